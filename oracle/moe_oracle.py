@@ -1,0 +1,356 @@
+"""CPU oracle for the weight-only 4-bit routed-expert MoE layer (W4A16).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the CPU
+baseline leg of bench.py may import this module.  The product path (the CUDA
+library and its Python binding) never calls it and shares no code with it.
+
+Plain, slow and meant to be checked by eye: NumPy, fp64 arithmetic unless a
+step's definition fixes another precision, no blocking or fusion.
+
+Sources, cited by page title and section:
+  [INT4]   "Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe: routed experts are
+           INT4, symmetric, group 128, round-to-nearest per group with min-max
+           scales, no calibration; the fused banks experts.gate_up_proj
+           [256, 1024, 2048] and experts.down_proj [256, 2048, 512].
+  [MXFP4]  "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary / What
+           was quantized / Quantization method: MXFP4 W4A16 experts (E2M1
+           codes, one shared power-of-two scale per 32 elements, one packed and
+           one scale tensor per matrix), scale exponents of the
+           floor(log2(x / 6)) family.
+  [ROUTE]  "cbert33/Nex-N2.5-mini-FP8-Calibrated", Artifact summary: 256
+           routed experts, 8 active per token; routers kept in bf16
+           ("Tech2wild/...", Recipe table).
+  [LAYOUT] "primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", What's quantized to
+           what: experts shipped as two batched 3-D tensors per layer; gate and
+           up are the two halves of the fused gate_up bank.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * INT4 scale s = bf16(fp32(amax) / 7): the group max maps to code +-7, code
+    -8 is never produced; q = clamp(round_half_even(fp32(w / s)), -8, 7);
+    stored as offset-binary nibbles q + 8, element 2j in the low nibble of
+    byte j.  Scales are bf16 in their own plane.  An all-zero group has s = 0
+    and codes 0.  The last group of a row holds K mod 128 elements.
+  * MXFP4 exponent e = floor(log2(amax / 6)), i.e. the largest integer with
+    6 * 2^e <= amax, clamped to [-127, 127]; e = -127 for an all-zero block.
+    Scale byte e + 127 (E8M0).  Codes: nearest point of the E2M1 magnitude
+    grid {0, .5, 1, 1.5, 2, 3, 4, 6} to w / 2^e, ties to the even code index,
+    values past 6 saturate to 6; nibble = sign << 3 | code, zero is +0.
+  * Router: fp32 logits (+ optional fp32 bias), top-k by value with ties to
+    the lower expert index, ids in descending-logit order; weights are the
+    softmax restricted to the selected k (= full softmax renormalised over
+    the top-k), in fp64.
+  * Expert MLP is SwiGLU: a = silu(gate) * up with gate = rows [0, I) of the
+    fused bank and up = rows [I, 2I); y = W_down a.
+  * Two bf16 roundings belong to the W4A16 method itself and are modelled:
+    the dequantised weight (bf16(q * s) for INT4; exact for MXFP4) and the
+    activation a that feeds the down projection.  Expert outputs y and the
+    routing-weighted sum stay in fp64 here.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+INT4_GROUP = 128
+MX_BLOCK = 32
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+
+FMT_INT4 = "int4_g128"
+FMT_MXFP4 = "mxfp4"
+
+
+# --------------------------------------------------------------------------
+# bf16 <-> float helpers (bit-level, no casts that could flush or double-round)
+# --------------------------------------------------------------------------
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> exact fp64 values."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    """Round fp64 values to bf16 with round-half-to-even; returns uint16 bits.
+
+    bf16 keeps 8 significant bits and the fp32 exponent range: normal numbers
+    down to 2^-126 and subnormals on the 2^-133 grid below that.  Rounding is
+    done exactly in fp64 (scaling by powers of two is exact, np.rint is
+    half-to-even), then the already-representable value is narrowed.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                       # x = m * 2^e, 0.5 <= |m| < 1
+    normal = e >= -125                        # |x| >= 2^-126
+    r_norm = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+    r_sub = np.ldexp(np.rint(np.ldexp(x, 133)), -133)
+    r = np.where(normal, r_norm, r_sub)
+    r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, x), r)
+    return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_round(x) -> np.ndarray:
+    """fp64 -> nearest bf16 value, returned as fp64."""
+    return bf16_to_f64(f64_to_bf16(x))
+
+
+# --------------------------------------------------------------------------
+# INT4 symmetric round-to-nearest, group 128, bf16 min-max scales   [INT4]
+# --------------------------------------------------------------------------
+
+def int4_groups(K: int):
+    """Column ranges of the 128-element groups of a row of length K."""
+    return [(g0, min(g0 + INT4_GROUP, K)) for g0 in range(0, K, INT4_GROUP)]
+
+
+def pack_int4_g128(w_bits):
+    """Quantise a bf16 bank [E, N, K] (or [N, K]) row by row, group by group.
+
+    Returns (codes uint8 [..., N, K/2], scales uint16 bf16 bits [..., N, G]).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    K = w_bits.shape[-1]
+    assert K % 2 == 0
+    w32 = bf16_to_f64(w_bits).astype(np.float32)        # exact
+    groups = int4_groups(K)
+    q = np.zeros(w32.shape, dtype=np.int32)
+    scales = np.zeros(w32.shape[:-1] + (len(groups),), dtype=np.uint16)
+    for gi, (a, b) in enumerate(groups):
+        wg = w32[..., a:b]
+        amax = np.max(np.abs(wg), axis=-1)               # fp32, exact
+        s32 = amax / np.float32(7.0)                      # fp32 correctly rounded quotient
+        s_bits = f64_to_bf16(s32.astype(np.float64))
+        s = bf16_to_f64(s_bits).astype(np.float32)[..., None]
+        safe = np.where(s == 0, np.float32(1.0), s)
+        quot = wg / safe                                  # fp32 correctly rounded quotient
+        qg = np.clip(np.rint(quot), -8, 7).astype(np.int32)
+        q[..., a:b] = np.where(s == 0, 0, qg)
+        scales[..., gi] = s_bits
+    u = (q + 8).astype(np.uint8)                          # offset binary 0..15
+    codes = (u[..., 0::2] | (u[..., 1::2] << np.uint8(4))).astype(np.uint8)
+    return codes, scales
+
+
+def unpack_nibbles(codes) -> np.ndarray:
+    """uint8 [..., K/2] -> uint8 nibbles [..., K], element 2j = low nibble of byte j."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = codes & np.uint8(0x0F)
+    out[..., 1::2] = codes >> np.uint8(4)
+    return out
+
+
+def int4_codes(codes) -> np.ndarray:
+    """Signed INT4 values q in [-8, 7] from packed offset-binary nibbles."""
+    return unpack_nibbles(codes).astype(np.int32) - 8
+
+
+def dequant_int4_g128(codes, scales) -> np.ndarray:
+    """w_hat = bf16(q * s) per element (q * s is exact in fp64), as fp64."""
+    q = int4_codes(codes).astype(np.float64)
+    K = q.shape[-1]
+    s = bf16_to_f64(scales)
+    s_full = np.empty_like(q)
+    for gi, (a, b) in enumerate(int4_groups(K)):
+        s_full[..., a:b] = s[..., gi:gi + 1]
+    return bf16_round(q * s_full)
+
+
+# --------------------------------------------------------------------------
+# MXFP4: E2M1 codes, E8M0 scale per 32 elements                      [MXFP4]
+# --------------------------------------------------------------------------
+
+def mx_exponent(amax) -> np.ndarray:
+    """Largest integer e with 6 * 2^e <= amax (= floor(log2(amax/6))), clamped
+    to [-127, 127]; -127 for amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    pos = amax > 0
+    safe = np.where(pos, amax, 6.0)
+    e = np.floor(np.log2(safe / 6.0)).astype(np.int64)
+    # fix up the fp64 log2 estimate with exact power-of-two comparisons
+    e = np.where(6.0 * np.ldexp(1.0, e + 1) <= safe, e + 1, e)
+    e = np.where(6.0 * np.ldexp(1.0, e) > safe, e - 1, e)
+    e = np.clip(e, -127, 127)
+    return np.where(pos, e, -127)
+
+
+def e2m1_nearest(v) -> np.ndarray:
+    """Magnitude code 0..7 of the E2M1 grid point nearest |v|; ties go to the
+    even code index (the grid point whose mantissa bit is 0)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    d = np.abs(a[..., None] - E2M1_GRID)                  # distance to each grid point
+    best = np.min(d, axis=-1, keepdims=True)
+    is_best = d == best
+    # among equally near points prefer an even index; there is never more than one
+    even_best = is_best & (np.arange(8) % 2 == 0)
+    pick = np.where(even_best.any(axis=-1), np.argmax(even_best, axis=-1), np.argmax(is_best, axis=-1))
+    return pick.astype(np.uint8)
+
+
+def pack_mxfp4(w_bits):
+    """Quantise a bf16 bank [..., N, K] in blocks of 32 along K.
+
+    Returns (codes uint8 [..., N, K/2], scales uint8 E8M0 [..., N, K/32]).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    K = w_bits.shape[-1]
+    assert K % MX_BLOCK == 0
+    w = bf16_to_f64(w_bits)
+    blocks = w.reshape(w.shape[:-1] + (K // MX_BLOCK, MX_BLOCK))
+    amax = np.max(np.abs(blocks), axis=-1)
+    e = mx_exponent(amax)
+    v = blocks / np.ldexp(1.0, e)[..., None]              # exact power-of-two scaling
+    mag = e2m1_nearest(v)
+    sign = ((blocks < 0) & (mag > 0)).astype(np.uint8)
+    nib = ((sign << np.uint8(3)) | mag).reshape(w.shape).astype(np.uint8)
+    codes = (nib[..., 0::2] | (nib[..., 1::2] << np.uint8(4))).astype(np.uint8)
+    scales = (e + 127).astype(np.uint8)
+    return codes, scales
+
+
+def e2m1_value(nibbles) -> np.ndarray:
+    nib = np.asarray(nibbles, dtype=np.uint8)
+    mag = E2M1_GRID[nib & np.uint8(7)]
+    return np.where(nib & np.uint8(8), -mag, mag)
+
+
+def dequant_mxfp4(codes, scales) -> np.ndarray:
+    """w_hat = e2m1(c) * 2^(scale - 127), exact (asserted representable in bf16)."""
+    vals = e2m1_value(unpack_nibbles(codes))
+    K = vals.shape[-1]
+    e = np.asarray(scales, dtype=np.int64) - 127
+    full = vals * np.repeat(np.ldexp(1.0, e), MX_BLOCK, axis=-1)[..., :K]
+    assert np.array_equal(bf16_round(full), full), "MXFP4 dequant not exact in bf16"
+    return full
+
+
+def pack(fmt: str, w_bits):
+    return pack_int4_g128(w_bits) if fmt == FMT_INT4 else pack_mxfp4(w_bits)
+
+
+def dequant(fmt: str, codes, scales):
+    return dequant_int4_g128(codes, scales) if fmt == FMT_INT4 else dequant_mxfp4(codes, scales)
+
+
+def packed_bytes_per_expert(fmt: str, hidden: int, inter: int) -> int:
+    """Bytes of codes + scales for one expert's gate_up [2I, H] and down [H, I]."""
+    def mat(N, K):
+        if fmt == FMT_INT4:
+            return N * K // 2 + N * len(int4_groups(K)) * 2
+        return N * K // 2 + N * (K // MX_BLOCK)
+    return mat(2 * inter, hidden) + mat(hidden, inter)
+
+
+# --------------------------------------------------------------------------
+# Router: logits -> top-k -> softmax over the selected k             [ROUTE]
+# --------------------------------------------------------------------------
+
+def router_logits(x_bits, router_bits) -> np.ndarray:
+    """fp32 logits = fp32(x . Wr^T) with the dot products taken in fp64."""
+    return (bf16_to_f64(x_bits) @ bf16_to_f64(router_bits).T).astype(np.float32)
+
+
+def route(logits32, bias32, k: int):
+    """Top-k of the fp32 logits (+ fp32 bias), ties to the lower expert index.
+
+    Returns (ids int32 [T, k] in descending-logit order, weights fp64 [T, k]).
+    """
+    L = np.asarray(logits32, dtype=np.float32)
+    if bias32 is not None:
+        L = (L + np.asarray(bias32, dtype=np.float32)[None, :]).astype(np.float32)
+    # a stable sort of -L keeps the lower index first among equal logits
+    ids = np.argsort(-L, axis=1, kind="stable")[:, :k].astype(np.int32)
+    sel = np.take_along_axis(L, ids, axis=1).astype(np.float64)
+    ex = np.exp(sel - sel[:, :1])                         # sel[:, 0] is the row max
+    return ids, ex / ex.sum(axis=1, keepdims=True)
+
+
+def permute(ids, num_experts: int):
+    """Stable counting sort of the flat (token, slot) index r = t*k + j by expert.
+
+    Returns (offsets int32 [E+1], sorted_rows int32 [T*k], pos int32 [T*k]) with
+    sorted_rows[offsets[e]:offsets[e+1]] the rows routed to expert e in
+    ascending r, and pos the inverse permutation.
+    """
+    flat = np.asarray(ids, dtype=np.int64).reshape(-1)
+    counts = np.bincount(flat, minlength=num_experts)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    sorted_rows = np.argsort(flat, kind="stable").astype(np.int32)
+    pos = np.empty_like(sorted_rows)
+    pos[sorted_rows] = np.arange(flat.size, dtype=np.int32)
+    return offsets, sorted_rows, pos
+
+
+# --------------------------------------------------------------------------
+# Expert MLP and combine                                         [INT4][LAYOUT]
+# --------------------------------------------------------------------------
+
+def silu(z):
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+class PackedBank:
+    """Codes + scales of one fused bank, dequantised lazily per expert."""
+
+    def __init__(self, fmt: str, codes, scales):
+        self.fmt, self.codes, self.scales = fmt, codes, scales
+        self._cache = {}
+
+    @classmethod
+    def from_bf16(cls, fmt: str, w_bits):
+        return cls(fmt, *pack(fmt, w_bits))
+
+    def expert(self, e: int) -> np.ndarray:
+        if e not in self._cache:
+            self._cache[e] = dequant(self.fmt, self.codes[e], self.scales[e])
+        return self._cache[e]
+
+
+def expert_mlp(x_rows, w_gate_up, w_down):
+    """SwiGLU expert on fp64 rows: a = bf16(silu(h_gate) * h_up), y = W_down a."""
+    inter = w_gate_up.shape[0] // 2
+    h = x_rows @ w_gate_up.T
+    a = bf16_round(silu(h[:, :inter]) * h[:, inter:])
+    return a, a @ w_down.T
+
+
+def forward_routed(x_bits, ids, weights, gate_up: PackedBank, down: PackedBank, num_experts: int):
+    """Layer output for given routing: out_t = sum_j w_tj * y(expert ids_tj, x_t).
+
+    Returns (out fp64 [T, H], a fp64 [T*k, I] in expert-sorted row order).
+    """
+    x = bf16_to_f64(x_bits)
+    T, k = ids.shape
+    offsets, sorted_rows, _ = permute(ids, num_experts)
+    out = np.zeros((T, x.shape[1]), dtype=np.float64)
+    a_sorted = None
+    wflat = np.asarray(weights, dtype=np.float64).reshape(-1)
+    for e in range(num_experts):
+        rows = sorted_rows[offsets[e]:offsets[e + 1]]
+        if rows.size == 0:
+            continue
+        toks = rows // k                                  # each token at most once per expert
+        a, y = expert_mlp(x[toks], gate_up.expert(e), down.expert(e))
+        if a_sorted is None:
+            a_sorted = np.zeros((T * k, a.shape[1]), dtype=np.float64)
+        a_sorted[offsets[e]:offsets[e + 1]] = a
+        out[toks] += wflat[rows][:, None] * y
+    return out, a_sorted
+
+
+def forward(x_bits, router_bits, bias32, gate_up: PackedBank, down: PackedBank, top_k: int):
+    """The whole layer: router logits -> route -> experts -> weighted combine."""
+    E = np.asarray(router_bits).shape[0]
+    logits = router_logits(x_bits, router_bits)
+    ids, w = route(logits, bias32, top_k)
+    out, a_sorted = forward_routed(x_bits, ids, w, gate_up, down, E)
+    return {"logits": logits, "ids": ids, "weights": w, "out": out, "a_sorted": a_sorted}
+
+
+def routing_margin(logits32, bias32, k: int) -> np.ndarray:
+    """Per token, the gap between the k-th and (k+1)-th largest (biased) logit."""
+    L = np.asarray(logits32, dtype=np.float64)
+    if bias32 is not None:
+        L = L + np.asarray(bias32, dtype=np.float64)[None, :]
+    s = -np.sort(-L, axis=1)
+    if s.shape[1] <= k:
+        return np.full(s.shape[0], np.inf)
+    return s[:, k - 1] - s[:, k]
