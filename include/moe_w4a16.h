@@ -1,0 +1,256 @@
+/*
+ * moe_w4a16.h - C ABI of the B200 (sm_100a) weight-only 4-bit routed-expert
+ * MoE layer (W4A16: 4-bit expert weights, bf16 activations).
+ *
+ * The operation is the forward pass of one Qwen3.5-MoE expert layer:
+ *
+ *   logits = x Wr^T (+ bias)                     router, fp32
+ *   ids, w = top-k(logits), softmax over the k   per token
+ *   h      = W_gate_up[e] x_t                    per (token, slot), e = ids
+ *   a      = bf16(silu(h[0:I]) * h[I:2I])        SwiGLU
+ *   y      = W_down[e] a
+ *   out_t  = sum_j w_tj y_tj                     bf16 output
+ *
+ * Sources (model cards of quantised builds of one 35B MoE model):
+ *   "Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe: routed experts INT4,
+ *     symmetric, group 128, round-to-nearest with min-max scales; the fused
+ *     banks experts.gate_up_proj [256, 1024, 2048] (gate rows then up rows)
+ *     and experts.down_proj [256, 2048, 512]; routers stay bf16.
+ *   "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary and
+ *     Quantization method: MXFP4 W4A16 experts (E2M1 codes, one E8M0 scale
+ *     per 32 elements, exponents of the floor(log2(x / 6)) family).
+ *   "cbert33/Nex-N2.5-mini-FP8-Calibrated", Artifact summary: 256 routed
+ *     experts per layer, 8 active per token.
+ * Where the cards are silent the library takes the plain reading documented
+ * at each entry point (softmax top-k renormalised, SwiGLU, ties to the lower
+ * expert index).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     16-byte aligned unless stated.  bf16 tensors are passed as uint16_t
+ *     bit patterns.
+ *   - Nothing allocates device memory: scratch comes from a caller-provided
+ *     workspace whose size a query function returns.
+ *   - Calls only enqueue work on `stream` (asynchronous, no host sync) and
+ *     keep no global mutable state, so they are reentrant across streams as
+ *     long as workspaces are not shared.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and leave every output untouched.
+ */
+#ifndef MOE_W4A16_H
+#define MOE_W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+/* Exported symbol marker (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape outside the supported envelope (see moe_shape_t) */
+  MOE_ERR_WORKSPACE = 3,     /* workspace null or smaller than the query returned */
+  MOE_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  MOE_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (reported by moe_workspace_status) */
+  MOE_ERR_NONFINITE = 6      /* NaN/Inf met while packing (reported through the count pointer) */
+} moe_status_t;
+
+typedef enum {
+  MOE_FMT_INT4_G128 = 1,     /* INT4 symmetric RTN, bf16 scale per 128 elements along K */
+  MOE_FMT_MXFP4_G32 = 2      /* MXFP4: E2M1 codes, E8M0 scale per 32 elements along K */
+} moe_format_t;
+
+/* Layer shape.  Supported: hidden and inter multiples of 64 (>= 64),
+ * 1 <= top_k <= 32, top_k <= num_experts <= 1024. */
+typedef struct {
+  int hidden;          /* H */
+  int inter;           /* I, expert intermediate size; gate_up bank is [E, 2I, H] */
+  int num_experts;     /* E */
+  int top_k;           /* k */
+  moe_format_t fmt;    /* format of both expert banks */
+} moe_shape_t;
+
+/* Returns a static, NUL-terminated description of a status code. */
+MOE_API const char* moe_status_str(moe_status_t status);
+
+/* Returns MOE_ABI_VERSION of the loaded library. */
+MOE_API int moe_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Packed bank layout
+ *
+ * A packed bank of E matrices [N, K] is ONE buffer:
+ *   bytes [0, E*N*K/2)          codes, [E][N][K/2]: element 2j of a row in the
+ *                               low nibble of byte j, element 2j+1 in the high
+ *                               nibble.  INT4: offset binary q + 8 (q in
+ *                               [-8, 7]).  MXFP4: sign<<3 | E2M1 magnitude code.
+ *   bytes [scale_offset, total) scales.  INT4: bf16 [E][N][ceil(K/128)] (the
+ *                               last group of a row holds K mod 128 elements).
+ *                               MXFP4: E8M0 uint8 [E][N][K/32], byte = e + 127.
+ * scale_offset is E*N*K/2 rounded up to 256 bytes.
+ * ---------------------------------------------------------------------- */
+
+/* Total bytes of a packed bank of E matrices [N, K]; 0 if the arguments are invalid. */
+MOE_API size_t moe_bank_bytes(moe_format_t fmt, int E, int N, int K);
+
+/* Byte offset of the scale plane inside a packed bank; 0 if invalid. */
+MOE_API size_t moe_bank_scale_offset(moe_format_t fmt, int E, int N, int K);
+
+/* Bytes of the packed gate_up bank (which = 0, [E, 2I, H]) or down bank
+ * (which = 1, [E, H, I]) of a layer; 0 if invalid. */
+MOE_API size_t moe_packed_bytes(const moe_shape_t* shape, int which);
+
+/* ------------------------------------------------------------------------
+ * Packing (offline step, bandwidth-bound)
+ * ---------------------------------------------------------------------- */
+
+/* Quantise a bf16 bank w [E, N, K] (device) to INT4 symmetric RTN with one
+ * bf16 scale per 128 consecutive K elements of a row
+ * ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe):
+ *   s = bf16_rne(fp32(amax) / 7)          (the group max maps to +-7)
+ *   q = clamp(rint_half_even(fp32(w / s)), -8, 7), q = 0 when s == 0.
+ * K must be a positive multiple of 32; N, E >= 1.  Writes moe_bank_bytes()
+ * bytes at `packed` (device, 256-byte aligned).  If `nonfinite_count`
+ * (device int32, nullable) is given, the number of NaN/Inf inputs is ADDED
+ * to it; such elements produce unspecified codes. */
+MOE_API moe_status_t moe_pack_int4_g128(const uint16_t* w, int E, int N, int K, void* packed,
+                                int32_t* nonfinite_count, cudaStream_t stream);
+
+/* Quantise a bf16 bank w [E, N, K] to MXFP4 ("kirillbilchenko/Nex-N2.5-mini-
+ * MXFP4-MxWave", Model summary and Quantization method), per block of 32
+ * consecutive K elements:
+ *   e = floor(log2(amax / 6)) clamped to [-127, 127] (-127 when amax == 0),
+ *   scale byte e + 127; code = nearest E2M1 magnitude of |w| / 2^e (ties to
+ *   the even code, saturating at 6), sign bit set only for nonzero codes.
+ * Same arguments and errors as moe_pack_int4_g128. */
+MOE_API moe_status_t moe_pack_mxfp4(const uint16_t* w, int E, int N, int K, void* packed,
+                            int32_t* nonfinite_count, cudaStream_t stream);
+
+/* Expand a packed bank back to bf16 w_out [E, N, K] (device):
+ * INT4 w = bf16_rne(q * s); MXFP4 w = e2m1(c) * 2^e (exact).  Debug and test
+ * entry; the forward pass dequantises inside its GEMMs instead. */
+MOE_API moe_status_t moe_dequant(const void* packed, moe_format_t fmt, int E, int N, int K,
+                         uint16_t* w_out, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Routing
+ * ---------------------------------------------------------------------- */
+
+/* Top-k routing of fp32 logits [T, E] (+ optional fp32 bias [E], nullable)
+ * ("cbert33/Nex-N2.5-mini-FP8-Calibrated", Artifact summary: 8 of 256
+ * experts active).  Per token: the k largest biased logits, equal values
+ * ordered by the lower expert index, written in that order to topk_ids
+ * [T, k] (int32); topk_w [T, k] (fp32) = exp(l_j - l_max) / sum over the
+ * selected k (the softmax over all experts renormalised over the top-k).
+ * T >= 0 (T == 0 is a no-op), 1 <= k <= min(32, E), E <= 1024.
+ * No 16-byte alignment requirement (4-byte alignment suffices). */
+MOE_API moe_status_t moe_route(const float* logits, const float* bias, int T, int E, int k,
+                       int32_t* topk_ids, float* topk_w, cudaStream_t stream);
+
+/* Workspace bytes moe_permute needs for T tokens. */
+MOE_API size_t moe_permute_workspace_bytes(int T, int E, int k);
+
+/* Stable counting sort of the flat (token, slot) rows r = t*k + j by expert
+ * id (topk_ids [T, k], values in [0, E)):
+ *   offsets [E+1]      offsets[e] = number of rows with expert < e
+ *   sorted_rows [T*k]  rows of expert e at [offsets[e], offsets[e+1]) in
+ *                      ascending r
+ *   pos [T*k]          inverse permutation: sorted_rows[pos[r]] = r.
+ * Ids outside [0, E) are a contract violation (results unspecified, no
+ * out-of-bounds access). */
+MOE_API moe_status_t moe_permute(const int32_t* topk_ids, int T, int E, int k, int32_t* offsets,
+                         int32_t* sorted_rows, int32_t* pos, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Layer forward
+ * ---------------------------------------------------------------------- */
+
+typedef enum {
+  MOE_PATH_AUTO = 0,      /* decode path for T <= 32, grouped tcgen05 GEMMs above */
+  MOE_PATH_DECODE = 1,    /* weight-streaming GEMV kernels (any T; meant for T <= 32) */
+  MOE_PATH_PREFILL = 2    /* grouped tcgen05 GEMMs (any T >= 1) */
+} moe_path_t;
+
+/* Number of timed stages moe_forward reports through stage_events. */
+#define MOE_NUM_STAGES 5
+/* Stage ids: 0 router logits, 1 top-k + permutation, 2 gate_up + SwiGLU,
+ * 3 down projection, 4 weighted combine / output conversion. */
+
+/* Optional extras of moe_forward / moe_forward_routed.  Every pointer may be
+ * NULL; a NULL opts pointer means all defaults. */
+typedef struct {
+  moe_path_t path;
+  int32_t* topk_ids_out;     /* [T, k]  routing ids (moe_forward only) */
+  float* topk_w_out;         /* [T, k]  routing weights (moe_forward only) */
+  float* logits_out;         /* [T, E]  fp32 router logits, before the bias */
+  int32_t* offsets_out;      /* [E+1]   per-expert row offsets */
+  int32_t* sorted_rows_out;  /* [T*k]   expert-sorted rows */
+  uint16_t* act_out;         /* [T*k, I] bf16 SwiGLU activations, expert-sorted rows */
+  cudaEvent_t* stage_events; /* [2*MOE_NUM_STAGES]: recorded before / after each stage */
+} moe_forward_opts_t;
+
+/* Workspace bytes moe_forward / moe_forward_routed need for T tokens. */
+MOE_API size_t moe_workspace_bytes(const moe_shape_t* shape, int T);
+
+/* Forward pass of the routed-expert layer.
+ *   x            [T, H] bf16 hidden states
+ *   router_w     [E, H] bf16 router weight (logits = x router_w^T, fp32 accumulation)
+ *   logit_bias   [E] fp32 added to the logits before top-k (nullable)
+ *   gate_up_packed  packed bank of [E, 2I, H] (gate rows [0, I), up rows [I, 2I))
+ *   down_packed     packed bank of [E, H, I]
+ *   workspace    >= moe_workspace_bytes(shape, T) bytes, 256-byte aligned
+ *   out          [T, H] bf16 output: sum_j w_tj W_down[e] bf16(silu(g) * u),
+ *                accumulated in fp32 and rounded to bf16 once.
+ * T >= 0 (T == 0 is a no-op).  Device-side waits are bounded; an expired
+ * wait is reported by moe_workspace_status. */
+MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T,
+                         const uint16_t* router_w, const float* logit_bias,
+                         const void* gate_up_packed, const void* down_packed,
+                         void* workspace, size_t workspace_bytes, uint16_t* out,
+                         const moe_forward_opts_t* opts, cudaStream_t stream);
+
+/* The same layer with the routing given: topk_ids [T, k] int32 (distinct
+ * experts per token, values in [0, E)) and topk_w [T, k] fp32.  Used to check
+ * the expert path on its own (e.g. with the oracle's routing). */
+MOE_API moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int T,
+                                const int32_t* topk_ids, const float* topk_w,
+                                const void* gate_up_packed, const void* down_packed,
+                                void* workspace, size_t workspace_bytes, uint16_t* out,
+                                const moe_forward_opts_t* opts, cudaStream_t stream);
+
+/* Zeroes the status word at the start of a workspace (enqueued on `stream`).
+ * Call once after allocating a workspace, before its first use. */
+MOE_API moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, then reports MOE_ERR_TIMEOUT if a bounded
+ * device-side wait of a previous moe_forward on this workspace expired (and
+ * clears the flag), MOE_OK otherwise. */
+MOE_API moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Self-test of the bounded device-side wait: launches one warp that waits on
+ * a barrier nothing ever arrives at, gives up after `limit_ns` nanoseconds of
+ * device time (at most 10 s) and raises the workspace status word, so that a
+ * following moe_workspace_status returns MOE_ERR_TIMEOUT.  The GPU context
+ * stays usable.  No counterpart on the model cards: this checks the library's
+ * own failure reporting. */
+MOE_API moe_status_t moe_selftest_bounded_wait(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
+                                       cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_W4A16_H */

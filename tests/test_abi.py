@@ -1,0 +1,138 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point
+include/moe_w4a16.h declares, answers size queries, and rejects bad arguments
+on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_synth
+import weight_only_bit_router_b200 as moe
+from conftest import ROOT
+from oracle import moe_oracle as o
+
+HEADER = os.path.join(ROOT, "include", "moe_w4a16.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_loads_and_reports_abi_version():
+    assert moe.moe_abi_version() == 1
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = declared_functions()
+    assert len(names) >= 15
+    handle = moe.lib()
+    for n in names:
+        assert hasattr(handle, n), n
+    assert sorted(moe.exported_symbols()) == names
+
+
+def test_status_strings():
+    assert moe.moe_status_str(0) == "ok"
+    assert "timeout" in moe.moe_status_str(5) or "expired" in moe.moe_status_str(5)
+
+
+@pytest.mark.parametrize("fmt", ["int4_g128", "mxfp4"])
+def test_bank_sizes_match_closed_form(fmt):
+    s = moe.make_shape(2048, 512, 256, 8, fmt)
+    gu, dn = moe.moe_packed_bytes(s, 0), moe.moe_packed_bytes(s, 1)
+    per_expert = o.packed_bytes_per_expert(o.FMT_INT4 if fmt == "int4_g128" else o.FMT_MXFP4, 2048, 512)
+    # two 256-byte alignment pads at most (codes -> scales, per bank)
+    assert 0 <= gu + dn - 256 * per_expert < 2 * 256
+    assert moe.moe_packed_bytes(s, 2) == 0
+    assert moe.moe_bank_scale_offset(fmt, 256, 1024, 2048) == 256 * 1024 * 1024
+
+
+def test_bank_bytes_rejects_bad_sizes():
+    assert moe.moe_bank_bytes("int4_g128", 1, 1, 48) == 0   # K % 32 != 0
+    assert moe.moe_bank_bytes("int4_g128", 0, 1, 64) == 0
+    assert moe.moe_bank_bytes(7, 1, 1, 64) == 0
+
+
+def test_workspace_bytes_grow_with_tokens_and_reject_bad_shapes():
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    a, b = moe.moe_workspace_bytes(s, 1), moe.moe_workspace_bytes(s, 8192)
+    assert 0 < a < b
+    assert moe.moe_workspace_bytes(s, -1) == 0
+    assert moe.moe_workspace_bytes(moe.make_shape(2000, 512, 256, 8, "int4_g128"), 4) == 0
+    assert moe.moe_workspace_bytes(moe.make_shape(2048, 512, 256, 33, "int4_g128"), 4) == 0
+
+
+def _c(fn, *args):
+    return getattr(moe.lib(), fn)(*args)
+
+
+def test_pack_rejects_null_and_bad_k_without_a_gpu():
+    L = moe.lib()
+    assert L.moe_pack_int4_g128(None, 1, 1, 64, 256, None, None) == 1
+    assert L.moe_pack_mxfp4(16, 1, 1, 48, 256, None, None) == 1        # K % 32
+    assert L.moe_pack_mxfp4(16, 1, 1, 64, 255, None, None) == 1        # misaligned output
+    assert L.moe_dequant(None, 1, 1, 1, 64, 16, None) == 1
+
+
+def test_route_and_permute_validation():
+    L = moe.lib()
+    assert L.moe_route(16, None, 4, 256, 33, 16, 16, None) == 2        # k > 32
+    assert L.moe_route(16, None, 4, 8, 9, 16, 16, None) == 2           # k > E
+    assert L.moe_route(16, None, -1, 8, 2, 16, 16, None) == 1
+    assert L.moe_route(None, None, 0, 8, 2, None, None, None) == 0      # T == 0 is a no-op
+    assert L.moe_permute(16, 4, 2000, 2, 256, 256, 256, 256, 1 << 20, None) == 2
+    assert L.moe_permute(16, 4, 8, 2, 256, 256, 256, None, 0, None) == 3
+
+
+def test_forward_validation_happens_on_the_host():
+    L = moe.lib()
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    ws = moe.moe_workspace_bytes(s, 4)
+    args = lambda **kw: [ctypes.byref(kw.get("shape", s)), kw.get("x", 256), kw.get("T", 4), kw.get("r", 256),
+                         None, kw.get("gu", 256), kw.get("dn", 256), kw.get("ws", 256), kw.get("wsb", ws),
+                         kw.get("out", 256), None, None]
+    assert L.moe_forward(*args(x=None)) == 1
+    assert L.moe_forward(*args(x=8)) == 1                  # x not 16-byte aligned
+    assert L.moe_forward(*args(gu=512 + 16)) == 1          # packed bank not 256-byte aligned
+    assert L.moe_forward(*args(ws=None)) == 3
+    assert L.moe_forward(*args(wsb=ws - 1)) == 3
+    assert L.moe_forward(*args(T=-2)) == 1
+    assert L.moe_forward(*args(shape=moe.make_shape(2048, 500, 256, 8, "int4_g128"))) == 2
+    assert L.moe_forward(*args(shape=moe.make_shape(2048, 512, 256, 8, 3))) == 1
+    assert L.moe_forward(*args(r=None)) == 1
+    opts = moe.ForwardOpts()
+    opts.path = 9
+    a = args()
+    a[10] = ctypes.byref(opts)
+    assert L.moe_forward(*a) == 1
+    # the decode path keeps [T*k, H] expert outputs: bounded token count
+    opts.path = moe.MOE_PATH_DECODE
+    big = moe.moe_workspace_bytes(s, 4096)
+    a = args(T=4096, wsb=big)
+    a[10] = ctypes.byref(opts)
+    assert L.moe_forward(*a) == 2
+    # T == 0 is a valid no-op
+    assert L.moe_forward(*args(T=0)) == 0
+
+
+def test_routed_forward_validation():
+    L = moe.lib()
+    s = moe.make_shape(256, 64, 8, 2, "mxfp4")
+    ws = moe.moe_workspace_bytes(s, 16)
+    assert L.moe_forward_routed(ctypes.byref(s), 256, 16, None, 256, 256, 256, 256, ws, 256, None, None) == 1
+
+
+def test_workspace_status_validation():
+    L = moe.lib()
+    assert L.moe_workspace_status(None, 256, None) == 3
+    assert L.moe_workspace_init(256, 100, None) == 3
+    assert L.moe_selftest_bounded_wait(256, 256, 11 * 10**9, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    w = moe_synth.gate_up_bank(moe_synth.TINY, seed=0)
+    with pytest.raises(ValueError):
+        moe.moe_pack_int4_g128(w, packed=torch.empty(10, dtype=torch.uint8))

@@ -1,0 +1,289 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Bit-exact: packed bytes, dequantised weights, routing ids on identical
+logits, permutations.  Tolerance: routing weights |dw| <= 1e-6 (1 + |w|);
+layer outputs |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref) per element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import weight_only_bit_router_b200 as moe
+from oracle import moe_oracle as o
+from parity_util import FMT_NAMES, LazyOracleBank, assert_out_close, assert_routing_consistent
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+FMTS = ["int4_g128", "mxfp4"]
+
+
+def pack_gpu(fmt, w):
+    return moe.moe_pack_int4_g128(w) if fmt == "int4_g128" else moe.moe_pack_mxfp4(w)
+
+
+def gpu_split(fmt, packed, E, N, K):
+    codes, scales = moe.split_bank(packed, fmt, E, N, K)
+    c = codes.cpu().numpy()
+    s = scales.cpu().numpy()
+    return c, (s.view(np.uint16) if fmt == "int4_g128" else s)
+
+
+# ---------------------------------------------------------------- packing
+
+def edge_bank():
+    """Rows that exercise the corners of both packers (K = 192: a short last
+    INT4 group of 64; MXFP4 blocks of 32)."""
+    rng = np.random.default_rng(0)
+    K = 192
+    rows = [
+        np.zeros(K),                                               # all-zero groups
+        rng.normal(size=K) * 0.02,
+        rng.normal(size=K) * 1e3,
+        np.concatenate([[1.75, -0.875, 0.125, 0.1875], np.zeros(K - 4)]),  # hand-worked ties
+        np.concatenate([[3.0, -0.3125, 1.25, 0.625], np.zeros(K - 4)]),
+        np.full(K, 2.0 ** -133),                                   # bf16 subnormals
+        rng.normal(size=K) * 1e-38,
+        np.concatenate([[3.0e38, -1.0], rng.normal(size=K - 2)]),  # near bf16 max
+        (rng.integers(-8, 8, size=K) * 0.25),                      # many exact ties
+        -np.abs(rng.normal(size=K)),
+    ]
+    w = np.stack(rows)[None]                                       # [1, 10, 192]
+    bits = o.f64_to_bf16(w)
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_pack_bit_exact_tiny_and_edges(fmt):
+    for w in (moe_synth.gate_up_bank(moe_synth.TINY, 0), moe_synth.down_bank(moe_synth.TINY, 0), edge_bank()):
+        E, N, K = w.shape
+        packed = pack_gpu(fmt, w.to(DEV))
+        torch.cuda.synchronize()
+        gc, gs = gpu_split(fmt, packed, E, N, K)
+        rc, rs = o.pack(FMT_NAMES[fmt], moe_synth.bf16_bits(w))
+        assert np.array_equal(gc, rc)
+        assert np.array_equal(gs, rs)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_dequant_bit_exact(fmt):
+    for w in (moe_synth.gate_up_bank(moe_synth.TINY, 1), edge_bank()):
+        E, N, K = w.shape
+        packed = pack_gpu(fmt, w.to(DEV))
+        deq = moe.moe_dequant(packed, fmt, E, N, K)
+        torch.cuda.synchronize()
+        ref = o.dequant(FMT_NAMES[fmt], *o.pack(FMT_NAMES[fmt], moe_synth.bf16_bits(w)))
+        got = o.bf16_to_f64(moe_synth.bf16_bits(deq))
+        assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_pack_bit_exact_full_layer_sampled_experts(fmt):
+    gu = moe_synth.gate_up_bank(moe_synth.NEX, seed=1000, device=DEV)
+    packed = pack_gpu(fmt, gu)
+    torch.cuda.synchronize()
+    E, N, K = gu.shape
+    codes, scales = moe.split_bank(packed, fmt, E, N, K)
+    for e in (0, 131, 255):
+        rc, rs = o.pack(FMT_NAMES[fmt], moe_synth.bf16_bits(gu[e]))
+        assert np.array_equal(codes[e].cpu().numpy(), rc)
+        s = scales[e].cpu().numpy()
+        assert np.array_equal(s.view(np.uint16) if fmt == "int4_g128" else s, rs)
+
+
+def test_pack_counts_nonfinite_inputs():
+    w = moe_synth.gate_up_bank(moe_synth.TINY, 2).to(DEV)
+    w[0, 0, 5] = float("nan")
+    w[3, 7, 100] = float("inf")
+    cnt = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_pack_int4_g128(w, nonfinite=cnt)
+    moe.moe_pack_mxfp4(w, nonfinite=cnt)
+    assert int(cnt.item()) == 4
+
+
+# ---------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("T,E,k", [(1, 256, 8), (1000, 256, 8), (77, 8, 2), (64, 1024, 32), (5, 40, 40)])
+def test_route_bit_exact_on_identical_logits(T, E, k):
+    g = torch.Generator().manual_seed(T * 31 + E)
+    logits = torch.randn(T, E, generator=g)
+    logits[: T // 2] = torch.round(logits[: T // 2] * 2) / 2     # exact ties
+    bias = moe_synth.zipf_bias(moe_synth.LayerShape(64, 64, E, k), seed=3) if E >= k else None
+    for b in (None, bias):
+        ids, w = moe.moe_route(logits.to(DEV), k, bias=None if b is None else b.to(DEV))
+        torch.cuda.synchronize()
+        rid, rw = o.route(logits.numpy(), None if b is None else b.numpy(), k)
+        assert np.array_equal(ids.cpu().numpy(), rid)
+        wg = w.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(wg - rw) <= 1e-6 * (1 + np.abs(rw)))
+        assert np.all(np.abs(wg.sum(1) - 1) <= 8 * 2.0 ** -23 * k)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 256, 8), (4, 256, 8), (32, 256, 8), (100, 8, 2), (8192, 256, 8),
+                                   (3000, 1024, 32), (129, 3, 1)])
+def test_permute_bit_exact(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    if T >= 100:  # skew: most tokens on a few experts
+        hot = torch.randperm(E, generator=g)[:k]
+        ids[: T // 2] = hot.to(torch.int32)
+    offsets, sorted_rows, pos = moe.moe_permute(ids.to(DEV), E)
+    torch.cuda.synchronize()
+    ro, rs, rp = o.permute(ids.numpy(), E)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(sorted_rows.cpu().numpy(), rs)
+    assert np.array_equal(pos.cpu().numpy(), rp)
+
+
+# ---------------------------------------------------------------- layer forward
+
+def run_forward(layer, fmt, path=None, routed=None):
+    s = layer.shape
+    shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
+    T = layer.x.shape[0]
+    gu = pack_gpu(fmt, layer.gate_up)
+    dn = pack_gpu(fmt, layer.down)
+    ws = moe.alloc_workspace(shape, T)
+    dbg = {
+        "logits_out": torch.empty(T, s.num_experts, dtype=torch.float32, device=DEV),
+        "topk_ids_out": torch.empty(T, s.top_k, dtype=torch.int32, device=DEV),
+        "topk_w_out": torch.empty(T, s.top_k, dtype=torch.float32, device=DEV),
+        "act_out": torch.empty(T * s.top_k, s.inter, dtype=torch.bfloat16, device=DEV),
+        "offsets_out": torch.empty(s.num_experts + 1, dtype=torch.int32, device=DEV),
+        "sorted_rows_out": torch.empty(T * s.top_k, dtype=torch.int32, device=DEV),
+    }
+    if routed is None:
+        out = moe.moe_forward(shape, layer.x, layer.router_w, gu, dn, ws, bias=layer.bias, path=path, debug=dbg)
+    else:
+        ids, w = routed
+        for key in ("logits_out", "topk_ids_out", "topk_w_out"):
+            dbg.pop(key)
+        out = moe.moe_forward_routed(shape, layer.x, ids, w, gu, dn, ws, path=path, debug=dbg)
+    assert moe.moe_workspace_status(ws) == moe.MOE_OK
+    return out, dbg
+
+
+def check_layer(layer, fmt, path=None, sample=None):
+    """Full forward on the GPU; the oracle recomputes the (sampled) tokens."""
+    s = layer.shape
+    out, dbg = run_forward(layer, fmt, path)
+    T = layer.x.shape[0]
+    tok = np.arange(T) if sample is None else np.asarray(sample)
+    xb = moe_synth.bf16_bits(layer.x)[tok]
+    bias = None if layer.bias is None else layer.bias.cpu().numpy()
+    ref_logits = o.router_logits(xb, moe_synth.bf16_bits(layer.router_w))
+    gpu_logits = dbg["logits_out"][torch.as_tensor(tok, device=DEV)]
+    gpu_ids = dbg["topk_ids_out"][torch.as_tensor(tok, device=DEV)]
+    assert_routing_consistent(gpu_logits, ref_logits, gpu_ids, bias, s.top_k)
+    # routing is bit-exact given the GPU's own logits
+    rid, rw = o.route(gpu_logits.cpu().numpy(), bias, s.top_k)
+    assert np.array_equal(rid, gpu_ids.cpu().numpy())
+    gw = dbg["topk_w_out"][torch.as_tensor(tok, device=DEV)].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gw - rw) <= 1e-6 * (1 + np.abs(rw)))
+    gu = LazyOracleBank(fmt, layer.gate_up)
+    dn = LazyOracleBank(fmt, layer.down)
+    ref_out, ref_act = o.forward_routed(xb, rid, rw, gu, dn, s.num_experts)
+    assert_out_close(out[torch.as_tensor(tok, device=DEV)], ref_out, f"{fmt} T={T}")
+    if sample is None:
+        # expert-sorted activations (bf16): the oracle rounds from fp64, the GPU from fp32
+        ga = o.bf16_to_f64(moe_synth.bf16_bits(dbg["act_out"]))
+        diff = np.abs(ga - ref_act)
+        assert np.all(diff <= 2.0 ** -7 * np.abs(ref_act) + 1e-3 * np.sqrt(np.mean(ref_act ** 2)))
+        ro, rs, _ = o.permute(rid, s.num_experts)
+        assert np.array_equal(dbg["offsets_out"].cpu().numpy(), ro)
+        assert np.array_equal(dbg["sorted_rows_out"].cpu().numpy(), rs)
+    return out
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("path", [moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL])
+def test_forward_tiny_layer(fmt, path):
+    layer = moe_synth.make_layer(moe_synth.TINY, T=16, seed=moe_synth.SEED_TINY, device=DEV)
+    check_layer(layer, fmt, path)
+
+
+@pytest.mark.parametrize("T", [1, 3, 33, 130, 300])
+def test_forward_tiny_shape_ragged_token_counts(T):
+    layer = moe_synth.make_layer(moe_synth.TINY, T=T, seed=40 + T, zipf=True, device=DEV)
+    check_layer(layer, "int4_g128", moe.MOE_PATH_PREFILL)
+    if T <= 256:
+        check_layer(layer, "mxfp4", moe.MOE_PATH_DECODE)
+
+
+def test_forward_odd_shapes_and_partial_tiles():
+    """I = 192 and H = 320: weight-row tiles of 128 end part-way, one INT4 group
+    of 64 closes every row of the down bank and of gate_up."""
+    shape = moe_synth.LayerShape(hidden=320, inter=192, num_experts=6, top_k=3)
+    layer = moe_synth.make_layer(shape, T=45, seed=77, device=DEV)
+    for fmt in FMTS:
+        for path in (moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL):
+            check_layer(layer, fmt, path)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_forward_nex_decode_int4(T):
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=100 + T, device=DEV)
+    check_layer(layer, "int4_g128")
+
+
+def test_forward_nex_concurrency32_zipf_int4():
+    layer = moe_synth.make_layer(moe_synth.NEX, T=32, seed=132, zipf=True, device=DEV)
+    check_layer(layer, "int4_g128")
+
+
+@pytest.mark.parametrize("zipf", [False, True])
+def test_forward_nex_prefill_8192_int4(zipf):
+    layer = moe_synth.make_layer(moe_synth.NEX, T=8192, seed=8192 + zipf, zipf=zipf, device=DEV)
+    sample = np.random.default_rng(5).choice(8192, 24, replace=False)
+    sample = np.concatenate([sample, [0, 8191]])
+    check_layer(layer, "int4_g128", sample=sample)
+
+
+@pytest.mark.parametrize("T", [4, 8192])
+def test_forward_nex_mxfp4(T):
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=4000 + T, device=DEV)
+    sample = None if T <= 32 else np.random.default_rng(6).choice(T, 24, replace=False)
+    check_layer(layer, "mxfp4", sample=sample)
+
+
+def test_prefill_and_decode_paths_agree():
+    layer = moe_synth.make_layer(moe_synth.NEX, T=24, seed=7, device=DEV)
+    a, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_DECODE)
+    b, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_PREFILL)
+    ref = b.float().cpu().numpy().astype(np.float64)
+    assert_out_close(a, ref, "decode vs prefill")
+
+
+def test_forward_routed_matches_forward():
+    layer = moe_synth.make_layer(moe_synth.NEX, T=40, seed=9, device=DEV)
+    out, dbg = run_forward(layer, "int4_g128")
+    out2, _ = run_forward(layer, "int4_g128", routed=(dbg["topk_ids_out"], dbg["topk_w_out"]))
+    # the grouped path sums expert outputs with fp32 atomics: equal up to order
+    assert_out_close(out2, out.float().cpu().numpy().astype(np.float64), "routed vs forward")
+    d1, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_DECODE)
+    d2, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_DECODE,
+                        routed=(dbg["topk_ids_out"], dbg["topk_w_out"]))
+    assert torch.equal(d1, d2)  # the decode path is deterministic
+
+
+def test_zero_tokens_is_a_no_op():
+    s = moe.make_shape(256, 64, 8, 2, "int4_g128")
+    ws = moe.alloc_workspace(s, 0)
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device=DEV)
+    r = torch.zeros(8, 256, dtype=torch.bfloat16, device=DEV)
+    gu = torch.zeros(moe.moe_packed_bytes(s, 0), dtype=torch.uint8, device=DEV)
+    dn = torch.zeros(moe.moe_packed_bytes(s, 1), dtype=torch.uint8, device=DEV)
+    out = moe.moe_forward(s, x, r, gu, dn, ws)
+    assert out.shape == (0, 256)
+
+
+# ---------------------------------------------------------------- failure reporting
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    s = moe.make_shape(256, 64, 8, 2, "int4_g128")
+    ws = moe.alloc_workspace(s, 16)
+    moe.moe_selftest_bounded_wait(ws, 20_000_000)  # 20 ms
+    assert moe.moe_workspace_status(ws) == moe.MOE_ERR_TIMEOUT
+    assert moe.moe_workspace_status(ws) == moe.MOE_OK  # reading clears it
+    layer = moe_synth.make_layer(moe_synth.TINY, T=16, seed=0, device=DEV)
+    check_layer(layer, "int4_g128")

@@ -1,0 +1,296 @@
+"""ctypes binding of libmoe_w4a16.so: argument marshalling only.
+
+Every function has the name of the C entry point it wraps and takes torch
+tensors (device memory owned by the caller) in place of raw pointers.  All
+computation happens in the library's CUDA kernels; there is no Python or CPU
+fallback.  A missing library or a non-CUDA tensor raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_w4a16.so")
+_lib = None
+
+MOE_OK = 0
+MOE_ERR_TIMEOUT = 5
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_NONFINITE"}
+
+MOE_FMT_INT4_G128 = 1
+MOE_FMT_MXFP4_G32 = 2
+FORMATS = {"int4_g128": MOE_FMT_INT4_G128, "mxfp4": MOE_FMT_MXFP4_G32}
+
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL = 0, 1, 2
+MOE_NUM_STAGES = 5
+STAGE_NAMES = ("router", "route_permute", "gate_up", "down", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("num_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("fmt", ctypes.c_int)]
+
+
+class ForwardOpts(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("topk_ids_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
+                ("logits_out", ctypes.c_void_p), ("offsets_out", ctypes.c_void_p),
+                ("sorted_rows_out", ctypes.c_void_p), ("act_out", ctypes.c_void_p),
+                ("stage_events", ctypes.c_void_p)]
+
+
+_SIGS = {
+    "moe_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_abi_version": (ctypes.c_int, []),
+    "moe_bank_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "moe_bank_scale_offset": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "moe_packed_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int]),
+    "moe_pack_int4_g128": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_pack_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_dequant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_permute_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "moe_permute": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_void_p]),
+    "moe_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int]),
+    "moe_forward": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_size_t, ctypes.c_void_p, ctypes.POINTER(ForwardOpts),
+                                   ctypes.c_void_p]),
+    "moe_forward_routed": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                          ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
+    "moe_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "moe_workspace_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64,
+                                                 ctypes.c_void_p]),
+}
+
+
+def lib():
+    """The loaded library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {_LIB_PATH} is missing "
+                               "(run `python -m weight_only_bit_router_b200.build`)")
+        handle = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _check(fn: str, status: int):
+    if status != MOE_OK:
+        raise MoeError(fn, status)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        return t  # already an address
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return stream
+
+
+def _bits(t):
+    """bf16 tensor -> the same memory (uint16 bit patterns for the C side)."""
+    if t is not None and t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected a bf16 tensor, got {t.dtype}")
+    return t
+
+
+def make_shape(hidden, inter, num_experts, top_k, fmt) -> MoeShape:
+    return MoeShape(hidden, inter, num_experts, top_k, FORMATS.get(fmt, fmt))
+
+
+# ------------------------------------------------------------------ queries
+
+def moe_abi_version() -> int:
+    return lib().moe_abi_version()
+
+
+def moe_status_str(status: int) -> str:
+    return lib().moe_status_str(status).decode()
+
+
+def moe_bank_bytes(fmt, E, N, K) -> int:
+    return lib().moe_bank_bytes(FORMATS.get(fmt, fmt), E, N, K)
+
+
+def moe_bank_scale_offset(fmt, E, N, K) -> int:
+    return lib().moe_bank_scale_offset(FORMATS.get(fmt, fmt), E, N, K)
+
+
+def moe_packed_bytes(shape: MoeShape, which: int) -> int:
+    return lib().moe_packed_bytes(ctypes.byref(shape), which)
+
+
+def moe_workspace_bytes(shape: MoeShape, T: int) -> int:
+    return lib().moe_workspace_bytes(ctypes.byref(shape), T)
+
+
+def moe_permute_workspace_bytes(T, E, k) -> int:
+    return lib().moe_permute_workspace_bytes(T, E, k)
+
+
+# ------------------------------------------------------------------ packing
+
+def _pack(name, fmt, w, packed, nonfinite, stream):
+    E, N, K = w.shape
+    if packed is None:
+        packed = torch.empty(moe_bank_bytes(fmt, E, N, K), dtype=torch.uint8, device=w.device)
+    _check(name, getattr(lib(), name)(_ptr(_bits(w)), E, N, K, _ptr(packed), _ptr(nonfinite), _stream(stream)))
+    return packed
+
+
+def moe_pack_int4_g128(w, packed=None, nonfinite=None, stream=None):
+    return _pack("moe_pack_int4_g128", MOE_FMT_INT4_G128, w, packed, nonfinite, stream)
+
+
+def moe_pack_mxfp4(w, packed=None, nonfinite=None, stream=None):
+    return _pack("moe_pack_mxfp4", MOE_FMT_MXFP4_G32, w, packed, nonfinite, stream)
+
+
+def moe_dequant(packed, fmt, E, N, K, out=None, stream=None):
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=packed.device)
+    _check("moe_dequant", lib().moe_dequant(_ptr(packed), FORMATS.get(fmt, fmt), E, N, K, _ptr(out),
+                                            _stream(stream)))
+    return out
+
+
+def split_bank(packed, fmt, E, N, K):
+    """(codes uint8 [E, N, K/2], scales) views of a packed bank (no copy)."""
+    fmt = FORMATS.get(fmt, fmt)
+    ncode = E * N * K // 2
+    off = moe_bank_scale_offset(fmt, E, N, K)
+    codes = packed[:ncode].view(E, N, K // 2)
+    if fmt == MOE_FMT_INT4_G128:
+        G = (K + 127) // 128
+        scales = packed[off:off + E * N * G * 2].view(torch.int16).view(E, N, G)
+    else:
+        scales = packed[off:off + E * N * (K // 32)].view(E, N, K // 32)
+    return codes, scales
+
+
+# ------------------------------------------------------------------ routing
+
+def moe_route(logits, k, bias=None, ids=None, weights=None, stream=None):
+    T, E = logits.shape
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if weights is None:
+        weights = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check("moe_route", lib().moe_route(_ptr(logits), _ptr(bias), T, E, k, _ptr(ids), _ptr(weights),
+                                        _stream(stream)))
+    return ids, weights
+
+
+def moe_permute(topk_ids, E, stream=None):
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_rows = torch.empty(T * k, dtype=torch.int32, device=dev)
+    pos = torch.empty(T * k, dtype=torch.int32, device=dev)
+    wsb = moe_permute_workspace_bytes(T, E, k)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    _check("moe_permute", lib().moe_permute(_ptr(topk_ids), T, E, k, _ptr(offsets), _ptr(sorted_rows), _ptr(pos),
+                                            _ptr(ws), wsb, _stream(stream)))
+    return offsets, sorted_rows, pos
+
+
+# ------------------------------------------------------------------ forward
+
+def alloc_workspace(shape: MoeShape, T: int, device="cuda", stream=None):
+    nbytes = moe_workspace_bytes(shape, T)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream=stream)
+    return ws
+
+
+def _opts(path, debug, events):
+    if path is None and not debug and events is None:
+        return None, None
+    o = ForwardOpts()
+    o.path = path or MOE_PATH_AUTO
+    for name, t in (debug or {}).items():
+        setattr(o, name, _ptr(t))
+    keep = None
+    if events is not None:
+        keep = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
+        o.stage_events = ctypes.cast(keep, ctypes.c_void_p)
+    return o, keep
+
+
+def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, workspace, out=None, bias=None,
+                path=None, debug=None, events=None, stream=None):
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
+    o, _keep = _opts(path, debug, events)
+    st = lib().moe_forward(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(_bits(router_w)), _ptr(bias),
+                           _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
+                           _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
+    _check("moe_forward", st)
+    return out
+
+
+def moe_forward_routed(shape: MoeShape, x, topk_ids, topk_w, gate_up_packed, down_packed, workspace, out=None,
+                       path=None, debug=None, events=None, stream=None):
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
+    o, _keep = _opts(path, debug, events)
+    st = lib().moe_forward_routed(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(topk_ids), _ptr(topk_w),
+                                  _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
+                                  _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
+    _check("moe_forward_routed", st)
+    return out
+
+
+def moe_workspace_init(workspace, stream=None):
+    _check("moe_workspace_init", lib().moe_workspace_init(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_workspace_status(workspace, stream=None) -> int:
+    """Synchronises the stream; returns the status code (MOE_OK or MOE_ERR_TIMEOUT)."""
+    return lib().moe_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def moe_selftest_bounded_wait(workspace, limit_ns: int, stream=None):
+    _check("moe_selftest_bounded_wait",
+           lib().moe_selftest_bounded_wait(_ptr(workspace), workspace.numel(), int(limit_ns), _stream(stream)))

@@ -1,0 +1,357 @@
+// C ABI of the W4A16 routed-expert MoE layer: argument validation, workspace
+// carve-up and the order of kernel launches on the caller's stream.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kDecodeMaxForced = 256;  // the decode path keeps [T*k, H] fp32 expert outputs
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_fmt(moe_format_t f) { return f == MOE_FMT_INT4_G128 || f == MOE_FMT_MXFP4_G32; }
+
+moe_status_t check_shape(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (!valid_fmt(s->fmt)) return MOE_ERR_INVALID_ARG;
+  if (s->hidden <= 0 || s->inter <= 0 || s->num_experts <= 0 || s->top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (s->hidden % 64 || s->inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (s->top_k > kMaxTopK || s->top_k > s->num_experts || s->num_experts > kMaxExperts)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_T(const moe_shape_t* s, int T) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (long(T) * s->top_k > (1L << 26)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                              \
+  do {                                             \
+    const moe_status_t _st = cuda_status(expr);    \
+    if (_st != MOE_OK) return _st;                 \
+  } while (0)
+
+Bank make_bank(const void* packed, moe_format_t fmt, int E, int N, int K) {
+  Bank b;
+  b.codes = static_cast<const uint8_t*>(packed);
+  b.scales = static_cast<const uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
+  b.N = N;
+  b.K = K;
+  return b;
+}
+
+// Record stage event `idx` (0 = before, 1 = after) if the caller asked for it.
+void mark(const moe_forward_opts_t* o, int stage, int after, cudaStream_t stream) {
+  if (o && o->stage_events) cudaEventRecord(o->stage_events[2 * stage + after], stream);
+}
+
+__global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    // nothing ever arrives: the wait has to give up by itself
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
+  Workspace w{};
+  const size_t R = size_t(T) * s.top_k;
+  const size_t E = s.num_experts, H = s.hidden, I = s.inter;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* r = p ? p + off : nullptr;
+    off += align_up(bytes, 256);
+    return r;
+  };
+  w.status = static_cast<uint32_t*>(take(256));
+  w.logits = static_cast<float*>(take(size_t(T) * E * 4));
+  w.topk_ids = static_cast<int32_t*>(take(R * 4));
+  w.topk_w = static_cast<float*>(take(R * 4));
+  w.offsets = static_cast<int32_t*>(take((E + 1) * 4));
+  w.sorted_rows = static_cast<int32_t*>(take(R * 4));
+  w.pos = static_cast<int32_t*>(take(R * 4));
+  w.touched = static_cast<int32_t*>(take((E + 1) * 4));
+  w.tile_base = static_cast<int32_t*>(take((E + 1) * 4));
+  w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
+  w.act = static_cast<uint16_t*>(take(R * I * 2));
+  w.y = static_cast<float*>(take(T <= kDecodeMaxForced ? R * H * 4 : 0));
+  w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
+  w.bytes = off;
+  return w;
+}
+
+cudaError_t launch_bounded_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream) {
+  bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+// Routing state (permutation + touched list + tile prefix) from ids in ws.
+moe_status_t build_permutation(const moe_shape_t& s, int T, const Workspace& ws, cudaStream_t stream) {
+  const long R = long(T) * s.top_k;
+  if (R <= 1024)
+    return cuda_status(launch_permute_small(ws.topk_ids, T, s.num_experts, s.top_k, ws.offsets, ws.sorted_rows,
+                                            ws.pos, ws.touched, ws.tile_base, kGemmBN, stream));
+  return cuda_status(launch_permute_large(ws.topk_ids, T, s.num_experts, s.top_k, ws.offsets, ws.sorted_rows,
+                                          ws.pos, ws.block_hist, ws.touched, ws.tile_base, kGemmBN, stream));
+}
+
+// Stages 2-4: experts and combine, given routing in the workspace.
+moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const void* gu_packed,
+                         const void* dn_packed, const Workspace& ws, uint16_t* out, bool decode,
+                         const moe_forward_opts_t* o, cudaStream_t stream) {
+  const Bank gu = make_bank(gu_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
+  const Bank dn = make_bank(dn_packed, s.fmt, s.num_experts, s.hidden, s.inter);
+  mark(o, 2, 0, stream);
+  if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, ws, stream));
+  else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, ws, stream));
+  mark(o, 2, 1, stream);
+  mark(o, 3, 0, stream);
+  if (decode) {
+    MOE_TRY(launch_decode_down(s, T, dn, ws, stream));
+  } else {
+    MOE_TRY(cudaMemsetAsync(ws.out_acc, 0, size_t(T) * s.hidden * 4, stream));
+    MOE_TRY(launch_grouped_down(s, T, dn, ws, stream));
+  }
+  mark(o, 3, 1, stream);
+  mark(o, 4, 0, stream);
+  if (decode) MOE_TRY(launch_decode_combine(s, T, ws, out, stream));
+  else MOE_TRY(launch_finalize_out(ws.out_acc, long(T) * s.hidden, out, stream));
+  mark(o, 4, 1, stream);
+  return MOE_OK;
+}
+
+moe_status_t copy_debug_outputs(const moe_shape_t& s, int T, const Workspace& ws, const moe_forward_opts_t* o,
+                                bool routed, cudaStream_t stream) {
+  if (!o) return MOE_OK;
+  const size_t R = size_t(T) * s.top_k;
+  auto cp = [&](void* dst, const void* src, size_t bytes) -> cudaError_t {
+    return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, stream) : cudaSuccess;
+  };
+  if (!routed) {
+    MOE_TRY(cp(o->topk_ids_out, ws.topk_ids, R * 4));
+    MOE_TRY(cp(o->topk_w_out, ws.topk_w, R * 4));
+    MOE_TRY(cp(o->logits_out, ws.logits, size_t(T) * s.num_experts * 4));
+  }
+  MOE_TRY(cp(o->offsets_out, ws.offsets, size_t(s.num_experts + 1) * 4));
+  MOE_TRY(cp(o->sorted_rows_out, ws.sorted_rows, R * 4));
+  MOE_TRY(cp(o->act_out, ws.act, R * s.inter * 2));
+  return MOE_OK;
+}
+
+moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, int T, const void* gu,
+                                  const void* dn, void* workspace, size_t ws_bytes, uint16_t* out,
+                                  const moe_forward_opts_t* opts, bool* decode) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if ((st = check_T(shape, T)) != MOE_OK) return st;
+  const moe_path_t path = opts ? opts->path : MOE_PATH_AUTO;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;  // nothing to do; pointers may be null
+  if (!x || !gu || !dn || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(gu, 256) || !aligned(dn, 256) || !aligned(out, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
+  *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  if (*decode && T > kDecodeMaxForced) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "bounded device wait expired";
+    case MOE_ERR_NONFINITE: return "non-finite input";
+  }
+  return "unknown status";
+}
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+size_t moe_bank_bytes(moe_format_t fmt, int E, int N, int K) {
+  if (!valid_fmt(fmt) || E <= 0 || N <= 0 || K <= 0 || K % 32) return 0;
+  return bank_scale_offset(fmt, E, N, K) + bank_scale_bytes(fmt, E, N, K);
+}
+
+size_t moe_bank_scale_offset(moe_format_t fmt, int E, int N, int K) {
+  if (!valid_fmt(fmt) || E <= 0 || N <= 0 || K <= 0 || K % 32) return 0;
+  return bank_scale_offset(fmt, E, N, K);
+}
+
+size_t moe_packed_bytes(const moe_shape_t* s, int which) {
+  if (check_shape(s) != MOE_OK) return 0;
+  if (which == 0) return moe_bank_bytes(s->fmt, s->num_experts, 2 * s->inter, s->hidden);
+  if (which == 1) return moe_bank_bytes(s->fmt, s->num_experts, s->hidden, s->inter);
+  return 0;
+}
+
+static moe_status_t pack_common(moe_format_t fmt, const uint16_t* w, int E, int N, int K, void* packed,
+                                int32_t* nonfinite, cudaStream_t stream) {
+  if (!w || !packed) return MOE_ERR_INVALID_ARG;
+  if (E <= 0 || N <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(packed, 256) || (nonfinite && !aligned(nonfinite, 4))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_pack(fmt, w, E, N, K, packed, nonfinite, stream));
+}
+
+moe_status_t moe_pack_int4_g128(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                                cudaStream_t stream) {
+  return pack_common(MOE_FMT_INT4_G128, w, E, N, K, packed, nonfinite, stream);
+}
+
+moe_status_t moe_pack_mxfp4(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                            cudaStream_t stream) {
+  return pack_common(MOE_FMT_MXFP4_G32, w, E, N, K, packed, nonfinite, stream);
+}
+
+moe_status_t moe_dequant(const void* packed, moe_format_t fmt, int E, int N, int K, uint16_t* w_out,
+                         cudaStream_t stream) {
+  if (!packed || !w_out || !valid_fmt(fmt)) return MOE_ERR_INVALID_ARG;
+  if (E <= 0 || N <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(packed, 256) || !aligned(w_out, 16)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_dequant(fmt, packed, E, N, K, w_out, stream));
+}
+
+moe_status_t moe_route(const float* logits, const float* bias, int T, int E, int k, int32_t* topk_ids,
+                       float* topk_w, cudaStream_t stream) {
+  if (T < 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > kMaxTopK || k > E) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) || (bias && !aligned(bias, 4)))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_topk(logits, bias, T, E, k, topk_ids, topk_w, stream));
+}
+
+size_t moe_permute_workspace_bytes(int T, int E, int k) {
+  if (T < 0 || E <= 0 || k <= 0) return 0;
+  return 4 * align_up(size_t(E + 1) * 4, 256) + align_up(permute_large_hist_bytes(T, E, k), 256) + 256;
+}
+
+moe_status_t moe_permute(const int32_t* topk_ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
+                         int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (T < 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > kMaxTopK || k > E) return MOE_ERR_UNSUPPORTED;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !sorted_rows || !pos)) return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < moe_permute_workspace_bytes(T, E, k))
+    return MOE_ERR_WORKSPACE;
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  int32_t* touched = reinterpret_cast<int32_t*>(p);
+  int32_t* tile_base = reinterpret_cast<int32_t*>(p + align_up(size_t(E + 1) * 4, 256));
+  int32_t* hist = reinterpret_cast<int32_t*>(p + 4 * align_up(size_t(E + 1) * 4, 256));
+  const long R = long(T) * k;
+  if (R <= 1024)
+    return cuda_status(
+        launch_permute_small(topk_ids, T, E, k, offsets, sorted_rows, pos, touched, tile_base, kGemmBN, stream));
+  return cuda_status(launch_permute_large(topk_ids, T, E, k, offsets, sorted_rows, pos, hist, touched, tile_base,
+                                          kGemmBN, stream));
+}
+
+size_t moe_workspace_bytes(const moe_shape_t* shape, int T) {
+  if (check_shape(shape) != MOE_OK || T < 0) return 0;
+  return carve_workspace(nullptr, *shape, T).bytes;
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, const uint16_t* router_w,
+                         const float* logit_bias, const void* gate_up_packed, const void* down_packed,
+                         void* workspace, size_t workspace_bytes, uint16_t* out, const moe_forward_opts_t* opts,
+                         cudaStream_t stream) {
+  bool decode = false;
+  moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
+                                         out, opts, &decode);
+  if (st != MOE_OK || T == 0) return st;
+  if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t& s = *shape;
+  const Workspace ws = carve_workspace(workspace, s, T);
+  mark(opts, 0, 0, stream);
+  if (T <= kDecodeMaxT)
+    MOE_TRY(launch_router_gemv(x, router_w, T, s.hidden, s.num_experts, ws.logits, stream));
+  else
+    MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
+  mark(opts, 0, 1, stream);
+  mark(opts, 1, 0, stream);
+  MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
+  if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
+  mark(opts, 1, 1, stream);
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
+  return copy_debug_outputs(s, T, ws, opts, false, stream);
+}
+
+moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int T, const int32_t* topk_ids,
+                                const float* topk_w, const void* gate_up_packed, const void* down_packed,
+                                void* workspace, size_t workspace_bytes, uint16_t* out,
+                                const moe_forward_opts_t* opts, cudaStream_t stream) {
+  bool decode = false;
+  moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
+                                         out, opts, &decode);
+  if (st != MOE_OK || T == 0) return st;
+  if (!topk_ids || !topk_w || !aligned(topk_ids, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t& s = *shape;
+  Workspace ws = carve_workspace(workspace, s, T);
+  ws.topk_ids = const_cast<int32_t*>(topk_ids);
+  ws.topk_w = const_cast<float*>(topk_w);
+  mark(opts, 1, 0, stream);
+  if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
+  mark(opts, 1, 1, stream);
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
+  return copy_debug_outputs(s, T, ws, opts, true, stream);
+}
+
+moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!workspace || workspace_bytes < 256 || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(workspace, 0, 256, stream));
+}
+
+moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!workspace || workspace_bytes < 256) return MOE_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & kStatusTimeout) {
+    if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_selftest_bounded_wait(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
+                                       cudaStream_t stream) {
+  if (!workspace || workspace_bytes < 256 || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  if (limit_ns > 10ull * 1000000000ull) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_bounded_wait_probe(static_cast<uint32_t*>(workspace), limit_ns, stream));
+}
+
+}  // extern "C"

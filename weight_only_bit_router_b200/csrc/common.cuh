@@ -1,0 +1,257 @@
+// Device helpers shared by the sm_100a kernels of the W4A16 MoE layer:
+// bf16 bit tricks, mbarriers with bounded waits, TMA and cp.async copies,
+// and thin wrappers over the tcgen05 (5th-generation tensor core) PTX.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MOE_DEV __device__ __forceinline__
+
+namespace moe {
+
+// --------------------------------------------------------------------------
+// status word shared with the host (lives in the caller's workspace)
+// --------------------------------------------------------------------------
+constexpr uint32_t kStatusTimeout = 1u;
+
+// Bounded waits give up after this many nanoseconds of device time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+MOE_DEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// --------------------------------------------------------------------------
+// bf16 helpers
+// --------------------------------------------------------------------------
+MOE_DEV float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+MOE_DEV float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+MOE_DEV float bf16_to_f32(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
+MOE_DEV uint16_t f32_to_bf16_rn(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+// two fp32 -> packed bf16x2 (lo = a), round to nearest even
+MOE_DEV uint32_t pack_bf16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+MOE_DEV uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+MOE_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  // (a & mask) | magic in one instruction
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
+  return r;
+}
+MOE_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// INT4 offset-binary nibbles -> bf16 pairs.  For a 32-bit word holding 8
+// nibbles u0..u7 (u0 lowest), int4_pairs(w, i) returns bf16x2 (u_i - 8,
+// u_{i+4} - 8) for i in 0..3: OR-ing a nibble into the mantissa of bf16 128.0
+// (0x4300) gives exactly 128 + u; subtracting 136 leaves u - 8 exactly.
+MOE_DEV uint32_t int4_pair(uint32_t w, int i) {
+  const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);
+  return bf16x2_sub(v, 0x43084308u);
+}
+
+// E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the
+// nibble pair at bit offsets 0 and 16 of `w` after shifting by 4*i.
+// Magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; looked up with two byte permutes.
+MOE_DEV uint32_t e2m1_pair(uint32_t w, int i) {
+  // high bytes of bf16(m) for m = code 0..7: 00 3F 3F 3F 40 40 40 40
+  // low bytes:                                00 00 80 C0 00 40 80 C0
+  const uint32_t hi0 = 0x3F3F3F00u, hi1 = 0x40404040u;
+  const uint32_t lo0 = 0xC0800000u, lo1 = 0xC0804000u;
+  const uint32_t s = w >> (4 * i);
+  // selector: code of the low element in nibble 0, of the high element in nibble 1
+  const uint32_t sel = (s & 0x7u) | ((s >> 12) & 0x70u);
+  const uint32_t hi = prmt(hi0, hi1, sel);   // bytes: hi(c0), hi(c1), ...
+  const uint32_t lo = prmt(lo0, lo1, sel);
+  uint32_t v = prmt(lo, hi, 0x5140u);        // lo(c0) hi(c0) lo(c1) hi(c1)
+  const uint32_t sign = ((s << 12) & 0x8000u) | ((s << 12) & 0x80000000u);
+  return v | sign;
+}
+
+// --------------------------------------------------------------------------
+// shared-memory addresses, fences
+// --------------------------------------------------------------------------
+MOE_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+MOE_DEV void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// --------------------------------------------------------------------------
+// mbarriers
+// --------------------------------------------------------------------------
+MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+MOE_DEV void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+MOE_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+MOE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity.  Gives up (returns
+// false) once `abort` is raised by another thread of the CTA or after
+// kWaitLimitNs, in which case it raises `abort` and the global status word.
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* gstatus) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 255u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        if (gstatus) atomicOr(gstatus, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// TMA (tensor memory accelerator) and cp.async
+// --------------------------------------------------------------------------
+MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+// 2-D tiled load of the box at (x, y) into shared memory; completion is
+// signalled on `bar` as transaction bytes.  x must be 16-byte aligned in bytes.
+MOE_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+MOE_DEV void cp_async_16(uint32_t smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+MOE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// --------------------------------------------------------------------------
+// tcgen05: tensor memory allocation, MMA, commit, loads
+// --------------------------------------------------------------------------
+MOE_DEV void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
+               "r"(ncols)
+               : "memory");
+}
+MOE_DEV void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+MOE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MOE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, kind::f16 (bf16 in, fp32 acc)
+MOE_DEV void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every previously issued tcgen05.mma of this thread completes.
+MOE_DEV void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, shape M x N (M = 128 here, N a multiple of 16 in [16, 256]).
+MOE_DEV uint32_t umma_idesc_bf16(uint32_t M, uint32_t N) {
+  return (1u << 4)            // D format: f32
+         | (1u << 7)          // A format: bf16
+         | (1u << 10)         // B format: bf16
+         | ((N >> 3) << 17)   // N / 8
+         | ((M >> 4) << 24);  // M / 16
+}
+
+// Shared-memory matrix descriptor for a K-major operand stored as rows of 128
+// bytes (64 bf16) with the 128-byte swizzle, 8-row groups 1024 bytes apart.
+// The tile base must be 1024-byte aligned; advancing K by 16 elements adds
+// 32 bytes to the start address.
+MOE_DEV uint64_t umma_desc_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr >> 4) & 0x3FFFu);  // start address
+  d |= uint64_t(1) << 16;                      // leading byte offset (unused for swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;              // stride byte offset: 8 rows x 128 B
+  d |= uint64_t(1) << 46;                      // descriptor version for sm_100
+  d |= uint64_t(2) << 61;                      // layout: 128-byte swizzle
+  return d;
+}
+
+// Load 32 consecutive fp32 columns of this warp's 32 TMEM lanes.
+MOE_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+MOE_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// --------------------------------------------------------------------------
+// misc
+// --------------------------------------------------------------------------
+MOE_DEV float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+MOE_DEV void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+MOE_DEV uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+}  // namespace moe

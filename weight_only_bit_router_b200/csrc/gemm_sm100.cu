@@ -1,0 +1,629 @@
+// Grouped GEMMs of the prefill path on the 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory).
+//
+// One persistent, warp-specialised kernel serves three products, all computed
+// "weights x tokens^T" so that a 128-row weight tile is the MMA's M side and
+// the tokens of one expert are its N side (N = the expert's token count
+// rounded up to 16, at most 128 per tile):
+//
+//   ROUTER   logits[t][e]   = Wr[e, :] . x[t, :]                (bf16 A by TMA)
+//   GATE_UP  act[p][f]      = bf16(silu(g_f . x_t) * (u_f . x_t)), two
+//                             accumulators (gate rows f, up rows I+f)
+//   DOWN     out_acc[t][f] += w_tj * (Wd[e, f, :] . act[p, :])
+//
+// The expert weights ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe: fused
+// banks gate_up [E, 2I, H], down [E, H, I]) arrive as packed 4-bit codes by
+// TMA, are dequantised to bf16 by a warpgroup straight into the 128-byte
+// swizzled K-major layout the MMA reads (W4A16: 4-bit weights, bf16
+// activations, "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary),
+// and the token rows of each expert are gathered by cp.async.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: code tiles (or router weight tiles)
+//   warp 1      TMEM allocation + single-thread tcgen05.mma issue
+//   warps 2-3   token-row gather (cp.async, 16 B per thread per copy)
+//   warps 4-7   dequantisation, one weight row per thread
+//   warps 8-11  epilogue, one TMEM lane (weight row) per thread
+// Every wait is bounded; an expired wait raises the workspace status word and
+// the CTA unwinds, frees its tensor memory and exits.
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+enum GemmMode { kRouter = 0, kGateUp = 1, kDown = 2 };
+
+constexpr int BM = 128;        // weight rows per tile (MMA M)
+constexpr int BN = kGemmBN;    // token columns per tile (max MMA N)
+constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int SO = 3;          // operand stages (bf16 A + gathered B)
+constexpr int SC = 4;          // code stages
+constexpr int kThreads = 384;
+constexpr int kTileBytes = BM * BK * 2;   // 16 KB bf16 operand tile
+constexpr int kCodeBytes = BM * BK / 2;   // 4 KB code tile
+
+struct GemmArgs {
+  int mode, fmt;
+  int K;                // reduction length
+  int M_total;          // rows of the weight side: E (router), I (gate_up), H (down)
+  int n_ftiles;         // weight-row tiles of 128
+  int T, top_k, I, H, E;
+  const uint16_t* bsrc;        // token operand: x [T, H] (router, gate_up) or act [T*k, I] (down)
+  const int32_t* offsets;      // [E+1]
+  const int32_t* sorted_rows;  // [T*k]
+  const int32_t* tile_base;    // [E+1] token-block prefix
+  const float* topk_w;         // [T*k]
+  const void* scales;          // scale plane of the packed bank
+  int scale_row_stride;        // scale elements per weight row
+  float* logits;
+  uint16_t* act;
+  float* out_acc;
+  uint32_t* status;
+};
+
+template <int MODE>
+struct Cfg {
+  static constexpr int NACC = MODE == kGateUp ? 2 : 1;                 // accumulators per tile
+  static constexpr uint32_t TMEM_COLS = MODE == kGateUp ? 512 : 256;   // 2 buffers x NACC x BN
+  static constexpr int SMEM_A = SO * NACC * kTileBytes;
+  static constexpr int SMEM_B = SO * kTileBytes;
+  static constexpr int SMEM_C = SC * NACC * kCodeBytes;
+  static constexpr int SMEM = SMEM_A + SMEM_B + SMEM_C + 1024 /*barriers*/ + 1024 /*align*/ +
+                             (kMaxExperts + 1) * 4;
+};
+
+struct Tile {
+  int e;        // expert (grouped modes)
+  int fb;       // weight-row tile
+  int p_begin;  // first sorted row (grouped) or first token (router)
+  int n;        // valid token columns (1..BN)
+};
+
+MOE_DEV Tile decode_tile(const GemmArgs& a, int tile, const int* s_tile_base) {
+  Tile t;
+  t.fb = tile % a.n_ftiles;
+  const int blk = tile / a.n_ftiles;
+  if (a.mode == kRouter) {
+    t.e = 0;
+    t.p_begin = blk * BN;
+    t.n = min(BN, a.T - t.p_begin);
+    return t;
+  }
+  // expert e with tile_base[e] <= blk < tile_base[e+1] (skip empty experts)
+  int lo = 0, hi = a.E;  // invariant: tile_base[lo] <= blk < tile_base[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_tile_base[mid] <= blk) lo = mid; else hi = mid;
+  }
+  t.e = lo;
+  const int tb = blk - s_tile_base[lo];
+  const int p0 = a.offsets[lo];
+  const int n_e = a.offsets[lo + 1] - p0;
+  t.p_begin = p0 + tb * BN;
+  t.n = min(BN, n_e - tb * BN);
+  return t;
+}
+
+MOE_DEV int num_tiles(const GemmArgs& a, const int* s_tile_base) {
+  if (a.mode == kRouter) return a.n_ftiles * ((a.T + BN - 1) / BN);
+  return s_tile_base[a.E] * a.n_ftiles;
+}
+
+// byte offset of 16-byte chunk c of row r inside a 128B-swizzled K-major tile
+MOE_DEV uint32_t sw128_offset(int r, int c) {
+  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+MOE_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// bf16x2 with both halves = 2^e (e in [-127, 127]).
+MOE_DEV uint32_t pow2x2(int e) {
+  const uint32_t b = e >= -126 ? uint32_t(e + 127) << 7 : 0x0040u;
+  return b | (b << 16);
+}
+
+// Dequantise 32 codes (one 16-byte chunk, k = 32*half .. +31 of the stage) of
+// one row and store them as four 16-byte bf16 chunks in swizzled layout.
+template <int FMT>
+MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint8_t* tile, int r, int half) {
+  const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t P[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t v = (FMT == MOE_FMT_INT4_G128) ? int4_pair(w[j], i) : e2m1_pair(w[j], i);
+      P[i] = bf16x2_mul(v, mult);  // (k+i, k+i+4)
+    }
+    uint4 o;
+    o.x = prmt(P[0], P[1], 0x5410u);  // k0 k1
+    o.y = prmt(P[2], P[3], 0x5410u);  // k2 k3
+    o.z = prmt(P[0], P[1], 0x7632u);  // k4 k5
+    o.w = prmt(P[2], P[3], 0x7632u);  // k6 k7
+    const int c = half * 4 + j;
+    *reinterpret_cast<uint4*>(tile + sw128_offset(r, c)) = o;
+  }
+}
+
+template <int MODE, int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const GemmArgs args) {
+  using C = Cfg<MODE>;
+  constexpr int NACC = C::NACC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                          // [SO][NACC][16 KB]
+  uint8_t* sB = sA + C::SMEM_A;                // [SO][16 KB]
+  uint8_t* sC = sB + C::SMEM_B;                // [SC][NACC][4 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::SMEM_C);
+  uint64_t* codes_full = bars;                 // [SC]
+  uint64_t* codes_empty = codes_full + SC;     // [SC]
+  uint64_t* opA_full = codes_empty + SC;       // [SO]
+  uint64_t* opB_full = opA_full + SO;          // [SO]
+  uint64_t* op_empty = opB_full + SO;          // [SO]
+  uint64_t* acc_full = op_empty + SO;          // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* drain = acc_empty + 2;             // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tile_base = reinterpret_cast<int*>(bars + 64);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GemmArgs& a = args;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SC; ++i) {
+      mbar_init(&codes_full[i], 1);
+      mbar_init(&codes_empty[i], 128);
+    }
+    for (int i = 0; i < SO; ++i) {
+      mbar_init(&opA_full[i], MODE == kRouter ? 1 : 128);
+      mbar_init(&opB_full[i], 64);
+      mbar_init(&op_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (MODE != kRouter)
+    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_tile_base[i] = a.tile_base[i];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_a);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = num_tiles(a, s_tile_base);
+  const int KS = a.K / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(a, tile, s_tile_base);
+        for (int ks = 0; ks < KS; ++ks, ++g) {
+          if (MODE == kRouter) {
+            const int s = g % SO;
+            if (!(ok = mbar_wait(&op_empty[s], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+            mbar_arrive_expect_tx(&opA_full[s], kTileBytes);
+            tma_load_2d(sA + s * NACC * kTileBytes, &tmap_a, &opA_full[s], ks * BK, t.fb * BM);
+          } else {
+            const int s = g % SC;
+            if (!(ok = mbar_wait(&codes_empty[s], ((g / SC) & 1) ^ 1, abort, a.status))) break;
+            mbar_arrive_expect_tx(&codes_full[s], NACC * kCodeBytes);
+            uint8_t* dst = sC + s * NACC * kCodeBytes;
+            if (MODE == kGateUp) {
+              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.e);
+              tma_load_3d(dst + kCodeBytes, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.e + 1);
+            } else {
+              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, t.e);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA unwinds
+        volatile int never = 0;
+        for (uint32_t i = 0; i < (MODE == kRouter ? SO : SC) && i < g; ++i) {
+          const uint32_t gg = g - 1 - i;
+          if (MODE == kRouter)
+            mbar_wait(&opA_full[gg % SO], (gg / SO) & 1, &never, nullptr);
+          else
+            mbar_wait(&codes_full[gg % SC], (gg / SC) & 1, &never, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+        const Tile t = decode_tile(a, tile, s_tile_base);
+        const int buf = it & 1;
+        if (!(ok = mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, a.status))) break;
+        tc_fence_after();
+        const uint32_t n16 = uint32_t((t.n + 15) & ~15);
+        const uint32_t idesc = umma_idesc_bf16(BM, n16);
+        const uint32_t d0 = tmem_base + uint32_t(buf * NACC * BN);
+        for (int ks = 0; ks < KS; ++ks, ++g) {
+          const int s = g % SO;
+          if (!(ok = mbar_wait(&opA_full[s], (g / SO) & 1, abort, a.status))) break;
+          if (!(ok = mbar_wait(&opB_full[s], (g / SO) & 1, abort, a.status))) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + s * NACC * kTileBytes);
+          const uint32_t b_addr = smem_u32(sB + s * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = umma_desc_sw128(b_addr + kk * 32);
+#pragma unroll
+            for (int c = 0; c < NACC; ++c) {
+              const uint64_t adesc = umma_desc_sw128(a_addr + c * kTileBytes + kk * 32);
+              umma_bf16(d0 + c * BN, adesc, bdesc, idesc, (ks | kk) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&op_empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+      }
+      if (!ok) {
+        volatile int never = 0;
+        umma_commit(drain);
+        mbar_wait(drain, 0, &never, nullptr);
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ token gather
+    // Copies of stage g are issued before stage g-2 is released, so two
+    // stages of 16-byte copies are in flight per thread.
+    constexpr uint32_t LAG = SO - 1;
+    const int lt = threadIdx.x - 64;  // 0..63
+    const int c = lt & 7;             // 16-byte chunk of the 128-byte row slice
+    const int r0 = lt >> 3;           // rows r0, r0+8, ..., r0+120
+    uint32_t g = 0, released = 0;
+    bool ok = true;
+    const int ld = (MODE == kDown) ? a.I : a.H;  // row length of the token operand
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const Tile t = decode_tile(a, tile, s_tile_base);
+      const int n16 = (t.n + 15) & ~15;
+      const uint16_t* src[BN / 8];
+#pragma unroll
+      for (int i = 0; i < BN / 8; ++i) {
+        const int r = r0 + 8 * i;
+        long row;
+        if (MODE == kGateUp) row = a.sorted_rows[t.p_begin + (r < t.n ? r : 0)] / a.top_k;
+        else row = t.p_begin + (r < t.n ? r : 0);
+        src[i] = a.bsrc + row * ld + c * 8;
+      }
+      for (int ks = 0; ks < KS; ++ks, ++g) {
+        const int s = g % SO;
+        if (!(ok = mbar_wait(&op_empty[s], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+        const uint32_t base = smem_u32(sB + s * kTileBytes);
+#pragma unroll
+        for (int i = 0; i < BN / 8; ++i) {
+          const int r = r0 + 8 * i;
+          if (r < n16) cp_async_16(base + sw128_offset(r, c), src[i] + ks * BK);
+        }
+        cp_async_commit();
+        if (g + 1 - released > LAG) {
+          cp_async_wait<LAG>();
+          fence_proxy_async_smem();
+          mbar_arrive(&opB_full[released % SO]);
+          ++released;
+        }
+      }
+    }
+    cp_async_wait<0>();
+    if (ok) {
+      fence_proxy_async_smem();
+      for (; released < g; ++released) mbar_arrive(&opB_full[released % SO]);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ dequantisation
+    if (MODE != kRouter) {
+      const int r = threadIdx.x - 128;  // weight row inside the tile
+      uint32_t g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(a, tile, s_tile_base);
+        const int f = t.fb * BM + r;
+        const bool valid = f < a.M_total;
+        long srow[NACC];
+        if (MODE == kGateUp) {
+          srow[0] = long(t.e) * 2 * a.I + f;
+          if (NACC > 1) srow[NACC - 1] = long(t.e) * 2 * a.I + a.I + f;
+        } else {
+          srow[0] = long(t.e) * a.H + f;
+        }
+        for (int ks = 0; ks < KS; ++ks, ++g) {
+          const int sc = g % SC, so = g % SO;
+          if (!(ok = mbar_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
+          if (!(ok = mbar_wait(&op_empty[so], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+#pragma unroll
+          for (int c = 0; c < NACC; ++c) {
+            const uint8_t* ctile = sC + (sc * NACC + c) * kCodeBytes + r * (BK / 2);
+            const uint4 c0 = *reinterpret_cast<const uint4*>(ctile);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + 16);
+            uint32_t m0 = 0, m1 = 0;
+            if (valid) {
+              if (FMT == MOE_FMT_INT4_G128) {
+                const uint32_t s = static_cast<const uint16_t*>(a.scales)[srow[c] * a.scale_row_stride +
+                                                                          (ks * BK) / 128];
+                m0 = m1 = s | (s << 16);
+              } else {
+                const uint8_t* sp = static_cast<const uint8_t*>(a.scales) + srow[c] * a.scale_row_stride +
+                                    (ks * BK) / 32;
+                m0 = pow2x2(int(sp[0]) - 127);
+                m1 = pow2x2(int(sp[1]) - 127);
+              }
+            }
+            uint8_t* atile = sA + (so * NACC + c) * kTileBytes;
+            dequant_store32<FMT>(c0, m0, atile, r, 0);
+            dequant_store32<FMT>(c1, m1, atile, r, 1);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&opA_full[so]);
+          mbar_arrive(&codes_empty[sc]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 8;          // TMEM lanes 32*ew .. 32*ew+31
+    const int r = ew * 32 + lane;     // weight row inside the tile
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      const Tile t = decode_tile(a, tile, s_tile_base);
+      const int buf = it & 1;
+      if (!(ok = mbar_wait(&acc_full[buf], (it >> 1) & 1, abort, a.status))) break;
+      tc_fence_after();
+      const int f = t.fb * BM + r;
+      const bool row_ok = f < a.M_total;
+      const uint32_t taddr = tmem_base + (uint32_t(ew * 32) << 16) + uint32_t(buf * NACC * BN);
+      for (int c0 = 0; c0 < t.n; c0 += 32) {
+        uint32_t v0[32];
+        tmem_ld32(taddr + c0, v0);
+        if (MODE == kGateUp) {
+          uint32_t v1[32];
+          tmem_ld32(taddr + BN + c0, v1);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < t.n)
+                a.act[size_t(t.p_begin + c0 + j) * a.I + f] =
+                    f32_to_bf16_rn(silu_mul(__uint_as_float(v0[j]), __uint_as_float(v1[j])));
+            }
+          }
+        } else if (MODE == kDown) {
+          tmem_ld_wait();
+          // routing of the 32 columns: lane j fetches column c0 + j
+          int tok = 0;
+          float wgt = 0.f;
+          if (c0 + lane < t.n) {
+            const int rr = a.sorted_rows[t.p_begin + c0 + lane];
+            tok = rr / a.top_k;
+            wgt = a.topk_w[rr];
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tj = __shfl_sync(0xffffffffu, tok, j);
+            const float wj = __shfl_sync(0xffffffffu, wgt, j);
+            if (row_ok && c0 + j < t.n) red_add_f32(a.out_acc + size_t(tj) * a.H + f, wj * __uint_as_float(v0[j]));
+          }
+        } else {
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < t.n) a.logits[size_t(t.p_begin + c0 + j) * a.E + f] = __uint_as_float(v0[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// fp32 accumulator -> bf16 output
+__global__ void finalize_kernel(const float* __restrict__ acc, long n, uint16_t* __restrict__ out) {
+  const long i = (long(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i >= n) return;
+  const float4 v = *reinterpret_cast<const float4*>(acc + i);
+  uint2 o;
+  o.x = pack_bf16x2(v.x, v.y);
+  o.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(out + i) = o;
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launches
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Codes of a packed bank viewed as [Z][rows][K/2] bytes, box 32 bytes x 128 rows.
+bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int K, int rows, long Z) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(K / 2), cuuint64_t(rows), cuuint64_t(Z)};
+  const cuuint64_t strides[2] = {cuuint64_t(K / 2), cuuint64_t(K / 2) * rows};
+  const cuuint32_t box[3] = {BK / 2, BM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows][K] with the 128-byte swizzle, box 64 x 128.
+bool make_bf16_sw128_map(CUtensorMap* m, const uint16_t* base, int K, int rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int MODE, int FMT>
+cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ctas, cudaStream_t stream) {
+  auto kern = grouped_gemm_kernel<MODE, FMT>;
+  const int smem = Cfg<MODE>::SMEM;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const int grid = max(1, min(sm_count(), max_ctas));
+  kern<<<grid, kThreads, smem, stream>>>(map, args);
+  return cudaGetLastError();
+}
+
+GemmArgs base_args(const moe_shape_t& s, int T, const Workspace& ws) {
+  GemmArgs a{};
+  a.fmt = int(s.fmt);
+  a.T = T;
+  a.top_k = s.top_k;
+  a.I = s.inter;
+  a.H = s.hidden;
+  a.E = s.num_experts;
+  a.offsets = ws.offsets;
+  a.sorted_rows = ws.sorted_rows;
+  a.tile_base = ws.tile_base;
+  a.topk_w = ws.topk_w;
+  a.logits = ws.logits;
+  a.act = ws.act;
+  a.out_acc = ws.out_acc;
+  a.status = ws.status;
+  return a;
+}
+
+// Upper bound of the grouped tile count (host side, no device read): every
+// row in its own expert's partial block, bounded by the full count.
+int grouped_tiles_bound(int T, int k, int E, int ftiles) {
+  const long rows = long(T) * k;
+  const long blocks = (rows + BN - 1) / BN + std::min<long>(E, rows);
+  return int(std::min<long>(blocks * ftiles, 1L << 30));
+}
+
+}  // namespace
+
+cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
+                               uint32_t* status, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  CUtensorMap map;
+  if (!make_bf16_sw128_map(&map, wr, H, E)) return cudaErrorInvalidValue;
+  GemmArgs a{};
+  a.mode = kRouter;
+  a.K = H;
+  a.M_total = E;
+  a.n_ftiles = (E + BM - 1) / BM;
+  a.T = T;
+  a.H = H;
+  a.E = E;
+  a.bsrc = x;
+  a.logits = logits;
+  a.status = status;
+  const int tiles = a.n_ftiles * ((T + BN - 1) / BN);
+  return launch_gemm<kRouter, 0>(map, a, tiles, stream);
+}
+
+cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
+                                   const Workspace& ws, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  CUtensorMap map;
+  if (!make_codes_map(&map, gu.codes, gu.K, s.inter, 2L * s.num_experts)) return cudaErrorInvalidValue;
+  GemmArgs a = base_args(s, T, ws);
+  a.mode = kGateUp;
+  a.K = s.hidden;
+  a.M_total = s.inter;
+  a.n_ftiles = (s.inter + BM - 1) / BM;
+  a.bsrc = x;
+  a.scales = gu.scales;
+  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(gu.K) : gu.K / 32;
+  const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
+  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kGateUp, MOE_FMT_INT4_G128>(map, a, bound, stream);
+  return launch_gemm<kGateUp, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
+}
+
+cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
+                                cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  CUtensorMap map;
+  if (!make_codes_map(&map, dn.codes, dn.K, s.hidden, s.num_experts)) return cudaErrorInvalidValue;
+  GemmArgs a = base_args(s, T, ws);
+  a.mode = kDown;
+  a.K = s.inter;
+  a.M_total = s.hidden;
+  a.n_ftiles = (s.hidden + BM - 1) / BM;
+  a.bsrc = ws.act;
+  a.scales = dn.scales;
+  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(dn.K) : dn.K / 32;
+  const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
+  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kDown, MOE_FMT_INT4_G128>(map, a, bound, stream);
+  return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
+}
+
+cudaError_t launch_finalize_out(const float* acc, long n, uint16_t* out, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int block = 256;
+  const long threads = (n + 3) / 4;
+  finalize_kernel<<<unsigned((threads + block - 1) / block), block, 0, stream>>>(acc, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

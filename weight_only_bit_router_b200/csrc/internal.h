@@ -1,0 +1,100 @@
+// Internal declarations shared by the host dispatcher (api.cu) and the kernel
+// translation units.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_w4a16.h"
+
+namespace moe {
+
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+constexpr int kDecodeMaxT = 32;  // MOE_PATH_AUTO switches to the grouped GEMMs above this
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t bank_codes_bytes(int E, int N, int K) { return size_t(E) * N * (K / 2); }
+__host__ __device__ inline int int4_groups(int K) { return (K + 127) / 128; }
+inline size_t bank_scale_offset(moe_format_t fmt, int E, int N, int K) {
+  (void)fmt;
+  return align_up(bank_codes_bytes(E, N, K), 256);
+}
+inline size_t bank_scale_bytes(moe_format_t fmt, int E, int N, int K) {
+  return fmt == MOE_FMT_INT4_G128 ? size_t(E) * N * int4_groups(K) * 2 : size_t(E) * N * (K / 32);
+}
+
+// Device view of one packed bank.
+struct Bank {
+  const uint8_t* codes;  // [E][N][K/2]
+  const void* scales;    // INT4: bf16 [E][N][G]; MXFP4: u8 [E][N][K/32]
+  int N, K;
+};
+
+// Workspace carve-up for T tokens (all offsets 256-byte aligned).
+struct Workspace {
+  uint32_t* status;       // [64] status word + scratch counters
+  float* logits;          // [T, E]
+  int32_t* topk_ids;      // [T, k]
+  float* topk_w;          // [T, k]
+  int32_t* offsets;       // [E+1]
+  int32_t* sorted_rows;   // [T*k]
+  int32_t* pos;           // [T*k]
+  int32_t* touched;       // [E+1]: number of experts with rows, then their ids ascending
+  int32_t* tile_base;     // [E+1]: prefix of per-expert token blocks (grouped GEMMs)
+  int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
+  uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
+  float* y;               // [T*k, H] fp32 expert outputs (decode path)
+  float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
+  size_t bytes;
+};
+
+Workspace carve_workspace(void* base, const moe_shape_t& s, int T);
+size_t permute_block_rows();
+
+// pack.cu
+cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K, void* packed,
+                        int32_t* nonfinite, cudaStream_t stream);
+cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, int K, uint16_t* out,
+                           cudaStream_t stream);
+
+// route.cu
+cudaError_t launch_router_gemv(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
+                               cudaStream_t stream);
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
+                        cudaStream_t stream);
+// Small-T routing state: permutation + touched-expert list in one CTA.
+cudaError_t launch_permute_small(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
+                                 int32_t* pos, int32_t* touched, int32_t* tile_base, int block_n,
+                                 cudaStream_t stream);
+// Any-T permutation (three kernels) + tile prefix for the grouped GEMMs.
+cudaError_t launch_permute_large(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
+                                 int32_t* pos, int32_t* block_hist, int32_t* touched, int32_t* tile_base,
+                                 int block_n, cudaStream_t stream);
+size_t permute_large_hist_bytes(int T, int E, int k);
+
+// decode.cu
+cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
+                                  const Workspace& ws, cudaStream_t stream);
+cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
+                               cudaStream_t stream);
+cudaError_t launch_decode_combine(const moe_shape_t& s, int T, const Workspace& ws, uint16_t* out,
+                                  cudaStream_t stream);
+
+// gemm_sm100.cu
+constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
+cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
+                               uint32_t* status, cudaStream_t stream);
+cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
+                                   const Workspace& ws, cudaStream_t stream);
+cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
+                                cudaStream_t stream);
+cudaError_t launch_finalize_out(const float* acc, long n, uint16_t* out, cudaStream_t stream);
+
+// selftest of the bounded device-side wait (api.cu)
+cudaError_t launch_bounded_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace moe

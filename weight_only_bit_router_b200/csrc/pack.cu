@@ -1,0 +1,193 @@
+// Packing of bf16 expert banks into the two 4-bit formats, and the debug
+// dequantiser.  One warp quantises 128 consecutive K elements of one row
+// (one INT4 group, or four MXFP4 blocks); each lane owns 4 elements.
+//
+// INT4: "Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe (symmetric, group 128,
+//       round-to-nearest with min-max scales).
+// MXFP4: "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary and
+//       Quantization method (E2M1 codes, E8M0 scale per 32 elements,
+//       exponent floor(log2(amax / 6))).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+// One warp per (row, 128-column chunk).  Lane l owns columns c0+4l .. c0+4l+3.
+__global__ void __launch_bounds__(256) pack_int4_kernel(const uint16_t* __restrict__ w, long rows, int K,
+                                                        uint8_t* __restrict__ codes, uint16_t* __restrict__ scales,
+                                                        int32_t* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  const int G = (K + 127) / 128;
+  const long task = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (task >= rows * G) return;
+  const long row = task / G;
+  const int g = int(task % G);
+  const int col = g * 128 + lane * 4;
+  const bool active = col < K;  // K % 4 == 0: a lane is wholly in or out
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(w + row * K + col);
+    v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
+  }
+  float amax = 0.f;
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bad |= !isfinite(v[i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (bad && nonfinite) atomicAdd(nonfinite, 1);
+  // s = bf16(fp32(amax) / 7): the group max maps to +-7
+  const uint16_t s_bits = f32_to_bf16_rn(__fdiv_rn(amax, 7.0f));
+  const float s = bf16_to_f32(s_bits);
+  if (!active) return;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int q = 0;
+    if (s != 0.f) q = max(-8, min(7, __float2int_rn(__fdiv_rn(v[i], s))));
+    packed |= uint32_t(q + 8) << (4 * i);
+  }
+  *reinterpret_cast<uint16_t*>(codes + row * (K / 2) + col / 2) = uint16_t(packed);
+  if (lane == 0) scales[row * G + g] = s_bits;
+}
+
+// E2M1 magnitude code of a non-negative fp32 v: nearest of {0,.5,1,1.5,2,3,4,6},
+// ties to the even code, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1_code(float a) {
+  if (a <= 0.25f) return 0;
+  if (a < 0.75f) return 1;
+  if (a <= 1.25f) return 2;
+  if (a < 1.75f) return 3;
+  if (a <= 2.5f) return 4;
+  if (a < 3.5f) return 5;
+  if (a <= 5.0f) return 6;
+  return 7;
+}
+
+// floor(log2(amax / 6)) for amax > 0, computed exactly from the fp32 bits:
+// amax = m * 2^E with m in [1, 2); 6 * 2^(E-2) <= amax iff m >= 1.5.
+__device__ __forceinline__ int mx_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int bias = 0;
+  if (amax < 1e-30f) { amax *= 18446744073709551616.0f; bias = 64; }  // 2^64, exact
+  const uint32_t b = __float_as_uint(amax);
+  const int E = int((b >> 23) & 0xFF) - 127 - bias;
+  const int e = ((b & 0x7FFFFF) >= 0x400000u) ? E - 2 : E - 3;
+  return max(-127, min(127, e));
+}
+
+// 2^p as fp32 for p in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float exp2i(int p) {
+  return p >= -126 ? __uint_as_float(uint32_t(p + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// One warp per (row, 128 columns) = 4 MXFP4 blocks; lanes 8b..8b+7 own block b.
+__global__ void __launch_bounds__(256) pack_mxfp4_kernel(const uint16_t* __restrict__ w, long rows, int K,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                         int32_t* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  const int C = (K + 127) / 128;
+  const long task = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (task >= rows * C) return;
+  const long row = task / C;
+  const int col = int(task % C) * 128 + lane * 4;
+  const bool active = col < K;  // K % 32 == 0: a block of 8 lanes is wholly in or out
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(w + row * K + col);
+    v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
+  }
+  float amax = 0.f;
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bad |= !isfinite(v[i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (bad && nonfinite) atomicAdd(nonfinite, 1);
+  if (!active) return;
+  const int e = mx_exponent(amax);
+  const float inv = exp2i(-e);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x = v[i] * inv;  // exact whenever it matters (|x| >= 2^-126)
+    const uint32_t c = e2m1_code(fabsf(x));
+    const uint32_t sgn = (v[i] < 0.f && c != 0) ? 8u : 0u;
+    packed |= (sgn | c) << (4 * i);
+  }
+  *reinterpret_cast<uint16_t*>(codes + row * (K / 2) + col / 2) = uint16_t(packed);
+  if ((lane & 7) == 0) scales[row * (K / 32) + col / 32] = uint8_t(e + 127);
+}
+
+// Debug dequantiser: one thread per code byte (two elements).
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales, int fmt,
+                               long rows, int K, uint16_t* __restrict__ out) {
+  const long i = long(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long nbytes = rows * (K / 2);
+  if (i >= nbytes) return;
+  const long row = i / (K / 2);
+  const int col = int(i % (K / 2)) * 2;
+  const uint32_t byte = codes[i];
+  uint16_t r[2];
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t nib = (byte >> (4 * h)) & 15u;
+    const int k = col + h;
+    float val;
+    if (fmt == MOE_FMT_INT4_G128) {
+      const int G = (K + 127) / 128;
+      const float s = bf16_to_f32(static_cast<const uint16_t*>(scales)[row * G + k / 128]);
+      val = float(int(nib) - 8) * s;  // exact in fp32, rounded once below
+    } else {
+      const int e = int(static_cast<const uint8_t*>(scales)[row * (K / 32) + k / 32]) - 127;
+      const float mags[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+      val = mags[nib & 7u] * exp2i(e);  // exact (subnormal products included)
+      if (nib & 8u) val = -val;
+    }
+    r[h] = f32_to_bf16_rn(val);
+  }
+  *reinterpret_cast<uint32_t*>(out + row * K + col) = uint32_t(r[0]) | (uint32_t(r[1]) << 16);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K, void* packed,
+                        int32_t* nonfinite, cudaStream_t stream) {
+  const long rows = long(E) * N;
+  const long chunks = rows * ((K + 127) / 128);
+  const long threads = chunks * 32;
+  const int block = 256;
+  const long grid = (threads + block - 1) / block;
+  uint8_t* codes = static_cast<uint8_t*>(packed);
+  void* scales = static_cast<uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
+  if (grid == 0) return cudaSuccess;
+  if (fmt == MOE_FMT_INT4_G128)
+    pack_int4_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, rows, K, codes, static_cast<uint16_t*>(scales),
+                                                                 nonfinite);
+  else
+    pack_mxfp4_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, rows, K, codes, static_cast<uint8_t*>(scales),
+                                                                  nonfinite);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, int K, uint16_t* out,
+                           cudaStream_t stream) {
+  const long rows = long(E) * N;
+  const long nbytes = rows * (K / 2);
+  if (nbytes == 0) return cudaSuccess;
+  const int block = 256;
+  const long grid = (nbytes + block - 1) / block;
+  const uint8_t* codes = static_cast<const uint8_t*>(packed);
+  const void* scales = static_cast<const uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
+  dequant_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(codes, scales, int(fmt), rows, K, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
