@@ -1,0 +1,538 @@
+"""Benchmark of the W4A16 routed-expert MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Workloads (Qwen3.5-MoE expert layer: hidden 2048, 256 experts, top-8, expert
+intermediate 512; synthetic seeded inputs, random-init weights):
+  decode4   (default) INT4 g128, 4 tokens per layer, a stack of 40 layers with
+            independently seeded weights (16.6 GB packed); one step = one CUDA
+            graph replay of moe_forward over all 40 layers on the same tokens
+  decode1   the same with 1 token
+  c32       INT4, 32 tokens with a Zipf(1.1) expert-popularity logit bias
+  prefill   INT4, 8192 tokens, one step = one layer (rotating over 40 layers)
+  prefill_zipf  the same with the Zipf logit bias
+  mx_decode4 / mx_prefill   the MXFP4 stack (17.1 GB packed) at 4 / 8192 tokens
+
+The metric is MoE-layer tokens per second: tokens x layers processed per
+second of device time, whole job (all ranks).  With --gpus N > 1 (launched by
+torch.distributed.run) every rank runs its own replica of the stack on its own
+tokens (data parallel, weak scaling); the only collective is the max-over-ranks
+reduction of the timed region.
+
+The JSON line carries the roofline of the dominant kernel (measured live with
+CUDA events around each stage inside a captured graph), the CPU oracle timed on
+a bounded sample (cpu_baseline), an end-to-end number through the host API
+with host<->device copies in the timed region (e2e), and the SM clocks sampled
+by nvidia-smi during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import moe_synth  # noqa: E402
+
+NUM_LAYERS = 40
+WORKLOADS = {
+    # name: (fmt, T, zipf, layers per step)
+    "decode4": ("int4_g128", 4, False, NUM_LAYERS),
+    "decode1": ("int4_g128", 1, False, NUM_LAYERS),
+    "c32": ("int4_g128", 32, True, NUM_LAYERS),
+    "prefill": ("int4_g128", 8192, False, 1),
+    "prefill_zipf": ("int4_g128", 8192, True, 1),
+    "mx_decode4": ("mxfp4", 4, False, NUM_LAYERS),
+    "mx_prefill": ("mxfp4", 8192, False, 1),
+}
+METRIC = "W4A16 MoE-layer tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    """(rank, local_rank, world_size) from the torchrun environment."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def dist_init(backend: str):
+    rank, local, world = dist_env()
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity on one process)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def rank_token_seed(rank: int, T: int) -> int:
+    """Each rank processes its own tokens (weak scaling): a distinct seed per rank."""
+    return 500_000 + 1000 * rank + T
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, period_ms: int = 100):
+        self.gpu_id, self.period_ms, self.proc = gpu_id, period_ms, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the layer stack
+
+class Stack:
+    """L layers of packed expert banks + bf16 router weights on one GPU."""
+
+    def __init__(self, moe, fmt: str, layers: int, device, zipf: bool):
+        s = moe_synth.NEX
+        self.moe, self.fmt, self.L = moe, fmt, layers
+        self.shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
+        gu_b, dn_b = moe.moe_packed_bytes(self.shape, 0), moe.moe_packed_bytes(self.shape, 1)
+        self.gate_up = torch.empty(layers, gu_b, dtype=torch.uint8, device=device)
+        self.down = torch.empty(layers, dn_b, dtype=torch.uint8, device=device)
+        self.router = torch.empty(layers, s.num_experts, s.hidden, dtype=torch.bfloat16, device=device)
+        self.bias = [moe_synth.zipf_bias(s, moe_synth.SEED_STACK_BASE + l).to(device) if zipf else None
+                     for l in range(layers)]
+        pack = moe.moe_pack_int4_g128 if fmt == "int4_g128" else moe.moe_pack_mxfp4
+        for l in range(layers):
+            seed = moe_synth.SEED_STACK_BASE + l
+            w = moe_synth.gate_up_bank(s, seed, device)
+            pack(w, packed=self.gate_up[l])
+            del w
+            w = moe_synth.down_bank(s, seed, device)
+            pack(w, packed=self.down[l])
+            del w
+            self.router[l].copy_(moe_synth.router_weight(s, seed, device))
+        torch.cuda.synchronize()
+        self.packed_bytes = (gu_b + dn_b) * layers
+
+    def layer_bf16(self, l: int):
+        """The bf16 source of layer l (regenerated from its seed; for the oracle)."""
+        s = moe_synth.NEX
+        seed = moe_synth.SEED_STACK_BASE + l
+        dev = self.gate_up.device
+        return moe_synth.gate_up_bank(s, seed, dev), moe_synth.down_bank(s, seed, dev)
+
+
+def capture_graph(fn):
+    """Capture fn() (a sequence of enqueues on the current stream) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm-up outside capture (also loads kernels)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def gate_up_bytes_per_expert(moe, shape):
+    return moe.moe_packed_bytes(shape, 0) // shape.num_experts
+
+
+def down_bytes_per_expert(moe, shape):
+    return moe.moe_packed_bytes(shape, 1) // shape.num_experts
+
+
+def stage_work(moe, shape, T: int, touched: float):
+    """Algorithmic bytes (decode) and flops (prefill) per layer-launch of each stage.
+
+    bytes: packed weights of the touched experts streamed once + activations in/out;
+    flops: 2 * rows * (2I*H) for gate_up, 2 * rows * (H*I) for down, 2*T*E*H router."""
+    H, I, E, k = shape.hidden, shape.inter, shape.num_experts, shape.top_k
+    R = T * k
+    return {
+        "router": {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H},
+        "gate_up": {"bytes": touched * gate_up_bytes_per_expert(moe, shape) + T * H * 2 + R * I * 2,
+                    "flops": 2 * R * 2 * I * H},
+        "down": {"bytes": touched * down_bytes_per_expert(moe, shape) + R * I * 2 + R * H * 4,
+                 "flops": 2 * R * H * I},
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, slots_per_token=None):
+    """Time the CPU oracle on a bounded sample of the workload.
+
+    Inputs (bf16 weights of the touched experts, packed by the oracle's own
+    packer) are prepared untimed; the timed part is the oracle's forward of
+    the sampled tokens: router logits, top-k, dequantisation of every touched
+    expert (cold), SwiGLU experts and the weighted combine.  Returns
+    (layer-tokens per second, description, threads)."""
+    from oracle import moe_oracle as o
+    from threadpoolctl import threadpool_info
+    fmt = o.FMT_INT4 if stack.fmt == "int4_g128" else o.FMT_MXFP4
+    E, k = stack.shape.num_experts, stack.shape.top_k
+    done_tokens, elapsed, used_layers = 0.0, 0.0, 0
+    xb_all = moe_synth.bf16_bits(x_bf16)
+    for l in range(min(max_layers, stack.L)):
+        if elapsed >= budget_s:
+            break
+        router = moe_synth.bf16_bits(stack.router[l])
+        b = None if bias[l] is None else bias[l].cpu().numpy()
+        ntok = min(T, 16)  # the oracle runs at most 16 tokens of a layer per sample
+        xb = xb_all[:ntok]
+        ids, _ = o.route(o.router_logits(xb, router), b, k)
+        touched = sorted(set(int(e) for e in ids.reshape(-1)))
+        gu_bf16, dn_bf16 = stack.layer_bf16(l)
+        gu_c, gu_s, dn_c, dn_s = {}, {}, {}, {}
+        for e in touched:
+            gu_c[e], gu_s[e] = o.pack(fmt, moe_synth.bf16_bits(gu_bf16[e]))
+            dn_c[e], dn_s[e] = o.pack(fmt, moe_synth.bf16_bits(dn_bf16[e]))
+        del gu_bf16, dn_bf16
+        gu = o.PackedBank(fmt, gu_c, gu_s)
+        dn = o.PackedBank(fmt, dn_c, dn_s)
+        t0 = time.perf_counter()
+        o.forward(xb, router, b, gu, dn, k)
+        elapsed += time.perf_counter() - t0
+        done_tokens += ntok
+        used_layers += 1
+    threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    desc = (f"CPU oracle (NumPy fp64) forward of {int(done_tokens)} token-layers "
+            f"({used_layers} layer(s) x up to 16 tokens of this workload, cold dequantisation of every touched "
+            f"expert; packing untimed)")
+    return done_tokens / max(elapsed, 1e-9), desc, int(threads), elapsed
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, local, world):
+    import weight_only_bit_router_b200 as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    fmt, T, zipf, layers_per_step = WORKLOADS[args.workload]
+    L = NUM_LAYERS
+    stack = Stack(moe, fmt, L, device, zipf)
+    shape = stack.shape
+    x = moe_synth.hidden_states(moe_synth.NEX, T, rank_token_seed(rank, T), device)
+    ws = moe.alloc_workspace(shape, T, device)
+    outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+    path = moe.MOE_PATH_AUTO
+
+    def layer_call(l, events=None):
+        moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
+                        bias=stack.bias[l], path=path, events=events, stream=torch.cuda.current_stream())
+
+    # one step: layers_per_step consecutive layers; graphs rotate over the stack
+    n_graphs = L // layers_per_step
+    graphs = []
+    for gi in range(n_graphs):
+        ls = list(range(gi * layers_per_step, (gi + 1) * layers_per_step))
+        graphs.append(capture_graph(lambda ls=ls: [layer_call(l) for l in ls]))
+    assert moe.moe_workspace_status(ws) == moe.MOE_OK
+
+    def step(i):
+        graphs[i % n_graphs].replay()
+
+    # warm-up
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+    ms_local = start.elapsed_time(end)
+    ms = reduce_max(ms_local, device)
+    tokens_per_step = T * layers_per_step
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    status = moe.moe_workspace_status(ws)
+
+    # ---- instrumented pass: per-stage device time inside a captured graph
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * moe.MOE_NUM_STAGES)] for _ in range(L)]
+    for evs in ev:
+        for e in evs:
+            e.record(stream)  # materialise the events before capture
+    torch.cuda.synchronize()
+    inst_graphs = []
+    for gi in range(n_graphs):
+        ls = list(range(gi * layers_per_step, (gi + 1) * layers_per_step))
+        inst_graphs.append(capture_graph(lambda ls=ls: [layer_call(l, ev[l]) for l in ls]))
+    stage_ms = {n: [] for n in moe.STAGE_NAMES}
+    reps = max(1, min(20, args.steps))
+    for r in range(reps):
+        inst_graphs[r % n_graphs].replay()
+        torch.cuda.synchronize()
+        gi = r % n_graphs
+        for l in range(gi * layers_per_step, (gi + 1) * layers_per_step):
+            for si, n in enumerate(moe.STAGE_NAMES):
+                stage_ms[n].append(ev[l][2 * si].elapsed_time(ev[l][2 * si + 1]))
+    stage_avg = {n: float(np.mean(v)) for n, v in stage_ms.items()}
+
+    # touched experts per layer (from the routing of each layer)
+    touched = []
+    ids_buf = torch.empty(T, shape.top_k, dtype=torch.int32, device=device)
+    for l in range(L):
+        moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
+                        bias=stack.bias[l], debug={"topk_ids_out": ids_buf})
+        touched.append(len(torch.unique(ids_buf)))
+    avg_touched = float(np.mean(touched))
+    work = stage_work(moe, shape, T, avg_touched)
+    peaks, peak_kind = load_peaks()
+    decode = T <= 32
+    dom = max(("router", "gate_up", "down"), key=lambda n: stage_avg[n])
+    if decode:
+        achieved = work[dom]["bytes"] / (stage_avg[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_kind": f"{peak_kind} STREAM-copy HBM bandwidth",
+                "algorithmic_bytes_per_launch": work[dom]["bytes"], "avg_launch_ms": stage_avg[dom]}
+    else:
+        achieved = work[dom]["flops"] / (stage_avg[dom] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_kind": f"{peak_kind} sustained cuBLAS bf16 GEMM",
+                "algorithmic_flops_per_launch": work[dom]["flops"], "avg_launch_ms": stage_avg[dom]}
+
+    # ---- end to end through the public API with host buffers
+    x_host = torch.empty_like(x, device="cpu").pin_memory()
+    x_host.copy_(x.cpu())
+    out_host = torch.empty(layers_per_step, T, shape.hidden, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step(i):
+        x.copy_(x_host, non_blocking=True)
+        graphs[i % n_graphs].replay()
+        gi = i % n_graphs
+        out_host.copy_(outs[gi * layers_per_step:(gi + 1) * layers_per_step], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+
+    launches = moe.moe_forward_launch_count(shape, T, path, False) * layers_per_step * args.steps
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads, secs = oracle_sample(stack, x, stack.bias, T, budget_s=args.cpu_budget)
+        cpu = {"value": v, "unit": "layer-tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": secs}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
+        "config": {"workload": f"nex_moe_{fmt}_T{T}{'_zipf' if zipf else ''}_{layers_per_step}layer_step_"
+                               f"of_{L}layer_stack",
+                   "hidden": shape.hidden, "experts": shape.num_experts, "top_k": shape.top_k,
+                   "inter": shape.inter, "tokens_per_layer": T, "layers_per_step": layers_per_step,
+                   "stack_layers": L, "packed_stack_bytes": stack.packed_bytes,
+                   "l2": "inputs larger than L2: steps rotate over a 40-layer stack of packed weights",
+                   "parallelism": f"dp{world} replicas (one stack per GPU)",
+                   "avg_touched_experts": avg_touched, "path": "decode GEMV" if decode else "tcgen05 grouped GEMM"},
+        "roofline": roof,
+        "stage_ms": stage_avg,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "layer-tokens/s", "h2d_bytes_per_step": x.numel() * 2,
+                "d2h_bytes_per_step": layers_per_step * T * shape.hidden * 2, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "device_status": moe.moe_status_str(status),
+    }
+    return line
+
+
+# ---------------------------------------------------------------- reference arm (the CPU oracle)
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores, on this workload's config and metric.
+    Each step is a bounded sample: one token of one layer (cold dequantisation
+    of its k experts), so that the whole run ends within a few minutes."""
+    if rank != 0:
+        return None
+    from oracle import moe_oracle as o
+    from threadpoolctl import threadpool_info
+    fmt_name, T, zipf, _ = WORKLOADS[args.workload]
+    fmt = o.FMT_INT4 if fmt_name == "int4_g128" else o.FMT_MXFP4
+    s = moe_synth.NEX
+    n_layers = 2
+    prepared = []
+    # inputs drawn with the same generator as our arm when a GPU is present
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    for l in range(n_layers):
+        seed = moe_synth.SEED_STACK_BASE + l
+        router = moe_synth.bf16_bits(moe_synth.router_weight(s, seed, gen_dev))
+        b = moe_synth.zipf_bias(s, seed).numpy() if zipf else None
+        x = moe_synth.bf16_bits(moe_synth.hidden_states(s, T, rank_token_seed(0, T), gen_dev))[:max(1, min(T, 64))]
+        ids, _ = o.route(o.router_logits(x, router), b, s.top_k)
+        touched = sorted(set(int(e) for e in ids.reshape(-1)))
+        gu = moe_synth.gate_up_bank(s, seed, gen_dev)
+        dn = moe_synth.down_bank(s, seed, gen_dev)
+        gu_p = {e: o.pack(fmt, moe_synth.bf16_bits(gu[e])) for e in touched}
+        dn_p = {e: o.pack(fmt, moe_synth.bf16_bits(dn[e])) for e in touched}
+        del gu, dn
+        prepared.append((router, b, x, gu_p, dn_p))
+    budget = 150.0 / max(1, args.steps + args.warmup)
+
+    def one_step(i):
+        router, b, x, gu_p, dn_p = prepared[i % n_layers]
+        t = i % x.shape[0]
+        gu = o.PackedBank(fmt, {e: v[0] for e, v in gu_p.items()}, {e: v[1] for e, v in gu_p.items()})
+        dn = o.PackedBank(fmt, {e: v[0] for e, v in dn_p.items()}, {e: v[1] for e, v in dn_p.items()})
+        t0 = time.perf_counter()
+        o.forward(x[t:t + 1], router, b, gu, dn, s.top_k)
+        return time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        one_step(i)
+    total = 0.0
+    steps_done = 0
+    for i in range(args.steps):
+        total += one_step(args.warmup + i)
+        steps_done += 1
+        if total > 170.0:
+            break
+    value = steps_done / total
+    threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    sample = ("CPU oracle (NumPy fp64) forward of one token of one layer per step (router, top-k, cold "
+              f"dequantisation of its {s.top_k} experts, SwiGLU, combine); packing untimed")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world,
+        "steps": steps_done, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, steps_done),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
+        "config": {"workload": f"nex_moe_{fmt_name}_T{T}{'_zipf' if zipf else ''}", "hidden": s.hidden,
+                   "experts": s.num_experts, "top_k": s.top_k, "inter": s.inter, "tokens_per_layer": T},
+        "cpu_baseline": {"value": value, "unit": "layer-tokens/s", "cores": int(threads), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "layer-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "per_step_budget_s": budget,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode4")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps are required")
+    rank, local, world = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    dist_init("nccl")
+    line = run_ours(args, rank, local, world)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -199,7 +199,9 @@ typedef struct {
   int32_t* offsets_out;      /* [E+1]   per-expert row offsets */
   int32_t* sorted_rows_out;  /* [T*k]   expert-sorted rows */
   uint16_t* act_out;         /* [T*k, I] bf16 SwiGLU activations, expert-sorted rows */
-  cudaEvent_t* stage_events; /* [2*MOE_NUM_STAGES]: recorded before / after each stage */
+  cudaEvent_t* stage_events; /* [2*MOE_NUM_STAGES]: recorded before / after each stage
+                                (as external event nodes when the stream is being
+                                captured into a CUDA graph) */
 } moe_forward_opts_t;
 
 /* Workspace bytes moe_forward / moe_forward_routed need for T tokens. */
@@ -234,6 +236,12 @@ MOE_API moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t
 /* Zeroes the status word at the start of a workspace (enqueued on `stream`).
  * Call once after allocating a workspace, before its first use. */
 MOE_API moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of kernels moe_forward (routed = 0) or moe_forward_routed
+ * (routed = 1) launches for T tokens on `path` (memsets and the optional
+ * debug copies are not kernels and are not counted); -1 if the arguments are
+ * invalid. */
+MOE_API int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed);
 
 /* Synchronises `stream`, then reports MOE_ERR_TIMEOUT if a bounded
  * device-side wait of a previous moe_forward on this workspace expired (and

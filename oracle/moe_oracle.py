@@ -304,12 +304,55 @@ class PackedBank:
         return self._cache[e]
 
 
-def expert_mlp(x_rows, w_gate_up, w_down):
-    """SwiGLU expert on fp64 rows: a = bf16(silu(h_gate) * h_up), y = W_down a."""
+def swiglu_exact(x_rows, w_gate_up):
+    """silu(h_gate) * h_up in fp64, before the activation's bf16 rounding."""
     inter = w_gate_up.shape[0] // 2
     h = x_rows @ w_gate_up.T
-    a = bf16_round(silu(h[:, :inter]) * h[:, inter:])
+    return silu(h[:, :inter]) * h[:, inter:]
+
+
+def expert_mlp(x_rows, w_gate_up, w_down):
+    """SwiGLU expert on fp64 rows: a = bf16(silu(h_gate) * h_up), y = W_down a."""
+    a = bf16_round(swiglu_exact(x_rows, w_gate_up))
     return a, a @ w_down.T
+
+
+def expert_activations(x_bits, ids, gate_up: PackedBank, num_experts: int):
+    """Expert-sorted activations of every (token, slot) row.
+
+    Returns (a_exact fp64 [T*k, I] before rounding, a = bf16(a_exact)) with
+    row q holding sorted_rows[q] of permute(ids).
+    """
+    x = bf16_to_f64(x_bits)
+    T, k = ids.shape
+    offsets, sorted_rows, _ = permute(ids, num_experts)
+    a_exact = None
+    for e in range(num_experts):
+        rows = sorted_rows[offsets[e]:offsets[e + 1]]
+        if rows.size == 0:
+            continue
+        ae = swiglu_exact(x[rows // k], gate_up.expert(e))
+        if a_exact is None:
+            a_exact = np.zeros((T * k, ae.shape[1]), dtype=np.float64)
+        a_exact[offsets[e]:offsets[e + 1]] = ae
+    return a_exact, bf16_round(a_exact)
+
+
+def down_and_combine(a_sorted, ids, weights, down: PackedBank, num_experts: int):
+    """out_t = sum_j w_tj * W_down[ids_tj] a_(t,j), from expert-sorted activations."""
+    T, k = ids.shape
+    offsets, sorted_rows, _ = permute(ids, num_experts)
+    wflat = np.asarray(weights, dtype=np.float64).reshape(-1)
+    out = None
+    for e in range(num_experts):
+        rows = sorted_rows[offsets[e]:offsets[e + 1]]
+        if rows.size == 0:
+            continue
+        y = a_sorted[offsets[e]:offsets[e + 1]] @ down.expert(e).T
+        if out is None:
+            out = np.zeros((T, y.shape[1]), dtype=np.float64)
+        out[rows // k] += wflat[rows][:, None] * y      # each token at most once per expert
+    return out
 
 
 def forward_routed(x_bits, ids, weights, gate_up: PackedBank, down: PackedBank, num_experts: int):
@@ -317,23 +360,8 @@ def forward_routed(x_bits, ids, weights, gate_up: PackedBank, down: PackedBank, 
 
     Returns (out fp64 [T, H], a fp64 [T*k, I] in expert-sorted row order).
     """
-    x = bf16_to_f64(x_bits)
-    T, k = ids.shape
-    offsets, sorted_rows, _ = permute(ids, num_experts)
-    out = np.zeros((T, x.shape[1]), dtype=np.float64)
-    a_sorted = None
-    wflat = np.asarray(weights, dtype=np.float64).reshape(-1)
-    for e in range(num_experts):
-        rows = sorted_rows[offsets[e]:offsets[e + 1]]
-        if rows.size == 0:
-            continue
-        toks = rows // k                                  # each token at most once per expert
-        a, y = expert_mlp(x[toks], gate_up.expert(e), down.expert(e))
-        if a_sorted is None:
-            a_sorted = np.zeros((T * k, a.shape[1]), dtype=np.float64)
-        a_sorted[offsets[e]:offsets[e + 1]] = a
-        out[toks] += wflat[rows][:, None] * y
-    return out, a_sorted
+    _, a_sorted = expert_activations(x_bits, ids, gate_up, num_experts)
+    return down_and_combine(a_sorted, ids, weights, down, num_experts), a_sorted
 
 
 def forward(x_bits, router_bits, bias32, gate_up: PackedBank, down: PackedBank, top_k: int):

@@ -15,7 +15,7 @@ from oracle import moe_oracle as o
 
 _orig = {name: getattr(o, name) for name in (
     "pack_int4_g128", "unpack_nibbles", "dequant_int4_g128", "mx_exponent", "e2m1_nearest",
-    "route", "expert_mlp", "permute", "f64_to_bf16")}
+    "route", "expert_mlp", "permute", "f64_to_bf16", "swiglu_exact", "expert_activations")}
 
 
 def _int4_pack_variant(div=7.0, rnd=np.rint):
@@ -63,16 +63,15 @@ def _route_variant(tie_high=False, full_softmax=False, unit_weights=False):
     return route
 
 
-def _mlp_variant(swap_gate_up=False, round_act=True):
-    def mlp(x_rows, w_gate_up, w_down):
-        inter = w_gate_up.shape[0] // 2
-        h = x_rows @ w_gate_up.T
-        g, u = (h[:, inter:], h[:, :inter]) if swap_gate_up else (h[:, :inter], h[:, inter:])
-        a = o.silu(g) * u
-        if round_act:
-            a = o.bf16_round(a)
-        return a, a @ w_down.T
-    return mlp
+def _swiglu_swapped(x_rows, w_gate_up):
+    inter = w_gate_up.shape[0] // 2
+    h = x_rows @ w_gate_up.T
+    return o.silu(h[:, inter:]) * h[:, :inter]
+
+
+def _activations_unrounded(x_bits, ids, gate_up, num_experts):
+    a_exact, _ = _orig["expert_activations"](x_bits, ids, gate_up, num_experts)
+    return a_exact, a_exact
 
 
 def _unstable_permute(ids, E):
@@ -119,8 +118,8 @@ MUTANTS = {
     "route ties to higher index": {"route": _route_variant(tie_high=True)},
     "route softmax over all experts": {"route": _route_variant(full_softmax=True)},
     "combine drops routing weight": {"route": _route_variant(unit_weights=True)},
-    "gate and up swapped": {"expert_mlp": _mlp_variant(swap_gate_up=True)},
-    "activation not rounded to bf16": {"expert_mlp": _mlp_variant(round_act=False)},
+    "gate and up swapped": {"swiglu_exact": _swiglu_swapped},
+    "activation not rounded to bf16": {"expert_activations": _activations_unrounded},
     "unstable permutation": {"permute": _unstable_permute},
     "bf16 rounding truncates": {"f64_to_bf16": _bf16_truncating},
 }

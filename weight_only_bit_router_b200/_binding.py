@@ -74,6 +74,8 @@ _SIGS = {
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
+    "moe_forward_launch_count": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int]),
     "moe_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_workspace_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64,
@@ -280,6 +282,10 @@ def moe_forward_routed(shape: MoeShape, x, topk_ids, topk_w, gate_up_packed, dow
                                   _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
     _check("moe_forward_routed", st)
     return out
+
+
+def moe_forward_launch_count(shape: MoeShape, T: int, path=MOE_PATH_AUTO, routed=False) -> int:
+    return lib().moe_forward_launch_count(ctypes.byref(shape), T, path, int(routed))
 
 
 def moe_workspace_init(workspace, stream=None):

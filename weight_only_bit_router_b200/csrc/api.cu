@@ -50,7 +50,8 @@ Bank make_bank(const void* packed, moe_format_t fmt, int E, int N, int K) {
 
 // Record stage event `idx` (0 = before, 1 = after) if the caller asked for it.
 void mark(const moe_forward_opts_t* o, int stage, int after, cudaStream_t stream) {
-  if (o && o->stage_events) cudaEventRecord(o->stage_events[2 * stage + after], stream);
+  if (o && o->stage_events)
+    cudaEventRecordWithFlags(o->stage_events[2 * stage + after], stream, cudaEventRecordExternal);
 }
 
 __global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
@@ -328,6 +329,18 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
   mark(opts, 1, 1, stream);
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
   return copy_debug_outputs(s, T, ws, opts, true, stream);
+}
+
+int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed) {
+  if (check_shape(shape) != MOE_OK || check_T(shape, T) != MOE_OK) return -1;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return -1;
+  if (T == 0) return 0;
+  const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  int n = routed ? 0 : 2;                                     // router logits, top-k
+  n += (long(T) * shape->top_k <= 1024) ? 1 : 3;              // permutation
+  n += 3;                                                     // gate_up, down, combine / finalize
+  (void)decode;
+  return n;
 }
 
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream) {

@@ -526,8 +526,15 @@ template <int MODE, int FMT>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ctas, cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<MODE, FMT>;
   const int smem = Cfg<MODE>::SMEM;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err != cudaSuccess) return err;
+  // once per process (and per device), outside any stream capture of later calls
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
   const int grid = max(1, min(sm_count(), max_ctas));
   kern<<<grid, kThreads, smem, stream>>>(map, args);
   return cudaGetLastError();
