@@ -66,20 +66,25 @@ def bf16_ulp(v):
     return np.where(a == 0, 2.0 ** -133, np.ldexp(1.0, np.maximum(e - 8, -133)))
 
 
-def flip_aware_activations(gpu_act, a_exact, a_round, rel=1e-4, abs_frac=1e-6):
+def flip_aware_activations(gpu_act, a_exact, a_round, rel=1e-4, abs_frac=2e-5, max_frac_differing=0.01):
     """The GPU's bf16 activations must be correct roundings of the exact SwiGLU
     value up to the GPU's fp32 accumulation error: every GPU value g must
     satisfy |g - a_exact| <= ulp(g)/2 + rel*|a_exact| + abs_frac*rms(a), i.e. g
-    is the bf16 rounding of some value within that error band.  Where g differs
-    from the oracle's own rounding both are correct results, and the reference
-    continues with the GPU's.  Returns (activations for the reference, number
-    of elements that differ from the oracle's rounding)."""
+    is the bf16 rounding of some value within that error band.  The band's
+    absolute part covers tensor-core fp32 accumulation over K (error ~1e-6 on
+    activations of rms ~0.4 at K = 2048), far below what a wrong weight, scale
+    or token would cause; at most `max_frac_differing` of the elements may
+    differ from the oracle's own rounding at all.  Where they differ both are
+    correct results and the reference continues with the GPU's.  Returns
+    (activations for the reference, number of elements that differ)."""
     diff = gpu_act != a_round
-    if diff.any():
+    n = int(diff.sum())
+    assert n <= max_frac_differing * gpu_act.size, f"{n} of {gpu_act.size} activations differ from the oracle"
+    if n:
         g, r, x = gpu_act[diff], a_round[diff], a_exact[diff]
         tol = rel * np.abs(x) + abs_frac * float(np.sqrt(np.mean(a_round ** 2)))
         bad = np.abs(g - x) > 0.5 * bf16_ulp(g) + tol
         assert not bad.any(), (f"{int(bad.sum())} of {gpu_act.size} activations differ from the oracle beyond "
                                f"fp32 accumulation error; e.g. gpu={g[bad][:4]} oracle={r[bad][:4]} "
                                f"exact={x[bad][:4]}")
-    return np.where(diff, gpu_act, a_round), int(diff.sum())
+    return np.where(diff, gpu_act, a_round), n

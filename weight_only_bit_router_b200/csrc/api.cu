@@ -48,10 +48,17 @@ Bank make_bank(const void* packed, moe_format_t fmt, int E, int N, int K) {
   return b;
 }
 
-// Record stage event `idx` (0 = before, 1 = after) if the caller asked for it.
-void mark(const moe_forward_opts_t* o, int stage, int after, cudaStream_t stream) {
-  if (o && o->stage_events)
-    cudaEventRecordWithFlags(o->stage_events[2 * stage + after], stream, cudaEventRecordExternal);
+// Record stage event (after = 0: before the stage, 1: after it) if the caller
+// asked for it; inside a stream capture it becomes an external event node so
+// that it can be timed when the graph is replayed.
+cudaError_t mark(const moe_forward_opts_t* o, int stage, int after, cudaStream_t stream) {
+  if (!o || !o->stage_events) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t err = cudaStreamIsCapturing(stream, &cs);
+  if (err != cudaSuccess) return err;
+  cudaEvent_t ev = o->stage_events[2 * stage + after];
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal)
+                                             : cudaEventRecord(ev, stream);
 }
 
 __global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
@@ -127,22 +134,22 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
                          const moe_forward_opts_t* o, cudaStream_t stream) {
   const Bank gu = make_bank(gu_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
   const Bank dn = make_bank(dn_packed, s.fmt, s.num_experts, s.hidden, s.inter);
-  mark(o, 2, 0, stream);
+  MOE_TRY(mark(o, 2, 0, stream));
   if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, ws, stream));
   else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, ws, stream));
-  mark(o, 2, 1, stream);
-  mark(o, 3, 0, stream);
+  MOE_TRY(mark(o, 2, 1, stream));
+  MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
     MOE_TRY(launch_decode_down(s, T, dn, ws, stream));
   } else {
     MOE_TRY(cudaMemsetAsync(ws.out_acc, 0, size_t(T) * s.hidden * 4, stream));
     MOE_TRY(launch_grouped_down(s, T, dn, ws, stream));
   }
-  mark(o, 3, 1, stream);
-  mark(o, 4, 0, stream);
+  MOE_TRY(mark(o, 3, 1, stream));
+  MOE_TRY(mark(o, 4, 0, stream));
   if (decode) MOE_TRY(launch_decode_combine(s, T, ws, out, stream));
   else MOE_TRY(launch_finalize_out(ws.out_acc, long(T) * s.hidden, out, stream));
-  mark(o, 4, 1, stream);
+  MOE_TRY(mark(o, 4, 1, stream));
   return MOE_OK;
 }
 
@@ -297,16 +304,16 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   const Workspace ws = carve_workspace(workspace, s, T);
-  mark(opts, 0, 0, stream);
+  MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT)
     MOE_TRY(launch_router_gemv(x, router_w, T, s.hidden, s.num_experts, ws.logits, stream));
   else
     MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
-  mark(opts, 0, 1, stream);
-  mark(opts, 1, 0, stream);
+  MOE_TRY(mark(opts, 0, 1, stream));
+  MOE_TRY(mark(opts, 1, 0, stream));
   MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
   if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
-  mark(opts, 1, 1, stream);
+  MOE_TRY(mark(opts, 1, 1, stream));
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
   return copy_debug_outputs(s, T, ws, opts, false, stream);
 }
@@ -324,9 +331,9 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
   Workspace ws = carve_workspace(workspace, s, T);
   ws.topk_ids = const_cast<int32_t*>(topk_ids);
   ws.topk_w = const_cast<float*>(topk_w);
-  mark(opts, 1, 0, stream);
+  MOE_TRY(mark(opts, 1, 0, stream));
   if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
-  mark(opts, 1, 1, stream);
+  MOE_TRY(mark(opts, 1, 1, stream));
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
   return copy_debug_outputs(s, T, ws, opts, true, stream);
 }
