@@ -286,7 +286,8 @@ def run_ours(args, rank, local, world):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fmt, T, zipf, layers_per_step = WORKLOADS[args.workload]
-    L = NUM_LAYERS
+    L = args.stack_layers
+    layers_per_step = min(layers_per_step, L)
     stack = Stack(moe, fmt, L, device, zipf)
     shape = stack.shape
     x = moe_synth.hidden_states(moe_synth.NEX, T, rank_token_seed(rank, T), device)
@@ -516,6 +517,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode4")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stack-layers", type=int, default=NUM_LAYERS,
+                    help="layers in the packed stack (smaller only for profiling captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps are required")

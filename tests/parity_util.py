@@ -1,4 +1,7 @@
 """Helpers shared by the GPU parity tests (the oracle side runs on the CPU)."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -88,3 +91,12 @@ def flip_aware_activations(gpu_act, a_exact, a_round, rel=1e-4, abs_frac=2e-5, m
                                f"fp32 accumulation error; e.g. gpu={g[bad][:4]} oracle={r[bad][:4]} "
                                f"exact={x[bad][:4]}")
     return np.where(diff, gpu_act, a_round), n
+
+
+def record_parity(rec: dict):
+    """Append one parity record to $MOE_PARITY_REPORT (a JSON-lines file) if set."""
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        rec = dict(rec, test=os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0])
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
