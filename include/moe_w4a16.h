@@ -233,8 +233,10 @@ MOE_API moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
                                 const moe_forward_opts_t* opts, cudaStream_t stream);
 
-/* Zeroes the status word at the start of a workspace (enqueued on `stream`).
- * Call once after allocating a workspace, before its first use. */
+/* Zeroes the status word and the kernels' completion counters at the start
+ * of a workspace (its first 4096 bytes; enqueued on `stream`).  Call once
+ * after allocating a workspace, before its first use; every forward leaves
+ * the counters at zero again. */
 MOE_API moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Number of kernels moe_forward (routed = 0) or moe_forward_routed

@@ -90,7 +90,9 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
     off += align_up(bytes, 256);
     return r;
   };
-  w.status = static_cast<uint32_t*>(take(256));
+  w.status = static_cast<uint32_t*>(take(kStatusBytes));
+  w.route_counter = p ? reinterpret_cast<int32_t*>(w.status) + 1 : nullptr;
+  w.tile_counters = p ? reinterpret_cast<int32_t*>(w.status) + 8 : nullptr;
   w.logits = static_cast<float*>(take(size_t(T) * E * 4));
   w.topk_ids = static_cast<int32_t*>(take(R * 4));
   w.topk_w = static_cast<float*>(take(R * 4));
@@ -140,15 +142,17 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   MOE_TRY(mark(o, 2, 1, stream));
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
-    MOE_TRY(launch_decode_down(s, T, dn, ws, stream));
+    // down projection and the combine are one kernel on this path
+    MOE_TRY(launch_decode_down_combine(s, T, dn, ws, out, stream));
+    MOE_TRY(mark(o, 3, 1, stream));
+    MOE_TRY(mark(o, 4, 0, stream));
   } else {
     MOE_TRY(cudaMemsetAsync(ws.out_acc, 0, size_t(T) * s.hidden * 4, stream));
     MOE_TRY(launch_grouped_down(s, T, dn, ws, stream));
+    MOE_TRY(mark(o, 3, 1, stream));
+    MOE_TRY(mark(o, 4, 0, stream));
+    MOE_TRY(launch_finalize_out(ws.out_acc, long(T) * s.hidden, out, stream));
   }
-  MOE_TRY(mark(o, 3, 1, stream));
-  MOE_TRY(mark(o, 4, 0, stream));
-  if (decode) MOE_TRY(launch_decode_combine(s, T, ws, out, stream));
-  else MOE_TRY(launch_finalize_out(ws.out_acc, long(T) * s.hidden, out, stream));
   MOE_TRY(mark(o, 4, 1, stream));
   return MOE_OK;
 }
@@ -305,14 +309,18 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
   const moe_shape_t& s = *shape;
   const Workspace ws = carve_workspace(workspace, s, T);
   MOE_TRY(mark(opts, 0, 0, stream));
-  if (T <= kDecodeMaxT)
-    MOE_TRY(launch_router_gemv(x, router_w, T, s.hidden, s.num_experts, ws.logits, stream));
-  else
+  if (T <= kDecodeMaxT) {
+    // router logits, top-k and the permutation in one kernel
+    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+  } else {
     MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
-  MOE_TRY(mark(opts, 0, 1, stream));
-  MOE_TRY(mark(opts, 1, 0, stream));
-  MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
-  if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+    MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
+    if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
+  }
   MOE_TRY(mark(opts, 1, 1, stream));
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
   return copy_debug_outputs(s, T, ws, opts, false, stream);
@@ -343,16 +351,18 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return -1;
   if (T == 0) return 0;
   const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
-  int n = routed ? 0 : 2;                                     // router logits, top-k
-  n += (long(T) * shape->top_k <= 1024) ? 1 : 3;              // permutation
-  n += 3;                                                     // gate_up, down, combine / finalize
-  (void)decode;
+  const int perm = (long(T) * shape->top_k <= 1024) ? 1 : 3;
+  int n = 0;
+  if (routed) n += perm;
+  else if (T <= kDecodeMaxT) n += 1;                          // fused router + top-k + permutation
+  else n += 2 + perm;                                         // router GEMM, top-k, permutation
+  n += decode ? 2 : 3;                                        // gate_up, down (+ combine) / finalize
   return n;
 }
 
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (!workspace || workspace_bytes < 256 || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(workspace, 0, 256, stream));
+  if (!workspace || workspace_bytes < kStatusBytes || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(workspace, 0, kStatusBytes, stream));
 }
 
 moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream) {

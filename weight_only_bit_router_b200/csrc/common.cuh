@@ -167,6 +167,23 @@ MOE_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 1-D bulk copy global -> shared (size and both addresses multiples of 16 B);
+// completion is signalled on `bar` as transaction bytes.
+MOE_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// --------------------------------------------------------------------------
+// programmatic dependent launch: wait for the preceding kernel's results /
+// allow the next kernel in the stream to start launching
+// --------------------------------------------------------------------------
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads
 // --------------------------------------------------------------------------

@@ -2,11 +2,13 @@
 //
 // The time goes into streaming the touched experts' packed weights from HBM
 // ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", Measured: at concurrency 32
-// the bottleneck is weight bandwidth).  Each warp owns 16 weight rows and a
-// slice of K; a lane loads 16 contiguous bytes (32 codes) per row and 128-k
-// block with one 128-bit load, dequantises them to bf16 in registers
-// (bf16(q*s) for INT4, e2m1*2^e for MXFP4) and feeds mma.sync m16n8k16 with
-// up to 8 tokens per tile.
+// the bottleneck is weight bandwidth).  A CTA owns one work unit, (touched
+// expert, a tile of output features): the unit's packed rows are one
+// contiguous range of the canonical [E][N][K/2] layout, so a single thread
+// starts 1-D bulk copies of the codes and scales into shared memory and every
+// byte of the unit is in flight at once.  Warps then dequantise in registers
+// (bf16(q*s) for INT4, e2m1*2^e for MXFP4) and feed mma.sync m16n8k16 with up
+// to 8 tokens per tile.
 //
 // Fragment k-permutation.  Inside a 128-k block, lane (g = lane/4, q = lane%4)
 // owns k in [32q, 32q+32).  For MMA step s = 2*j + h (j = 32-bit code word,
@@ -17,15 +19,16 @@
 // fragment register directly.
 #include "common.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
 namespace {
 
-constexpr int kDecWarps = 4;   // warps per CTA
-constexpr int kDecRows = 16;   // weight rows (features) per warp tile
-constexpr int kDecPF = 4;      // 128-k blocks prefetched per warp at once
-constexpr int kDecNT = 4;      // token tiles of 8 held in registers at once
+constexpr int kDecWarps = 4;       // warps per CTA
+constexpr int kDecRows = 16;       // weight rows (features) per warp tile
+constexpr int kDecNT = 4;          // token tiles of 8 held in registers at once
+constexpr int kDownFeatures = kDecRows * kDecWarps;  // features per down CTA
 
 MOE_DEV void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -41,13 +44,6 @@ MOE_DEV uint32_t pow2_bf16x2(int e) {
   return b | (b << 16);
 }
 
-// Per-row dequantisation state for one 128-k block: the 16 code bytes of the
-// lane's k-slice and the bf16x2 multiplier (scale, or 2^e for MXFP4).
-struct RowChunk {
-  uint4 codes;
-  uint32_t mult;
-};
-
 template <int FMT>
 MOE_DEV uint32_t dq_pair(uint32_t word, int i, uint32_t mult) {
   const uint32_t v = (FMT == MOE_FMT_INT4_G128) ? int4_pair(word, i) : e2m1_pair(word, i);
@@ -58,20 +54,30 @@ MOE_DEV uint32_t word_of(const uint4& c, int j) {
   return j == 0 ? c.x : j == 1 ? c.y : j == 2 ? c.z : c.w;
 }
 
-// Load one row's 16-byte code chunk and its multiplier for the lane's k-slice
-// [kb + 32q, kb + 32q + 32).  Slices past K read as zero weights.
+// Scale bytes per weight row of a bank with reduction length K.
+__host__ __device__ inline int scale_row_bytes(int fmt, int K) {
+  return fmt == MOE_FMT_INT4_G128 ? int4_groups(K) * 2 : K / 32;
+}
+
+// One row's 16 code bytes for the lane's k-slice [kb + 32q, kb + 32q + 32) and
+// the bf16x2 multiplier (scale, or 2^e for MXFP4), read from shared memory.
+// Slices past K read as zero weights.
+struct RowChunk {
+  uint4 codes;
+  uint32_t mult;
+};
+
 template <int FMT>
-MOE_DEV RowChunk load_row_chunk(const Bank& bk, long row, int kb, int q) {
+MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int r, int K, int kb, int q) {
   RowChunk rc;
   const int k = kb + 32 * q;
-  if (k < bk.K) {
-    rc.codes = ldg_nc_v4(bk.codes + row * (bk.K / 2) + k / 2);
+  if (k < K) {
+    rc.codes = *reinterpret_cast<const uint4*>(codes + r * (K / 2) + k / 2);
     if (FMT == MOE_FMT_INT4_G128) {
-      const uint32_t s = static_cast<const uint16_t*>(bk.scales)[row * int4_groups(bk.K) + k / 128];
+      const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[r * int4_groups(K) + k / 128];
       rc.mult = s | (s << 16);
     } else {
-      const int e = int(static_cast<const uint8_t*>(bk.scales)[row * (bk.K / 32) + k / 32]) - 127;
-      rc.mult = pow2_bf16x2(e);
+      rc.mult = pow2_bf16x2(int(scales[r * (K / 32) + k / 32]) - 127);
     }
   } else {
     rc.codes = make_uint4(0, 0, 0, 0);  // INT4 nibble 0 would be -8: zero the multiplier instead
@@ -106,7 +112,7 @@ MOE_DEV void load_act_frags(const uint16_t* rowp, int K, int kb, int q, bool val
   }
 }
 
-// acc[4] += W(rows r, r+8; one 128-k block) x act fragments, for one 16-row tile.
+// acc[4] += W(rows r, r+8; one 128-k block) x activation fragments.
 template <int FMT>
 MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, const uint32_t (&b)[8][2]) {
 #pragma unroll
@@ -124,99 +130,126 @@ MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, 
   }
 }
 
+// Stage `rows` consecutive weight rows (codes + scales) of a bank into shared
+// memory with two bulk copies on `bar`; one thread calls this.
+template <int FMT>
+MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, uint8_t* s_scales, uint64_t* bar) {
+  const uint32_t cbytes = uint32_t(rows) * (bk.K / 2);
+  const int sb = scale_row_bytes(FMT, bk.K);
+  const uint32_t sbytes = uint32_t(rows) * sb;
+  mbar_arrive_expect_tx(bar, cbytes + sbytes);
+  bulk_g2s(s_codes, bk.codes + row0 * (bk.K / 2), cbytes, bar);
+  bulk_g2s(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, sbytes, bar);
+}
+
+// Wait for the staged rows (bounded); false if the wait gave up.
+MOE_DEV bool wait_staged(uint64_t* bar, uint32_t* status) {
+  volatile int never = 0;
+  return mbar_wait(bar, 0, &never, status);
+}
+
 // ---------------------------------------------------------------------------
-// gate_up + SwiGLU.  grid = (max experts touched) x (I / 16).  The CTA's 4
-// warps split K; partial tiles are summed in shared memory, then
+// gate_up + SwiGLU.  grid = (max experts touched) x (I / 16).  A CTA stages
+// the 16 gate rows and the 16 matching up rows of its expert; its 4 warps
+// split K, partial tiles are summed in shared memory, and
 // a = bf16(silu(gate) * up) goes to act[p][f] for the expert's sorted rows p.
 // ---------------------------------------------------------------------------
-template <int FMT>
+template <int FMT, int NT>
 __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act) {
-  __shared__ float red[kDecWarps][kDecNT][2][4][32];
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act,
+    uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int K = gu.K;
+  const int cbytes = kDecRows * (K / 2);
+  const int sbytes = kDecRows * scale_row_bytes(FMT, K);
+  const int red_bytes = kDecWarps * NT * 2 * 4 * 32 * 4;
+  uint8_t* s_cg = smem;                              // gate codes, later the reduction buffer
+  uint8_t* s_cu = s_cg + cbytes;                     // up codes
+  uint8_t* s_sg = smem + max(2 * cbytes, red_bytes); // gate scales
+  uint8_t* s_su = s_sg + sbytes;                     // up scales
+  uint64_t* bar = reinterpret_cast<uint64_t*>(s_su + ((sbytes + 15) & ~15));
+  float* red = reinterpret_cast<float*>(smem);       // [warp][tile][gate/up][4][lane]
+
+  pdl_wait();
+  pdl_trigger();
   const int ftiles = I / kDecRows;
   const int slot = blockIdx.x / ftiles;
   const int f0 = (blockIdx.x % ftiles) * kDecRows;
   if (slot >= touched[0]) return;
   const int e = touched[1 + slot];
+  const long row_g = long(e) * gu.N + f0;
+  const long row_u = row_g + I;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    stage_rows<FMT>(gu, row_g, kDecRows, s_cg, s_sg, bar);
+    stage_rows<FMT>(gu, row_u, kDecRows, s_cu, s_su, bar);
+  }
   const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int K = gu.K, N = gu.N;
   const int nblk = (K + 127) / 128;
-  const long row_g = long(e) * N + f0 + g;       // gate rows g, g+8
-  const long row_u = long(e) * N + I + f0 + g;   // up rows g, g+8
   const int ntiles = (n_e + 7) / 8;
+  __syncthreads();  // barrier initialised before anyone waits on it
+  const bool ok = wait_staged(bar, status);
 
-  for (int nt0 = 0; nt0 < ntiles; nt0 += kDecNT) {
-    float acc[kDecNT][2][4];
+  for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
+    float acc[NT][2][4];
 #pragma unroll
-    for (int j = 0; j < kDecNT; ++j)
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[j][t][i] = 0.f;
-    // token row of this lane in each of the tiles
-    const uint16_t* xrow[kDecNT];
-    bool xval[kDecNT];
+    const uint16_t* xrow[NT];
+    bool xval[NT];
 #pragma unroll
-    for (int j = 0; j < kDecNT; ++j) {
+    for (int j = 0; j < NT; ++j) {
       const int c = (nt0 + j) * 8 + g;
       xval[j] = c < n_e;
       xrow[j] = x + size_t(xval[j] ? sorted_rows[p0 + c] / top_k : 0) * K;
     }
-    for (int b0 = warp; b0 < nblk; b0 += kDecWarps * kDecPF) {
-      RowChunk cg[kDecPF][2], cu[kDecPF][2];
+    if (ok) {
+      for (int b = warp; b < nblk; b += kDecWarps) {
+        const int kb = b * 128;
+        const RowChunk g0 = smem_row_chunk<FMT>(s_cg, s_sg, g, K, kb, q);
+        const RowChunk g1 = smem_row_chunk<FMT>(s_cg, s_sg, g + 8, K, kb, q);
+        const RowChunk u0 = smem_row_chunk<FMT>(s_cu, s_su, g, K, kb, q);
+        const RowChunk u1 = smem_row_chunk<FMT>(s_cu, s_su, g + 8, K, kb, q);
 #pragma unroll
-      for (int u = 0; u < kDecPF; ++u) {
-        const int kb = (b0 + u * kDecWarps) * 128;
-        const bool ok = kb < K;
-        cg[u][0] = load_row_chunk<FMT>(gu, row_g, ok ? kb : K, q);
-        cg[u][1] = load_row_chunk<FMT>(gu, row_g + 8, ok ? kb : K, q);
-        cu[u][0] = load_row_chunk<FMT>(gu, row_u, ok ? kb : K, q);
-        cu[u][1] = load_row_chunk<FMT>(gu, row_u + 8, ok ? kb : K, q);
-      }
-#pragma unroll
-      for (int u = 0; u < kDecPF; ++u) {
-        const int kb = (b0 + u * kDecWarps) * 128;
-        if (kb >= K) break;
-#pragma unroll
-        for (int j = 0; j < kDecNT; ++j) {
+        for (int j = 0; j < NT; ++j) {
           if (nt0 + j >= ntiles) break;
           uint32_t bf[8][2];
           load_act_frags(xrow[j], K, kb, q, xval[j], bf);
-          mma_block<FMT>(acc[j][0], cg[u][0], cg[u][1], bf);
-          mma_block<FMT>(acc[j][1], cu[u][0], cu[u][1], bf);
+          mma_block<FMT>(acc[j][0], g0, g1, bf);
+          mma_block<FMT>(acc[j][1], u0, u1, bf);
         }
       }
     }
+    __syncthreads();  // the codes buffer becomes the reduction buffer
 #pragma unroll
-    for (int j = 0; j < kDecNT; ++j)
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) red[warp][j][t][i][lane] = acc[j][t][i];
+        for (int i = 0; i < 4; ++i) red[(((warp * NT + j) * 2 + t) * 4 + i) * 32 + lane] = acc[j][t][i];
     __syncthreads();
-    // warp w finishes token tile nt0 + w
+    // warp w < NT finishes token tile nt0 + w
     const int j = warp;
-    if (nt0 + j < ntiles) {
-      float gsum[4], usum[4];
+    if (ok && j < NT && nt0 + j < ntiles) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        gsum[i] = 0.f;
-        usum[i] = 0.f;
+        float gs = 0.f, us = 0.f;
 #pragma unroll
         for (int w = 0; w < kDecWarps; ++w) {
-          gsum[i] += red[w][j][0][i][lane];
-          usum[i] += red[w][j][1][i][lane];
+          gs += red[(((w * NT + j) * 2 + 0) * 4 + i) * 32 + lane];
+          us += red[(((w * NT + j) * 2 + 1) * 4 + i) * 32 + lane];
         }
-      }
-      // c0,c1: feature g, tokens 2q, 2q+1; c2,c3: feature g+8
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
+        // c0,c1: feature g, tokens 2q, 2q+1; c2,c3: feature g+8
         const int col = (nt0 + j) * 8 + 2 * q + (i & 1);
         const int f = f0 + g + ((i >> 1) << 3);
-        if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(gsum[i], usum[i]));
+        if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(gs, us));
       }
     }
     __syncthreads();
@@ -224,55 +257,70 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// down projection.  grid = (max experts touched) x (H / 64): each warp owns 16
-// output features over the whole K = I; y[p][f] is written in fp32.
+// down projection + deterministic combine.  grid = (max experts touched) x
+// (H / 64).  A CTA stages 64 rows of its expert's down bank; each warp owns
+// 16 features over K = I and writes y[p][f] in fp32.  The last CTA to finish
+// a feature tile (counted in the workspace) sums the k expert outputs of every
+// token in slot order j = 0..k-1 and writes the bf16 output for that tile.
 // ---------------------------------------------------------------------------
-template <int FMT>
+template <int FMT, int NT>
 __global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
-    Bank dn, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
-    const uint16_t* __restrict__ act, float* __restrict__ y) {
+    Bank dn, int T, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
+    const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ pos,
+    float* __restrict__ y, uint16_t* __restrict__ out, uint32_t* status, int32_t* tile_counters) {
+  extern __shared__ __align__(128) uint8_t smem[];
   const int H = dn.N, K = dn.K;  // K = I
-  const int ftiles = H / (kDecRows * kDecWarps);
+  const int cbytes = kDownFeatures * (K / 2);
+  const int sbytes = kDownFeatures * scale_row_bytes(FMT, K);
+  uint8_t* s_c = smem;
+  uint8_t* s_s = smem + cbytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(s_s + ((sbytes + 15) & ~15));
+  __shared__ int s_last;
+
+  pdl_wait();
+  pdl_trigger();
+  const int ftiles = H / kDownFeatures;
   const int slot = blockIdx.x / ftiles;
-  if (slot >= touched[0]) return;
+  const int ft = blockIdx.x % ftiles;
+  const int n_touched = touched[0];
+  if (slot >= n_touched) return;
+  const int e = touched[1 + slot];
+  const int fbase = ft * kDownFeatures;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    stage_rows<FMT>(dn, long(e) * H + fbase, kDownFeatures, s_c, s_s, bar);
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int f0 = (blockIdx.x % ftiles) * (kDecRows * kDecWarps) + warp * kDecRows;
-  const int e = touched[1 + slot];
+  const int f0 = fbase + warp * kDecRows;
   const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
   const int nblk = (K + 127) / 128;
-  const long row = long(e) * H + f0 + g;
   const int ntiles = (n_e + 7) / 8;
-  for (int nt0 = 0; nt0 < ntiles; nt0 += kDecNT) {
-    float acc[kDecNT][4];
+  __syncthreads();
+  const bool ok = wait_staged(bar, status);
+  const int r0 = warp * kDecRows + g;  // staged row of this lane
+  for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
+    float acc[NT][4];
 #pragma unroll
-    for (int j = 0; j < kDecNT; ++j)
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-    for (int b0 = 0; b0 < nblk; b0 += kDecPF) {
-      RowChunk c[kDecPF][2];
+    for (int b = 0; b < nblk; ++b) {
+      const int kb = b * 128;
+      const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, r0, K, kb, q);
+      const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, r0 + 8, K, kb, q);
 #pragma unroll
-      for (int u = 0; u < kDecPF; ++u) {
-        const int kb = (b0 + u) * 128;
-        c[u][0] = load_row_chunk<FMT>(dn, row, kb < K ? kb : K, q);
-        c[u][1] = load_row_chunk<FMT>(dn, row + 8, kb < K ? kb : K, q);
-      }
-#pragma unroll
-      for (int u = 0; u < kDecPF; ++u) {
-        const int kb = (b0 + u) * 128;
-        if (kb >= K) break;
-#pragma unroll
-        for (int j = 0; j < kDecNT; ++j) {
-          if (nt0 + j >= ntiles) break;
-          const int col = (nt0 + j) * 8 + g;
-          uint32_t bf[8][2];
-          load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
-          mma_block<FMT>(acc[j], c[u][0], c[u][1], bf);
-        }
+      for (int j = 0; j < NT; ++j) {
+        if (nt0 + j >= ntiles) break;
+        const int col = (nt0 + j) * 8 + g;
+        uint32_t bf[8][2];
+        load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
+        mma_block<FMT>(acc[j], c0, c1, bf);
       }
     }
 #pragma unroll
-    for (int j = 0; j < kDecNT; ++j) {
+    for (int j = 0; j < NT; ++j) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int col = (nt0 + j) * 8 + 2 * q + (i & 1);
@@ -281,35 +329,94 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
       }
     }
   }
-}
-
-// out[t][h] = bf16(sum_j w[t][j] * y[pos[t*k+j]][h]), slots in order j = 0..k-1.
-__global__ void decode_combine_kernel(const float* __restrict__ y, const float* __restrict__ w,
-                                      const int32_t* __restrict__ pos, int T, int H, int k,
-                                      uint16_t* __restrict__ out) {
-  const long i = long(blockIdx.x) * blockDim.x + threadIdx.x;  // one thread per 4 outputs
-  const long n4 = long(T) * H / 4;
-  if (i >= n4) return;
-  const int t = int(i / (H / 4));
-  const int h = int(i % (H / 4)) * 4;
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int p = pos[size_t(t) * k + j];
-    if (p < 0) continue;
-    const float wj = w[size_t(t) * k + j];
-    const float4 v = *reinterpret_cast<const float4*>(y + size_t(p) * H + h);
-    s.x = fmaf(wj, v.x, s.x);
-    s.y = fmaf(wj, v.y, s.y);
-    s.z = fmaf(wj, v.z, s.z);
-    s.w = fmaf(wj, v.w, s.w);
+  // the last CTA of this feature tile combines it
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&tile_counters[ft], 1) == n_touched - 1;
   }
-  uint2 o;
-  o.x = pack_bf16x2(s.x, s.y);
-  o.y = pack_bf16x2(s.z, s.w);
-  *reinterpret_cast<uint2*>(out + size_t(t) * H + h) = o;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < T * kDownFeatures; i += blockDim.x) {
+    const int t = i / kDownFeatures;
+    const int f = fbase + i % kDownFeatures;
+    float s = 0.f;
+    for (int j = 0; j < top_k; ++j) {
+      const int p = pos[size_t(t) * top_k + j];
+      if (p < 0) continue;
+      s = fmaf(topk_w[size_t(t) * top_k + j], __ldcg(y + size_t(p) * H + f), s);
+    }
+    out[size_t(t) * H + f] = f32_to_bf16_rn(s);
+  }
+  if (threadIdx.x == 0) tile_counters[ft] = 0;  // ready for the next call
 }
 
 int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
+
+size_t gate_up_smem(int fmt, int K) {
+  const int cbytes = kDecRows * (K / 2);
+  const int sbytes = kDecRows * scale_row_bytes(fmt, K);
+  const int red_bytes = kDecWarps * kDecNT * 2 * 4 * 32 * 4;
+  return size_t(std::max(2 * cbytes, red_bytes)) + 2 * size_t((sbytes + 15) & ~15) + 16;
+}
+
+size_t down_smem(int fmt, int K) {
+  const int cbytes = kDownFeatures * (K / 2);
+  const int sbytes = kDownFeatures * scale_row_bytes(fmt, K);
+  return size_t(cbytes) + size_t((sbytes + 15) & ~15) + 16;
+}
+
+template <typename Kern>
+cudaError_t allow_smem(Kern k, size_t smem) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+}
+
+}  // namespace
+
+size_t decode_gate_up_smem_bytes(int fmt, int K) { return gate_up_smem(fmt, K); }
+
+namespace {
+
+template <int FMT, int NT>
+cudaError_t gate_up_nt(const moe_shape_t& s, const uint16_t* x, const Bank& gu, const Workspace& ws, int grid,
+                       size_t smem, cudaStream_t stream) {
+  auto k = decode_gate_up_kernel<FMT, NT>;
+  cudaError_t err = allow_smem(k, smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, x, gu, s.inter, s.top_k,
+                    (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows, ws.act,
+                    ws.status);
+}
+
+template <int FMT>
+cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws, int grid,
+                        size_t smem, cudaStream_t stream) {
+  // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, x, gu, ws, grid, smem, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, x, gu, ws, grid, smem, stream);
+  return gate_up_nt<FMT, kDecNT>(s, x, gu, ws, grid, smem, stream);
+}
+
+template <int FMT, int NT>
+cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int grid,
+                    size_t smem, cudaStream_t stream) {
+  auto k = decode_down_kernel<FMT, NT>;
+  cudaError_t err = allow_smem(k, smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, dn, T, s.top_k, (const int32_t*)ws.touched,
+                    (const int32_t*)ws.offsets, (const uint16_t*)ws.act, (const float*)ws.topk_w,
+                    (const int32_t*)ws.pos, ws.y, out, ws.status, ws.tile_counters);
+}
+
+template <int FMT>
+cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int grid,
+                     size_t smem, cudaStream_t stream) {
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, grid, smem, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, grid, smem, stream);
+  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, grid, smem, stream);
+}
 
 }  // namespace
 
@@ -318,37 +425,19 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
   const int slots = max_touched(T, s.top_k, s.num_experts);
   const int grid = slots * (s.inter / kDecRows);
   if (grid == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128)
-    decode_gate_up_kernel<MOE_FMT_INT4_G128><<<grid, kDecWarps * 32, 0, stream>>>(
-        x, gu, s.inter, s.top_k, ws.touched, ws.offsets, ws.sorted_rows, ws.act);
-  else
-    decode_gate_up_kernel<MOE_FMT_MXFP4_G32><<<grid, kDecWarps * 32, 0, stream>>>(
-        x, gu, s.inter, s.top_k, ws.touched, ws.offsets, ws.sorted_rows, ws.act);
-  return cudaGetLastError();
+  const size_t smem = gate_up_smem(s.fmt, s.hidden);
+  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, grid, smem, stream);
+  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, grid, smem, stream);
 }
 
-cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                               cudaStream_t stream) {
+cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
+                                       uint16_t* out, cudaStream_t stream) {
   const int slots = max_touched(T, s.top_k, s.num_experts);
-  const int grid = slots * (s.hidden / (kDecRows * kDecWarps));
+  const int grid = slots * (s.hidden / kDownFeatures);
   if (grid == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128)
-    decode_down_kernel<MOE_FMT_INT4_G128><<<grid, kDecWarps * 32, 0, stream>>>(dn, ws.touched, ws.offsets,
-                                                                                ws.act, ws.y);
-  else
-    decode_down_kernel<MOE_FMT_MXFP4_G32><<<grid, kDecWarps * 32, 0, stream>>>(dn, ws.touched, ws.offsets,
-                                                                                ws.act, ws.y);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_decode_combine(const moe_shape_t& s, int T, const Workspace& ws, uint16_t* out,
-                                  cudaStream_t stream) {
-  const long n4 = long(T) * s.hidden / 4;
-  if (n4 == 0) return cudaSuccess;
-  const int block = 256;
-  decode_combine_kernel<<<unsigned((n4 + block - 1) / block), block, 0, stream>>>(ws.y, ws.topk_w, ws.pos, T,
-                                                                                  s.hidden, s.top_k, out);
-  return cudaGetLastError();
+  const size_t smem = down_smem(s.fmt, s.inter);
+  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, grid, smem, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, grid, smem, stream);
 }
 
 }  // namespace moe

@@ -35,8 +35,15 @@ struct Bank {
 };
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
+// The first kStatusBytes of a workspace: the status word, the fused-routing
+// completion counter and per-feature-tile combine counters.  Zeroed once by
+// moe_workspace_init; every kernel that counts resets its counter to zero.
+constexpr size_t kStatusBytes = 4096;
+
 struct Workspace {
-  uint32_t* status;       // [64] status word + scratch counters
+  uint32_t* status;       // status word (device-side failures)
+  int32_t* route_counter; // CTAs done in the fused small-batch routing kernel
+  int32_t* tile_counters; // decode down kernel: CTAs done per 64-feature tile
   float* logits;          // [T, E]
   int32_t* topk_ids;      // [T, k]
   float* topk_w;          // [T, k]
@@ -62,11 +69,13 @@ cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, i
                            cudaStream_t stream);
 
 // route.cu
-cudaError_t launch_router_gemv(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
-                               cudaStream_t stream);
+// Fused router GEMV + top-k + permutation for T <= kDecodeMaxT.
+cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                               const Workspace& ws, int block_n, cudaStream_t stream);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t stream);
-// Small-T routing state: permutation + touched-expert list in one CTA.
+// Small-T permutation (R = T*k <= 1024) in one CTA, with the touched-expert
+// list and the token-block prefix.
 cudaError_t launch_permute_small(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
                                  int32_t* pos, int32_t* touched, int32_t* tile_base, int block_n,
                                  cudaStream_t stream);
@@ -79,10 +88,8 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 // decode.cu
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const Workspace& ws, cudaStream_t stream);
-cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                               cudaStream_t stream);
-cudaError_t launch_decode_combine(const moe_shape_t& s, int T, const Workspace& ws, uint16_t* out,
-                                  cudaStream_t stream);
+cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
+                                       uint16_t* out, cudaStream_t stream);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile

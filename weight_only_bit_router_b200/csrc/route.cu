@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
@@ -21,11 +22,10 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kRgExpertsPerCta = 2;
 constexpr int kRgWarpsPerExpert = 4;
+constexpr int kRgThreads = 32 * kRgExpertsPerCta * kRgWarpsPerExpert;
 
-__global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __restrict__ x,
-                                                          const uint16_t* __restrict__ wr, int T, int H, int E,
-                                                          float* __restrict__ logits) {
-  __shared__ float part[kRgExpertsPerCta][kRgWarpsPerExpert][kDecodeMaxT];
+MOE_DEV void router_gemv_block(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, int T, int H, int E,
+                               float* __restrict__ logits, float (*part)[kRgWarpsPerExpert][kDecodeMaxT]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int le = warp / kRgWarpsPerExpert, ks = warp % kRgWarpsPerExpert;
   const int e = blockIdx.x * kRgExpertsPerCta + le;
@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
     const int span = H / kRgWarpsPerExpert;  // multiple of 16
     const int c0 = ks * span;
     for (int c = c0 + lane * 8; c < c0 + span; c += 256) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wr + size_t(e) * H + c);
+      const uint4 wv = ldg_nc_v4(wr + size_t(e) * H + c);
       const float w8[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
                            bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
 #pragma unroll
@@ -78,12 +78,12 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
 // top-k: one warp per token.  Lane l holds experts l, l+32, ... (E <= 1024).
 // Each round takes the largest remaining value, ties to the lower index.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                                                   int T, int E, int k, int32_t* __restrict__ ids,
-                                                   float* __restrict__ wout) {
+// Top-k of one token's logits by one warp (lane l holds experts l, l+32, ...,
+// E <= 1024); each round takes the largest remaining value, ties to the lower
+// index.  Logits are read through L2 (they may come from other CTAs).
+MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
+                       int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
   float v[32];
   const int per = (E + 31) / 32;
 #pragma unroll
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     const int e = i * 32 + lane;
     float val = -FLT_MAX;
     if (i < per && e < E) {
-      val = logits[size_t(t) * E + e];
+      val = __ldcg(row + e);
       if (bias) val = val + bias[e];  // fp32 add
     }
     v[i] = val;
@@ -100,7 +100,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    // local best among untaken entries (smallest index first on ties: i ascending)
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
@@ -125,9 +124,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane < k) {
-    ids[size_t(t) * k + lane] = my_id;
-    wout[size_t(t) * k + lane] = ex / sum;
+    ids[lane] = my_id;
+    wout[lane] = ex / sum;
   }
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                   int T, int E, int k, int32_t* __restrict__ ids,
+                                                   float* __restrict__ wout) {
+  pdl_wait();
+  pdl_trigger();
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  warp_topk(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k);
 }
 
 // Exclusive scan of n <= 1024 ints held in smem by a 1024-thread block; the
@@ -161,60 +170,153 @@ __device__ int block_exclusive_scan_1024(int* data, int n, int* warp_tot) {
   return total;
 }
 
-// ---------------------------------------------------------------------------
-// Small permutation: one 1024-thread CTA, R = T*k <= 1024 rows.
-// Also writes the touched-expert list and the per-expert token-block prefix.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __restrict__ ids, int R, int E,
-                                                             int32_t* __restrict__ offsets,
-                                                             int32_t* __restrict__ sorted_rows,
-                                                             int32_t* __restrict__ pos,
-                                                             int32_t* __restrict__ touched,
-                                                             int32_t* __restrict__ tile_base, int block_n) {
-  __shared__ int s_ids[1024];
-  __shared__ int s_cnt[kMaxExperts];
-  __shared__ int s_off[kMaxExperts];
-  __shared__ int s_aux[kMaxExperts];
-  __shared__ int s_wt[33];
-  const int tid = threadIdx.x;
-  int my_e = -1;
-  if (tid < R) {
-    my_e = ids[tid];
-    if (my_e < 0 || my_e >= E) my_e = -1;  // contract violation: row dropped
-    s_ids[tid] = my_e;
+// Exclusive scan of n <= 4 * blockDim.x ints in smem by a block of 256
+// threads (4 consecutive items per thread); returns the total.
+__device__ int block_exclusive_scan_256x4(int* data, int n, int* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int loc[4], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = tid * 4 + i;
+    loc[i] = idx < n ? data[idx] : 0;
+    sum += loc[i];
   }
-  if (tid < E) s_cnt[tid] = 0;
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
-  if (my_e >= 0) atomicAdd(&s_cnt[my_e], 1);
-  __syncthreads();
-  if (tid < E) {
-    s_off[tid] = s_cnt[tid];
-    s_aux[tid] = s_cnt[tid] > 0 ? 1 : 0;
+  if (warp == 0) {
+    const int w = lane < 8 ? warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < 8) warp_tot[lane] = wi - w;
+    if (lane == 7) warp_tot[32] = wi;
   }
   __syncthreads();
-  const int total = block_exclusive_scan_1024(s_off, E, s_wt);
-  if (tid < E) offsets[tid] = s_off[tid];
+  int run = incl - sum + warp_tot[warp];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = tid * 4 + i;
+    if (idx < n) data[idx] = run;
+    run += loc[i];
+  }
+  const int total = warp_tot[32];
+  __syncthreads();
+  return total;
+}
+
+struct SmallPermSmem {
+  int ids[1024];
+  int cnt[kMaxExperts];
+  int off[kMaxExperts];
+  int aux[kMaxExperts];
+  int wt[33];
+};
+
+// Stable counting sort of R <= 1024 rows by expert in one 256-thread block,
+// plus the touched-expert list and the per-expert token-block prefix.  The
+// block's ids must already be in sm.ids (values outside [0, E) are dropped).
+__device__ void small_permutation_block(SmallPermSmem& sm, int R, int E, int32_t* __restrict__ offsets,
+                                        int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
+                                        int32_t* __restrict__ touched, int32_t* __restrict__ tile_base,
+                                        int block_n) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int e = tid; e < E; e += nt) sm.cnt[e] = 0;
+  __syncthreads();
+  for (int r = tid; r < R; r += nt) {
+    const int e = sm.ids[r];
+    if (e >= 0 && e < E) atomicAdd(&sm.cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += nt) {
+    sm.off[e] = sm.cnt[e];
+    sm.aux[e] = sm.cnt[e] > 0 ? 1 : 0;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan_256x4(sm.off, E, sm.wt);
+  for (int e = tid; e < E; e += nt) offsets[e] = sm.off[e];
   if (tid == 0) offsets[E] = total;
-  // stable rank: rows of the same expert with a lower index
-  if (my_e >= 0) {
+  for (int r = tid; r < R; r += nt) {
+    const int e = sm.ids[r];
+    if (e < 0 || e >= E) {
+      pos[r] = -1;
+      continue;
+    }
     int rank = 0;
-    for (int r = 0; r < tid; ++r) rank += (s_ids[r] == my_e);
-    const int p = s_off[my_e] + rank;
-    sorted_rows[p] = tid;
-    pos[tid] = p;
-  } else if (tid < R) {
-    pos[tid] = -1;
+    for (int r2 = 0; r2 < r; ++r2) rank += (sm.ids[r2] == e);
+    const int p = sm.off[e] + rank;
+    sorted_rows[p] = r;
+    pos[r] = p;
   }
-  // touched experts, ascending
-  const int ntouched = block_exclusive_scan_1024(s_aux, E, s_wt);
-  if (tid < E && s_cnt[tid] > 0) touched[1 + s_aux[tid]] = tid;
+  const int ntouched = block_exclusive_scan_256x4(sm.aux, E, sm.wt);
+  for (int e = tid; e < E; e += nt)
+    if (sm.cnt[e] > 0) touched[1 + sm.aux[e]] = e;
   if (tid == 0) touched[0] = ntouched;
-  // token-block prefix for the grouped GEMMs
-  if (tid < E) s_aux[tid] = (s_cnt[tid] + block_n - 1) / block_n;
   __syncthreads();
-  const int nblocks = block_exclusive_scan_1024(s_aux, E, s_wt);
-  if (tid < E) tile_base[tid] = s_aux[tid];
+  for (int e = tid; e < E; e += nt) sm.aux[e] = (sm.cnt[e] + block_n - 1) / block_n;
+  __syncthreads();
+  const int nblocks = block_exclusive_scan_256x4(sm.aux, E, sm.wt);
+  for (int e = tid; e < E; e += nt) tile_base[e] = sm.aux[e];
   if (tid == 0) tile_base[E] = nblocks;
+}
+
+__global__ void __launch_bounds__(256) permute_small_kernel(const int32_t* __restrict__ ids, int R, int E,
+                                                            int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ sorted_rows,
+                                                            int32_t* __restrict__ pos,
+                                                            int32_t* __restrict__ touched,
+                                                            int32_t* __restrict__ tile_base, int block_n) {
+  __shared__ SmallPermSmem sm;
+  pdl_wait();
+  pdl_trigger();
+  for (int r = threadIdx.x; r < R; r += blockDim.x) sm.ids[r] = ids[r];
+  __syncthreads();
+  small_permutation_block(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+}
+
+// ---------------------------------------------------------------------------
+// Fused small-batch routing (T <= 32): every CTA computes the logits of two
+// experts for all tokens; the last CTA to finish (counted in the workspace)
+// runs top-k for every token (one warp per token), then the stable
+// permutation, the touched-expert list and the token-block prefix.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kRgThreads) route_small_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
+    int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
+    int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n, int32_t* done_counter) {
+  __shared__ float part[kRgExpertsPerCta][kRgWarpsPerExpert][kDecodeMaxT];
+  __shared__ SmallPermSmem sm;
+  __shared__ int s_last;
+  pdl_wait();
+  pdl_trigger();
+  router_gemv_block(x, wr, T, H, E, logits, part);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(done_counter, 1) == int(gridDim.x) - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int t = warp; t < T; t += nwarps)
+    warp_topk(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k);
+  __syncthreads();
+  __threadfence_block();
+  const int R = T * k;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) sm.ids[r] = __ldcg(ids + r);
+  __syncthreads();
+  small_permutation_block(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  if (threadIdx.x == 0) *done_counter = 0;  // ready for the next call
 }
 
 // ---------------------------------------------------------------------------
@@ -229,6 +331,8 @@ __global__ void __launch_bounds__(kPermRows) permute_hist_kernel(const int32_t* 
                                                                  int32_t* __restrict__ block_hist,
                                                                  int32_t* __restrict__ row_rank) {
   extern __shared__ int warp_cnt[];  // [8][E]
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = blockIdx.x * kPermRows + tid;
   for (int i = tid; i < 8 * E; i += kPermRows) warp_cnt[i] = 0;
@@ -269,6 +373,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int nblk, int E, int
   __shared__ int s_off[kMaxExperts];
   __shared__ int s_aux[kMaxExperts];
   __shared__ int s_wt[33];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int e = tid / G, sub = tid % G;
   const int chunk = (nblk + G - 1) / G;
@@ -324,6 +430,8 @@ __global__ void __launch_bounds__(kPermRows) permute_place_kernel(const int32_t*
                                                                   const int32_t* __restrict__ block_base,
                                                                   int32_t* __restrict__ sorted_rows,
                                                                   int32_t* __restrict__ pos) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x * kPermRows + threadIdx.x;
   if (r >= R) return;
   const int e = ids[r];
@@ -347,11 +455,12 @@ size_t permute_large_hist_bytes(int T, int E, int k) {
   return nblk * size_t(E) * sizeof(int32_t);
 }
 
-cudaError_t launch_router_gemv(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
-                               cudaStream_t stream) {
+cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                               const Workspace& ws, int block_n, cudaStream_t stream) {
   const int grid = (E + kRgExpertsPerCta - 1) / kRgExpertsPerCta;
-  router_gemv_kernel<<<grid, 32 * kRgExpertsPerCta * kRgWarpsPerExpert, 0, stream>>>(x, wr, T, H, E, logits);
-  return cudaGetLastError();
+  return launch_pdl(route_small_kernel, dim3(grid), dim3(kRgThreads), 0, stream, x, wr, bias, T, H, E, k, ws.logits,
+                    ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched, ws.tile_base, block_n,
+                    ws.route_counter);
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
@@ -359,16 +468,14 @@ cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, in
   if (T == 0) return cudaSuccess;
   const int warps_per_block = 8;
   const int grid = (T + warps_per_block - 1) / warps_per_block;
-  topk_kernel<<<grid, 32 * warps_per_block, 0, stream>>>(logits, bias, T, E, k, ids, w);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(grid), dim3(32 * warps_per_block), 0, stream, logits, bias, T, E, k, ids, w);
 }
 
 cudaError_t launch_permute_small(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
                                  int32_t* pos, int32_t* touched, int32_t* tile_base, int block_n,
                                  cudaStream_t stream) {
-  permute_small_kernel<<<1, 1024, 0, stream>>>(ids, T * k, E, offsets, sorted_rows, pos, touched, tile_base,
-                                               block_n);
-  return cudaGetLastError();
+  return launch_pdl(permute_small_kernel, dim3(1), dim3(256), 0, stream, ids, T * k, E, offsets, sorted_rows, pos,
+                    touched, tile_base, block_n);
 }
 
 cudaError_t launch_permute_large(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* sorted_rows,
@@ -378,12 +485,16 @@ cudaError_t launch_permute_large(const int32_t* ids, int T, int E, int k, int32_
   const int nblk = (R + kPermRows - 1) / kPermRows;
   if (nblk == 0) return cudaSuccess;
   const size_t smem = size_t(8) * E * sizeof(int);
-  permute_hist_kernel<<<nblk, kPermRows, smem, stream>>>(ids, R, E, block_hist, pos);
+  cudaError_t err = launch_pdl(permute_hist_kernel, dim3(nblk), dim3(kPermRows), smem, stream, ids, R, E,
+                               block_hist, pos);
+  if (err != cudaSuccess) return err;
   int G = 1;
   while (G * 2 * E <= 1024) G *= 2;
-  permute_scan_kernel<<<1, 1024, 0, stream>>>(nblk, E, G, block_hist, offsets, touched, tile_base, block_n);
-  permute_place_kernel<<<nblk, kPermRows, 0, stream>>>(ids, R, E, block_hist, sorted_rows, pos);
-  return cudaGetLastError();
+  err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, nblk, E, G, block_hist, offsets, touched,
+                   tile_base, block_n);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(permute_place_kernel, dim3(nblk), dim3(kPermRows), 0, stream, ids, R, E,
+                    (const int32_t*)block_hist, sorted_rows, pos);
 }
 
 }  // namespace moe
