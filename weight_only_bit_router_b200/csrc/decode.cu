@@ -130,16 +130,21 @@ MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, 
   }
 }
 
-// Stage `rows` consecutive weight rows (codes + scales) of a bank into shared
-// memory with two bulk copies on `bar`; one thread calls this.
+// Bytes staged for `rows` consecutive weight rows (codes + scales).
+template <int FMT>
+MOE_DEV uint32_t staged_bytes(const Bank& bk, int rows) {
+  return uint32_t(rows) * (bk.K / 2) + uint32_t(rows) * scale_row_bytes(FMT, bk.K);
+}
+
+// Start the two bulk copies (codes, scales) of `rows` consecutive weight rows
+// of a bank into shared memory, completing on `bar`.  The caller has already
+// announced the total bytes with ONE arrive.expect_tx on `bar`.
 template <int FMT>
 MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, uint8_t* s_scales, uint64_t* bar) {
   const uint32_t cbytes = uint32_t(rows) * (bk.K / 2);
   const int sb = scale_row_bytes(FMT, bk.K);
-  const uint32_t sbytes = uint32_t(rows) * sb;
-  mbar_arrive_expect_tx(bar, cbytes + sbytes);
   bulk_g2s(s_codes, bk.codes + row0 * (bk.K / 2), cbytes, bar);
-  bulk_g2s(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, sbytes, bar);
+  bulk_g2s(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar);
 }
 
 // Wait for the staged rows (bounded); false if the wait gave up.
@@ -183,6 +188,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar, 2 * staged_bytes<FMT>(gu, kDecRows));
     stage_rows<FMT>(gu, row_g, kDecRows, s_cg, s_sg, bar);
     stage_rows<FMT>(gu, row_u, kDecRows, s_cu, s_su, bar);
   }
@@ -289,6 +295,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar, staged_bytes<FMT>(dn, kDownFeatures));
     stage_rows<FMT>(dn, long(e) * H + fbase, kDownFeatures, s_c, s_s, bar);
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
