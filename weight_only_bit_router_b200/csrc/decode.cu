@@ -17,6 +17,8 @@
 // depend on the order of its terms, so weights and activations only need the
 // same assignment; this one lets one nibble-extraction instruction produce a
 // fragment register directly.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "launch.h"
@@ -153,12 +155,40 @@ MOE_DEV bool wait_staged(uint64_t* bar, uint32_t* status) {
   return mbar_wait(bar, 0, &never, status);
 }
 
+// Per-stage shared-memory layout of a work unit: codes then scales, each
+// matrix slice 16-byte aligned.
+struct UnitLayout {
+  int cbytes, sbytes, sbytes_pad, stage_bytes;
+};
+
+MOE_DEV UnitLayout unit_layout(int fmt, int K, int rows, int mats) {
+  UnitLayout l;
+  l.cbytes = rows * (K / 2);
+  l.sbytes = rows * scale_row_bytes(fmt, K);
+  l.sbytes_pad = (l.sbytes + 15) & ~15;
+  l.stage_bytes = mats * (l.cbytes + l.sbytes_pad);
+  return l;
+}
+
 // ---------------------------------------------------------------------------
-// gate_up + SwiGLU.  grid = (max experts touched) x (I / 16).  A CTA stages
-// the 16 gate rows and the 16 matching up rows of its expert; its 4 warps
-// split K, partial tiles are summed in shared memory, and
-// a = bf16(silu(gate) * up) goes to act[p][f] for the expert's sorted rows p.
+// gate_up + SwiGLU, persistent.  Work unit u = (touched slot u / (I/16),
+// features 16*(u % (I/16)) ...): the 16 gate rows and the 16 matching up rows
+// of that expert.  A CTA walks units u = blockIdx.x + i * gridDim.x with two
+// shared-memory stages: the bulk copies of unit i+2 start as soon as unit i's
+// stage is free, so weight streaming overlaps the MMAs.  The CTA's 4 warps
+// split K; partial tiles are summed in shared memory; a = bf16(silu(gate) *
+// up) goes to act[p][f] for the expert's sorted rows p.
 // ---------------------------------------------------------------------------
+template <int FMT>
+MOE_DEV void issue_gate_up_unit(const Bank& gu, int I, const int32_t* touched, int ftiles, int u, uint8_t* stage,
+                                const UnitLayout& L, uint64_t* bar) {
+  const int e = touched[1 + u / ftiles];
+  const long row_g = long(e) * gu.N + (u % ftiles) * kDecRows;
+  mbar_arrive_expect_tx(bar, 2 * staged_bytes<FMT>(gu, kDecRows));
+  stage_rows<FMT>(gu, row_g, kDecRows, stage, stage + 2 * L.cbytes, bar);
+  stage_rows<FMT>(gu, row_g + I, kDecRows, stage + L.cbytes, stage + 2 * L.cbytes + L.sbytes_pad, bar);
+}
+
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
@@ -166,109 +196,127 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
     uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = gu.K;
-  const int cbytes = kDecRows * (K / 2);
-  const int sbytes = kDecRows * scale_row_bytes(FMT, K);
-  const int red_bytes = kDecWarps * NT * 2 * 4 * 32 * 4;
-  uint8_t* s_cg = smem;                              // gate codes, later the reduction buffer
-  uint8_t* s_cu = s_cg + cbytes;                     // up codes
-  uint8_t* s_sg = smem + max(2 * cbytes, red_bytes); // gate scales
-  uint8_t* s_su = s_sg + sbytes;                     // up scales
-  uint64_t* bar = reinterpret_cast<uint64_t*>(s_su + ((sbytes + 15) & ~15));
-  float* red = reinterpret_cast<float*>(smem);       // [warp][tile][gate/up][4][lane]
+  // stage layout: [gate codes][up codes][gate scales][up scales]
+  const UnitLayout L = unit_layout(FMT, K, kDecRows, 2);
+  float* red = reinterpret_cast<float*>(smem + 2 * L.stage_bytes);  // [warp][tile][gate/up][4][lane]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kDecWarps * NT * 2 * 4 * 32);
 
   pdl_wait();
   pdl_trigger();
   const int ftiles = I / kDecRows;
-  const int slot = blockIdx.x / ftiles;
-  const int f0 = (blockIdx.x % ftiles) * kDecRows;
-  if (slot >= touched[0]) return;
-  const int e = touched[1 + slot];
-  const long row_g = long(e) * gu.N + f0;
-  const long row_u = row_g + I;
+  const int n_units = touched[0] * ftiles;
+  if (int(blockIdx.x) >= n_units) return;
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar, 2 * staged_bytes<FMT>(gu, kDecRows));
-    stage_rows<FMT>(gu, row_g, kDecRows, s_cg, s_sg, bar);
-    stage_rows<FMT>(gu, row_u, kDecRows, s_cu, s_su, bar);
+    for (int st = 0; st < 2; ++st) {
+      const int u = blockIdx.x + st * gridDim.x;
+      if (u < n_units) issue_gate_up_unit<FMT>(gu, I, touched, ftiles, u, smem + st * L.stage_bytes, L, &bars[st]);
+    }
   }
-  const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
+  __syncthreads();  // barriers initialised before anyone waits on them
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const int nblk = (K + 127) / 128;
-  const int ntiles = (n_e + 7) / 8;
-  __syncthreads();  // barrier initialised before anyone waits on it
-  const bool ok = wait_staged(bar, status);
-
-  for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
-    float acc[NT][2][4];
+  int i = 0;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+    const int st = i & 1;
+    const uint8_t* s_cg = smem + st * L.stage_bytes;
+    const uint8_t* s_cu = s_cg + L.cbytes;
+    const uint8_t* s_sg = s_cg + 2 * L.cbytes;
+    const uint8_t* s_su = s_sg + L.sbytes_pad;
+    const int e = touched[1 + u / ftiles];
+    const int f0 = (u % ftiles) * kDecRows;
+    const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
+    const int ntiles = (n_e + 7) / 8;
+    volatile int never = 0;
+    const bool ok = mbar_wait(&bars[st], (i >> 1) & 1, &never, status);
+    for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
+      float acc[NT][2][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+      for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[j][t][i] = 0.f;
-    const uint16_t* xrow[NT];
-    bool xval[NT];
+          for (int c = 0; c < 4; ++c) acc[j][t][c] = 0.f;
+      const uint16_t* xrow[NT];
+      bool xval[NT];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int c = (nt0 + j) * 8 + g;
-      xval[j] = c < n_e;
-      xrow[j] = x + size_t(xval[j] ? sorted_rows[p0 + c] / top_k : 0) * K;
-    }
-    if (ok) {
-      for (int b = warp; b < nblk; b += kDecWarps) {
-        const int kb = b * 128;
-        const RowChunk g0 = smem_row_chunk<FMT>(s_cg, s_sg, g, K, kb, q);
-        const RowChunk g1 = smem_row_chunk<FMT>(s_cg, s_sg, g + 8, K, kb, q);
-        const RowChunk u0 = smem_row_chunk<FMT>(s_cu, s_su, g, K, kb, q);
-        const RowChunk u1 = smem_row_chunk<FMT>(s_cu, s_su, g + 8, K, kb, q);
+      for (int j = 0; j < NT; ++j) {
+        const int c = (nt0 + j) * 8 + g;
+        xval[j] = c < n_e;
+        xrow[j] = x + size_t(xval[j] ? sorted_rows[p0 + c] / top_k : 0) * K;
+      }
+      if (ok) {
+        for (int b = warp; b < nblk; b += kDecWarps) {
+          const int kb = b * 128;
+          const RowChunk g0 = smem_row_chunk<FMT>(s_cg, s_sg, g, K, kb, q);
+          const RowChunk g1 = smem_row_chunk<FMT>(s_cg, s_sg, g + 8, K, kb, q);
+          const RowChunk u0 = smem_row_chunk<FMT>(s_cu, s_su, g, K, kb, q);
+          const RowChunk u1 = smem_row_chunk<FMT>(s_cu, s_su, g + 8, K, kb, q);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (nt0 + j >= ntiles) break;
-          uint32_t bf[8][2];
-          load_act_frags(xrow[j], K, kb, q, xval[j], bf);
-          mma_block<FMT>(acc[j][0], g0, g1, bf);
-          mma_block<FMT>(acc[j][1], u0, u1, bf);
+          for (int j = 0; j < NT; ++j) {
+            if (nt0 + j >= ntiles) break;
+            uint32_t bf[8][2];
+            load_act_frags(xrow[j], K, kb, q, xval[j], bf);
+            mma_block<FMT>(acc[j][0], g0, g1, bf);
+            mma_block<FMT>(acc[j][1], u0, u1, bf);
+          }
         }
       }
-    }
-    __syncthreads();  // the codes buffer becomes the reduction buffer
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+      for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) red[(((warp * NT + j) * 2 + t) * 4 + i) * 32 + lane] = acc[j][t][i];
-    __syncthreads();
-    // warp w < NT finishes token tile nt0 + w
-    const int j = warp;
-    if (ok && j < NT && nt0 + j < ntiles) {
+          for (int c = 0; c < 4; ++c) red[(((warp * NT + j) * 2 + t) * 4 + c) * 32 + lane] = acc[j][t][c];
+      __syncthreads();
+      // warp w < NT finishes token tile nt0 + w
+      const int j = warp;
+      if (ok && j < NT && nt0 + j < ntiles) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float gs = 0.f, us = 0.f;
+        for (int c = 0; c < 4; ++c) {
+          float gs = 0.f, us = 0.f;
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-          gs += red[(((w * NT + j) * 2 + 0) * 4 + i) * 32 + lane];
-          us += red[(((w * NT + j) * 2 + 1) * 4 + i) * 32 + lane];
+          for (int w = 0; w < kDecWarps; ++w) {
+            gs += red[(((w * NT + j) * 2 + 0) * 4 + c) * 32 + lane];
+            us += red[(((w * NT + j) * 2 + 1) * 4 + c) * 32 + lane];
+          }
+          // c0,c1: feature g, tokens 2q, 2q+1; c2,c3: feature g+8
+          const int col = (nt0 + j) * 8 + 2 * q + (c & 1);
+          const int f = f0 + g + ((c >> 1) << 3);
+          if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(gs, us));
         }
-        // c0,c1: feature g, tokens 2q, 2q+1; c2,c3: feature g+8
-        const int col = (nt0 + j) * 8 + 2 * q + (i & 1);
-        const int f = f0 + g + ((i >> 1) << 3);
-        if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(gs, us));
       }
+      __syncthreads();
     }
-    __syncthreads();
+    // stage st is free again: start the unit two steps ahead
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();  // the stage's generic-proxy reads before the bulk copies refill it
+      const int u2 = u + 2 * gridDim.x;
+      if (u2 < n_units) issue_gate_up_unit<FMT>(gu, I, touched, ftiles, u2, smem + st * L.stage_bytes, L, &bars[st]);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// down projection + deterministic combine.  grid = (max experts touched) x
-// (H / 64).  A CTA stages 64 rows of its expert's down bank; each warp owns
-// 16 features over K = I and writes y[p][f] in fp32.  The last CTA to finish
-// a feature tile (counted in the workspace) sums the k expert outputs of every
-// token in slot order j = 0..k-1 and writes the bf16 output for that tile.
+// down projection + deterministic combine, persistent.  Work unit u = (touched
+// slot u / (H/64), features 64*(u % (H/64)) ...): 64 rows of the expert's
+// down bank, two shared-memory stages as above.  Each warp owns 16 features
+// over K = I and writes y[p][f] in fp32.  The CTA that completes the last
+// unit of a feature tile (counted in the workspace) sums the k expert outputs
+// of every token in slot order j = 0..k-1 and writes that tile's bf16 output.
 // ---------------------------------------------------------------------------
+template <int FMT>
+MOE_DEV void issue_down_unit(const Bank& dn, const int32_t* touched, int ftiles, int u, uint8_t* stage,
+                             const UnitLayout& L, uint64_t* bar) {
+  const int e = touched[1 + u / ftiles];
+  const long row0 = long(e) * dn.N + (u % ftiles) * kDownFeatures;
+  mbar_arrive_expect_tx(bar, staged_bytes<FMT>(dn, kDownFeatures));
+  stage_rows<FMT>(dn, row0, kDownFeatures, stage, stage + L.cbytes, bar);
+}
+
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
     Bank dn, int T, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
@@ -276,102 +324,140 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
     float* __restrict__ y, uint16_t* __restrict__ out, uint32_t* status, int32_t* tile_counters) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = dn.N, K = dn.K;  // K = I
-  const int cbytes = kDownFeatures * (K / 2);
-  const int sbytes = kDownFeatures * scale_row_bytes(FMT, K);
-  uint8_t* s_c = smem;
-  uint8_t* s_s = smem + cbytes;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(s_s + ((sbytes + 15) & ~15));
+  const UnitLayout L = unit_layout(FMT, K, kDownFeatures, 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * L.stage_bytes);
   __shared__ int s_last;
 
   pdl_wait();
   pdl_trigger();
   const int ftiles = H / kDownFeatures;
-  const int slot = blockIdx.x / ftiles;
-  const int ft = blockIdx.x % ftiles;
   const int n_touched = touched[0];
-  if (slot >= n_touched) return;
-  const int e = touched[1 + slot];
-  const int fbase = ft * kDownFeatures;
+  const int n_units = n_touched * ftiles;
+  if (int(blockIdx.x) >= n_units) return;
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar, staged_bytes<FMT>(dn, kDownFeatures));
-    stage_rows<FMT>(dn, long(e) * H + fbase, kDownFeatures, s_c, s_s, bar);
+    for (int st = 0; st < 2; ++st) {
+      const int u = blockIdx.x + st * gridDim.x;
+      if (u < n_units) issue_down_unit<FMT>(dn, touched, ftiles, u, smem + st * L.stage_bytes, L, &bars[st]);
+    }
   }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int f0 = fbase + warp * kDecRows;
-  const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
   const int nblk = (K + 127) / 128;
-  const int ntiles = (n_e + 7) / 8;
-  __syncthreads();
-  const bool ok = wait_staged(bar, status);
   const int r0 = warp * kDecRows + g;  // staged row of this lane
-  for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
-    float acc[NT][4];
+  int i = 0;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+    const int st = i & 1;
+    const uint8_t* s_c = smem + st * L.stage_bytes;
+    const uint8_t* s_s = s_c + L.cbytes;
+    const int e = touched[1 + u / ftiles];
+    const int ft = u % ftiles;
+    const int f0 = ft * kDownFeatures + warp * kDecRows;
+    const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
+    const int ntiles = (n_e + 7) / 8;
+    volatile int never = 0;
+    const bool ok = mbar_wait(&bars[st], (i >> 1) & 1, &never, status);
+    for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
+      float acc[NT][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+      for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-    for (int b = 0; b < nblk; ++b) {
-      const int kb = b * 128;
-      const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, r0, K, kb, q);
-      const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, r0 + 8, K, kb, q);
+        for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
+      for (int b = 0; b < nblk; ++b) {
+        const int kb = b * 128;
+        const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, r0, K, kb, q);
+        const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, r0 + 8, K, kb, q);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (nt0 + j >= ntiles) break;
+          const int col = (nt0 + j) * 8 + g;
+          uint32_t bf[8][2];
+          load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
+          mma_block<FMT>(acc[j], c0, c1, bf);
+        }
+      }
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        if (nt0 + j >= ntiles) break;
-        const int col = (nt0 + j) * 8 + g;
-        uint32_t bf[8][2];
-        load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
-        mma_block<FMT>(acc[j], c0, c1, bf);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = (nt0 + j) * 8 + 2 * q + (c & 1);
+          const int f = f0 + g + ((c >> 1) << 3);
+          if (nt0 + j < ntiles && col < n_e) y[size_t(p0 + col) * H + f] = acc[j][c];
+        }
       }
     }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = (nt0 + j) * 8 + 2 * q + (i & 1);
-        const int f = f0 + g + ((i >> 1) << 3);
-        if (nt0 + j < ntiles && col < n_e) y[size_t(p0 + col) * H + f] = acc[j][i];
+    __syncthreads();  // stage st consumed, y tile written
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();
+      const int u2 = u + 2 * gridDim.x;
+      if (u2 < n_units) issue_down_unit<FMT>(dn, touched, ftiles, u2, smem + st * L.stage_bytes, L, &bars[st]);
+      __threadfence();
+      s_last = atomicAdd(&tile_counters[ft], 1) == n_touched - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      // every expert's y for this feature tile is written: combine it
+      __threadfence();
+      const int fbase = ft * kDownFeatures;
+      for (int idx = threadIdx.x; idx < T * kDownFeatures; idx += blockDim.x) {
+        const int t = idx / kDownFeatures;
+        const int f = fbase + idx % kDownFeatures;
+        float sum = 0.f;
+        for (int j = 0; j < top_k; ++j) {
+          const int p = pos[size_t(t) * top_k + j];
+          if (p < 0) continue;
+          sum = fmaf(topk_w[size_t(t) * top_k + j], __ldcg(y + size_t(p) * H + f), sum);
+        }
+        out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
       }
+      if (threadIdx.x == 0) tile_counters[ft] = 0;  // ready for the next call
+      __syncthreads();
     }
   }
-  // the last CTA of this feature tile combines it
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(&tile_counters[ft], 1) == n_touched - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < T * kDownFeatures; i += blockDim.x) {
-    const int t = i / kDownFeatures;
-    const int f = fbase + i % kDownFeatures;
-    float s = 0.f;
-    for (int j = 0; j < top_k; ++j) {
-      const int p = pos[size_t(t) * top_k + j];
-      if (p < 0) continue;
-      s = fmaf(topk_w[size_t(t) * top_k + j], __ldcg(y + size_t(p) * H + f), s);
-    }
-    out[size_t(t) * H + f] = f32_to_bf16_rn(s);
-  }
-  if (threadIdx.x == 0) tile_counters[ft] = 0;  // ready for the next call
 }
 
 int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
 
-size_t gate_up_smem(int fmt, int K) {
-  const int cbytes = kDecRows * (K / 2);
-  const int sbytes = kDecRows * scale_row_bytes(fmt, K);
-  const int red_bytes = kDecWarps * kDecNT * 2 * 4 * 32 * 4;
-  return size_t(std::max(2 * cbytes, red_bytes)) + 2 * size_t((sbytes + 15) & ~15) + 16;
+size_t unit_stage_bytes(int fmt, int K, int rows, int mats) {
+  const int cbytes = rows * (K / 2);
+  const int sbytes = rows * scale_row_bytes(fmt, K);
+  return size_t(mats) * (cbytes + ((sbytes + 15) & ~15));
 }
 
-size_t down_smem(int fmt, int K) {
-  const int cbytes = kDownFeatures * (K / 2);
-  const int sbytes = kDownFeatures * scale_row_bytes(fmt, K);
-  return size_t(cbytes) + size_t((sbytes + 15) & ~15) + 16;
+// two unit stages + the cross-warp reduction buffer + two barriers
+size_t gate_up_smem(int fmt, int K, int nt) {
+  return 2 * unit_stage_bytes(fmt, K, kDecRows, 2) + size_t(kDecWarps) * nt * 2 * 4 * 32 * 4 + 16;
+}
+
+size_t down_smem(int fmt, int K) { return 2 * unit_stage_bytes(fmt, K, kDownFeatures, 1) + 16; }
+
+int sm_count_cached() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Persistent grid: as many CTAs as fit on the GPU at once (at most `units`).
+// (computed once per kernel instantiation and shared-memory size)
+template <typename Kern>
+int persistent_grid(Kern k, size_t smem, int units) {
+  static size_t cached_smem = 0;
+  static int per_sm = 0;
+  if (per_sm == 0 || cached_smem != smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kDecWarps * 32, smem) != cudaSuccess || n < 1) n = 1;
+    per_sm = n;
+    cached_smem = smem;
+  }
+  return std::max(1, std::min(units, per_sm * sm_count_cached()));
 }
 
 template <typename Kern>
@@ -382,69 +468,67 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 
 }  // namespace
 
-size_t decode_gate_up_smem_bytes(int fmt, int K) { return gate_up_smem(fmt, K); }
-
 namespace {
 
 template <int FMT, int NT>
-cudaError_t gate_up_nt(const moe_shape_t& s, const uint16_t* x, const Bank& gu, const Workspace& ws, int grid,
-                       size_t smem, cudaStream_t stream) {
+cudaError_t gate_up_nt(const moe_shape_t& s, const uint16_t* x, const Bank& gu, const Workspace& ws, int units,
+                       cudaStream_t stream) {
   auto k = decode_gate_up_kernel<FMT, NT>;
+  const size_t smem = gate_up_smem(FMT, s.hidden, NT);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
+  const int grid = persistent_grid(k, smem, units);
   return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, x, gu, s.inter, s.top_k,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows, ws.act,
                     ws.status);
 }
 
 template <int FMT>
-cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws, int grid,
-                        size_t smem, cudaStream_t stream) {
+cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws,
+                        int units, cudaStream_t stream) {
   // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
-  if (T <= 8) return gate_up_nt<FMT, 1>(s, x, gu, ws, grid, smem, stream);
-  if (T <= 16) return gate_up_nt<FMT, 2>(s, x, gu, ws, grid, smem, stream);
-  return gate_up_nt<FMT, kDecNT>(s, x, gu, ws, grid, smem, stream);
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, x, gu, ws, units, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, x, gu, ws, units, stream);
+  return gate_up_nt<FMT, kDecNT>(s, x, gu, ws, units, stream);
 }
 
 template <int FMT, int NT>
-cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int grid,
-                    size_t smem, cudaStream_t stream) {
+cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int units,
+                    cudaStream_t stream) {
   auto k = decode_down_kernel<FMT, NT>;
+  const size_t smem = down_smem(FMT, s.inter);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
+  const int grid = persistent_grid(k, smem, units);
   return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, dn, T, s.top_k, (const int32_t*)ws.touched,
                     (const int32_t*)ws.offsets, (const uint16_t*)ws.act, (const float*)ws.topk_w,
                     (const int32_t*)ws.pos, ws.y, out, ws.status, ws.tile_counters);
 }
 
 template <int FMT>
-cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int grid,
-                     size_t smem, cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, grid, smem, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, grid, smem, stream);
-  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, grid, smem, stream);
+cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int units,
+                     cudaStream_t stream) {
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, units, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, units, stream);
+  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, units, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const Workspace& ws, cudaStream_t stream) {
-  const int slots = max_touched(T, s.top_k, s.num_experts);
-  const int grid = slots * (s.inter / kDecRows);
-  if (grid == 0) return cudaSuccess;
-  const size_t smem = gate_up_smem(s.fmt, s.hidden);
-  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, grid, smem, stream);
-  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, grid, smem, stream);
+  const int units = max_touched(T, s.top_k, s.num_experts) * (s.inter / kDecRows);
+  if (units == 0) return cudaSuccess;
+  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, units, stream);
+  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, units, stream);
 }
 
 cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
                                        uint16_t* out, cudaStream_t stream) {
-  const int slots = max_touched(T, s.top_k, s.num_experts);
-  const int grid = slots * (s.hidden / kDownFeatures);
-  if (grid == 0) return cudaSuccess;
-  const size_t smem = down_smem(s.fmt, s.inter);
-  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, grid, smem, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, grid, smem, stream);
+  const int units = max_touched(T, s.top_k, s.num_experts) * (s.hidden / kDownFeatures);
+  if (units == 0) return cudaSuccess;
+  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, units, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, units, stream);
 }
 
 }  // namespace moe

@@ -79,34 +79,39 @@ MOE_DEV void router_gemv_block(const uint16_t* __restrict__ x, const uint16_t* _
 // Each round takes the largest remaining value, ties to the lower index.
 // ---------------------------------------------------------------------------
 // Top-k of one token's logits by one warp (lane l holds experts l, l+32, ...,
-// E <= 1024); each round takes the largest remaining value, ties to the lower
-// index.  Logits are read through L2 (they may come from other CTAs).
-MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
-                       int32_t* __restrict__ ids, float* __restrict__ wout) {
+// PER = ceil(E/32) of them); each round takes the largest remaining value,
+// ties to the lower index.  Logits are read through L2 (they may come from
+// other CTAs).
+template <int PER>
+MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
+                         int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
-  float v[32];
-  const int per = (E + 31) / 32;
+  float v[PER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < PER; ++i) {
     const int e = i * 32 + lane;
-    float val = -FLT_MAX;
-    if (i < per && e < E) {
+    float val = -INFINITY;
+    if (e < E) {
       val = __ldcg(row + e);
       if (bias) val = val + bias[e];  // fp32 add
     }
     v[i] = val;
   }
-  uint32_t taken = 0;
+  uint32_t avail = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i)
+    if (i * 32 + lane < E) avail |= 1u << i;
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
+    // local best among available entries; i ascending keeps the lower index on ties
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = i * 32 + lane;
-      if (i < per && e < E && !((taken >> i) & 1u)) {
-        if (v[i] > bv || (v[i] == bv && e < bi)) { bv = v[i]; bi = e; }
+    for (int i = 0; i < PER; ++i) {
+      if (((avail >> i) & 1u) && (v[i] > bv || bi == 0x7fffffff)) {
+        bv = v[i];
+        bi = i * 32 + lane;
       }
     }
 #pragma unroll
@@ -115,7 +120,7 @@ MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ 
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if ((bi & 31) == lane) avail &= ~(1u << (bi >> 5));
     if (lane == j) { my_val = bv; my_id = bi; }
   }
   const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
@@ -127,6 +132,17 @@ MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ 
     ids[lane] = my_id;
     wout[lane] = ex / sum;
   }
+}
+
+MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
+                       int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int per = (E + 31) / 32;
+  if (per <= 1) warp_topk_t<1>(row, bias, E, k, ids, wout);
+  else if (per <= 2) warp_topk_t<2>(row, bias, E, k, ids, wout);
+  else if (per <= 4) warp_topk_t<4>(row, bias, E, k, ids, wout);
+  else if (per <= 8) warp_topk_t<8>(row, bias, E, k, ids, wout);
+  else if (per <= 16) warp_topk_t<16>(row, bias, E, k, ids, wout);
+  else warp_topk_t<32>(row, bias, E, k, ids, wout);
 }
 
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
