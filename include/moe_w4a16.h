@@ -250,6 +250,30 @@ MOE_API int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t
  * clears the flag), MOE_OK otherwise. */
 MOE_API moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* moe_forward for callers that cannot allocate device memory.  The model
+ * cards have no counterpart to this entry point; it exists for callers that
+ * record their GPU work ahead of time and replay it (a captured CUDA graph, a
+ * pre-built command buffer), where a cudaMalloc inside the recorded region is
+ * not possible, and for runtimes or plugins that reserve all device memory
+ * up front or do not own the allocator.  The caller passes only inputs and
+ * outputs (same meaning, layout and alignment as moe_forward); the scratch
+ * is a fixed array inside the library (moe_noalloc_scratch_bytes(), 8 MiB),
+ * held by every GPU that loads the library until the process exits.
+ *   - Returns MOE_ERR_UNSUPPORTED when moe_workspace_bytes(shape, T) exceeds
+ *     that size (e.g. large prefill batches); nothing is enqueued then.
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture.
+ *   - Calls on one device share the array: each clears its status/counter
+ *     region, and calls that overlap on the GPU (unordered streams) race.
+ *   - No device allocation and no freeing happen inside this call. */
+MOE_API moe_status_t moe_forward_noalloc(const moe_shape_t* shape, const uint16_t* x, int T,
+                                         const uint16_t* router_w, const float* logit_bias,
+                                         const void* gate_up_packed, const void* down_packed,
+                                         uint16_t* out, cudaStream_t stream);
+
+/* Size in bytes of moe_forward_noalloc's fixed scratch array. */
+MOE_API size_t moe_noalloc_scratch_bytes(void);
+
 /* Self-test of the bounded device-side wait: launches one warp that waits on
  * a barrier nothing ever arrives at, gives up after `limit_ns` nanoseconds of
  * device time (at most 10 s) and raises the workspace status word, so that a

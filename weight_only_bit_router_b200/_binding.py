@@ -76,6 +76,10 @@ _SIGS = {
                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
     "moe_forward_launch_count": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int,
                                                 ctypes.c_int]),
+    "moe_forward_noalloc": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "moe_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_workspace_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64,
@@ -286,6 +290,22 @@ def moe_forward_routed(shape: MoeShape, x, topk_ids, topk_w, gate_up_packed, dow
 
 def moe_forward_launch_count(shape: MoeShape, T: int, path=MOE_PATH_AUTO, routed=False) -> int:
     return lib().moe_forward_launch_count(ctypes.byref(shape), T, path, int(routed))
+
+
+def moe_noalloc_scratch_bytes() -> int:
+    return lib().moe_noalloc_scratch_bytes()
+
+
+def moe_forward_noalloc(shape: MoeShape, x, router_w, gate_up_packed, down_packed, out=None, bias=None,
+                        stream=None):
+    """moe_forward on the library's fixed scratch array (no workspace argument)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
+    st = lib().moe_forward_noalloc(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(_bits(router_w)), _ptr(bias),
+                                   _ptr(gate_up_packed), _ptr(down_packed), _ptr(out), _stream(stream))
+    _check("moe_forward_noalloc", st)
+    return out
 
 
 def moe_workspace_init(workspace, stream=None):
