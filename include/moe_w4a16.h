@@ -180,7 +180,8 @@ MOE_API moe_status_t moe_permute(const int32_t* topk_ids, int T, int E, int k, i
 
 typedef enum {
   MOE_PATH_AUTO = 0,      /* decode path for T <= 32, grouped tcgen05 GEMMs above */
-  MOE_PATH_DECODE = 1,    /* weight-streaming GEMV kernels (any T; meant for T <= 32) */
+  MOE_PATH_DECODE = 1,    /* weight-streaming GEMV kernels (any T; meant for T <= 32: above that
+                             the down projection re-streams its weights per 32 tokens) */
   MOE_PATH_PREFILL = 2    /* grouped tcgen05 GEMMs (any T >= 1) */
 } moe_path_t;
 

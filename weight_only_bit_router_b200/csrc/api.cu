@@ -9,8 +9,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kDecodeMaxForced = 256;  // the decode path keeps [T*k, H] fp32 expert outputs
-
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool valid_fmt(moe_format_t f) { return f == MOE_FMT_INT4_G128 || f == MOE_FMT_MXFP4_G32; }
@@ -92,7 +90,6 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   };
   w.status = static_cast<uint32_t*>(take(kStatusBytes));
   w.route_counter = p ? reinterpret_cast<int32_t*>(w.status) + 1 : nullptr;
-  w.tile_counters = p ? reinterpret_cast<int32_t*>(w.status) + 8 : nullptr;
   w.logits = static_cast<float*>(take(size_t(T) * E * 4));
   w.topk_ids = static_cast<int32_t*>(take(R * 4));
   w.topk_w = static_cast<float*>(take(R * 4));
@@ -103,7 +100,6 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.tile_base = static_cast<int32_t*>(take((E + 1) * 4));
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
-  w.y = static_cast<float*>(take(T <= kDecodeMaxForced ? R * H * 4 : 0));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
   w.bytes = off;
   return w;
@@ -190,7 +186,6 @@ moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, i
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
   *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
-  if (*decode && T > kDecodeMaxForced) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 

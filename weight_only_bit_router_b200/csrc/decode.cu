@@ -30,7 +30,6 @@ namespace {
 constexpr int kDecWarps = 4;       // warps per CTA
 constexpr int kDecRows = 16;       // weight rows (features) per warp tile
 constexpr int kDecNT = 4;          // token tiles of 8 held in registers at once
-constexpr int kDownFeatures = kDecRows * kDecWarps;  // features per down CTA
 
 MOE_DEV void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -171,22 +170,28 @@ MOE_DEV UnitLayout unit_layout(int fmt, int K, int rows, int mats) {
 }
 
 // ---------------------------------------------------------------------------
-// gate_up + SwiGLU, persistent.  Work unit u = (touched slot u / (I/16),
-// features 16*(u % (I/16)) ...): the 16 gate rows and the 16 matching up rows
-// of that expert.  A CTA walks units u = blockIdx.x + i * gridDim.x with two
-// shared-memory stages: the bulk copies of unit i+2 start as soon as unit i's
-// stage is free, so weight streaming overlaps the MMAs.  The CTA's 4 warps
-// split K; partial tiles are summed in shared memory; a = bf16(silu(gate) *
-// up) goes to act[p][f] for the expert's sorted rows p.
+// gate_up + SwiGLU, persistent.  Work unit u = (touched slot u / (I/8),
+// features f0 = 8*(u % (I/8)) .. f0+7).  Its 16 weight rows are the 8 gate
+// rows f0.. and the 8 matching up rows I+f0.., staged as one 16-row tile
+// (gate rows 0-7, up rows 8-15), so the MMA's C fragment holds gate (c0, c1)
+// and up (c2, c3) of the same feature and token: SwiGLU needs no shuffle.
+// A CTA walks units u = blockIdx.x + i * gridDim.x with two shared-memory
+// stages: the bulk copies of unit i+2 start as soon as unit i's stage is
+// free.  The CTA's 4 warps split K; partial tiles are summed in shared memory;
+// a = bf16(silu(gate) * up) goes to act[p][f] for the expert's sorted rows p.
 // ---------------------------------------------------------------------------
+constexpr int kGuFeatures = kDecRows / 2;  // features per gate_up unit
+
 template <int FMT>
 MOE_DEV void issue_gate_up_unit(const Bank& gu, int I, const int32_t* touched, int ftiles, int u, uint8_t* stage,
                                 const UnitLayout& L, uint64_t* bar) {
   const int e = touched[1 + u / ftiles];
-  const long row_g = long(e) * gu.N + (u % ftiles) * kDecRows;
-  mbar_arrive_expect_tx(bar, 2 * staged_bytes<FMT>(gu, kDecRows));
-  stage_rows<FMT>(gu, row_g, kDecRows, stage, stage + 2 * L.cbytes, bar);
-  stage_rows<FMT>(gu, row_g + I, kDecRows, stage + L.cbytes, stage + 2 * L.cbytes + L.sbytes_pad, bar);
+  const long row_g = long(e) * gu.N + (u % ftiles) * kGuFeatures;
+  const int sb = scale_row_bytes(FMT, gu.K);
+  const uint32_t half_codes = uint32_t(kGuFeatures) * (gu.K / 2);
+  mbar_arrive_expect_tx(bar, staged_bytes<FMT>(gu, kDecRows));
+  stage_rows<FMT>(gu, row_g, kGuFeatures, stage, stage + L.cbytes, bar);
+  stage_rows<FMT>(gu, row_g + I, kGuFeatures, stage + half_codes, stage + L.cbytes + kGuFeatures * sb, bar);
 }
 
 template <int FMT, int NT>
@@ -196,14 +201,14 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
     uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = gu.K;
-  // stage layout: [gate codes][up codes][gate scales][up scales]
-  const UnitLayout L = unit_layout(FMT, K, kDecRows, 2);
-  float* red = reinterpret_cast<float*>(smem + 2 * L.stage_bytes);  // [warp][tile][gate/up][4][lane]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kDecWarps * NT * 2 * 4 * 32);
+  // stage layout: [16 rows of codes: gate 0-7, up 8-15][16 rows of scales]
+  const UnitLayout L = unit_layout(FMT, K, kDecRows, 1);
+  float* red = reinterpret_cast<float*>(smem + 2 * L.stage_bytes);  // [warp][tile][4][lane]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kDecWarps * NT * 4 * 32);
 
   pdl_wait();
   pdl_trigger();
-  const int ftiles = I / kDecRows;
+  const int ftiles = I / kGuFeatures;
   const int n_units = touched[0] * ftiles;
   if (int(blockIdx.x) >= n_units) return;
   if (threadIdx.x == 0) {
@@ -222,24 +227,20 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
   int i = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
     const int st = i & 1;
-    const uint8_t* s_cg = smem + st * L.stage_bytes;
-    const uint8_t* s_cu = s_cg + L.cbytes;
-    const uint8_t* s_sg = s_cg + 2 * L.cbytes;
-    const uint8_t* s_su = s_sg + L.sbytes_pad;
+    const uint8_t* s_c = smem + st * L.stage_bytes;
+    const uint8_t* s_s = s_c + L.cbytes;
     const int e = touched[1 + u / ftiles];
-    const int f0 = (u % ftiles) * kDecRows;
+    const int f0 = (u % ftiles) * kGuFeatures;
     const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
     const int ntiles = (n_e + 7) / 8;
     volatile int never = 0;
     const bool ok = mbar_wait(&bars[st], (i >> 1) & 1, &never, status);
     for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
-      float acc[NT][2][4];
+      float acc[NT][4];
 #pragma unroll
       for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[j][t][c] = 0.f;
+        for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
       const uint16_t* xrow[NT];
       bool xval[NT];
 #pragma unroll
@@ -251,42 +252,38 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
       if (ok) {
         for (int b = warp; b < nblk; b += kDecWarps) {
           const int kb = b * 128;
-          const RowChunk g0 = smem_row_chunk<FMT>(s_cg, s_sg, g, K, kb, q);
-          const RowChunk g1 = smem_row_chunk<FMT>(s_cg, s_sg, g + 8, K, kb, q);
-          const RowChunk u0 = smem_row_chunk<FMT>(s_cu, s_su, g, K, kb, q);
-          const RowChunk u1 = smem_row_chunk<FMT>(s_cu, s_su, g + 8, K, kb, q);
+          const RowChunk gate = smem_row_chunk<FMT>(s_c, s_s, g, K, kb, q);
+          const RowChunk up = smem_row_chunk<FMT>(s_c, s_s, g + 8, K, kb, q);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
             uint32_t bf[8][2];
             load_act_frags(xrow[j], K, kb, q, xval[j], bf);
-            mma_block<FMT>(acc[j][0], g0, g1, bf);
-            mma_block<FMT>(acc[j][1], u0, u1, bf);
+            mma_block<FMT>(acc[j], gate, up, bf);
           }
         }
       }
 #pragma unroll
       for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) red[(((warp * NT + j) * 2 + t) * 4 + c) * 32 + lane] = acc[j][t][c];
+        for (int c = 0; c < 4; ++c) red[((warp * NT + j) * 4 + c) * 32 + lane] = acc[j][c];
       __syncthreads();
       // warp w < NT finishes token tile nt0 + w
       const int j = warp;
       if (ok && j < NT && nt0 + j < ntiles) {
+        float sum[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float gs = 0.f, us = 0.f;
+          sum[c] = 0.f;
 #pragma unroll
-          for (int w = 0; w < kDecWarps; ++w) {
-            gs += red[(((w * NT + j) * 2 + 0) * 4 + c) * 32 + lane];
-            us += red[(((w * NT + j) * 2 + 1) * 4 + c) * 32 + lane];
-          }
-          // c0,c1: feature g, tokens 2q, 2q+1; c2,c3: feature g+8
-          const int col = (nt0 + j) * 8 + 2 * q + (c & 1);
-          const int f = f0 + g + ((c >> 1) << 3);
-          if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(gs, us));
+          for (int w = 0; w < kDecWarps; ++w) sum[c] += red[((w * NT + j) * 4 + c) * 32 + lane];
+        }
+        // c0, c1: gate of feature f0+g at tokens 2q, 2q+1; c2, c3: up of the same
+        const int f = f0 + g;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col = (nt0 + j) * 8 + 2 * q + h;
+          if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(sum[h], sum[2 + h]));
         }
       }
       __syncthreads();
@@ -301,121 +298,140 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// down projection + deterministic combine, persistent.  Work unit u = (touched
-// slot u / (H/64), features 64*(u % (H/64)) ...): 64 rows of the expert's
-// down bank, two shared-memory stages as above.  Each warp owns 16 features
-// over K = I and writes y[p][f] in fp32.  The CTA that completes the last
-// unit of a feature tile (counted in the workspace) sums the k expert outputs
-// of every token in slot order j = 0..k-1 and writes that tile's bf16 output.
+// down projection + deterministic combine.  One CTA per 16-feature tile of
+// the output; its 16 warps own the touched experts (warp w takes slots w,
+// w+16, ...), each streaming its experts' 16 down rows (all of K = I) through
+// its own two-stage ring of bulk copies.  A warp multiplies the expert's rows
+// with the activations of the expert's tokens and adds w_tj * y into its own
+// shared-memory accumulator [token][feature]; the 16 accumulators are then
+// summed in warp order and written as bf16.  The summation order is fixed, so
+// the output is deterministic.  Tokens are processed in chunks of 32 (one
+// chunk for T <= 32).
 // ---------------------------------------------------------------------------
+constexpr int kDnWarps = 16;
+constexpr int kDnStages = 2;
+constexpr int kDnTokens = 32;  // token chunk per pass
+
 template <int FMT>
-MOE_DEV void issue_down_unit(const Bank& dn, const int32_t* touched, int ftiles, int u, uint8_t* stage,
-                             const UnitLayout& L, uint64_t* bar) {
-  const int e = touched[1 + u / ftiles];
-  const long row0 = long(e) * dn.N + (u % ftiles) * kDownFeatures;
-  mbar_arrive_expect_tx(bar, staged_bytes<FMT>(dn, kDownFeatures));
-  stage_rows<FMT>(dn, row0, kDownFeatures, stage, stage + L.cbytes, bar);
+MOE_DEV void issue_down_rows(const Bank& dn, int e, int f0, uint8_t* stage, const UnitLayout& L, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, staged_bytes<FMT>(dn, kDecRows));
+  stage_rows<FMT>(dn, long(e) * dn.N + f0, kDecRows, stage, stage + L.cbytes, bar);
 }
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kDecWarps * 32) decode_down_kernel(
+__global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
     Bank dn, int T, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
-    const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ pos,
-    float* __restrict__ y, uint16_t* __restrict__ out, uint32_t* status, int32_t* tile_counters) {
+    const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ sorted_rows,
+    uint16_t* __restrict__ out, uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = dn.N, K = dn.K;  // K = I
-  const UnitLayout L = unit_layout(FMT, K, kDownFeatures, 1);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * L.stage_bytes);
-  __shared__ int s_last;
+  const UnitLayout L = unit_layout(FMT, K, kDecRows, 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  uint8_t* ring = smem + warp * kDnStages * L.stage_bytes;
+  float* accs = reinterpret_cast<float*>(smem + kDnWarps * kDnStages * L.stage_bytes);  // [warp][token][16]
+  float* acc_w = accs + warp * kDnTokens * kDecRows;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(accs + kDnWarps * kDnTokens * kDecRows) + warp * kDnStages;
 
   pdl_wait();
   pdl_trigger();
-  const int ftiles = H / kDownFeatures;
+  const int f0 = blockIdx.x * kDecRows;
   const int n_touched = touched[0];
-  const int n_units = n_touched * ftiles;
-  if (int(blockIdx.x) >= n_units) return;
-  if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_mbar_init();
-    for (int st = 0; st < 2; ++st) {
-      const int u = blockIdx.x + st * gridDim.x;
-      if (u < n_units) issue_down_unit<FMT>(dn, touched, ftiles, u, smem + st * L.stage_bytes, L, &bars[st]);
-    }
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, q = lane & 3;
   const int nblk = (K + 127) / 128;
-  const int r0 = warp * kDecRows + g;  // staged row of this lane
-  int i = 0;
-  for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
-    const int st = i & 1;
-    const uint8_t* s_c = smem + st * L.stage_bytes;
-    const uint8_t* s_s = s_c + L.cbytes;
-    const int e = touched[1 + u / ftiles];
-    const int ft = u % ftiles;
-    const int f0 = ft * kDownFeatures + warp * kDecRows;
-    const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
-    const int ntiles = (n_e + 7) / 8;
-    volatile int never = 0;
-    const bool ok = mbar_wait(&bars[st], (i >> 1) & 1, &never, status);
-    for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
-      float acc[NT][4];
+  if (lane == 0) {
+    for (int st = 0; st < kDnStages; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  int uses = 0;  // ring slots consumed so far by this warp (over all chunks)
+  for (int t0 = 0; t0 < T; t0 += kDnTokens) {
+    const int t1 = min(T, t0 + kDnTokens);
+    for (int i = lane; i < kDnTokens * kDecRows; i += 32) acc_w[i] = 0.f;
+    // prologue: first experts of this warp into the ring
+    if (lane == 0) {
+      for (int st = 0; st < kDnStages; ++st) {
+        const int slot = warp + st * kDnWarps;
+        if (slot < n_touched) {
+          fence_proxy_async_smem();
+          issue_down_rows<FMT>(dn, touched[1 + slot], f0, ring + ((uses + st) % kDnStages) * L.stage_bytes, L,
+                               &bars[(uses + st) % kDnStages]);
+        }
+      }
+    }
+    __syncwarp();
+    for (int slot = warp, n = 0; slot < n_touched; slot += kDnWarps, ++n) {
+      const int st = (uses + n) % kDnStages;
+      const uint32_t parity = ((uses + n) / kDnStages) & 1;
+      const uint8_t* s_c = ring + st * L.stage_bytes;
+      const uint8_t* s_s = s_c + L.cbytes;
+      const int e = touched[1 + slot];
+      // rows of expert e whose token lies in [t0, t1): a contiguous sub-range
+      // (sorted rows ascend with the token index)
+      int p0 = offsets[e], p1 = offsets[e + 1];
+      while (p0 < p1 && sorted_rows[p0] / top_k < t0) ++p0;
+      int pe = p0;
+      while (pe < p1 && sorted_rows[pe] / top_k < t1) ++pe;
+      const int n_e = pe - p0;
+      volatile int never = 0;
+      const bool ok = mbar_wait(&bars[st], parity, &never, status);
+      const int ntiles = (n_e + 7) / 8;
+      for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
+        float acc[NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j)
+        for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
-      for (int b = 0; b < nblk; ++b) {
-        const int kb = b * 128;
-        const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, r0, K, kb, q);
-        const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, r0 + 8, K, kb, q);
+          for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
+        for (int b = 0; b < nblk; ++b) {
+          const int kb = b * 128;
+          const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, g, K, kb, q);
+          const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, g + 8, K, kb, q);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            if (nt0 + j >= ntiles) break;
+            const int col = (nt0 + j) * 8 + g;
+            uint32_t bf[8][2];
+            load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
+            mma_block<FMT>(acc[j], c0, c1, bf);
+          }
+        }
+        // c0,c1: feature g, rows 2q, 2q+1 of the tile; c2,c3: feature g+8
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          if (nt0 + j >= ntiles) break;
-          const int col = (nt0 + j) * 8 + g;
-          uint32_t bf[8][2];
-          load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
-          mma_block<FMT>(acc[j], c0, c1, bf);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col = (nt0 + j) * 8 + 2 * q + h;
+            if (nt0 + j < ntiles && col < n_e) {
+              const int r = sorted_rows[p0 + col];
+              const int t = r / top_k - t0;
+              const float w = topk_w[r];
+              acc_w[t * kDecRows + g] += w * acc[j][h];
+              acc_w[t * kDecRows + g + 8] += w * acc[j][2 + h];
+            }
+          }
         }
       }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = (nt0 + j) * 8 + 2 * q + (c & 1);
-          const int f = f0 + g + ((c >> 1) << 3);
-          if (nt0 + j < ntiles && col < n_e) y[size_t(p0 + col) * H + f] = acc[j][c];
+      __syncwarp();  // ring slot st consumed by every lane
+      if (lane == 0) {
+        const int next = slot + kDnStages * kDnWarps;
+        if (next < n_touched) {
+          fence_proxy_async_smem();
+          issue_down_rows<FMT>(dn, touched[1 + next], f0, ring + st * L.stage_bytes, L, &bars[st]);
         }
       }
+      __syncwarp();
     }
-    __syncthreads();  // stage st consumed, y tile written
-    if (threadIdx.x == 0) {
-      fence_proxy_async_smem();
-      const int u2 = u + 2 * gridDim.x;
-      if (u2 < n_units) issue_down_unit<FMT>(dn, touched, ftiles, u2, smem + st * L.stage_bytes, L, &bars[st]);
-      __threadfence();
-      s_last = atomicAdd(&tile_counters[ft], 1) == n_touched - 1;
+    // every warp's ring slots used in this chunk
+    uses += (n_touched > warp) ? (n_touched - warp + kDnWarps - 1) / kDnWarps : 0;
+    __syncthreads();
+    // sum the warps' accumulators in a fixed order
+    for (int idx = threadIdx.x; idx < (t1 - t0) * kDecRows; idx += blockDim.x) {
+      float sum = 0.f;
+#pragma unroll 4
+      for (int w = 0; w < kDnWarps; ++w) sum += accs[w * kDnTokens * kDecRows + idx];
+      const int t = t0 + idx / kDecRows, f = f0 + idx % kDecRows;
+      out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
     }
     __syncthreads();
-    if (s_last) {
-      // every expert's y for this feature tile is written: combine it
-      __threadfence();
-      const int fbase = ft * kDownFeatures;
-      for (int idx = threadIdx.x; idx < T * kDownFeatures; idx += blockDim.x) {
-        const int t = idx / kDownFeatures;
-        const int f = fbase + idx % kDownFeatures;
-        float sum = 0.f;
-        for (int j = 0; j < top_k; ++j) {
-          const int p = pos[size_t(t) * top_k + j];
-          if (p < 0) continue;
-          sum = fmaf(topk_w[size_t(t) * top_k + j], __ldcg(y + size_t(p) * H + f), sum);
-        }
-        out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
-      }
-      if (threadIdx.x == 0) tile_counters[ft] = 0;  // ready for the next call
-      __syncthreads();
-    }
   }
 }
 
@@ -429,10 +445,14 @@ size_t unit_stage_bytes(int fmt, int K, int rows, int mats) {
 
 // two unit stages + the cross-warp reduction buffer + two barriers
 size_t gate_up_smem(int fmt, int K, int nt) {
-  return 2 * unit_stage_bytes(fmt, K, kDecRows, 2) + size_t(kDecWarps) * nt * 2 * 4 * 32 * 4 + 16;
+  return 2 * unit_stage_bytes(fmt, K, kDecRows, 1) + size_t(kDecWarps) * nt * 4 * 32 * 4 + 16;
 }
 
-size_t down_smem(int fmt, int K) { return 2 * unit_stage_bytes(fmt, K, kDownFeatures, 1) + 16; }
+// per-warp rings + per-warp accumulators + per-warp barriers
+size_t down_smem(int fmt, int K) {
+  return size_t(kDnWarps) * kDnStages * unit_stage_bytes(fmt, K, kDecRows, 1) +
+         size_t(kDnWarps) * kDnTokens * kDecRows * 4 + size_t(kDnWarps) * kDnStages * 8;
+}
 
 int sm_count_cached() {
   static int n = 0;
@@ -493,31 +513,30 @@ cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Ba
 }
 
 template <int FMT, int NT>
-cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int units,
+cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
                     cudaStream_t stream) {
   auto k = decode_down_kernel<FMT, NT>;
   const size_t smem = down_smem(FMT, s.inter);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(k, smem, units);
-  return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, dn, T, s.top_k, (const int32_t*)ws.touched,
-                    (const int32_t*)ws.offsets, (const uint16_t*)ws.act, (const float*)ws.topk_w,
-                    (const int32_t*)ws.pos, ws.y, out, ws.status, ws.tile_counters);
+  return launch_pdl(k, dim3(s.hidden / kDecRows), dim3(kDnWarps * 32), smem, stream, dn, T, s.top_k,
+                    (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const uint16_t*)ws.act,
+                    (const float*)ws.topk_w, (const int32_t*)ws.sorted_rows, out, ws.status);
 }
 
 template <int FMT>
-cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out, int units,
+cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
                      cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, units, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, units, stream);
-  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, units, stream);
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, stream);
+  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const Workspace& ws, cudaStream_t stream) {
-  const int units = max_touched(T, s.top_k, s.num_experts) * (s.inter / kDecRows);
+  const int units = max_touched(T, s.top_k, s.num_experts) * (s.inter / kGuFeatures);
   if (units == 0) return cudaSuccess;
   if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, units, stream);
   return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, units, stream);
@@ -525,10 +544,9 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
 
 cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
                                        uint16_t* out, cudaStream_t stream) {
-  const int units = max_touched(T, s.top_k, s.num_experts) * (s.hidden / kDownFeatures);
-  if (units == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, units, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, units, stream);
+  if (T == 0) return cudaSuccess;
+  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, stream);
 }
 
 }  // namespace moe

@@ -35,15 +35,14 @@ struct Bank {
 };
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
-// The first kStatusBytes of a workspace: the status word, the fused-routing
-// completion counter and per-feature-tile combine counters.  Zeroed once by
-// moe_workspace_init; every kernel that counts resets its counter to zero.
+// The first kStatusBytes of a workspace: the status word and the fused-routing
+// completion counter.  Zeroed once by moe_workspace_init; the counting kernel
+// resets its counter to zero.
 constexpr size_t kStatusBytes = 4096;
 
 struct Workspace {
   uint32_t* status;       // status word (device-side failures)
   int32_t* route_counter; // CTAs done in the fused small-batch routing kernel
-  int32_t* tile_counters; // decode down kernel: CTAs done per 64-feature tile
   float* logits;          // [T, E]
   int32_t* topk_ids;      // [T, k]
   float* topk_w;          // [T, k]
@@ -54,7 +53,6 @@ struct Workspace {
   int32_t* tile_base;     // [E+1]: prefix of per-expert token blocks (grouped GEMMs)
   int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
-  float* y;               // [T*k, H] fp32 expert outputs (decode path)
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
   size_t bytes;
 };

@@ -20,68 +20,17 @@ namespace {
 // A CTA owns 2 experts; 4 warps split H for each expert; lanes read 16-byte
 // chunks of the router row and of every token row.
 // ---------------------------------------------------------------------------
-constexpr int kRgExpertsPerCta = 2;
-constexpr int kRgWarpsPerExpert = 4;
-constexpr int kRgThreads = 32 * kRgExpertsPerCta * kRgWarpsPerExpert;
-
-MOE_DEV void router_gemv_block(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, int T, int H, int E,
-                               float* __restrict__ logits, float (*part)[kRgWarpsPerExpert][kDecodeMaxT]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int le = warp / kRgWarpsPerExpert, ks = warp % kRgWarpsPerExpert;
-  const int e = blockIdx.x * kRgExpertsPerCta + le;
-  float acc[kDecodeMaxT];
-#pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.f;
-  if (e < E) {
-    const int span = H / kRgWarpsPerExpert;  // multiple of 16
-    const int c0 = ks * span;
-    for (int c = c0 + lane * 8; c < c0 + span; c += 256) {
-      const uint4 wv = ldg_nc_v4(wr + size_t(e) * H + c);
-      const float w8[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
-                           bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
-#pragma unroll
-      for (int t = 0; t < kDecodeMaxT; ++t) {
-        if (t < T) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * H + c));
-          float s = acc[t];
-          s = fmaf(w8[0], bf16_lo(xv.x), s); s = fmaf(w8[1], bf16_hi(xv.x), s);
-          s = fmaf(w8[2], bf16_lo(xv.y), s); s = fmaf(w8[3], bf16_hi(xv.y), s);
-          s = fmaf(w8[4], bf16_lo(xv.z), s); s = fmaf(w8[5], bf16_hi(xv.z), s);
-          s = fmaf(w8[6], bf16_lo(xv.w), s); s = fmaf(w8[7], bf16_hi(xv.w), s);
-          acc[t] = s;
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) {
-    if (t < T) {
-      float s = acc[t];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) part[le][ks][t] = s;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kRgExpertsPerCta * T; i += blockDim.x) {
-    const int l = i / T, t = i % T;
-    const int ee = blockIdx.x * kRgExpertsPerCta + l;
-    if (ee < E) {
-      float s = 0.f;
-      for (int w = 0; w < kRgWarpsPerExpert; ++w) s += part[l][w][t];
-      logits[size_t(t) * E + ee] = s;
-    }
-  }
+// Order-preserving map of a non-NaN fp32 value to uint32 (-0 and +0 equal).
+MOE_DEV uint32_t orderable(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 + 0 = +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// ---------------------------------------------------------------------------
-// top-k: one warp per token.  Lane l holds experts l, l+32, ... (E <= 1024).
-// Each round takes the largest remaining value, ties to the lower index.
-// ---------------------------------------------------------------------------
 // Top-k of one token's logits by one warp (lane l holds experts l, l+32, ...,
-// PER = ceil(E/32) of them); each round takes the largest remaining value,
-// ties to the lower index.  Logits are read through L2 (they may come from
-// other CTAs).
+// PER = ceil(E/32) of them).  Each round takes the largest remaining value
+// with two warp reductions (max of the value key, then min of the expert
+// index among the lanes holding that value: ties go to the lower index).
+// Logits are read through L2 (they may come from other CTAs).
 template <int PER>
 MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
                          int32_t* __restrict__ ids, float* __restrict__ wout) {
@@ -90,7 +39,7 @@ MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict_
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = i * 32 + lane;
-    float val = -INFINITY;
+    float val = 0.f;
     if (e < E) {
       val = __ldcg(row + e);
       if (bias) val = val + bias[e];  // fp32 add
@@ -104,24 +53,27 @@ MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict_
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    // local best among available entries; i ascending keeps the lower index on ties
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    // this lane's best remaining entry (i ascending keeps its lower index on ties)
+    uint32_t bkey = 0;
+    int bi = 0;
+    float bv = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      if (((avail >> i) & 1u) && (v[i] > bv || bi == 0x7fffffff)) {
+      const uint32_t key = orderable(v[i]);
+      if (((avail >> i) & 1u) && (key > bkey || bkey == 0)) {
+        bkey = key;
+        bi = i;
         bv = v[i];
-        bi = i * 32 + lane;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if ((bi & 31) == lane) avail &= ~(1u << (bi >> 5));
-    if (lane == j) { my_val = bv; my_id = bi; }
+    const uint32_t has = avail != 0;
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, has ? bkey : 0u);
+    const uint32_t cand = (has && bkey == kmax) ? uint32_t(bi * 32 + lane) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if (int(win & 31) == lane) avail &= ~(1u << (win >> 5));
+    // the winner's value reaches lane j through a shuffle
+    const float wv = __shfl_sync(0xffffffffu, bv, int(win & 31));
+    if (lane == j) { my_val = wv; my_id = int(win); }
   }
   const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
   const float ex = lane < k ? expf(my_val - vmax) : 0.f;
@@ -299,22 +251,182 @@ __global__ void __launch_bounds__(256) permute_small_kernel(const int32_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// Fused small-batch routing (T <= 32): every CTA computes the logits of two
-// experts for all tokens; the last CTA to finish (counted in the workspace)
-// runs top-k for every token (one warp per token), then the stable
-// permutation, the touched-expert list and the token-block prefix.
+// Stable counting sort of R rows by expert with ONE warp (ids in smem, values
+// outside [0, E) dropped), plus the touched-expert list and the token-block
+// prefix.  Rows are taken 32 at a time in ascending order; __match_any_sync
+// groups a chunk's rows by expert and the running per-expert counts in smem
+// give each row its rank, so equal experts keep ascending row order.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kRgThreads) route_small_kernel(
+MOE_DEV void warp_permutation(const int* s_ids, int* s_cnt, int* s_rank, int R, int E, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
+                              int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n) {
+  const int lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+  __syncwarp();
+  for (int r0 = 0; r0 < R; r0 += 32) {
+    const int r = r0 + lane;
+    int e = r < R ? s_ids[r] : -1;
+    if (e >= E) e = -1;
+    const unsigned m = __match_any_sync(full, e);
+    const int before = __popc(m & ((1u << lane) - 1u));
+    const int base = e >= 0 ? s_cnt[e] : 0;
+    __syncwarp();
+    if (e >= 0 && before == 0) s_cnt[e] = base + __popc(m);
+    if (r < R) s_rank[r] = e >= 0 ? base + before : -1;
+    __syncwarp();
+  }
+  // per-lane contiguous expert ranges [lane*per, lane*per + per)
+  const int per = (E + 31) / 32;
+  const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  int cnt_sum = 0, nz = 0, blk = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = s_cnt[e];
+    cnt_sum += c;
+    nz += c > 0;
+    blk += (c + block_n - 1) / block_n;
+  }
+  int c_incl = cnt_sum, nz_incl = nz, b_incl = blk;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(full, c_incl, o), b = __shfl_up_sync(full, nz_incl, o),
+              c = __shfl_up_sync(full, b_incl, o);
+    if (lane >= o) { c_incl += a; nz_incl += b; b_incl += c; }
+  }
+  int run = c_incl - cnt_sum, tpos = nz_incl - nz, brun = b_incl - blk;
+  for (int e = e0; e < e1; ++e) {
+    const int c = s_cnt[e];
+    offsets[e] = run;
+    tile_base[e] = brun;
+    s_cnt[e] = run;  // becomes the expert's first sorted position
+    if (c > 0) touched[1 + tpos++] = e;
+    run += c;
+    brun += (c + block_n - 1) / block_n;
+  }
+  if (lane == 31) {
+    offsets[E] = c_incl;
+    tile_base[E] = b_incl;
+    touched[0] = nz_incl;
+  }
+  __syncwarp();
+  for (int r = lane; r < R; r += 32) {
+    const int e = s_ids[r];
+    if (e < 0 || e >= E) {
+      pos[r] = -1;
+      continue;
+    }
+    const int p = s_cnt[e] + s_rank[r];
+    sorted_rows[p] = r;
+    pos[r] = p;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused small-batch routing (T <= 32).  Each CTA owns 16 experts; its 8 warps
+// split K and compute logits for all tokens with mma.sync (bf16 router
+// weights and tokens, fp32 accumulation), reduce them in shared memory and
+// store them.  The last CTA to finish (device counter) runs top-k for every
+// token (one warp per token) and one warp builds the permutation.
+// ---------------------------------------------------------------------------
+constexpr int kRsExperts = 16;
+constexpr int kRsWarps = 8;
+constexpr int kRsThreads = 32 * kRsWarps;
+
+MOE_DEV void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 row slice [k, k+32) of `rowp` permuted into the fragment order the
+// decode kernels use: for MMA step 2j+h the pairs (v[k0+2h], v[k0+2h+4]) and
+// (v[k0+2h+1], v[k0+2h+5]) with k0 = k + 8j.
+MOE_DEV void bf16_frags(const uint16_t* rowp, bool valid, uint32_t (&b)[8][2]) {
+  uint32_t X[16];
+  if (valid) {
+    const uint4* p = reinterpret_cast<const uint4*>(rowp);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = __ldg(p + i);
+      X[4 * i] = v.x; X[4 * i + 1] = v.y; X[4 * i + 2] = v.z; X[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) X[i] = 0;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    b[2 * j][0] = prmt(X[4 * j], X[4 * j + 2], 0x5410u);
+    b[2 * j][1] = prmt(X[4 * j], X[4 * j + 2], 0x7632u);
+    b[2 * j + 1][0] = prmt(X[4 * j + 1], X[4 * j + 3], 0x5410u);
+    b[2 * j + 1][1] = prmt(X[4 * j + 1], X[4 * j + 3], 0x7632u);
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kRsThreads) route_small_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
     int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
     int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n, int32_t* done_counter) {
-  __shared__ float part[kRgExpertsPerCta][kRgWarpsPerExpert][kDecodeMaxT];
-  __shared__ SmallPermSmem sm;
+  __shared__ float red[kRsWarps][NT][4][32];
+  __shared__ int s_ids[32 * kMaxTopK];
+  __shared__ int s_rank[32 * kMaxTopK];
+  __shared__ int s_cnt[kMaxExperts];
   __shared__ int s_last;
   pdl_wait();
   pdl_trigger();
-  router_gemv_block(x, wr, T, H, E, logits, part);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int e0 = blockIdx.x * kRsExperts;
+  const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
+  const uint16_t* wlo = wr + size_t(r_lo ? e0 + g : 0) * H;
+  const uint16_t* whi = wr + size_t(r_hi ? e0 + g + 8 : 0) * H;
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
+  const int nblk = H / 128;  // H is a multiple of 64: a last half block is handled below
+  for (int b = warp; b * 128 < H; b += kRsWarps) {
+    const int k = b * 128 + 32 * q;
+    const bool kin = k < H;
+    uint32_t alo[8][2], ahi[8][2];
+    bf16_frags(wlo + k, r_lo && kin, alo);
+    bf16_frags(whi + k, r_hi && kin, ahi);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int t = j * 8 + g;
+      uint32_t bf[8][2];
+      bf16_frags(x + size_t(t < T ? t : 0) * H + k, t < T && kin, bf);
+#pragma unroll
+      for (int st = 0; st < 8; ++st) {
+        const uint32_t a[4] = {alo[st][0], ahi[st][0], alo[st][1], ahi[st][1]};
+        mma_16816(acc[j], a, bf[st][0], bf[st][1]);
+      }
+    }
+  }
+  (void)nblk;
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[warp][j][c][lane] = acc[j][c];
+  __syncthreads();
+  if (warp < NT) {
+    const int j = warp;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRsWarps; ++w) sum += red[w][j][c][lane];
+      // c0,c1: expert e0+g, tokens 2q, 2q+1; c2,c3: expert e0+g+8
+      const int t = j * 8 + 2 * q + (c & 1);
+      const int e = e0 + g + ((c >> 1) << 3);
+      if (t < T && e < E) logits[size_t(t) * E + e] = sum;
+    }
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -323,15 +435,13 @@ __global__ void __launch_bounds__(kRgThreads) route_small_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = warp; t < T; t += nwarps)
+  for (int t = warp; t < T; t += kRsWarps)
     warp_topk(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k);
   __syncthreads();
-  __threadfence_block();
   const int R = T * k;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) sm.ids[r] = __ldcg(ids + r);
+  for (int r = threadIdx.x; r < R; r += blockDim.x) s_ids[r] = __ldcg(ids + r);
   __syncthreads();
-  small_permutation_block(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  if (warp == 0) warp_permutation(s_ids, s_cnt, s_rank, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
   if (threadIdx.x == 0) *done_counter = 0;  // ready for the next call
 }
 
@@ -473,10 +583,16 @@ size_t permute_large_hist_bytes(int T, int E, int k) {
 
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream) {
-  const int grid = (E + kRgExpertsPerCta - 1) / kRgExpertsPerCta;
-  return launch_pdl(route_small_kernel, dim3(grid), dim3(kRgThreads), 0, stream, x, wr, bias, T, H, E, k, ws.logits,
-                    ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched, ws.tile_base, block_n,
-                    ws.route_counter);
+  const int grid = (E + kRsExperts - 1) / kRsExperts;
+  const int nt = (T + 7) / 8;
+#define MOE_ROUTE_SMALL(NT_)                                                                                   \
+  return launch_pdl(route_small_kernel<NT_>, dim3(grid), dim3(kRsThreads), 0, stream, x, wr, bias, T, H, E, k, \
+                    ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched,          \
+                    ws.tile_base, block_n, ws.route_counter)
+  if (nt <= 1) MOE_ROUTE_SMALL(1);
+  if (nt <= 2) MOE_ROUTE_SMALL(2);
+  MOE_ROUTE_SMALL(4);
+#undef MOE_ROUTE_SMALL
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
