@@ -51,6 +51,11 @@ MOE_DEV uint32_t dq_pair(uint32_t word, int i, uint32_t mult) {
   return bf16x2_mul(v, mult);
 }
 
+// Nibbles i and i+4 of `word` moved to bits 4-7 / 20-23 (for int4_pair_fma).
+MOE_DEV uint32_t nibble_pair_at4(uint32_t word, int i) {
+  return i == 0 ? word << 4 : i == 1 ? word : i == 2 ? word >> 4 : word >> 8;
+}
+
 MOE_DEV uint32_t word_of(const uint4& c, int j) {
   return j == 0 ? c.x : j == 1 ? c.y : j == 2 ? c.z : c.w;
 }
@@ -65,7 +70,9 @@ __host__ __device__ inline int scale_row_bytes(int fmt, int K) {
 // Slices past K read as zero weights.
 struct RowChunk {
   uint4 codes;
-  uint32_t mult;
+  uint32_t mult;  // bf16x2 multiplier: the INT4 scale (or s/16 on the fused path), or 2^e for MXFP4
+  uint32_t add;   // INT4 fused path: bf16x2 -16s
+  bool fused;     // INT4: s/16 is a normal bf16, so int4_pair_fma is exact
 };
 
 template <int FMT>
@@ -76,13 +83,30 @@ MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int
     rc.codes = *reinterpret_cast<const uint4*>(codes + r * (K / 2) + k / 2);
     if (FMT == MOE_FMT_INT4_G128) {
       const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[r * int4_groups(K) + k / 128];
-      rc.mult = s | (s << 16);
+      const uint32_t ex = (s >> 7) & 0xFFu;
+      rc.fused = (ex >= 5u && ex <= 250u) || (s & 0x7FFFu) == 0u;
+      if (rc.fused && (s & 0x7FFFu) != 0u) {
+        const uint32_t d16 = s - (4u << 7);  // s / 16: exponent - 4
+        const uint32_t m16 = (s + (4u << 7)) ^ 0x8000u;  // -16 s: exponent + 4, sign flipped
+        rc.mult = d16 | (d16 << 16);
+        rc.add = m16 | (m16 << 16);
+      } else if (rc.fused) {
+        rc.mult = 0;   // s == 0: q * s = 0
+        rc.add = 0;
+      } else {
+        rc.mult = s | (s << 16);
+        rc.add = 0;
+      }
     } else {
       rc.mult = pow2_bf16x2(int(scales[r * (K / 32) + k / 32]) - 127);
+      rc.add = 0;
+      rc.fused = false;
     }
   } else {
-    rc.codes = make_uint4(0, 0, 0, 0);  // INT4 nibble 0 would be -8: zero the multiplier instead
+    rc.codes = make_uint4(0, 0, 0, 0);  // zero weights: multiplier 0 on both paths
     rc.mult = 0;
+    rc.add = 0;
+    rc.fused = true;
   }
   return rc;
 }
@@ -113,6 +137,13 @@ MOE_DEV void load_act_frags(const uint16_t* rowp, int K, int kb, int q, bool val
   }
 }
 
+// One bf16 pair (nibbles i, i+4 of `word`) of a row chunk.
+template <int FMT>
+MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i) {
+  if (FMT == MOE_FMT_INT4_G128 && rc.fused) return int4_pair_fma(nibble_pair_at4(word, i), rc.mult, rc.add);
+  return dq_pair<FMT>(word, i, rc.mult);
+}
+
 // acc[4] += W(rows r, r+8; one 128-k block) x activation fragments.
 template <int FMT>
 MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, const uint32_t (&b)[8][2]) {
@@ -122,10 +153,10 @@ MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t a[4];
-      a[0] = dq_pair<FMT>(wl, 2 * h, lo.mult);
-      a[1] = dq_pair<FMT>(wh, 2 * h, hi.mult);
-      a[2] = dq_pair<FMT>(wl, 2 * h + 1, lo.mult);
-      a[3] = dq_pair<FMT>(wh, 2 * h + 1, hi.mult);
+      a[0] = dq<FMT>(lo, wl, 2 * h);
+      a[1] = dq<FMT>(hi, wh, 2 * h);
+      a[2] = dq<FMT>(lo, wl, 2 * h + 1);
+      a[3] = dq<FMT>(hi, wh, 2 * h + 1);
       mma_bf16_16816(acc, a, b[2 * j + h][0], b[2 * j + h][1]);
     }
   }
@@ -148,12 +179,6 @@ MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, u
   bulk_g2s(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar);
 }
 
-// Wait for the staged rows (bounded); false if the wait gave up.
-MOE_DEV bool wait_staged(uint64_t* bar, uint32_t* status) {
-  volatile int never = 0;
-  return mbar_wait(bar, 0, &never, status);
-}
-
 // Per-stage shared-memory layout of a work unit: codes then scales, each
 // matrix slice 16-byte aligned.
 struct UnitLayout {
@@ -170,32 +195,31 @@ MOE_DEV UnitLayout unit_layout(int fmt, int K, int rows, int mats) {
 }
 
 // ---------------------------------------------------------------------------
-// gate_up + SwiGLU, persistent.  Work unit u = (touched slot u / (I/8),
-// features f0 = 8*(u % (I/8)) .. f0+7).  Its 16 weight rows are the 8 gate
-// rows f0.. and the 8 matching up rows I+f0.., staged as one 16-row tile
-// (gate rows 0-7, up rows 8-15), so the MMA's C fragment holds gate (c0, c1)
-// and up (c2, c3) of the same feature and token: SwiGLU needs no shuffle.
-// A CTA walks units u = blockIdx.x + i * gridDim.x with two shared-memory
-// stages: the bulk copies of unit i+2 start as soon as unit i's stage is
-// free.  The CTA's 4 warps split K; partial tiles are summed in shared memory;
-// a = bf16(silu(gate) * up) goes to act[p][f] for the expert's sorted rows p.
+// gate_up + SwiGLU, persistent, warp-specialised.  Work unit u = (touched slot
+// u / (I/8), features f0 = 8*(u % (I/8)) .. f0+7).  Its 16 weight rows are the
+// 8 gate rows f0.. and the 8 matching up rows I+f0.., staged as one 16-row
+// tile (gate rows 0-7, up rows 8-15), so the MMA's C fragment holds gate
+// (c0, c1) and up (c2, c3) of the same feature and token: SwiGLU needs no
+// shuffle.  A producer warp walks the CTA's units u = blockIdx.x + i*gridDim.x:
+// it writes each unit's routing metadata (expert, first sorted row, row count,
+// token of each row) into a header in shared memory and starts the bulk
+// copies of its codes and scales, two stages ahead.  Eight compute warps split
+// K, sum their partial tiles in shared memory and write a = bf16(silu(gate) *
+// up) to act[p][f] for the expert's sorted rows p.
 // ---------------------------------------------------------------------------
 constexpr int kGuFeatures = kDecRows / 2;  // features per gate_up unit
+constexpr int kGuWarps = 8;                // compute warps (split K)
+constexpr int kGuThreads = (kGuWarps + 1) * 32;
+constexpr int kGuStages = 2;
+constexpr int kHdrTokens = 32;             // token rows carried in a unit header
 
-template <int FMT>
-MOE_DEV void issue_gate_up_unit(const Bank& gu, int I, const int32_t* touched, int ftiles, int u, uint8_t* stage,
-                                const UnitLayout& L, uint64_t* bar) {
-  const int e = touched[1 + u / ftiles];
-  const long row_g = long(e) * gu.N + (u % ftiles) * kGuFeatures;
-  const int sb = scale_row_bytes(FMT, gu.K);
-  const uint32_t half_codes = uint32_t(kGuFeatures) * (gu.K / 2);
-  mbar_arrive_expect_tx(bar, staged_bytes<FMT>(gu, kDecRows));
-  stage_rows<FMT>(gu, row_g, kGuFeatures, stage, stage + L.cbytes, bar);
-  stage_rows<FMT>(gu, row_g + I, kGuFeatures, stage + half_codes, stage + L.cbytes + kGuFeatures * sb, bar);
-}
+struct UnitHeader {
+  int e, p0, n_e, pad;
+  int tok[kHdrTokens];  // token of sorted row p0 + i (i < min(n_e, 32))
+};
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act,
     uint32_t* status) {
@@ -203,38 +227,74 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
   const int K = gu.K;
   // stage layout: [16 rows of codes: gate 0-7, up 8-15][16 rows of scales]
   const UnitLayout L = unit_layout(FMT, K, kDecRows, 1);
-  float* red = reinterpret_cast<float*>(smem + 2 * L.stage_bytes);  // [warp][tile][4][lane]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kDecWarps * NT * 4 * 32);
+  UnitHeader* hdr = reinterpret_cast<UnitHeader*>(smem + kGuStages * L.stage_bytes);
+  float* red = reinterpret_cast<float*>(hdr + kGuStages);  // [warp][tile][4][lane]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + kGuWarps * NT * 4 * 32);
+  uint64_t* empty = full + kGuStages;
+  __shared__ int s_units;
+  __shared__ volatile int s_abort;  // raised by the first wait that gives up
 
   pdl_wait();
   pdl_trigger();
-  const int ftiles = I / kGuFeatures;
-  const int n_units = touched[0] * ftiles;
-  if (int(blockIdx.x) >= n_units) return;
-  if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    fence_mbar_init();
-    for (int st = 0; st < 2; ++st) {
-      const int u = blockIdx.x + st * gridDim.x;
-      if (u < n_units) issue_gate_up_unit<FMT>(gu, I, touched, ftiles, u, smem + st * L.stage_bytes, L, &bars[st]);
-    }
-  }
-  __syncthreads();  // barriers initialised before anyone waits on them
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ftiles = I / kGuFeatures;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    s_units = touched[0] * ftiles;
+    for (int st = 0; st < kGuStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kGuWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int n_units = s_units;
+  if (int(blockIdx.x) >= n_units) return;
+
+  if (warp == kGuWarps) {
+    // ---------------------------------------------------------------- producer
+    int i = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+      const int st = i % kGuStages;
+      if (!mbar_wait(&empty[st], ((i / kGuStages) & 1) ^ 1, &s_abort, status)) break;
+      const int e = touched[1 + u / ftiles];
+      const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
+      UnitHeader& h = hdr[st];
+      if (lane < n_e) h.tok[lane] = sorted_rows[p0 + lane] / top_k;
+      if (lane == 0) {
+        h.e = e;
+        h.p0 = p0;
+        h.n_e = n_e;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
+        const long row_g = long(e) * gu.N + (u % ftiles) * kGuFeatures;
+        const int sb = scale_row_bytes(FMT, K);
+        uint8_t* stage = smem + st * L.stage_bytes;
+        mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(gu, kDecRows));
+        stage_rows<FMT>(gu, row_g, kGuFeatures, stage, stage + L.cbytes, &full[st]);
+        stage_rows<FMT>(gu, row_g + I, kGuFeatures, stage + kGuFeatures * (K / 2), stage + L.cbytes + kGuFeatures * sb,
+                        &full[st]);
+      }
+      __syncwarp();
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------------- compute
   const int g = lane >> 2, q = lane & 3;
   const int nblk = (K + 127) / 128;
   int i = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
-    const int st = i & 1;
+    const int st = i % kGuStages;
+    const bool ok = mbar_wait(&full[st], (i / kGuStages) & 1, &s_abort, status);
     const uint8_t* s_c = smem + st * L.stage_bytes;
     const uint8_t* s_s = s_c + L.cbytes;
-    const int e = touched[1 + u / ftiles];
+    const UnitHeader& h = hdr[st];
+    const int p0 = h.p0, n_e = h.n_e;
     const int f0 = (u % ftiles) * kGuFeatures;
-    const int p0 = offsets[e], n_e = offsets[e + 1] - p0;
     const int ntiles = (n_e + 7) / 8;
-    volatile int never = 0;
-    const bool ok = mbar_wait(&bars[st], (i >> 1) & 1, &never, status);
     for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
       float acc[NT][4];
 #pragma unroll
@@ -247,10 +307,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
       for (int j = 0; j < NT; ++j) {
         const int c = (nt0 + j) * 8 + g;
         xval[j] = c < n_e;
-        xrow[j] = x + size_t(xval[j] ? sorted_rows[p0 + c] / top_k : 0) * K;
+        const int tok = !xval[j] ? 0 : (c < kHdrTokens ? h.tok[c] : sorted_rows[p0 + c] / top_k);
+        xrow[j] = x + size_t(tok) * K;
       }
       if (ok) {
-        for (int b = warp; b < nblk; b += kDecWarps) {
+        for (int b = warp; b < nblk; b += kGuWarps) {
           const int kb = b * 128;
           const RowChunk gate = smem_row_chunk<FMT>(s_c, s_s, g, K, kb, q);
           const RowChunk up = smem_row_chunk<FMT>(s_c, s_s, g + 8, K, kb, q);
@@ -267,7 +328,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
       for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int c = 0; c < 4; ++c) red[((warp * NT + j) * 4 + c) * 32 + lane] = acc[j][c];
-      __syncthreads();
+      named_barrier_sync(1, kGuWarps * 32);
       // warp w < NT finishes token tile nt0 + w
       const int j = warp;
       if (ok && j < NT && nt0 + j < ntiles) {
@@ -276,24 +337,20 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
         for (int c = 0; c < 4; ++c) {
           sum[c] = 0.f;
 #pragma unroll
-          for (int w = 0; w < kDecWarps; ++w) sum[c] += red[((w * NT + j) * 4 + c) * 32 + lane];
+          for (int w = 0; w < kGuWarps; ++w) sum[c] += red[((w * NT + j) * 4 + c) * 32 + lane];
         }
         // c0, c1: gate of feature f0+g at tokens 2q, 2q+1; c2, c3: up of the same
         const int f = f0 + g;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col = (nt0 + j) * 8 + 2 * q + h;
-          if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(sum[h], sum[2 + h]));
+        for (int hh = 0; hh < 2; ++hh) {
+          const int col = (nt0 + j) * 8 + 2 * q + hh;
+          if (col < n_e) act[size_t(p0 + col) * I + f] = f32_to_bf16_rn(silu_mul(sum[hh], sum[2 + hh]));
         }
       }
-      __syncthreads();
+      named_barrier_sync(1, kGuWarps * 32);
     }
-    // stage st is free again: start the unit two steps ahead
-    if (threadIdx.x == 0) {
-      fence_proxy_async_smem();  // the stage's generic-proxy reads before the bulk copies refill it
-      const int u2 = u + 2 * gridDim.x;
-      if (u2 < n_units) issue_gate_up_unit<FMT>(gu, I, touched, ftiles, u2, smem + st * L.stage_bytes, L, &bars[st]);
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
   }
 }
 
@@ -311,6 +368,18 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_gate_up_kernel(
 constexpr int kDnWarps = 16;
 constexpr int kDnStages = 2;
 constexpr int kDnTokens = 32;  // token chunk per pass
+
+// First sorted row in [p0, p1) whose token is >= t (rows ascend with the
+// token index), found 32 rows at a time with a warp ballot.
+MOE_DEV int chunk_bound(const int32_t* __restrict__ sorted_rows, int p0, int p1, int top_k, int t) {
+  const int lane = threadIdx.x & 31;
+  for (int p = p0; p < p1; p += 32) {
+    const bool below = p + lane < p1 && sorted_rows[p + lane] / top_k < t;
+    const unsigned m = __ballot_sync(0xffffffffu, below);
+    if (m != 0xffffffffu) return p + __popc(m);
+  }
+  return p1;
+}
 
 template <int FMT>
 MOE_DEV void issue_down_rows(const Bank& dn, int e, int f0, uint8_t* stage, const UnitLayout& L, uint64_t* bar) {
@@ -333,16 +402,18 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
   float* acc_w = accs + warp * kDnTokens * kDecRows;
   uint64_t* bars = reinterpret_cast<uint64_t*>(accs + kDnWarps * kDnTokens * kDecRows) + warp * kDnStages;
 
+  __shared__ volatile int s_abort;
   pdl_wait();
   pdl_trigger();
   const int f0 = blockIdx.x * kDecRows;
   const int n_touched = touched[0];
   const int nblk = (K + 127) / 128;
+  if (threadIdx.x == 0) s_abort = 0;
   if (lane == 0) {
     for (int st = 0; st < kDnStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
-  __syncwarp();
+  __syncthreads();
   int uses = 0;  // ring slots consumed so far by this warp (over all chunks)
   for (int t0 = 0; t0 < T; t0 += kDnTokens) {
     const int t1 = min(T, t0 + kDnTokens);
@@ -366,16 +437,25 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
       const uint8_t* s_s = s_c + L.cbytes;
       const int e = touched[1 + slot];
       // rows of expert e whose token lies in [t0, t1): a contiguous sub-range
-      // (sorted rows ascend with the token index)
-      int p0 = offsets[e], p1 = offsets[e + 1];
-      while (p0 < p1 && sorted_rows[p0] / top_k < t0) ++p0;
-      int pe = p0;
-      while (pe < p1 && sorted_rows[pe] / top_k < t1) ++pe;
+      // (sorted rows ascend with the token index); one chunk when T <= 32
+      int p0 = offsets[e], pe = offsets[e + 1];
+      if (T > kDnTokens) {
+        pe = chunk_bound(sorted_rows, p0, pe, top_k, t1);
+        p0 = chunk_bound(sorted_rows, p0, pe, top_k, t0);
+      }
       const int n_e = pe - p0;
-      volatile int never = 0;
-      const bool ok = mbar_wait(&bars[st], parity, &never, status);
+      const bool ok = mbar_wait(&bars[st], parity, &s_abort, status);
       const int ntiles = (n_e + 7) / 8;
       for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
+        // routing of the next 32 rows: lane l holds row nt0*8 + l
+        const int rl = nt0 * 8 + lane;
+        int my_tok = 0;
+        float my_w = 0.f;
+        if (rl < n_e) {
+          const int r = sorted_rows[p0 + rl];
+          my_tok = r / top_k - t0;
+          my_w = topk_w[r];
+        }
         float acc[NT][4];
 #pragma unroll
         for (int j = 0; j < NT; ++j)
@@ -399,11 +479,10 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
         for (int j = 0; j < NT; ++j) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int col = (nt0 + j) * 8 + 2 * q + h;
-            if (nt0 + j < ntiles && col < n_e) {
-              const int r = sorted_rows[p0 + col];
-              const int t = r / top_k - t0;
-              const float w = topk_w[r];
+            const int lr = j * 8 + 2 * q + h;  // row within this group of 32
+            const int t = __shfl_sync(0xffffffffu, my_tok, lr);
+            const float w = __shfl_sync(0xffffffffu, my_w, lr);
+            if (nt0 + j < ntiles && (nt0 + j) * 8 + 2 * q + h < n_e) {
               acc_w[t * kDecRows + g] += w * acc[j][h];
               acc_w[t * kDecRows + g + 8] += w * acc[j][2 + h];
             }
@@ -443,9 +522,10 @@ size_t unit_stage_bytes(int fmt, int K, int rows, int mats) {
   return size_t(mats) * (cbytes + ((sbytes + 15) & ~15));
 }
 
-// two unit stages + the cross-warp reduction buffer + two barriers
+// stages + unit headers + the cross-warp reduction buffer + barriers
 size_t gate_up_smem(int fmt, int K, int nt) {
-  return 2 * unit_stage_bytes(fmt, K, kDecRows, 1) + size_t(kDecWarps) * nt * 4 * 32 * 4 + 16;
+  return kGuStages * unit_stage_bytes(fmt, K, kDecRows, 1) + kGuStages * sizeof(UnitHeader) +
+         size_t(kGuWarps) * nt * 4 * 32 * 4 + 2 * kGuStages * 8;
 }
 
 // per-warp rings + per-warp accumulators + per-warp barriers
@@ -468,12 +548,12 @@ int sm_count_cached() {
 // Persistent grid: as many CTAs as fit on the GPU at once (at most `units`).
 // (computed once per kernel instantiation and shared-memory size)
 template <typename Kern>
-int persistent_grid(Kern k, size_t smem, int units) {
+int persistent_grid(Kern k, size_t smem, int units, int threads) {
   static size_t cached_smem = 0;
   static int per_sm = 0;
   if (per_sm == 0 || cached_smem != smem) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kDecWarps * 32, smem) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 1) n = 1;
     per_sm = n;
     cached_smem = smem;
   }
@@ -497,8 +577,8 @@ cudaError_t gate_up_nt(const moe_shape_t& s, const uint16_t* x, const Bank& gu, 
   const size_t smem = gate_up_smem(FMT, s.hidden, NT);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(k, smem, units);
-  return launch_pdl(k, dim3(grid), dim3(kDecWarps * 32), smem, stream, x, gu, s.inter, s.top_k,
+  const int grid = persistent_grid(k, smem, units, kGuThreads);
+  return launch_pdl(k, dim3(grid), dim3(kGuThreads), smem, stream, x, gu, s.inter, s.top_k,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows, ws.act,
                     ws.status);
 }

@@ -7,7 +7,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/moe_w4a16.h"
+#include "moe_w4a16.h"
 
 namespace moe {
 

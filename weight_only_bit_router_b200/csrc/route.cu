@@ -26,54 +26,73 @@ MOE_DEV uint32_t orderable(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Top-k of one token's logits by one warp (lane l holds experts l, l+32, ...,
-// PER = ceil(E/32) of them).  Each round takes the largest remaining value
-// with two warp reductions (max of the value key, then min of the expert
-// index among the lanes holding that value: ties go to the lower index).
-// Logits are read through L2 (they may come from other CTAs).
+// Inverse of orderable().
+MOE_DEV float from_orderable(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k of one token's logits by one warp.  Lane l holds experts l, l+32, ...
+// (PER = ceil(E/32) of them) and first sorts them by (value descending, expert
+// ascending) with a bitonic network in registers.  Each round then takes the
+// largest head with two warp reductions (max of the value key, then min of the
+// expert index among lanes whose head has that value: ties go to the lower
+// expert) and the winning lane drops its head.  Logits are read through L2
+// (they may come from other CTAs).
 template <int PER>
 MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
                          int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
-  float v[PER];
+  uint32_t key[PER];
+  int slot[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = i * 32 + lane;
-    float val = 0.f;
+    slot[i] = i;
+    key[i] = 0u;  // empty: below every real key
     if (e < E) {
-      val = __ldcg(row + e);
+      float val = __ldcg(row + e);
       if (bias) val = val + bias[e];  // fp32 add
+      key[i] = orderable(val);
     }
-    v[i] = val;
   }
-  uint32_t avail = 0;
+  // bitonic sort into ascending "worse" order: position 0 ends up the best
 #pragma unroll
-  for (int i = 0; i < PER; ++i)
-    if (i * 32 + lane < E) avail |= 1u << i;
+  for (int size = 2; size <= PER; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int l = i ^ stride;
+        if (l > i) {
+          // better(a, b): larger key, or equal key and lower slot
+          const bool l_better = key[l] > key[i] || (key[l] == key[i] && slot[l] < slot[i]);
+          const bool swap = ((i & size) == 0) ? l_better : !l_better;
+          if (swap) {
+            const uint32_t tk = key[i]; key[i] = key[l]; key[l] = tk;
+            const int ts = slot[i]; slot[i] = slot[l]; slot[l] = ts;
+          }
+        }
+      }
+    }
+  }
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    // this lane's best remaining entry (i ascending keeps its lower index on ties)
-    uint32_t bkey = 0;
-    int bi = 0;
-    float bv = 0.f;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const uint32_t key = orderable(v[i]);
-      if (((avail >> i) & 1u) && (key > bkey || bkey == 0)) {
-        bkey = key;
-        bi = i;
-        bv = v[i];
-      }
-    }
-    const uint32_t has = avail != 0;
-    const uint32_t kmax = __reduce_max_sync(0xffffffffu, has ? bkey : 0u);
-    const uint32_t cand = (has && bkey == kmax) ? uint32_t(bi * 32 + lane) : 0xffffffffu;
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t cand = (key[0] != 0u && key[0] == kmax) ? uint32_t(slot[0] * 32 + lane) : 0xffffffffu;
     const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    if (int(win & 31) == lane) avail &= ~(1u << (win >> 5));
-    // the winner's value reaches lane j through a shuffle
-    const float wv = __shfl_sync(0xffffffffu, bv, int(win & 31));
-    if (lane == j) { my_val = wv; my_id = int(win); }
+    if (int(win & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i + 1 < PER; ++i) {
+        key[i] = key[i + 1];
+        slot[i] = slot[i + 1];
+      }
+      key[PER - 1] = 0u;
+    }
+    if (lane == j) {
+      my_val = from_orderable(kmax);
+      my_id = int(win);
+    }
   }
   const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
   const float ex = lane < k ? expf(my_val - vmax) : 0.f;
@@ -365,7 +384,7 @@ MOE_DEV void bf16_frags(const uint16_t* rowp, bool valid, uint32_t (&b)[8][2]) {
   }
 }
 
-template <int NT>
+template <int NT, int PER>
 __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
     int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
@@ -436,7 +455,7 @@ __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
   if (!s_last) return;
   __threadfence();
   for (int t = warp; t < T; t += kRsWarps)
-    warp_topk(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k);
+    warp_topk_t<PER>(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k);
   __syncthreads();
   const int R = T * k;
   for (int r = threadIdx.x; r < R; r += blockDim.x) s_ids[r] = __ldcg(ids + r);
@@ -581,18 +600,30 @@ size_t permute_large_hist_bytes(int T, int E, int k) {
   return nblk * size_t(E) * sizeof(int32_t);
 }
 
+template <int NT>
+cudaError_t route_small_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                           const Workspace& ws, int block_n, cudaStream_t stream) {
+  const int grid = (E + kRsExperts - 1) / kRsExperts;
+  const int per = (E + 31) / 32;
+#define MOE_ROUTE_SMALL(PER_)                                                                                    \
+  return launch_pdl(route_small_kernel<NT, PER_>, dim3(grid), dim3(kRsThreads), 0, stream, x, wr, bias, T, H, E, \
+                    k, ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched,         \
+                    ws.tile_base, block_n, ws.route_counter)
+  if (per <= 1) MOE_ROUTE_SMALL(1);
+  if (per <= 2) MOE_ROUTE_SMALL(2);
+  if (per <= 4) MOE_ROUTE_SMALL(4);
+  if (per <= 8) MOE_ROUTE_SMALL(8);
+  if (per <= 16) MOE_ROUTE_SMALL(16);
+  MOE_ROUTE_SMALL(32);
+#undef MOE_ROUTE_SMALL
+}
+
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream) {
-  const int grid = (E + kRsExperts - 1) / kRsExperts;
   const int nt = (T + 7) / 8;
-#define MOE_ROUTE_SMALL(NT_)                                                                                   \
-  return launch_pdl(route_small_kernel<NT_>, dim3(grid), dim3(kRsThreads), 0, stream, x, wr, bias, T, H, E, k, \
-                    ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched,          \
-                    ws.tile_base, block_n, ws.route_counter)
-  if (nt <= 1) MOE_ROUTE_SMALL(1);
-  if (nt <= 2) MOE_ROUTE_SMALL(2);
-  MOE_ROUTE_SMALL(4);
-#undef MOE_ROUTE_SMALL
+  if (nt <= 1) return route_small_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+  if (nt <= 2) return route_small_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+  return route_small_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
 }
 
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
