@@ -76,17 +76,6 @@ MOE_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// INT4 dequantisation of a nibble pair straight to bf16(q * s) with one FMA.
-// OR-ing a nibble u into mantissa bits 4-7 of bf16 128.0 gives 128 + 16u;
-// (128 + 16u) * (s/16) - 16s = (u - 8) * s = q * s exactly, and the fused
-// multiply-add rounds that exact value once.  s/16 and 16s are exact when s/16
-// is a normal bf16 (exponent field >= 5); callers use int4_pair otherwise.
-// `w4` holds the pair's nibbles at bits 4-7 and 20-23.
-MOE_DEV uint32_t int4_pair_fma(uint32_t w4, uint32_t s_div16, uint32_t neg16s) {
-  const uint32_t v = lop3_and_or(w4, 0x00F000F0u, 0x43004300u);
-  return bf16x2_fma(v, s_div16, neg16s);
-}
-
 // E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the
 // nibble pair at bit offsets 0 and 16 of `w` after shifting by 4*i.
 // Magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; looked up with two byte permutes.

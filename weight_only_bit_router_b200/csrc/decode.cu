@@ -51,11 +51,6 @@ MOE_DEV uint32_t dq_pair(uint32_t word, int i, uint32_t mult) {
   return bf16x2_mul(v, mult);
 }
 
-// Nibbles i and i+4 of `word` moved to bits 4-7 / 20-23 (for int4_pair_fma).
-MOE_DEV uint32_t nibble_pair_at4(uint32_t word, int i) {
-  return i == 0 ? word << 4 : i == 1 ? word : i == 2 ? word >> 4 : word >> 8;
-}
-
 MOE_DEV uint32_t word_of(const uint4& c, int j) {
   return j == 0 ? c.x : j == 1 ? c.y : j == 2 ? c.z : c.w;
 }
@@ -70,9 +65,7 @@ __host__ __device__ inline int scale_row_bytes(int fmt, int K) {
 // Slices past K read as zero weights.
 struct RowChunk {
   uint4 codes;
-  uint32_t mult;  // bf16x2 multiplier: the INT4 scale (or s/16 on the fused path), or 2^e for MXFP4
-  uint32_t add;   // INT4 fused path: bf16x2 -16s
-  bool fused;     // INT4: s/16 is a normal bf16, so int4_pair_fma is exact
+  uint32_t mult;  // bf16x2 multiplier: the INT4 scale, or 2^e for MXFP4
 };
 
 template <int FMT>
@@ -83,30 +76,13 @@ MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int
     rc.codes = *reinterpret_cast<const uint4*>(codes + r * (K / 2) + k / 2);
     if (FMT == MOE_FMT_INT4_G128) {
       const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[r * int4_groups(K) + k / 128];
-      const uint32_t ex = (s >> 7) & 0xFFu;
-      rc.fused = (ex >= 5u && ex <= 250u) || (s & 0x7FFFu) == 0u;
-      if (rc.fused && (s & 0x7FFFu) != 0u) {
-        const uint32_t d16 = s - (4u << 7);  // s / 16: exponent - 4
-        const uint32_t m16 = (s + (4u << 7)) ^ 0x8000u;  // -16 s: exponent + 4, sign flipped
-        rc.mult = d16 | (d16 << 16);
-        rc.add = m16 | (m16 << 16);
-      } else if (rc.fused) {
-        rc.mult = 0;   // s == 0: q * s = 0
-        rc.add = 0;
-      } else {
-        rc.mult = s | (s << 16);
-        rc.add = 0;
-      }
+      rc.mult = s | (s << 16);
     } else {
       rc.mult = pow2_bf16x2(int(scales[r * (K / 32) + k / 32]) - 127);
-      rc.add = 0;
-      rc.fused = false;
     }
   } else {
-    rc.codes = make_uint4(0, 0, 0, 0);  // zero weights: multiplier 0 on both paths
+    rc.codes = make_uint4(0, 0, 0, 0);  // INT4 nibble 0 would be -8: zero the multiplier instead
     rc.mult = 0;
-    rc.add = 0;
-    rc.fused = true;
   }
   return rc;
 }
@@ -140,7 +116,6 @@ MOE_DEV void load_act_frags(const uint16_t* rowp, int K, int kb, int q, bool val
 // One bf16 pair (nibbles i, i+4 of `word`) of a row chunk.
 template <int FMT>
 MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i) {
-  if (FMT == MOE_FMT_INT4_G128 && rc.fused) return int4_pair_fma(nibble_pair_at4(word, i), rc.mult, rc.add);
   return dq_pair<FMT>(word, i, rc.mult);
 }
 
