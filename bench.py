@@ -221,6 +221,12 @@ def stage_work(moe, shape, T: int, touched: float):
                     "flops": 2 * R * 2 * I * H},
         "down": {"bytes": touched * down_bytes_per_expert(moe, shape) + R * I * 2 + R * H * 4,
                  "flops": 2 * R * H * I},
+        # the whole layer as one kernel: router weight, tokens in, touched experts' packed
+        # banks, output; the intermediates (logits, SwiGLU rows, per-row down outputs) stay in L2
+        "layer": {"bytes": E * H * 2 + T * H * 2
+                  + touched * (gate_up_bytes_per_expert(moe, shape) + down_bytes_per_expert(moe, shape))
+                  + T * H * 2,
+                  "flops": 2 * T * E * H + 2 * R * 3 * I * H},
     }
 
 
@@ -294,7 +300,8 @@ def run_ours(args, rank, local, world):
     ws = moe.alloc_workspace(shape, T, device)
     outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
-    path = moe.MOE_PATH_AUTO
+    path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL,
+            "fused": moe.MOE_PATH_FUSED}[args.path]
 
     def layer_call(l, events=None):
         moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
@@ -361,13 +368,19 @@ def run_ours(args, rank, local, world):
     ids_buf = torch.empty(T, shape.top_k, dtype=torch.int32, device=device)
     for l in range(L):
         moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
-                        bias=stack.bias[l], debug={"topk_ids_out": ids_buf})
+                        bias=stack.bias[l], path=path, debug={"topk_ids_out": ids_buf})
         touched.append(len(torch.unique(ids_buf)))
     avg_touched = float(np.mean(touched))
     work = stage_work(moe, shape, T, avg_touched)
     peaks, peak_kind = load_peaks()
     decode = T <= 32
-    dom = max(("router", "gate_up", "down"), key=lambda n: stage_avg[n])
+    single_kernel = moe.moe_forward_launch_count(shape, T, path, False) == 1
+    if single_kernel:
+        # one launch does every stage: stage 0's events bracket it
+        dom = "layer"
+        stage_avg = {"layer": stage_avg["router"]}
+    else:
+        dom = max(("router", "gate_up", "down"), key=lambda n: stage_avg[n])
     if decode:
         achieved = work[dom]["bytes"] / (stage_avg[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -427,7 +440,9 @@ def run_ours(args, rank, local, world):
                    "stack_layers": L, "packed_stack_bytes": stack.packed_bytes,
                    "l2": "inputs larger than L2: steps rotate over a 40-layer stack of packed weights",
                    "parallelism": f"dp{world} replicas (one stack per GPU)",
-                   "avg_touched_experts": avg_touched, "path": "decode GEMV" if decode else "tcgen05 grouped GEMM"},
+                   "avg_touched_experts": avg_touched,
+                   "path": ("single-kernel decode layer" if single_kernel else "decode GEMV") if decode
+                   else "tcgen05 grouped GEMM", "path_option": args.path},
         "roofline": roof,
         "stage_ms": stage_avg,
         "cpu_baseline": cpu,
@@ -517,6 +532,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode4")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["auto", "decode", "prefill", "fused"], default="auto",
+                    help="kernel path of moe_forward (auto: decode kernels up to 32 tokens, grouped GEMMs above)")
     ap.add_argument("--stack-layers", type=int, default=NUM_LAYERS,
                     help="layers in the packed stack (smaller only for profiling captures)")
     args = ap.parse_args(argv)

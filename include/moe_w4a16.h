@@ -182,13 +182,19 @@ typedef enum {
   MOE_PATH_AUTO = 0,      /* decode path for T <= 32, grouped tcgen05 GEMMs above */
   MOE_PATH_DECODE = 1,    /* weight-streaming GEMV kernels (any T; meant for T <= 32: above that
                              the down projection re-streams its weights per 32 tokens) */
-  MOE_PATH_PREFILL = 2    /* grouped tcgen05 GEMMs (any T >= 1) */
+  MOE_PATH_PREFILL = 2,   /* grouped tcgen05 GEMMs (any T >= 1) */
+  MOE_PATH_FUSED = 3      /* the whole layer as ONE persistent cooperative kernel (every CTA
+                             resident at once): 1 <= T <= 8, H <= 2048, I <= 512, H % 64 == 0;
+                             MOE_ERR_UNSUPPORTED otherwise */
 } moe_path_t;
 
 /* Number of timed stages moe_forward reports through stage_events. */
 #define MOE_NUM_STAGES 5
 /* Stage ids: 0 router logits, 1 top-k + permutation, 2 gate_up + SwiGLU,
- * 3 down projection, 4 weighted combine / output conversion. */
+ * 3 down projection, 4 weighted combine / output conversion.  When the layer
+ * runs as a single kernel (moe_forward_launch_count() == 1) stage 0's
+ * "before" event precedes that kernel and every other event follows it:
+ * stage 0 then times the whole layer and stages 1-4 read zero. */
 
 /* Optional extras of moe_forward / moe_forward_routed.  Every pointer may be
  * NULL; a NULL opts pointer means all defaults. */
@@ -243,12 +249,13 @@ MOE_API moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes,
 /* Number of kernels moe_forward (routed = 0) or moe_forward_routed
  * (routed = 1) launches for T tokens on `path` (memsets and the optional
  * debug copies are not kernels and are not counted); -1 if the arguments are
- * invalid. */
+ * invalid or the path does not support them. */
 MOE_API int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed);
 
 /* Synchronises `stream`, then reports MOE_ERR_TIMEOUT if a bounded
  * device-side wait of a previous moe_forward on this workspace expired (and
- * clears the flag), MOE_OK otherwise. */
+ * clears the flag together with every device counter of the workspace, as
+ * moe_workspace_init does), MOE_OK otherwise. */
 MOE_API moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* moe_forward for callers that cannot allocate device memory.  The model

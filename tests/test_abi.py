@@ -109,6 +109,13 @@ def test_forward_validation_happens_on_the_host():
     assert L.moe_forward(*a) == 1
     # T == 0 is a valid no-op
     assert L.moe_forward(*args(T=0)) == 0
+    # the single-kernel path takes at most 8 tokens
+    opts.path = moe.MOE_PATH_FUSED
+    a = args(T=9)
+    a[10] = ctypes.byref(opts)
+    assert L.moe_forward(*a) == 2
+    assert moe.moe_forward_launch_count(s, 9, moe.MOE_PATH_FUSED, False) == -1
+    assert moe.moe_forward_launch_count(s, 8, moe.MOE_PATH_FUSED, False) == 1
 
 
 def test_routed_forward_validation():

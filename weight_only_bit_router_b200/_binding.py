@@ -24,7 +24,7 @@ MOE_FMT_INT4_G128 = 1
 MOE_FMT_MXFP4_G32 = 2
 FORMATS = {"int4_g128": MOE_FMT_INT4_G128, "mxfp4": MOE_FMT_MXFP4_G32}
 
-MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_FUSED = 0, 1, 2, 3
 MOE_NUM_STAGES = 5
 STAGE_NAMES = ("router", "route_permute", "gate_up", "down", "combine")
 

@@ -101,6 +101,7 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
+  w.ypart = static_cast<float*>(take(decode_fused_ypart_bytes(s, T)));
   w.bytes = off;
   return w;
 }
@@ -171,20 +172,37 @@ moe_status_t copy_debug_outputs(const moe_shape_t& s, int T, const Workspace& ws
   return MOE_OK;
 }
 
+// On the single-kernel path every stage runs inside one launch: stage 0's
+// "before" event precedes it and all the other events follow it.
+moe_status_t mark_single_kernel_rest(const moe_forward_opts_t* o, cudaStream_t stream) {
+  MOE_TRY(mark(o, 0, 1, stream));
+  for (int st = 1; st < MOE_NUM_STAGES; ++st) {
+    MOE_TRY(mark(o, st, 0, stream));
+    MOE_TRY(mark(o, st, 1, stream));
+  }
+  return MOE_OK;
+}
+
+bool valid_path(moe_path_t p) {
+  return p == MOE_PATH_AUTO || p == MOE_PATH_DECODE || p == MOE_PATH_PREFILL || p == MOE_PATH_FUSED;
+}
+
 moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, int T, const void* gu,
                                   const void* dn, void* workspace, size_t ws_bytes, uint16_t* out,
-                                  const moe_forward_opts_t* opts, bool* decode) {
+                                  const moe_forward_opts_t* opts, bool* decode, bool* fused) {
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   if ((st = check_T(shape, T)) != MOE_OK) return st;
   const moe_path_t path = opts ? opts->path : MOE_PATH_AUTO;
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+  if (!valid_path(path)) return MOE_ERR_INVALID_ARG;
+  if (path == MOE_PATH_FUSED && T > 0 && !decode_fused_supported(*shape, T)) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;  // nothing to do; pointers may be null
   if (!x || !gu || !dn || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gu, 256) || !aligned(dn, 256) || !aligned(out, 16))
     return MOE_ERR_INVALID_ARG;
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
+  *fused = path == MOE_PATH_FUSED;
   *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
   return MOE_OK;
 }
@@ -296,13 +314,21 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
                          const float* logit_bias, const void* gate_up_packed, const void* down_packed,
                          void* workspace, size_t workspace_bytes, uint16_t* out, const moe_forward_opts_t* opts,
                          cudaStream_t stream) {
-  bool decode = false;
+  bool decode = false, fused = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
-                                         out, opts, &decode);
+                                         out, opts, &decode, &fused);
   if (st != MOE_OK || T == 0) return st;
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   const Workspace ws = carve_workspace(workspace, s, T);
+  if (fused) {
+    const Bank gu = make_bank(gate_up_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
+    const Bank dn = make_bank(down_packed, s.fmt, s.num_experts, s.hidden, s.inter);
+    MOE_TRY(mark(opts, 0, 0, stream));
+    MOE_TRY(launch_decode_fused(s, T, x, router_w, logit_bias, nullptr, nullptr, gu, dn, ws, out, stream));
+    if ((st = mark_single_kernel_rest(opts, stream)) != MOE_OK) return st;
+    return copy_debug_outputs(s, T, ws, opts, false, stream);
+  }
   MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT) {
     // router logits, top-k and the permutation in one kernel
@@ -325,15 +351,23 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
                                 const float* topk_w, const void* gate_up_packed, const void* down_packed,
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
                                 const moe_forward_opts_t* opts, cudaStream_t stream) {
-  bool decode = false;
+  bool decode = false, fused = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
-                                         out, opts, &decode);
+                                         out, opts, &decode, &fused);
   if (st != MOE_OK || T == 0) return st;
   if (!topk_ids || !topk_w || !aligned(topk_ids, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   Workspace ws = carve_workspace(workspace, s, T);
   ws.topk_ids = const_cast<int32_t*>(topk_ids);
   ws.topk_w = const_cast<float*>(topk_w);
+  if (fused) {
+    const Bank gu = make_bank(gate_up_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
+    const Bank dn = make_bank(down_packed, s.fmt, s.num_experts, s.hidden, s.inter);
+    MOE_TRY(mark(opts, 0, 0, stream));
+    MOE_TRY(launch_decode_fused(s, T, x, nullptr, nullptr, topk_ids, topk_w, gu, dn, ws, out, stream));
+    if ((st = mark_single_kernel_rest(opts, stream)) != MOE_OK) return st;
+    return copy_debug_outputs(s, T, ws, opts, true, stream);
+  }
   MOE_TRY(mark(opts, 1, 0, stream));
   if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
   MOE_TRY(mark(opts, 1, 1, stream));
@@ -343,9 +377,10 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
 
 int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed) {
   if (check_shape(shape) != MOE_OK || check_T(shape, T) != MOE_OK) return -1;
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return -1;
+  if (!valid_path(path)) return -1;
   if (T == 0) return 0;
   const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  if (path == MOE_PATH_FUSED) return decode_fused_supported(*shape, T) ? 1 : -1;  // the whole layer in one kernel
   const int perm = (long(T) * shape->top_k <= 1024) ? 1 : 3;
   int n = 0;
   if (routed) n += perm;
@@ -366,7 +401,9 @@ moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaS
   uint32_t word = 0;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (word & kStatusTimeout) {
-    if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+    // an expired wait can leave device counters mid-count: clear them all
+    if (cudaMemset(workspace, 0, workspace_bytes < kStatusBytes ? workspace_bytes : kStatusBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
     return MOE_ERR_TIMEOUT;
   }
   return MOE_OK;

@@ -149,6 +149,51 @@ MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint
   }
 }
 
+// Wait for the phase of `bar` with the given parity, ignoring any abort flag;
+// gives up (false) after limit_ns.  Used to drain copies still in flight.
+MOE_DEV bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// --------------------------------------------------------------------------
+// device-wide counters (CTAs of one cooperative grid waiting on each other)
+// --------------------------------------------------------------------------
+MOE_DEV uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+MOE_DEV uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Spin until *ctr >= target (acquire).  Gives up (returns false) when `abort`
+// is raised, when another CTA has already reported a timeout in the status
+// word, or after kWaitLimitNs, in which case it raises both.
+MOE_DEV bool spin_until_geq(const uint32_t* ctr, uint32_t target, volatile int* abort, uint32_t* gstatus) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (*abort) return false;
+    if (ld_relaxed_gpu(gstatus) & kStatusTimeout) {
+      *abort = 1;
+      return false;
+    }
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicOr(gstatus, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
 // --------------------------------------------------------------------------
 // TMA (tensor memory accelerator) and cp.async
 // --------------------------------------------------------------------------
@@ -269,6 +314,10 @@ MOE_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: 
 // misc
 // --------------------------------------------------------------------------
 MOE_DEV float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+MOE_DEV void red_add_u32(uint32_t* addr, uint32_t v) {
+  asm volatile("red.global.add.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
 
 MOE_DEV void red_add_f32(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");

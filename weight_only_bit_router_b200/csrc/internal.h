@@ -35,9 +35,10 @@ struct Bank {
 };
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
-// The first kStatusBytes of a workspace: the status word and the fused-routing
-// completion counter.  Zeroed once by moe_workspace_init; the counting kernel
-// resets its counter to zero.
+// The first kStatusBytes of a workspace: the status word and the kernels'
+// device counters (small-batch routing completion; the single-kernel decode
+// path's grid-wide counters).  Zeroed once by moe_workspace_init; every kernel
+// that counts leaves its counters at zero when it finishes.
 constexpr size_t kStatusBytes = 4096;
 
 struct Workspace {
@@ -54,6 +55,7 @@ struct Workspace {
   int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
+  float* ypart;           // [T*k, H] fp32 per-row down outputs (single-kernel decode path)
   size_t bytes;
 };
 
@@ -88,6 +90,14 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
                                   const Workspace& ws, cudaStream_t stream);
 cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
                                        uint16_t* out, cudaStream_t stream);
+
+// decode_fused.cu: the whole layer as one cooperative kernel for T <= 8
+bool decode_fused_supported(const moe_shape_t& s, int T);
+size_t decode_fused_ypart_bytes(const moe_shape_t& s, int T);
+// ids_in / w_in: the given routing (moe_forward_routed), or null to route from router_w
+cudaError_t launch_decode_fused(const moe_shape_t& s, int T, const uint16_t* x, const uint16_t* router_w,
+                                const float* bias, const int32_t* ids_in, const float* w_in, const Bank& gu,
+                                const Bank& dn, const Workspace& ws, uint16_t* out, cudaStream_t stream);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile

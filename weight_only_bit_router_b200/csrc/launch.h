@@ -26,4 +26,33 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Cooperative launch (every CTA resident at once, so CTAs may wait on one
+// another), with programmatic stream serialization when the driver accepts
+// both attributes together.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cooperative(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               Args&&... args) {
+  static int with_pdl = 1;  // cleared once the driver refuses the combination
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = with_pdl ? 2 : 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (err != cudaSuccess && with_pdl) {
+    (void)cudaGetLastError();
+    with_pdl = 0;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  }
+  return err;
+}
+
 }  // namespace moe

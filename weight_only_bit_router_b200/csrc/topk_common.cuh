@@ -1,0 +1,107 @@
+// Warp-level top-k of one token's router logits with the renormalised
+// softmax over the selected experts (ties to the lower expert index).
+#pragma once
+
+#include <float.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Order-preserving map of a non-NaN fp32 value to uint32 (-0 and +0 equal).
+MOE_DEV uint32_t orderable(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 + 0 = +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of orderable().
+MOE_DEV float from_orderable(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k of one token's logits by one warp.  Lane l holds experts l, l+32, ...
+// (PER = ceil(E/32) of them) and first sorts them by (value descending, expert
+// ascending) with a bitonic network in registers.  Each round then takes the
+// largest head with two warp reductions (max of the value key, then min of the
+// expert index among lanes whose head has that value: ties go to the lower
+// expert) and the winning lane drops its head.  Logits are read through L2
+// (they may come from other CTAs).
+template <int PER>
+MOE_DEV void warp_topk_t(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
+                         int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[PER];
+  int slot[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = i * 32 + lane;
+    slot[i] = i;
+    key[i] = 0u;  // empty: below every real key
+    if (e < E) {
+      float val = __ldcg(row + e);
+      if (bias) val = val + bias[e];  // fp32 add
+      key[i] = orderable(val);
+    }
+  }
+  // bitonic sort into ascending "worse" order: position 0 ends up the best
+#pragma unroll
+  for (int size = 2; size <= PER; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int l = i ^ stride;
+        if (l > i) {
+          // better(a, b): larger key, or equal key and lower slot
+          const bool l_better = key[l] > key[i] || (key[l] == key[i] && slot[l] < slot[i]);
+          const bool swap = ((i & size) == 0) ? l_better : !l_better;
+          if (swap) {
+            const uint32_t tk = key[i]; key[i] = key[l]; key[l] = tk;
+            const int ts = slot[i]; slot[i] = slot[l]; slot[l] = ts;
+          }
+        }
+      }
+    }
+  }
+  float my_val = 0.f;
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t cand = (key[0] != 0u && key[0] == kmax) ? uint32_t(slot[0] * 32 + lane) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if (int(win & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i + 1 < PER; ++i) {
+        key[i] = key[i + 1];
+        slot[i] = slot[i + 1];
+      }
+      key[PER - 1] = 0u;
+    }
+    if (lane == j) {
+      my_val = from_orderable(kmax);
+      my_id = int(win);
+    }
+  }
+  const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
+  const float ex = lane < k ? expf(my_val - vmax) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) {
+    ids[lane] = my_id;
+    wout[lane] = ex / sum;
+  }
+}
+
+MOE_DEV void warp_topk(const float* __restrict__ row, const float* __restrict__ bias, int E, int k,
+                       int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int per = (E + 31) / 32;
+  if (per <= 1) warp_topk_t<1>(row, bias, E, k, ids, wout);
+  else if (per <= 2) warp_topk_t<2>(row, bias, E, k, ids, wout);
+  else if (per <= 4) warp_topk_t<4>(row, bias, E, k, ids, wout);
+  else if (per <= 8) warp_topk_t<8>(row, bias, E, k, ids, wout);
+  else if (per <= 16) warp_topk_t<16>(row, bias, E, k, ids, wout);
+  else warp_topk_t<32>(row, bias, E, k, ids, wout);
+}
+
+}  // namespace moe
