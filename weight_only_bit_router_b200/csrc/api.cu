@@ -102,6 +102,7 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
   w.ypart = static_cast<float*>(take(decode_fused_ypart_bytes(s, T)));
+  w.route_part = static_cast<float*>(take(T <= kDecodeMaxT ? route_part_bytes(T, int(H), int(E), s.top_k) : 0));
   w.bytes = off;
   return w;
 }

@@ -228,6 +228,24 @@ MOE_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t
       : "memory");
 }
 
+// L2 cache policy for data read once per launch (streamed expert weights):
+// evicted first, so the stream does not push out kernel code, router weights
+// and small activations that every launch reuses.
+MOE_DEV uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// bulk_g2s with an L2 cache policy (see l2_policy_evict_first).
+MOE_DEV void bulk_g2s_hint(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // --------------------------------------------------------------------------
 // programmatic dependent launch: wait for the preceding kernel's results /
 // allow the next kernel in the stream to start launching

@@ -169,8 +169,10 @@ template <int FMT>
 MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, uint8_t* s_scales, uint64_t* bar) {
   const uint32_t cbytes = uint32_t(rows) * (bk.K / 2);
   const int sb = scale_row_bytes(FMT, bk.K);
-  bulk_g2s(s_codes, bk.codes + row0 * (bk.K / 2), cbytes, bar);
-  bulk_g2s(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar);
+  // packed weights are read once per launch: evict them first from L2
+  const uint64_t policy = l2_policy_evict_first();
+  bulk_g2s_hint(s_codes, bk.codes + row0 * (bk.K / 2), cbytes, bar, policy);
+  bulk_g2s_hint(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar, policy);
 }
 
 // Per-stage shared-memory layout of a work unit: codes then scales, each

@@ -56,6 +56,7 @@ struct Workspace {
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
   float* ypart;           // [T*k, H] fp32 per-row down outputs (single-kernel decode path)
+  float* route_part;      // [H/256, T, E] fp32 split-K router partials (small-batch routing)
   size_t bytes;
 };
 
@@ -72,6 +73,8 @@ cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, i
 // Fused router GEMV + top-k + permutation for T <= kDecodeMaxT.
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream);
+// split-K partial logits of the small-batch routing kernel (0 when it does not apply)
+size_t route_part_bytes(int T, int H, int E, int k);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t stream);
 // Small-T permutation (R = T*k <= 1024) in one CTA, with the touched-expert

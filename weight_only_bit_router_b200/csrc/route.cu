@@ -58,8 +58,10 @@ __device__ int block_exclusive_scan_1024(int* data, int n, int* warp_tot) {
 }
 
 // Exclusive scan of n <= 4 * blockDim.x ints in smem by a block of 256
-// threads (4 consecutive items per thread); returns the total.
-__device__ int block_exclusive_scan_256x4(int* data, int n, int* warp_tot) {
+// threads (4 consecutive items per thread); returns the total.  Not inlined:
+// callers run it several times once per launch, and one shared copy of the
+// code stays in the instruction cache.
+__device__ __noinline__ int block_exclusive_scan_256x4(int* data, int n, int* warp_tot) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int loc[4], sum = 0;
 #pragma unroll
@@ -365,6 +367,207 @@ __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Fused small-batch routing, split-K (T <= 32, E <= 256, k <= 8).  CTA
+// (tile, s) computes, with mma.sync, the partial logits of experts
+// [16 tile, 16 tile + 16) over k in [256 s, 256 s + 256) for every token and
+// stores them; spreading the router weight over (E/16) x (H/256) CTAs keeps
+// every SM's share of it small.  The last CTA to finish (device counter) sums
+// the partials in split order (deterministic), keeps the logits in shared
+// memory, runs the merge top-k (one warp per token) and the stable
+// permutation with the whole block.
+// ---------------------------------------------------------------------------
+constexpr int kRfK = 256;  // k per CTA
+constexpr int kRfMaxT = 32, kRfMaxE = 256, kRfMaxR = kRfMaxT * 8;
+constexpr int kRfMaxSplits = 8;  // H <= 8 * kRfK
+
+struct __align__(16) RouteFastSmem {
+  union __align__(16) {
+    float red[kRsWarps][4][32];                // GEMV: one C fragment per warp
+    float logit[kRfMaxT * kRfMaxE];             // last CTA: summed logits [T][E]
+  } u;
+  int ids[kRfMaxR];
+  int rank[kRfMaxR];
+  int wcnt[kRsWarps][kRfMaxE];                 // per-warp row counts, then per-warp bases
+  int off[kRfMaxE];                            // expert totals, then offsets
+  int last;
+};
+
+// Stable counting sort of R <= 256 rows (32 per warp) by expert (E <= 256)
+// with the whole 256-thread block and four block barriers, plus the
+// touched-expert list and the token-block prefix.  Ids outside [0, E) are
+// dropped.  Warp w ranks its rows with __match_any_sync; the experts' totals
+// and per-warp bases come from a pass over the 8 warps' counts; one warp then
+// scans the E totals with shuffles (8 experts per lane).
+__device__ void block_permutation_256(RouteFastSmem& sm, int R, int E, int32_t* __restrict__ offsets,
+                                      int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
+                                      int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned full = 0xffffffffu;
+  for (int i = tid; i < kRsWarps * E; i += blockDim.x) sm.wcnt[i / E][i % E] = 0;
+  __syncthreads();
+  const int r = warp * 32 + lane;
+  int e = r < R ? sm.ids[r] : -1;
+  if (e >= E) e = -1;
+  const unsigned mm = __match_any_sync(full, e);
+  const int before = __popc(mm & ((1u << lane) - 1u));
+  if (e >= 0 && before == 0) sm.wcnt[warp][e] = __popc(mm);
+  __syncthreads();
+  // per expert: bases over warps (in warp order) and the total
+  for (int x = tid; x < E; x += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kRsWarps; ++w) {
+      const int c = sm.wcnt[w][x];
+      sm.wcnt[w][x] = run;
+      run += c;
+    }
+    sm.off[x] = run;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // lane owns experts [8 lane, 8 lane + 8): totals, touched flags, token blocks
+    int c[8], cs = 0, nz = 0, bl = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = 8 * lane + u;
+      c[u] = x < E ? sm.off[x] : 0;
+      cs += c[u];
+      nz += c[u] > 0;
+      bl += (c[u] + block_n - 1) / block_n;
+    }
+    int ci = cs, ni = nz, bi = bl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a0 = __shfl_up_sync(full, ci, o), a1 = __shfl_up_sync(full, ni, o), a2 = __shfl_up_sync(full, bi, o);
+      if (lane >= o) {
+        ci += a0;
+        ni += a1;
+        bi += a2;
+      }
+    }
+    int run = ci - cs, tp = ni - nz, brun = bi - bl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = 8 * lane + u;
+      if (x < E) {
+        sm.off[x] = run;
+        offsets[x] = run;
+        tile_base[x] = brun;
+        if (c[u] > 0) touched[1 + tp++] = x;
+      }
+      run += c[u];
+      brun += (c[u] + block_n - 1) / block_n;
+    }
+    if (lane == 31) {
+      offsets[E] = ci;
+      tile_base[E] = bi;
+      touched[0] = ni;
+    }
+  }
+  __syncthreads();
+  if (r < R) {
+    if (e < 0) {
+      pos[r] = -1;
+    } else {
+      const int p = sm.off[e] + sm.wcnt[warp][e] + before;
+      sorted_rows[p] = r;
+      pos[r] = p;
+    }
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
+    int E, int k, float* __restrict__ logits, float* __restrict__ part, int32_t* __restrict__ ids,
+    float* __restrict__ wout, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
+    int32_t* __restrict__ pos, int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n,
+    int32_t* done_counter) {
+  __shared__ RouteFastSmem sm;
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int e0 = blockIdx.x * kRsExperts, ks = blockIdx.y, KS = gridDim.y;
+  // warp: k-block b of this split, token tile jt
+  const int b = warp & 1, jt = warp >> 1;
+  const int kblk = ks * kRfK + b * 128 + 32 * q;
+  const bool kin = kblk < H;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (jt < NT) {
+    const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
+    uint32_t alo[8][2], ahi[8][2], bf[8][2];
+    bf16_frags(wr + size_t(r_lo ? e0 + g : 0) * H + kblk, r_lo && kin, alo);
+    bf16_frags(wr + size_t(r_hi ? e0 + g + 8 : 0) * H + kblk, r_hi && kin, ahi);
+    const int t = jt * 8 + g;
+    bf16_frags(x + size_t(t < T ? t : 0) * H + kblk, t < T && kin, bf);
+#pragma unroll
+    for (int st = 0; st < 8; ++st) {
+      const uint32_t a[4] = {alo[st][0], ahi[st][0], alo[st][1], ahi[st][1]};
+      mma_16816(acc, a, bf[st][0], bf[st][1]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sm.u.red[warp][c][lane] = acc[c];
+  __syncthreads();
+  if (b == 0 && jt < NT) {
+    // this CTA's partial logits of token tile jt: the two k-blocks in order
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float v = sm.u.red[warp][c][lane] + sm.u.red[warp + 1][c][lane];
+      // c0, c1: expert e0+g, tokens 2q, 2q+1; c2, c3: expert e0+g+8
+      const int t = jt * 8 + 2 * q + (c & 1);
+      const int e = e0 + g + ((c >> 1) << 3);
+      if (t < T && e < E) part[(size_t(ks) * T + t) * E + e] = v;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    sm.last = atomicAdd(done_counter, 1) == int(gridDim.x * gridDim.y) - 1;
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  // logits = sum of the split partials, in split order; four logits per
+  // thread-step, every split's load in flight at once (KS <= kRfMaxSplits)
+  const int n4 = T * E / 4;
+  const float4* part4 = reinterpret_cast<const float4*>(part);
+  for (int i0 = threadIdx.x; i0 < n4; i0 += 2 * blockDim.x) {
+    float4 v[2][kRfMaxSplits];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int s2 = 0; s2 < kRfMaxSplits; ++s2) {
+        const int idx = i0 + h * blockDim.x;
+        v[h][s2] = (s2 < KS && idx < n4) ? __ldcg(part4 + size_t(s2) * n4 + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int idx = i0 + h * blockDim.x;
+      if (idx >= n4) continue;
+      float4 sum = v[h][0];
+#pragma unroll
+      for (int s2 = 1; s2 < kRfMaxSplits; ++s2) {
+        sum.x += v[h][s2].x;
+        sum.y += v[h][s2].y;
+        sum.z += v[h][s2].z;
+        sum.w += v[h][s2].w;
+      }
+      reinterpret_cast<float4*>(sm.u.logit)[idx] = sum;
+      reinterpret_cast<float4*>(logits)[idx] = sum;
+    }
+  }
+  __syncthreads();
+  for (int t = warp; t < T; t += kRsWarps) warp_topk8(sm.u.logit + t * E, bias, E, k, sm.ids + t * k, wout + t * k);
+  __syncthreads();
+  const int R = T * k;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) ids[r] = sm.ids[r];
+  block_permutation_256(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  if (threadIdx.x == 0) *done_counter = 0;  // ready for the next call
+}
+
+// ---------------------------------------------------------------------------
 // Large permutation, any R.  Blocks of 256 rows.
 // K1: per-block histogram + stable rank of each row inside its block.
 // K2: one CTA scans counts over experts and over blocks (bases per block).
@@ -518,9 +721,31 @@ cudaError_t route_small_nt(const uint16_t* x, const uint16_t* wr, const float* b
 #undef MOE_ROUTE_SMALL
 }
 
+template <int NT>
+cudaError_t route_fast_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                          const Workspace& ws, int block_n, cudaStream_t stream) {
+  const dim3 grid((E + kRsExperts - 1) / kRsExperts, (H + kRfK - 1) / kRfK);
+  return launch_pdl(route_fast_kernel<NT>, grid, dim3(kRsThreads), 0, stream, x, wr, bias, T, H, E, k, ws.logits,
+                    ws.route_part, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched,
+                    ws.tile_base, block_n, ws.route_counter);
+}
+
+bool route_fast_applies(int T, int H, int E, int k) {
+  return T <= kRfMaxT && E <= kRfMaxE && E % 4 == 0 && k <= 8 && H <= kRfMaxSplits * kRfK;
+}
+
+size_t route_part_bytes(int T, int H, int E, int k) {
+  return route_fast_applies(T, H, E, k) ? size_t((H + kRfK - 1) / kRfK) * T * E * sizeof(float) : 0;
+}
+
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream) {
   const int nt = (T + 7) / 8;
+  if (route_fast_applies(T, H, E, k)) {
+    if (nt <= 1) return route_fast_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+    if (nt <= 2) return route_fast_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+    return route_fast_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+  }
   if (nt <= 1) return route_small_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
   if (nt <= 2) return route_small_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
   return route_small_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
