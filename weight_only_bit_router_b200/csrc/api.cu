@@ -205,6 +205,7 @@ moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, i
   if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
   *fused = path == MOE_PATH_FUSED;
   *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  if (!*fused && !*decode && !grouped_supported(*shape)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 

@@ -18,12 +18,15 @@
 // activations, "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary),
 // and the token rows of each expert are gathered by cp.async.
 //
-// Warp roles (384 threads):
-//   warp 0      TMA producer: code tiles (or router weight tiles)
-//   warp 1      TMEM allocation + single-thread tcgen05.mma issue
-//   warps 2-3   token-row gather (cp.async, 16 B per thread per copy)
-//   warps 4-7   dequantisation, one weight row per thread
-//   warps 8-11  epilogue, one TMEM lane (weight row) per thread
+// Warp roles (512 threads):
+//   warp 0       TMA producer: code tiles (or router weight tiles), and once
+//                per tile a bulk copy of the tile's scale rows
+//   warp 1       TMEM allocation + single-thread tcgen05.mma issue
+//   warps 2-3    token-row gather (cp.async, 16 B per thread per copy)
+//   warps 4-11   dequantisation, two threads per weight row (32 k each)
+//   warps 12-15  epilogue, one TMEM lane (weight row) per thread; the down
+//                product's weighted tile goes through shared memory and is
+//                added into the fp32 output with one bulk reduction per token
 // Every wait is bounded; an expired wait raises the workspace status word and
 // the CTA unwinds, frees its tensor memory and exits.
 #include <stdio.h>
@@ -42,9 +45,13 @@ enum GemmMode { kRouter = 0, kGateUp = 1, kDown = 2 };
 constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BN = kGemmBN;    // token columns per tile (max MMA N)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int SO = 3;          // operand stages (bf16 A + gathered B)
-constexpr int SC = 4;          // code stages
-constexpr int kThreads = 384;
+constexpr int SA = 2;          // bf16 weight-operand stages (dequantised, or router weights by TMA)
+constexpr int SB = 6;          // gathered token-operand stages (the gather waits out L2/HBM latency)
+constexpr int SC = 3;          // code stages
+constexpr int kThreads = 512;
+constexpr int kDqThreads = 256;           // dequantisation threads (warps 4-11)
+constexpr int kEpiWarp0 = 12;             // first epilogue warp
+constexpr int kMaxScaleRow = 64;          // scale bytes per weight row (K <= 2048)
 constexpr int kTileBytes = BM * BK * 2;   // 16 KB bf16 operand tile
 constexpr int kCodeBytes = BM * BK / 2;   // 4 KB code tile
 
@@ -71,11 +78,14 @@ template <int MODE>
 struct Cfg {
   static constexpr int NACC = MODE == kGateUp ? 2 : 1;                 // accumulators per tile
   static constexpr uint32_t TMEM_COLS = MODE == kGateUp ? 512 : 256;   // 2 buffers x NACC x BN
-  static constexpr int SMEM_A = SO * NACC * kTileBytes;
-  static constexpr int SMEM_B = SO * kTileBytes;
+  static constexpr int SMEM_A = SA * NACC * kTileBytes;
+  static constexpr int SMEM_B = SB * kTileBytes;
   static constexpr int SMEM_C = SC * NACC * kCodeBytes;
-  static constexpr int SMEM = SMEM_A + SMEM_B + SMEM_C + 1024 /*barriers*/ + 1024 /*align*/ +
+  static constexpr int SMEM_S = MODE == kRouter ? 0 : 2 * NACC * BM * kMaxScaleRow;  // two tiles of scale rows
+  static constexpr int SMEM_D = MODE == kDown ? BN * BM * 4 : 0;                     // down: [token][row] fp32
+  static constexpr int SMEM = SMEM_A + SMEM_B + SMEM_C + SMEM_S + SMEM_D + 1024 /*barriers*/ + 1024 /*align*/ +
                              (kMaxExperts + 1) * 4;
+  static_assert(SMEM <= 232448, "shared memory of one CTA");
 };
 
 struct Tile {
@@ -164,38 +174,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NACC = C::NACC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                          // [SO][NACC][16 KB]
-  uint8_t* sB = sA + C::SMEM_A;                // [SO][16 KB]
+  uint8_t* sA = smem;                          // [SA][NACC][16 KB]
+  uint8_t* sB = sA + C::SMEM_A;                // [SB][16 KB]
   uint8_t* sC = sB + C::SMEM_B;                // [SC][NACC][4 KB]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::SMEM_C);
+  uint8_t* sS = sC + C::SMEM_C;                // [2][NACC][BM rows][scale row bytes]
+  float* sD = reinterpret_cast<float*>(sS + C::SMEM_S);  // down: [BN tokens][BM rows]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + C::SMEM_S + C::SMEM_D);
   uint64_t* codes_full = bars;                 // [SC]
   uint64_t* codes_empty = codes_full + SC;     // [SC]
-  uint64_t* opA_full = codes_empty + SC;       // [SO]
-  uint64_t* opB_full = opA_full + SO;          // [SO]
-  uint64_t* op_empty = opB_full + SO;          // [SO]
-  uint64_t* acc_full = op_empty + SO;          // [2]
+  uint64_t* opA_full = codes_empty + SC;       // [SA]
+  uint64_t* opA_empty = opA_full + SA;         // [SA]
+  uint64_t* opB_full = opA_empty + SA;         // [SB]
+  uint64_t* opB_empty = opB_full + SB;         // [SB]
+  uint64_t* acc_full = opB_empty + SB;         // [2]
   uint64_t* acc_empty = acc_full + 2;          // [2]
   uint64_t* drain = acc_empty + 2;             // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sc_full = drain + 1;               // [2] scale rows of a tile
+  uint64_t* sc_empty = sc_full + 2;            // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sc_empty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_tile_base = reinterpret_cast<int*>(bars + 64);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmArgs& a = args;
+  // scale bytes per weight row (INT4: bf16 per 128 k; MXFP4: one byte per 32 k)
+  const int sb = FMT == MOE_FMT_INT4_G128 ? 2 * a.scale_row_stride : a.scale_row_stride;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SC; ++i) {
       mbar_init(&codes_full[i], 1);
-      mbar_init(&codes_empty[i], 128);
+      mbar_init(&codes_empty[i], kDqThreads / 32);
     }
-    for (int i = 0; i < SO; ++i) {
-      mbar_init(&opA_full[i], MODE == kRouter ? 1 : 128);
+    for (int i = 0; i < SA; ++i) {
+      mbar_init(&opA_full[i], MODE == kRouter ? 1 : kDqThreads / 32);
+      mbar_init(&opA_empty[i], 1);
+    }
+    for (int i = 0; i < SB; ++i) {
       mbar_init(&opB_full[i], 64);
-      mbar_init(&op_empty[i], 1);
+      mbar_init(&opB_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], 4);
+      mbar_init(&sc_full[i], 1);
+      mbar_init(&sc_empty[i], kDqThreads / 32);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -220,12 +242,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t g = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const Tile t = decode_tile(a, tile, s_tile_base);
+        if (MODE != kRouter) {
+          // the tile's scale rows: contiguous rows of the scale plane, once per tile
+          const int slot = it & 1;
+          if (!(ok = mbar_wait(&sc_empty[slot], ((it >> 1) & 1) ^ 1, abort, a.status))) break;
+          const int f0 = t.fb * BM;
+          const int rows = min(BM, a.M_total - f0);
+          const uint32_t bytes = uint32_t(rows * sb);
+          mbar_arrive_expect_tx(&sc_full[slot], NACC * bytes);
+          const uint8_t* sp = static_cast<const uint8_t*>(a.scales);
+#pragma unroll
+          for (int c = 0; c < NACC; ++c) {
+            long row0;
+            if (MODE == kGateUp) row0 = long(t.e) * 2 * a.I + (c ? a.I : 0) + f0;
+            else row0 = long(t.e) * a.H + f0;
+            bulk_g2s(sS + (slot * NACC + c) * BM * kMaxScaleRow, sp + row0 * sb, bytes, &sc_full[slot]);
+          }
+        }
         for (int ks = 0; ks < KS; ++ks, ++g) {
           if (MODE == kRouter) {
-            const int s = g % SO;
-            if (!(ok = mbar_wait(&op_empty[s], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+            const int s = g % SA;
+            if (!(ok = mbar_wait(&opA_empty[s], ((g / SA) & 1) ^ 1, abort, a.status))) break;
             mbar_arrive_expect_tx(&opA_full[s], kTileBytes);
             tma_load_2d(sA + s * NACC * kTileBytes, &tmap_a, &opA_full[s], ks * BK, t.fb * BM);
           } else {
@@ -245,12 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         // let copies already in flight land before the CTA unwinds
         volatile int never = 0;
-        for (uint32_t i = 0; i < (MODE == kRouter ? SO : SC) && i < g; ++i) {
+        for (uint32_t i = 0; i < (MODE == kRouter ? SA : SC) && i < g; ++i) {
           const uint32_t gg = g - 1 - i;
           if (MODE == kRouter)
-            mbar_wait(&opA_full[gg % SO], (gg / SO) & 1, &never, nullptr);
+            mbar_wait(&opA_full[gg % SA], (gg / SA) & 1, &never, nullptr);
           else
             mbar_wait(&codes_full[gg % SC], (gg / SC) & 1, &never, nullptr);
+        }
+        if (MODE != kRouter && it > 0) {
+          const int last = it - 1;
+          mbar_wait(&sc_full[last & 1], (last >> 1) & 1, &never, nullptr);
         }
       }
     }
@@ -269,12 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc = umma_idesc_bf16(BM, n16);
         const uint32_t d0 = tmem_base + uint32_t(buf * NACC * BN);
         for (int ks = 0; ks < KS; ++ks, ++g) {
-          const int s = g % SO;
-          if (!(ok = mbar_wait(&opA_full[s], (g / SO) & 1, abort, a.status))) break;
-          if (!(ok = mbar_wait(&opB_full[s], (g / SO) & 1, abort, a.status))) break;
+          const int sa = g % SA, sbuf = g % SB;
+          if (!(ok = mbar_wait(&opA_full[sa], (g / SA) & 1, abort, a.status))) break;
+          if (!(ok = mbar_wait(&opB_full[sbuf], (g / SB) & 1, abort, a.status))) break;
+          // the token rows landed through cp.async (generic proxy): order them
+          // before the tensor core's (async proxy) reads
+          fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + s * NACC * kTileBytes);
-          const uint32_t b_addr = smem_u32(sB + s * kTileBytes);
+          const uint32_t a_addr = smem_u32(sA + sa * NACC * kTileBytes);
+          const uint32_t b_addr = smem_u32(sB + sbuf * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(b_addr + kk * 32);
@@ -284,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_bf16(d0 + c * BN, adesc, bdesc, idesc, (ks | kk) != 0 ? 1u : 0u);
             }
           }
-          umma_commit(&op_empty[s]);
+          umma_commit(&opA_empty[sa]);
+          umma_commit(&opB_empty[sbuf]);
         }
         if (!ok) break;
         umma_commit(&acc_full[buf]);
@@ -297,13 +345,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ token gather
-    // Copies of stage g are issued before stage g-2 is released, so two
-    // stages of 16-byte copies are in flight per thread.
-    constexpr uint32_t LAG = SO - 1;
+    // The stage's copies signal its full barrier themselves when they land
+    // (cp.async.mbarrier.arrive.noinc), so the gather never waits on its own
+    // copies and runs up to SB stages ahead of the tensor core.
     const int lt = threadIdx.x - 64;  // 0..63
     const int c = lt & 7;             // 16-byte chunk of the 128-byte row slice
     const int r0 = lt >> 3;           // rows r0, r0+8, ..., r0+120
-    uint32_t g = 0, released = 0;
+    uint32_t g = 0;
     bool ok = true;
     const int ld = (MODE == kDown) ? a.I : a.H;  // row length of the token operand
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -319,80 +367,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         src[i] = a.bsrc + row * ld + c * 8;
       }
       for (int ks = 0; ks < KS; ++ks, ++g) {
-        const int s = g % SO;
-        if (!(ok = mbar_wait(&op_empty[s], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+        const int s = g % SB;
+        if (!(ok = mbar_wait(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status))) break;
         const uint32_t base = smem_u32(sB + s * kTileBytes);
 #pragma unroll
         for (int i = 0; i < BN / 8; ++i) {
           const int r = r0 + 8 * i;
           if (r < n16) cp_async_16(base + sw128_offset(r, c), src[i] + ks * BK);
         }
-        cp_async_commit();
-        if (g + 1 - released > LAG) {
-          cp_async_wait<LAG>();
-          fence_proxy_async_smem();
-          mbar_arrive(&opB_full[released % SO]);
-          ++released;
-        }
+        cp_async_mbar_arrive_noinc(&opB_full[s]);
       }
     }
-    cp_async_wait<0>();
-    if (ok) {
-      fence_proxy_async_smem();
-      for (; released < g; ++released) mbar_arrive(&opB_full[released % SO]);
-    }
-  } else if (warp >= 4 && warp < 8) {
+    cp_async_wait<0>();  // nothing in flight into shared memory when the CTA exits
+  } else if (warp >= 4 && warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantisation
+    // Two threads per weight row: thread half h writes the row's 32 k at
+    // 32 h .. 32 h + 31 of every 64-wide stage.
     if (MODE != kRouter) {
-      const int r = threadIdx.x - 128;  // weight row inside the tile
+      const int d = threadIdx.x - 128;  // 0..255
+      const int r = d >> 1, h = d & 1;
       uint32_t g = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const Tile t = decode_tile(a, tile, s_tile_base);
         const int f = t.fb * BM + r;
         const bool valid = f < a.M_total;
-        long srow[NACC];
-        if (MODE == kGateUp) {
-          srow[0] = long(t.e) * 2 * a.I + f;
-          if (NACC > 1) srow[NACC - 1] = long(t.e) * 2 * a.I + a.I + f;
-        } else {
-          srow[0] = long(t.e) * a.H + f;
-        }
+        const int slot = it & 1;
+        if (!(ok = mbar_wait(&sc_full[slot], (it >> 1) & 1, abort, a.status))) break;
+        const uint8_t* srows = sS + slot * NACC * BM * kMaxScaleRow + r * sb;
         for (int ks = 0; ks < KS; ++ks, ++g) {
-          const int sc = g % SC, so = g % SO;
+          const int sc = g % SC, so = g % SA;
           if (!(ok = mbar_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
-          if (!(ok = mbar_wait(&op_empty[so], ((g / SO) & 1) ^ 1, abort, a.status))) break;
+          if (!(ok = mbar_wait(&opA_empty[so], ((g / SA) & 1) ^ 1, abort, a.status))) break;
 #pragma unroll
           for (int c = 0; c < NACC; ++c) {
             const uint8_t* ctile = sC + (sc * NACC + c) * kCodeBytes + r * (BK / 2);
-            const uint4 c0 = *reinterpret_cast<const uint4*>(ctile);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(ctile + 16);
-            uint32_t m0 = 0, m1 = 0;
+            const uint4 cw = *reinterpret_cast<const uint4*>(ctile + 16 * h);
+            uint32_t m = 0;
             if (valid) {
+              const uint8_t* srow = srows + c * BM * kMaxScaleRow;
               if (FMT == MOE_FMT_INT4_G128) {
-                const uint32_t s = static_cast<const uint16_t*>(a.scales)[srow[c] * a.scale_row_stride +
-                                                                          (ks * BK) / 128];
-                m0 = m1 = s | (s << 16);
+                const uint32_t sv = reinterpret_cast<const uint16_t*>(srow)[(ks * BK) / 128];
+                m = sv | (sv << 16);
               } else {
-                const uint8_t* sp = static_cast<const uint8_t*>(a.scales) + srow[c] * a.scale_row_stride +
-                                    (ks * BK) / 32;
-                m0 = pow2x2(int(sp[0]) - 127);
-                m1 = pow2x2(int(sp[1]) - 127);
+                m = pow2x2(int(srow[(ks * BK) / 32 + h]) - 127);
               }
             }
-            uint8_t* atile = sA + (so * NACC + c) * kTileBytes;
-            dequant_store32<FMT>(c0, m0, atile, r, 0);
-            dequant_store32<FMT>(c1, m1, atile, r, 1);
+            dequant_store32<FMT>(cw, m, sA + (so * NACC + c) * kTileBytes, r, h);
           }
+          // this thread's bf16 stores before the tensor core reads them
           fence_proxy_async_smem();
-          mbar_arrive(&opA_full[so]);
-          mbar_arrive(&codes_empty[sc]);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&opA_full[so]);
+            mbar_arrive(&codes_empty[sc]);
+          }
         }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sc_empty[slot]);  // the tile's scale rows are no longer read
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 8;          // TMEM lanes 32*ew .. 32*ew+31
+    const int ew = warp - kEpiWarp0;  // TMEM lanes 32*ew .. 32*ew+31
     const int r = ew * 32 + lane;     // weight row inside the tile
     int it = 0;
     bool ok = true;
@@ -404,6 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int f = t.fb * BM + r;
       const bool row_ok = f < a.M_total;
       const uint32_t taddr = tmem_base + (uint32_t(ew * 32) << 16) + uint32_t(buf * NACC * BN);
+      if (MODE == kDown) {
+        // the previous tile's bulk reductions must have read the staging buffer
+        if (it > 0) {
+          if (r < BN) bulk_wait_read_all();
+          named_barrier_sync(1, 128);
+        }
+      }
       for (int c0 = 0; c0 < t.n; c0 += 32) {
         uint32_t v0[32];
         tmem_ld32(taddr + c0, v0);
@@ -421,19 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else if (MODE == kDown) {
           tmem_ld_wait();
-          // routing of the 32 columns: lane j fetches column c0 + j
-          int tok = 0;
+          // weights of the 32 columns: lane j fetches column c0 + j
           float wgt = 0.f;
-          if (c0 + lane < t.n) {
-            const int rr = a.sorted_rows[t.p_begin + c0 + lane];
-            tok = rr / a.top_k;
-            wgt = a.topk_w[rr];
-          }
+          if (c0 + lane < t.n) wgt = a.topk_w[a.sorted_rows[t.p_begin + c0 + lane]];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int tj = __shfl_sync(0xffffffffu, tok, j);
             const float wj = __shfl_sync(0xffffffffu, wgt, j);
-            if (row_ok && c0 + j < t.n) red_add_f32(a.out_acc + size_t(tj) * a.H + f, wj * __uint_as_float(v0[j]));
+            sD[(c0 + j) * BM + r] = wj * __uint_as_float(v0[j]);  // row-contiguous per token
           }
         } else {
           tmem_ld_wait();
@@ -445,8 +485,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (MODE == kDown) {
+        // every row of the weighted tile is staged: one bulk add per token
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (r < t.n) {
+          const int tok = a.sorted_rows[t.p_begin + r] / a.top_k;
+          const int rows = min(BM, a.M_total - t.fb * BM);
+          bulk_reduce_add_f32(a.out_acc + size_t(tok) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
+          bulk_commit_group();
+        }
+      }
     }
+    if (MODE == kDown) bulk_wait_all();  // the reductions are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -587,6 +640,12 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int
   a.status = status;
   const int tiles = a.n_ftiles * ((T + BN - 1) / BN);
   return launch_gemm<kRouter, 0>(map, a, tiles, stream);
+}
+
+bool grouped_supported(const moe_shape_t& s) {
+  // a tile's scale rows are staged in shared memory, kMaxScaleRow bytes per row
+  const auto row_bytes = [&](int K) { return s.fmt == MOE_FMT_INT4_G128 ? 2 * int4_groups(K) : K / 32; };
+  return row_bytes(s.hidden) <= kMaxScaleRow && row_bytes(s.inter) <= kMaxScaleRow;
 }
 
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,

@@ -104,6 +104,8 @@ cudaError_t launch_decode_fused(const moe_shape_t& s, int T, const uint16_t* x, 
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
+// the grouped GEMMs support the shape (scale rows of a tile fit their staging buffer)
+bool grouped_supported(const moe_shape_t& s);
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
                                uint32_t* status, cudaStream_t stream);
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
