@@ -45,8 +45,8 @@ enum GemmMode { kRouter = 0, kGateUp = 1, kDown = 2 };
 constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BN = kGemmBN;    // token columns per tile (max MMA N)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int SA = 2;          // bf16 weight-operand stages (dequantised, or router weights by TMA)
-constexpr int SB = 6;          // gathered token-operand stages (the gather waits out L2/HBM latency)
+constexpr int SA = 3;          // bf16 weight-operand stages (dequantised, or router weights by TMA)
+constexpr int SB = 4;          // gathered token-operand stages (copies signal their own arrival)
 constexpr int SC = 3;          // code stages
 constexpr int kThreads = 512;
 constexpr int kDqThreads = 256;           // dequantisation threads (warps 4-11)
