@@ -58,6 +58,15 @@ WORKLOADS = {
 METRIC = "W4A16 MoE-layer tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of the current kernel (profiles/decode_gate_up_int4_T4_ncu.md and
+# profiles/prefill_gate_up_int4_T8192_ncu.md); workloads without a capture of
+# their dominant kernel report null.
+MEASURED_TRAFFIC = {
+    ("decode4", "gate_up"): 32.475904e6,
+    ("prefill", "gate_up"): 375.163392e6 + 57.828864e6,
+}
+
 
 # ---------------------------------------------------------------- distributed plumbing
 
@@ -384,14 +393,16 @@ def run_ours(args, rank, local, world):
     if decode:
         achieved = work[dom]["bytes"] / (stage_avg[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if args.path == "auto" else None,
                 "peak_kind": f"{peak_kind} STREAM-copy HBM bandwidth",
                 "algorithmic_bytes_per_launch": work[dom]["bytes"], "avg_launch_ms": stage_avg[dom]}
     else:
         achieved = work[dom]["flops"] / (stage_avg[dom] / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak,
+                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if args.path == "auto" else None,
                 "peak_kind": f"{peak_kind} sustained cuBLAS bf16 GEMM",
                 "algorithmic_flops_per_launch": work[dom]["flops"], "avg_launch_ms": stage_avg[dom]}
 
