@@ -45,9 +45,12 @@ struct UnitHeader {
   int tok[kHdrTokens];  // token of sorted row p0 + i (i < min(n_e, 32))
 };
 
-template <int FMT, int NT>
+// With X_SMEM (small T), the producer warp first stages the T token rows of x
+// into shared memory (one bulk copy per row, padded row stride), and the
+// compute warps read their activation fragments from there.
+template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
-    const uint16_t* __restrict__ x, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
+    const uint16_t* __restrict__ x, int T, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act,
     uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -58,6 +61,9 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
   float* red = reinterpret_cast<float*>(hdr + kGuStages);  // [warp][tile][4][lane]
   uint64_t* full = reinterpret_cast<uint64_t*>(red + kGuWarps * NT * 4 * 32);
   uint64_t* empty = full + kGuStages;
+  uint64_t* x_bar = empty + kGuStages;
+  uint8_t* x_s = reinterpret_cast<uint8_t*>(x_bar + 2);  // [T][staged_row_stride(K)]
+  const int xstride = staged_row_stride(K);
   __shared__ int s_units;
   __shared__ volatile int s_abort;  // raised by the first wait that gives up
 
@@ -72,6 +78,7 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
       mbar_init(&full[st], 1);
       mbar_init(&empty[st], kGuWarps);
     }
+    if (X_SMEM) mbar_init(x_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -80,6 +87,11 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
 
   if (warp == kGuWarps) {
     // ---------------------------------------------------------------- producer
+    if (X_SMEM) {
+      if (lane == 0) mbar_arrive_expect_tx(x_bar, uint32_t(T) * uint32_t(2 * K));
+      __syncwarp();
+      stage_act_rows(x_s, x, T, K, x_bar);
+    }
     int i = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
       const int st = i % kGuStages;
@@ -112,10 +124,11 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
   // -------------------------------------------------------------------- compute
   const int g = lane >> 2, q = lane & 3;
   const int nblk = (K + 127) / 128;
+  const bool x_ok = !X_SMEM || mbar_wait(x_bar, 0, &s_abort, status);
   int i = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
     const int st = i % kGuStages;
-    const bool ok = mbar_wait(&full[st], (i / kGuStages) & 1, &s_abort, status);
+    const bool ok = mbar_wait(&full[st], (i / kGuStages) & 1, &s_abort, status) && x_ok;
     const uint8_t* s_c = smem + st * L.stage_bytes;
     const uint8_t* s_s = s_c + L.cbytes;
     const UnitHeader& h = hdr[st];
@@ -128,14 +141,13 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
       for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
-      const uint16_t* xrow[NT];
+      int xtok[NT];
       bool xval[NT];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         const int c = (nt0 + j) * 8 + g;
         xval[j] = c < n_e;
-        const int tok = !xval[j] ? 0 : (c < kHdrTokens ? h.tok[c] : sorted_rows[p0 + c] / top_k);
-        xrow[j] = x + size_t(tok) * K;
+        xtok[j] = !xval[j] ? 0 : (c < kHdrTokens ? h.tok[c] : sorted_rows[p0 + c] / top_k);
       }
       if (ok) {
         for (int b = warp; b < nblk; b += kGuWarps) {
@@ -146,7 +158,8 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
             uint32_t bf[8][2];
-            load_act_frags(xrow[j], K, kb, q, xval[j], bf);
+            if (X_SMEM) load_act_frags_smem(smem_u32(x_s) + uint32_t(xtok[j] * xstride), K, kb, q, xval[j], bf);
+            else load_act_frags(x + size_t(xtok[j]) * K, K, kb, q, xval[j], bf);
             mma_block<FMT>(acc[j], gate, up, bf);
           }
         }
@@ -214,7 +227,11 @@ MOE_DEV void issue_down_rows(const Bank& dn, int e, int f0, uint8_t* stage, cons
   stage_rows<FMT>(dn, long(e) * dn.N + f0, kDecRows, stage, stage + L.cbytes, bar);
 }
 
-template <int FMT, int NT>
+// With ACT_SMEM (T <= kDnTokens and the rows fit), one warp first stages all
+// T*k activation rows into shared memory with one bulk copy per row, so the
+// fragment loads of the expert loop read shared memory instead of waiting on
+// L2 once per k-block.
+template <int FMT, int NT, bool ACT_SMEM>
 __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
     Bank dn, int T, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
     const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ sorted_rows,
@@ -224,10 +241,15 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
   const UnitLayout L = unit_layout(FMT, K, kDecRows, 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
+  const int tchunk = min(T, kDnTokens);  // tokens per pass
   uint8_t* ring = smem + warp * kDnStages * L.stage_bytes;
   float* accs = reinterpret_cast<float*>(smem + kDnWarps * kDnStages * L.stage_bytes);  // [warp][token][16]
-  float* acc_w = accs + warp * kDnTokens * kDecRows;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(accs + kDnWarps * kDnTokens * kDecRows) + warp * kDnStages;
+  float* acc_w = accs + warp * tchunk * kDecRows;
+  uint64_t* all_bars = reinterpret_cast<uint64_t*>(accs + kDnWarps * tchunk * kDecRows);
+  uint64_t* bars = all_bars + warp * kDnStages;
+  uint64_t* act_bar = all_bars + kDnWarps * kDnStages;
+  uint8_t* act_s = reinterpret_cast<uint8_t*>(act_bar + 2);  // [T*k][staged_row_stride(K)]
+  const int astride = staged_row_stride(K);
 
   __shared__ volatile int s_abort;
   pdl_wait();
@@ -235,16 +257,25 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
   const int f0 = blockIdx.x * kDecRows;
   const int n_touched = touched[0];
   const int nblk = (K + 127) / 128;
-  if (threadIdx.x == 0) s_abort = 0;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    if (ACT_SMEM) mbar_init(act_bar, 1);
+  }
   if (lane == 0) {
     for (int st = 0; st < kDnStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
   __syncthreads();
+  if (ACT_SMEM && warp == 0) {
+    const int R = T * top_k;
+    if (lane == 0) mbar_arrive_expect_tx(act_bar, uint32_t(R) * uint32_t(2 * K));
+    __syncwarp();
+    stage_act_rows(act_s, act, R, K, act_bar);
+  }
   int uses = 0;  // ring slots consumed so far by this warp (over all chunks)
   for (int t0 = 0; t0 < T; t0 += kDnTokens) {
     const int t1 = min(T, t0 + kDnTokens);
-    for (int i = lane; i < kDnTokens * kDecRows; i += 32) acc_w[i] = 0.f;
+    for (int i = lane; i < tchunk * kDecRows; i += 32) acc_w[i] = 0.f;
     // prologue: first experts of this warp into the ring
     if (lane == 0) {
       for (int st = 0; st < kDnStages; ++st) {
@@ -257,6 +288,8 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
       }
     }
     __syncwarp();
+    // the staged activation rows (one chunk: T <= kDnTokens)
+    const bool act_ok = !ACT_SMEM || n_touched <= warp || mbar_wait(act_bar, 0, &s_abort, status);
     for (int slot = warp, n = 0; slot < n_touched; slot += kDnWarps, ++n) {
       const int st = (uses + n) % kDnStages;
       const uint32_t parity = ((uses + n) / kDnStages) & 1;
@@ -271,7 +304,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
         p0 = chunk_bound(sorted_rows, p0, pe, top_k, t0);
       }
       const int n_e = pe - p0;
-      const bool ok = mbar_wait(&bars[st], parity, &s_abort, status);
+      const bool ok = mbar_wait(&bars[st], parity, &s_abort, status) && act_ok;
       const int ntiles = (n_e + 7) / 8;
       for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
         // routing of the next 32 rows: lane l holds row nt0*8 + l
@@ -296,8 +329,10 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
             const int col = (nt0 + j) * 8 + g;
+            const int prow = p0 + (col < n_e ? col : 0);
             uint32_t bf[8][2];
-            load_act_frags(act + size_t(p0 + (col < n_e ? col : 0)) * K, K, kb, q, col < n_e, bf);
+            if (ACT_SMEM) load_act_frags_smem(smem_u32(act_s) + uint32_t(prow * astride), K, kb, q, col < n_e, bf);
+            else load_act_frags(act + size_t(prow) * K, K, kb, q, col < n_e, bf);
             mma_block<FMT>(acc[j], c0, c1, bf);
           }
         }
@@ -333,11 +368,15 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
     for (int idx = threadIdx.x; idx < (t1 - t0) * kDecRows; idx += blockDim.x) {
       float sum = 0.f;
 #pragma unroll 4
-      for (int w = 0; w < kDnWarps; ++w) sum += accs[w * kDnTokens * kDecRows + idx];
+      for (int w = 0; w < kDnWarps; ++w) sum += accs[w * tchunk * kDecRows + idx];
       const int t = t0 + idx / kDecRows, f = f0 + idx % kDecRows;
       out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
     }
     __syncthreads();
+  }
+  if (ACT_SMEM && warp == 0 && n_touched <= 0) {
+    // nothing waited on the staged rows: let the copies land before exiting
+    mbar_wait_drain(act_bar, 0, kWaitLimitNs);
   }
 }
 
@@ -349,17 +388,27 @@ size_t unit_stage_bytes(int fmt, int K, int rows, int mats) {
   return size_t(mats) * (cbytes + ((sbytes + 15) & ~15));
 }
 
-// stages + unit headers + the cross-warp reduction buffer + barriers
-size_t gate_up_smem(int fmt, int K, int nt) {
+// stages + unit headers + the cross-warp reduction buffer + barriers + the
+// token rows' barrier (16 bytes) and, with x_rows > 0, those rows
+size_t gate_up_smem(int fmt, int K, int nt, int x_rows) {
   return kGuStages * unit_stage_bytes(fmt, K, kDecRows, 1) + kGuStages * sizeof(UnitHeader) +
-         size_t(kGuWarps) * nt * 4 * 32 * 4 + 2 * kGuStages * 8;
+         size_t(kGuWarps) * nt * 4 * 32 * 4 + 2 * kGuStages * 8 + 16 + size_t(x_rows) * staged_row_stride(K);
 }
 
-// per-warp rings + per-warp accumulators + per-warp barriers
-size_t down_smem(int fmt, int K) {
+// Token rows staged in shared memory by the gate_up kernel up to this many
+// bytes: 4 rows of hidden 2048 keep four CTAs resident per SM.
+constexpr size_t kGuMaxStagedX = 4 * (2 * 2048 + 16);
+
+// per-warp rings + per-warp accumulators + per-warp barriers + the staged
+// activation rows' barrier (16 bytes) and, with act_rows > 0, those rows
+size_t down_smem(int fmt, int K, int T, int act_rows) {
+  const int tchunk = std::min(T, kDnTokens);
   return size_t(kDnWarps) * kDnStages * unit_stage_bytes(fmt, K, kDecRows, 1) +
-         size_t(kDnWarps) * kDnTokens * kDecRows * 4 + size_t(kDnWarps) * kDnStages * 8;
+         size_t(kDnWarps) * tchunk * kDecRows * 4 + size_t(kDnWarps) * kDnStages * 8 + 16 +
+         size_t(act_rows) * staged_row_stride(K);
 }
+
+constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving room for static
 
 int sm_count_cached() {
   static int n = 0;
@@ -373,16 +422,29 @@ int sm_count_cached() {
 }
 
 // Persistent grid: as many CTAs as fit on the GPU at once (at most `units`).
-// (computed once per kernel instantiation and shared-memory size)
+// The occupancy of each (kernel, shared-memory size) is computed once and kept
+// in a small table (instantiations of one template share a function type, so
+// the kernel's address is part of the key).
 template <typename Kern>
 int persistent_grid(Kern k, size_t smem, int units, int threads) {
-  static size_t cached_smem = 0;
-  static int per_sm = 0;
-  if (per_sm == 0 || cached_smem != smem) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 1) n = 1;
-    per_sm = n;
-    cached_smem = smem;
+  struct Entry {
+    const void* fn;
+    size_t smem;
+    int per_sm;
+  };
+  static Entry cache[16] = {};
+  const void* fn = reinterpret_cast<const void*>(k);
+  int per_sm = 0;
+  for (const Entry& e : cache)
+    if (e.fn == fn && e.smem == smem) per_sm = e.per_sm;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    for (Entry& e : cache)
+      if (e.fn == nullptr) {
+        e = Entry{fn, smem, per_sm};
+        break;
+      }
   }
   return std::max(1, std::min(units, per_sm * sm_count_cached()));
 }
@@ -398,14 +460,15 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 namespace {
 
 template <int FMT, int NT>
-cudaError_t gate_up_nt(const moe_shape_t& s, const uint16_t* x, const Bank& gu, const Workspace& ws, int units,
-                       cudaStream_t stream) {
-  auto k = decode_gate_up_kernel<FMT, NT>;
-  const size_t smem = gate_up_smem(FMT, s.hidden, NT);
+cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws,
+                       int units, cudaStream_t stream) {
+  const bool x_smem = size_t(T) * staged_row_stride(s.hidden) <= kGuMaxStagedX;
+  auto k = x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
+  const size_t smem = gate_up_smem(FMT, s.hidden, NT, x_smem ? T : 0);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(k, smem, units, kGuThreads);
-  return launch_pdl(k, dim3(grid), dim3(kGuThreads), smem, stream, x, gu, s.inter, s.top_k,
+  return launch_pdl(k, dim3(grid), dim3(kGuThreads), smem, stream, x, T, gu, s.inter, s.top_k,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows, ws.act,
                     ws.status);
 }
@@ -414,16 +477,19 @@ template <int FMT>
 cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws,
                         int units, cudaStream_t stream) {
   // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
-  if (T <= 8) return gate_up_nt<FMT, 1>(s, x, gu, ws, units, stream);
-  if (T <= 16) return gate_up_nt<FMT, 2>(s, x, gu, ws, units, stream);
-  return gate_up_nt<FMT, kDecNT>(s, x, gu, ws, units, stream);
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, ws, units, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, ws, units, stream);
+  return gate_up_nt<FMT, kDecNT>(s, T, x, gu, ws, units, stream);
 }
 
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
                     cudaStream_t stream) {
-  auto k = decode_down_kernel<FMT, NT>;
-  const size_t smem = down_smem(FMT, s.inter);
+  // stage all T*k activation rows in shared memory when they fit
+  const int R = T * s.top_k;
+  const bool act_smem = T <= kDnTokens && down_smem(FMT, s.inter, T, R) <= kMaxSmemPerCta;
+  auto k = act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
+  const size_t smem = down_smem(FMT, s.inter, T, act_smem ? R : 0);
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
   return launch_pdl(k, dim3(s.hidden / kDecRows), dim3(kDnWarps * 32), smem, stream, dn, T, s.top_k,

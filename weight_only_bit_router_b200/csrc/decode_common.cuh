@@ -102,6 +102,53 @@ MOE_DEV void load_act_frags(const uint16_t* rowp, int K, int kb, int q, bool val
   }
 }
 
+// Raw words X[m] = (v[32q+2m], v[32q+2m+1]) -> the permuted fragment pairs of
+// the 8 MMA steps (see the fragment k-permutation above).
+MOE_DEV void act_frags_from_raw(const uint32_t (&X)[16], uint32_t (&b)[8][2]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    b[2 * j][0] = prmt(X[4 * j], X[4 * j + 2], 0x5410u);
+    b[2 * j][1] = prmt(X[4 * j], X[4 * j + 2], 0x7632u);
+    b[2 * j + 1][0] = prmt(X[4 * j + 1], X[4 * j + 3], 0x5410u);
+    b[2 * j + 1][1] = prmt(X[4 * j + 1], X[4 * j + 3], 0x7632u);
+  }
+}
+
+// Activation fragments of one 128-k block for one token row held in shared
+// memory (`rowp` is the row's shared-memory address); same layout and
+// permutation as load_act_frags.
+MOE_DEV void load_act_frags_smem(uint32_t rowp, int K, int kb, int q, bool valid, uint32_t (&b)[8][2]) {
+  uint32_t X[16];
+  const int k = kb + 32 * q;
+  if (valid && k < K) {
+    const uint32_t a = rowp + uint32_t(k) * 2u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(X[4 * i]), "=r"(X[4 * i + 1]), "=r"(X[4 * i + 2]), "=r"(X[4 * i + 3])
+                   : "r"(a + 16u * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) X[i] = 0;
+  }
+  act_frags_from_raw(X, b);
+}
+
+// Row stride of bf16 activation rows of length K staged in shared memory:
+// 16 bytes of padding shift consecutive rows by four banks, so the eight rows
+// of an MMA fragment load do not all start in the same bank.
+__host__ __device__ inline int staged_row_stride(int K) { return 2 * K + 16; }
+
+// Start one bulk copy per bf16 row of length K (rows [lane, lane+32, ...) <
+// `rows`) from global `src` into shared memory at `dst` with the padded row
+// stride, all completing on `bar`.  Called by every lane of one warp after
+// lane 0 announced rows * 2K bytes on `bar`.
+MOE_DEV void stage_act_rows(uint8_t* dst, const uint16_t* src, int rows, int K, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  const int stride = staged_row_stride(K);
+  for (int r = lane; r < rows; r += 32) bulk_g2s(dst + size_t(r) * stride, src + size_t(r) * K, uint32_t(2 * K), bar);
+}
+
 // The 16 raw activation words of one 128-k block for the lane's k-slice,
 // read through L2 (ld.global.cg): for data that other CTAs of the same grid
 // wrote.  Rows past K, or an invalid row, read as zeros.
@@ -117,18 +164,6 @@ MOE_DEV void load_act_raw_cg(const uint16_t* rowp, int K, int kb, int q, bool va
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) X[i] = 0;
-  }
-}
-
-// Raw words X[m] = (v[32q+2m], v[32q+2m+1]) -> the permuted fragment pairs of
-// the 8 MMA steps (see the fragment k-permutation above).
-MOE_DEV void act_frags_from_raw(const uint32_t (&X)[16], uint32_t (&b)[8][2]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    b[2 * j][0] = prmt(X[4 * j], X[4 * j + 2], 0x5410u);
-    b[2 * j][1] = prmt(X[4 * j], X[4 * j + 2], 0x7632u);
-    b[2 * j + 1][0] = prmt(X[4 * j + 1], X[4 * j + 3], 0x5410u);
-    b[2 * j + 1][1] = prmt(X[4 * j + 1], X[4 * j + 3], 0x7632u);
   }
 }
 

@@ -476,6 +476,76 @@ __device__ void block_permutation_256(RouteFastSmem& sm, int R, int E, int32_t* 
   }
 }
 
+// Stable counting sort of R <= 32 rows by expert (E <= 256) by one warp, with
+// no block barrier: the same results as block_permutation_256 (offsets,
+// sorted rows and their inverse, the touched-expert list and the token-block
+// prefix).  Lane r ranks row r among the rows of its expert with
+// __match_any_sync; the per-expert counts go through shared memory, where
+// lane l owns experts [8l, 8l + 8) for the scan.
+__device__ void warp_permutation_32(RouteFastSmem& sm, int R, int E, int32_t* __restrict__ offsets,
+                                    int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
+                                    int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n) {
+  const int lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) sm.off[8 * lane + u] = 0;
+  __syncwarp();
+  const int r = lane;
+  int e = r < R ? sm.ids[r] : -1;
+  if (e < 0 || e >= E) e = -1;
+  const unsigned mm = __match_any_sync(full, e);
+  const int before = __popc(mm & ((1u << lane) - 1u));
+  if (e >= 0 && before == 0) sm.off[e] = __popc(mm);
+  __syncwarp();
+  int c[8], cs = 0, nz = 0, bl = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    c[u] = sm.off[8 * lane + u];
+    cs += c[u];
+    nz += c[u] > 0;
+    bl += (c[u] + block_n - 1) / block_n;
+  }
+  int ci = cs, ni = nz, bi = bl;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a0 = __shfl_up_sync(full, ci, o), a1 = __shfl_up_sync(full, ni, o), a2 = __shfl_up_sync(full, bi, o);
+    if (lane >= o) {
+      ci += a0;
+      ni += a1;
+      bi += a2;
+    }
+  }
+  int run = ci - cs, tp = ni - nz, brun = bi - bl;
+  __syncwarp();  // every lane has read its counts before they become offsets
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int x = 8 * lane + u;
+    if (x < E) {
+      sm.off[x] = run;
+      offsets[x] = run;
+      tile_base[x] = brun;
+      if (c[u] > 0) touched[1 + tp++] = x;
+    }
+    run += c[u];
+    brun += (c[u] + block_n - 1) / block_n;
+  }
+  if (lane == 31) {
+    offsets[E] = ci;
+    tile_base[E] = bi;
+    touched[0] = ni;
+  }
+  __syncwarp();
+  if (r < R) {
+    if (e < 0) {
+      pos[r] = -1;
+    } else {
+      const int p = sm.off[e] + before;
+      sorted_rows[p] = r;
+      pos[r] = p;
+    }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
@@ -563,7 +633,11 @@ __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
   __syncthreads();
   const int R = T * k;
   for (int r = threadIdx.x; r < R; r += blockDim.x) ids[r] = sm.ids[r];
-  block_permutation_256(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  if (R <= 32) {
+    if (warp == 0) warp_permutation_32(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  } else {
+    block_permutation_256(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
+  }
   if (threadIdx.x == 0) *done_counter = 0;  // ready for the next call
 }
 
