@@ -138,6 +138,41 @@ MOE_API moe_status_t moe_pack_int4_g128(const uint16_t* w, int E, int N, int K, 
 MOE_API moe_status_t moe_pack_mxfp4(const uint16_t* w, int E, int N, int K, void* packed,
                             int32_t* nonfinite_count, cudaStream_t stream);
 
+/* Exponent rules of the MXFP4 packer (all members of the floor(log2(x / 6))
+ * family of "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Quantization
+ * method), per block of 32 with amax = max |w| (amax == 0 always gives
+ * e = -127 and zero codes; every e is clamped to [-127, 127]):
+ *   MOE_MX_EXP_FLOOR  e = floor(log2(amax / 6)): largest e with 6 * 2^e <=
+ *                     amax (the block max may clip to 6 * 2^e); this is what
+ *                     moe_pack_mxfp4 uses.
+ *   MOE_MX_EXP_CEIL   e = ceil(log2(amax / 6)): smallest e with amax <=
+ *                     6 * 2^e (nothing clips; the card's "smallest exponent
+ *                     that avoids clipping").
+ *   MOE_MX_EXP_OCP    e = floor(log2(amax)) - 2 (2 = largest E2M1 exponent).
+ *   MOE_MX_EXP_MSE    the card's scale search: candidates e0 - 4 ... e0 + 1
+ *                     with e0 = floor(log2(p / 6)), p the block's 99.5th
+ *                     percentile of |w| (v30 + 0.845 * (v31 - v30) of the
+ *                     sorted magnitudes, fp64, multiply rounded before the
+ *                     add), plus the CEIL exponent; the candidate with the
+ *                     smallest sum of squared reconstruction errors wins (fp64,
+ *                     squares of exact differences summed pairwise: element i
+ *                     with i + 16, then i + 8, i + 4, i + 2, i + 1), ties to
+ *                     the smaller exponent. */
+typedef enum {
+  MOE_MX_EXP_FLOOR = 0,
+  MOE_MX_EXP_CEIL = 1,
+  MOE_MX_EXP_OCP = 2,
+  MOE_MX_EXP_MSE = 3
+} moe_mx_exp_rule_t;
+
+/* moe_pack_mxfp4 with the given exponent rule (codes are always the nearest
+ * E2M1 magnitude of |w| / 2^e, ties to the even code, saturating at 6).  The
+ * packed layout is the same for every rule, so moe_forward consumes any of
+ * them.  Same arguments and errors as moe_pack_int4_g128, plus
+ * MOE_ERR_INVALID_ARG for an unknown rule. */
+MOE_API moe_status_t moe_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed,
+                                 int32_t* nonfinite_count, moe_mx_exp_rule_t rule, cudaStream_t stream);
+
 /* Expand a packed bank back to bf16 w_out [E, N, K] (device):
  * INT4 w = bf16_rne(q * s); MXFP4 w = e2m1(c) * 2^e (exact).  Debug and test
  * entry; the forward pass dequantises inside its GEMMs instead. */

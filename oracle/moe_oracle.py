@@ -157,17 +157,21 @@ def dequant_int4_g128(codes, scales) -> np.ndarray:
 # MXFP4: E2M1 codes, E8M0 scale per 32 elements                      [MXFP4]
 # --------------------------------------------------------------------------
 
+def floor_log2_div6(x) -> np.ndarray:
+    """Largest integer e with 6 * 2^e <= x, for x > 0 (no clamping)."""
+    x = np.asarray(x, dtype=np.float64)
+    e = np.floor(np.log2(x / 6.0)).astype(np.int64)
+    # fix up the fp64 log2 estimate with exact power-of-two comparisons
+    e = np.where(6.0 * np.ldexp(1.0, e + 1) <= x, e + 1, e)
+    return np.where(6.0 * np.ldexp(1.0, e) > x, e - 1, e)
+
+
 def mx_exponent(amax) -> np.ndarray:
     """Largest integer e with 6 * 2^e <= amax (= floor(log2(amax/6))), clamped
     to [-127, 127]; -127 for amax == 0."""
     amax = np.asarray(amax, dtype=np.float64)
     pos = amax > 0
-    safe = np.where(pos, amax, 6.0)
-    e = np.floor(np.log2(safe / 6.0)).astype(np.int64)
-    # fix up the fp64 log2 estimate with exact power-of-two comparisons
-    e = np.where(6.0 * np.ldexp(1.0, e + 1) <= safe, e + 1, e)
-    e = np.where(6.0 * np.ldexp(1.0, e) > safe, e - 1, e)
-    e = np.clip(e, -127, 127)
+    e = np.clip(floor_log2_div6(np.where(pos, amax, 6.0)), -127, 127)
     return np.where(pos, e, -127)
 
 
@@ -184,8 +188,88 @@ def e2m1_nearest(v) -> np.ndarray:
     return pick.astype(np.uint8)
 
 
-def pack_mxfp4(w_bits):
-    """Quantise a bf16 bank [..., N, K] in blocks of 32 along K.
+# Exponent rules of the MXFP4 packer.  FLOOR is the one above; the others are
+# the members of the same family that the MxWave card compares against or
+# searches over ("kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Quantization
+# method: the "smallest exponent that avoids clipping", and the MSE search).
+MX_RULE_FLOOR = "floor"   # largest e with 6 * 2^e <= amax (block max may clip)
+MX_RULE_CEIL = "ceil"     # smallest e with amax <= 6 * 2^e (nothing clips)
+MX_RULE_OCP = "ocp"       # floor(log2(amax)) - 2: the OCP MX shared-exponent rule for E2M1
+MX_RULE_MSE = "mse"       # MxWave: lowest-MSE exponent among the candidates below
+MX_P995_FRACTION = 0.845  # 99.5th percentile of 32 values: index 0.995 * 31 = 30.845
+
+
+def mx_exponent_ceil(amax) -> np.ndarray:
+    """Smallest integer e with amax <= 6 * 2^e (= ceil(log2(amax/6))), clamped
+    to [-127, 127]; -127 for amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    pos = amax > 0
+    safe = np.where(pos, amax, 6.0)
+    e = np.ceil(np.log2(safe / 6.0)).astype(np.int64)
+    e = np.where(6.0 * np.ldexp(1.0, e - 1) >= safe, e - 1, e)
+    e = np.where(6.0 * np.ldexp(1.0, e) < safe, e + 1, e)
+    e = np.clip(e, -127, 127)
+    return np.where(pos, e, -127)
+
+
+def mx_exponent_ocp(amax) -> np.ndarray:
+    """floor(log2(amax)) - 2 (2 = the largest exponent of an E2M1 value), clamped
+    to [-127, 127]; -127 for amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    pos = amax > 0
+    _, ex = np.frexp(np.where(pos, amax, 1.0))            # amax = m * 2^ex, 0.5 <= m < 1
+    e = np.clip(ex.astype(np.int64) - 1 - 2, -127, 127)
+    return np.where(pos, e, -127)
+
+
+def mx_p995(mag_blocks) -> np.ndarray:
+    """99.5th percentile of each block's 32 magnitudes, linear interpolation
+    between order statistics: v30 + 0.845 * (v31 - v30) of the sorted values,
+    in fp64 with the multiply rounded before the add."""
+    v = np.sort(np.asarray(mag_blocks, dtype=np.float64), axis=-1)
+    v30, v31 = v[..., 30], v[..., 31]
+    return v30 + (v31 - v30) * MX_P995_FRACTION
+
+
+def mx_block_sq_error(blocks, e) -> np.ndarray:
+    """Squared reconstruction error of each block quantised with exponent e
+    (array over blocks), summed over the 32 elements pairwise in halving order
+    (element i with i + 16, then with i + 8, ...), in fp64."""
+    v = blocks / np.ldexp(1.0, e)[..., None]
+    mag = e2m1_nearest(v)
+    w_hat = np.where(blocks < 0, -1.0, 1.0) * E2M1_GRID[mag] * np.ldexp(1.0, e)[..., None]
+    sq = (blocks - w_hat) * (blocks - w_hat)                 # both exact in fp64
+    n = sq.shape[-1]
+    while n > 1:
+        n //= 2
+        sq = sq[..., :n] + sq[..., n:2 * n]
+    return sq[..., 0]
+
+
+def mx_exponent_mse(blocks) -> np.ndarray:
+    """MxWave's scale search per block of 32: the candidates are
+    floor(log2(p995 / 6)) - 4 ... + 1 and the smallest exponent that avoids
+    clipping, each clamped to [-127, 127]; the one with the lowest squared
+    error wins, ties to the smaller exponent.  An all-zero block gets -127."""
+    blocks = np.asarray(blocks, dtype=np.float64)
+    mags = np.abs(blocks)
+    amax = np.max(mags, axis=-1)
+    p = mx_p995(mags)
+    e0 = floor_log2_div6(np.where(amax > 0, p, 6.0))      # largest e with 6 * 2^e <= p995
+    cands = [np.clip(e0 + d, -127, 127) for d in range(-4, 2)] + [mx_exponent_ceil(amax)]
+    best_e = cands[0]
+    best_err = mx_block_sq_error(blocks, best_e)
+    for c in cands[1:]:                                    # ascending exponents
+        err = mx_block_sq_error(blocks, c)
+        better = err < best_err
+        best_e = np.where(better, c, best_e)
+        best_err = np.where(better, err, best_err)
+    return np.where(amax > 0, best_e, -127)
+
+
+def pack_mxfp4(w_bits, rule: str = MX_RULE_FLOOR):
+    """Quantise a bf16 bank [..., N, K] in blocks of 32 along K with the given
+    exponent rule.
 
     Returns (codes uint8 [..., N, K/2], scales uint8 E8M0 [..., N, K/32]).
     """
@@ -195,7 +279,16 @@ def pack_mxfp4(w_bits):
     w = bf16_to_f64(w_bits)
     blocks = w.reshape(w.shape[:-1] + (K // MX_BLOCK, MX_BLOCK))
     amax = np.max(np.abs(blocks), axis=-1)
-    e = mx_exponent(amax)
+    if rule == MX_RULE_FLOOR:
+        e = mx_exponent(amax)
+    elif rule == MX_RULE_CEIL:
+        e = mx_exponent_ceil(amax)
+    elif rule == MX_RULE_OCP:
+        e = mx_exponent_ocp(amax)
+    elif rule == MX_RULE_MSE:
+        e = mx_exponent_mse(blocks)
+    else:
+        raise ValueError(f"unknown MXFP4 exponent rule {rule!r}")
     v = blocks / np.ldexp(1.0, e)[..., None]              # exact power-of-two scaling
     mag = e2m1_nearest(v)
     sign = ((blocks < 0) & (mag > 0)).astype(np.uint8)

@@ -57,6 +57,8 @@ _SIGS = {
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_pack_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_pack_mxfp4_rule": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "moe_dequant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_void_p, ctypes.c_void_p]),
     "moe_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -189,6 +191,20 @@ def moe_pack_int4_g128(w, packed=None, nonfinite=None, stream=None):
 
 def moe_pack_mxfp4(w, packed=None, nonfinite=None, stream=None):
     return _pack("moe_pack_mxfp4", MOE_FMT_MXFP4_G32, w, packed, nonfinite, stream)
+
+
+MX_EXP_RULES = {"floor": 0, "ceil": 1, "ocp": 2, "mse": 3}
+
+
+def moe_pack_mxfp4_rule(w, rule, packed=None, nonfinite=None, stream=None):
+    """MXFP4 packing with an exponent rule: "floor" | "ceil" | "ocp" | "mse" (or its enum value)."""
+    E, N, K = w.shape
+    if packed is None:
+        packed = torch.empty(moe_bank_bytes(MOE_FMT_MXFP4_G32, E, N, K), dtype=torch.uint8, device=w.device)
+    _check("moe_pack_mxfp4_rule",
+           lib().moe_pack_mxfp4_rule(_ptr(_bits(w)), E, N, K, _ptr(packed), _ptr(nonfinite),
+                                     MX_EXP_RULES.get(rule, rule), _stream(stream)))
+    return packed
 
 
 def moe_dequant(packed, fmt, E, N, K, out=None, stream=None):

@@ -263,6 +263,16 @@ moe_status_t moe_pack_mxfp4(const uint16_t* w, int E, int N, int K, void* packed
   return pack_common(MOE_FMT_MXFP4_G32, w, E, N, K, packed, nonfinite, stream);
 }
 
+moe_status_t moe_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                                 moe_mx_exp_rule_t rule, cudaStream_t stream) {
+  if (rule != MOE_MX_EXP_FLOOR && rule != MOE_MX_EXP_CEIL && rule != MOE_MX_EXP_OCP && rule != MOE_MX_EXP_MSE)
+    return MOE_ERR_INVALID_ARG;
+  if (!w || !packed) return MOE_ERR_INVALID_ARG;
+  if (E <= 0 || N <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(packed, 256) || (nonfinite && !aligned(nonfinite, 4))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_pack_mxfp4_rule(w, E, N, K, packed, nonfinite, int(rule), stream));
+}
+
 moe_status_t moe_dequant(const void* packed, moe_format_t fmt, int E, int N, int K, uint16_t* w_out,
                          cudaStream_t stream) {
   if (!packed || !w_out || !valid_fmt(fmt)) return MOE_ERR_INVALID_ARG;

@@ -49,7 +49,7 @@ struct UnitHeader {
 // into shared memory (one bulk copy per row, padded row stride), and the
 // compute warps read their activation fragments from there.
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kGuThreads, NT == 1 ? 4 : 1) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int top_k, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act,
     uint32_t* status) {
@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
   const int g = lane >> 2, q = lane & 3;
   const int nblk = (K + 127) / 128;
   const bool x_ok = !X_SMEM || mbar_wait(x_bar, 0, &s_abort, status);
+  const int srow = scale_row_bytes(FMT, K);
+  const int nb_q = lane_kblocks(K, q);
   int i = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
     const int st = i % kGuStages;
@@ -150,16 +152,21 @@ __global__ void __launch_bounds__(kGuThreads) decode_gate_up_kernel(
         xtok[j] = !xval[j] ? 0 : (c < kHdrTokens ? h.tok[c] : sorted_rows[p0 + c] / top_k);
       }
       if (ok) {
+        // the lane's rows g (gate) and g + 8 (up) at its k-slice, and their scales
+        const uint8_t* c_gate = s_c + g * (K / 2) + 16 * q;
+        const uint8_t* c_up = c_gate + 8 * (K / 2);
+        const uint8_t* sc_gate = s_s + g * srow;
+        const uint8_t* sc_up = sc_gate + 8 * srow;
         for (int b = warp; b < nblk; b += kGuWarps) {
-          const int kb = b * 128;
-          const RowChunk gate = smem_row_chunk<FMT>(s_c, s_s, g, K, kb, q);
-          const RowChunk up = smem_row_chunk<FMT>(s_c, s_s, g + 8, K, kb, q);
+          const bool in = b < nb_q;
+          const RowChunk gate = row_chunk_at<FMT>(c_gate, sc_gate, b, q, in);
+          const RowChunk up = row_chunk_at<FMT>(c_up, sc_up, b, q, in);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
             uint32_t bf[8][2];
-            if (X_SMEM) load_act_frags_smem(smem_u32(x_s) + uint32_t(xtok[j] * xstride), K, kb, q, xval[j], bf);
-            else load_act_frags(x + size_t(xtok[j]) * K, K, kb, q, xval[j], bf);
+            if (X_SMEM) load_act_frags_smem(x_s + xtok[j] * xstride + 256 * b + 64 * q, in && xval[j], bf);
+            else load_act_frags(x + size_t(xtok[j]) * K, K, b * 128, q, xval[j], bf);
             mma_block<FMT>(acc[j], gate, up, bf);
           }
         }
@@ -242,6 +249,8 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const int tchunk = min(T, kDnTokens);  // tokens per pass
+  const int srow = scale_row_bytes(FMT, K);
+  const int nb_q = lane_kblocks(K, q);
   uint8_t* ring = smem + warp * kDnStages * L.stage_bytes;
   float* accs = reinterpret_cast<float*>(smem + kDnWarps * kDnStages * L.stage_bytes);  // [warp][token][16]
   float* acc_w = accs + warp * tchunk * kDecRows;
@@ -321,18 +330,22 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
         for (int j = 0; j < NT; ++j)
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
+        const uint8_t* c_lo = s_c + g * (K / 2) + 16 * q;
+        const uint8_t* c_hi = c_lo + 8 * (K / 2);
+        const uint8_t* sc_lo = s_s + g * srow;
+        const uint8_t* sc_hi = sc_lo + 8 * srow;
         for (int b = 0; b < nblk; ++b) {
-          const int kb = b * 128;
-          const RowChunk c0 = smem_row_chunk<FMT>(s_c, s_s, g, K, kb, q);
-          const RowChunk c1 = smem_row_chunk<FMT>(s_c, s_s, g + 8, K, kb, q);
+          const bool in = b < nb_q;
+          const RowChunk c0 = row_chunk_at<FMT>(c_lo, sc_lo, b, q, in);
+          const RowChunk c1 = row_chunk_at<FMT>(c_hi, sc_hi, b, q, in);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
             const int col = (nt0 + j) * 8 + g;
             const int prow = p0 + (col < n_e ? col : 0);
             uint32_t bf[8][2];
-            if (ACT_SMEM) load_act_frags_smem(smem_u32(act_s) + uint32_t(prow * astride), K, kb, q, col < n_e, bf);
-            else load_act_frags(act + size_t(prow) * K, K, kb, q, col < n_e, bf);
+            if (ACT_SMEM) load_act_frags_smem(act_s + prow * astride + 256 * b + 64 * q, in && col < n_e, bf);
+            else load_act_frags(act + size_t(prow) * K, K, b * 128, q, col < n_e, bf);
             mma_block<FMT>(acc[j], c0, c1, bf);
           }
         }

@@ -21,7 +21,8 @@ constexpr int kDecRows = 16;       // weight rows (features) per warp tile
 constexpr int kDecNT = 4;          // token tiles of 8 held in registers at once
 
 MOE_DEV void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  // not volatile: a pure function of its registers, free to be scheduled
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -115,24 +116,50 @@ MOE_DEV void act_frags_from_raw(const uint32_t (&X)[16], uint32_t (&b)[8][2]) {
 }
 
 // Activation fragments of one 128-k block for one token row held in shared
-// memory (`rowp` is the row's shared-memory address); same layout and
-// permutation as load_act_frags.
-MOE_DEV void load_act_frags_smem(uint32_t rowp, int K, int kb, int q, bool valid, uint32_t (&b)[8][2]) {
+// memory: `p` points at the lane's 64-byte k-slice (row + 2 * (kb + 32q));
+// same layout and permutation as load_act_frags.  Plain loads, so that the
+// compiler orders them after the barrier waits that make the data visible.
+MOE_DEV void load_act_frags_smem(const uint8_t* p, bool valid, uint32_t (&b)[8][2]) {
   uint32_t X[16];
-  const int k = kb + 32 * q;
-  if (valid && k < K) {
-    const uint32_t a = rowp + uint32_t(k) * 2u;
+  if (valid) {
+    const uint4* v = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(X[4 * i]), "=r"(X[4 * i + 1]), "=r"(X[4 * i + 2]), "=r"(X[4 * i + 3])
-                   : "r"(a + 16u * i));
+    for (int i = 0; i < 4; ++i) {
+      const uint4 w = v[i];
+      X[4 * i] = w.x; X[4 * i + 1] = w.y; X[4 * i + 2] = w.z; X[4 * i + 3] = w.w;
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) X[i] = 0;
   }
   act_frags_from_raw(X, b);
 }
+
+// A lane's 16 code bytes and multiplier of k-block b of one staged weight
+// row: `codes` points at the row's codes plus the lane's slice offset 16q,
+// `scales` at the row's scales; `in` is false for a slice past K (zero
+// weights).
+template <int FMT>
+MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b, int q, bool in) {
+  RowChunk rc;
+  if (in) {
+    rc.codes = *reinterpret_cast<const uint4*>(codes + 64 * b);
+    if (FMT == MOE_FMT_INT4_G128) {
+      const uint32_t sc = reinterpret_cast<const uint16_t*>(scales)[b];  // group b = k-block b
+      rc.mult = sc | (sc << 16);
+    } else {
+      rc.mult = pow2_bf16x2(int(scales[4 * b + q]) - 127);  // the slice is one 32-element block
+    }
+  } else {
+    rc.codes = make_uint4(0, 0, 0, 0);
+    rc.mult = 0;
+  }
+  return rc;
+}
+
+// Number of 128-k blocks in which lane slice q (k in [kb + 32q, kb + 32q + 32))
+// lies inside K (K a multiple of 32).
+MOE_DEV int lane_kblocks(int K, int q) { return (K - 32 * q + 127) >> 7; }
 
 // Row stride of bf16 activation rows of length K staged in shared memory:
 // 16 bytes of padding shift consecutive rows by four banks, so the eight rows

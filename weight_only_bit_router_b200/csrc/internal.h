@@ -66,6 +66,9 @@ size_t permute_block_rows();
 // pack.cu
 cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K, void* packed,
                         int32_t* nonfinite, cudaStream_t stream);
+// MXFP4 packing with an exponent rule (moe_mx_exp_rule_t as int)
+cudaError_t launch_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                                   int rule, cudaStream_t stream);
 cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, int K, uint16_t* out,
                            cudaStream_t stream);
 

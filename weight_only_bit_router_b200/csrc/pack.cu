@@ -127,6 +127,122 @@ __global__ void __launch_bounds__(256) pack_mxfp4_kernel(const uint16_t* __restr
   if ((lane & 7) == 0) scales[row * (K / 32) + col / 32] = uint8_t(e + 127);
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4 with a selectable exponent rule (the floor(log2(x / 6)) family of
+// "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Quantization method).  One
+// warp per block of 32; lane i owns element i.  The MSE rule evaluates its
+// candidates in fp64 with explicitly rounded operations (no contraction), so
+// that its integer decision is reproducible.
+// ---------------------------------------------------------------------------
+
+// ceil(log2(amax / 6)) for amax > 0: amax = m * 2^E, m in [1, 2);
+// 6 * 2^(E-2) = 1.5 * 2^E >= amax iff m <= 1.5, else 6 * 2^(E-1) >= amax.
+__device__ __forceinline__ int mx_exponent_ceil(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int bias = 0;
+  if (amax < 1e-30f) { amax *= 18446744073709551616.0f; bias = 64; }  // 2^64, exact
+  const uint32_t b = __float_as_uint(amax);
+  const int E = int((b >> 23) & 0xFF) - 127 - bias;
+  const int e = ((b & 0x7FFFFF) <= 0x400000u) ? E - 2 : E - 1;
+  return max(-127, min(127, e));
+}
+
+// floor(log2(amax)) - 2 for amax > 0.
+__device__ __forceinline__ int mx_exponent_ocp(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int bias = 0;
+  if (amax < 1e-30f) { amax *= 18446744073709551616.0f; bias = 64; }
+  const int E = int((__float_as_uint(amax) >> 23) & 0xFF) - 127 - bias;
+  return max(-127, min(127, E - 2));
+}
+
+// Largest e with 6 * 2^e <= p for a normal fp64 p > 0: p = m * 2^E, m in
+// [1, 2); 6 * 2^(E-2) <= p iff m >= 1.5.
+__device__ __forceinline__ int mx_exponent_f64(double p) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(p));
+  const int E = int((b >> 52) & 0x7FF) - 1023;
+  return (b & (1ull << 51)) ? E - 2 : E - 3;
+}
+
+__device__ __forceinline__ double exp2i_f64(int p) {  // 2^p, p in [-1022, 1023]
+  return __longlong_as_double(static_cast<long long>(p + 1023) << 52);
+}
+
+// E2M1 magnitude code of a non-negative fp64 a (same thresholds as e2m1_code).
+__device__ __forceinline__ uint32_t e2m1_code_f64(double a) {
+  if (a <= 0.25) return 0;
+  if (a < 0.75) return 1;
+  if (a <= 1.25) return 2;
+  if (a < 1.75) return 3;
+  if (a <= 2.5) return 4;
+  if (a < 3.5) return 5;
+  if (a <= 5.0) return 6;
+  return 7;
+}
+
+__constant__ double kE2m1Grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+// Sum over the warp of the squared error of quantising this lane's w with
+// exponent e; pairwise in halving order, identical in every lane.
+__device__ __forceinline__ double mx_block_sq_error(double w, int e) {
+  const double a = fabs(w) * exp2i_f64(-e);  // exact power-of-two scaling
+  const double mag = kE2m1Grid[e2m1_code_f64(a)] * exp2i_f64(e);
+  const double d = __dsub_rn(w, w < 0.0 ? -mag : mag);  // exact
+  double sq = __dmul_rn(d, d);                          // exact
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq = __dadd_rn(sq, __shfl_xor_sync(0xffffffffu, sq, o));
+  return sq;
+}
+
+__global__ void __launch_bounds__(256) pack_mxfp4_rule_kernel(const uint16_t* __restrict__ w, long nblocks,
+                                                              uint8_t* __restrict__ codes,
+                                                              uint8_t* __restrict__ scales, int32_t* nonfinite,
+                                                              int rule) {
+  const unsigned full = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const long blk = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (blk >= nblocks) return;
+  const float v = bf16_to_f32(w[blk * 32 + lane]);
+  if (!isfinite(v) && nonfinite) atomicAdd(nonfinite, 1);
+  const float a = fabsf(v);
+  // magnitudes are non-negative: their fp32 bit patterns order like the values
+  const float amax = __uint_as_float(__reduce_max_sync(full, __float_as_uint(a)));
+  int e;
+  if (!(amax > 0.f)) {
+    e = -127;
+  } else if (rule == MOE_MX_EXP_CEIL) {
+    e = mx_exponent_ceil(amax);
+  } else if (rule == MOE_MX_EXP_OCP) {
+    e = mx_exponent_ocp(amax);
+  } else if (rule == MOE_MX_EXP_MSE) {
+    // 99.5th percentile of the 32 magnitudes: v30 + 0.845 * (v31 - v30)
+    const int n_max = __popc(__ballot_sync(full, a == amax));
+    const float v30 = n_max >= 2 ? amax
+                                 : __uint_as_float(__reduce_max_sync(full, a == amax ? 0u : __float_as_uint(a)));
+    const double p = __dadd_rn(double(v30), __dmul_rn(__dsub_rn(double(amax), double(v30)), 0.845));
+    const int e0 = mx_exponent_f64(p);
+    const double wv = double(v);
+    e = max(-127, min(127, e0 - 4));
+    double best = mx_block_sq_error(wv, e);
+    for (int d = -3; d <= 2; ++d) {  // e0 - 3 ... e0 + 1, then the no-clip exponent
+      const int c = d <= 1 ? max(-127, min(127, e0 + d)) : mx_exponent_ceil(amax);
+      const double err = mx_block_sq_error(wv, c);
+      if (err < best) {
+        best = err;
+        e = c;
+      }
+    }
+  } else {
+    e = mx_exponent(amax);
+  }
+  const float x = v * exp2i(-e);  // exact whenever it matters (|x| >= 2^-126)
+  const uint32_t c = e2m1_code(fabsf(x));
+  const uint32_t nib = ((v < 0.f && c != 0) ? 8u : 0u) | c;
+  const uint32_t hi = __shfl_down_sync(full, nib, 1);
+  if ((lane & 1) == 0) codes[blk * 16 + lane / 2] = uint8_t(nib | (hi << 4));
+  if (lane == 0) scales[blk] = uint8_t(e + 127);
+}
+
 // Debug dequantiser: one thread per code byte (two elements).
 __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales, int fmt,
                                long rows, int K, uint16_t* __restrict__ out) {
@@ -174,6 +290,19 @@ cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K
   else
     pack_mxfp4_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, rows, K, codes, static_cast<uint8_t*>(scales),
                                                                   nonfinite);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                                   int rule, cudaStream_t stream) {
+  if (rule == MOE_MX_EXP_FLOOR) return launch_pack(MOE_FMT_MXFP4_G32, w, E, N, K, packed, nonfinite, stream);
+  const long nblocks = long(E) * N * (K / 32);
+  if (nblocks == 0) return cudaSuccess;
+  const int block = 256;
+  const long grid = (nblocks * 32 + block - 1) / block;
+  uint8_t* codes = static_cast<uint8_t*>(packed);
+  uint8_t* scales = codes + bank_scale_offset(MOE_FMT_MXFP4_G32, E, N, K);
+  pack_mxfp4_rule_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, nblocks, codes, scales, nonfinite, rule);
   return cudaGetLastError();
 }
 
