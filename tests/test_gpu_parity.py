@@ -248,6 +248,15 @@ def test_forward_odd_shapes_and_partial_tiles():
             check_layer(layer, fmt, path)
 
 
+def test_forward_odd_shapes_small_batch():
+    """H = 320, I = 192 at 5 tokens: a k-block of the gate_up rows ends
+    part-way and four rows of scales are not a whole number of 16-byte units."""
+    shape = moe_synth.LayerShape(hidden=320, inter=192, num_experts=6, top_k=3)
+    layer = moe_synth.make_layer(shape, T=5, seed=78, device=DEV)
+    for fmt in FMTS:
+        check_layer(layer, fmt, moe.MOE_PATH_DECODE)
+
+
 @pytest.mark.parametrize("T", [1, 4])
 def test_forward_nex_decode_int4(T):
     layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=100 + T, device=DEV)
