@@ -56,6 +56,10 @@ E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
 
 FMT_INT4 = "int4_g128"
 FMT_MXFP4 = "mxfp4"
+FMT_NVFP4 = "nvfp4"
+NV_BLOCK = 16
+E4M3_MAX = 448.0
+NV_GLOBAL_DIVISOR = 6.0 * E4M3_MAX   # largest E2M1 magnitude x largest E4M3 value
 
 
 # --------------------------------------------------------------------------
@@ -314,12 +318,103 @@ def dequant_mxfp4(codes, scales) -> np.ndarray:
     return full
 
 
+# --------------------------------------------------------------------------
+# NVFP4 as W4A16: E2M1 codes, E4M3 scale per 16 elements, one fp32 global
+# scale per expert matrix                                              [NVFP4]
+# ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", What's quantized to what:
+# NVFP4 experts with group 16; gate and up share one weight_global_scale per
+# expert; weights-only round-to-nearest, no calibration)
+# --------------------------------------------------------------------------
+
+def e4m3_value(code) -> np.ndarray:
+    """Value of an E4M3 (fn) byte without its sign bit: 4 exponent bits (bias 7),
+    3 mantissa bits, subnormals m * 2^-9."""
+    c = np.asarray(code, dtype=np.int64) & 0x7F
+    e, m = c >> 3, c & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+
+
+_E4M3_CODES = np.arange(0x7F)                      # 0x7F is NaN in E4M3fn: never produced
+_E4M3_VALUES = e4m3_value(_E4M3_CODES)             # increasing
+
+
+def e4m3_nearest(t) -> np.ndarray:
+    """Code of the E4M3 value nearest t >= 0, ties to the even code (mantissa
+    bit 0), saturating at 448."""
+    t = np.asarray(t, dtype=np.float64)
+    d = np.abs(t[..., None] - _E4M3_VALUES)
+    best = d == d.min(axis=-1, keepdims=True)
+    even_best = best & (_E4M3_CODES % 2 == 0)
+    pick = np.where(even_best.any(axis=-1), np.argmax(even_best, axis=-1), np.argmax(best, axis=-1))
+    return pick.astype(np.uint8)
+
+
+def nv_global_scale(w_bits) -> np.ndarray:
+    """Per matrix (leading dims kept): g = fp32(amax / 2688), so that the block
+    with the matrix's largest magnitude gets the E4M3 scale 448."""
+    w = bf16_to_f64(w_bits).astype(np.float32)
+    amax = np.max(np.abs(w.reshape(w.shape[:-2] + (-1,))), axis=-1)
+    return (amax / np.float32(NV_GLOBAL_DIVISOR)).astype(np.float32)
+
+
+def nv_multiplier(scale_codes, g) -> np.ndarray:
+    """Per block: bf16(fp32(e4m3(code) * g)), the bf16 multiplier of the block's
+    E2M1 codes, as fp64."""
+    v = e4m3_value(scale_codes).astype(np.float32)
+    prod = (v * np.asarray(g, dtype=np.float32)[..., None, None]).astype(np.float32)
+    return bf16_round(prod.astype(np.float64))
+
+
+def pack_nvfp4(w_bits):
+    """Quantise a bf16 bank [E, N, K] (or one matrix [N, K]) to NVFP4:
+    g = fp32(amax / 2688) per matrix; per block of 16 along K the scale code
+    e4m3_nearest(fp32(amax_b / fp32(6 g))); the block multiplier
+    d = bf16(fp32(e4m3(code) g)); codes = nearest E2M1 magnitude of
+    fp32(w / d) (ties to the even code, saturating at 6), sign bit set only
+    for nonzero codes; all zero when d == 0.
+
+    Returns (codes uint8 [..., N, K/2], (scales uint8 [..., N, K/16], g fp32 [...])).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    K = w_bits.shape[-1]
+    assert K % NV_BLOCK == 0
+    w32 = bf16_to_f64(w_bits).astype(np.float32)
+    g = nv_global_scale(w_bits)
+    blocks = w32.reshape(w32.shape[:-1] + (K // NV_BLOCK, NV_BLOCK))
+    amax_b = np.max(np.abs(blocks), axis=-1)
+    six_g = (np.float32(6.0) * g).astype(np.float32)[..., None, None]
+    safe = np.where(six_g == 0, np.float32(1.0), six_g)
+    t = np.where(six_g == 0, np.float32(0.0), (amax_b / safe).astype(np.float32))
+    scales = e4m3_nearest(t.astype(np.float64))
+    d = nv_multiplier(scales, g)                                   # fp64, bf16 values
+    d32 = d.astype(np.float32)[..., None]
+    quot = np.where(d32 == 0, np.float32(0.0), blocks / np.where(d32 == 0, np.float32(1.0), d32))
+    mag = np.where(d32 == 0, 0, e2m1_nearest(quot.astype(np.float32).astype(np.float64))).astype(np.uint8)
+    sign = ((blocks < 0) & (mag > 0)).astype(np.uint8)
+    nib = ((sign << np.uint8(3)) | mag).reshape(w32.shape).astype(np.uint8)
+    codes = (nib[..., 0::2] | (nib[..., 1::2] << np.uint8(4))).astype(np.uint8)
+    return codes, (scales, g)
+
+
+def dequant_nvfp4(codes, scales_g) -> np.ndarray:
+    """w_hat = bf16(e2m1(c) * d), d the block's bf16 multiplier (one rounding of
+    an exact product), as fp64."""
+    scales, g = scales_g
+    vals = e2m1_value(unpack_nibbles(codes))
+    d = nv_multiplier(scales, g)
+    return bf16_round(vals * np.repeat(d, NV_BLOCK, axis=-1))
+
+
 def pack(fmt: str, w_bits):
-    return pack_int4_g128(w_bits) if fmt == FMT_INT4 else pack_mxfp4(w_bits)
+    if fmt == FMT_INT4:
+        return pack_int4_g128(w_bits)
+    return pack_mxfp4(w_bits) if fmt == FMT_MXFP4 else pack_nvfp4(w_bits)
 
 
 def dequant(fmt: str, codes, scales):
-    return dequant_int4_g128(codes, scales) if fmt == FMT_INT4 else dequant_mxfp4(codes, scales)
+    if fmt == FMT_INT4:
+        return dequant_int4_g128(codes, scales)
+    return dequant_mxfp4(codes, scales) if fmt == FMT_MXFP4 else dequant_nvfp4(codes, scales)
 
 
 def packed_bytes_per_expert(fmt: str, hidden: int, inter: int) -> int:
@@ -327,6 +422,8 @@ def packed_bytes_per_expert(fmt: str, hidden: int, inter: int) -> int:
     def mat(N, K):
         if fmt == FMT_INT4:
             return N * K // 2 + N * len(int4_groups(K)) * 2
+        if fmt == FMT_NVFP4:
+            return N * K // 2 + N * (K // NV_BLOCK) + 4
         return N * K // 2 + N * (K // MX_BLOCK)
     return mat(2 * inter, hidden) + mat(hidden, inter)
 
@@ -393,7 +490,11 @@ class PackedBank:
 
     def expert(self, e: int) -> np.ndarray:
         if e not in self._cache:
-            self._cache[e] = dequant(self.fmt, self.codes[e], self.scales[e])
+            if isinstance(self.scales, dict) or self.fmt != FMT_NVFP4:
+                sc = self.scales[e]                             # per-expert entries
+            else:
+                sc = (self.scales[0][e], self.scales[1][e])     # (block scales, global scales)
+            self._cache[e] = dequant(self.fmt, self.codes[e], sc)
         return self._cache[e]
 
 
