@@ -12,6 +12,7 @@ intermediate 512; synthetic seeded inputs, random-init weights):
   prefill   INT4, 8192 tokens, one step = one layer (rotating over 40 layers)
   prefill_zipf  the same with the Zipf logit bias
   mx_decode4 / mx_prefill   the MXFP4 stack (17.1 GB packed) at 4 / 8192 tokens
+  nv_decode4 / nv_prefill   the NVFP4 stack (E4M3 scale per 16 elements) at 4 / 8192 tokens
 
 The metric is MoE-layer tokens per second: tokens x layers processed per
 second of device time, whole job (all ranks).  With --gpus N > 1 (launched by
@@ -54,6 +55,8 @@ WORKLOADS = {
     "prefill_zipf": ("int4_g128", 8192, True, 1),
     "mx_decode4": ("mxfp4", 4, False, NUM_LAYERS),
     "mx_prefill": ("mxfp4", 8192, False, 1),
+    "nv_decode4": ("nvfp4", 4, False, NUM_LAYERS),
+    "nv_prefill": ("nvfp4", 8192, False, 1),
 }
 METRIC = "W4A16 MoE-layer tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -171,7 +174,7 @@ class Stack:
         self.router = torch.empty(layers, s.num_experts, s.hidden, dtype=torch.bfloat16, device=device)
         self.bias = [moe_synth.zipf_bias(s, moe_synth.SEED_STACK_BASE + l).to(device) if zipf else None
                      for l in range(layers)]
-        pack = moe.moe_pack_int4_g128 if fmt == "int4_g128" else moe.moe_pack_mxfp4
+        pack = {"int4_g128": moe.moe_pack_int4_g128, "mxfp4": moe.moe_pack_mxfp4, "nvfp4": moe.moe_pack_nvfp4}[fmt]
         for l in range(layers):
             seed = moe_synth.SEED_STACK_BASE + l
             w = moe_synth.gate_up_bank(s, seed, device)
@@ -261,7 +264,7 @@ def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, 
     (layer-tokens per second, description, threads)."""
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
-    fmt = o.FMT_INT4 if stack.fmt == "int4_g128" else o.FMT_MXFP4
+    fmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[stack.fmt]
     E, k = stack.shape.num_experts, stack.shape.top_k
     done_tokens, elapsed, used_layers = 0.0, 0.0, 0
     xb_all = moe_synth.bf16_bits(x_bf16)
@@ -477,7 +480,7 @@ def run_reference(args, rank, world):
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
     fmt_name, T, zipf, _ = WORKLOADS[args.workload]
-    fmt = o.FMT_INT4 if fmt_name == "int4_g128" else o.FMT_MXFP4
+    fmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[fmt_name]
     s = moe_synth.NEX
     n_layers = 2
     prepared = []

@@ -69,7 +69,8 @@ typedef enum {
 
 typedef enum {
   MOE_FMT_INT4_G128 = 1,     /* INT4 symmetric RTN, bf16 scale per 128 elements along K */
-  MOE_FMT_MXFP4_G32 = 2      /* MXFP4: E2M1 codes, E8M0 scale per 32 elements along K */
+  MOE_FMT_MXFP4_G32 = 2,     /* MXFP4: E2M1 codes, E8M0 scale per 32 elements along K */
+  MOE_FMT_NVFP4_G16 = 3      /* NVFP4: E2M1 codes, E4M3 scale per 16 elements along K, fp32 scale per matrix */
 } moe_format_t;
 
 /* Layer shape.  Supported: hidden and inter multiples of 64 (>= 64),
@@ -96,10 +97,16 @@ MOE_API int moe_abi_version(void);
  *                               low nibble of byte j, element 2j+1 in the high
  *                               nibble.  INT4: offset binary q + 8 (q in
  *                               [-8, 7]).  MXFP4: sign<<3 | E2M1 magnitude code.
- *   bytes [scale_offset, total) scales.  INT4: bf16 [E][N][ceil(K/128)] (the
+ *                               NVFP4: the same E2M1 nibbles as MXFP4.
+ *   bytes [scale_offset, ...)   scales.  INT4: bf16 [E][N][ceil(K/128)] (the
  *                               last group of a row holds K mod 128 elements).
  *                               MXFP4: E8M0 uint8 [E][N][K/32], byte = e + 127.
- * scale_offset is E*N*K/2 rounded up to 256 bytes.
+ *                               NVFP4: E4M3 uint8 [E][N][K/16].
+ *   NVFP4 only: fp32 [E] global scales (one per matrix; for a gate_up bank the
+ *                               gate and up halves of an expert share it) at
+ *                               scale_offset + E*N*K/16 rounded up to 256 bytes.
+ * scale_offset is E*N*K/2 rounded up to 256 bytes; the total is what
+ * moe_bank_bytes returns.
  * ---------------------------------------------------------------------- */
 
 /* Total bytes of a packed bank of E matrices [N, K]; 0 if the arguments are invalid. */
@@ -173,8 +180,29 @@ typedef enum {
 MOE_API moe_status_t moe_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed,
                                  int32_t* nonfinite_count, moe_mx_exp_rule_t rule, cudaStream_t stream);
 
+/* Quantise a bf16 bank w [E, N, K] to NVFP4 with bf16 block multipliers
+ * (W4A16) ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", What's quantized to
+ * what: NVFP4 experts with group 16, one weight_global_scale per expert shared
+ * by gate and up, weights-only round-to-nearest).  Per matrix e (all N rows,
+ * the gate and up halves of a gate_up bank together):
+ *   g    = fp32(amax_e / 2688)            (2688 = 6 * 448: the largest E2M1
+ *                                          times the largest E4M3 value)
+ * per block of 16 consecutive K elements of a row:
+ *   code = E4M3 nearest to fp32(amax_b / fp32(6 g)), ties to even, saturating
+ *          at 448
+ *   d    = bf16_rne(fp32(e4m3(code) * g)) the block's multiplier
+ *   c    = nearest E2M1 magnitude of fp32(w / d) (ties to the even code,
+ *          saturating at 6), sign bit only for nonzero codes; 0 when d == 0
+ * and the forward pass dequantises w = bf16_rne(e2m1(c) * d).  K must be a
+ * positive multiple of 32.  The call enqueues four kernels (matrix maxima,
+ * global scales, codes); otherwise arguments and errors as
+ * moe_pack_int4_g128. */
+MOE_API moe_status_t moe_pack_nvfp4(const uint16_t* w, int E, int N, int K, void* packed,
+                            int32_t* nonfinite_count, cudaStream_t stream);
+
 /* Expand a packed bank back to bf16 w_out [E, N, K] (device):
- * INT4 w = bf16_rne(q * s); MXFP4 w = e2m1(c) * 2^e (exact).  Debug and test
+ * INT4 w = bf16_rne(q * s); MXFP4 w = e2m1(c) * 2^e (exact); NVFP4
+ * w = bf16_rne(e2m1(c) * d).  Debug and test
  * entry; the forward pass dequantises inside its GEMMs instead. */
 MOE_API moe_status_t moe_dequant(const void* packed, moe_format_t fmt, int E, int N, int K,
                          uint16_t* w_out, cudaStream_t stream);

@@ -8,7 +8,7 @@ import torch
 import moe_synth
 from oracle import moe_oracle as o
 
-FMT_NAMES = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4}
+FMT_NAMES = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}
 
 
 class LazyOracleBank:

@@ -38,13 +38,15 @@ def test_status_strings():
     assert "timeout" in moe.moe_status_str(5) or "expired" in moe.moe_status_str(5)
 
 
-@pytest.mark.parametrize("fmt", ["int4_g128", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4_g128", "mxfp4", "nvfp4"])
 def test_bank_sizes_match_closed_form(fmt):
     s = moe.make_shape(2048, 512, 256, 8, fmt)
     gu, dn = moe.moe_packed_bytes(s, 0), moe.moe_packed_bytes(s, 1)
-    per_expert = o.packed_bytes_per_expert(o.FMT_INT4 if fmt == "int4_g128" else o.FMT_MXFP4, 2048, 512)
-    # two 256-byte alignment pads at most (codes -> scales, per bank)
-    assert 0 <= gu + dn - 256 * per_expert < 2 * 256
+    ofmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[fmt]
+    per_expert = o.packed_bytes_per_expert(ofmt, 2048, 512)
+    # 256-byte alignment pads (codes -> scales, and for NVFP4 scales -> global scales, per bank)
+    pads = 4 if fmt == "nvfp4" else 2
+    assert 0 <= gu + dn - 256 * per_expert < pads * 256
     assert moe.moe_packed_bytes(s, 2) == 0
     assert moe.moe_bank_scale_offset(fmt, 256, 1024, 2048) == 256 * 1024 * 1024
 
@@ -100,7 +102,7 @@ def test_forward_validation_happens_on_the_host():
     assert L.moe_forward(*args(wsb=ws - 1)) == 3
     assert L.moe_forward(*args(T=-2)) == 1
     assert L.moe_forward(*args(shape=moe.make_shape(2048, 500, 256, 8, "int4_g128"))) == 2
-    assert L.moe_forward(*args(shape=moe.make_shape(2048, 512, 256, 8, 3))) == 1
+    assert L.moe_forward(*args(shape=moe.make_shape(2048, 512, 256, 8, 4))) == 1   # unknown format
     assert L.moe_forward(*args(r=None)) == 1
     opts = moe.ForwardOpts()
     opts.path = 9

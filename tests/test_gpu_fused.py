@@ -9,7 +9,9 @@ import torch
 
 import moe_synth
 import weight_only_bit_router_b200 as moe
-from test_gpu_parity import DEV, FMTS, check_layer, pack_gpu, run_forward
+from test_gpu_parity import DEV, check_layer, pack_gpu, run_forward
+
+FMTS = ["int4_g128", "mxfp4"]  # NVFP4 banks run on the three-kernel decode path
 
 pytestmark = pytest.mark.gpu
 
@@ -28,6 +30,13 @@ def test_single_kernel_path_launch_counts():
         assert moe.moe_forward_launch_count(s, T, FUSED, 0) == 1
         assert moe.moe_forward_launch_count(s, T, FUSED, 1) == 1
     assert moe.moe_forward_launch_count(s, 9, FUSED, 0) == -1   # above the path's token limit
+    assert moe.moe_forward_launch_count(moe.make_shape(2048, 512, 256, 8, "nvfp4"), 4, FUSED, 0) == -1
+
+
+def test_single_kernel_path_rejects_nvfp4():
+    layer = moe_synth.make_layer(moe_synth.TINY, T=4, seed=3, device=DEV)
+    with pytest.raises(moe.MoeError):
+        run_forward(layer, "nvfp4", FUSED)
 
 
 @pytest.mark.parametrize("fmt", FMTS)

@@ -16,18 +16,27 @@ from parity_util import (FMT_NAMES, LazyOracleBank, assert_out_close, assert_rou
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-FMTS = ["int4_g128", "mxfp4"]
+FMTS = ["int4_g128", "mxfp4", "nvfp4"]
+PACKERS = {"int4_g128": moe.moe_pack_int4_g128, "mxfp4": moe.moe_pack_mxfp4, "nvfp4": moe.moe_pack_nvfp4}
 
 
 def pack_gpu(fmt, w):
-    return moe.moe_pack_int4_g128(w) if fmt == "int4_g128" else moe.moe_pack_mxfp4(w)
+    return PACKERS[fmt](w)
 
 
 def gpu_split(fmt, packed, E, N, K):
     codes, scales = moe.split_bank(packed, fmt, E, N, K)
     c = codes.cpu().numpy()
+    if fmt == "nvfp4":
+        return c, (scales[0].cpu().numpy(), scales[1].cpu().numpy())
     s = scales.cpu().numpy()
     return c, (s.view(np.uint16) if fmt == "int4_g128" else s)
+
+
+def scales_equal(fmt, a, b):
+    if fmt == "nvfp4":
+        return np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), np.asarray(b[1], np.float32).view(np.uint32))
+    return np.array_equal(a, b)
 
 
 # ---------------------------------------------------------------- packing
@@ -63,7 +72,7 @@ def test_pack_bit_exact_tiny_and_edges(fmt):
         gc, gs = gpu_split(fmt, packed, E, N, K)
         rc, rs = o.pack(FMT_NAMES[fmt], moe_synth.bf16_bits(w))
         assert np.array_equal(gc, rc)
-        assert np.array_equal(gs, rs)
+        assert scales_equal(fmt, gs, rs)
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -88,8 +97,12 @@ def test_pack_bit_exact_full_layer_sampled_experts(fmt):
     for e in (0, 131, 255):
         rc, rs = o.pack(FMT_NAMES[fmt], moe_synth.bf16_bits(gu[e]))
         assert np.array_equal(codes[e].cpu().numpy(), rc)
-        s = scales[e].cpu().numpy()
-        assert np.array_equal(s.view(np.uint16) if fmt == "int4_g128" else s, rs)
+        if fmt == "nvfp4":
+            s = (scales[0][e].cpu().numpy(), scales[1][e:e + 1].cpu().numpy()[0])
+        else:
+            s = scales[e].cpu().numpy()
+            s = s.view(np.uint16) if fmt == "int4_g128" else s
+        assert scales_equal(fmt, s, rs)
 
 
 def test_pack_counts_nonfinite_inputs():
@@ -99,7 +112,8 @@ def test_pack_counts_nonfinite_inputs():
     cnt = torch.zeros(1, dtype=torch.int32, device=DEV)
     moe.moe_pack_int4_g128(w, nonfinite=cnt)
     moe.moe_pack_mxfp4(w, nonfinite=cnt)
-    assert int(cnt.item()) == 4
+    moe.moe_pack_nvfp4(w, nonfinite=cnt)
+    assert int(cnt.item()) == 6
 
 
 # ---------------------------------------------------------------- routing
@@ -281,6 +295,13 @@ def test_forward_nex_mxfp4(T):
     layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=4000 + T, device=DEV)
     sample = None if T <= 32 else np.random.default_rng(6).choice(T, 24, replace=False)
     check_layer(layer, "mxfp4", sample=sample)
+
+
+@pytest.mark.parametrize("T", [4, 8192])
+def test_forward_nex_nvfp4(T):
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=5000 + T, device=DEV)
+    sample = None if T <= 32 else np.random.default_rng(7).choice(T, 24, replace=False)
+    check_layer(layer, "nvfp4", sample=sample)
 
 
 def test_decode_and_grouped_paths_on_one_nex_layer():

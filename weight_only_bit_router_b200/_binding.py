@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 
 MOE_FMT_INT4_G128 = 1
 MOE_FMT_MXFP4_G32 = 2
-FORMATS = {"int4_g128": MOE_FMT_INT4_G128, "mxfp4": MOE_FMT_MXFP4_G32}
+MOE_FMT_NVFP4_G16 = 3
+FORMATS = {"int4_g128": MOE_FMT_INT4_G128, "mxfp4": MOE_FMT_MXFP4_G32, "nvfp4": MOE_FMT_NVFP4_G16}
 
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_FUSED = 0, 1, 2, 3
 MOE_NUM_STAGES = 5
@@ -56,6 +57,8 @@ _SIGS = {
     "moe_pack_int4_g128": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_pack_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_pack_nvfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_pack_mxfp4_rule": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
@@ -193,6 +196,10 @@ def moe_pack_mxfp4(w, packed=None, nonfinite=None, stream=None):
     return _pack("moe_pack_mxfp4", MOE_FMT_MXFP4_G32, w, packed, nonfinite, stream)
 
 
+def moe_pack_nvfp4(w, packed=None, nonfinite=None, stream=None):
+    return _pack("moe_pack_nvfp4", MOE_FMT_NVFP4_G16, w, packed, nonfinite, stream)
+
+
 MX_EXP_RULES = {"floor": 0, "ceil": 1, "ocp": 2, "mse": 3}
 
 
@@ -224,6 +231,11 @@ def split_bank(packed, fmt, E, N, K):
     if fmt == MOE_FMT_INT4_G128:
         G = (K + 127) // 128
         scales = packed[off:off + E * N * G * 2].view(torch.int16).view(E, N, G)
+    elif fmt == MOE_FMT_NVFP4_G16:
+        # (E4M3 block scales [E, N, K/16], fp32 global scales [E])
+        nsc = E * N * (K // 16)
+        goff = (off + nsc + 255) // 256 * 256
+        scales = (packed[off:off + nsc].view(E, N, K // 16), packed[goff:goff + 4 * E].view(torch.float32))
     else:
         scales = packed[off:off + E * N * (K // 32)].view(E, N, K // 32)
     return codes, scales

@@ -11,7 +11,9 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool valid_fmt(moe_format_t f) { return f == MOE_FMT_INT4_G128 || f == MOE_FMT_MXFP4_G32; }
+bool valid_fmt(moe_format_t f) {
+  return f == MOE_FMT_INT4_G128 || f == MOE_FMT_MXFP4_G32 || f == MOE_FMT_NVFP4_G16;
+}
 
 moe_status_t check_shape(const moe_shape_t* s) {
   if (!s) return MOE_ERR_INVALID_ARG;
@@ -41,6 +43,9 @@ Bank make_bank(const void* packed, moe_format_t fmt, int E, int N, int K) {
   Bank b;
   b.codes = static_cast<const uint8_t*>(packed);
   b.scales = static_cast<const uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
+  b.gscale = fmt == MOE_FMT_NVFP4_G16
+                 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(packed) + bank_gscale_offset(fmt, E, N, K))
+                 : nullptr;
   b.N = N;
   b.K = K;
   return b;
@@ -230,7 +235,7 @@ int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 size_t moe_bank_bytes(moe_format_t fmt, int E, int N, int K) {
   if (!valid_fmt(fmt) || E <= 0 || N <= 0 || K <= 0 || K % 32) return 0;
-  return bank_scale_offset(fmt, E, N, K) + bank_scale_bytes(fmt, E, N, K);
+  return bank_total_bytes(fmt, E, N, K);
 }
 
 size_t moe_bank_scale_offset(moe_format_t fmt, int E, int N, int K) {
@@ -261,6 +266,11 @@ moe_status_t moe_pack_int4_g128(const uint16_t* w, int E, int N, int K, void* pa
 moe_status_t moe_pack_mxfp4(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
                             cudaStream_t stream) {
   return pack_common(MOE_FMT_MXFP4_G32, w, E, N, K, packed, nonfinite, stream);
+}
+
+moe_status_t moe_pack_nvfp4(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,
+                            cudaStream_t stream) {
+  return pack_common(MOE_FMT_NVFP4_G16, w, E, N, K, packed, nonfinite, stream);
 }
 
 moe_status_t moe_pack_mxfp4_rule(const uint16_t* w, int E, int N, int K, void* packed, int32_t* nonfinite,

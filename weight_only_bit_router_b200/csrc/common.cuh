@@ -76,6 +76,18 @@ MOE_DEV uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// E4M3 (fn) scale byte, sign bit ignored -> its fp32 value (exact): 4
+// exponent bits with bias 7, 3 mantissa bits, subnormals m * 2^-9.
+MOE_DEV float e4m3_to_f32(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : float(m) * 0.001953125f;
+}
+
+// NVFP4 block multiplier as bf16 bits: bf16_rne(fp32(e4m3(byte) * g)).
+MOE_DEV uint32_t nv_mult_bits(uint32_t scale_byte, float g) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e4m3_to_f32(scale_byte), g)));
+}
+
 // E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the
 // nibble pair at bit offsets 0 and 16 of `w` after shifting by 4*i.
 // Magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; looked up with two byte permutes.

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kGuThreads, NT == 1 ? 4 : 1) decode_gate_up_ke
     const uint8_t* s_s = s_c + L.cbytes;
     const UnitHeader& h = hdr[st];
     const int p0 = h.p0, n_e = h.n_e;
+    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[h.e] : 0.f;
     const int f0 = (u % ftiles) * kGuFeatures;
     const int ntiles = (n_e + 7) / 8;
     for (int nt0 = 0; nt0 < ntiles; nt0 += NT) {
@@ -159,8 +160,8 @@ __global__ void __launch_bounds__(kGuThreads, NT == 1 ? 4 : 1) decode_gate_up_ke
         const uint8_t* sc_up = sc_gate + 8 * srow;
         for (int b = warp; b < nblk; b += kGuWarps) {
           const bool in = b < nb_q;
-          const RowChunk gate = row_chunk_at<FMT>(c_gate, sc_gate, b, q, in);
-          const RowChunk up = row_chunk_at<FMT>(c_up, sc_up, b, q, in);
+          const RowChunk gate = row_chunk_at<FMT>(c_gate, sc_gate, b, q, in, gsc);
+          const RowChunk up = row_chunk_at<FMT>(c_up, sc_up, b, q, in, gsc);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
         p0 = chunk_bound(sorted_rows, p0, pe, top_k, t0);
       }
       const int n_e = pe - p0;
+      const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e] : 0.f;
       const bool ok = mbar_wait(&bars[st], parity, &s_abort, status) && act_ok;
       const int ntiles = (n_e + 7) / 8;
       for (int nt0 = 0; ok && nt0 < ntiles; nt0 += NT) {
@@ -336,8 +338,8 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
         const uint8_t* sc_hi = sc_lo + 8 * srow;
         for (int b = 0; b < nblk; ++b) {
           const bool in = b < nb_q;
-          const RowChunk c0 = row_chunk_at<FMT>(c_lo, sc_lo, b, q, in);
-          const RowChunk c1 = row_chunk_at<FMT>(c_hi, sc_hi, b, q, in);
+          const RowChunk c0 = row_chunk_at<FMT>(c_lo, sc_lo, b, q, in, gsc);
+          const RowChunk c1 = row_chunk_at<FMT>(c_hi, sc_hi, b, q, in, gsc);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
             if (nt0 + j >= ntiles) break;
@@ -525,6 +527,7 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
   const int units = max_touched(T, s.top_k, s.num_experts) * (s.inter / kGuFeatures);
   if (units == 0) return cudaSuccess;
   if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, units, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, ws, units, stream);
   return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, units, stream);
 }
 
@@ -532,6 +535,7 @@ cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& 
                                        uint16_t* out, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, ws, out, stream);
   return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, stream);
 }
 

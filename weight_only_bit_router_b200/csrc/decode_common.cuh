@@ -47,7 +47,7 @@ MOE_DEV uint32_t word_of(const uint4& c, int j) {
 
 // Scale bytes per weight row of a bank with reduction length K.
 __host__ __device__ inline int scale_row_bytes(int fmt, int K) {
-  return fmt == MOE_FMT_INT4_G128 ? int4_groups(K) * 2 : K / 32;
+  return fmt == MOE_FMT_INT4_G128 ? int4_groups(K) * 2 : fmt == MOE_FMT_NVFP4_G16 ? K / 16 : K / 32;
 }
 
 // One row's 16 code bytes for the lane's k-slice [kb + 32q, kb + 32q + 32) and
@@ -55,11 +55,13 @@ __host__ __device__ inline int scale_row_bytes(int fmt, int K) {
 // Slices past K read as zero weights.
 struct RowChunk {
   uint4 codes;
-  uint32_t mult;  // bf16x2 multiplier: the INT4 scale, or 2^e for MXFP4
+  uint32_t mult;   // bf16x2 multiplier: the INT4 scale, 2^e for MXFP4, or (NVFP4) the first 16-block's
+  uint32_t mult2;  // NVFP4: the second 16-block's multiplier (code words 2 and 3); otherwise = mult
 };
 
 template <int FMT>
 MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int r, int K, int kb, int q) {
+  static_assert(FMT != MOE_FMT_NVFP4_G16, "NVFP4 chunks come from row_chunk_at");
   RowChunk rc;
   const int k = kb + 32 * q;
   if (k < K) {
@@ -74,6 +76,7 @@ MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int
     rc.codes = make_uint4(0, 0, 0, 0);  // INT4 nibble 0 would be -8: zero the multiplier instead
     rc.mult = 0;
   }
+  rc.mult2 = rc.mult;
   return rc;
 }
 
@@ -135,24 +138,32 @@ MOE_DEV void load_act_frags_smem(const uint8_t* p, bool valid, uint32_t (&b)[8][
   act_frags_from_raw(X, b);
 }
 
-// A lane's 16 code bytes and multiplier of k-block b of one staged weight
+// A lane's 16 code bytes and multiplier(s) of k-block b of one staged weight
 // row: `codes` points at the row's codes plus the lane's slice offset 16q,
 // `scales` at the row's scales; `in` is false for a slice past K (zero
-// weights).
+// weights); `g` is the matrix's NVFP4 global scale (unused otherwise).
 template <int FMT>
-MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b, int q, bool in) {
+MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b, int q, bool in, float g = 0.f) {
   RowChunk rc;
   if (in) {
     rc.codes = *reinterpret_cast<const uint4*>(codes + 64 * b);
     if (FMT == MOE_FMT_INT4_G128) {
       const uint32_t sc = reinterpret_cast<const uint16_t*>(scales)[b];  // group b = k-block b
       rc.mult = sc | (sc << 16);
+      rc.mult2 = rc.mult;
+    } else if (FMT == MOE_FMT_NVFP4_G16) {
+      // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
+      const uint32_t m0 = nv_mult_bits(scales[8 * b + 2 * q], g), m1 = nv_mult_bits(scales[8 * b + 2 * q + 1], g);
+      rc.mult = m0 | (m0 << 16);
+      rc.mult2 = m1 | (m1 << 16);
     } else {
       rc.mult = pow2_bf16x2(int(scales[4 * b + q]) - 127);  // the slice is one 32-element block
+      rc.mult2 = rc.mult;
     }
   } else {
     rc.codes = make_uint4(0, 0, 0, 0);
     rc.mult = 0;
+    rc.mult2 = 0;
   }
   return rc;
 }
@@ -194,10 +205,10 @@ MOE_DEV void load_act_raw_cg(const uint16_t* rowp, int K, int kb, int q, bool va
   }
 }
 
-// One bf16 pair (nibbles i, i+4 of `word`) of a row chunk.
+// One bf16 pair (nibbles i, i+4 of code word j) of a row chunk.
 template <int FMT>
-MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i) {
-  return dq_pair<FMT>(word, i, rc.mult);
+MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i, int j = 0) {
+  return dq_pair<FMT>(word, i, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? rc.mult2 : rc.mult);
 }
 
 // acc[4] += W(rows r, r+8; one 128-k block) x activation fragments.
@@ -209,10 +220,10 @@ MOE_DEV void mma_block(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t a[4];
-      a[0] = dq<FMT>(lo, wl, 2 * h);
-      a[1] = dq<FMT>(hi, wh, 2 * h);
-      a[2] = dq<FMT>(lo, wl, 2 * h + 1);
-      a[3] = dq<FMT>(hi, wh, 2 * h + 1);
+      a[0] = dq<FMT>(lo, wl, 2 * h, j);
+      a[1] = dq<FMT>(hi, wh, 2 * h, j);
+      a[2] = dq<FMT>(lo, wl, 2 * h + 1, j);
+      a[3] = dq<FMT>(hi, wh, 2 * h + 1, j);
       mma_bf16_16816(acc, a, b[2 * j + h][0], b[2 * j + h][1]);
     }
   }

@@ -778,8 +778,9 @@ cudaError_t fused_launch(const FusedArgs& args, cudaStream_t stream) {
 }  // namespace
 
 bool decode_fused_supported(const moe_shape_t& s, int T) {
-  // gate_up: two 128-k blocks per warp of a group (H <= 2048); down: one (I <= 512)
-  return T >= 1 && T <= kFuMaxT && s.hidden <= 128 * kFuGuBlocks * kFuGroupWarps && s.inter <= 128 * kFuDnKBlocks &&
+  // gate_up: two 128-k blocks per warp of a group (H <= 2048); down: one (I <= 512);
+  // INT4 and MXFP4 banks (NVFP4 runs on the three-kernel decode path)
+  return s.fmt != MOE_FMT_NVFP4_G16 && T >= 1 && T <= kFuMaxT && s.hidden <= 128 * kFuGuBlocks * kFuGroupWarps && s.inter <= 128 * kFuDnKBlocks &&
          s.hidden % kFuDnRows == 0 && s.inter % kFuGuFeatures == 0 && kCtrHr + s.hidden / kFuDnRows <= kCtrSlot &&
          kCtrSlot + kFuMaxR <= int(kStatusBytes / 4) && s.num_experts <= kMaxExperts && s.top_k <= kMaxTopK;
 }

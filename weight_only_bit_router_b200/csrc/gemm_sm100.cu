@@ -45,13 +45,16 @@ enum GemmMode { kRouter = 0, kGateUp = 1, kDown = 2 };
 constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BN = kGemmBN;    // token columns per tile (max MMA N)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int SA = 3;          // bf16 weight-operand stages (dequantised, or router weights by TMA)
+constexpr int SA_DEFAULT = 3;  // bf16 weight-operand stages (dequantised, or router weights by TMA)
 constexpr int SB = 4;          // gathered token-operand stages (copies signal their own arrival)
 constexpr int SC = 3;          // code stages
 constexpr int kThreads = 512;
 constexpr int kDqThreads = 256;           // dequantisation threads (warps 4-11)
 constexpr int kEpiWarp0 = 12;             // first epilogue warp
-constexpr int kMaxScaleRow = 64;          // scale bytes per weight row (K <= 2048)
+// scale bytes staged per weight row: K <= 2048 for INT4 and MXFP4; NVFP4 keeps
+// one E4M3 byte per 16 k and, to make room, one bf16 operand stage less
+constexpr int kMaxScaleRow = 64;
+constexpr int kMaxScaleRowNv = 128;
 constexpr int kTileBytes = BM * BK * 2;   // 16 KB bf16 operand tile
 constexpr int kCodeBytes = BM * BK / 2;   // 4 KB code tile
 
@@ -67,6 +70,7 @@ struct GemmArgs {
   const int32_t* tile_base;    // [E+1] token-block prefix
   const float* topk_w;         // [T*k]
   const void* scales;          // scale plane of the packed bank
+  const float* gscale;         // NVFP4: per-expert global scales (null otherwise)
   int scale_row_stride;        // scale elements per weight row
   float* logits;
   uint16_t* act;
@@ -74,14 +78,17 @@ struct GemmArgs {
   uint32_t* status;
 };
 
-template <int MODE>
+template <int MODE, int FMT>
 struct Cfg {
+  static constexpr bool NV_WIDE = FMT == MOE_FMT_NVFP4_G16 && MODE == kGateUp;
+  static constexpr int SA = NV_WIDE ? SA_DEFAULT - 1 : SA_DEFAULT;
+  static constexpr int SROW = FMT == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv : kMaxScaleRow;
   static constexpr int NACC = MODE == kGateUp ? 2 : 1;                 // accumulators per tile
   static constexpr uint32_t TMEM_COLS = MODE == kGateUp ? 512 : 256;   // 2 buffers x NACC x BN
   static constexpr int SMEM_A = SA * NACC * kTileBytes;
   static constexpr int SMEM_B = SB * kTileBytes;
   static constexpr int SMEM_C = SC * NACC * kCodeBytes;
-  static constexpr int SMEM_S = MODE == kRouter ? 0 : 2 * NACC * BM * kMaxScaleRow;  // two tiles of scale rows
+  static constexpr int SMEM_S = MODE == kRouter ? 0 : 2 * NACC * BM * SROW;  // two tiles of scale rows
   static constexpr int SMEM_D = MODE == kDown ? BN * BM * 4 : 0;                     // down: [token][row] fp32
   static constexpr int SMEM = SMEM_A + SMEM_B + SMEM_C + SMEM_S + SMEM_D + 1024 /*barriers*/ + 1024 /*align*/ +
                              (kMaxExperts + 1) * 4;
@@ -146,8 +153,10 @@ MOE_DEV uint32_t pow2x2(int e) {
 
 // Dequantise 32 codes (one 16-byte chunk, k = 32*half .. +31 of the stage) of
 // one row and store them as four 16-byte bf16 chunks in swizzled layout.
+// Code words 0-1 use `mult`, words 2-3 `mult2` (the two 16-element NVFP4
+// blocks of the chunk; equal for the other formats).
 template <int FMT>
-MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint8_t* tile, int r, int half) {
+MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint32_t mult2, uint8_t* tile, int r, int half) {
   const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -155,7 +164,7 @@ MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint8_t* tile, int r, i
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t v = (FMT == MOE_FMT_INT4_G128) ? int4_pair(w[j], i) : e2m1_pair(w[j], i);
-      P[i] = bf16x2_mul(v, mult);  // (k+i, k+i+4)
+      P[i] = bf16x2_mul(v, j < 2 ? mult : mult2);  // (k+i, k+i+4)
     }
     uint4 o;
     o.x = prmt(P[0], P[1], 0x5410u);  // k0 k1
@@ -170,7 +179,9 @@ MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint8_t* tile, int r, i
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const GemmArgs args) {
-  using C = Cfg<MODE>;
+  using C = Cfg<MODE, FMT>;
+  constexpr int SA = C::SA;
+  constexpr int kSrow = C::SROW;
   constexpr int NACC = C::NACC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmArgs& a = args;
   // scale bytes per weight row (INT4: bf16 per 128 k; MXFP4: one byte per 32 k)
-  const int sb = FMT == MOE_FMT_INT4_G128 ? 2 * a.scale_row_stride : a.scale_row_stride;
+  const int sb = FMT == MOE_FMT_INT4_G128 ? 2 * a.scale_row_stride : a.scale_row_stride;  // bytes
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SC; ++i) {
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             long row0;
             if (MODE == kGateUp) row0 = long(t.e) * 2 * a.I + (c ? a.I : 0) + f0;
             else row0 = long(t.e) * a.H + f0;
-            bulk_g2s(sS + (slot * NACC + c) * BM * kMaxScaleRow, sp + row0 * sb, bytes, &sc_full[slot]);
+            bulk_g2s(sS + (slot * NACC + c) * BM * kSrow, sp + row0 * sb, bytes, &sc_full[slot]);
           }
         }
         for (int ks = 0; ks < KS; ++ks, ++g) {
@@ -395,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = f < a.M_total;
         const int slot = it & 1;
         if (!(ok = mbar_wait(&sc_full[slot], (it >> 1) & 1, abort, a.status))) break;
-        const uint8_t* srows = sS + slot * NACC * BM * kMaxScaleRow + r * sb;
+        const uint8_t* srows = sS + slot * NACC * BM * kSrow + r * sb;
+        const float gsc = FMT == MOE_FMT_NVFP4_G16 ? a.gscale[t.e] : 0.f;
         for (int ks = 0; ks < KS; ++ks, ++g) {
           const int sc = g % SC, so = g % SA;
           if (!(ok = mbar_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
@@ -404,17 +416,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < NACC; ++c) {
             const uint8_t* ctile = sC + (sc * NACC + c) * kCodeBytes + r * (BK / 2);
             const uint4 cw = *reinterpret_cast<const uint4*>(ctile + 16 * h);
-            uint32_t m = 0;
+            uint32_t m = 0, m2 = 0;
             if (valid) {
-              const uint8_t* srow = srows + c * BM * kMaxScaleRow;
+              const uint8_t* srow = srows + c * BM * kSrow;
               if (FMT == MOE_FMT_INT4_G128) {
                 const uint32_t sv = reinterpret_cast<const uint16_t*>(srow)[(ks * BK) / 128];
                 m = sv | (sv << 16);
+                m2 = m;
+              } else if (FMT == MOE_FMT_NVFP4_G16) {
+                // blocks of 16: (ks * 64 + 32 h) / 16 and the next one
+                const int blk = (ks * BK) / 16 + 2 * h;
+                const uint32_t b0 = nv_mult_bits(srow[blk], gsc), b1 = nv_mult_bits(srow[blk + 1], gsc);
+                m = b0 | (b0 << 16);
+                m2 = b1 | (b1 << 16);
               } else {
                 m = pow2x2(int(srow[(ks * BK) / 32 + h]) - 127);
+                m2 = m;
               }
             }
-            dequant_store32<FMT>(cw, m, sA + (so * NACC + c) * kTileBytes, r, h);
+            dequant_store32<FMT>(cw, m, m2, sA + (so * NACC + c) * kTileBytes, r, h);
           }
           // this thread's bf16 stores before the tensor core reads them
           fence_proxy_async_smem();
@@ -578,7 +598,7 @@ int sm_count() {
 template <int MODE, int FMT>
 cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ctas, cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<MODE, FMT>;
-  const int smem = Cfg<MODE>::SMEM;
+  const int smem = Cfg<MODE, FMT>::SMEM;
   // once per process (and per device), outside any stream capture of later calls
   static int configured_device = -1;
   int dev = 0;
@@ -643,9 +663,12 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int
 }
 
 bool grouped_supported(const moe_shape_t& s) {
-  // a tile's scale rows are staged in shared memory, kMaxScaleRow bytes per row
-  const auto row_bytes = [&](int K) { return s.fmt == MOE_FMT_INT4_G128 ? 2 * int4_groups(K) : K / 32; };
-  return row_bytes(s.hidden) <= kMaxScaleRow && row_bytes(s.inter) <= kMaxScaleRow;
+  // a tile's scale rows are staged in shared memory, up to kMaxScaleRow(Nv) bytes per row
+  const auto row_bytes = [&](int K) {
+    return s.fmt == MOE_FMT_INT4_G128 ? 2 * int4_groups(K) : s.fmt == MOE_FMT_NVFP4_G16 ? K / 16 : K / 32;
+  };
+  const int cap = s.fmt == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv : kMaxScaleRow;
+  return row_bytes(s.hidden) <= cap && row_bytes(s.inter) <= cap;
 }
 
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
@@ -660,9 +683,11 @@ cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* 
   a.n_ftiles = (s.inter + BM - 1) / BM;
   a.bsrc = x;
   a.scales = gu.scales;
-  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(gu.K) : gu.K / 32;
+  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(gu.K) : s.fmt == MOE_FMT_NVFP4_G16 ? gu.K / 16 : gu.K / 32;
+  a.gscale = gu.gscale;
   const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
   if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kGateUp, MOE_FMT_INT4_G128>(map, a, bound, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kGateUp, MOE_FMT_NVFP4_G16>(map, a, bound, stream);
   return launch_gemm<kGateUp, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
 }
 
@@ -678,9 +703,11 @@ cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, con
   a.n_ftiles = (s.hidden + BM - 1) / BM;
   a.bsrc = ws.act;
   a.scales = dn.scales;
-  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(dn.K) : dn.K / 32;
+  a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(dn.K) : s.fmt == MOE_FMT_NVFP4_G16 ? dn.K / 16 : dn.K / 32;
+  a.gscale = dn.gscale;
   const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
   if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kDown, MOE_FMT_INT4_G128>(map, a, bound, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kDown, MOE_FMT_NVFP4_G16>(map, a, bound, stream);
   return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
 }
 

@@ -24,13 +24,23 @@ inline size_t bank_scale_offset(moe_format_t fmt, int E, int N, int K) {
   return align_up(bank_codes_bytes(E, N, K), 256);
 }
 inline size_t bank_scale_bytes(moe_format_t fmt, int E, int N, int K) {
-  return fmt == MOE_FMT_INT4_G128 ? size_t(E) * N * int4_groups(K) * 2 : size_t(E) * N * (K / 32);
+  if (fmt == MOE_FMT_INT4_G128) return size_t(E) * N * int4_groups(K) * 2;
+  return fmt == MOE_FMT_NVFP4_G16 ? size_t(E) * N * (K / 16) : size_t(E) * N * (K / 32);
+}
+// NVFP4: the per-matrix fp32 global scales follow the block scales
+inline size_t bank_gscale_offset(moe_format_t fmt, int E, int N, int K) {
+  return align_up(bank_scale_offset(fmt, E, N, K) + bank_scale_bytes(fmt, E, N, K), 256);
+}
+inline size_t bank_total_bytes(moe_format_t fmt, int E, int N, int K) {
+  if (fmt == MOE_FMT_NVFP4_G16) return bank_gscale_offset(fmt, E, N, K) + size_t(E) * 4;
+  return bank_scale_offset(fmt, E, N, K) + bank_scale_bytes(fmt, E, N, K);
 }
 
 // Device view of one packed bank.
 struct Bank {
   const uint8_t* codes;  // [E][N][K/2]
-  const void* scales;    // INT4: bf16 [E][N][G]; MXFP4: u8 [E][N][K/32]
+  const void* scales;    // INT4: bf16 [E][N][G]; MXFP4: u8 [E][N][K/32]; NVFP4: E4M3 u8 [E][N][K/16]
+  const float* gscale;   // NVFP4: fp32 [E] per-matrix global scales; null otherwise
   int N, K;
 };
 

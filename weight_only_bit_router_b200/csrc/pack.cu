@@ -7,6 +7,10 @@
 // MXFP4: "kirillbilchenko/Nex-N2.5-mini-MXFP4-MxWave", Model summary and
 //       Quantization method (E2M1 codes, E8M0 scale per 32 elements,
 //       exponent floor(log2(amax / 6))).
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -243,9 +247,79 @@ __global__ void __launch_bounds__(256) pack_mxfp4_rule_kernel(const uint16_t* __
   if (lane == 0) scales[blk] = uint8_t(e + 127);
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 as W4A16 ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", What's
+// quantized to what: group 16, one global scale per expert shared by gate and
+// up, weights-only round-to-nearest).  Three steps: the maximum magnitude of
+// every matrix (as fp32 bits, atomically, into the global-scale slots), the
+// global scales g = fp32(amax / 2688) in place, then codes and E4M3 block
+// scales (one warp per (row, 128 columns); four lanes per block of 16).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nv_amax_kernel(const uint16_t* __restrict__ w, long per_matrix,
+                                                      uint32_t* __restrict__ amax_bits) {
+  const int e = blockIdx.y;
+  const uint16_t* m = w + long(e) * per_matrix;
+  uint32_t mx = 0;
+  for (long i = long(blockIdx.x) * blockDim.x + threadIdx.x; i < per_matrix; i += long(gridDim.x) * blockDim.x) {
+    const float v = fabsf(bf16_to_f32(m[i]));
+    if (isfinite(v)) mx = max(mx, __float_as_uint(v));  // non-negative floats order like their bits
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if ((threadIdx.x & 31) == 0 && mx) atomicMax(&amax_bits[e], mx);
+}
+
+__global__ void nv_gscale_kernel(uint32_t* __restrict__ slots, int E) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < E) reinterpret_cast<float*>(slots)[e] = __fdiv_rn(__uint_as_float(slots[e]), 2688.0f);
+}
+
+__global__ void __launch_bounds__(256) pack_nvfp4_kernel(const uint16_t* __restrict__ w, long rows, int N, int K,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                         const float* __restrict__ gscale, int32_t* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  const int C = (K + 127) / 128;
+  const long task = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (task >= rows * C) return;
+  const long row = task / C;
+  const int col = int(task % C) * 128 + lane * 4;
+  const bool active = col < K;  // K % 32 == 0: a block of 4 lanes is wholly in or out
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(w + row * K + col);
+    v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
+  }
+  float amax = 0.f;
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bad |= !isfinite(v[i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (bad && nonfinite) atomicAdd(nonfinite, 1);
+  if (!active) return;
+  const float g = gscale[row / N];
+  const float six_g = __fmul_rn(6.0f, g);
+  const float t = six_g == 0.f ? 0.f : __fdiv_rn(amax, six_g);
+  // nearest E4M3, ties to even, saturating at 448
+  const uint32_t code = uint32_t(__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3));
+  const float d = bf16_to_f32(uint16_t(nv_mult_bits(code, g)));
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t c = d == 0.f ? 0u : e2m1_code(fabsf(__fdiv_rn(v[i], d)));
+    const uint32_t sgn = (v[i] < 0.f && c != 0) ? 8u : 0u;
+    packed |= (sgn | c) << (4 * i);
+  }
+  *reinterpret_cast<uint16_t*>(codes + row * (K / 2) + col / 2) = uint16_t(packed);
+  if ((lane & 3) == 0) scales[row * (K / 16) + col / 16] = uint8_t(code);
+}
+
 // Debug dequantiser: one thread per code byte (two elements).
-__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales, int fmt,
-                               long rows, int K, uint16_t* __restrict__ out) {
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales,
+                               const float* __restrict__ gscale, int fmt, long rows, int N, int K,
+                               uint16_t* __restrict__ out) {
   const long i = long(blockIdx.x) * blockDim.x + threadIdx.x;
   const long nbytes = rows * (K / 2);
   if (i >= nbytes) return;
@@ -261,6 +335,12 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const void* __
       const int G = (K + 127) / 128;
       const float s = bf16_to_f32(static_cast<const uint16_t*>(scales)[row * G + k / 128]);
       val = float(int(nib) - 8) * s;  // exact in fp32, rounded once below
+    } else if (fmt == MOE_FMT_NVFP4_G16) {
+      const uint32_t sbyte = static_cast<const uint8_t*>(scales)[row * (K / 16) + k / 16];
+      const float d = bf16_to_f32(uint16_t(nv_mult_bits(sbyte, gscale[row / N])));
+      const float mags[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+      val = mags[nib & 7u] * d;  // exact in fp32, rounded once below
+      if (nib & 8u) val = -val;
     } else {
       const int e = int(static_cast<const uint8_t*>(scales)[row * (K / 32) + k / 32]) - 127;
       const float mags[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
@@ -284,6 +364,18 @@ cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K
   uint8_t* codes = static_cast<uint8_t*>(packed);
   void* scales = static_cast<uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
   if (grid == 0) return cudaSuccess;
+  if (fmt == MOE_FMT_NVFP4_G16) {
+    uint32_t* slots = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(packed) + bank_gscale_offset(fmt, E, N, K));
+    cudaError_t err = cudaMemsetAsync(slots, 0, size_t(E) * 4, stream);
+    if (err != cudaSuccess) return err;
+    const long per_matrix = long(N) * K;
+    const int bx = int(std::min<long>(64, (per_matrix + 255) / 256));
+    nv_amax_kernel<<<dim3(bx, E), 256, 0, stream>>>(w, per_matrix, slots);
+    nv_gscale_kernel<<<(E + 255) / 256, 256, 0, stream>>>(slots, E);
+    pack_nvfp4_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, rows, N, K, codes, static_cast<uint8_t*>(scales),
+                                                                  reinterpret_cast<const float*>(slots), nonfinite);
+    return cudaGetLastError();
+  }
   if (fmt == MOE_FMT_INT4_G128)
     pack_int4_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(w, rows, K, codes, static_cast<uint16_t*>(scales),
                                                                  nonfinite);
@@ -315,7 +407,10 @@ cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, i
   const long grid = (nbytes + block - 1) / block;
   const uint8_t* codes = static_cast<const uint8_t*>(packed);
   const void* scales = static_cast<const uint8_t*>(packed) + bank_scale_offset(fmt, E, N, K);
-  dequant_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(codes, scales, int(fmt), rows, K, out);
+  const float* gscale = fmt == MOE_FMT_NVFP4_G16 ? reinterpret_cast<const float*>(
+                                                       static_cast<const uint8_t*>(packed) + bank_gscale_offset(fmt, E, N, K))
+                                                 : nullptr;
+  dequant_kernel<<<dim3(unsigned(grid)), block, 0, stream>>>(codes, scales, gscale, int(fmt), rows, N, K, out);
   return cudaGetLastError();
 }
 
