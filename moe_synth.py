@@ -33,6 +33,7 @@ import torch
 
 # tensor ids for the per-tensor generator seeds
 _X, _ROUTER, _GATE_UP, _DOWN, _BIAS = 0, 1, 2, 3, 4
+_SH_GATE_UP, _SH_DOWN, _SH_GATE = 5, 6, 7
 
 ZIPF_S = 1.1
 WEIGHT_STD = 0.02
@@ -87,6 +88,16 @@ def gate_up_bank(shape: LayerShape, seed: int, device="cpu") -> torch.Tensor:
 
 def down_bank(shape: LayerShape, seed: int, device="cpu") -> torch.Tensor:
     return normal_bf16(shape.down_shape, WEIGHT_STD, seed, _DOWN, device)
+
+
+def shared_expert(shape: LayerShape, inter_shared: int, seed: int, device="cpu"):
+    """bf16 weights of the dense shared expert beside the routed ones: gate_up
+    [2 I_s, H] (gate rows then up rows), down [H, I_s], and the shared-expert
+    gate vector [H], all N(0, 0.02)."""
+    H = shape.hidden
+    return (normal_bf16((2 * inter_shared, H), WEIGHT_STD, seed, _SH_GATE_UP, device),
+            normal_bf16((H, inter_shared), WEIGHT_STD, seed, _SH_DOWN, device),
+            normal_bf16((H,), WEIGHT_STD, seed, _SH_GATE, device))
 
 
 def zipf_bias(shape: LayerShape, seed: int, s: float = ZIPF_S) -> torch.Tensor:

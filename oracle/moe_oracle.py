@@ -23,6 +23,10 @@ Sources, cited by page title and section:
   [LAYOUT] "primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", What's quantized to
            what: experts shipped as two batched 3-D tensors per layer; gate and
            up are the two halves of the fused gate_up bank.
+  [NVFP4]  the same section: NVFP4 experts, group 16, one global scale per
+           expert shared by gate and up, round-to-nearest.
+  [SHARED] the dense shared expert and its sigmoid gate (Int4-Int8Mix Recipe
+           table; MxWave What was quantized: kept in bf16).
 
 Readings where the pages are silent (each also listed in the design notes):
   * INT4 scale s = bf16(fp32(amax) / 7): the group max maps to code +-7, code
@@ -565,6 +569,37 @@ def forward(x_bits, router_bits, bias32, gate_up: PackedBank, down: PackedBank, 
     ids, w = route(logits, bias32, top_k)
     out, a_sorted = forward_routed(x_bits, ids, w, gate_up, down, E)
     return {"logits": logits, "ids": ids, "weights": w, "out": out, "a_sorted": a_sorted}
+
+
+# --------------------------------------------------------------------------
+# Shared expert beside the routed ones                              [SHARED]
+# ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe table: shared expert
+# gate/up/down_proj and a separate shared_expert_gate; "kirillbilchenko/Nex-
+# N2.5-mini-MXFP4-MxWave", What was quantized: shared experts stay bf16;
+# "primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8": shared experts, routers and
+# norms hold 0.15 B parameters, i.e. an intermediate size of 512)
+# --------------------------------------------------------------------------
+
+def shared_expert(x_bits, gate_up_bits, down_bits, gate_bits):
+    """Dense SwiGLU expert on every token, scaled by its gate:
+    g_t = sigmoid(x_t . w_gate), a = bf16(silu(h_gate) * h_up) (the same bf16
+    activation rounding as the routed experts), y = W_down a; in fp64 on the
+    bf16 weights.  Returns (g [T], y [T, H])."""
+    x = bf16_to_f64(x_bits)
+    a = bf16_round(swiglu_exact(x, bf16_to_f64(gate_up_bits)))
+    y = a @ bf16_to_f64(down_bits).T
+    z = x @ bf16_to_f64(gate_bits)
+    return 1.0 / (1.0 + np.exp(-z)), y
+
+
+def forward_with_shared(x_bits, router_bits, bias32, gate_up: PackedBank, down: PackedBank, top_k: int,
+                        shared_bits):
+    """The layer with its shared expert: out_t = sum_j w_tj y_tj + g_t y_shared,t."""
+    r = forward(x_bits, router_bits, bias32, gate_up, down, top_k)
+    g, ys = shared_expert(x_bits, *shared_bits)
+    r["shared_gate"], r["shared_y"] = g, ys
+    r["out"] = r["out"] + g[:, None] * ys
+    return r
 
 
 def routing_margin(logits32, bias32, k: int) -> np.ndarray:
