@@ -13,6 +13,7 @@ intermediate 512; synthetic seeded inputs, random-init weights):
   prefill_zipf  the same with the Zipf logit bias
   mx_decode4 / mx_prefill   the MXFP4 stack (17.1 GB packed) at 4 / 8192 tokens
   nv_decode4 / nv_prefill   the NVFP4 stack (E4M3 scale per 16 elements) at 4 / 8192 tokens
+  sh_decode4 / sh_prefill   the INT4 stack with each layer's bf16 shared expert (moe_forward_shared)
 
 The metric is MoE-layer tokens per second: tokens x layers processed per
 second of device time, whole job (all ranks).  With --gpus N > 1 (launched by
@@ -57,7 +58,11 @@ WORKLOADS = {
     "mx_prefill": ("mxfp4", 8192, False, 1),
     "nv_decode4": ("nvfp4", 4, False, NUM_LAYERS),
     "nv_prefill": ("nvfp4", 8192, False, 1),
+    "sh_decode4": ("int4_g128", 4, False, NUM_LAYERS),
+    "sh_prefill": ("int4_g128", 8192, False, 1),
 }
+# workloads whose layers carry the bf16 shared expert (intermediate 512)
+SHARED_INTER = {"sh_decode4": 512, "sh_prefill": 512}
 METRIC = "W4A16 MoE-layer tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -309,15 +314,20 @@ def run_ours(args, rank, local, world):
     stack = Stack(moe, fmt, L, device, zipf)
     shape = stack.shape
     x = moe_synth.hidden_states(moe_synth.NEX, T, rank_token_seed(rank, T), device)
-    ws = moe.alloc_workspace(shape, T, device)
+    inter_sh = SHARED_INTER.get(args.workload)
+    shared = ([moe_synth.shared_expert(moe_synth.NEX, inter_sh, moe_synth.SEED_STACK_BASE + l, device)
+               for l in range(L)] if inter_sh else None)
+    ws = moe.alloc_workspace_shared(shape, inter_sh, T, device) if inter_sh else moe.alloc_workspace(shape, T, device)
     outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
     path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL,
             "fused": moe.MOE_PATH_FUSED}[args.path]
 
     def layer_call(l, events=None):
-        moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
-                        bias=stack.bias[l], path=path, events=events, stream=torch.cuda.current_stream())
+        fwd = (lambda *a, **k: moe.moe_forward_shared(shape, shared[l], *a, **k)) if shared else \
+            (lambda *a, **k: moe.moe_forward(shape, *a, **k))
+        fwd(x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
+            bias=stack.bias[l], path=path, events=events, stream=torch.cuda.current_stream())
 
     # one step: layers_per_step consecutive layers; graphs rotate over the stack
     n_graphs = L // layers_per_step
@@ -379,8 +389,10 @@ def run_ours(args, rank, local, world):
     touched = []
     ids_buf = torch.empty(T, shape.top_k, dtype=torch.int32, device=device)
     for l in range(L):
-        moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
-                        bias=stack.bias[l], path=path, debug={"topk_ids_out": ids_buf})
+        fwd = (lambda *a, **k: moe.moe_forward_shared(shape, shared[l], *a, **k)) if shared else \
+            (lambda *a, **k: moe.moe_forward(shape, *a, **k))
+        fwd(x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
+            bias=stack.bias[l], path=path, debug={"topk_ids_out": ids_buf})
         touched.append(len(torch.unique(ids_buf)))
     avg_touched = float(np.mean(touched))
     work = stage_work(moe, shape, T, avg_touched)
@@ -434,7 +446,8 @@ def run_ours(args, rank, local, world):
     e2e_ms = reduce_max(e0.elapsed_time(e1), device)
     e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
 
-    launches = moe.moe_forward_launch_count(shape, T, path, False) * layers_per_step * args.steps
+    per_layer = moe.moe_forward_launch_count(shape, T, path, False) + (3 if shared else 0)  # shared: 2 GEMMs + SwiGLU
+    launches = per_layer * layers_per_step * args.steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -447,7 +460,7 @@ def run_ours(args, rank, local, world):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
-        "config": {"workload": f"nex_moe_{fmt}_T{T}{'_zipf' if zipf else ''}_{layers_per_step}layer_step_"
+        "config": {"workload": f"nex_moe_{fmt}_T{T}{'_zipf' if zipf else ''}{f'_shared{inter_sh}' if inter_sh else ''}_{layers_per_step}layer_step_"
                                f"of_{L}layer_stack",
                    "hidden": shape.hidden, "experts": shape.num_experts, "top_k": shape.top_k,
                    "inter": shape.inter, "tokens_per_layer": T, "layers_per_step": layers_per_step,

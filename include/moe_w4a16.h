@@ -303,6 +303,39 @@ MOE_API moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
                                 const moe_forward_opts_t* opts, cudaStream_t stream);
 
+/* The dense shared expert of a Qwen3.5-MoE block, beside the routed ones
+ * ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe table: shared expert
+ * gate/up/down_proj and shared_expert_gate; "kirillbilchenko/Nex-N2.5-mini-
+ * MXFP4-MxWave", What was quantized: shared experts stay bf16).  Weights are
+ * bf16 (not quantised), device pointers, 16-byte aligned. */
+typedef struct {
+  int inter;                /* I_s, a positive multiple of 64 (512 in the cards' model) */
+  const uint16_t* gate_up;  /* [2*I_s, H] bf16: gate rows [0, I_s), up rows [I_s, 2*I_s) */
+  const uint16_t* down;     /* [H, I_s] bf16 */
+  const uint16_t* gate;     /* [H] bf16 weight of the shared_expert_gate (H -> 1) */
+} moe_shared_expert_t;
+
+/* Workspace bytes moe_forward_shared needs for T tokens (the routed layer's
+ * workspace plus the shared expert's fp32 and bf16 intermediates); 0 if the
+ * arguments are invalid. */
+MOE_API size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_shared, int T);
+
+/* moe_forward plus the shared expert:
+ *   g_t   = sigmoid(x_t . w_gate)                     fp32
+ *   a_s   = bf16(silu(W_gate_s x_t) * (W_up_s x_t))   (the routed experts' rounding)
+ *   out_t = bf16( sum_j w_tj y_tj  +  g_t * (W_down_s a_s) )   one final rounding
+ * The shared expert runs on the tensor cores (tcgen05) for every T; its
+ * contribution is added to the routed combine in fp32 before the output's
+ * single bf16 rounding.  Paths MOE_PATH_AUTO, _DECODE and _PREFILL; the
+ * single-kernel path returns MOE_ERR_UNSUPPORTED.  Other arguments, errors
+ * and the workspace rules as moe_forward (workspace >=
+ * moe_workspace_bytes_shared bytes). */
+MOE_API moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_expert_t* shared,
+                                const uint16_t* x, int T, const uint16_t* router_w,
+                                const float* logit_bias, const void* gate_up_packed,
+                                const void* down_packed, void* workspace, size_t workspace_bytes,
+                                uint16_t* out, const moe_forward_opts_t* opts, cudaStream_t stream);
+
 /* Zeroes the status word and the kernels' completion counters at the start
  * of a workspace (its first 4096 bytes; enqueued on `stream`).  Call once
  * after allocating a workspace, before its first use; every forward leaves

@@ -1,0 +1,95 @@
+"""The layer with its bf16 shared expert (moe_forward_shared) against the CPU
+oracle, through the C ABI (needs a B200).
+
+Per element |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref), ref = the oracle's
+routed combine of the GPU's own bf16 activations (where fp32 accumulation put
+an activation across a bf16 rounding boundary both neighbours are correct;
+see parity_util.flip_aware_activations) plus the oracle's gated shared expert.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import weight_only_bit_router_b200 as moe
+from oracle import moe_oracle as o
+from parity_util import LazyOracleBank, assert_out_close, assert_routing_consistent, flip_aware_activations
+from test_gpu_parity import DEV, gpu_activations_in_oracle_order, pack_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
+    s = layer.shape
+    shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
+    T = layer.x.shape[0]
+    shared = moe_synth.shared_expert(s, inter_shared, seed, DEV)
+    gu, dn = pack_gpu(fmt, layer.gate_up), pack_gpu(fmt, layer.down)
+    ws = moe.alloc_workspace_shared(shape, inter_shared, T)
+    dbg = {
+        "logits_out": torch.empty(T, s.num_experts, dtype=torch.float32, device=DEV),
+        "topk_ids_out": torch.empty(T, s.top_k, dtype=torch.int32, device=DEV),
+        "topk_w_out": torch.empty(T, s.top_k, dtype=torch.float32, device=DEV),
+        "act_out": torch.empty(T * s.top_k, s.inter, dtype=torch.bfloat16, device=DEV),
+        "offsets_out": torch.empty(s.num_experts + 1, dtype=torch.int32, device=DEV),
+        "sorted_rows_out": torch.empty(T * s.top_k, dtype=torch.int32, device=DEV),
+    }
+    out = moe.moe_forward_shared(shape, shared, layer.x, layer.router_w, gu, dn, ws, bias=layer.bias, path=path,
+                                 debug=dbg)
+    assert moe.moe_workspace_status(ws) == moe.MOE_OK
+    tok = np.arange(T) if sample is None else np.asarray(sample)
+    tok_d = torch.as_tensor(tok, device=DEV)
+    xb = moe_synth.bf16_bits(layer.x)[tok]
+    bias = None if layer.bias is None else layer.bias.cpu().numpy()
+    ref_logits = o.router_logits(xb, moe_synth.bf16_bits(layer.router_w))
+    assert_routing_consistent(dbg["logits_out"][tok_d], ref_logits, dbg["topk_ids_out"][tok_d], bias, s.top_k)
+    rid, rw = o.route(dbg["logits_out"][tok_d].cpu().numpy(), bias, s.top_k)
+    assert np.array_equal(rid, dbg["topk_ids_out"][tok_d].cpu().numpy())
+    gub, dnb = LazyOracleBank(fmt, layer.gate_up), LazyOracleBank(fmt, layer.down)
+    a_exact, a_round = o.expert_activations(xb, rid, gub, s.num_experts)
+    act_used, n_diff = flip_aware_activations(gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k),
+                                              a_exact, a_round)
+    routed = o.down_and_combine(act_used, rid, rw, dnb, s.num_experts)
+    g, ys = o.shared_expert(xb, *(moe_synth.bf16_bits(t) for t in shared))
+    assert np.all((g > 0.01) & (g < 0.99))  # the gate is not saturated on these inputs
+    ref = routed + g[:, None] * ys
+    assert_out_close(out[tok_d], ref, f"{fmt} shared T={T} ({n_diff} routed activations rounded the other way)")
+    # the shared expert changes the output: the routed-only oracle must not pass
+    n_far = int(np.sum(np.abs(out[tok_d].float().cpu().numpy() - routed) > 1e-2 * np.abs(routed) +
+                       1e-3 * np.sqrt(np.mean(routed ** 2))))
+    assert n_far > out[tok_d].numel() // 4
+    return out
+
+
+@pytest.mark.parametrize("fmt", ["int4_g128", "nvfp4"])
+@pytest.mark.parametrize("path", [moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL])
+def test_shared_tiny_layer(fmt, path):
+    layer = moe_synth.make_layer(moe_synth.TINY, T=16, seed=moe_synth.SEED_TINY, device=DEV)
+    check_shared(layer, fmt, 64, path, seed=3)
+
+
+def test_shared_nex_decode():
+    layer = moe_synth.make_layer(moe_synth.NEX, T=4, seed=104, device=DEV)
+    check_shared(layer, "int4_g128", 512, seed=104)
+
+
+def test_shared_nex_prefill_sampled():
+    layer = moe_synth.make_layer(moe_synth.NEX, T=2048, seed=2048, device=DEV)
+    sample = np.random.default_rng(9).choice(2048, 24, replace=False)
+    check_shared(layer, "mxfp4", 512, sample=sample, seed=2048)
+
+
+def test_shared_expert_rejects_single_kernel_path_and_bad_sizes():
+    layer = moe_synth.make_layer(moe_synth.TINY, T=4, seed=1, device=DEV)
+    s = layer.shape
+    shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, "int4_g128")
+    gu, dn = pack_gpu("int4_g128", layer.gate_up), pack_gpu("int4_g128", layer.down)
+    ws = moe.alloc_workspace_shared(shape, 64, 4)
+    with pytest.raises(moe.MoeError):
+        moe.moe_forward_shared(shape, moe_synth.shared_expert(s, 64, 1, DEV), layer.x, layer.router_w, gu, dn, ws,
+                               path=moe.MOE_PATH_FUSED)
+    small = torch.empty(moe.moe_workspace_bytes(shape, 4), dtype=torch.uint8, device=DEV)
+    moe.moe_workspace_init(small)
+    with pytest.raises(moe.MoeError):   # the routed layer's workspace is too small for the shared expert
+        moe.moe_forward_shared(shape, moe_synth.shared_expert(s, 64, 1, DEV), layer.x, layer.router_w, gu, dn, small)
+    assert moe.moe_workspace_bytes_shared(shape, 96, 4) == 0   # I_s not a multiple of 64

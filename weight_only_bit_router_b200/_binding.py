@@ -41,6 +41,11 @@ class MoeShape(ctypes.Structure):
                 ("top_k", ctypes.c_int), ("fmt", ctypes.c_int)]
 
 
+class SharedExpert(ctypes.Structure):
+    _fields_ = [("inter", ctypes.c_int), ("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p),
+                ("gate", ctypes.c_void_p)]
+
+
 class ForwardOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("topk_ids_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
                 ("logits_out", ctypes.c_void_p), ("offsets_out", ctypes.c_void_p),
@@ -78,6 +83,11 @@ _SIGS = {
     "moe_forward_routed": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int,
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                          ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
+    "moe_workspace_bytes_shared": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int]),
+    "moe_forward_shared": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.POINTER(SharedExpert), ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
     "moe_forward_launch_count": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int,
                                                 ctypes.c_int]),
@@ -300,6 +310,34 @@ def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, works
                            _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
                            _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
     _check("moe_forward", st)
+    return out
+
+
+def moe_workspace_bytes_shared(shape: MoeShape, inter_shared: int, T: int) -> int:
+    return lib().moe_workspace_bytes_shared(ctypes.byref(shape), inter_shared, T)
+
+
+def alloc_workspace_shared(shape: MoeShape, inter_shared: int, T: int, device="cuda", stream=None):
+    nbytes = moe_workspace_bytes_shared(shape, inter_shared, T)
+    ws = torch.empty(max(nbytes, 4096), dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream=stream)
+    return ws
+
+
+def moe_forward_shared(shape: MoeShape, shared, x, router_w, gate_up_packed, down_packed, workspace, out=None,
+                       bias=None, path=None, debug=None, events=None, stream=None):
+    """moe_forward plus the bf16 shared expert; shared = (gate_up [2 I_s, H], down [H, I_s], gate [H])."""
+    gu_s, dn_s, gate_s = shared
+    sh = SharedExpert(int(dn_s.shape[1]), _ptr(_bits(gu_s)), _ptr(_bits(dn_s)), _ptr(_bits(gate_s)))
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
+    o, _keep = _opts(path, debug, events)
+    st = lib().moe_forward_shared(ctypes.byref(shape), ctypes.byref(sh), _ptr(_bits(x)), T, _ptr(_bits(router_w)),
+                                  _ptr(bias), _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace),
+                                  workspace.numel(), _ptr(out), ctypes.byref(o) if o is not None else None,
+                                  _stream(stream))
+    _check("moe_forward_shared", st)
     return out
 
 

@@ -133,10 +133,13 @@ moe_status_t build_permutation(const moe_shape_t& s, int T, const Workspace& ws,
                                           ws.pos, ws.block_hist, ws.touched, ws.tile_base, kGemmBN, stream));
 }
 
-// Stages 2-4: experts and combine, given routing in the workspace.
+// Stages 2-4: experts and combine, given routing in the workspace.  sh_gate /
+// sh_y (nullable): the shared expert's gate [T] and output [T, H], added before
+// the output's bf16 rounding.
 moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const void* gu_packed,
                          const void* dn_packed, const Workspace& ws, uint16_t* out, bool decode,
-                         const moe_forward_opts_t* o, cudaStream_t stream) {
+                         const moe_forward_opts_t* o, cudaStream_t stream, const float* sh_gate = nullptr,
+                         const float* sh_y = nullptr) {
   const Bank gu = make_bank(gu_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
   const Bank dn = make_bank(dn_packed, s.fmt, s.num_experts, s.hidden, s.inter);
   MOE_TRY(mark(o, 2, 0, stream));
@@ -146,7 +149,7 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
     // down projection and the combine are one kernel on this path
-    MOE_TRY(launch_decode_down_combine(s, T, dn, ws, out, stream));
+    MOE_TRY(launch_decode_down_combine(s, T, dn, ws, out, sh_gate, sh_y, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
   } else {
@@ -154,7 +157,7 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
     MOE_TRY(launch_grouped_down(s, T, dn, ws, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
-    MOE_TRY(launch_finalize_out(ws.out_acc, long(T) * s.hidden, out, stream));
+    MOE_TRY(launch_finalize_out(ws.out_acc, T, s.hidden, sh_gate, sh_y, out, stream));
   }
   MOE_TRY(mark(o, 4, 1, stream));
   return MOE_OK;
@@ -395,6 +398,82 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
   MOE_TRY(mark(opts, 1, 1, stream));
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
   return copy_debug_outputs(s, T, ws, opts, true, stream);
+}
+
+// The shared expert's intermediates after the routed layer's workspace.
+struct SharedWs {
+  float* h;      // [T, 2 I_s] fp32 gate_up product
+  uint16_t* a;   // [T, I_s] bf16 SwiGLU
+  float* g;      // [T] fp32 sigmoid gate
+  float* y;      // [T, H] fp32 down product
+  size_t bytes;  // total workspace bytes, routed part included
+};
+
+static SharedWs carve_shared(void* base, const moe_shape_t& s, int I_s, int T) {
+  SharedWs w{};
+  size_t off = carve_workspace(nullptr, s, T).bytes;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  auto take = [&](size_t bytes) -> void* {
+    void* r = p ? p + off : nullptr;
+    off += align_up(bytes, 256);
+    return r;
+  };
+  w.h = static_cast<float*>(take(size_t(T) * 2 * I_s * 4));
+  w.a = static_cast<uint16_t*>(take(size_t(T) * I_s * 2));
+  w.g = static_cast<float*>(take(size_t(T) * 4));
+  w.y = static_cast<float*>(take(size_t(T) * s.hidden * 4));
+  w.bytes = off;
+  return w;
+}
+
+size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_shared, int T) {
+  if (check_shape(shape) != MOE_OK || T < 0 || inter_shared <= 0 || inter_shared % 64) return 0;
+  return carve_shared(nullptr, *shape, inter_shared, T).bytes;
+}
+
+moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_expert_t* shared, const uint16_t* x,
+                                int T, const uint16_t* router_w, const float* logit_bias,
+                                const void* gate_up_packed, const void* down_packed, void* workspace,
+                                size_t workspace_bytes, uint16_t* out, const moe_forward_opts_t* opts,
+                                cudaStream_t stream) {
+  if (!shared) return MOE_ERR_INVALID_ARG;
+  if (shared->inter <= 0) return MOE_ERR_INVALID_ARG;
+  if (shared->inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (opts && opts->path == MOE_PATH_FUSED) return MOE_ERR_UNSUPPORTED;
+  bool decode = false, fused = false;
+  moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
+                                         out, opts, &decode, &fused);
+  if (st != MOE_OK || T == 0) return st;
+  if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
+  if (!shared->gate_up || !shared->down || !shared->gate || !aligned(shared->gate_up, 16) ||
+      !aligned(shared->down, 16) || !aligned(shared->gate, 16))
+    return MOE_ERR_INVALID_ARG;
+  const moe_shape_t& s = *shape;
+  const int I_s = shared->inter;
+  if (workspace_bytes < carve_shared(nullptr, s, I_s, T).bytes) return MOE_ERR_WORKSPACE;
+  const Workspace ws = carve_workspace(workspace, s, T);
+  const SharedWs sw = carve_shared(workspace, s, I_s, T);
+  // the shared expert needs only x: gate_up product, SwiGLU and gate, down product
+  MOE_TRY(launch_router_gemm(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, ws.status, stream));
+  MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, T, s.hidden, I_s, sw.a, sw.g, stream));
+  MOE_TRY(launch_router_gemm(sw.a, shared->down, T, I_s, s.hidden, sw.y, ws.status, stream));
+  // the routed experts, their combine and the shared expert's gated output
+  MOE_TRY(mark(opts, 0, 0, stream));
+  if (T <= kDecodeMaxT) {
+    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+  } else {
+    MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+    MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
+    if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
+  }
+  MOE_TRY(mark(opts, 1, 1, stream));
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream, sw.g, sw.y)) != MOE_OK)
+    return st;
+  return copy_debug_outputs(s, T, ws, opts, false, stream);
 }
 
 int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed) {

@@ -243,7 +243,7 @@ template <int FMT, int NT, bool ACT_SMEM>
 __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
     Bank dn, int T, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
     const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ sorted_rows,
-    uint16_t* __restrict__ out, uint32_t* status) {
+    uint16_t* __restrict__ out, const float* __restrict__ sh_gate, const float* __restrict__ sh_y, uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = dn.N, K = dn.K;  // K = I
   const UnitLayout L = unit_layout(FMT, K, kDecRows, 1);
@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) decode_down_kernel(
 #pragma unroll 4
       for (int w = 0; w < kDnWarps; ++w) sum += accs[w * tchunk * kDecRows + idx];
       const int t = t0 + idx / kDecRows, f = f0 + idx % kDecRows;
+      if (sh_y) sum += sh_gate[t] * sh_y[size_t(t) * H + f];  // the shared expert, before the one rounding
       out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
     }
     __syncthreads();
@@ -499,7 +500,7 @@ cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Ba
 
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
-                    cudaStream_t stream) {
+                    const float* sh_gate, const float* sh_y, cudaStream_t stream) {
   // stage all T*k activation rows in shared memory when they fit
   const int R = T * s.top_k;
   const bool act_smem = T <= kDnTokens && down_smem(FMT, s.inter, T, R) <= kMaxSmemPerCta;
@@ -509,15 +510,15 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace
   if (err != cudaSuccess) return err;
   return launch_pdl(k, dim3(s.hidden / kDecRows), dim3(kDnWarps * 32), smem, stream, dn, T, s.top_k,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const uint16_t*)ws.act,
-                    (const float*)ws.topk_w, (const int32_t*)ws.sorted_rows, out, ws.status);
+                    (const float*)ws.topk_w, (const int32_t*)ws.sorted_rows, out, sh_gate, sh_y, ws.status);
 }
 
 template <int FMT>
 cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
-                     cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, stream);
-  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, stream);
+                     const float* sh_gate, const float* sh_y, cudaStream_t stream) {
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+  return down_nt<FMT, kDecNT>(s, T, dn, ws, out, sh_gate, sh_y, stream);
 }
 
 }  // namespace
@@ -532,11 +533,12 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
 }
 
 cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                       uint16_t* out, cudaStream_t stream) {
+                                       uint16_t* out, const float* sh_gate, const float* sh_y,
+                                       cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, ws, out, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, stream);
+  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, sh_gate, sh_y, stream);
 }
 
 }  // namespace moe

@@ -528,11 +528,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
-// fp32 accumulator -> bf16 output
-__global__ void finalize_kernel(const float* __restrict__ acc, long n, uint16_t* __restrict__ out) {
+// fp32 accumulator (+ the shared expert's gated output) -> bf16 output
+__global__ void finalize_kernel(const float* __restrict__ acc, long n, int H, const float* __restrict__ sh_gate,
+                                const float* __restrict__ sh_y, uint16_t* __restrict__ out) {
   const long i = (long(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i >= n) return;
-  const float4 v = *reinterpret_cast<const float4*>(acc + i);
+  float4 v = *reinterpret_cast<const float4*>(acc + i);
+  if (sh_y) {
+    const float g = sh_gate[i / H];  // H % 4 == 0: the four elements share a token
+    const float4 y = *reinterpret_cast<const float4*>(sh_y + i);
+    v.x += g * y.x;
+    v.y += g * y.y;
+    v.z += g * y.z;
+    v.w += g * y.w;
+  }
   uint2 o;
   o.x = pack_bf16x2(v.x, v.y);
   o.y = pack_bf16x2(v.z, v.w);
@@ -711,11 +720,13 @@ cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, con
   return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
 }
 
-cudaError_t launch_finalize_out(const float* acc, long n, uint16_t* out, cudaStream_t stream) {
+cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_gate, const float* sh_y,
+                                uint16_t* out, cudaStream_t stream) {
+  const long n = long(T) * H;
   if (n == 0) return cudaSuccess;
   const int block = 256;
   const long threads = (n + 3) / 4;
-  finalize_kernel<<<unsigned((threads + block - 1) / block), block, 0, stream>>>(acc, n, out);
+  finalize_kernel<<<unsigned((threads + block - 1) / block), block, 0, stream>>>(acc, n, H, sh_gate, sh_y, out);
   return cudaGetLastError();
 }
 

@@ -104,8 +104,11 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 // decode.cu
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const Workspace& ws, cudaStream_t stream);
+// sh_gate [T] / sh_y [T, H] (both null, or both given): the shared expert's
+// gate and output, added as sh_gate[t] * sh_y[t][f] before the bf16 rounding
 cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                       uint16_t* out, cudaStream_t stream);
+                                       uint16_t* out, const float* sh_gate, const float* sh_y,
+                                       cudaStream_t stream);
 
 // decode_fused.cu: the whole layer as one cooperative kernel for T <= 8
 bool decode_fused_supported(const moe_shape_t& s, int T);
@@ -125,7 +128,14 @@ cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* 
                                    const Workspace& ws, cudaStream_t stream);
 cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
                                 cudaStream_t stream);
-cudaError_t launch_finalize_out(const float* acc, long n, uint16_t* out, cudaStream_t stream);
+// out = bf16(acc [+ sh_gate[t] * sh_y[t][f]]) over [T, H] (sh_* nullable)
+cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_gate, const float* sh_y,
+                                uint16_t* out, cudaStream_t stream);
+
+// shared.cu: the shared expert's SwiGLU and sigmoid gate from the fp32 gate_up
+// product h [T, 2 I_s]: a [T, I_s] bf16, g [T] fp32 (g = sigmoid(x . w_gate))
+cudaError_t launch_shared_swiglu_gate(const uint16_t* x, const uint16_t* w_gate, const float* h, int T, int H,
+                                      int I_s, uint16_t* a, float* g, cudaStream_t stream);
 
 // selftest of the bounded device-side wait (api.cu)
 cudaError_t launch_bounded_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
