@@ -2,9 +2,13 @@
 oracle, through the C ABI (needs a B200).
 
 Per element |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref), ref = the oracle's
-routed combine of the GPU's own bf16 activations (where fp32 accumulation put
-an activation across a bf16 rounding boundary both neighbours are correct;
-see parity_util.flip_aware_activations) plus the oracle's gated shared expert.
+routed combine of the GPU's own bf16 activations plus the oracle's gated
+shared expert on the GPU's own shared-expert activations: where fp32
+accumulation put an activation across a bf16 rounding boundary both
+neighbours are correct (parity_util.flip_aware_activations checks each such
+activation against the exact value).  The shared expert's bf16 activations
+are read from their place in the workspace, right after the routed layer's
+part (at offset moe_workspace_bytes).
 """
 import numpy as np
 import pytest
@@ -50,8 +54,17 @@ def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
     act_used, n_diff = flip_aware_activations(gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k),
                                               a_exact, a_round)
     routed = o.down_and_combine(act_used, rid, rw, dnb, s.num_experts)
-    g, ys = o.shared_expert(xb, *(moe_synth.bf16_bits(t) for t in shared))
+    sh_bits = [moe_synth.bf16_bits(t) for t in shared]
+    g, ys_oracle = o.shared_expert(xb, *sh_bits)
     assert np.all((g > 0.01) & (g < 0.99))  # the gate is not saturated on these inputs
+    # the GPU's shared-expert activations, checked and used like the routed ones
+    off = moe.moe_workspace_bytes(shape, T)
+    a_gpu = ws[off:off + T * inter_shared * 2].view(torch.bfloat16).view(T, inter_shared)[tok_d]
+    a_s_exact = o.swiglu_exact(o.bf16_to_f64(xb), o.bf16_to_f64(sh_bits[0]))
+    a_s_used, n_sh = flip_aware_activations(o.bf16_to_f64(moe_synth.bf16_bits(a_gpu)), a_s_exact,
+                                            o.bf16_round(a_s_exact))
+    ys = a_s_used @ o.bf16_to_f64(sh_bits[1]).T
+    assert np.allclose(ys, ys_oracle, rtol=1e-2, atol=1e-3 * np.sqrt(np.mean(ys_oracle ** 2)))
     ref = routed + g[:, None] * ys
     assert_out_close(out[tok_d], ref, f"{fmt} shared T={T} ({n_diff} routed activations rounded the other way)")
     # the shared expert changes the output: the routed-only oracle must not pass
@@ -68,9 +81,10 @@ def test_shared_tiny_layer(fmt, path):
     check_shared(layer, fmt, 64, path, seed=3)
 
 
-def test_shared_nex_decode():
-    layer = moe_synth.make_layer(moe_synth.NEX, T=4, seed=104, device=DEV)
-    check_shared(layer, "int4_g128", 512, seed=104)
+@pytest.mark.parametrize("T", [4, 24])
+def test_shared_nex_decode(T):
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=100 + T, device=DEV)
+    check_shared(layer, "int4_g128", 512, seed=100 + T)
 
 
 def test_shared_nex_prefill_sampled():

@@ -402,10 +402,11 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
 
 // The shared expert's intermediates after the routed layer's workspace.
 struct SharedWs {
-  float* h;      // [T, 2 I_s] fp32 gate_up product
-  uint16_t* a;   // [T, I_s] bf16 SwiGLU
+  uint16_t* a;   // [T, I_s] bf16 SwiGLU (first: its offset is the routed workspace's size)
   float* g;      // [T] fp32 sigmoid gate
   float* y;      // [T, H] fp32 down product
+  float* h;      // [splits][T, 2 I_s] fp32 gate_up product (split-K partials for T <= 32)
+  int splits;
   size_t bytes;  // total workspace bytes, routed part included
 };
 
@@ -418,10 +419,11 @@ static SharedWs carve_shared(void* base, const moe_shape_t& s, int I_s, int T) {
     off += align_up(bytes, 256);
     return r;
   };
-  w.h = static_cast<float*>(take(size_t(T) * 2 * I_s * 4));
+  w.splits = T <= kDecodeMaxT ? shared_gemv_splits(s.hidden) : 1;
   w.a = static_cast<uint16_t*>(take(size_t(T) * I_s * 2));
   w.g = static_cast<float*>(take(size_t(T) * 4));
-  w.y = static_cast<float*>(take(size_t(T) * s.hidden * 4));
+  w.y = static_cast<float*>(take(size_t(T) * s.hidden * 4 * (T <= kDecodeMaxT ? shared_gemv_splits(I_s) : 1)));
+  w.h = static_cast<float*>(take(size_t(w.splits) * T * 2 * I_s * 4));
   w.bytes = off;
   return w;
 }
@@ -453,10 +455,17 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   if (workspace_bytes < carve_shared(nullptr, s, I_s, T).bytes) return MOE_ERR_WORKSPACE;
   const Workspace ws = carve_workspace(workspace, s, T);
   const SharedWs sw = carve_shared(workspace, s, I_s, T);
-  // the shared expert needs only x: gate_up product, SwiGLU and gate, down product
-  MOE_TRY(launch_router_gemm(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, ws.status, stream));
-  MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, T, s.hidden, I_s, sw.a, sw.g, stream));
-  MOE_TRY(launch_router_gemm(sw.a, shared->down, T, I_s, s.hidden, sw.y, ws.status, stream));
+  // the shared expert needs only x: gate_up product, SwiGLU and gate, down
+  // product (split-K mma.sync for small batches, tcgen05 above)
+  if (T <= kDecodeMaxT && I_s <= 512) {
+    MOE_TRY(launch_shared_gemv(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, stream));
+    MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, sw.splits, T, s.hidden, I_s, sw.a, sw.g, stream));
+    MOE_TRY(launch_shared_gemv(sw.a, shared->down, T, I_s, s.hidden, sw.y, stream));  // one split: I_s <= 512
+  } else {
+    MOE_TRY(launch_router_gemm(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, ws.status, stream));
+    MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, 1, T, s.hidden, I_s, sw.a, sw.g, stream));
+    MOE_TRY(launch_router_gemm(sw.a, shared->down, T, I_s, s.hidden, sw.y, ws.status, stream));
+  }
   // the routed experts, their combine and the shared expert's gated output
   MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT) {

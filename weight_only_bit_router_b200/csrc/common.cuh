@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -86,6 +87,20 @@ MOE_DEV float e4m3_to_f32(uint32_t b) {
 // NVFP4 block multiplier as bf16 bits: bf16_rne(fp32(e4m3(byte) * g)).
 MOE_DEV uint32_t nv_mult_bits(uint32_t scale_byte, float g) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e4m3_to_f32(scale_byte), g)));
+}
+
+// Multipliers of two adjacent NVFP4 blocks (scale bytes p[0], p[1]; p even)
+// as bf16x2 pairs with both halves equal: the hardware E4M3 -> f16
+// conversion is exact, f16 -> fp32 too, so this equals nv_mult_bits.
+MOE_DEV void nv_mult_pair(const uint8_t* p, float g, uint32_t& m0, uint32_t& m1) {
+  const uint16_t two = *reinterpret_cast<const uint16_t*>(p);
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+  const float f0 = __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
+  const float f1 = __half2float(__ushort_as_half(uint16_t(h2 >> 16)));
+  const float v0 = __fmul_rn(f0, g), v1 = __fmul_rn(f1, g);
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m0) : "f"(v0));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m1) : "f"(v1));
 }
 
 // E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the

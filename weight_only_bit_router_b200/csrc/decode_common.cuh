@@ -153,9 +153,7 @@ MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b
       rc.mult2 = rc.mult;
     } else if (FMT == MOE_FMT_NVFP4_G16) {
       // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
-      const uint32_t m0 = nv_mult_bits(scales[8 * b + 2 * q], g), m1 = nv_mult_bits(scales[8 * b + 2 * q + 1], g);
-      rc.mult = m0 | (m0 << 16);
-      rc.mult2 = m1 | (m1 << 16);
+      nv_mult_pair(scales + 8 * b + 2 * q, g, rc.mult, rc.mult2);
     } else {
       rc.mult = pow2_bf16x2(int(scales[4 * b + q]) - 127);  // the slice is one 32-element block
       rc.mult2 = rc.mult;

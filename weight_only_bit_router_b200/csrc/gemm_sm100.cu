@@ -425,10 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m2 = m;
               } else if (FMT == MOE_FMT_NVFP4_G16) {
                 // blocks of 16: (ks * 64 + 32 h) / 16 and the next one
-                const int blk = (ks * BK) / 16 + 2 * h;
-                const uint32_t b0 = nv_mult_bits(srow[blk], gsc), b1 = nv_mult_bits(srow[blk + 1], gsc);
-                m = b0 | (b0 << 16);
-                m2 = b1 | (b1 << 16);
+                nv_mult_pair(srow + (ks * BK) / 16 + 2 * h, gsc, m, m2);
               } else {
                 m = pow2x2(int(srow[(ks * BK) / 32 + h]) - 127);
                 m2 = m;

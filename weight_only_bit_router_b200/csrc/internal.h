@@ -134,8 +134,12 @@ cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_
 
 // shared.cu: the shared expert's SwiGLU and sigmoid gate from the fp32 gate_up
 // product h [T, 2 I_s]: a [T, I_s] bf16, g [T] fp32 (g = sigmoid(x . w_gate))
-cudaError_t launch_shared_swiglu_gate(const uint16_t* x, const uint16_t* w_gate, const float* h, int T, int H,
-                                      int I_s, uint16_t* a, float* g, cudaStream_t stream);
+cudaError_t launch_shared_swiglu_gate(const uint16_t* x, const uint16_t* w_gate, const float* h, int splits, int T,
+                                      int H, int I_s, uint16_t* a, float* g, cudaStream_t stream);
+// T <= 32: part [splits][T][N] fp32 = W [N][K] x [T][K]^T per 512-k split (N % 16 == 0, K % 64 == 0)
+int shared_gemv_splits(int K);
+cudaError_t launch_shared_gemv(const uint16_t* x, const uint16_t* w, int T, int K, int N, float* part,
+                               cudaStream_t stream);
 
 // selftest of the bounded device-side wait (api.cu)
 cudaError_t launch_bounded_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
