@@ -324,9 +324,9 @@ MOE_API size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_sh
  *   g_t   = sigmoid(x_t . w_gate)                     fp32
  *   a_s   = bf16(silu(W_gate_s x_t) * (W_up_s x_t))   (the routed experts' rounding)
  *   out_t = bf16( sum_j w_tj y_tj  +  g_t * (W_down_s a_s) )   one final rounding
- * The shared expert runs on the tensor cores (tcgen05) for every T; its
- * contribution is added to the routed combine in fp32 before the output's
- * single bf16 rounding.  Paths MOE_PATH_AUTO, _DECODE and _PREFILL; the
+ * The shared expert's products run on tcgen05 above 32 tokens and as a
+ * split-K mma.sync product up to 32; its contribution is added to the routed
+ * combine in fp32 before the output's single bf16 rounding.  Paths MOE_PATH_AUTO, _DECODE and _PREFILL; the
  * single-kernel path returns MOE_ERR_UNSUPPORTED.  Other arguments, errors
  * and the workspace rules as moe_forward (workspace >=
  * moe_workspace_bytes_shared bytes). */
