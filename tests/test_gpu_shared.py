@@ -55,7 +55,7 @@ def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
                                               a_exact, a_round)
     routed = o.down_and_combine(act_used, rid, rw, dnb, s.num_experts)
     sh_bits = [moe_synth.bf16_bits(t) for t in shared]
-    g, ys_oracle = o.shared_expert(xb, *sh_bits)
+    g, _ = o.shared_expert(xb, *sh_bits)
     assert np.all((g > 0.01) & (g < 0.99))  # the gate is not saturated on these inputs
     # the GPU's shared-expert activations, checked and used like the routed ones
     off = moe.moe_workspace_bytes(shape, T)
@@ -64,7 +64,6 @@ def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
     a_s_used, n_sh = flip_aware_activations(o.bf16_to_f64(moe_synth.bf16_bits(a_gpu)), a_s_exact,
                                             o.bf16_round(a_s_exact))
     ys = a_s_used @ o.bf16_to_f64(sh_bits[1]).T
-    assert np.allclose(ys, ys_oracle, rtol=1e-2, atol=1e-3 * np.sqrt(np.mean(ys_oracle ** 2)))
     ref = routed + g[:, None] * ys
     assert_out_close(out[tok_d], ref, f"{fmt} shared T={T} ({n_diff} routed activations rounded the other way)")
     # the shared expert changes the output: the routed-only oracle must not pass

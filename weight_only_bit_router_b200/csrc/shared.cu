@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "decode_common.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
@@ -46,6 +47,8 @@ __global__ void __launch_bounds__(128) shared_gemv_kernel(const uint16_t* __rest
                                                           const uint16_t* __restrict__ w, int T, int K, int N,
                                                           float* __restrict__ part) {
   __shared__ float red[4][NT][4][32];
+  pdl_wait();  // the previous kernel on the stream may still read `part`
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int n0 = blockIdx.x * 16;
   const int k = blockIdx.y * kSgK + warp * 128 + 32 * q;  // this lane's 32-k slice
@@ -92,6 +95,8 @@ __global__ void __launch_bounds__(256) shared_swiglu_gate_kernel(const uint16_t*
                                                                  const float* __restrict__ h, int splits, int T,
                                                                  int H, int I, uint16_t* __restrict__ a,
                                                                  float* __restrict__ g) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   for (int i = threadIdx.x; i < I; i += blockDim.x) {
     float hg = 0.f, hu = 0.f;
@@ -120,17 +125,15 @@ cudaError_t launch_shared_gemv(const uint16_t* x, const uint16_t* w, int T, int 
                                cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const dim3 grid(N / 16, shared_gemv_splits(K));
-  if (T <= 8) shared_gemv_kernel<1><<<grid, 128, 0, stream>>>(x, w, T, K, N, part);
-  else if (T <= 16) shared_gemv_kernel<2><<<grid, 128, 0, stream>>>(x, w, T, K, N, part);
-  else shared_gemv_kernel<4><<<grid, 128, 0, stream>>>(x, w, T, K, N, part);
-  return cudaGetLastError();
+  if (T <= 8) return launch_pdl(shared_gemv_kernel<1>, grid, dim3(128), 0, stream, x, w, T, K, N, part);
+  if (T <= 16) return launch_pdl(shared_gemv_kernel<2>, grid, dim3(128), 0, stream, x, w, T, K, N, part);
+  return launch_pdl(shared_gemv_kernel<4>, grid, dim3(128), 0, stream, x, w, T, K, N, part);
 }
 
 cudaError_t launch_shared_swiglu_gate(const uint16_t* x, const uint16_t* w_gate, const float* h, int splits, int T,
                                       int H, int I_s, uint16_t* a, float* g, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  shared_swiglu_gate_kernel<<<T, 256, 0, stream>>>(x, w_gate, h, splits, T, H, I_s, a, g);
-  return cudaGetLastError();
+  return launch_pdl(shared_swiglu_gate_kernel, dim3(T), dim3(256), 0, stream, x, w_gate, h, splits, T, H, I_s, a, g);
 }
 
 }  // namespace moe
