@@ -71,8 +71,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/prefill_gate_up_int4_T8192_ncu.md); workloads without a capture of
 # their dominant kernel report null.
 MEASURED_TRAFFIC = {
-    ("decode4", "gate_up"): 32.475904e6,
-    ("prefill", "gate_up"): 375.163392e6 + 57.828864e6,
+    ("decode4", "gate_up"): 32.480768e6 + 768.0,
+    ("prefill", "gate_up"): 375.213568e6 + 56.956672e6,
 }
 
 
