@@ -103,6 +103,37 @@ MOE_DEV void nv_mult_pair(const uint8_t* p, float g, uint32_t& m0, uint32_t& m1)
   asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m1) : "f"(v1));
 }
 
+// E2M1 nibbles i and i+4 of `w` -> bf16x2 bit patterns of (value * 2^-126),
+// exact: the magnitude code's three bits land on bf16 bits [8:6] (the two low
+// exponent bits and the first mantissa bit, so code 1 = 0.5 becomes the
+// subnormal 2^-127 and code (e, m) with e >= 1 the normal 2^(e-127) (1 + m/2)),
+// the sign bit on bit 15.  One bf16 multiply by (multiplier * 2^126) then
+// yields bf16(value * multiplier) with a single rounding.
+MOE_DEV uint32_t e2m1_pair_scaled(uint32_t w, int i) {
+  const uint32_t t = w >> (4 * i);
+  return ((t << 6) & 0x01C001C0u) | ((t << 12) & 0x80008000u);
+}
+constexpr uint32_t kBf16x2Pow126 = 0x7E807E80u;  // 2^126 in both halves
+
+// Like nv_mult_pair, but the multipliers come pre-scaled by 2^126 for
+// e2m1_pair_scaled codes (two = 0) whenever that is exact: both fp32 products
+// within [2^-126, 3.9), i.e. the bf16 rounding is in the normal range and the
+// scaled value stays finite; otherwise the plain multipliers (two = 1, and
+// the caller first multiplies the codes by 2^126).
+MOE_DEV void nv_mult_pair_scaled(const uint8_t* p, float g, uint32_t& m0, uint32_t& m1, uint32_t& two) {
+  const uint16_t pair = *reinterpret_cast<const uint16_t*>(p);
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+  const float v0 = __fmul_rn(__half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu))), g);
+  const float v1 = __fmul_rn(__half2float(__ushort_as_half(uint16_t(h2 >> 16))), g);
+  const bool fold = v0 >= 0x1p-126f && v0 < 3.9f && v1 >= 0x1p-126f && v1 < 3.9f;
+  const float sc = fold ? 0x1p126f : 1.0f;
+  const float a = __fmul_rn(v0, sc), b = __fmul_rn(v1, sc);
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m0) : "f"(a));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m1) : "f"(b));
+  two = fold ? 0u : 1u;
+}
+
 // E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the
 // nibble pair at bit offsets 0 and 16 of `w` after shifting by 4*i.
 // Magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; looked up with two byte permutes.

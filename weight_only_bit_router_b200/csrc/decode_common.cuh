@@ -35,10 +35,22 @@ MOE_DEV uint32_t pow2_bf16x2(int e) {
   return b | (b << 16);
 }
 
+// One bf16 pair (nibbles i, i+4 of `word`) times its multiplier.  E2M1 codes
+// enter as value * 2^-126 (e2m1_pair_scaled) and `mult` carries the 2^126
+// unless `two` is set, in which case the codes are first scaled back.
 template <int FMT>
-MOE_DEV uint32_t dq_pair(uint32_t word, int i, uint32_t mult) {
-  const uint32_t v = (FMT == MOE_FMT_INT4_G128) ? int4_pair(word, i) : e2m1_pair(word, i);
+MOE_DEV uint32_t dq_pair(uint32_t word, int i, uint32_t mult, uint32_t two = 0) {
+  if (FMT == MOE_FMT_INT4_G128) return bf16x2_mul(int4_pair(word, i), mult);
+  uint32_t v = e2m1_pair_scaled(word, i);
+  if (two) v = bf16x2_mul(v, kBf16x2Pow126);
   return bf16x2_mul(v, mult);
+}
+
+// MXFP4 multiplier of exponent e for dq_pair: 2^(e + 126) when that is a
+// bf16 value (e <= 1), else 2^e with the two-step flag.
+MOE_DEV void mx_mult(int e, uint32_t& mult, uint32_t& two) {
+  two = e > 1 ? 1u : 0u;
+  mult = pow2_bf16x2(two ? e : e + 126);
 }
 
 MOE_DEV uint32_t word_of(const uint4& c, int j) {
@@ -57,6 +69,7 @@ struct RowChunk {
   uint4 codes;
   uint32_t mult;   // bf16x2 multiplier: the INT4 scale, 2^e for MXFP4, or (NVFP4) the first 16-block's
   uint32_t mult2;  // NVFP4: the second 16-block's multiplier (code words 2 and 3); otherwise = mult
+  uint32_t two;    // E2M1 formats: 1 if the multipliers do not carry the 2^126 (see dq_pair)
 };
 
 template <int FMT>
@@ -69,12 +82,14 @@ MOE_DEV RowChunk smem_row_chunk(const uint8_t* codes, const uint8_t* scales, int
     if (FMT == MOE_FMT_INT4_G128) {
       const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[r * int4_groups(K) + k / 128];
       rc.mult = s | (s << 16);
+      rc.two = 0;
     } else {
-      rc.mult = pow2_bf16x2(int(scales[r * (K / 32) + k / 32]) - 127);
+      mx_mult(int(scales[r * (K / 32) + k / 32]) - 127, rc.mult, rc.two);
     }
   } else {
     rc.codes = make_uint4(0, 0, 0, 0);  // INT4 nibble 0 would be -8: zero the multiplier instead
     rc.mult = 0;
+    rc.two = 0;
   }
   rc.mult2 = rc.mult;
   return rc;
@@ -151,17 +166,19 @@ MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b
       const uint32_t sc = reinterpret_cast<const uint16_t*>(scales)[b];  // group b = k-block b
       rc.mult = sc | (sc << 16);
       rc.mult2 = rc.mult;
+      rc.two = 0;
     } else if (FMT == MOE_FMT_NVFP4_G16) {
       // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
-      nv_mult_pair(scales + 8 * b + 2 * q, g, rc.mult, rc.mult2);
+      nv_mult_pair_scaled(scales + 8 * b + 2 * q, g, rc.mult, rc.mult2, rc.two);
     } else {
-      rc.mult = pow2_bf16x2(int(scales[4 * b + q]) - 127);  // the slice is one 32-element block
+      mx_mult(int(scales[4 * b + q]) - 127, rc.mult, rc.two);  // the slice is one 32-element block
       rc.mult2 = rc.mult;
     }
   } else {
     rc.codes = make_uint4(0, 0, 0, 0);
     rc.mult = 0;
     rc.mult2 = 0;
+    rc.two = 0;
   }
   return rc;
 }
@@ -206,7 +223,7 @@ MOE_DEV void load_act_raw_cg(const uint16_t* rowp, int K, int kb, int q, bool va
 // One bf16 pair (nibbles i, i+4 of code word j) of a row chunk.
 template <int FMT>
 MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i, int j = 0) {
-  return dq_pair<FMT>(word, i, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? rc.mult2 : rc.mult);
+  return dq_pair<FMT>(word, i, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? rc.mult2 : rc.mult, rc.two);
 }
 
 // acc[4] += W(rows r, r+8; one 128-k block) x activation fragments.

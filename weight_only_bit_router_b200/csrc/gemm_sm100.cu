@@ -156,14 +156,22 @@ MOE_DEV uint32_t pow2x2(int e) {
 // Code words 0-1 use `mult`, words 2-3 `mult2` (the two 16-element NVFP4
 // blocks of the chunk; equal for the other formats).
 template <int FMT>
-MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint32_t mult2, uint8_t* tile, int r, int half) {
+MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint32_t mult2, uint32_t two, uint8_t* tile, int r,
+                             int half) {
   const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t P[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t v = (FMT == MOE_FMT_INT4_G128) ? int4_pair(w[j], i) : e2m1_pair(w[j], i);
+      uint32_t v;
+      if (FMT == MOE_FMT_INT4_G128) {
+        v = int4_pair(w[j], i);
+      } else {
+        // E2M1 codes as value * 2^-126; the multipliers carry 2^126 unless `two`
+        v = e2m1_pair_scaled(w[j], i);
+        if (two) v = bf16x2_mul(v, kBf16x2Pow126);
+      }
       P[i] = bf16x2_mul(v, j < 2 ? mult : mult2);  // (k+i, k+i+4)
     }
     uint4 o;
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < NACC; ++c) {
             const uint8_t* ctile = sC + (sc * NACC + c) * kCodeBytes + r * (BK / 2);
             const uint4 cw = *reinterpret_cast<const uint4*>(ctile + 16 * h);
-            uint32_t m = 0, m2 = 0;
+            uint32_t m = 0, m2 = 0, two = 0;
             if (valid) {
               const uint8_t* srow = srows + c * BM * kSrow;
               if (FMT == MOE_FMT_INT4_G128) {
@@ -425,13 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m2 = m;
               } else if (FMT == MOE_FMT_NVFP4_G16) {
                 // blocks of 16: (ks * 64 + 32 h) / 16 and the next one
-                nv_mult_pair(srow + (ks * BK) / 16 + 2 * h, gsc, m, m2);
+                nv_mult_pair_scaled(srow + (ks * BK) / 16 + 2 * h, gsc, m, m2, two);
               } else {
-                m = pow2x2(int(srow[(ks * BK) / 32 + h]) - 127);
+                const int e = int(srow[(ks * BK) / 32 + h]) - 127;
+                two = e > 1 ? 1u : 0u;
+                m = pow2x2(two ? e : e + 126);
                 m2 = m;
               }
             }
-            dequant_store32<FMT>(cw, m, m2, sA + (so * NACC + c) * kTileBytes, r, h);
+            dequant_store32<FMT>(cw, m, m2, two, sA + (so * NACC + c) * kTileBytes, r, h);
           }
           // this thread's bf16 stores before the tensor core reads them
           fence_proxy_async_smem();
