@@ -259,7 +259,8 @@ def load_peaks():
 
 # ---------------------------------------------------------------- CPU oracle timing
 
-def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, slots_per_token=None):
+def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, slots_per_token=None,
+                  shared=None):
     """Time the CPU oracle on a bounded sample of the workload.
 
     Inputs (bf16 weights of the touched experts, packed by the oracle's own
@@ -290,15 +291,19 @@ def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, 
         del gu_bf16, dn_bf16
         gu = o.PackedBank(fmt, gu_c, gu_s)
         dn = o.PackedBank(fmt, dn_c, dn_s)
+        sh = None if shared is None else [moe_synth.bf16_bits(t) for t in shared[l]]
         t0 = time.perf_counter()
-        o.forward(xb, router, b, gu, dn, k)
+        if sh is None:
+            o.forward(xb, router, b, gu, dn, k)
+        else:
+            o.forward_with_shared(xb, router, b, gu, dn, k, sh)
         elapsed += time.perf_counter() - t0
         done_tokens += ntok
         used_layers += 1
     threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
     desc = (f"CPU oracle (NumPy fp64) forward of {int(done_tokens)} token-layers "
             f"({used_layers} layer(s) x up to 16 tokens of this workload, cold dequantisation of every touched "
-            f"expert; packing untimed)")
+            f"expert{', the bf16 shared expert' if shared is not None else ''}; packing untimed)")
     return done_tokens / max(elapsed, 1e-9), desc, int(threads), elapsed
 
 
@@ -451,7 +456,7 @@ def run_ours(args, rank, local, world):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, threads, secs = oracle_sample(stack, x, stack.bias, T, budget_s=args.cpu_budget)
+        v, desc, threads, secs = oracle_sample(stack, x, stack.bias, T, budget_s=args.cpu_budget, shared=shared)
         cpu = {"value": v, "unit": "layer-tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": secs}
 
@@ -492,8 +497,9 @@ def run_reference(args, rank, world):
         return None
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
-    fmt_name, T, zipf, _ = WORKLOADS[args.workload]
+    fmt_name, T, zipf, layers_per_step = WORKLOADS[args.workload]
     fmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[fmt_name]
+    inter_sh = SHARED_INTER.get(args.workload)
     s = moe_synth.NEX
     n_layers = 2
     prepared = []
@@ -511,16 +517,21 @@ def run_reference(args, rank, world):
         gu_p = {e: o.pack(fmt, moe_synth.bf16_bits(gu[e])) for e in touched}
         dn_p = {e: o.pack(fmt, moe_synth.bf16_bits(dn[e])) for e in touched}
         del gu, dn
-        prepared.append((router, b, x, gu_p, dn_p))
+        sh = ([moe_synth.bf16_bits(t) for t in moe_synth.shared_expert(s, inter_sh, seed, gen_dev)]
+              if inter_sh else None)
+        prepared.append((router, b, x, gu_p, dn_p, sh))
     budget = 150.0 / max(1, args.steps + args.warmup)
 
     def one_step(i):
-        router, b, x, gu_p, dn_p = prepared[i % n_layers]
+        router, b, x, gu_p, dn_p, sh = prepared[i % n_layers]
         t = i % x.shape[0]
         gu = o.PackedBank(fmt, {e: v[0] for e, v in gu_p.items()}, {e: v[1] for e, v in gu_p.items()})
         dn = o.PackedBank(fmt, {e: v[0] for e, v in dn_p.items()}, {e: v[1] for e, v in dn_p.items()})
         t0 = time.perf_counter()
-        o.forward(x[t:t + 1], router, b, gu, dn, s.top_k)
+        if sh is None:
+            o.forward(x[t:t + 1], router, b, gu, dn, s.top_k)
+        else:
+            o.forward_with_shared(x[t:t + 1], router, b, gu, dn, s.top_k, sh)
         return time.perf_counter() - t0
 
     for i in range(args.warmup):
@@ -535,13 +546,16 @@ def run_reference(args, rank, world):
     value = steps_done / total
     threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
     sample = ("CPU oracle (NumPy fp64) forward of one token of one layer per step (router, top-k, cold "
-              f"dequantisation of its {s.top_k} experts, SwiGLU, combine); packing untimed")
+              f"dequantisation of its {s.top_k} experts, SwiGLU, combine"
+              f"{', the bf16 shared expert' if inter_sh else ''}); packing untimed")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world,
         "steps": steps_done, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, steps_done),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
-        "config": {"workload": f"nex_moe_{fmt_name}_T{T}{'_zipf' if zipf else ''}", "hidden": s.hidden,
+        "config": {"workload": f"nex_moe_{fmt_name}_T{T}{'_zipf' if zipf else ''}"
+                               f"{f'_shared{inter_sh}' if inter_sh else ''}_{layers_per_step}layer_step_"
+                               f"of_{NUM_LAYERS}layer_stack", "hidden": s.hidden,
                    "experts": s.num_experts, "top_k": s.top_k, "inter": s.inter, "tokens_per_layer": T},
         "cpu_baseline": {"value": value, "unit": "layer-tokens/s", "cores": int(threads), "kind": "oracle",
                          "sample": sample},

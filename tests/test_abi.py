@@ -78,6 +78,39 @@ def test_pack_rejects_null_and_bad_k_without_a_gpu():
     assert L.moe_dequant(None, 1, 1, 1, 64, 16, None) == 1
 
 
+def test_new_packers_reject_bad_arguments_without_a_gpu():
+    L = moe.lib()
+    assert L.moe_pack_nvfp4(None, 1, 1, 64, 256, None, None) == 1
+    assert L.moe_pack_nvfp4(16, 1, 1, 48, 256, None, None) == 1        # K % 32
+    assert L.moe_pack_mxfp4_rule(16, 1, 1, 64, 256, None, 4, None) == 1  # unknown rule
+    assert L.moe_pack_mxfp4_rule(16, 1, 1, 64, 255, None, 3, None) == 1  # misaligned output
+    assert L.moe_bank_bytes(3, 1, 1, 48) == 0                           # NVFP4 K % 32
+
+
+def test_forward_shared_validation_happens_on_the_host():
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    ws_plain = moe.moe_workspace_bytes(s, 4)
+    ws_sh = moe.moe_workspace_bytes_shared(s, 512, 4)
+    assert ws_sh > ws_plain
+    assert moe.moe_workspace_bytes_shared(s, 500, 4) == 0               # I_s % 64
+    assert moe.moe_workspace_bytes_shared(s, 0, 4) == 0
+    L = moe.lib()
+    sh = moe.SharedExpert(512, 256, 256, 256)
+    def call(shared=ctypes.byref(sh), ws=4096, wsb=None, opts=None, T=4):
+        return L.moe_forward_shared(ctypes.byref(s), shared, 256, T, 256, None, 256, 512, ws,
+                                    ws_sh if wsb is None else wsb, 256, opts, None)
+    assert call(shared=None) == 1
+    assert call(wsb=ws_plain) == 3                                       # the routed workspace is too small
+    bad = moe.SharedExpert(96, 256, 256, 256)
+    assert call(shared=ctypes.byref(bad)) == 2                           # I_s not a multiple of 64
+    unaligned = moe.SharedExpert(512, 258, 256, 256)
+    assert call(shared=ctypes.byref(unaligned)) == 1
+    o = moe.ForwardOpts()
+    o.path = moe.MOE_PATH_FUSED
+    assert call(opts=ctypes.byref(o)) == 2                               # no single-kernel path
+    assert call(T=0) == 0                                                # nothing to do
+
+
 def test_route_and_permute_validation():
     L = moe.lib()
     assert L.moe_route(16, None, 4, 256, 33, 16, 16, None) == 2        # k > 32

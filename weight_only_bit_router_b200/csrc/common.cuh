@@ -134,24 +134,6 @@ MOE_DEV void nv_mult_pair_scaled(const uint8_t* p, float g, uint32_t& m0, uint32
   two = fold ? 0u : 1u;
 }
 
-// E2M1 nibble (sign<<3 | magnitude code) -> bf16 bits of its value, for the
-// nibble pair at bit offsets 0 and 16 of `w` after shifting by 4*i.
-// Magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; looked up with two byte permutes.
-MOE_DEV uint32_t e2m1_pair(uint32_t w, int i) {
-  // high bytes of bf16(m) for m = code 0..7: 00 3F 3F 3F 40 40 40 40
-  // low bytes:                                00 00 80 C0 00 40 80 C0
-  const uint32_t hi0 = 0x3F3F3F00u, hi1 = 0x40404040u;
-  const uint32_t lo0 = 0xC0800000u, lo1 = 0xC0804000u;
-  const uint32_t s = w >> (4 * i);
-  // selector: code of the low element in nibble 0, of the high element in nibble 1
-  const uint32_t sel = (s & 0x7u) | ((s >> 12) & 0x70u);
-  const uint32_t hi = prmt(hi0, hi1, sel);   // bytes: hi(c0), hi(c1), ...
-  const uint32_t lo = prmt(lo0, lo1, sel);
-  uint32_t v = prmt(lo, hi, 0x5140u);        // lo(c0) hi(c0) lo(c1) hi(c1)
-  const uint32_t sign = ((s << 12) & 0x8000u) | ((s << 12) & 0x80000000u);
-  return v | sign;
-}
-
 // --------------------------------------------------------------------------
 // shared-memory addresses, fences
 // --------------------------------------------------------------------------
