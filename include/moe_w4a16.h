@@ -31,9 +31,12 @@
  *     bit patterns.
  *   - Nothing allocates device memory: scratch comes from a caller-provided
  *     workspace whose size a query function returns.
- *   - Calls only enqueue work on `stream` (asynchronous, no host sync) and
- *     keep no global mutable state, so they are reentrant across streams as
- *     long as workspaces are not shared.
+ *   - Calls only enqueue work on `stream` (asynchronous, no host sync); the
+ *     only process-wide state is a set of thread-safe caches of launch
+ *     parameters (SM count, occupancy, kernel attributes), so calls are
+ *     reentrant across host threads and streams as long as workspaces are not
+ *     shared.  (moe_workspace_status synchronises its stream; the no-alloc
+ *     entry point shares one scratch array, see there.)
  *   - Argument errors are detected on the host before anything is enqueued
  *     and leave every output untouched.
  */

@@ -11,6 +11,8 @@
 // to 8 tokens per tile.
 // (The fragment k-permutation is described in decode_common.cuh.)
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -427,12 +429,13 @@ size_t down_smem(int fmt, int K, int T, int act_rows) {
 constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving room for static
 
 int sm_count_cached() {
-  static int n = 0;
+  static std::atomic<int> cached{0};
+  int n = cached.load(std::memory_order_relaxed);
   if (!n) {
     int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached.store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -449,6 +452,9 @@ int persistent_grid(Kern k, size_t smem, int units, int threads) {
     int per_sm;
   };
   static Entry cache[16] = {};
+  static std::mutex mu;  // host threads may launch concurrently
+  const int sms = sm_count_cached();
+  std::lock_guard<std::mutex> lock(mu);
   const void* fn = reinterpret_cast<const void*>(k);
   int per_sm = 0;
   for (const Entry& e : cache)
@@ -462,7 +468,7 @@ int persistent_grid(Kern k, size_t smem, int units, int threads) {
         break;
       }
   }
-  return std::max(1, std::min(units, per_sm * sm_count_cached()));
+  return std::max(1, std::min(units, per_sm * sms));
 }
 
 template <typename Kern>

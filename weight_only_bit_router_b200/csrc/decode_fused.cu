@@ -56,6 +56,8 @@
 #include "launch.h"
 #include "topk_common.cuh"
 
+#include <mutex>
+
 namespace moe {
 
 namespace {
@@ -742,9 +744,11 @@ cudaError_t fused_launch(const FusedArgs& args, cudaStream_t stream) {
   static FusedPlan plan;
   static int plan_stage_bytes = -1;
   static int plan_dev = -1;
+  static std::mutex mu;  // host threads may launch concurrently
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  std::unique_lock<std::mutex> lock(mu);
   if (plan_stage_bytes != args.stage_bytes || plan_dev != dev) {
     int sms = 0, max_optin = 0;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
@@ -770,9 +774,11 @@ cudaError_t fused_launch(const FusedArgs& args, cudaStream_t stream) {
     plan_stage_bytes = args.stage_bytes;
     plan_dev = dev;
   }
+  const FusedPlan use = plan;
+  lock.unlock();
   FusedArgs a = args;
-  a.stages = plan.stages;
-  return launch_cooperative(kern, dim3(plan.grid), dim3(kFuThreads), plan.smem, stream, a);
+  a.stages = use.stages;
+  return launch_cooperative(kern, dim3(use.grid), dim3(kFuThreads), use.smem, stream, a);
 }
 
 }  // namespace

@@ -32,6 +32,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -563,13 +564,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load();
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cached.store(fn);
+    }
   }
   return fn;
 }
@@ -601,12 +605,13 @@ bool make_bf16_sw128_map(CUtensorMap* m, const uint16_t* base, int K, int rows) 
 }
 
 int sm_count() {
-  static int n = 0;
+  static std::atomic<int> cached{0};
+  int n = cached.load(std::memory_order_relaxed);
   if (!n) {
     int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached.store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -616,13 +621,13 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ct
   auto kern = grouped_gemm_kernel<MODE, FMT>;
   const int smem = Cfg<MODE, FMT>::SMEM;
   // once per process (and per device), outside any stream capture of later calls
-  static int configured_device = -1;
+  static std::atomic<int> configured_device{-1};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  if (configured_device.load() != dev) {  // setting it twice from two threads is harmless
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    configured_device = dev;
+    configured_device.store(dev);
   }
   const int grid = max(1, min(sm_count(), max_ctas));
   kern<<<grid, kThreads, smem, stream>>>(map, args);

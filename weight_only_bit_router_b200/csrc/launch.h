@@ -6,6 +6,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <utility>
 
 namespace moe {
@@ -32,7 +33,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 template <typename... KArgs, typename... Args>
 cudaError_t launch_cooperative(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                                Args&&... args) {
-  static int with_pdl = 1;  // cleared once the driver refuses the combination
+  static std::atomic<int> with_pdl{1};  // cleared once the driver refuses the combination
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -44,11 +45,11 @@ cudaError_t launch_cooperative(void (*kern)(KArgs...), dim3 grid, dim3 block, si
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = with_pdl ? 2 : 1;
+  cfg.numAttrs = with_pdl.load() ? 2 : 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-  if (err != cudaSuccess && with_pdl) {
+  if (err != cudaSuccess && cfg.numAttrs == 2) {
     (void)cudaGetLastError();
-    with_pdl = 0;
+    with_pdl.store(0);
     cfg.numAttrs = 1;
     err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   }
