@@ -325,8 +325,7 @@ def run_ours(args, rank, local, world):
     ws = moe.alloc_workspace_shared(shape, inter_sh, T, device) if inter_sh else moe.alloc_workspace(shape, T, device)
     outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
-    path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL,
-            "fused": moe.MOE_PATH_FUSED}[args.path]
+    path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL}[args.path]
 
     def layer_call(l, events=None):
         fwd = (lambda *a, **k: moe.moe_forward_shared(shape, shared[l], *a, **k)) if shared else \
@@ -573,7 +572,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode4")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", choices=["auto", "decode", "prefill", "fused"], default="auto",
+    ap.add_argument("--path", choices=["auto", "decode", "prefill"], default="auto",
                     help="kernel path of moe_forward (auto: decode kernels up to 32 tokens, grouped GEMMs above)")
     ap.add_argument("--stack-layers", type=int, default=NUM_LAYERS,
                     help="layers in the packed stack (smaller only for profiling captures)")

@@ -248,19 +248,16 @@ typedef enum {
   MOE_PATH_AUTO = 0,      /* decode path for T <= 32, grouped tcgen05 GEMMs above */
   MOE_PATH_DECODE = 1,    /* weight-streaming GEMV kernels (any T; meant for T <= 32: above that
                              the down projection re-streams its weights per 32 tokens) */
-  MOE_PATH_PREFILL = 2,   /* grouped tcgen05 GEMMs (any T >= 1) */
-  MOE_PATH_FUSED = 3      /* the whole layer as ONE persistent cooperative kernel (every CTA
-                             resident at once): 1 <= T <= 8, H <= 2048, I <= 512, H % 64 == 0;
-                             MOE_ERR_UNSUPPORTED otherwise */
+  MOE_PATH_PREFILL = 2    /* grouped tcgen05 GEMMs (any T >= 1) */
 } moe_path_t;
 
 /* Number of timed stages moe_forward reports through stage_events. */
 #define MOE_NUM_STAGES 5
 /* Stage ids: 0 router logits, 1 top-k + permutation, 2 gate_up + SwiGLU,
- * 3 down projection, 4 weighted combine / output conversion.  When the layer
- * runs as a single kernel (moe_forward_launch_count() == 1) stage 0's
- * "before" event precedes that kernel and every other event follows it:
- * stage 0 then times the whole layer and stages 1-4 read zero. */
+ * 3 down projection, 4 weighted combine / output conversion.  Where one
+ * kernel does two stages (small batches: routing and permutation in one, down
+ * projection and combine in one) the second stage's events bracket nothing
+ * and it reads zero. */
 
 /* Optional extras of moe_forward / moe_forward_routed.  Every pointer may be
  * NULL; a NULL opts pointer means all defaults. */
@@ -329,10 +326,9 @@ MOE_API size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_sh
  *   out_t = bf16( sum_j w_tj y_tj  +  g_t * (W_down_s a_s) )   one final rounding
  * The shared expert's products run on tcgen05 above 32 tokens and as a
  * split-K mma.sync product up to 32; its contribution is added to the routed
- * combine in fp32 before the output's single bf16 rounding.  Paths MOE_PATH_AUTO, _DECODE and _PREFILL; the
- * single-kernel path returns MOE_ERR_UNSUPPORTED.  Other arguments, errors
- * and the workspace rules as moe_forward (workspace >=
- * moe_workspace_bytes_shared bytes). */
+ * combine in fp32 before the output's single bf16 rounding.  Other
+ * arguments, paths, errors and the workspace rules as moe_forward (workspace
+ * >= moe_workspace_bytes_shared bytes). */
 MOE_API moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_expert_t* shared,
                                 const uint16_t* x, int T, const uint16_t* router_w,
                                 const float* logit_bias, const void* gate_up_packed,
@@ -358,20 +354,27 @@ MOE_API int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t
 MOE_API moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* moe_forward for callers that cannot allocate device memory.  The model
- * cards have no counterpart to this entry point; it exists for callers that
- * record their GPU work ahead of time and replay it (a captured CUDA graph, a
- * pre-built command buffer), where a cudaMalloc inside the recorded region is
- * not possible, and for runtimes or plugins that reserve all device memory
- * up front or do not own the allocator.  The caller passes only inputs and
- * outputs (same meaning, layout and alignment as moe_forward); the scratch
- * is a fixed array inside the library (moe_noalloc_scratch_bytes(), 8 MiB),
- * held by every GPU that loads the library until the process exits.
+ * cards have no counterpart to this entry point.  It serves code that may
+ * not call cudaMalloc while it issues its work: runtimes and inference
+ * engines that reserve their whole device-memory budget at start-up, plugins
+ * whose host framework owns the device allocator, and code that records its
+ * GPU work for later replay, where an allocation inside the recorded region
+ * is not allowed.  The caller passes only inputs and outputs (same meaning,
+ * layout and alignment as moe_forward); the scratch is a fixed array inside
+ * the library (moe_noalloc_scratch_bytes(), 8 MiB), held by every GPU that
+ * loads the library until the process exits.
  *   - Returns MOE_ERR_UNSUPPORTED when moe_workspace_bytes(shape, T) exceeds
- *     that size (e.g. large prefill batches); nothing is enqueued then.
- *   - The first call on a device looks up the array's device address; make
- *     that first call before any stream capture.
- *   - Calls on one device share the array: each clears its status/counter
- *     region, and calls that overlap on the GPU (unordered streams) race.
+ *     that size (e.g. large prefill batches), MOE_ERR_INVALID_ARG for the
+ *     argument errors of moe_forward; nothing is enqueued then.
+ *   - The first call on a device (and the first after that device's context
+ *     was re-created, e.g. by cudaDeviceReset) looks up the array's device
+ *     address; make that first call before any stream capture.
+ *   - Calls on one device share the array and it keeps the last call's
+ *     contents: each call clears the device counters it needs at zero, and
+ *     calls that overlap on the GPU (unordered streams) race.
+ *   - An expired bounded device wait is recorded in the array's status word,
+ *     which later calls leave set (while it is set, their device-wide waits
+ *     give up at once); moe_noalloc_status reports and clears it.
  *   - No device allocation and no freeing happen inside this call. */
 MOE_API moe_status_t moe_forward_noalloc(const moe_shape_t* shape, const uint16_t* x, int T,
                                          const uint16_t* router_w, const float* logit_bias,
@@ -381,12 +384,20 @@ MOE_API moe_status_t moe_forward_noalloc(const moe_shape_t* shape, const uint16_
 /* Size in bytes of moe_forward_noalloc's fixed scratch array. */
 MOE_API size_t moe_noalloc_scratch_bytes(void);
 
+/* Synchronises `stream`, then reports MOE_ERR_TIMEOUT if a bounded device
+ * wait of a moe_forward_noalloc call on the current device expired since the
+ * last report (and clears the status word and the device counters of the
+ * scratch array), MOE_OK otherwise.  Allocates nothing. */
+MOE_API moe_status_t moe_noalloc_status(cudaStream_t stream);
+
 /* Self-test of the bounded device-side wait: launches one warp that waits on
  * a barrier nothing ever arrives at, gives up after `limit_ns` nanoseconds of
  * device time (at most 10 s) and raises the workspace status word, so that a
- * following moe_workspace_status returns MOE_ERR_TIMEOUT.  The GPU context
- * stays usable.  No counterpart on the model cards: this checks the library's
- * own failure reporting. */
+ * following moe_workspace_status returns MOE_ERR_TIMEOUT.  With workspace ==
+ * NULL it raises the status word of moe_forward_noalloc's scratch array on
+ * the current device instead (reported by moe_noalloc_status).  The GPU
+ * context stays usable.  No counterpart on the model cards: this checks the
+ * library's own failure reporting. */
 MOE_API moe_status_t moe_selftest_bounded_wait(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
                                        cudaStream_t stream);
 

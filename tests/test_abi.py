@@ -106,8 +106,8 @@ def test_forward_shared_validation_happens_on_the_host():
     unaligned = moe.SharedExpert(512, 258, 256, 256)
     assert call(shared=ctypes.byref(unaligned)) == 1
     o = moe.ForwardOpts()
-    o.path = moe.MOE_PATH_FUSED
-    assert call(opts=ctypes.byref(o)) == 2                               # no single-kernel path
+    o.path = 3
+    assert call(opts=ctypes.byref(o)) == 1                               # unknown path
     assert call(T=0) == 0                                                # nothing to do
 
 
@@ -144,13 +144,7 @@ def test_forward_validation_happens_on_the_host():
     assert L.moe_forward(*a) == 1
     # T == 0 is a valid no-op
     assert L.moe_forward(*args(T=0)) == 0
-    # the single-kernel path takes at most 8 tokens
-    opts.path = moe.MOE_PATH_FUSED
-    a = args(T=9)
-    a[10] = ctypes.byref(opts)
-    assert L.moe_forward(*a) == 2
-    assert moe.moe_forward_launch_count(s, 9, moe.MOE_PATH_FUSED, False) == -1
-    assert moe.moe_forward_launch_count(s, 8, moe.MOE_PATH_FUSED, False) == 1
+    assert moe.moe_forward_launch_count(s, 4, 3, False) == -1     # unknown path
 
 
 def test_routed_forward_validation():
@@ -165,6 +159,28 @@ def test_workspace_status_validation():
     assert L.moe_workspace_status(None, 256, None) == 3
     assert L.moe_workspace_init(256, 100, None) == 3
     assert L.moe_selftest_bounded_wait(256, 256, 11 * 10**9, None) == 1
+    assert L.moe_selftest_bounded_wait(None, 0, 11 * 10**9, None) == 1
+    assert L.moe_selftest_bounded_wait(256, 100, 1000, None) == 3
+
+
+def test_noalloc_validation_happens_before_anything_is_enqueued():
+    """Argument errors of moe_forward_noalloc come back before it touches
+    the device (no GPU here: a call that got past the checks would fail with
+    MOE_ERR_CUDA instead)."""
+    L = moe.lib()
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    args = lambda **kw: [ctypes.byref(kw.get("shape", s)), kw.get("x", 256), kw.get("T", 4), kw.get("r", 256),
+                         kw.get("bias", None), kw.get("gu", 256), kw.get("dn", 256), kw.get("out", 256), None]
+    assert L.moe_forward_noalloc(*args(x=None)) == 1
+    assert L.moe_forward_noalloc(*args(x=8)) == 1
+    assert L.moe_forward_noalloc(*args(r=None)) == 1
+    assert L.moe_forward_noalloc(*args(bias=2)) == 1       # bias not 4-byte aligned
+    assert L.moe_forward_noalloc(*args(gu=512 + 16)) == 1
+    assert L.moe_forward_noalloc(*args(out=None)) == 1
+    assert L.moe_forward_noalloc(*args(T=-1)) == 1
+    assert L.moe_forward_noalloc(*args(shape=moe.make_shape(2048, 500, 256, 8, "int4_g128"))) == 2
+    assert L.moe_forward_noalloc(*args(T=8192)) == 2       # workspace beyond the fixed scratch
+    assert L.moe_forward_noalloc(*args(T=0)) == 0
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -11,8 +11,9 @@ import torch
 import moe_synth
 import weight_only_bit_router_b200 as moe
 from oracle import moe_oracle as o
-from parity_util import (FMT_NAMES, LazyOracleBank, assert_out_close, assert_routing_consistent,
-                         flip_aware_activations, out_tolerance_report, record_parity)
+from parity_util import (FMT_NAMES, LazyOracleBank, assert_layer_parity, assert_out_close,
+                         assert_routing_consistent, flip_allowance, flip_aware_activations, out_tolerance_report,
+                         record_parity)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -152,12 +153,14 @@ def test_permute_bit_exact(T, E, k):
 
 # ---------------------------------------------------------------- layer forward
 
-def run_forward(layer, fmt, path=None, routed=None):
+def run_forward(layer, fmt, path=None, routed=None, packed=None):
+    """moe_forward (or moe_forward_routed) of a layer with every debug output;
+    `packed` = (gate_up, down) banks already packed on the GPU, else they are
+    packed here."""
     s = layer.shape
     shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
     T = layer.x.shape[0]
-    gu = pack_gpu(fmt, layer.gate_up)
-    dn = pack_gpu(fmt, layer.down)
+    gu, dn = packed if packed is not None else (pack_gpu(fmt, layer.gate_up), pack_gpu(fmt, layer.down))
     ws = moe.alloc_workspace(shape, T)
     dbg = {
         "logits_out": torch.empty(T, s.num_experts, dtype=torch.float32, device=DEV),
@@ -190,16 +193,26 @@ def gpu_activations_in_oracle_order(dbg, tok, rid, E, k):
     return act[pos[gpu_rows]]
 
 
-def check_layer(layer, fmt, path=None, sample=None):
+def check_layer(layer, fmt, path=None, sample=None, name="", packed=None):
     """Full forward on the GPU; the oracle recomputes the (sampled) tokens.
 
     Routing is checked bit-exact on the GPU's own fp32 logits, which must agree
-    with the oracle's to fp32 accumulation error.  The bf16 SwiGLU activations
-    must equal the oracle's except at rounding ties (see
-    flip_aware_activations); the output is compared, per element, with the
-    oracle's down projection and combine of those activations."""
+    with the oracle's to fp32 accumulation error.  The layer output is held to
+    |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref) against the oracle's own layer
+    (its own bf16 activation rounding, no GPU value): exactly for tokens whose
+    bf16 SwiGLU activations all equal the oracle's, and up to the flip
+    allowance (parity_util.flip_allowance) for tokens where fp32 accumulation
+    put an activation across a bf16 rounding boundary.  Each such activation is
+    itself checked to be a correct rounding (flip_aware_activations), and the
+    output of those tokens is also checked stage-wise: against the oracle's down
+    projection and combine of the activations the GPU chose."""
+    out, dbg = run_forward(layer, fmt, path, packed=packed)
+    return verify_layer(layer, fmt, out, dbg, path, sample, name)
+
+
+def verify_layer(layer, fmt, out, dbg, path=None, sample=None, name=""):
+    """The checks of check_layer on a forward's output and debug outputs."""
     s = layer.shape
-    out, dbg = run_forward(layer, fmt, path)
     T = layer.x.shape[0]
     tok = np.arange(T) if sample is None else np.asarray(sample)
     tok_d = torch.as_tensor(tok, device=DEV)
@@ -208,7 +221,7 @@ def check_layer(layer, fmt, path=None, sample=None):
     ref_logits = o.router_logits(xb, moe_synth.bf16_bits(layer.router_w))
     gpu_logits = dbg["logits_out"][tok_d]
     gpu_ids = dbg["topk_ids_out"][tok_d]
-    assert_routing_consistent(gpu_logits, ref_logits, gpu_ids, bias, s.top_k)
+    n_near_ties = assert_routing_consistent(gpu_logits, ref_logits, gpu_ids, bias, s.top_k)
     rid, rw = o.route(gpu_logits.cpu().numpy(), bias, s.top_k)
     assert np.array_equal(rid, gpu_ids.cpu().numpy())
     gw = dbg["topk_w_out"][tok_d].cpu().numpy().astype(np.float64)
@@ -222,19 +235,20 @@ def check_layer(layer, fmt, path=None, sample=None):
     a_exact, a_round = o.expert_activations(xb, rid, gu, s.num_experts)
     gpu_act = gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k)
     act_used, n_diff = flip_aware_activations(gpu_act, a_exact, a_round)
-    ref_out = o.down_and_combine(act_used, rid, rw, dn, s.num_experts)
-    assert_out_close(out[tok_d], ref_out, f"{fmt} T={T} ({n_diff} activations rounded the other way)")
-    # recorded, not asserted: the output against the oracle's own activation
-    # rounding (differs where fp32 accumulation put an activation across a bf16
-    # rounding boundary)
+    out_sel = out[tok_d]
+    # the layer against the pure oracle
     pure = o.down_and_combine(a_round, rid, rw, dn, s.num_experts)
-    n_bad, worst = out_tolerance_report(out[tok_d], pure)
-    _, worst_stage = out_tolerance_report(out[tok_d], ref_out)
-    record_parity(dict(fmt=fmt, T=T, path=int(path or 0), shape=[s.hidden, s.inter, s.num_experts, s.top_k],
-                       sampled_tokens=int(tok.size), activations=int(gpu_act.size),
-                       activations_rounded_other_way=n_diff, stagewise_worst_ratio=worst_stage,
-                       end_to_end_outside=n_bad, end_to_end_elements=int(pure.size),
-                       end_to_end_worst_ratio=worst))
+    allow, flipped = flip_allowance(gpu_act, a_exact, a_round, rid, rw, dn, s.num_experts)
+    what = f"{fmt} T={T} path={int(path or 0)} ({n_diff} activations rounded the other way)"
+    summary = assert_layer_parity(out_sel, pure, allow, flipped, what)
+    # stage-wise: the down projection and combine of the GPU's own activations
+    ref_stage = o.down_and_combine(act_used, rid, rw, dn, s.num_experts)
+    assert_out_close(out_sel, ref_stage, what + " stage-wise")
+    _, worst_stage = out_tolerance_report(out_sel, ref_stage)
+    record_parity(dict(case=name or f"{fmt}_T{T}", fmt=fmt, T=T, path=int(path or 0),
+                       shape=[s.hidden, s.inter, s.num_experts, s.top_k], sampled_tokens=int(tok.size),
+                       routing_near_ties=n_near_ties, activations=int(gpu_act.size),
+                       activations_rounded_other_way=n_diff, stagewise_worst_ratio=worst_stage, **summary))
     return out
 
 

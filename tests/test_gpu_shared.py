@@ -2,13 +2,16 @@
 oracle, through the C ABI (needs a B200).
 
 Per element |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref), ref = the oracle's
-routed combine of the GPU's own bf16 activations plus the oracle's gated
-shared expert on the GPU's own shared-expert activations: where fp32
-accumulation put an activation across a bf16 rounding boundary both
-neighbours are correct (parity_util.flip_aware_activations checks each such
-activation against the exact value).  The shared expert's bf16 activations
-are read from their place in the workspace, right after the routed layer's
-part (at offset moe_workspace_bytes).
+own layer: its routed combine plus its gated shared expert, each with the
+oracle's own bf16 activation rounding.  Tokens where fp32 accumulation put a
+routed or shared activation across a bf16 rounding boundary (both neighbours
+are correct, parity_util.flip_aware_activations checks each against the exact
+value) may exceed the bound by at most the flips' own effect on the output
+(parity_util.flip_allowance, and the same bound for the shared expert's down
+projection scaled by its gate); their output is also checked stage-wise
+against the oracle's down projections of the GPU's own activations.  The
+shared expert's bf16 activations are read from their place in the workspace,
+right after the routed layer's part (at offset moe_workspace_bytes).
 """
 import numpy as np
 import pytest
@@ -17,7 +20,8 @@ import torch
 import moe_synth
 import weight_only_bit_router_b200 as moe
 from oracle import moe_oracle as o
-from parity_util import LazyOracleBank, assert_out_close, assert_routing_consistent, flip_aware_activations
+from parity_util import (LazyOracleBank, assert_layer_parity, assert_out_close, assert_routing_consistent,
+                         bf16_ulp, flip_allowance, flip_aware_activations, record_parity)
 from test_gpu_parity import DEV, gpu_activations_in_oracle_order, pack_gpu
 
 pytestmark = pytest.mark.gpu
@@ -51,21 +55,38 @@ def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
     assert np.array_equal(rid, dbg["topk_ids_out"][tok_d].cpu().numpy())
     gub, dnb = LazyOracleBank(fmt, layer.gate_up), LazyOracleBank(fmt, layer.down)
     a_exact, a_round = o.expert_activations(xb, rid, gub, s.num_experts)
-    act_used, n_diff = flip_aware_activations(gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k),
-                                              a_exact, a_round)
+    gpu_act = gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k)
+    act_used, n_diff = flip_aware_activations(gpu_act, a_exact, a_round)
     routed = o.down_and_combine(act_used, rid, rw, dnb, s.num_experts)
     sh_bits = [moe_synth.bf16_bits(t) for t in shared]
     g, _ = o.shared_expert(xb, *sh_bits)
     assert np.all((g > 0.01) & (g < 0.99))  # the gate is not saturated on these inputs
-    # the GPU's shared-expert activations, checked and used like the routed ones
+    # the GPU's shared-expert activations, checked like the routed ones
     off = moe.moe_workspace_bytes(shape, T)
     a_gpu = ws[off:off + T * inter_shared * 2].view(torch.bfloat16).view(T, inter_shared)[tok_d]
+    a_gpu = o.bf16_to_f64(moe_synth.bf16_bits(a_gpu))
     a_s_exact = o.swiglu_exact(o.bf16_to_f64(xb), o.bf16_to_f64(sh_bits[0]))
-    a_s_used, n_sh = flip_aware_activations(o.bf16_to_f64(moe_synth.bf16_bits(a_gpu)), a_s_exact,
-                                            o.bf16_round(a_s_exact))
-    ys = a_s_used @ o.bf16_to_f64(sh_bits[1]).T
-    ref = routed + g[:, None] * ys
-    assert_out_close(out[tok_d], ref, f"{fmt} shared T={T} ({n_diff} routed activations rounded the other way)")
+    a_s_round = o.bf16_round(a_s_exact)
+    a_s_used, n_sh = flip_aware_activations(a_gpu, a_s_exact, a_s_round)
+    wd_s = o.bf16_to_f64(sh_bits[1])
+    out_sel = out[tok_d]
+    what = f"{fmt} shared T={T} ({n_diff} routed, {n_sh} shared activations rounded the other way)"
+    # against the pure oracle: the oracle's own layer with its shared expert
+    pure = o.down_and_combine(a_round, rid, rw, dnb, s.num_experts) + g[:, None] * (a_s_round @ wd_s.T)
+    allow, flipped = flip_allowance(gpu_act, a_exact, a_round, rid, rw, dnb, s.num_experts)
+    if allow is None:
+        allow = np.zeros_like(pure)
+    for t, i in zip(*np.nonzero(a_gpu != a_s_round)):
+        allow[t] += abs(float(g[t])) * np.abs(wd_s[:, i]) * float(bf16_ulp(a_s_exact[t, i]))
+        flipped[t] = True
+    summary = assert_layer_parity(out_sel, pure, allow, flipped, what)
+    # stage-wise: the oracle's down projections of the GPU's own activations
+    ref = routed + g[:, None] * (a_s_used @ wd_s.T)
+    assert_out_close(out_sel, ref, what + " stage-wise")
+    record_parity(dict(case=f"shared_{fmt}_T{T}", fmt=fmt, T=T, path=int(path or 0),
+                       shape=[s.hidden, s.inter, s.num_experts, s.top_k, inter_shared],
+                       sampled_tokens=int(tok.size), activations_rounded_other_way=n_diff,
+                       shared_activations_rounded_other_way=n_sh, **summary))
     # the shared expert changes the output: the routed-only oracle must not pass
     n_far = int(np.sum(np.abs(out[tok_d].float().cpu().numpy() - routed) > 1e-2 * np.abs(routed) +
                        1e-3 * np.sqrt(np.mean(routed ** 2))))
@@ -92,15 +113,11 @@ def test_shared_nex_prefill_sampled():
     check_shared(layer, "mxfp4", 512, sample=sample, seed=2048)
 
 
-def test_shared_expert_rejects_single_kernel_path_and_bad_sizes():
+def test_shared_expert_rejects_bad_sizes():
     layer = moe_synth.make_layer(moe_synth.TINY, T=4, seed=1, device=DEV)
     s = layer.shape
     shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, "int4_g128")
     gu, dn = pack_gpu("int4_g128", layer.gate_up), pack_gpu("int4_g128", layer.down)
-    ws = moe.alloc_workspace_shared(shape, 64, 4)
-    with pytest.raises(moe.MoeError):
-        moe.moe_forward_shared(shape, moe_synth.shared_expert(s, 64, 1, DEV), layer.x, layer.router_w, gu, dn, ws,
-                               path=moe.MOE_PATH_FUSED)
     small = torch.empty(moe.moe_workspace_bytes(shape, 4), dtype=torch.uint8, device=DEV)
     moe.moe_workspace_init(small)
     with pytest.raises(moe.MoeError):   # the routed layer's workspace is too small for the shared expert

@@ -25,7 +25,7 @@ MOE_FMT_MXFP4_G32 = 2
 MOE_FMT_NVFP4_G16 = 3
 FORMATS = {"int4_g128": MOE_FMT_INT4_G128, "mxfp4": MOE_FMT_MXFP4_G32, "nvfp4": MOE_FMT_NVFP4_G16}
 
-MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_FUSED = 0, 1, 2, 3
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL = 0, 1, 2
 MOE_NUM_STAGES = 5
 STAGE_NAMES = ("router", "route_permute", "gate_up", "down", "combine")
 
@@ -95,6 +95,7 @@ _SIGS = {
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_void_p]),
     "moe_noalloc_scratch_bytes": (ctypes.c_size_t, []),
+    "moe_noalloc_status": (ctypes.c_int, [ctypes.c_void_p]),
     "moe_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_workspace_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64,
@@ -374,6 +375,12 @@ def moe_forward_noalloc(shape: MoeShape, x, router_w, gate_up_packed, down_packe
     return out
 
 
+def moe_noalloc_status(stream=None) -> int:
+    """Synchronises the stream; MOE_ERR_TIMEOUT if a no-alloc call's bounded
+    device wait expired since the last report (the report clears it), else MOE_OK."""
+    return lib().moe_noalloc_status(_stream(stream))
+
+
 def moe_workspace_init(workspace, stream=None):
     _check("moe_workspace_init", lib().moe_workspace_init(_ptr(workspace), workspace.numel(), _stream(stream)))
 
@@ -384,5 +391,7 @@ def moe_workspace_status(workspace, stream=None) -> int:
 
 
 def moe_selftest_bounded_wait(workspace, limit_ns: int, stream=None):
+    """workspace None: the status word of the no-alloc scratch array on the current device."""
     _check("moe_selftest_bounded_wait",
-           lib().moe_selftest_bounded_wait(_ptr(workspace), workspace.numel(), int(limit_ns), _stream(stream)))
+           lib().moe_selftest_bounded_wait(_ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                           int(limit_ns), _stream(stream)))

@@ -106,7 +106,6 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
-  w.ypart = static_cast<float*>(take(decode_fused_ypart_bytes(s, T)));
   w.route_part = static_cast<float*>(take(T <= kDecodeMaxT ? route_part_bytes(T, int(H), int(E), s.top_k) : 0));
   w.bytes = off;
   return w;
@@ -181,43 +180,53 @@ moe_status_t copy_debug_outputs(const moe_shape_t& s, int T, const Workspace& ws
   return MOE_OK;
 }
 
-// On the single-kernel path every stage runs inside one launch: stage 0's
-// "before" event precedes it and all the other events follow it.
-moe_status_t mark_single_kernel_rest(const moe_forward_opts_t* o, cudaStream_t stream) {
-  MOE_TRY(mark(o, 0, 1, stream));
-  for (int st = 1; st < MOE_NUM_STAGES; ++st) {
-    MOE_TRY(mark(o, st, 0, stream));
-    MOE_TRY(mark(o, st, 1, stream));
-  }
-  return MOE_OK;
-}
-
 bool valid_path(moe_path_t p) {
-  return p == MOE_PATH_AUTO || p == MOE_PATH_DECODE || p == MOE_PATH_PREFILL || p == MOE_PATH_FUSED;
+  return p == MOE_PATH_AUTO || p == MOE_PATH_DECODE || p == MOE_PATH_PREFILL;
 }
 
-moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, int T, const void* gu,
-                                  const void* dn, void* workspace, size_t ws_bytes, uint16_t* out,
-                                  const moe_forward_opts_t* opts, bool* decode, bool* fused) {
+// Everything moe_forward checks except the workspace; `decode` gets the path.
+moe_status_t check_forward_inputs(const moe_shape_t* shape, const uint16_t* x, int T, const void* gu,
+                                  const void* dn, uint16_t* out, const moe_forward_opts_t* opts, bool* decode) {
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   if ((st = check_T(shape, T)) != MOE_OK) return st;
   const moe_path_t path = opts ? opts->path : MOE_PATH_AUTO;
   if (!valid_path(path)) return MOE_ERR_INVALID_ARG;
-  if (path == MOE_PATH_FUSED && T > 0 && !decode_fused_supported(*shape, T)) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;  // nothing to do; pointers may be null
   if (!x || !gu || !dn || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gu, 256) || !aligned(dn, 256) || !aligned(out, 16))
     return MOE_ERR_INVALID_ARG;
+  *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  if (!*decode && !grouped_supported(*shape)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, int T, const void* gu,
+                                  const void* dn, void* workspace, size_t ws_bytes, uint16_t* out,
+                                  const moe_forward_opts_t* opts, bool* decode) {
+  moe_status_t st = check_forward_inputs(shape, x, T, gu, dn, out, opts, decode);
+  if (st != MOE_OK || T == 0) return st;
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
-  *fused = path == MOE_PATH_FUSED;
-  *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
-  if (!*fused && !*decode && !grouped_supported(*shape)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
 }  // namespace
+
+namespace moe {
+
+// The argument checks of moe_forward that do not involve the workspace (for
+// entry points that supply their own scratch).
+moe_status_t check_forward_args(const moe_shape_t* shape, const uint16_t* x, int T, const uint16_t* router_w,
+                                const float* logit_bias, const void* gu, const void* dn, uint16_t* out) {
+  bool decode = false;
+  const moe_status_t st = check_forward_inputs(shape, x, T, gu, dn, out, nullptr, &decode);
+  if (st != MOE_OK || T == 0) return st;
+  if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace moe
 
 extern "C" {
 
@@ -339,21 +348,13 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
                          const float* logit_bias, const void* gate_up_packed, const void* down_packed,
                          void* workspace, size_t workspace_bytes, uint16_t* out, const moe_forward_opts_t* opts,
                          cudaStream_t stream) {
-  bool decode = false, fused = false;
+  bool decode = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
-                                         out, opts, &decode, &fused);
+                                         out, opts, &decode);
   if (st != MOE_OK || T == 0) return st;
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   const Workspace ws = carve_workspace(workspace, s, T);
-  if (fused) {
-    const Bank gu = make_bank(gate_up_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
-    const Bank dn = make_bank(down_packed, s.fmt, s.num_experts, s.hidden, s.inter);
-    MOE_TRY(mark(opts, 0, 0, stream));
-    MOE_TRY(launch_decode_fused(s, T, x, router_w, logit_bias, nullptr, nullptr, gu, dn, ws, out, stream));
-    if ((st = mark_single_kernel_rest(opts, stream)) != MOE_OK) return st;
-    return copy_debug_outputs(s, T, ws, opts, false, stream);
-  }
   MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT) {
     // router logits, top-k and the permutation in one kernel
@@ -376,23 +377,15 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
                                 const float* topk_w, const void* gate_up_packed, const void* down_packed,
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
                                 const moe_forward_opts_t* opts, cudaStream_t stream) {
-  bool decode = false, fused = false;
+  bool decode = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
-                                         out, opts, &decode, &fused);
+                                         out, opts, &decode);
   if (st != MOE_OK || T == 0) return st;
   if (!topk_ids || !topk_w || !aligned(topk_ids, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   Workspace ws = carve_workspace(workspace, s, T);
   ws.topk_ids = const_cast<int32_t*>(topk_ids);
   ws.topk_w = const_cast<float*>(topk_w);
-  if (fused) {
-    const Bank gu = make_bank(gate_up_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
-    const Bank dn = make_bank(down_packed, s.fmt, s.num_experts, s.hidden, s.inter);
-    MOE_TRY(mark(opts, 0, 0, stream));
-    MOE_TRY(launch_decode_fused(s, T, x, nullptr, nullptr, topk_ids, topk_w, gu, dn, ws, out, stream));
-    if ((st = mark_single_kernel_rest(opts, stream)) != MOE_OK) return st;
-    return copy_debug_outputs(s, T, ws, opts, true, stream);
-  }
   MOE_TRY(mark(opts, 1, 0, stream));
   if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
   MOE_TRY(mark(opts, 1, 1, stream));
@@ -441,10 +434,9 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   if (!shared) return MOE_ERR_INVALID_ARG;
   if (shared->inter <= 0) return MOE_ERR_INVALID_ARG;
   if (shared->inter % 64) return MOE_ERR_UNSUPPORTED;
-  if (opts && opts->path == MOE_PATH_FUSED) return MOE_ERR_UNSUPPORTED;
-  bool decode = false, fused = false;
+  bool decode = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
-                                         out, opts, &decode, &fused);
+                                         out, opts, &decode);
   if (st != MOE_OK || T == 0) return st;
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   if (!shared->gate_up || !shared->down || !shared->gate || !aligned(shared->gate_up, 16) ||
@@ -490,7 +482,6 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   if (!valid_path(path)) return -1;
   if (T == 0) return 0;
   const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
-  if (path == MOE_PATH_FUSED) return decode_fused_supported(*shape, T) ? 1 : -1;  // the whole layer in one kernel
   const int perm = (long(T) * shape->top_k <= 1024) ? 1 : 3;
   int n = 0;
   if (routed) n += perm;
@@ -521,8 +512,15 @@ moe_status_t moe_workspace_status(void* workspace, size_t workspace_bytes, cudaS
 
 moe_status_t moe_selftest_bounded_wait(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
                                        cudaStream_t stream) {
-  if (!workspace || workspace_bytes < 256 || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
   if (limit_ns > 10ull * 1000000000ull) return MOE_ERR_INVALID_ARG;
+  if (!workspace) {
+    // the status word of moe_forward_noalloc's scratch array on this device
+    void* scratch = nullptr;
+    MOE_TRY(noalloc_scratch_address(stream, &scratch));
+    workspace = scratch;
+  } else if (workspace_bytes < 256 || !aligned(workspace, 256)) {
+    return MOE_ERR_WORKSPACE;
+  }
   return cuda_status(launch_bounded_wait_probe(static_cast<uint32_t*>(workspace), limit_ns, stream));
 }
 

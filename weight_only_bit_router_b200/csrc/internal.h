@@ -46,8 +46,7 @@ struct Bank {
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
 // The first kStatusBytes of a workspace: the status word and the kernels'
-// device counters (small-batch routing completion; the single-kernel decode
-// path's grid-wide counters).  Zeroed once by moe_workspace_init; every kernel
+// device counters (small-batch routing completion).  Zeroed once by moe_workspace_init; every kernel
 // that counts leaves its counters at zero when it finishes.
 constexpr size_t kStatusBytes = 4096;
 
@@ -65,7 +64,6 @@ struct Workspace {
   int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
-  float* ypart;           // [T*k, H] fp32 per-row down outputs (single-kernel decode path)
   float* route_part;      // [H/256, T, E] fp32 split-K router partials (small-batch routing)
   size_t bytes;
 };
@@ -110,14 +108,6 @@ cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& 
                                        uint16_t* out, const float* sh_gate, const float* sh_y,
                                        cudaStream_t stream);
 
-// decode_fused.cu: the whole layer as one cooperative kernel for T <= 8
-bool decode_fused_supported(const moe_shape_t& s, int T);
-size_t decode_fused_ypart_bytes(const moe_shape_t& s, int T);
-// ids_in / w_in: the given routing (moe_forward_routed), or null to route from router_w
-cudaError_t launch_decode_fused(const moe_shape_t& s, int T, const uint16_t* x, const uint16_t* router_w,
-                                const float* bias, const int32_t* ids_in, const float* w_in, const Bank& gu,
-                                const Bank& dn, const Workspace& ws, uint16_t* out, cudaStream_t stream);
-
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
 // the grouped GEMMs support the shape (scale rows of a tile fit their staging buffer)
@@ -143,5 +133,14 @@ cudaError_t launch_shared_gemv(const uint16_t* x, const uint16_t* w, int T, int 
 
 // selftest of the bounded device-side wait (api.cu)
 cudaError_t launch_bounded_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+// moe_forward's argument checks without the workspace (api.cu)
+moe_status_t check_forward_args(const moe_shape_t* shape, const uint16_t* x, int T, const uint16_t* router_w,
+                                const float* logit_bias, const void* gu, const void* dn, uint16_t* out);
+
+// Device address of moe_forward_noalloc's scratch array on the current device
+// (noalloc.cu); looked up when the device's context is new to the library,
+// which is refused while `stream` is being captured.
+cudaError_t noalloc_scratch_address(cudaStream_t stream, void** out);
 
 }  // namespace moe
