@@ -294,6 +294,27 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, in
                          void* workspace, size_t workspace_bytes, uint16_t* out,
                          const moe_forward_opts_t* opts, cudaStream_t stream);
 
+/* Workspace bytes moe_forward_host needs for T tokens: moe_forward's plus
+ * device staging for the hidden states and the output; 0 if invalid. */
+MOE_API size_t moe_workspace_bytes_host(const moe_shape_t* shape, int T);
+
+/* moe_forward with the hidden states and the output in HOST memory (the
+ * weights, router and workspace stay device memory): enqueues on `stream` the
+ * copy of x_host [T, H] bf16 into the workspace, the forward pass, and the
+ * copy of the output back to out_host [T, H] bf16.  Asynchronous like every
+ * other call: out_host holds the result once the stream has been
+ * synchronised, and x_host must stay unchanged until then.  Page-locked host
+ * buffers (cudaHostAlloc / cudaHostRegister) make the copies asynchronous;
+ * pageable ones work but the copies then synchronise with the host.
+ * workspace >= moe_workspace_bytes_host(shape, T) bytes, 256-byte aligned;
+ * other arguments, paths and errors as moe_forward (the debug outputs of
+ * opts, if given, are device pointers). */
+MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const uint16_t* x_host, int T,
+                                      const uint16_t* router_w, const float* logit_bias,
+                                      const void* gate_up_packed, const void* down_packed, void* workspace,
+                                      size_t workspace_bytes, uint16_t* out_host, const moe_forward_opts_t* opts,
+                                      cudaStream_t stream);
+
 /* The same layer with the routing given: topk_ids [T, k] int32 (distinct
  * experts per token, values in [0, E)) and topk_w [T, k] fp32.  Used to check
  * the expert path on its own (e.g. with the oracle's routing). */

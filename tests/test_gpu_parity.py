@@ -259,11 +259,16 @@ def test_forward_tiny_layer(fmt, path):
     check_layer(layer, fmt, path)
 
 
-@pytest.mark.parametrize("T", [1, 3, 33, 130, 300])
+@pytest.mark.parametrize("T", [1, 3, 29, 32, 33, 130, 300])
 def test_forward_tiny_shape_ragged_token_counts(T):
     layer = moe_synth.make_layer(moe_synth.TINY, T=T, seed=40 + T, zipf=True, device=DEV)
     check_layer(layer, "int4_g128", moe.MOE_PATH_PREFILL)
-    check_layer(layer, "mxfp4", moe.MOE_PATH_DECODE)
+    if T <= 32:
+        check_layer(layer, "mxfp4", moe.MOE_PATH_DECODE)
+    else:
+        # the decode kernels take at most 32 tokens
+        with pytest.raises(moe.MoeError):
+            run_forward(layer, "mxfp4", moe.MOE_PATH_DECODE)
 
 
 def test_forward_odd_shapes_and_partial_tiles():
@@ -271,9 +276,10 @@ def test_forward_odd_shapes_and_partial_tiles():
     of 64 closes every row of the down bank and of gate_up."""
     shape = moe_synth.LayerShape(hidden=320, inter=192, num_experts=6, top_k=3)
     layer = moe_synth.make_layer(shape, T=45, seed=77, device=DEV)
+    small = moe_synth.make_layer(shape, T=30, seed=76, device=DEV)
     for fmt in FMTS:
-        for path in (moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL):
-            check_layer(layer, fmt, path)
+        check_layer(layer, fmt, moe.MOE_PATH_PREFILL)
+        check_layer(small, fmt, moe.MOE_PATH_DECODE)
 
 
 def test_forward_odd_shapes_small_batch():
@@ -330,10 +336,39 @@ def test_forward_routed_matches_forward():
     out2, _ = run_forward(layer, "int4_g128", routed=(dbg["topk_ids_out"], dbg["topk_w_out"]))
     # the grouped path sums expert outputs with fp32 atomics: equal up to order
     assert_out_close(out2, out.float().cpu().numpy().astype(np.float64), "routed vs forward")
-    d1, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_DECODE)
-    d2, _ = run_forward(layer, "int4_g128", moe.MOE_PATH_DECODE,
-                        routed=(dbg["topk_ids_out"], dbg["topk_w_out"]))
+    small = moe_synth.make_layer(moe_synth.NEX, T=24, seed=10, device=DEV)
+    d1, dbg1 = run_forward(small, "int4_g128", moe.MOE_PATH_DECODE)
+    d2, _ = run_forward(small, "int4_g128", moe.MOE_PATH_DECODE,
+                        routed=(dbg1["topk_ids_out"], dbg1["topk_w_out"]))
     assert torch.equal(d1, d2)  # the decode path is deterministic
+    d3, _ = run_forward(small, "int4_g128", moe.MOE_PATH_DECODE)
+    assert torch.equal(d1, d3)
+
+
+def scaled_layer(shape, T, seed, gate_up_scale=1.0, down_scale=1.0, x_scale=1.0):
+    """A layer whose banks (and tokens) are multiplied by powers of two, rounded
+    to bf16 again (exact unless the scaled value leaves bf16's normal range)."""
+    layer = moe_synth.make_layer(shape, T=T, seed=seed, device=DEV)
+    scale = lambda t, f: (t.float() * f).to(torch.bfloat16) if f != 1.0 else t
+    return moe_synth.Layer(shape=shape, x=scale(layer.x, x_scale), router_w=layer.router_w,
+                           gate_up=scale(layer.gate_up, gate_up_scale), down=scale(layer.down, down_scale),
+                           bias=None)
+
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL])
+def test_forward_int4_scales_outside_the_single_fma_range(path):
+    """INT4 scales at or above 2^-5 (weights x 16) and subnormal scales (gate_up
+    weights x 2^-122, tokens x 2^100 to keep the activations representable)
+    take the kernels' two-step dequantisation; zero groups too."""
+    s = moe_synth.TINY
+    big = scaled_layer(s, 32, 301, gate_up_scale=16.0, down_scale=16.0)
+    big.gate_up[1, :4, :128] = 0  # whole zero groups: scale 0
+    check_layer(big, "int4_g128", path, name="int4_scales_ge_2^-5")
+    tiny = scaled_layer(s, 32, 302, gate_up_scale=2.0 ** -122, x_scale=2.0 ** 100)
+    gu = LazyOracleBank("int4_g128", tiny.gate_up)
+    scales = np.concatenate([gu.packed(e)[1].ravel() for e in range(s.num_experts)])
+    assert np.mean((scales > 0) & (scales < 0x0080)) > 0.5   # most scales are subnormal bf16
+    check_layer(tiny, "int4_g128", path, name="int4_subnormal_scales")
 
 
 def test_zero_tokens_is_a_no_op():

@@ -84,6 +84,11 @@ _SIGS = {
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
+    "moe_workspace_bytes_host": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int]),
+    "moe_forward_host": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_size_t, ctypes.c_void_p, ctypes.POINTER(ForwardOpts),
+                                        ctypes.c_void_p]),
     "moe_workspace_bytes_shared": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int]),
     "moe_forward_shared": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.POINTER(SharedExpert), ctypes.c_void_p,
                                           ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -312,6 +317,30 @@ def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, works
                            _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
     _check("moe_forward", st)
     return out
+
+
+def moe_workspace_bytes_host(shape: MoeShape, T: int) -> int:
+    return lib().moe_workspace_bytes_host(ctypes.byref(shape), T)
+
+
+def _host_ptr(t):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise ValueError("host-buffer arguments must be contiguous CPU tensors")
+    return t.data_ptr()
+
+
+def moe_forward_host(shape: MoeShape, x_host, router_w, gate_up_packed, down_packed, workspace, out_host,
+                     bias=None, path=None, stream=None):
+    """moe_forward with x_host / out_host [T, H] bf16 in (preferably pinned) host
+    memory; asynchronous: out_host is valid after the stream is synchronised."""
+    T = x_host.shape[0]
+    o, _keep = _opts(path, None, None)
+    st = lib().moe_forward_host(ctypes.byref(shape), _host_ptr(_bits(x_host)), T, _ptr(_bits(router_w)), _ptr(bias),
+                                _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
+                                _host_ptr(_bits(out_host)), ctypes.byref(o) if o is not None else None,
+                                _stream(stream))
+    _check("moe_forward_host", st)
+    return out_host
 
 
 def moe_workspace_bytes_shared(shape: MoeShape, inter_shared: int, T: int) -> int:

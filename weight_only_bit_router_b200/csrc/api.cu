@@ -106,6 +106,7 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
+  w.ypart = static_cast<float*>(take(decode_ypart_bytes(s, T)));
   w.route_part = static_cast<float*>(take(T <= kDecodeMaxT ? route_part_bytes(T, int(H), int(E), s.top_k) : 0));
   w.bytes = off;
   return w;
@@ -196,7 +197,9 @@ moe_status_t check_forward_inputs(const moe_shape_t* shape, const uint16_t* x, i
   if (!x || !gu || !dn || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gu, 256) || !aligned(dn, 256) || !aligned(out, 16))
     return MOE_ERR_INVALID_ARG;
-  *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  const bool dec_ok = decode_supported(*shape, T);
+  if (path == MOE_PATH_DECODE && !dec_ok) return MOE_ERR_UNSUPPORTED;
+  *decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && dec_ok);
   if (!*decode && !grouped_supported(*shape)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -373,6 +376,39 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
   return copy_debug_outputs(s, T, ws, opts, false, stream);
 }
 
+size_t moe_workspace_bytes_host(const moe_shape_t* shape, int T) {
+  const size_t base = moe_workspace_bytes(shape, T);
+  if (base == 0) return 0;
+  return base + 2 * align_up(size_t(T) * shape->hidden * 2, 256);
+}
+
+moe_status_t moe_forward_host(const moe_shape_t* shape, const uint16_t* x_host, int T, const uint16_t* router_w,
+                              const float* logit_bias, const void* gate_up_packed, const void* down_packed,
+                              void* workspace, size_t workspace_bytes, uint16_t* out_host,
+                              const moe_forward_opts_t* opts, cudaStream_t stream) {
+  if (check_shape(shape) != MOE_OK || T < 0) return check_shape(shape) != MOE_OK ? check_shape(shape) : MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < moe_workspace_bytes_host(shape, T))
+    return MOE_ERR_WORKSPACE;
+  // device staging of x and out after the forward's own workspace
+  const size_t base = moe_workspace_bytes(shape, T);
+  const size_t io = size_t(T) * shape->hidden * 2;
+  uint16_t* x_dev = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + base);
+  uint16_t* out_dev = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + base + align_up(io, 256));
+  bool decode = false;
+  moe_status_t st = check_forward_common(shape, x_dev, T, gate_up_packed, down_packed, workspace, base, out_dev,
+                                         opts, &decode);
+  if (st != MOE_OK) return st;
+  if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(cudaMemcpyAsync(x_dev, x_host, io, cudaMemcpyHostToDevice, stream));
+  if ((st = moe_forward(shape, x_dev, T, router_w, logit_bias, gate_up_packed, down_packed, workspace, base, out_dev,
+                        opts, stream)) != MOE_OK)
+    return st;
+  MOE_TRY(cudaMemcpyAsync(out_host, out_dev, io, cudaMemcpyDeviceToHost, stream));
+  return MOE_OK;
+}
+
 moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int T, const int32_t* topk_ids,
                                 const float* topk_w, const void* gate_up_packed, const void* down_packed,
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
@@ -481,7 +517,10 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   if (check_shape(shape) != MOE_OK || check_T(shape, T) != MOE_OK) return -1;
   if (!valid_path(path)) return -1;
   if (T == 0) return 0;
-  const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && T <= kDecodeMaxT);
+  const bool dec_ok = decode_supported(*shape, T);
+  if (path == MOE_PATH_DECODE && !dec_ok) return -1;
+  const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && dec_ok);
+  if (!decode && !grouped_supported(*shape)) return -1;
   const int perm = (long(T) * shape->top_k <= 1024) ? 1 : 3;
   int n = 0;
   if (routed) n += perm;

@@ -156,10 +156,36 @@ MOE_DEV uint32_t pow2x2(int e) {
 // one row and store them as four 16-byte bf16 chunks in swizzled layout.
 // Code words 0-1 use `mult`, words 2-3 `mult2` (the two 16-element NVFP4
 // blocks of the chunk; equal for the other formats).
+//
+// INT4 with a scale s in [2^-126, 2^-5): byte c of a code word holds the
+// adjacent elements 2c (low nibble u0) and 2c + 1 (high nibble u1).  The byte
+// copied into both halves of a word and masked with 0x00F0000F gives the bf16
+// values u0 * 2^-133 (low half) and u1 * 2^-129 (high half): bit patterns
+// below 256 are linear in value.  One bf16 fused multiply-add with the
+// multipliers (s * 2^133, s * 2^129) and -8 s in both halves yields
+// (bf16((u0 - 8) s), bf16((u1 - 8) s)), exact before its single rounding, in
+// the order the swizzled K-major tile wants.  Other scales take the two-step
+// path (the exact integer q, then one multiply).
 template <int FMT>
 MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint32_t mult2, uint32_t two, uint8_t* tile, int r,
                              int half) {
   const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+  if (FMT == MOE_FMT_INT4_G128) {
+    const uint32_t sv = mult & 0xFFFFu;
+    if (sv - 0x0080u < 0x3D00u - 0x0080u) {
+      const uint32_t m = (sv + 0x4280u) | ((sv + 0x4080u) << 16);  // (s 2^133, s 2^129)
+      const uint32_t bias = mult + 0x81808180u;                     // -8 s in both halves
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          o[c] = bf16x2_fma(prmt(w[j], 0u, 0x4040u | uint32_t(c) | (uint32_t(c) << 8)) & 0x00F0000Fu, m, bias);
+        *reinterpret_cast<uint4*>(tile + sw128_offset(r, half * 4 + j)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      return;
+    }
+  }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t P[4];

@@ -46,7 +46,8 @@ struct Bank {
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
 // The first kStatusBytes of a workspace: the status word and the kernels'
-// device counters (small-batch routing completion).  Zeroed once by moe_workspace_init; every kernel
+// device counters (small-batch routing completion at int32 index 1, the decode
+// down kernel's feature-tile counters from index 16).  Zeroed once by moe_workspace_init; every kernel
 // that counts leaves its counters at zero when it finishes.
 constexpr size_t kStatusBytes = 4096;
 
@@ -64,6 +65,7 @@ struct Workspace {
   int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
+  float* ypart;           // [T*k, H] fp32 per-row down outputs (decode path, T <= kDecodeMaxT)
   float* route_part;      // [H/256, T, E] fp32 split-K router partials (small-batch routing)
   size_t bytes;
 };
@@ -100,6 +102,10 @@ cudaError_t launch_permute_large(const int32_t* ids, int T, int E, int k, int32_
 size_t permute_large_hist_bytes(int T, int E, int k);
 
 // decode.cu
+// the decode kernels take this shape and token count (T <= kDecodeMaxT and the
+// stages fit in shared memory)
+bool decode_supported(const moe_shape_t& s, int T);
+size_t decode_ypart_bytes(const moe_shape_t& s, int T);
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const Workspace& ws, cudaStream_t stream);
 // sh_gate [T] / sh_y [T, H] (both null, or both given): the shared expert's
