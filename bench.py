@@ -21,17 +21,26 @@ torch.distributed.run) every rank runs its own replica of the stack on its own
 tokens (data parallel, weak scaling); the only collective is the max-over-ranks
 reduction of the timed region.
 
-The JSON line carries the roofline of the dominant kernel (measured live with
-CUDA events around each stage inside a captured graph), the CPU oracle timed on
-a bounded sample (cpu_baseline), an end-to-end number through the host API
-with host<->device copies in the timed region (e2e), and the SM clocks sampled
-by nvidia-smi during the timed region.
+The default run prints ONE JSON line for decode4 that also carries a
+`prefill` record: the INT4 8192-token prefill on the same stack, timed the
+same way with its own steps, clocks and roofline.
+
+Roofline: the whole layer's algorithmic bytes (decode) or flops (prefill) over
+the device-timed time per layer, and the same for the dominant kernel.  A
+kernel's time is the per-layer time times its share of the layer, the share
+measured live with CUDA events recorded around each stage in a replay of the
+same graph (events inside a graph stop programmatic launch overlap, so their
+raw durations, also reported, overstate the kernels).  `traffic` is DRAM read
++ write bytes of one ncu capture of the dominant kernel, reported only while
+the kernel sources still match the capture's digest (null otherwise).
+`e2e` times moe_forward_host (the C ABI call with the hidden states and the
+output in pinned host memory, copies in the timed region), one call per layer.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
-import math
 import os
 import subprocess
 import sys
@@ -47,33 +56,34 @@ if ROOT not in sys.path:
 import moe_synth  # noqa: E402
 
 NUM_LAYERS = 40
+PREFILL_T = 8192
 WORKLOADS = {
     # name: (fmt, T, zipf, layers per step)
     "decode4": ("int4_g128", 4, False, NUM_LAYERS),
     "decode1": ("int4_g128", 1, False, NUM_LAYERS),
     "c32": ("int4_g128", 32, True, NUM_LAYERS),
-    "prefill": ("int4_g128", 8192, False, 1),
-    "prefill_zipf": ("int4_g128", 8192, True, 1),
+    "prefill": ("int4_g128", PREFILL_T, False, 1),
+    "prefill_zipf": ("int4_g128", PREFILL_T, True, 1),
     "mx_decode4": ("mxfp4", 4, False, NUM_LAYERS),
-    "mx_prefill": ("mxfp4", 8192, False, 1),
+    "mx_prefill": ("mxfp4", PREFILL_T, False, 1),
     "nv_decode4": ("nvfp4", 4, False, NUM_LAYERS),
-    "nv_prefill": ("nvfp4", 8192, False, 1),
+    "nv_prefill": ("nvfp4", PREFILL_T, False, 1),
     "sh_decode4": ("int4_g128", 4, False, NUM_LAYERS),
-    "sh_prefill": ("int4_g128", 8192, False, 1),
+    "sh_prefill": ("int4_g128", PREFILL_T, False, 1),
 }
 # workloads whose layers carry the bf16 shared expert (intermediate 512)
 SHARED_INTER = {"sh_decode4": 512, "sh_prefill": 512}
 METRIC = "W4A16 MoE-layer tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
-# capture of the current kernel (profiles/decode_gate_up_int4_T4_ncu.md and
-# profiles/prefill_gate_up_int4_T8192_ncu.md); workloads without a capture of
-# their dominant kernel report null.
-MEASURED_TRAFFIC = {
-    ("decode4", "gate_up"): 32.480768e6 + 768.0,
-    ("prefill", "gate_up"): 375.213568e6 + 56.956672e6,
+CSRC = os.path.join(ROOT, "weight_only_bit_router_b200", "csrc")
+# the sources of each kernel family (their digest keys a traffic capture)
+KERNEL_SOURCES = {
+    "decode": ("decode.cu", "decode_common.cuh", "common.cuh", "internal.h"),
+    "grouped": ("gemm_sm100.cu", "common.cuh", "internal.h"),
 }
+# DRAM bytes (read + write) per launch of a workload's dominant kernel from one
+# ncu capture: (workload, kernel) -> (bytes, kernel family, digest of its sources)
+MEASURED_TRAFFIC = {}
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -111,6 +121,23 @@ def rank_token_seed(rank: int, T: int) -> int:
     return 500_000 + 1000 * rank + T
 
 
+def source_digest(family: str) -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[family]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, kernel: str):
+    """ncu DRAM bytes of the kernel, or None when no capture matches its current sources."""
+    rec = MEASURED_TRAFFIC.get((workload, kernel))
+    if rec is None:
+        return None
+    nbytes, family, digest = rec
+    return nbytes if source_digest(family) == digest else None
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -127,7 +154,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 f"-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
         time.sleep(0.25)
@@ -169,7 +196,7 @@ class ClockSampler:
 class Stack:
     """L layers of packed expert banks + bf16 router weights on one GPU."""
 
-    def __init__(self, moe, fmt: str, layers: int, device, zipf: bool):
+    def __init__(self, moe, fmt: str, layers: int, device):
         s = moe_synth.NEX
         self.moe, self.fmt, self.L = moe, fmt, layers
         self.shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
@@ -177,8 +204,7 @@ class Stack:
         self.gate_up = torch.empty(layers, gu_b, dtype=torch.uint8, device=device)
         self.down = torch.empty(layers, dn_b, dtype=torch.uint8, device=device)
         self.router = torch.empty(layers, s.num_experts, s.hidden, dtype=torch.bfloat16, device=device)
-        self.bias = [moe_synth.zipf_bias(s, moe_synth.SEED_STACK_BASE + l).to(device) if zipf else None
-                     for l in range(layers)]
+        self.zipf_bias = [moe_synth.zipf_bias(s, moe_synth.SEED_STACK_BASE + l).to(device) for l in range(layers)]
         pack = {"int4_g128": moe.moe_pack_int4_g128, "mxfp4": moe.moe_pack_mxfp4, "nvfp4": moe.moe_pack_nvfp4}[fmt]
         for l in range(layers):
             seed = moe_synth.SEED_STACK_BASE + l
@@ -191,6 +217,9 @@ class Stack:
             self.router[l].copy_(moe_synth.router_weight(s, seed, device))
         torch.cuda.synchronize()
         self.packed_bytes = (gu_b + dn_b) * layers
+
+    def bias(self, zipf: bool):
+        return self.zipf_bias if zipf else [None] * self.L
 
     def layer_bf16(self, l: int):
         """The bf16 source of layer l (regenerated from its seed; for the oracle)."""
@@ -217,34 +246,24 @@ def capture_graph(fn):
 
 # ---------------------------------------------------------------- algorithmic work
 
-def gate_up_bytes_per_expert(moe, shape):
-    return moe.moe_packed_bytes(shape, 0) // shape.num_experts
+def layer_work(moe, shape, T: int, touched: float):
+    """Algorithmic bytes (decode) and flops (prefill) per layer of each kernel
+    stage and of the whole layer.
 
-
-def down_bytes_per_expert(moe, shape):
-    return moe.moe_packed_bytes(shape, 1) // shape.num_experts
-
-
-def stage_work(moe, shape, T: int, touched: float):
-    """Algorithmic bytes (decode) and flops (prefill) per layer-launch of each stage.
-
-    bytes: packed weights of the touched experts streamed once + activations in/out;
-    flops: 2 * rows * (2I*H) for gate_up, 2 * rows * (H*I) for down, 2*T*E*H router."""
+    bytes: packed weights of the touched experts streamed once + the stage's
+    inputs and outputs (intermediates that the method does not define, such as
+    per-row fp32 partials, are not counted); flops: 2*T*E*H for the router,
+    2*R*(2I)*H for gate_up, 2*R*H*I for down, R = T*k."""
     H, I, E, k = shape.hidden, shape.inter, shape.num_experts, shape.top_k
     R = T * k
-    return {
-        "router": {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H},
-        "gate_up": {"bytes": touched * gate_up_bytes_per_expert(moe, shape) + T * H * 2 + R * I * 2,
-                    "flops": 2 * R * 2 * I * H},
-        "down": {"bytes": touched * down_bytes_per_expert(moe, shape) + R * I * 2 + R * H * 4,
-                 "flops": 2 * R * H * I},
-        # the whole layer as one kernel: router weight, tokens in, touched experts' packed
-        # banks, output; the intermediates (logits, SwiGLU rows, per-row down outputs) stay in L2
-        "layer": {"bytes": E * H * 2 + T * H * 2
-                  + touched * (gate_up_bytes_per_expert(moe, shape) + down_bytes_per_expert(moe, shape))
-                  + T * H * 2,
-                  "flops": 2 * T * E * H + 2 * R * 3 * I * H},
-    }
+    gu_e = moe.moe_packed_bytes(shape, 0) // E
+    dn_e = moe.moe_packed_bytes(shape, 1) // E
+    router = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
+    gate_up = {"bytes": touched * gu_e + T * H * 2 + R * I * 2, "flops": 2 * R * 2 * I * H}
+    down = {"bytes": touched * dn_e + R * I * 2 + T * H * 2, "flops": 2 * R * H * I}
+    layer = {"bytes": E * H * 2 + T * H * 2 + touched * (gu_e + dn_e) + T * H * 2,
+             "flops": router["flops"] + gate_up["flops"] + down["flops"]}
+    return {"router": router, "gate_up": gate_up, "down": down, "layer": layer}
 
 
 def load_peaks():
@@ -257,21 +276,36 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def workload_config(name: str, world: int, stack_layers: int):
+    """The `config` object of a workload's JSON line (identical in both arms)."""
+    fmt, T, zipf, layers_per_step = WORKLOADS[name]
+    layers_per_step = min(layers_per_step, stack_layers)
+    inter_sh = SHARED_INTER.get(name)
+    s = moe_synth.NEX
+    return {
+        "workload": (f"nex_moe_{fmt}_T{T}{'_zipf' if zipf else ''}{f'_shared{inter_sh}' if inter_sh else ''}"
+                     f"_{layers_per_step}layer_step_of_{stack_layers}layer_stack"),
+        "hidden": s.hidden, "experts": s.num_experts, "top_k": s.top_k, "inter": s.inter,
+        "tokens_per_layer": T, "layers_per_step": layers_per_step, "stack_layers": stack_layers,
+        "l2": "inputs larger than L2: steps rotate over a stack of packed layers larger than L2",
+        "parallelism": f"dp{world} replicas (one stack per GPU)",
+    }
+
+
 # ---------------------------------------------------------------- CPU oracle timing
 
-def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, slots_per_token=None,
-                  shared=None):
+def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, shared=None):
     """Time the CPU oracle on a bounded sample of the workload.
 
     Inputs (bf16 weights of the touched experts, packed by the oracle's own
     packer) are prepared untimed; the timed part is the oracle's forward of
     the sampled tokens: router logits, top-k, dequantisation of every touched
     expert (cold), SwiGLU experts and the weighted combine.  Returns
-    (layer-tokens per second, description, threads)."""
+    (layer-tokens per second, description, threads, seconds)."""
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
     fmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[stack.fmt]
-    E, k = stack.shape.num_experts, stack.shape.top_k
+    k = stack.shape.top_k
     done_tokens, elapsed, used_layers = 0.0, 0.0, 0
     xb_all = moe_synth.bf16_bits(x_bf16)
     for l in range(min(max_layers, stack.L)):
@@ -309,180 +343,191 @@ def oracle_sample(stack, x_bf16, bias, T, budget_s: float, max_layers: int = 3, 
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args, rank, local, world):
-    import weight_only_bit_router_b200 as moe
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    fmt, T, zipf, layers_per_step = WORKLOADS[args.workload]
-    L = args.stack_layers
-    layers_per_step = min(layers_per_step, L)
-    stack = Stack(moe, fmt, L, device, zipf)
-    shape = stack.shape
-    x = moe_synth.hidden_states(moe_synth.NEX, T, rank_token_seed(rank, T), device)
-    inter_sh = SHARED_INTER.get(args.workload)
-    shared = ([moe_synth.shared_expert(moe_synth.NEX, inter_sh, moe_synth.SEED_STACK_BASE + l, device)
-               for l in range(L)] if inter_sh else None)
-    ws = moe.alloc_workspace_shared(shape, inter_sh, T, device) if inter_sh else moe.alloc_workspace(shape, T, device)
-    outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
-    stream = torch.cuda.current_stream()
-    path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL}[args.path]
-
-    def layer_call(l, events=None):
-        fwd = (lambda *a, **k: moe.moe_forward_shared(shape, shared[l], *a, **k)) if shared else \
-            (lambda *a, **k: moe.moe_forward(shape, *a, **k))
-        fwd(x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
-            bias=stack.bias[l], path=path, events=events, stream=torch.cuda.current_stream())
-
-    # one step: layers_per_step consecutive layers; graphs rotate over the stack
-    n_graphs = L // layers_per_step
-    graphs = []
-    for gi in range(n_graphs):
-        ls = list(range(gi * layers_per_step, (gi + 1) * layers_per_step))
-        graphs.append(capture_graph(lambda ls=ls: [layer_call(l) for l in ls]))
-    assert moe.moe_workspace_status(ws) == moe.MOE_OK
-
-    def step(i):
-        graphs[i % n_graphs].replay()
-
-    # warm-up
-    for i in range(args.warmup):
-        step(i)
+def time_replays(replay, steps: int, warmup: int, stream, device, gpu_id):
+    """Device time of `steps` calls of replay(i) after `warmup` untimed ones:
+    barrier + synchronize on both sides, CUDA events on the stream, max over
+    ranks, nvidia-smi clocks sampled during the timed region."""
+    for i in range(warmup):
+        replay(i)
     torch.cuda.synchronize()
     barrier()
-    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id) as clk:
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         start.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i)
+        for i in range(steps):
+            replay(warmup + i)
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
-    ms_local = start.elapsed_time(end)
-    ms = reduce_max(ms_local, device)
-    tokens_per_step = T * layers_per_step
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
-    status = moe.moe_workspace_status(ws)
+    return reduce_max(start.elapsed_time(end), device), clk.summary()
 
-    # ---- instrumented pass: per-stage device time inside a captured graph
+
+def measure(moe, stack, name: str, steps: int, warmup: int, path: int, rank: int, world: int, device,
+            cpu_budget: float, with_cpu: bool):
+    """One workload on a packed stack: the device-timed value, the roofline,
+    the end-to-end number and (optionally) the CPU oracle beside it."""
+    fmt, T, zipf, layers_per_step = WORKLOADS[name]
+    L = stack.L
+    layers_per_step = min(layers_per_step, L)
+    shape = stack.shape
+    bias = stack.bias(zipf)
+    x = moe_synth.hidden_states(moe_synth.NEX, T, rank_token_seed(rank, T), device)
+    inter_sh = SHARED_INTER.get(name)
+    shared = ([moe_synth.shared_expert(moe_synth.NEX, inter_sh, moe_synth.SEED_STACK_BASE + l, device)
+               for l in range(L)] if inter_sh else None)
+    ws = moe.alloc_workspace_shared(shape, inter_sh, T, device) if inter_sh else moe.alloc_workspace(shape, T, device)
+    outs = torch.empty(L, T, shape.hidden, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+
+    def layer_call(l, events=None, debug=None):
+        if shared:
+            moe.moe_forward_shared(shape, shared[l], x, stack.router[l], stack.gate_up[l], stack.down[l], ws,
+                                   out=outs[l], bias=bias[l], path=path, events=events, debug=debug,
+                                   stream=torch.cuda.current_stream())
+        else:
+            moe.moe_forward(shape, x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
+                            bias=bias[l], path=path, events=events, debug=debug,
+                            stream=torch.cuda.current_stream())
+
+    def step_layers(gi):
+        return list(range(gi * layers_per_step, (gi + 1) * layers_per_step))
+
+    # one step: layers_per_step consecutive layers; graphs rotate over the stack
+    n_graphs = L // layers_per_step
+    graphs = [capture_graph(lambda ls=step_layers(gi): [layer_call(l) for l in ls]) for gi in range(n_graphs)]
+    assert moe.moe_workspace_status(ws) == moe.MOE_OK
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    ms, clocks = time_replays(lambda i: graphs[i % n_graphs].replay(), steps, warmup, stream, device, gpu_id)
+    value = world * T * layers_per_step * steps / (ms / 1e3)
+    status = moe.moe_workspace_status(ws)
+    layer_ms = ms / steps / layers_per_step
+    del graphs
+
+    # ---- stage shares: events around each stage in an instrumented replay
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * moe.MOE_NUM_STAGES)] for _ in range(L)]
     for evs in ev:
         for e in evs:
             e.record(stream)  # materialise the events before capture
     torch.cuda.synchronize()
-    inst_graphs = []
-    for gi in range(n_graphs):
-        ls = list(range(gi * layers_per_step, (gi + 1) * layers_per_step))
-        inst_graphs.append(capture_graph(lambda ls=ls: [layer_call(l, ev[l]) for l in ls]))
+    inst = [capture_graph(lambda ls=step_layers(gi): [layer_call(l, ev[l]) for l in ls]) for gi in range(n_graphs)]
     stage_ms = {n: [] for n in moe.STAGE_NAMES}
-    reps = max(1, min(20, args.steps))
-    for r in range(reps):
-        inst_graphs[r % n_graphs].replay()
-        torch.cuda.synchronize()
+    for r in range(max(1, min(20, steps))):
         gi = r % n_graphs
-        for l in range(gi * layers_per_step, (gi + 1) * layers_per_step):
+        inst[gi].replay()
+        torch.cuda.synchronize()
+        for l in step_layers(gi):
             for si, n in enumerate(moe.STAGE_NAMES):
                 stage_ms[n].append(ev[l][2 * si].elapsed_time(ev[l][2 * si + 1]))
-    stage_avg = {n: float(np.mean(v)) for n, v in stage_ms.items()}
+    del inst
+    stage_events = {n: float(np.mean(v)) for n, v in stage_ms.items()}
+    total_events = sum(stage_events.values())
+    stage_share = {n: v / total_events for n, v in stage_events.items()}
 
     # touched experts per layer (from the routing of each layer)
     touched = []
     ids_buf = torch.empty(T, shape.top_k, dtype=torch.int32, device=device)
     for l in range(L):
-        fwd = (lambda *a, **k: moe.moe_forward_shared(shape, shared[l], *a, **k)) if shared else \
-            (lambda *a, **k: moe.moe_forward(shape, *a, **k))
-        fwd(x, stack.router[l], stack.gate_up[l], stack.down[l], ws, out=outs[l],
-            bias=stack.bias[l], path=path, debug={"topk_ids_out": ids_buf})
+        layer_call(l, debug={"topk_ids_out": ids_buf})
         touched.append(len(torch.unique(ids_buf)))
     avg_touched = float(np.mean(touched))
-    work = stage_work(moe, shape, T, avg_touched)
+    work = layer_work(moe, shape, T, avg_touched)
     peaks, peak_kind = load_peaks()
-    decode = T <= 32
-    single_kernel = moe.moe_forward_launch_count(shape, T, path, False) == 1
-    if single_kernel:
-        # one launch does every stage: stage 0's events bracket it
-        dom = "layer"
-        stage_avg = {"layer": stage_avg["router"]}
-    else:
-        dom = max(("router", "gate_up", "down"), key=lambda n: stage_avg[n])
+    decode = T <= 32 and path != moe.MOE_PATH_PREFILL
+    dom = max(("router", "gate_up", "down"), key=lambda n: stage_share[n])
+    dom_ms = layer_ms * stage_share[dom]
     if decode:
-        achieved = work[dom]["bytes"] / (stage_avg[dom] / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if args.path == "auto" else None,
-                "peak_kind": f"{peak_kind} STREAM-copy HBM bandwidth",
-                "algorithmic_bytes_per_launch": work[dom]["bytes"], "avg_launch_ms": stage_avg[dom]}
+        peak, unit, key, scale = peaks["hbm_gbs"], "GB/s", "bytes", 1e9
+        bound, pk = "hbm", f"{peak_kind} STREAM-copy HBM bandwidth"
     else:
-        achieved = work[dom]["flops"] / (stage_avg[dom] / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if args.path == "auto" else None,
-                "peak_kind": f"{peak_kind} sustained cuBLAS bf16 GEMM",
-                "algorithmic_flops_per_launch": work[dom]["flops"], "avg_launch_ms": stage_avg[dom]}
+        peak, unit, key, scale = peaks["bf16_tflops_sustained"], "TFLOP/s", "flops", 1e12
+        bound, pk = "tensor", f"{peak_kind} sustained cuBLAS bf16 GEMM"
+    achieved = work[dom][key] / (dom_ms / 1e3) / scale
+    layer_ach = work["layer"][key] / (layer_ms / 1e3) / scale
+    roof = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": measured_traffic(name, dom) if path == moe.MOE_PATH_AUTO else None,
+            "peak_kind": pk, f"algorithmic_{key}_per_launch": work[dom][key], "avg_launch_ms": dom_ms,
+            "avg_launch_ms_event_bracketed": stage_events[dom],
+            "layer": {"achieved": layer_ach, "frac": layer_ach / peak, f"algorithmic_{key}": work["layer"][key],
+                      "ms": layer_ms}}
 
-    # ---- end to end through the public API with host buffers
-    x_host = torch.empty_like(x, device="cpu").pin_memory()
-    x_host.copy_(x.cpu())
-    out_host = torch.empty(layers_per_step, T, shape.hidden, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
+    # ---- end to end through the C ABI with host buffers (one call per layer)
+    e2e = None
+    if not shared:
+        ws_h = torch.empty(moe.moe_workspace_bytes_host(shape, T), dtype=torch.uint8, device=device)
+        moe.moe_workspace_init(ws_h)
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty(layers_per_step, T, shape.hidden, dtype=torch.bfloat16).pin_memory()
 
-    def e2e_step(i):
-        x.copy_(x_host, non_blocking=True)
-        graphs[i % n_graphs].replay()
-        gi = i % n_graphs
-        out_host.copy_(outs[gi * layers_per_step:(gi + 1) * layers_per_step], non_blocking=True)
+        def host_step(i):
+            for j, l in enumerate(step_layers(i % n_graphs)):
+                moe.moe_forward_host(shape, x_host, stack.router[l], stack.gate_up[l], stack.down[l], ws_h,
+                                     out_host[j], bias=bias[l], path=path, stream=stream)
 
-    for i in range(3):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
-    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+        e2e_steps = max(3, min(steps, 50))
+        e2e_ms, _ = time_replays(host_step, e2e_steps, 3, stream, device, gpu_id)
+        assert moe.moe_workspace_status(ws_h) == moe.MOE_OK
+        e2e = {"value": world * T * layers_per_step * e2e_steps / (e2e_ms / 1e3), "unit": "layer-tokens/s",
+               "h2d_bytes_per_step": layers_per_step * T * shape.hidden * 2,
+               "d2h_bytes_per_step": layers_per_step * T * shape.hidden * 2, "steps": e2e_steps,
+               "call": "moe_forward_host per layer, pinned host buffers"}
+        del ws_h
 
-    per_layer = moe.moe_forward_launch_count(shape, T, path, False) + (3 if shared else 0)  # shared: 2 GEMMs + SwiGLU
-    launches = per_layer * layers_per_step * args.steps
-
+    per_layer = moe.moe_forward_launch_count(shape, T, path, False) + (3 if shared else 0)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, threads, secs = oracle_sample(stack, x, stack.bias, T, budget_s=args.cpu_budget, shared=shared)
+    if with_cpu and rank == 0 and world == 1:
+        v, desc, threads, secs = oracle_sample(stack, x, bias, T, budget_s=cpu_budget, shared=shared)
         cpu = {"value": v, "unit": "layer-tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": secs}
+    del ws, outs
+    torch.cuda.empty_cache()
+    return {
+        "value": value, "ms_per_step": ms / steps, "steps": steps, "warmup": warmup,
+        "roofline": roof, "stage_ms_event_bracketed": stage_events, "stage_share": stage_share,
+        "e2e": e2e, "gpu_launches": per_layer * layers_per_step * steps, "clocks": clocks,
+        "cpu_baseline": cpu, "device_status": moe.moe_status_str(status),
+        "avg_touched_experts": avg_touched,
+        "path": "decode GEMV kernels" if decode else "tcgen05 grouped GEMMs",
+    }
 
+
+def run_ours(args, rank, local, world):
+    import weight_only_bit_router_b200 as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    fmt = WORKLOADS[args.workload][0]
+    stack = Stack(moe, fmt, args.stack_layers, device)
+    path = {"auto": moe.MOE_PATH_AUTO, "decode": moe.MOE_PATH_DECODE, "prefill": moe.MOE_PATH_PREFILL}[args.path]
+    m = measure(moe, stack, args.workload, args.steps, args.warmup, path, rank, world, device, args.cpu_budget,
+                not args.no_cpu_baseline)
+    details = {k: m[k] for k in ("stage_ms_event_bracketed", "stage_share", "device_status", "avg_touched_experts",
+                                 "path")}
+    details.update(packed_stack_bytes=stack.packed_bytes, path_option=args.path)
     line = {
-        "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": m["value"], "unit": "layer-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
-        "config": {"workload": f"nex_moe_{fmt}_T{T}{'_zipf' if zipf else ''}{f'_shared{inter_sh}' if inter_sh else ''}_{layers_per_step}layer_step_"
-                               f"of_{L}layer_stack",
-                   "hidden": shape.hidden, "experts": shape.num_experts, "top_k": shape.top_k,
-                   "inter": shape.inter, "tokens_per_layer": T, "layers_per_step": layers_per_step,
-                   "stack_layers": L, "packed_stack_bytes": stack.packed_bytes,
-                   "l2": "inputs larger than L2: steps rotate over a 40-layer stack of packed weights",
-                   "parallelism": f"dp{world} replicas (one stack per GPU)",
-                   "avg_touched_experts": avg_touched,
-                   "path": ("single-kernel decode layer" if single_kernel else "decode GEMV") if decode
-                   else "tcgen05 grouped GEMM", "path_option": args.path},
-        "roofline": roof,
-        "stage_ms": stage_avg,
-        "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "layer-tokens/s", "h2d_bytes_per_step": x.numel() * 2,
-                "d2h_bytes_per_step": layers_per_step * T * shape.hidden * 2, "steps": e2e_steps},
-        "gpu_launches": launches,
-        "clocks": clk.summary(),
-        "device_status": moe.moe_status_str(status),
+        "config": workload_config(args.workload, world, stack.L),
+        "roofline": m["roofline"], "cpu_baseline": m["cpu_baseline"], "e2e": m["e2e"],
+        "gpu_launches": m["gpu_launches"], "clocks": m["clocks"], "details": details,
     }
+    if (args.prefill_record and WORKLOADS[args.workload][1] <= 32 and fmt == "int4_g128"
+            and args.workload not in SHARED_INTER):
+        # the INT4 8192-token prefill on the same stack: its own steps, clocks and roofline
+        steps = max(3, min(args.steps, 40))
+        p = measure(moe, stack, "prefill", steps, args.warmup, moe.MOE_PATH_AUTO, rank, world, device, 0.0, False)
+        line["prefill"] = {
+            "workload": workload_config("prefill", world, stack.L)["workload"], "value": p["value"],
+            "unit": "layer-tokens/s", "ms_per_step": p["ms_per_step"], "steps": steps, "warmup": args.warmup,
+            "roofline": p["roofline"], "e2e": p["e2e"], "gpu_launches": p["gpu_launches"], "clocks": p["clocks"],
+            "details": {k: p[k] for k in ("stage_ms_event_bracketed", "stage_share", "device_status",
+                                          "avg_touched_experts", "path")},
+        }
+        line["gpu_launches"] += p["gpu_launches"]
     return line
 
 
@@ -496,7 +541,7 @@ def run_reference(args, rank, world):
         return None
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
-    fmt_name, T, zipf, layers_per_step = WORKLOADS[args.workload]
+    fmt_name, T, zipf, _ = WORKLOADS[args.workload]
     fmt = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}[fmt_name]
     inter_sh = SHARED_INTER.get(args.workload)
     s = moe_synth.NEX
@@ -519,7 +564,6 @@ def run_reference(args, rank, world):
         sh = ([moe_synth.bf16_bits(t) for t in moe_synth.shared_expert(s, inter_sh, seed, gen_dev)]
               if inter_sh else None)
         prepared.append((router, b, x, gu_p, dn_p, sh))
-    budget = 150.0 / max(1, args.steps + args.warmup)
 
     def one_step(i):
         router, b, x, gu_p, dn_p, sh = prepared[i % n_layers]
@@ -552,14 +596,10 @@ def run_reference(args, rank, world):
         "steps": steps_done, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, steps_done),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic seeded N(0,1) tokens, N(0,0.02) random-init weights",
-        "config": {"workload": f"nex_moe_{fmt_name}_T{T}{'_zipf' if zipf else ''}"
-                               f"{f'_shared{inter_sh}' if inter_sh else ''}_{layers_per_step}layer_step_"
-                               f"of_{NUM_LAYERS}layer_stack", "hidden": s.hidden,
-                   "experts": s.num_experts, "top_k": s.top_k, "inter": s.inter, "tokens_per_layer": T},
+        "config": workload_config(args.workload, world, args.stack_layers),
         "cpu_baseline": {"value": value, "unit": "layer-tokens/s", "cores": int(threads), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "layer-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "per_step_budget_s": budget,
     }
 
 
@@ -572,6 +612,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode4")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill-record", dest="prefill_record", action="store_false",
+                    help="leave out the 8192-token prefill record of the decode workloads")
     ap.add_argument("--path", choices=["auto", "decode", "prefill"], default="auto",
                     help="kernel path of moe_forward (auto: decode kernels up to 32 tokens, grouped GEMMs above)")
     ap.add_argument("--stack-layers", type=int, default=NUM_LAYERS,

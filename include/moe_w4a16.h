@@ -324,6 +324,40 @@ MOE_API moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t
                                 void* workspace, size_t workspace_bytes, uint16_t* out,
                                 const moe_forward_opts_t* opts, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Serving: the
+ * model runs with expert parallelism over a pair of GPUs).  Each GPU holds the
+ * packed banks of a contiguous range of experts; every GPU routes all tokens
+ * over all E experts (the router weight is replicated), computes the
+ * contribution of its own experts, and the fp32 contributions are summed
+ * across GPUs (the caller's collective, e.g. an NCCL reduce-scatter) before
+ * the single bf16 rounding of moe_partial_to_bf16.
+ * ---------------------------------------------------------------------- */
+
+/* The routed layer restricted to experts [expert_begin, expert_begin +
+ * num_local_experts) of the layer's E:
+ *   partial_out [T, H] fp32 = sum over the slots j whose expert e = ids[t, j]
+ *                             lies in the range of w_tj W_down[e] a_tj,
+ * not rounded (zero for tokens with no local expert).  The routing (logits,
+ * top-k, weights) is over all E experts, exactly as moe_forward's, so the sum
+ * of partial_out over a partition of the experts, rounded once to bf16, is
+ * moe_forward's output.  gate_up_local / down_local are packed banks of
+ * num_local_experts matrices ([n, 2I, H] and [n, H, I], the range's experts
+ * in order; moe_bank_bytes with E = n).  shape->num_experts is the layer's E.
+ * partial_out is 16-byte aligned device memory; the workspace is
+ * moe_workspace_bytes(shape, T).  Other arguments, paths and errors as
+ * moe_forward; MOE_ERR_INVALID_ARG for a range outside [0, E). */
+MOE_API moe_status_t moe_forward_partial(const moe_shape_t* shape, const uint16_t* x, int T,
+                                         const uint16_t* router_w, const float* logit_bias, int expert_begin,
+                                         int num_local_experts, const void* gate_up_local,
+                                         const void* down_local, void* workspace, size_t workspace_bytes,
+                                         float* partial_out, const moe_forward_opts_t* opts, cudaStream_t stream);
+
+/* out [T, H] bf16 = bf16_rne(partial [T, H] fp32): the layer output from the
+ * summed expert-parallel contributions.  H a multiple of 4, both pointers
+ * 16-byte aligned device memory. */
+MOE_API moe_status_t moe_partial_to_bf16(const float* partial, int T, int H, uint16_t* out, cudaStream_t stream);
+
 /* The dense shared expert of a Qwen3.5-MoE block, beside the routed ones
  * ("Tech2wild/Nex-N2.5-mini-Int4-Int8Mix", Recipe table: shared expert
  * gate/up/down_proj and shared_expert_gate; "kirillbilchenko/Nex-N2.5-mini-

@@ -89,6 +89,12 @@ _SIGS = {
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_size_t, ctypes.c_void_p, ctypes.POINTER(ForwardOpts),
                                         ctypes.c_void_p]),
+    "moe_forward_partial": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
+    "moe_partial_to_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p]),
     "moe_workspace_bytes_shared": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int]),
     "moe_forward_shared": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.POINTER(SharedExpert), ctypes.c_void_p,
                                           ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -316,6 +322,29 @@ def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, works
                            _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
                            _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
     _check("moe_forward", st)
+    return out
+
+
+def moe_forward_partial(shape: MoeShape, x, router_w, expert_begin: int, num_local: int, gate_up_local, down_local,
+                        workspace, partial_out=None, bias=None, path=None, debug=None, stream=None):
+    """The layer's fp32 contribution of experts [expert_begin, expert_begin + num_local)."""
+    T = x.shape[0]
+    if partial_out is None:
+        partial_out = torch.empty((T, shape.hidden), dtype=torch.float32, device=x.device)
+    o, _keep = _opts(path, debug, None)
+    st = lib().moe_forward_partial(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(_bits(router_w)), _ptr(bias),
+                                   int(expert_begin), int(num_local), _ptr(gate_up_local), _ptr(down_local),
+                                   _ptr(workspace), workspace.numel(), _ptr(partial_out),
+                                   ctypes.byref(o) if o is not None else None, _stream(stream))
+    _check("moe_forward_partial", st)
+    return partial_out
+
+
+def moe_partial_to_bf16(partial, out=None, stream=None):
+    T, H = partial.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=partial.device)
+    _check("moe_partial_to_bf16", lib().moe_partial_to_bf16(_ptr(partial), T, H, _ptr(out), _stream(stream)))
     return out
 
 

@@ -133,31 +133,59 @@ moe_status_t build_permutation(const moe_shape_t& s, int T, const Workspace& ws,
                                           ws.pos, ws.block_hist, ws.touched, ws.tile_base, kGemmBN, stream));
 }
 
-// Stages 2-4: experts and combine, given routing in the workspace.  sh_gate /
-// sh_y (nullable): the shared expert's gate [T] and output [T, H], added before
+// Stages 0-1: router logits, top-k and the permutation over all E experts.
+moe_status_t route_all(const moe_shape_t& s, int T, const uint16_t* x, const uint16_t* router_w,
+                       const float* logit_bias, const Workspace& ws, const moe_forward_opts_t* opts,
+                       cudaStream_t stream) {
+  MOE_TRY(mark(opts, 0, 0, stream));
+  if (T <= kDecodeMaxT) {
+    // router logits, top-k and the permutation in one kernel
+    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+  } else {
+    MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+    MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
+    moe_status_t st = build_permutation(s, T, ws, stream);
+    if (st != MOE_OK) return st;
+  }
+  MOE_TRY(mark(opts, 1, 1, stream));
+  return MOE_OK;
+}
+
+// Stages 2-4: experts and combine, given routing in the workspace.  The banks
+// hold the experts of `er`; with partial_out the result is the fp32 sum over
+// those experts (no rounding), else the bf16 output.  sh_gate / sh_y
+// (nullable): the shared expert's gate [T] and output [T, H], added before
 // the output's bf16 rounding.
 moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const void* gu_packed,
-                         const void* dn_packed, const Workspace& ws, uint16_t* out, bool decode,
-                         const moe_forward_opts_t* o, cudaStream_t stream, const float* sh_gate = nullptr,
-                         const float* sh_y = nullptr) {
-  const Bank gu = make_bank(gu_packed, s.fmt, s.num_experts, 2 * s.inter, s.hidden);
-  const Bank dn = make_bank(dn_packed, s.fmt, s.num_experts, s.hidden, s.inter);
+                         const void* dn_packed, const ExpertRange& er, const Workspace& ws, uint16_t* out,
+                         float* partial_out, bool decode, const moe_forward_opts_t* o, cudaStream_t stream,
+                         const float* sh_gate = nullptr, const float* sh_y = nullptr) {
+  const int n_bank = er.hi - er.lo;
+  const Bank gu = make_bank(gu_packed, s.fmt, n_bank, 2 * s.inter, s.hidden);
+  const Bank dn = make_bank(dn_packed, s.fmt, n_bank, s.hidden, s.inter);
   MOE_TRY(mark(o, 2, 0, stream));
-  if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, ws, stream));
-  else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, ws, stream));
+  if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, er, ws, stream));
+  else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
   MOE_TRY(mark(o, 2, 1, stream));
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
-    // down projection and the combine are one kernel on this path
-    MOE_TRY(launch_decode_down_combine(s, T, dn, ws, out, sh_gate, sh_y, stream));
+    // down projection and the combine are one kernel on this path; a shard
+    // without routed rows writes nothing, so its partial output starts at zero
+    if (partial_out) MOE_TRY(cudaMemsetAsync(partial_out, 0, size_t(T) * s.hidden * 4, stream));
+    MOE_TRY(launch_decode_down_combine(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
   } else {
-    MOE_TRY(cudaMemsetAsync(ws.out_acc, 0, size_t(T) * s.hidden * 4, stream));
-    MOE_TRY(launch_grouped_down(s, T, dn, ws, stream));
+    float* acc = partial_out ? partial_out : ws.out_acc;
+    MOE_TRY(cudaMemsetAsync(acc, 0, size_t(T) * s.hidden * 4, stream));
+    MOE_TRY(launch_grouped_down(s, T, dn, er, ws, acc, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
-    MOE_TRY(launch_finalize_out(ws.out_acc, T, s.hidden, sh_gate, sh_y, out, stream));
+    if (!partial_out) MOE_TRY(launch_finalize_out(ws.out_acc, T, s.hidden, sh_gate, sh_y, out, stream));
   }
   MOE_TRY(mark(o, 4, 1, stream));
   return MOE_OK;
@@ -358,22 +386,42 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
   const Workspace ws = carve_workspace(workspace, s, T);
-  MOE_TRY(mark(opts, 0, 0, stream));
-  if (T <= kDecodeMaxT) {
-    // router logits, top-k and the permutation in one kernel
-    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
-    MOE_TRY(mark(opts, 0, 1, stream));
-    MOE_TRY(mark(opts, 1, 0, stream));
-  } else {
-    MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
-    MOE_TRY(mark(opts, 0, 1, stream));
-    MOE_TRY(mark(opts, 1, 0, stream));
-    MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
-    if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
-  }
-  MOE_TRY(mark(opts, 1, 1, stream));
-  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
+  if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream)) != MOE_OK) return st;
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr, decode,
+                        opts, stream)) != MOE_OK)
+    return st;
   return copy_debug_outputs(s, T, ws, opts, false, stream);
+}
+
+moe_status_t moe_forward_partial(const moe_shape_t* shape, const uint16_t* x, int T, const uint16_t* router_w,
+                                 const float* logit_bias, int expert_begin, int num_local_experts,
+                                 const void* gate_up_local, const void* down_local, void* workspace,
+                                 size_t workspace_bytes, float* partial_out, const moe_forward_opts_t* opts,
+                                 cudaStream_t stream) {
+  bool decode = false;
+  // the checks of moe_forward, with the fp32 output in place of the bf16 one
+  moe_status_t st = check_forward_common(shape, x, T, gate_up_local, down_local, workspace, workspace_bytes,
+                                         reinterpret_cast<uint16_t*>(partial_out), opts, &decode);
+  if (st != MOE_OK) return st;
+  if (expert_begin < 0 || num_local_experts < 1 || long(expert_begin) + num_local_experts > shape->num_experts)
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t& s = *shape;
+  const Workspace ws = carve_workspace(workspace, s, T);
+  if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream)) != MOE_OK) return st;
+  const ExpertRange er{expert_begin, expert_begin + num_local_experts};
+  if ((st = run_experts(s, T, x, gate_up_local, down_local, er, ws, nullptr, partial_out, decode, opts, stream)) !=
+      MOE_OK)
+    return st;
+  return copy_debug_outputs(s, T, ws, opts, false, stream);
+}
+
+moe_status_t moe_partial_to_bf16(const float* partial, int T, int H, uint16_t* out, cudaStream_t stream) {
+  if (T < 0 || H <= 0 || H % 4) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!partial || !out || !aligned(partial, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_finalize_out(partial, T, H, nullptr, nullptr, out, stream));
 }
 
 size_t moe_workspace_bytes_host(const moe_shape_t* shape, int T) {
@@ -425,7 +473,9 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
   MOE_TRY(mark(opts, 1, 0, stream));
   if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
   MOE_TRY(mark(opts, 1, 1, stream));
-  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream)) != MOE_OK) return st;
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr, decode,
+                        opts, stream)) != MOE_OK)
+    return st;
   return copy_debug_outputs(s, T, ws, opts, true, stream);
 }
 
@@ -508,7 +558,8 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
     if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
   }
   MOE_TRY(mark(opts, 1, 1, stream));
-  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ws, out, decode, opts, stream, sw.g, sw.y)) != MOE_OK)
+  if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr, decode,
+                        opts, stream, sw.g, sw.y)) != MOE_OK)
     return st;
   return copy_debug_outputs(s, T, ws, opts, false, stream);
 }

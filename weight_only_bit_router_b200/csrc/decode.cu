@@ -41,6 +41,32 @@ MOE_DEV void load_routing(int* s_touched, int* s_off, const int32_t* touched, co
   }
 }
 
+// The touched experts of the bank's range [e_lo, e_hi) are a contiguous slice
+// [*t_lo, *t_hi) of the ascending touched list: counted by the whole CTA.
+// Called by every thread after the routing state is in shared memory; ends
+// with a block barrier.
+MOE_DEV void local_slice(const int* s_touched, int e_lo, int e_hi, int E, int* s_cnt, int* t_lo, int* t_hi) {
+  const int n = s_touched[0];
+  if (e_lo == 0 && e_hi == E) {
+    *t_lo = 0;
+    *t_hi = n;
+    return;
+  }
+  if (threadIdx.x < 2) s_cnt[threadIdx.x] = 0;
+  __syncthreads();
+  int below = 0, inside = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = s_touched[1 + i];
+    below += e < e_lo;
+    inside += e >= e_lo && e < e_hi;
+  }
+  if (below) atomicAdd(&s_cnt[0], below);
+  if (inside) atomicAdd(&s_cnt[1], inside);
+  __syncthreads();
+  *t_lo = s_cnt[0];
+  *t_hi = s_cnt[0] + s_cnt[1];
+}
+
 // Let the last bulk copies of this CTA's producer land before its shared
 // memory is released (bounded: they complete unless the GPU is failing).
 MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
@@ -62,9 +88,9 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kernel(
-    const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, const int32_t* __restrict__ touched,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, uint16_t* __restrict__ act,
-    uint32_t* status) {
+    const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
+    const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
+    uint16_t* __restrict__ act, uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int G = kGroups, S = kStages;
   const int K = gu.K, R = T * top_k;
@@ -81,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
   uint64_t* empty = full + S;
   uint64_t* x_bar = empty + S;
   __shared__ volatile int s_abort;  // raised by the first wait that gives up
+  __shared__ int s_cnt[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -97,8 +124,11 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
   load_routing(s_touched, s_off, touched, offsets, E);
   for (int p = threadIdx.x; p < R; p += blockDim.x) s_tok[p] = __ldcg(sorted_rows + p) / top_k;
   __syncthreads();
+  int t_lo, t_hi;
+  local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
+  const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
   const int ftiles = I / 8;
-  const int n_units = s_touched[0] * ftiles;
+  const int n_units = (t_hi - t_lo) * ftiles;
   if (int(blockIdx.x) >= n_units) return;
 
   if (warp == G * kGroupWarps) {
@@ -116,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
         if (u >= n_units) break;
         const int st = i % S;
         if (i >= S && !mbar_wait(&empty[st], ((i / S) - 1) & 1, &s_abort, status)) break;
-        const int e = s_touched[1 + u / ftiles];
-        const long row_g = long(e) * gu.N + (u % ftiles) * 8;
+        const int e = s_local[u / ftiles];
+        const long row_g = long(e - e_lo) * gu.N + (u % ftiles) * 8;
         uint8_t* stage = ring + st * L.stage_bytes;
         fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
         mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(gu, 16));
@@ -140,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
     if (u >= n_units) break;
     const int st = i % S;
     const bool ok = x_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status);
-    const int e = s_touched[1 + u / ftiles];
+    const int e = s_local[u / ftiles];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
     const int f0 = (u % ftiles) * 8;
     const uint8_t* s_c = ring + st * L.stage_bytes;
@@ -148,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
     const uint8_t* c_up = c_gate + 8 * (K / 2);
     const uint8_t* sc_gate = s_c + L.cbytes + g * srow;
     const uint8_t* sc_up = sc_gate + 8 * srow;
-    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[e] : 0.f;
+    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[e - e_lo] : 0.f;
     const int ntiles = min(NT, (n_e + 7) / 8);
     // token of column 8j + g (a valid token's row for the padding columns)
     int xtok[NT];
@@ -235,10 +265,11 @@ constexpr int kDnCounterBase = 16;    // first tile counter in the workspace's s
 
 template <int FMT, int NT, bool ACT_SMEM>
 __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
-    Bank dn, int T, int E, int top_k, const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets,
-    const uint16_t* __restrict__ act, const float* __restrict__ topk_w, const int32_t* __restrict__ pos,
-    float* __restrict__ ypart, uint16_t* __restrict__ out, const float* __restrict__ sh_gate,
-    const float* __restrict__ sh_y, uint32_t* status) {
+    Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
+    const int32_t* __restrict__ offsets, const uint16_t* __restrict__ act, const float* __restrict__ topk_w,
+    const int32_t* __restrict__ pos, float* __restrict__ ypart, uint16_t* __restrict__ out,
+    float* __restrict__ partial_out, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
+    uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int G = kGroups, S = kStages;
   const int H = dn.N, K = dn.K;  // K = I
@@ -257,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
   uint64_t* act_bar = empty + S;
   uint32_t* tile_cnt = status + kDnCounterBase;
   __shared__ volatile int s_abort;
+  __shared__ int s_cnt[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -275,7 +307,10 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
     s_w[r] = __ldcg(topk_w + r);
   }
   __syncthreads();
-  const int n_t = s_touched[0];
+  int t_lo, t_hi;
+  local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
+  const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
+  const int n_t = t_hi - t_lo;
   const int ftiles = H / kDnRows;
   const int n_units = n_t * ftiles;
   if (int(blockIdx.x) >= n_units) {
@@ -294,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
         if (u >= n_units) break;
         const int st = i % S;
         if (i >= S && !mbar_wait(&empty[st], ((i / S) - 1) & 1, &s_abort, status)) break;
-        const int e = s_touched[1 + u % n_t];
-        const long row0 = long(e) * H + (u / n_t) * kDnRows;
+        const int e = s_local[u % n_t];
+        const long row0 = long(e - e_lo) * H + (u / n_t) * kDnRows;
         uint8_t* stage = ring + st * L.stage_bytes;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(dn, kDnRows));
@@ -326,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
     if (u >= n_units) break;
     const int st = i % S;
     const bool ok = act_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status);
-    const int e = s_touched[1 + u % n_t];
+    const int e = s_local[u % n_t];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
     const int rt = (u / n_t) * (kDnRows / 16) + wj;  // this warp's 16-row feature tile
     const uint8_t* s_c = ring + st * L.stage_bytes;
@@ -334,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
     const uint8_t* c_hi = c_lo + 8 * (K / 2);
     const uint8_t* sc_lo = s_c + L.cbytes + (16 * wj + g) * srow;
     const uint8_t* sc_hi = sc_lo + 8 * srow;
-    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e] : 0.f;
+    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
     const int ntiles = min(NT, (n_e + 7) / 8);
     float acc[NT][4];
 #pragma unroll
@@ -384,17 +419,21 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
     }
     if (__shfl_sync(0xffffffffu, last, 0)) {
       // every touched expert's rows of this tile are written: the combine
+      // over the slots whose expert is in the bank's range (sorted positions
+      // [offsets[e_lo], offsets[e_hi]))
       __threadfence();
+      const int p_lo = s_off[e_lo], p_hi = s_off[e_hi];
       for (int idx = lane; idx < T * 16; idx += 32) {
         const int t = idx >> 4, f = 16 * rt + (idx & 15);
         float sum = 0.f;
         for (int j = 0; j < top_k; ++j) {
           const int r = t * top_k + j;
           const int p = s_pos[r];
-          if (p >= 0) sum += s_w[r] * __ldcg(ypart + size_t(p) * H + f);
+          if (p >= p_lo && p < p_hi) sum += s_w[r] * __ldcg(ypart + size_t(p) * H + f);
         }
         if (sh_y) sum += sh_gate[t] * sh_y[size_t(t) * H + f];  // the shared expert, before the one rounding
-        out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
+        if (partial_out) partial_out[size_t(t) * H + f] = sum;
+        else out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
       }
       if (lane == 0) tile_cnt[rt] = 0u;  // ready for the next call
     }
@@ -472,8 +511,8 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 }
 
 template <int FMT, int NT>
-cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws,
-                       int units, cudaStream_t stream) {
+cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const ExpertRange& er,
+                       const Workspace& ws, int units, cudaStream_t stream) {
   const int R = T * s.top_k;
   const bool x_smem = size_t(T) * staged_row_stride(s.hidden) <= kMaxStagedX;
   auto k = x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
@@ -482,23 +521,23 @@ cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Ban
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(k, smem, units, kThreads);
-  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k,
-                    (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows, ws.act,
-                    ws.status);
+  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k, er.lo,
+                    er.hi, (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
+                    ws.act, ws.status);
 }
 
 template <int FMT>
-cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Workspace& ws,
-                        int units, cudaStream_t stream) {
+cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const ExpertRange& er,
+                        const Workspace& ws, int units, cudaStream_t stream) {
   // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
-  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, ws, units, stream);
-  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, ws, units, stream);
-  return gate_up_nt<FMT, 4>(s, T, x, gu, ws, units, stream);
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, er, ws, units, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, er, ws, units, stream);
+  return gate_up_nt<FMT, 4>(s, T, x, gu, er, ws, units, stream);
 }
 
 template <int FMT, int NT>
-cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
-                    const float* sh_gate, const float* sh_y, cudaStream_t stream) {
+cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
+                    uint16_t* out, float* partial_out, const float* sh_gate, const float* sh_y, cudaStream_t stream) {
   const int R = T * s.top_k;
   const bool act_smem = size_t(R) * staged_row_stride(s.inter) <= kMaxStagedAct;
   auto k = act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
@@ -506,19 +545,21 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const Workspace
   if (smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
   cudaError_t err = allow_smem(k, smem);
   if (err != cudaSuccess) return err;
-  const int units = max_touched(T, s.top_k, s.num_experts) * (s.hidden / kDnRows);
-  const int grid = persistent_grid(k, smem, units, kThreads);
-  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, dn, T, s.num_experts, s.top_k,
+  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.hidden / kDnRows);
+  const int grid = persistent_grid(k, smem, std::max(units, 1), kThreads);
+  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const uint16_t*)ws.act,
-                    (const float*)ws.topk_w, (const int32_t*)ws.pos, ws.ypart, out, sh_gate, sh_y, ws.status);
+                    (const float*)ws.topk_w, (const int32_t*)ws.pos, ws.ypart, out, partial_out, sh_gate, sh_y,
+                    ws.status);
 }
 
 template <int FMT>
-cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws, uint16_t* out,
-                     const float* sh_gate, const float* sh_y, cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, ws, out, sh_gate, sh_y, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, ws, out, sh_gate, sh_y, stream);
-  return down_nt<FMT, 4>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
+                     uint16_t* out, float* partial_out, const float* sh_gate, const float* sh_y,
+                     cudaStream_t stream) {
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  return down_nt<FMT, 4>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
 }
 
 }  // namespace
@@ -539,21 +580,23 @@ size_t decode_ypart_bytes(const moe_shape_t& s, int T) {
 }
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
-                                  const Workspace& ws, cudaStream_t stream) {
-  const int units = max_touched(T, s.top_k, s.num_experts) * (s.inter / 8);
-  if (units == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, ws, units, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, ws, units, stream);
-  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, ws, units, stream);
+                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
+  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / 8);
+  if (units <= 0) return cudaSuccess;
+  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, er, ws, units, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, er, ws, units, stream);
+  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, er, ws, units, stream);
 }
 
-cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                       uint16_t* out, const float* sh_gate, const float* sh_y,
-                                       cudaStream_t stream) {
+cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                                       const Workspace& ws, uint16_t* out, float* partial_out, const float* sh_gate,
+                                       const float* sh_y, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, ws, out, sh_gate, sh_y, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, ws, out, sh_gate, sh_y, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, ws, out, sh_gate, sh_y, stream);
+  if (s.fmt == MOE_FMT_INT4_G128)
+    return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16)
+    return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
 }
 
 }  // namespace moe

@@ -65,6 +65,7 @@ struct GemmArgs {
   int M_total;          // rows of the weight side: E (router), I (gate_up), H (down)
   int n_ftiles;         // weight-row tiles of 128
   int T, top_k, I, H, E;
+  int e_lo, e_hi;              // grouped modes: the bank holds experts [e_lo, e_hi)
   const uint16_t* bsrc;        // token operand: x [T, H] (router, gate_up) or act [T*k, I] (down)
   const int32_t* offsets;      // [E+1]
   const int32_t* sorted_rows;  // [T*k]
@@ -98,6 +99,7 @@ struct Cfg {
 
 struct Tile {
   int e;        // expert (grouped modes)
+  int eb;       // its index in the bank (e - e_lo)
   int fb;       // weight-row tile
   int p_begin;  // first sorted row (grouped) or first token (router)
   int n;        // valid token columns (1..BN)
@@ -109,18 +111,22 @@ MOE_DEV Tile decode_tile(const GemmArgs& a, int tile, const int* s_tile_base) {
   const int blk = tile / a.n_ftiles;
   if (a.mode == kRouter) {
     t.e = 0;
+    t.eb = 0;
     t.p_begin = blk * BN;
     t.n = min(BN, a.T - t.p_begin);
     return t;
   }
-  // expert e with tile_base[e] <= blk < tile_base[e+1] (skip empty experts)
-  int lo = 0, hi = a.E;  // invariant: tile_base[lo] <= blk < tile_base[hi]
+  // expert e with tile_base[e] <= blk' < tile_base[e+1] (skip empty experts),
+  // blk' counted from the bank's first expert
+  const int gblk = blk + s_tile_base[a.e_lo];
+  int lo = a.e_lo, hi = a.e_hi;  // invariant: tile_base[lo] <= gblk < tile_base[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (s_tile_base[mid] <= blk) lo = mid; else hi = mid;
+    if (s_tile_base[mid] <= gblk) lo = mid; else hi = mid;
   }
   t.e = lo;
-  const int tb = blk - s_tile_base[lo];
+  t.eb = lo - a.e_lo;
+  const int tb = gblk - s_tile_base[lo];
   const int p0 = a.offsets[lo];
   const int n_e = a.offsets[lo + 1] - p0;
   t.p_begin = p0 + tb * BN;
@@ -130,7 +136,7 @@ MOE_DEV Tile decode_tile(const GemmArgs& a, int tile, const int* s_tile_base) {
 
 MOE_DEV int num_tiles(const GemmArgs& a, const int* s_tile_base) {
   if (a.mode == kRouter) return a.n_ftiles * ((a.T + BN - 1) / BN);
-  return s_tile_base[a.E] * a.n_ftiles;
+  return (s_tile_base[a.e_hi] - s_tile_base[a.e_lo]) * a.n_ftiles;
 }
 
 // byte offset of 16-byte chunk c of row r inside a 128B-swizzled K-major tile
@@ -303,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < NACC; ++c) {
             long row0;
-            if (MODE == kGateUp) row0 = long(t.e) * 2 * a.I + (c ? a.I : 0) + f0;
-            else row0 = long(t.e) * a.H + f0;
+            if (MODE == kGateUp) row0 = long(t.eb) * 2 * a.I + (c ? a.I : 0) + f0;
+            else row0 = long(t.eb) * a.H + f0;
             bulk_g2s(sS + (slot * NACC + c) * BM * kSrow, sp + row0 * sb, bytes, &sc_full[slot]);
           }
         }
@@ -320,10 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&codes_full[s], NACC * kCodeBytes);
             uint8_t* dst = sC + s * NACC * kCodeBytes;
             if (MODE == kGateUp) {
-              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.e);
-              tma_load_3d(dst + kCodeBytes, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.e + 1);
+              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.eb);
+              tma_load_3d(dst + kCodeBytes, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.eb + 1);
             } else {
-              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, t.e);
+              tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, t.eb);
             }
           }
         }
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = it & 1;
         if (!(ok = mbar_wait(&sc_full[slot], (it >> 1) & 1, abort, a.status))) break;
         const uint8_t* srows = sS + slot * NACC * BM * kSrow + r * sb;
-        const float gsc = FMT == MOE_FMT_NVFP4_G16 ? a.gscale[t.e] : 0.f;
+        const float gsc = FMT == MOE_FMT_NVFP4_G16 ? a.gscale[t.eb] : 0.f;
         for (int ks = 0; ks < KS; ++ks, ++g) {
           const int sc = g % SC, so = g % SA;
           if (!(ok = mbar_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
@@ -660,8 +666,10 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ct
   return cudaGetLastError();
 }
 
-GemmArgs base_args(const moe_shape_t& s, int T, const Workspace& ws) {
+GemmArgs base_args(const moe_shape_t& s, int T, const ExpertRange& er, const Workspace& ws) {
   GemmArgs a{};
+  a.e_lo = er.lo;
+  a.e_hi = er.hi;
   a.fmt = int(s.fmt);
   a.T = T;
   a.top_k = s.top_k;
@@ -719,11 +727,11 @@ bool grouped_supported(const moe_shape_t& s) {
 }
 
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
-                                   const Workspace& ws, cudaStream_t stream) {
-  if (T == 0) return cudaSuccess;
+                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
+  if (T == 0 || er.hi <= er.lo) return cudaSuccess;
   CUtensorMap map;
-  if (!make_codes_map(&map, gu.codes, gu.K, s.inter, 2L * s.num_experts)) return cudaErrorInvalidValue;
-  GemmArgs a = base_args(s, T, ws);
+  if (!make_codes_map(&map, gu.codes, gu.K, s.inter, 2L * (er.hi - er.lo))) return cudaErrorInvalidValue;
+  GemmArgs a = base_args(s, T, er, ws);
   a.mode = kGateUp;
   a.K = s.hidden;
   a.M_total = s.inter;
@@ -738,12 +746,13 @@ cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* 
   return launch_gemm<kGateUp, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
 }
 
-cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                cudaStream_t stream) {
-  if (T == 0) return cudaSuccess;
+cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                                const Workspace& ws, float* acc, cudaStream_t stream) {
+  if (T == 0 || er.hi <= er.lo) return cudaSuccess;
   CUtensorMap map;
-  if (!make_codes_map(&map, dn.codes, dn.K, s.hidden, s.num_experts)) return cudaErrorInvalidValue;
-  GemmArgs a = base_args(s, T, ws);
+  if (!make_codes_map(&map, dn.codes, dn.K, s.hidden, er.hi - er.lo)) return cudaErrorInvalidValue;
+  GemmArgs a = base_args(s, T, er, ws);
+  a.out_acc = acc;
   a.mode = kDown;
   a.K = s.inter;
   a.M_total = s.hidden;

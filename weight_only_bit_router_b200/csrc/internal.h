@@ -36,6 +36,12 @@ inline size_t bank_total_bytes(moe_format_t fmt, int E, int N, int K) {
   return bank_scale_offset(fmt, E, N, K) + bank_scale_bytes(fmt, E, N, K);
 }
 
+// The experts a packed bank holds: [lo, hi) of the layer's E (all of them,
+// or one expert-parallel shard).  Routing always runs over all E experts.
+struct ExpertRange {
+  int lo, hi;
+};
+
 // Device view of one packed bank.
 struct Bank {
   const uint8_t* codes;  // [E][N][K/2]
@@ -107,12 +113,14 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 bool decode_supported(const moe_shape_t& s, int T);
 size_t decode_ypart_bytes(const moe_shape_t& s, int T);
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
-                                  const Workspace& ws, cudaStream_t stream);
+                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
 // sh_gate [T] / sh_y [T, H] (both null, or both given): the shared expert's
-// gate and output, added as sh_gate[t] * sh_y[t][f] before the bf16 rounding
-cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                       uint16_t* out, const float* sh_gate, const float* sh_y,
-                                       cudaStream_t stream);
+// gate and output, added as sh_gate[t] * sh_y[t][f] before the bf16 rounding.
+// partial_out (nullable): the fp32 sum over the bank's experts instead of the
+// bf16 output (every element written when the bank has routed rows).
+cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                                       const Workspace& ws, uint16_t* out, float* partial_out, const float* sh_gate,
+                                       const float* sh_y, cudaStream_t stream);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
@@ -121,9 +129,10 @@ bool grouped_supported(const moe_shape_t& s);
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int H, int E, float* logits,
                                uint32_t* status, cudaStream_t stream);
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
-                                   const Workspace& ws, cudaStream_t stream);
-cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const Workspace& ws,
-                                cudaStream_t stream);
+                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
+// adds the weighted expert outputs into acc [T, H] fp32 (zeroed by the caller)
+cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                                const Workspace& ws, float* acc, cudaStream_t stream);
 // out = bf16(acc [+ sh_gate[t] * sh_y[t][f]]) over [T, H] (sh_* nullable)
 cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_gate, const float* sh_y,
                                 uint16_t* out, cudaStream_t stream);
