@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 /* Exported symbol marker (the library is built with hidden default visibility). */
 #if defined(__GNUC__)
@@ -269,13 +269,28 @@ typedef struct {
   int32_t* offsets_out;      /* [E+1]   per-expert row offsets */
   int32_t* sorted_rows_out;  /* [T*k]   expert-sorted rows */
   uint16_t* act_out;         /* [T*k, I] bf16 SwiGLU activations, expert-sorted rows */
+  uint32_t flags;            /* MOE_FLAG_* bits (0: defaults) */
   cudaEvent_t* stage_events; /* [2*MOE_NUM_STAGES]: recorded before / after each stage
                                 (as external event nodes when the stream is being
                                 captured into a CUDA graph) */
 } moe_forward_opts_t;
 
+/* moe_forward_opts_t.flags: MOE_FLAG_DETERMINISTIC makes the grouped
+ * (above 32 tokens) path's combine run-to-run deterministic: every (token,
+ * slot) row's weighted expert output is stored in its own fp32 row and each
+ * token's k rows are summed in slot order, instead of being added into the
+ * output accumulator in arrival order.  It needs the larger workspace of
+ * moe_workspace_bytes_flags.  The decode path (up to 32 tokens) is always
+ * deterministic. */
+#define MOE_FLAG_DETERMINISTIC 1u
+
 /* Workspace bytes moe_forward / moe_forward_routed need for T tokens. */
 MOE_API size_t moe_workspace_bytes(const moe_shape_t* shape, int T);
+
+/* Workspace bytes for T tokens with the given MOE_FLAG_* bits (flags = 0:
+ * moe_workspace_bytes; MOE_FLAG_DETERMINISTIC above 32 tokens adds T*k*H*4
+ * bytes for the per-row outputs). */
+MOE_API size_t moe_workspace_bytes_flags(const moe_shape_t* shape, int T, uint32_t flags);
 
 /* Forward pass of the routed-expert layer.
  *   x            [T, H] bf16 hidden states
@@ -308,7 +323,8 @@ MOE_API size_t moe_workspace_bytes_host(const moe_shape_t* shape, int T);
  * pageable ones work but the copies then synchronise with the host.
  * workspace >= moe_workspace_bytes_host(shape, T) bytes, 256-byte aligned;
  * other arguments, paths and errors as moe_forward (the debug outputs of
- * opts, if given, are device pointers). */
+ * opts, if given, are device pointers; opts->flags must be 0, else
+ * MOE_ERR_UNSUPPORTED). */
 MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const uint16_t* x_host, int T,
                                       const uint16_t* router_w, const float* logit_bias,
                                       const void* gate_up_packed, const void* down_packed, void* workspace,
@@ -383,7 +399,8 @@ MOE_API size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_sh
  * split-K mma.sync product up to 32; its contribution is added to the routed
  * combine in fp32 before the output's single bf16 rounding.  Other
  * arguments, paths, errors and the workspace rules as moe_forward (workspace
- * >= moe_workspace_bytes_shared bytes). */
+ * >= moe_workspace_bytes_shared bytes; opts->flags must be 0, else
+ * MOE_ERR_UNSUPPORTED). */
 MOE_API moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_expert_t* shared,
                                 const uint16_t* x, int T, const uint16_t* router_w,
                                 const float* logit_bias, const void* gate_up_packed,

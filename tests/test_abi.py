@@ -21,7 +21,7 @@ def declared_functions():
 
 
 def test_library_loads_and_reports_abi_version():
-    assert moe.moe_abi_version() == 1
+    assert moe.moe_abi_version() == 2
 
 
 def test_every_declared_symbol_is_exported_and_bound():
@@ -145,6 +145,34 @@ def test_forward_validation_happens_on_the_host():
     # T == 0 is a valid no-op
     assert L.moe_forward(*args(T=0)) == 0
     assert moe.moe_forward_launch_count(s, 4, 3, False) == -1     # unknown path
+
+
+def test_workspace_query_with_flags():
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    base = moe.moe_workspace_bytes(s, 8192)
+    assert moe.moe_workspace_bytes_flags(s, 8192, 0) == base
+    assert moe.moe_workspace_bytes_flags(s, 8192, moe.MOE_FLAG_DETERMINISTIC) >= base + 8192 * 8 * 2048 * 4
+    # the decode path's per-row buffer is always there: the flag adds nothing at 32 tokens or fewer
+    assert moe.moe_workspace_bytes_flags(s, 32, moe.MOE_FLAG_DETERMINISTIC) == moe.moe_workspace_bytes(s, 32)
+    assert moe.moe_workspace_bytes_flags(s, 4, 2) == 0          # unknown flag
+    assert moe.moe_workspace_bytes_host(s, 4) >= moe.moe_workspace_bytes(s, 4) + 2 * 4 * 2048 * 2
+
+
+def test_partial_and_host_validation():
+    L = moe.lib()
+    s = moe.make_shape(256, 64, 8, 2, "int4_g128")
+    wsb = moe.moe_workspace_bytes(s, 4)
+    part = lambda b, n, **kw: L.moe_forward_partial(ctypes.byref(s), 256, 4, 256, None, b, n, 256, 256, 256, wsb,
+                                                   kw.get("out", 256), None, None)
+    assert part(6, 3) == 1           # the range leaves the layer's experts
+    assert part(-1, 2) == 1
+    assert part(2, 0) == 1
+    assert part(0, 8, out=None) == 1
+    assert L.moe_partial_to_bf16(None, 4, 256, 256, None) == 1
+    assert L.moe_partial_to_bf16(256, 4, 250, 256, None) == 1   # H not a multiple of 4
+    assert L.moe_partial_to_bf16(None, 0, 256, None, None) == 0
+    assert L.moe_forward_host(ctypes.byref(s), None, 4, 256, None, 256, 256, 256, 1 << 20, 256, None, None) == 1
+    assert L.moe_forward_host(ctypes.byref(s), 256, 4, 256, None, 256, 256, 256, 16, 256, None, None) == 3
 
 
 def test_routed_forward_validation():

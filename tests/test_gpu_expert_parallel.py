@@ -23,25 +23,25 @@ from weight_only_bit_router_b200.expert_parallel import expert_range
 pytestmark = pytest.mark.gpu
 
 
-def sharded_forward(layer, fmt, blocks, path=None):
+def sharded_forward(layer, fmt, blocks, path=None, flags=0):
     """Sum of moe_forward_partial over the expert blocks [(begin, count)], rounded once."""
     s = layer.shape
     shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
     T = layer.x.shape[0]
-    ws = moe.alloc_workspace(shape, T)
+    ws = moe.alloc_workspace(shape, T, flags=flags)
     total = torch.zeros(T, s.hidden, dtype=torch.float32, device=DEV)
     for begin, count in blocks:
         gu = PACKERS[fmt](layer.gate_up[begin:begin + count].contiguous())
         dn = PACKERS[fmt](layer.down[begin:begin + count].contiguous())
         part = moe.moe_forward_partial(shape, layer.x, layer.router_w, begin, count, gu, dn, ws, bias=layer.bias,
-                                       path=path)
+                                       path=path, flags=flags)
         assert moe.moe_workspace_status(ws) == moe.MOE_OK
         total += part
     return moe.moe_partial_to_bf16(total)
 
 
-def check_sharded(layer, fmt, blocks, path=None, sample=None, name=""):
-    ep = sharded_forward(layer, fmt, blocks, path)
+def check_sharded(layer, fmt, blocks, path=None, sample=None, name="", flags=0):
+    ep = sharded_forward(layer, fmt, blocks, path, flags)
     full, dbg = run_forward(layer, fmt, path)
     # against moe_forward: the same kernels, only the fp32 summation order differs
     assert_out_close(ep, full.float().cpu().numpy().astype(np.float64), f"{name}: shards vs whole banks")
@@ -67,12 +67,13 @@ def test_uneven_shards_and_an_empty_one_decode_path():
     check_sharded(layer, "int4_g128", blocks, name="ep_uneven_T4")
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_shards_grouped_path(world):
+@pytest.mark.parametrize("world,flags", [(2, 0), (4, 0), (2, moe.MOE_FLAG_DETERMINISTIC)])
+def test_shards_grouped_path(world, flags):
     layer = moe_synth.make_layer(moe_synth.NEX, T=300, seed=2300 + world, device=DEV)
     blocks = [expert_range(256, r, world) for r in range(world)]
     sample = np.random.default_rng(world).choice(300, 16, replace=False)
-    check_sharded(layer, "int4_g128", blocks, moe.MOE_PATH_PREFILL, sample=sample, name=f"ep{world}_T300")
+    check_sharded(layer, "int4_g128", blocks, moe.MOE_PATH_PREFILL, sample=sample, name=f"ep{world}_T300_f{flags}",
+                  flags=flags)
 
 
 def test_shards_tiny_layer_both_paths():

@@ -153,7 +153,7 @@ def test_permute_bit_exact(T, E, k):
 
 # ---------------------------------------------------------------- layer forward
 
-def run_forward(layer, fmt, path=None, routed=None, packed=None):
+def run_forward(layer, fmt, path=None, routed=None, packed=None, flags=0):
     """moe_forward (or moe_forward_routed) of a layer with every debug output;
     `packed` = (gate_up, down) banks already packed on the GPU, else they are
     packed here."""
@@ -161,7 +161,7 @@ def run_forward(layer, fmt, path=None, routed=None, packed=None):
     shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
     T = layer.x.shape[0]
     gu, dn = packed if packed is not None else (pack_gpu(fmt, layer.gate_up), pack_gpu(fmt, layer.down))
-    ws = moe.alloc_workspace(shape, T)
+    ws = moe.alloc_workspace(shape, T, flags=flags)
     dbg = {
         "logits_out": torch.empty(T, s.num_experts, dtype=torch.float32, device=DEV),
         "topk_ids_out": torch.empty(T, s.top_k, dtype=torch.int32, device=DEV),
@@ -171,12 +171,13 @@ def run_forward(layer, fmt, path=None, routed=None, packed=None):
         "sorted_rows_out": torch.empty(T * s.top_k, dtype=torch.int32, device=DEV),
     }
     if routed is None:
-        out = moe.moe_forward(shape, layer.x, layer.router_w, gu, dn, ws, bias=layer.bias, path=path, debug=dbg)
+        out = moe.moe_forward(shape, layer.x, layer.router_w, gu, dn, ws, bias=layer.bias, path=path, debug=dbg,
+                              flags=flags)
     else:
         ids, w = routed
         for key in ("logits_out", "topk_ids_out", "topk_w_out"):
             dbg.pop(key)
-        out = moe.moe_forward_routed(shape, layer.x, ids, w, gu, dn, ws, path=path, debug=dbg)
+        out = moe.moe_forward_routed(shape, layer.x, ids, w, gu, dn, ws, path=path, debug=dbg, flags=flags)
     assert moe.moe_workspace_status(ws) == moe.MOE_OK
     return out, dbg
 
@@ -343,6 +344,39 @@ def test_forward_routed_matches_forward():
     assert torch.equal(d1, d2)  # the decode path is deterministic
     d3, _ = run_forward(small, "int4_g128", moe.MOE_PATH_DECODE)
     assert torch.equal(d1, d3)
+
+
+@pytest.mark.parametrize("fmt,T,zipf", [("int4_g128", 300, True), ("nvfp4", 2048, False)])
+def test_deterministic_grouped_combine(fmt, T, zipf):
+    """MOE_FLAG_DETERMINISTIC: the grouped path's output is bit-identical from run
+    to run (each token's slot rows summed in slot order) and meets the oracle."""
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=6000 + T, zipf=zipf, device=DEV)
+    packed = (pack_gpu(fmt, layer.gate_up), pack_gpu(fmt, layer.down))
+    det = moe.MOE_FLAG_DETERMINISTIC
+    s = layer.shape
+    shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, fmt)
+    assert moe.moe_workspace_bytes_flags(shape, T, det) == moe.moe_workspace_bytes(shape, T) + T * 8 * 2048 * 4
+    out1, dbg = run_forward(layer, fmt, packed=packed, flags=det)
+    for _ in range(3):
+        out2, _ = run_forward(layer, fmt, packed=packed, flags=det)
+        assert torch.equal(out1, out2)
+    sample = np.random.default_rng(T).choice(T, 16, replace=False)
+    verify_layer(layer, fmt, out1, dbg, sample=sample, name=f"deterministic_{fmt}_T{T}")
+    # the default (arrival-order) combine agrees within the tolerance
+    out3, _ = run_forward(layer, fmt, packed=packed)
+    assert_out_close(out3, out1.float().cpu().numpy().astype(np.float64), "default vs deterministic combine")
+
+
+def test_deterministic_flag_needs_its_workspace():
+    layer = moe_synth.make_layer(moe_synth.TINY, T=40, seed=12, device=DEV)
+    s = layer.shape
+    shape = moe.make_shape(s.hidden, s.inter, s.num_experts, s.top_k, "int4_g128")
+    gu, dn = pack_gpu("int4_g128", layer.gate_up), pack_gpu("int4_g128", layer.down)
+    small = moe.alloc_workspace(shape, 40)
+    with pytest.raises(moe.MoeError):
+        moe.moe_forward(shape, layer.x, layer.router_w, gu, dn, small, flags=moe.MOE_FLAG_DETERMINISTIC)
+    with pytest.raises(moe.MoeError):
+        moe.moe_forward(shape, layer.x, layer.router_w, gu, dn, small, flags=2)   # unknown flag
 
 
 def scaled_layer(shape, T, seed, gate_up_scale=1.0, down_scale=1.0, x_scale=1.0):

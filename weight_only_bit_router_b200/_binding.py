@@ -50,7 +50,10 @@ class ForwardOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("topk_ids_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
                 ("logits_out", ctypes.c_void_p), ("offsets_out", ctypes.c_void_p),
                 ("sorted_rows_out", ctypes.c_void_p), ("act_out", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p)]
+                ("flags", ctypes.c_uint32), ("stage_events", ctypes.c_void_p)]
+
+
+MOE_FLAG_DETERMINISTIC = 1
 
 
 _SIGS = {
@@ -76,6 +79,7 @@ _SIGS = {
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                    ctypes.c_void_p]),
     "moe_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int]),
+    "moe_workspace_bytes_flags": (ctypes.c_size_t, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_uint32]),
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_size_t, ctypes.c_void_p, ctypes.POINTER(ForwardOpts),
@@ -196,6 +200,10 @@ def moe_workspace_bytes(shape: MoeShape, T: int) -> int:
     return lib().moe_workspace_bytes(ctypes.byref(shape), T)
 
 
+def moe_workspace_bytes_flags(shape: MoeShape, T: int, flags: int) -> int:
+    return lib().moe_workspace_bytes_flags(ctypes.byref(shape), T, int(flags))
+
+
 def moe_permute_workspace_bytes(T, E, k) -> int:
     return lib().moe_permute_workspace_bytes(T, E, k)
 
@@ -291,18 +299,19 @@ def moe_permute(topk_ids, E, stream=None):
 
 # ------------------------------------------------------------------ forward
 
-def alloc_workspace(shape: MoeShape, T: int, device="cuda", stream=None):
-    nbytes = moe_workspace_bytes(shape, T)
+def alloc_workspace(shape: MoeShape, T: int, device="cuda", stream=None, flags=0):
+    nbytes = moe_workspace_bytes_flags(shape, T, flags)
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
     moe_workspace_init(ws, stream=stream)
     return ws
 
 
-def _opts(path, debug, events):
-    if path is None and not debug and events is None:
+def _opts(path, debug, events, flags=0):
+    if path is None and not debug and events is None and not flags:
         return None, None
     o = ForwardOpts()
     o.path = path or MOE_PATH_AUTO
+    o.flags = int(flags)
     for name, t in (debug or {}).items():
         setattr(o, name, _ptr(t))
     keep = None
@@ -313,11 +322,11 @@ def _opts(path, debug, events):
 
 
 def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, workspace, out=None, bias=None,
-                path=None, debug=None, events=None, stream=None):
+                path=None, debug=None, events=None, stream=None, flags=0):
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
-    o, _keep = _opts(path, debug, events)
+    o, _keep = _opts(path, debug, events, flags)
     st = lib().moe_forward(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(_bits(router_w)), _ptr(bias),
                            _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
                            _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))
@@ -326,12 +335,12 @@ def moe_forward(shape: MoeShape, x, router_w, gate_up_packed, down_packed, works
 
 
 def moe_forward_partial(shape: MoeShape, x, router_w, expert_begin: int, num_local: int, gate_up_local, down_local,
-                        workspace, partial_out=None, bias=None, path=None, debug=None, stream=None):
+                        workspace, partial_out=None, bias=None, path=None, debug=None, stream=None, flags=0):
     """The layer's fp32 contribution of experts [expert_begin, expert_begin + num_local)."""
     T = x.shape[0]
     if partial_out is None:
         partial_out = torch.empty((T, shape.hidden), dtype=torch.float32, device=x.device)
-    o, _keep = _opts(path, debug, None)
+    o, _keep = _opts(path, debug, None, flags)
     st = lib().moe_forward_partial(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(_bits(router_w)), _ptr(bias),
                                    int(expert_begin), int(num_local), _ptr(gate_up_local), _ptr(down_local),
                                    _ptr(workspace), workspace.numel(), _ptr(partial_out),
@@ -401,11 +410,11 @@ def moe_forward_shared(shape: MoeShape, shared, x, router_w, gate_up_packed, dow
 
 
 def moe_forward_routed(shape: MoeShape, x, topk_ids, topk_w, gate_up_packed, down_packed, workspace, out=None,
-                       path=None, debug=None, events=None, stream=None):
+                       path=None, debug=None, events=None, stream=None, flags=0):
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, shape.hidden), dtype=torch.bfloat16, device=x.device)
-    o, _keep = _opts(path, debug, events)
+    o, _keep = _opts(path, debug, events, flags)
     st = lib().moe_forward_routed(ctypes.byref(shape), _ptr(_bits(x)), T, _ptr(topk_ids), _ptr(topk_w),
                                   _ptr(gate_up_packed), _ptr(down_packed), _ptr(workspace), workspace.numel(),
                                   _ptr(out), ctypes.byref(o) if o is not None else None, _stream(stream))

@@ -1,5 +1,6 @@
 // C ABI of the W4A16 routed-expert MoE layer: argument validation, workspace
 // carve-up and the order of kernel launches on the caller's stream.
+#include <nvtx3/nvToolsExt.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -10,6 +11,18 @@ namespace moe {
 namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+uint32_t opt_flags(const moe_forward_opts_t* o) { return o ? o->flags : 0u; }
+
+// NVTX range over the host code that enqueues one stage (or one call): a
+// profiler shows which stage each kernel launch belongs to.  NVTX is header
+// only; without an attached tool a range costs a pointer check.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool valid_fmt(moe_format_t f) {
   return f == MOE_FMT_INT4_G128 || f == MOE_FMT_MXFP4_G32 || f == MOE_FMT_NVFP4_G16;
@@ -82,7 +95,7 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
 
 }  // namespace
 
-Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
+Workspace carve_workspace(void* base, const moe_shape_t& s, int T, uint32_t flags) {
   Workspace w{};
   const size_t R = size_t(T) * s.top_k;
   const size_t E = s.num_experts, H = s.hidden, I = s.inter;
@@ -106,7 +119,11 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T) {
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
-  w.ypart = static_cast<float*>(take(decode_ypart_bytes(s, T)));
+  // per-row down outputs: the decode path's (T <= kDecodeMaxT), or the
+  // deterministic grouped combine's
+  const size_t ypart_bytes = T <= kDecodeMaxT ? decode_ypart_bytes(s, T)
+                             : (flags & MOE_FLAG_DETERMINISTIC) ? R * H * 4 : 0;
+  w.ypart = static_cast<float*>(take(ypart_bytes));
   w.route_part = static_cast<float*>(take(T <= kDecodeMaxT ? route_part_bytes(T, int(H), int(E), s.top_k) : 0));
   w.bytes = off;
   return w;
@@ -137,6 +154,7 @@ moe_status_t build_permutation(const moe_shape_t& s, int T, const Workspace& ws,
 moe_status_t route_all(const moe_shape_t& s, int T, const uint16_t* x, const uint16_t* router_w,
                        const float* logit_bias, const Workspace& ws, const moe_forward_opts_t* opts,
                        cudaStream_t stream) {
+  NvtxRange range("moe.route");
   MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT) {
     // router logits, top-k and the permutation in one kernel
@@ -167,10 +185,14 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   const int n_bank = er.hi - er.lo;
   const Bank gu = make_bank(gu_packed, s.fmt, n_bank, 2 * s.inter, s.hidden);
   const Bank dn = make_bank(dn_packed, s.fmt, n_bank, s.hidden, s.inter);
-  MOE_TRY(mark(o, 2, 0, stream));
-  if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, er, ws, stream));
-  else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
-  MOE_TRY(mark(o, 2, 1, stream));
+  {
+    NvtxRange range("moe.gate_up");
+    MOE_TRY(mark(o, 2, 0, stream));
+    if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, er, ws, stream));
+    else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
+    MOE_TRY(mark(o, 2, 1, stream));
+  }
+  NvtxRange range(decode ? "moe.down_combine" : "moe.down");
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
     // down projection and the combine are one kernel on this path; a shard
@@ -179,10 +201,17 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
     MOE_TRY(launch_decode_down_combine(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
+  } else if (opt_flags(o) & MOE_FLAG_DETERMINISTIC) {
+    // every (token, slot) row's weighted output in its own row, then the
+    // k rows of each token summed in slot order
+    MOE_TRY(launch_grouped_down(s, T, dn, er, ws, nullptr, ws.ypart, stream));
+    MOE_TRY(mark(o, 3, 1, stream));
+    MOE_TRY(mark(o, 4, 0, stream));
+    MOE_TRY(launch_combine_rows(s, T, er, ws, ws.ypart, sh_gate, sh_y, out, partial_out, stream));
   } else {
     float* acc = partial_out ? partial_out : ws.out_acc;
     MOE_TRY(cudaMemsetAsync(acc, 0, size_t(T) * s.hidden * 4, stream));
-    MOE_TRY(launch_grouped_down(s, T, dn, er, ws, acc, stream));
+    MOE_TRY(launch_grouped_down(s, T, dn, er, ws, acc, nullptr, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
     if (!partial_out) MOE_TRY(launch_finalize_out(ws.out_acc, T, s.hidden, sh_gate, sh_y, out, stream));
@@ -236,9 +265,12 @@ moe_status_t check_forward_common(const moe_shape_t* shape, const uint16_t* x, i
                                   const void* dn, void* workspace, size_t ws_bytes, uint16_t* out,
                                   const moe_forward_opts_t* opts, bool* decode) {
   moe_status_t st = check_forward_inputs(shape, x, T, gu, dn, out, opts, decode);
-  if (st != MOE_OK || T == 0) return st;
+  if (st != MOE_OK) return st;
+  const uint32_t flags = opts ? opts->flags : 0u;
+  if (flags & ~MOE_FLAG_DETERMINISTIC) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
   if (!workspace || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
-  if (ws_bytes < moe_workspace_bytes(shape, T)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_bytes_flags(shape, T, flags)) return MOE_ERR_WORKSPACE;
   return MOE_OK;
 }
 
@@ -375,6 +407,11 @@ size_t moe_workspace_bytes(const moe_shape_t* shape, int T) {
   return carve_workspace(nullptr, *shape, T).bytes;
 }
 
+size_t moe_workspace_bytes_flags(const moe_shape_t* shape, int T, uint32_t flags) {
+  if (check_shape(shape) != MOE_OK || T < 0 || (flags & ~MOE_FLAG_DETERMINISTIC)) return 0;
+  return carve_workspace(nullptr, *shape, T, flags).bytes;
+}
+
 moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, const uint16_t* router_w,
                          const float* logit_bias, const void* gate_up_packed, const void* down_packed,
                          void* workspace, size_t workspace_bytes, uint16_t* out, const moe_forward_opts_t* opts,
@@ -385,7 +422,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, int T, con
   if (st != MOE_OK || T == 0) return st;
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
-  const Workspace ws = carve_workspace(workspace, s, T);
+  const Workspace ws = carve_workspace(workspace, s, T, opt_flags(opts));
   if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream)) != MOE_OK) return st;
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr, decode,
                         opts, stream)) != MOE_OK)
@@ -408,7 +445,7 @@ moe_status_t moe_forward_partial(const moe_shape_t* shape, const uint16_t* x, in
   if (T == 0) return MOE_OK;
   if (!router_w || !aligned(router_w, 16) || (logit_bias && !aligned(logit_bias, 4))) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
-  const Workspace ws = carve_workspace(workspace, s, T);
+  const Workspace ws = carve_workspace(workspace, s, T, opt_flags(opts));
   if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream)) != MOE_OK) return st;
   const ExpertRange er{expert_begin, expert_begin + num_local_experts};
   if ((st = run_experts(s, T, x, gate_up_local, down_local, er, ws, nullptr, partial_out, decode, opts, stream)) !=
@@ -435,6 +472,7 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const uint16_t* x_host, 
                               void* workspace, size_t workspace_bytes, uint16_t* out_host,
                               const moe_forward_opts_t* opts, cudaStream_t stream) {
   if (check_shape(shape) != MOE_OK || T < 0) return check_shape(shape) != MOE_OK ? check_shape(shape) : MOE_ERR_INVALID_ARG;
+  if (opt_flags(opts)) return MOE_ERR_UNSUPPORTED;  // the flags' larger workspace is not laid out here
   if (T == 0) return MOE_OK;
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < moe_workspace_bytes_host(shape, T))
@@ -467,7 +505,7 @@ moe_status_t moe_forward_routed(const moe_shape_t* shape, const uint16_t* x, int
   if (st != MOE_OK || T == 0) return st;
   if (!topk_ids || !topk_w || !aligned(topk_ids, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
   const moe_shape_t& s = *shape;
-  Workspace ws = carve_workspace(workspace, s, T);
+  Workspace ws = carve_workspace(workspace, s, T, opt_flags(opts));
   ws.topk_ids = const_cast<int32_t*>(topk_ids);
   ws.topk_w = const_cast<float*>(topk_w);
   MOE_TRY(mark(opts, 1, 0, stream));
@@ -520,6 +558,7 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   if (!shared) return MOE_ERR_INVALID_ARG;
   if (shared->inter <= 0) return MOE_ERR_INVALID_ARG;
   if (shared->inter % 64) return MOE_ERR_UNSUPPORTED;
+  if (opt_flags(opts)) return MOE_ERR_UNSUPPORTED;  // the flags' larger workspace is not laid out here
   bool decode = false;
   moe_status_t st = check_forward_common(shape, x, T, gate_up_packed, down_packed, workspace, workspace_bytes,
                                          out, opts, &decode);
@@ -531,7 +570,7 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   const moe_shape_t& s = *shape;
   const int I_s = shared->inter;
   if (workspace_bytes < carve_shared(nullptr, s, I_s, T).bytes) return MOE_ERR_WORKSPACE;
-  const Workspace ws = carve_workspace(workspace, s, T);
+  const Workspace ws = carve_workspace(workspace, s, T, opt_flags(opts));
   const SharedWs sw = carve_shared(workspace, s, I_s, T);
   // the shared expert needs only x: gate_up product, SwiGLU and gate, down
   // product (split-K mma.sync for small batches, tcgen05 above)

@@ -299,6 +299,13 @@ MOE_DEV void bulk_reduce_add_f32(float* gdst, const void* ssrc, uint32_t bytes) 
                "r"(smem_u32(ssrc)), "r"(bytes)
                : "memory");
 }
+// Copy `bytes` of shared memory to global memory (both addresses 16-byte
+// aligned, bytes a multiple of 16), tracked by the thread's bulk async-group.
+MOE_DEV void bulk_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
 MOE_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every bulk operation this thread committed has finished reading
 // its shared-memory source.

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
@@ -77,6 +78,7 @@ struct GemmArgs {
   float* logits;
   uint16_t* act;
   float* out_acc;
+  float* ypart;                // down: per-row outputs [T*k][H] instead of out_acc (deterministic combine)
   uint32_t* status;
 };
 
@@ -552,9 +554,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_barrier_sync(1, 128);
         if (r < t.n) {
-          const int tok = a.sorted_rows[t.p_begin + r] / a.top_k;
           const int rows = min(BM, a.M_total - t.fb * BM);
-          bulk_reduce_add_f32(a.out_acc + size_t(tok) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
+          if (a.ypart) {
+            // the row's own slot of the per-row outputs: summed in slot order later
+            bulk_s2g(a.ypart + size_t(t.p_begin + r) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
+          } else {
+            const int tok = a.sorted_rows[t.p_begin + r] / a.top_k;
+            bulk_reduce_add_f32(a.out_acc + size_t(tok) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
+          }
           bulk_commit_group();
         }
       }
@@ -576,6 +583,49 @@ __global__ void finalize_kernel(const float* __restrict__ acc, long n, int H, co
   float4 v = *reinterpret_cast<const float4*>(acc + i);
   if (sh_y) {
     const float g = sh_gate[i / H];  // H % 4 == 0: the four elements share a token
+    const float4 y = *reinterpret_cast<const float4*>(sh_y + i);
+    v.x += g * y.x;
+    v.y += g * y.y;
+    v.z += g * y.z;
+    v.w += g * y.w;
+  }
+  uint2 o;
+  o.x = pack_bf16x2(v.x, v.y);
+  o.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(out + i) = o;
+}
+
+// out[t] = bf16(sum over slots j in order of ypart[pos[t k + j]] (+ the shared
+// expert's gated output)): the deterministic combine of per-row outputs that
+// already carry their routing weight.  With partial_out, the fp32 sum over
+// the slots whose sorted position lies in [offsets[e_lo], offsets[e_hi]) (an
+// expert-parallel shard's experts) instead.  One thread per 4 features.
+__global__ void combine_rows_kernel(const float* __restrict__ ypart, const int32_t* __restrict__ pos,
+                                    const int32_t* __restrict__ offsets, int e_lo, int e_hi, int T, int H, int k,
+                                    const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
+                                    uint16_t* __restrict__ out, float* __restrict__ partial_out) {
+  pdl_wait();
+  pdl_trigger();
+  const long i = (long(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i >= long(T) * H) return;
+  const int t = int(i / H), f = int(i % H);
+  const int p_lo = offsets[e_lo], p_hi = offsets[e_hi];
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int p = pos[size_t(t) * k + j];
+    if (p < p_lo || p >= p_hi) continue;
+    const float4 y = *reinterpret_cast<const float4*>(ypart + size_t(p) * H + f);
+    v.x += y.x;
+    v.y += y.y;
+    v.z += y.z;
+    v.w += y.w;
+  }
+  if (partial_out) {
+    *reinterpret_cast<float4*>(partial_out + i) = v;
+    return;
+  }
+  if (sh_y) {
+    const float g = sh_gate[t];
     const float4 y = *reinterpret_cast<const float4*>(sh_y + i);
     v.x += g * y.x;
     v.y += g * y.y;
@@ -747,12 +797,13 @@ cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* 
 }
 
 cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                                const Workspace& ws, float* acc, cudaStream_t stream) {
+                                const Workspace& ws, float* acc, float* ypart, cudaStream_t stream) {
   if (T == 0 || er.hi <= er.lo) return cudaSuccess;
   CUtensorMap map;
   if (!make_codes_map(&map, dn.codes, dn.K, s.hidden, er.hi - er.lo)) return cudaErrorInvalidValue;
   GemmArgs a = base_args(s, T, er, ws);
   a.out_acc = acc;
+  a.ypart = ypart;
   a.mode = kDown;
   a.K = s.inter;
   a.M_total = s.hidden;
@@ -765,6 +816,18 @@ cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, con
   if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kDown, MOE_FMT_INT4_G128>(map, a, bound, stream);
   if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kDown, MOE_FMT_NVFP4_G16>(map, a, bound, stream);
   return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
+}
+
+cudaError_t launch_combine_rows(const moe_shape_t& s, int T, const ExpertRange& er, const Workspace& ws,
+                                const float* ypart, const float* sh_gate, const float* sh_y, uint16_t* out,
+                                float* partial_out, cudaStream_t stream) {
+  const long n = long(T) * s.hidden;
+  if (n == 0) return cudaSuccess;
+  const int block = 256;
+  const long threads = (n + 3) / 4;
+  return launch_pdl(combine_rows_kernel, dim3(unsigned((threads + block - 1) / block)), dim3(block), 0, stream,
+                    ypart, (const int32_t*)ws.pos, (const int32_t*)ws.offsets, er.lo, er.hi, T, s.hidden, s.top_k,
+                    sh_gate, sh_y, out, partial_out);
 }
 
 cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_gate, const float* sh_y,

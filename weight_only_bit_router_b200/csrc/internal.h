@@ -76,7 +76,9 @@ struct Workspace {
   size_t bytes;
 };
 
-Workspace carve_workspace(void* base, const moe_shape_t& s, int T);
+// flags: MOE_FLAG_* of the call (the deterministic grouped combine adds the
+// per-row output buffer above kDecodeMaxT tokens)
+Workspace carve_workspace(void* base, const moe_shape_t& s, int T, uint32_t flags = 0);
 size_t permute_block_rows();
 
 // pack.cu
@@ -130,9 +132,16 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int
                                uint32_t* status, cudaStream_t stream);
 cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                    const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
-// adds the weighted expert outputs into acc [T, H] fp32 (zeroed by the caller)
+// adds the weighted expert outputs into acc [T, H] fp32 (zeroed by the
+// caller), or with ypart stores each (token, slot) row's weighted output in
+// ypart [T*k, H] (sorted-row order) for combine_rows
 cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                                const Workspace& ws, float* acc, cudaStream_t stream);
+                                const Workspace& ws, float* acc, float* ypart, cudaStream_t stream);
+// out = bf16(sum over slots in order of ypart rows (+ shared)), or the fp32 sum
+// over the range's slots into partial_out
+cudaError_t launch_combine_rows(const moe_shape_t& s, int T, const ExpertRange& er, const Workspace& ws,
+                                const float* ypart, const float* sh_gate, const float* sh_y, uint16_t* out,
+                                float* partial_out, cudaStream_t stream);
 // out = bf16(acc [+ sh_gate[t] * sh_y[t][f]]) over [T, H] (sh_* nullable)
 cudaError_t launch_finalize_out(const float* acc, int T, int H, const float* sh_gate, const float* sh_y,
                                 uint16_t* out, cudaStream_t stream);

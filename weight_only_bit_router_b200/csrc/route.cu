@@ -554,8 +554,6 @@ __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
     int32_t* __restrict__ pos, int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n,
     int32_t* done_counter) {
   __shared__ RouteFastSmem sm;
-  pdl_wait();
-  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const int e0 = blockIdx.x * kRsExperts, ks = blockIdx.y, KS = gridDim.y;
@@ -563,12 +561,19 @@ __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
   const int b = warp & 1, jt = warp >> 1;
   const int kblk = ks * kRfK + b * 128 + 32 * q;
   const bool kin = kblk < H;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // the router weight does not depend on the kernels before: its fragments
+  // are loaded before the programmatic-launch wait
+  uint32_t alo[8][2], ahi[8][2];
   if (jt < NT) {
     const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
-    uint32_t alo[8][2], ahi[8][2], bf[8][2];
     bf16_frags(wr + size_t(r_lo ? e0 + g : 0) * H + kblk, r_lo && kin, alo);
     bf16_frags(wr + size_t(r_hi ? e0 + g + 8 : 0) * H + kblk, r_hi && kin, ahi);
+  }
+  pdl_wait();
+  pdl_trigger();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (jt < NT) {
+    uint32_t bf[8][2];
     const int t = jt * 8 + g;
     bf16_frags(x + size_t(t < T ? t : 0) * H + kblk, t < T && kin, bf);
 #pragma unroll
