@@ -221,7 +221,8 @@ MOE_DEV void dequant_store32(uint4 codes, uint32_t mult, uint32_t mult2, uint32_
 
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const GemmArgs args) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const GemmArgs args) {
   using C = Cfg<MODE, FMT>;
   constexpr int SA = C::SA;
   constexpr int kSrow = C::SROW;
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&opA_empty[i], 1);
     }
     for (int i = 0; i < SB; ++i) {
-      mbar_init(&opB_full[i], 64);
+      mbar_init(&opB_full[i], MODE == kDown ? 1 : 64);
       mbar_init(&opB_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -283,7 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_a);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_a);
+    if (MODE == kDown) tma_prefetch_desc(&tmap_b);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -395,6 +399,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int never = 0;
         umma_commit(drain);
         mbar_wait(drain, 0, &never, nullptr);
+      }
+    }
+  } else if (MODE == kDown && (warp == 2 || warp == 3)) {
+    // ------------------------------------------------------------ activation tiles
+    // The expert's activation rows are contiguous in sorted-row order: one
+    // 2-D TMA copy (64 k x 128 rows, 128-byte swizzle) per stage.  Rows past
+    // the expert's count belong to the next experts (their columns are not
+    // used); rows past the array read as zeros.
+    if (warp == 2 && lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(a, tile, s_tile_base);
+        for (int ks = 0; ks < KS; ++ks, ++g) {
+          const int s = g % SB;
+          if (!(ok = mbar_wait(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status))) break;
+          mbar_arrive_expect_tx(&opB_full[s], kTileBytes);
+          tma_load_2d(sB + s * kTileBytes, &tmap_b, &opB_full[s], ks * BK, t.p_begin);
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA unwinds
+        volatile int never = 0;
+        for (uint32_t i = 0; i < SB && i < g; ++i) {
+          const uint32_t gg = g - 1 - i;
+          mbar_wait(&opB_full[gg % SB], (gg / SB) & 1, &never, nullptr);
+        }
       }
     }
   } else if (warp == 2 || warp == 3) {
@@ -699,7 +730,8 @@ int sm_count() {
 }
 
 template <int MODE, int FMT>
-cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ctas, cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& map_b, const GemmArgs& args, int max_ctas,
+                        cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<MODE, FMT>;
   const int smem = Cfg<MODE, FMT>::SMEM;
   // once per process (and per device), outside any stream capture of later calls
@@ -712,7 +744,7 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int max_ct
     configured_device.store(dev);
   }
   const int grid = max(1, min(sm_count(), max_ctas));
-  kern<<<grid, kThreads, smem, stream>>>(map, args);
+  kern<<<grid, kThreads, smem, stream>>>(map, map_b, args);
   return cudaGetLastError();
 }
 
@@ -764,7 +796,7 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wr, int T, int
   a.logits = logits;
   a.status = status;
   const int tiles = a.n_ftiles * ((T + BN - 1) / BN);
-  return launch_gemm<kRouter, 0>(map, a, tiles, stream);
+  return launch_gemm<kRouter, 0>(map, map, a, tiles, stream);
 }
 
 bool grouped_supported(const moe_shape_t& s) {
@@ -791,9 +823,9 @@ cudaError_t launch_grouped_gate_up(const moe_shape_t& s, int T, const uint16_t* 
   a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(gu.K) : s.fmt == MOE_FMT_NVFP4_G16 ? gu.K / 16 : gu.K / 32;
   a.gscale = gu.gscale;
   const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
-  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kGateUp, MOE_FMT_INT4_G128>(map, a, bound, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kGateUp, MOE_FMT_NVFP4_G16>(map, a, bound, stream);
-  return launch_gemm<kGateUp, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
+  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kGateUp, MOE_FMT_INT4_G128>(map, map, a, bound, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kGateUp, MOE_FMT_NVFP4_G16>(map, map, a, bound, stream);
+  return launch_gemm<kGateUp, MOE_FMT_MXFP4_G32>(map, map, a, bound, stream);
 }
 
 cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
@@ -813,9 +845,12 @@ cudaError_t launch_grouped_down(const moe_shape_t& s, int T, const Bank& dn, con
   a.scale_row_stride = s.fmt == MOE_FMT_INT4_G128 ? int4_groups(dn.K) : s.fmt == MOE_FMT_NVFP4_G16 ? dn.K / 16 : dn.K / 32;
   a.gscale = dn.gscale;
   const int bound = grouped_tiles_bound(T, s.top_k, s.num_experts, a.n_ftiles);
-  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kDown, MOE_FMT_INT4_G128>(map, a, bound, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kDown, MOE_FMT_NVFP4_G16>(map, a, bound, stream);
-  return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, a, bound, stream);
+  // the activation rows [T*k, I] bf16 in sorted order, tiles of 64 k x 128 rows
+  CUtensorMap map_b;
+  if (!make_bf16_sw128_map(&map_b, ws.act, s.inter, T * s.top_k)) return cudaErrorInvalidValue;
+  if (s.fmt == MOE_FMT_INT4_G128) return launch_gemm<kDown, MOE_FMT_INT4_G128>(map, map_b, a, bound, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return launch_gemm<kDown, MOE_FMT_NVFP4_G16>(map, map_b, a, bound, stream);
+  return launch_gemm<kDown, MOE_FMT_MXFP4_G32>(map, map_b, a, bound, stream);
 }
 
 cudaError_t launch_combine_rows(const moe_shape_t& s, int T, const ExpertRange& er, const Workspace& ws,
