@@ -26,10 +26,20 @@ namespace {
 
 constexpr int kGroupWarps = 4;  // consumer warps per work unit
 
-// Number of consumer groups (units in flight through compute) per CTA and
-// shared-memory stages per CTA.
-constexpr int kGroups = 2;
-constexpr int kStages = 4;
+// Number of consumer groups (units in flight through compute) per CTA,
+// shared-memory stages per CTA, and CTAs per SM the register budget is sized
+// for (build-time tuning knobs; the defaults are the measured best).
+#ifndef MOE_DEC_GROUPS
+#define MOE_DEC_GROUPS 2
+#endif
+#ifndef MOE_DEC_STAGES
+#define MOE_DEC_STAGES 4
+#endif
+#ifndef MOE_DEC_MIN_CTAS
+#define MOE_DEC_MIN_CTAS 2
+#endif
+constexpr int kGroups = MOE_DEC_GROUPS;
+constexpr int kStages = MOE_DEC_STAGES;
 constexpr int kThreads = (kGroups * kGroupWarps + 1) * 32;
 
 // The routing state every CTA keeps in shared memory: the touched-expert list
@@ -87,7 +97,7 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // shared memory (one bulk copy per row, padded row stride).
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
     uint16_t* __restrict__ act, uint32_t* status) {
@@ -169,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
     const int u = blockIdx.x + i * gridDim.x;
     if (u >= n_units) break;
     const int st = i % S;
-    const bool ok = x_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status);
+    // warp-uniform: the MMAs below run only if every lane saw the data land
+    const bool ok = __all_sync(0xffffffffu, x_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status));
     const int e = s_local[u / ftiles];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
     const int f0 = (u % ftiles) * 8;
@@ -196,7 +207,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_gate_up_kern
       auto block = [&](int b, bool in) {
         const RowChunk lo = row_chunk_at<FMT>(c_gate, sc_gate, b, q, in, gsc);
         const RowChunk hi = row_chunk_at<FMT>(c_up, sc_up, b, q, in, gsc);
-        const bool fast = (lo.fast & hi.fast) != 0u;
+        // warp-uniform: mma.sync needs the whole warp on one path (the
+        // two-step path is exact for every scale)
+        const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           if (j >= ntiles) break;
@@ -264,7 +277,7 @@ constexpr int kDnRows = 64;           // output features per unit
 constexpr int kDnCounterBase = 16;    // first tile counter in the workspace's status region (int32 index)
 
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
+__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const uint16_t* __restrict__ act, const float* __restrict__ topk_w,
     const int32_t* __restrict__ pos, float* __restrict__ ypart, uint16_t* __restrict__ out,
@@ -360,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
     const int u = blockIdx.x + i * gridDim.x;
     if (u >= n_units) break;
     const int st = i % S;
-    const bool ok = act_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status);
+    const bool ok = __all_sync(0xffffffffu, act_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status));
     const int e = s_local[u % n_t];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
     const int rt = (u / n_t) * (kDnRows / 16) + wj;  // this warp's 16-row feature tile
@@ -380,7 +393,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
       auto block = [&](int b, bool in) {
         const RowChunk lo = row_chunk_at<FMT>(c_lo, sc_lo, b, q, in, gsc);
         const RowChunk hi = row_chunk_at<FMT>(c_hi, sc_hi, b, q, in, gsc);
-        const bool fast = (lo.fast & hi.fast) != 0u;
+        // warp-uniform: mma.sync needs the whole warp on one path (the
+        // two-step path is exact for every scale)
+        const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           if (j >= ntiles) break;
@@ -426,10 +441,17 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : 2) decode_down_kernel(
       for (int idx = lane; idx < T * 16; idx += 32) {
         const int t = idx >> 4, f = 16 * rt + (idx & 15);
         float sum = 0.f;
-        for (int j = 0; j < top_k; ++j) {
-          const int r = t * top_k + j;
-          const int p = s_pos[r];
-          if (p >= p_lo && p < p_hi) sum += s_w[r] * __ldcg(ypart + size_t(p) * H + f);
+        // eight slots' loads in flight at once, summed in slot order
+        for (int j0 = 0; j0 < top_k; j0 += 8) {
+          float v[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int r = t * top_k + j0 + jj;
+            const int p = j0 + jj < top_k ? s_pos[r] : -1;
+            v[jj] = (p >= p_lo && p < p_hi) ? s_w[r] * __ldcg(ypart + size_t(p) * H + f) : 0.f;
+          }
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) sum += v[jj];
         }
         if (sh_y) sum += sh_gate[t] * sh_y[size_t(t) * H + f];  // the shared expert, before the one rounding
         if (partial_out) partial_out[size_t(t) * H + f] = sum;
