@@ -291,6 +291,12 @@ MOE_DEV void bulk_g2s_hint(void* smem_dst, const void* gsrc, uint32_t bytes, uin
       : "memory");
 }
 
+// Prefetch `bytes` of global memory into L2 (address 16-byte aligned, bytes a
+// multiple of 16): a later bulk copy of the range then reads L2, not HBM.
+MOE_DEV void bulk_prefetch_l2(const void* gsrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
+}
+
 // Element-wise fp32 add of `bytes` of shared memory into global memory
 // (performed at L2; both addresses 16-byte aligned, bytes a multiple of 16),
 // tracked by the issuing thread's bulk async-group.

@@ -163,6 +163,13 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
         mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(gu, 16));
         stage_rows<FMT>(gu, row_g, 8, stage, stage + L.cbytes, &full[st], policy);
         stage_rows<FMT>(gu, row_g + I, 8, stage + 8 * (K / 2), stage + L.cbytes + 8 * srow, &full[st], policy);
+        // the unit that will refill this stage, into L2 ahead of time
+        const int un = u + S * gridDim.x;
+        if (un < n_units) {
+          const long rn = long(s_local[un / ftiles] - e_lo) * gu.N + (un % ftiles) * 8;
+          prefetch_rows<FMT>(gu, rn, 8);
+          prefetch_rows<FMT>(gu, rn + I, 8);
+        }
       }
       drain_stages(full, i, S);
     }
@@ -348,6 +355,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(dn, kDnRows));
         stage_rows<FMT>(dn, row0, kDnRows, stage, stage + L.cbytes, &full[st], policy);
+        // the unit that will refill this stage, into L2 ahead of time
+        const int un = u + S * gridDim.x;
+        if (un < n_units) prefetch_rows<FMT>(dn, long(s_local[un % n_t] - e_lo) * H + (un / n_t) * kDnRows, kDnRows);
       }
       drain_stages(full, i, S);
     }

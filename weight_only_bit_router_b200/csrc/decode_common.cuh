@@ -221,6 +221,14 @@ MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, u
   bulk_g2s_hint(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar, policy);
 }
 
+// Prefetch into L2 the codes and scales of `rows` consecutive weight rows.
+template <int FMT>
+MOE_DEV void prefetch_rows(const Bank& bk, long row0, int rows) {
+  const int sb = scale_row_bytes(FMT, bk.K);
+  bulk_prefetch_l2(bk.codes + row0 * (bk.K / 2), uint32_t(rows) * (bk.K / 2));
+  bulk_prefetch_l2(static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb);
+}
+
 // Shared-memory layout of one staged work unit of `rows` weight rows: codes,
 // then scales padded to 16 bytes.
 struct UnitLayout {

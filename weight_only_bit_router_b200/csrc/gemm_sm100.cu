@@ -154,6 +154,17 @@ MOE_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, 
       : "memory");
 }
 
+// Prefetch the box at (x, y, z) of a 3-D tensor map into L2.
+MOE_DEV void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+// Code tiles this many k-stages ahead of the producer are prefetched into L2.
+constexpr int kCodePrefetch = 8;
+
 // bf16x2 with both halves = 2^e (e in [-127, 127]).
 MOE_DEV uint32_t pow2x2(int e) {
   const uint32_t b = e >= -126 ? uint32_t(e + 127) << 7 : 0x0040u;
@@ -303,6 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const Tile t = decode_tile(a, tile, s_tile_base);
+        // the CTA's next tile, for the L2 prefetch of code tiles ahead of the ring
+        const bool has_next = tile + int(gridDim.x) < ntiles;
+        const Tile tn = has_next ? decode_tile(a, tile + gridDim.x, s_tile_base) : t;
         if (MODE != kRouter) {
           // the tile's scale rows: contiguous rows of the scale plane, once per tile
           const int slot = it & 1;
@@ -336,6 +350,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(dst + kCodeBytes, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, 2 * t.eb + 1);
             } else {
               tma_load_3d(dst, &tmap_a, &codes_full[s], ks * (BK / 2), t.fb * BM, t.eb);
+            }
+            // the code tile kCodePrefetch stages ahead, into L2
+            const int kp = ks + kCodePrefetch;
+            if (kp < KS || has_next) {
+              const Tile& tp = kp < KS ? t : tn;
+              const int kq = kp < KS ? kp : kp - KS;
+              if (kq < KS) {
+                if (MODE == kGateUp) {
+                  tma_prefetch_3d(&tmap_a, kq * (BK / 2), tp.fb * BM, 2 * tp.eb);
+                  tma_prefetch_3d(&tmap_a, kq * (BK / 2), tp.fb * BM, 2 * tp.eb + 1);
+                } else {
+                  tma_prefetch_3d(&tmap_a, kq * (BK / 2), tp.fb * BM, tp.eb);
+                }
+              }
             }
           }
         }
