@@ -255,9 +255,8 @@ typedef enum {
 #define MOE_NUM_STAGES 5
 /* Stage ids: 0 router logits, 1 top-k + permutation, 2 gate_up + SwiGLU,
  * 3 down projection, 4 weighted combine / output conversion.  Where one
- * kernel does two stages (small batches: routing and permutation in one, down
- * projection and combine in one) the second stage's events bracket nothing
- * and it reads zero. */
+ * kernel does two stages (small batches: routing and permutation in one) the
+ * second stage's events bracket nothing and it reads zero. */
 
 /* Optional extras of moe_forward / moe_forward_routed.  Every pointer may be
  * NULL; a NULL opts pointer means all defaults. */

@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests (the oracle side runs on the CPU)."""
+import concurrent.futures
 import json
+import multiprocessing
 import os
 
 import numpy as np
@@ -11,10 +13,29 @@ from oracle import moe_oracle as o
 FMT_NAMES = {"int4_g128": o.FMT_INT4, "mxfp4": o.FMT_MXFP4, "nvfp4": o.FMT_NVFP4}
 
 
+_POOL = None
+
+
+def oracle_pool():
+    """Worker processes for the oracle's per-expert packing (started with
+    spawn: the test process already holds a CUDA context)."""
+    global _POOL
+    if _POOL is None:
+        workers = max(1, min(16, (os.cpu_count() or 2) - 1))
+        _POOL = concurrent.futures.ProcessPoolExecutor(max_workers=workers,
+                                                       mp_context=multiprocessing.get_context("spawn"))
+    return _POOL
+
+
+def _pack_dequant(fmt, bits):
+    return o.dequant(fmt, *o.pack(fmt, bits))
+
+
 class LazyOracleBank:
     """Oracle-packed, oracle-dequantised experts of a bf16 bank that lives on
     the GPU; each expert is copied to the host and packed by the oracle on
-    first use (so big banks are only packed where a test needs them)."""
+    first use (so big banks are only packed where a test needs them).
+    prefetch() packs a set of experts in parallel worker processes."""
 
     def __init__(self, fmt: str, bank_bf16: torch.Tensor):
         self.fmt = FMT_NAMES[fmt]
@@ -23,6 +44,14 @@ class LazyOracleBank:
 
     def packed(self, e: int):
         return o.pack(self.fmt, moe_synth.bf16_bits(self.bank[e]))
+
+    def prefetch(self, experts):
+        todo = sorted(set(int(e) for e in np.asarray(experts).ravel()) - set(self._cache))
+        if len(todo) < 2:
+            return
+        futs = {e: oracle_pool().submit(_pack_dequant, self.fmt, moe_synth.bf16_bits(self.bank[e])) for e in todo}
+        for e, f in futs.items():
+            self._cache[e] = f.result()
 
     def expert(self, e: int):
         if e not in self._cache:

@@ -233,6 +233,8 @@ def verify_layer(layer, fmt, out, dbg, path=None, sample=None, name=""):
         assert np.array_equal(dbg["sorted_rows_out"].cpu().numpy(), rs)
     gu = LazyOracleBank(fmt, layer.gate_up)
     dn = LazyOracleBank(fmt, layer.down)
+    gu.prefetch(rid)
+    dn.prefetch(rid)
     a_exact, a_round = o.expert_activations(xb, rid, gu, s.num_experts)
     gpu_act = gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k)
     act_used, n_diff = flip_aware_activations(gpu_act, a_exact, a_round)
@@ -380,11 +382,13 @@ def test_deterministic_flag_needs_its_workspace():
 
 
 def scaled_layer(shape, T, seed, gate_up_scale=1.0, down_scale=1.0, x_scale=1.0):
-    """A layer whose banks (and tokens) are multiplied by powers of two, rounded
-    to bf16 again (exact unless the scaled value leaves bf16's normal range)."""
+    """A layer whose banks and tokens are multiplied by powers of two, rounded
+    to bf16 again (exact unless the scaled value leaves bf16's normal range);
+    the router weight takes the inverse of the tokens' factor, so the logits
+    keep their size."""
     layer = moe_synth.make_layer(shape, T=T, seed=seed, device=DEV)
     scale = lambda t, f: (t.float() * f).to(torch.bfloat16) if f != 1.0 else t
-    return moe_synth.Layer(shape=shape, x=scale(layer.x, x_scale), router_w=layer.router_w,
+    return moe_synth.Layer(shape=shape, x=scale(layer.x, x_scale), router_w=scale(layer.router_w, 1.0 / x_scale),
                            gate_up=scale(layer.gate_up, gate_up_scale), down=scale(layer.down, down_scale),
                            bias=None)
 

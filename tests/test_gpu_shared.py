@@ -54,6 +54,8 @@ def check_shared(layer, fmt, inter_shared, path=None, sample=None, seed=0):
     rid, rw = o.route(dbg["logits_out"][tok_d].cpu().numpy(), bias, s.top_k)
     assert np.array_equal(rid, dbg["topk_ids_out"][tok_d].cpu().numpy())
     gub, dnb = LazyOracleBank(fmt, layer.gate_up), LazyOracleBank(fmt, layer.down)
+    gub.prefetch(rid)
+    dnb.prefetch(rid)
     a_exact, a_round = o.expert_activations(xb, rid, gub, s.num_experts)
     gpu_act = gpu_activations_in_oracle_order(dbg, tok, rid, s.num_experts, s.top_k)
     act_used, n_diff = flip_aware_activations(gpu_act, a_exact, a_round)

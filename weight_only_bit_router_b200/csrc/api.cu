@@ -192,15 +192,14 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
     else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
     MOE_TRY(mark(o, 2, 1, stream));
   }
-  NvtxRange range(decode ? "moe.down_combine" : "moe.down");
+  NvtxRange range("moe.down_combine");
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
-    // down projection and the combine are one kernel on this path; a shard
-    // without routed rows writes nothing, so its partial output starts at zero
-    if (partial_out) MOE_TRY(cudaMemsetAsync(partial_out, 0, size_t(T) * s.hidden * 4, stream));
-    MOE_TRY(launch_decode_down_combine(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream));
+    // routing-weighted per-row outputs, then each token's slot rows summed in order
+    MOE_TRY(launch_decode_down(s, T, dn, er, ws, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
+    MOE_TRY(launch_combine_rows(s, T, er, ws, ws.ypart, sh_gate, sh_y, out, partial_out, stream));
   } else if (opt_flags(o) & MOE_FLAG_DETERMINISTIC) {
     // every (token, slot) row's weighted output in its own row, then the
     // k rows of each token summed in slot order
@@ -616,7 +615,7 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   if (routed) n += perm;
   else if (T <= kDecodeMaxT) n += 1;                          // fused router + top-k + permutation
   else n += 2 + perm;                                         // router GEMM, top-k, permutation
-  n += decode ? 2 : 3;                                        // gate_up, down (+ combine) / finalize
+  n += 3;                                                     // gate_up, down, combine / finalize
   return n;
 }
 

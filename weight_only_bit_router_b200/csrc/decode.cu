@@ -38,6 +38,11 @@ constexpr int kGroupWarps = 4;  // consumer warps per work unit
 #ifndef MOE_DEC_MIN_CTAS
 #define MOE_DEC_MIN_CTAS 2
 #endif
+// registers per thread that keep MOE_DEC_MIN_CTAS CTAs per SM (65536 per SM,
+// allocated in multiples of 8 per thread); one CTA per SM above 8 tokens
+constexpr int kDecRegs = (65536 / (MOE_DEC_MIN_CTAS * (MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8;
+constexpr int kDecRegsWide = (65536 / ((MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8 > 255
+                                 ? 248 : (65536 / ((MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8;
 constexpr int kGroups = MOE_DEC_GROUPS;
 constexpr int kStages = MOE_DEC_STAGES;
 constexpr int kThreads = (kGroups * kGroupWarps + 1) * 32;
@@ -77,6 +82,35 @@ MOE_DEV void local_slice(const int* s_touched, int e_lo, int e_hi, int E, int* s
   *t_hi = s_cnt[0] + s_cnt[1];
 }
 
+// Activation fragments of the gate_up kernel: token rows of x (staged in
+// shared memory, or read through L1) for the token tiles of one unit.
+template <int NT, bool X_SMEM>
+struct XFrags {
+  const uint16_t* x;      // global x [T, K]
+  const uint8_t* x_s;     // staged rows (X_SMEM)
+  int xstride, K, q;
+  int tok[NT];            // token of column 8j + g
+  MOE_DEV void load(int j, int b, bool in, uint32_t (&bf)[8][2]) const {
+    if (X_SMEM) act_frags<0>(reinterpret_cast<const uint16_t*>(x_s + tok[j] * xstride) + 128 * b + 32 * q, in, bf);
+    else act_frags<1>(x + size_t(tok[j]) * K + 128 * b + 32 * q, in, bf);
+  }
+};
+
+// Activation fragments of the down kernel: the expert's bf16 SwiGLU rows p
+// (staged in shared memory, or read through L2: another kernel wrote them).
+template <bool ACT_SMEM>
+struct ActFrags {
+  const uint16_t* act;    // global act [T*k, K]
+  const uint8_t* act_s;   // staged rows (ACT_SMEM)
+  int astride, K, q, g, p0, n_e;
+  MOE_DEV void load(int j, int b, bool in, uint32_t (&bf)[8][2]) const {
+    const int c = 8 * j + g;
+    const int p = p0 + (c < n_e ? c : 0);
+    if (ACT_SMEM) act_frags<0>(reinterpret_cast<const uint16_t*>(act_s + p * astride) + 128 * b + 32 * q, in, bf);
+    else act_frags<2>(act + size_t(p) * K + 128 * b + 32 * q, in, bf);
+  }
+};
+
 // Let the last bulk copies of this CTA's producer land before its shared
 // memory is released (bounded: they complete unless the GPU is failing).
 MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
@@ -97,7 +131,7 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // shared memory (one bulk copy per row, padded row stride).
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) decode_gate_up_kernel(
+__global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
     uint16_t* __restrict__ act, uint32_t* status) {
@@ -198,40 +232,31 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
     const uint8_t* sc_up = sc_gate + 8 * srow;
     const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[e - e_lo] : 0.f;
     const int ntiles = min(NT, (n_e + 7) / 8);
+    XFrags<NT, X_SMEM> xf;
+    xf.x = x;
+    xf.x_s = x_s;
+    xf.xstride = xstride;
+    xf.K = K;
+    xf.q = q;
     // token of column 8j + g (a valid token's row for the padding columns)
-    int xtok[NT];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int c = 8 * j + g;
-      xtok[j] = s_tok[p0 + (c < n_e ? c : 0)];
+      xf.tok[j] = s_tok[p0 + (c < n_e ? c : 0)];
     }
+    float acc2[NT][2][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc2[j][0][c] = acc2[j][1][c] = 0.f;
+    if (ok)
+      stream_kblocks<FMT, NT>(acc2, wj, kGroupWarps, nblk_full, (tail && nblk_full % kGroupWarps == wj) ? nblk_full : -1,
+                              K, q, c_gate, c_up, sc_gate, sc_up, gsc, ntiles, xf);
     float acc[NT][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
-    if (ok) {
-      auto block = [&](int b, bool in) {
-        const RowChunk lo = row_chunk_at<FMT>(c_gate, sc_gate, b, q, in, gsc);
-        const RowChunk hi = row_chunk_at<FMT>(c_up, sc_up, b, q, in, gsc);
-        // warp-uniform: mma.sync needs the whole warp on one path (the
-        // two-step path is exact for every scale)
-        const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j >= ntiles) break;
-          uint32_t bf[8][2];
-          if (X_SMEM)
-            act_frags<0>(reinterpret_cast<const uint16_t*>(x_s + xtok[j] * xstride) + 128 * b + 32 * q, in, bf);
-          else
-            act_frags<1>(x + size_t(xtok[j]) * K + 128 * b + 32 * q, in, bf);
-          if (fast) mma_block_path<FMT, true>(acc[j], lo, hi, bf);
-          else mma_block_path<FMT, false>(acc[j], lo, hi, bf);
-        }
-      };
-      for (int b = wj; b < nblk_full; b += kGroupWarps) block(b, true);
-      if (tail && nblk_full % kGroupWarps == wj) block(nblk_full, 128 * nblk_full + 32 * q < K);
-    }
+      for (int c = 0; c < 4; ++c) acc[j][c] = acc2[j][0][c] + acc2[j][1][c];
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
     // the group's partial tiles, double-buffered by unit parity
@@ -264,32 +289,25 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
 }
 
 // ---------------------------------------------------------------------------
-// down projection + deterministic combine.  Work unit u = (feature tile
-// ft = u / n of 64 output features, touched slot u % n): the expert's 64 down
-// rows (all of K = I).  Consumer warp w of the unit's group takes rows
-// 16 w .. 16 w + 15 over every k-block and writes y = Wd a for each of the
-// expert's rows p (fp32, unweighted) to ypart[p][f].  A counter per 16-row
-// feature tile counts the warps that wrote it; the warp that completes it
-// (last of n touched experts) sums, for every token t and feature f of the
-// tile, w_tj * ypart[pos(t, j)][f] over the slots j in order (plus the shared
-// expert's gated output) and rounds once to bf16.  The sum order is fixed, so
-// the output is deterministic.
+// down projection.  Work unit u = (feature tile ft = u / n of 64 output
+// features, touched slot u % n): the expert's 64 down rows (all of K = I).
+// Consumer warp w of the unit's group takes rows 16 w .. 16 w + 15 over every
+// k-block and writes w_tj * (Wd a) for each of the expert's sorted rows p
+// (fp32, scaled by the row's routing weight) to ypart[p][f].  The combine
+// kernel that follows sums each token's k rows in slot order (deterministic).
 // The weights do not depend on the gate_up kernel that runs just before: the
 // producer reads the routing state (written two launches back, and the kernel
 // in between triggers its dependents only after its own wait) and starts the
 // weight copies before the programmatic-launch wait; only the consumers wait.
 // With ACT_SMEM (small T) one consumer warp stages the T*k activation rows.
 // ---------------------------------------------------------------------------
-constexpr int kDnRows = 64;           // output features per unit
-constexpr int kDnCounterBase = 16;    // first tile counter in the workspace's status region (int32 index)
+constexpr int kDnRows = 64;  // output features per unit
 
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) decode_down_kernel(
+__global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
-    const int32_t* __restrict__ offsets, const uint16_t* __restrict__ act, const float* __restrict__ topk_w,
-    const int32_t* __restrict__ pos, float* __restrict__ ypart, uint16_t* __restrict__ out,
-    float* __restrict__ partial_out, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
-    uint32_t* status) {
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
+    const float* __restrict__ topk_w, float* __restrict__ ypart, uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int G = kGroups, S = kStages;
   const int H = dn.N, K = dn.K;  // K = I
@@ -301,12 +319,10 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
   uint8_t* act_s = ring + S * L.stage_bytes;             // [R][astride] (ACT_SMEM)
   int* s_touched = reinterpret_cast<int*>(act_s + (ACT_SMEM ? R * astride : 0));
   int* s_off = s_touched + (E + 1);
-  int* s_pos = s_off + (E + 1);                          // [R] sorted position of row r = t*k + j
-  float* s_w = reinterpret_cast<float*>(s_pos + R);      // [R] routing weight of row r
-  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_w + R) + 7) & ~uintptr_t(7));
+  float* s_wrow = reinterpret_cast<float*>(s_off + (E + 1));  // [R] routing weight of sorted row p
+  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_wrow + R) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + S;
   uint64_t* act_bar = empty + S;
-  uint32_t* tile_cnt = status + kDnCounterBase;
   __shared__ volatile int s_abort;
   __shared__ int s_cnt[2];
 
@@ -322,10 +338,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
   }
   // routing state: written two launches back (see above), read through L2
   load_routing(s_touched, s_off, touched, offsets, E);
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    s_pos[r] = __ldcg(pos + r);
-    s_w[r] = __ldcg(topk_w + r);
-  }
+  for (int p = threadIdx.x; p < R; p += blockDim.x) s_wrow[p] = __ldcg(topk_w + __ldcg(sorted_rows + p));
   __syncthreads();
   int t_lo, t_hi;
   local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
@@ -367,12 +380,12 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
   }
 
   // -------------------------------------------------------------------- consumers
-  pdl_wait();  // the activations (and the outputs' previous readers) of the kernels before
+  pdl_wait();  // the activations (and the previous readers of ypart) of the kernels before
   pdl_trigger();
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
   const int nblk_full = K / 128;
-  const bool tail = (K % 128) != 0;
+  const int tail = (K % 128) != 0 ? nblk_full : -1;
   if (ACT_SMEM && warp == 0) {
     if (lane == 0) mbar_arrive_expect_tx(act_bar, uint32_t(R) * uint32_t(2 * K));
     __syncwarp();
@@ -383,10 +396,11 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
     const int u = blockIdx.x + i * gridDim.x;
     if (u >= n_units) break;
     const int st = i % S;
+    // warp-uniform: the MMAs below run only if every lane saw the data land
     const bool ok = __all_sync(0xffffffffu, act_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status));
     const int e = s_local[u % n_t];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-    const int rt = (u / n_t) * (kDnRows / 16) + wj;  // this warp's 16-row feature tile
+    const int f0 = (u / n_t) * kDnRows + 16 * wj;  // this warp's 16 output features
     const uint8_t* s_c = ring + st * L.stage_bytes;
     const uint8_t* c_lo = s_c + (16 * wj + g) * (K / 2) + 16 * q;
     const uint8_t* c_hi = c_lo + 8 * (K / 2);
@@ -394,80 +408,34 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 1 : MOE_DEC_MIN_CTAS) deco
     const uint8_t* sc_hi = sc_lo + 8 * srow;
     const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
     const int ntiles = min(NT, (n_e + 7) / 8);
-    float acc[NT][4];
+    ActFrags<ACT_SMEM> af;
+    af.act = act;
+    af.act_s = act_s;
+    af.astride = astride;
+    af.K = K;
+    af.q = q;
+    af.g = g;
+    af.p0 = p0;
+    af.n_e = n_e;
+    float acc2[NT][2][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
-    if (ok) {
-      auto block = [&](int b, bool in) {
-        const RowChunk lo = row_chunk_at<FMT>(c_lo, sc_lo, b, q, in, gsc);
-        const RowChunk hi = row_chunk_at<FMT>(c_hi, sc_hi, b, q, in, gsc);
-        // warp-uniform: mma.sync needs the whole warp on one path (the
-        // two-step path is exact for every scale)
-        const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j >= ntiles) break;
-          const int c = 8 * j + g;
-          const int p = p0 + (c < n_e ? c : 0);
-          uint32_t bf[8][2];
-          if (ACT_SMEM)
-            act_frags<0>(reinterpret_cast<const uint16_t*>(act_s + p * astride) + 128 * b + 32 * q, in, bf);
-          else
-            act_frags<2>(act + size_t(p) * K + 128 * b + 32 * q, in, bf);
-          if (fast) mma_block_path<FMT, true>(acc[j], lo, hi, bf);
-          else mma_block_path<FMT, false>(acc[j], lo, hi, bf);
-        }
-      };
-      for (int b = 0; b < nblk_full; ++b) block(b, true);
-      if (tail) block(nblk_full, 128 * nblk_full + 32 * q < K);
-    }
+      for (int c = 0; c < 4; ++c) acc2[j][0][c] = acc2[j][1][c] = 0.f;
+    if (ok) stream_kblocks<FMT, NT>(acc2, 0, 1, nblk_full, tail, K, q, c_lo, c_hi, sc_lo, sc_hi, gsc, ntiles, af);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     if (!ok) continue;
-    // c0, c1: feature 16 rt + g at columns 2q, 2q+1; c2, c3: feature + 8
+    // c0, c1: feature f0 + g at columns 2q, 2q+1; c2, c3: feature + 8
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       if (j >= ntiles) break;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col = 8 * j + 2 * q + (c & 1);
-        if (col < n_e) ypart[size_t(p0 + col) * H + 16 * rt + g + 8 * (c >> 1)] = acc[j][c];
+        if (col < n_e)
+          ypart[size_t(p0 + col) * H + f0 + g + 8 * (c >> 1)] = s_wrow[p0 + col] * (acc2[j][0][c] + acc2[j][1][c]);
       }
-    }
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(&tile_cnt[rt], 1u) == uint32_t(n_t - 1);
-    }
-    if (__shfl_sync(0xffffffffu, last, 0)) {
-      // every touched expert's rows of this tile are written: the combine
-      // over the slots whose expert is in the bank's range (sorted positions
-      // [offsets[e_lo], offsets[e_hi]))
-      __threadfence();
-      const int p_lo = s_off[e_lo], p_hi = s_off[e_hi];
-      for (int idx = lane; idx < T * 16; idx += 32) {
-        const int t = idx >> 4, f = 16 * rt + (idx & 15);
-        float sum = 0.f;
-        // eight slots' loads in flight at once, summed in slot order
-        for (int j0 = 0; j0 < top_k; j0 += 8) {
-          float v[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int r = t * top_k + j0 + jj;
-            const int p = j0 + jj < top_k ? s_pos[r] : -1;
-            v[jj] = (p >= p_lo && p < p_hi) ? s_w[r] * __ldcg(ypart + size_t(p) * H + f) : 0.f;
-          }
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) sum += v[jj];
-        }
-        if (sh_y) sum += sh_gate[t] * sh_y[size_t(t) * H + f];  // the shared expert, before the one rounding
-        if (partial_out) partial_out[size_t(t) * H + f] = sum;
-        else out[size_t(t) * H + f] = f32_to_bf16_rn(sum);
-      }
-      if (lane == 0) tile_cnt[rt] = 0u;  // ready for the next call
     }
   }
 }
@@ -484,7 +452,7 @@ size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows) {
 
 size_t down_smem(int fmt, int K, int E, int R, int act_rows) {
   const UnitLayout L = unit_layout(fmt, K, kDnRows);
-  return size_t(kStages) * L.stage_bytes + size_t(act_rows) * staged_row_stride(K) + size_t(2 * (E + 1) + 2 * R) * 4 +
+  return size_t(kStages) * L.stage_bytes + size_t(act_rows) * staged_row_stride(K) + size_t(2 * (E + 1) + R) * 4 +
          8 + (2 * kStages + 1) * 8;
 }
 
@@ -569,7 +537,7 @@ cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Ba
 
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
-                    uint16_t* out, float* partial_out, const float* sh_gate, const float* sh_y, cudaStream_t stream) {
+                    cudaStream_t stream) {
   const int R = T * s.top_k;
   const bool act_smem = size_t(R) * staged_row_stride(s.inter) <= kMaxStagedAct;
   auto k = act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
@@ -580,25 +548,22 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRan
   const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.hidden / kDnRows);
   const int grid = persistent_grid(k, smem, std::max(units, 1), kThreads);
   return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
-                    (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const uint16_t*)ws.act,
-                    (const float*)ws.topk_w, (const int32_t*)ws.pos, ws.ypart, out, partial_out, sh_gate, sh_y,
-                    ws.status);
+                    (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
+                    (const uint16_t*)ws.act, (const float*)ws.topk_w, ws.ypart, ws.status);
 }
 
 template <int FMT>
 cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
-                     uint16_t* out, float* partial_out, const float* sh_gate, const float* sh_y,
                      cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
-  return down_nt<FMT, 4>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, stream);
+  return down_nt<FMT, 4>(s, T, dn, er, ws, stream);
 }
 
 }  // namespace
 
 bool decode_supported(const moe_shape_t& s, int T) {
   if (T > kDecodeMaxT) return false;
-  if (s.hidden / 16 > int(kStatusBytes / 4) - kDnCounterBase) return false;  // down tile counters
   const int R = T * s.top_k;
   const int NT = T <= 8 ? 1 : T <= 16 ? 2 : 4;
   const bool x_smem = size_t(T) * staged_row_stride(s.hidden) <= kMaxStagedX;
@@ -620,15 +585,12 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
   return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, er, ws, units, stream);
 }
 
-cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                                       const Workspace& ws, uint16_t* out, float* partial_out, const float* sh_gate,
-                                       const float* sh_y, cudaStream_t stream) {
+cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                               const Workspace& ws, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128)
-    return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16)
-    return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, out, partial_out, sh_gate, sh_y, stream);
+  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, stream);
 }
 
 }  // namespace moe

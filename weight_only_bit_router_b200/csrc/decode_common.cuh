@@ -133,9 +133,11 @@ MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i, int j) {
   return bf16x2_mul(v, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? rc.m1 : rc.m0);
 }
 
-// acc[4] += W(rows r, r+8; one 128-k block) x activation fragments.
+// acc[h][4] += W(rows r, r+8; one 128-k block) x activation fragments: the
+// MMA steps of a block alternate between two accumulators (h = 0 / 1), so two
+// independent dependency chains are in flight instead of one.
 template <int FMT, bool FAST>
-MOE_DEV void mma_block_path(float (&acc)[4], const RowChunk& lo, const RowChunk& hi, const uint32_t (&b)[8][2]) {
+MOE_DEV void mma_block2(float (&acc)[2][4], const RowChunk& lo, const RowChunk& hi, const uint32_t (&b)[8][2]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t wl = word_of(lo.codes, j), wh = word_of(hi.codes, j);
@@ -146,7 +148,7 @@ MOE_DEV void mma_block_path(float (&acc)[4], const RowChunk& lo, const RowChunk&
       a[1] = dq<FMT, FAST>(hi, wh, 2 * h, j);
       a[2] = dq<FMT, FAST>(lo, wl, 2 * h + 1, j);
       a[3] = dq<FMT, FAST>(hi, wh, 2 * h + 1, j);
-      mma_bf16_16816(acc, a, b[2 * j + h][0], b[2 * j + h][1]);
+      mma_bf16_16816(acc[h], a, b[2 * j + h][0], b[2 * j + h][1]);
     }
   }
 }
@@ -182,6 +184,70 @@ MOE_DEV void act_frags(const uint16_t* p, bool valid, uint32_t (&b)[8][2]) {
     for (int i = 0; i < 16; ++i) X[i] = 0;
   }
   act_frags_from_raw(X, b);
+}
+
+// One warp's pass over the 128-k blocks b0, b0 + step, ... below nblk_full of
+// one 16-row weight tile (rows r and r + 8 of the lane: codes c_lo / c_hi and
+// scales sc_lo / sc_hi in shared memory), then the optional block `tail`
+// (>= 0) whose lane slices may lie past K.  The next block's weights and first
+// token tile's activations are loaded before the current block's math (two
+// register buffers, no copies).  `act.load(j, b, in, bf)` gives token tile j's
+// fragments of block b.  acc[j][h] are the two accumulator chains of tile j.
+template <int FMT, int NT, typename Act>
+MOE_DEV void stream_kblocks(float (&acc)[NT][2][4], int b0, int step, int nblk_full, int tail, int K, int q,
+                            const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo, const uint8_t* sc_hi,
+                            float gsc, int ntiles, const Act& act) {
+  auto compute = [&](const RowChunk& lo, const RowChunk& hi, const uint32_t (&f0)[8][2], int b, bool in) {
+    // warp-uniform: mma.sync needs the whole warp on one path (the two-step
+    // path is exact for every scale)
+    const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
+    if (fast) mma_block2<FMT, true>(acc[0], lo, hi, f0);
+    else mma_block2<FMT, false>(acc[0], lo, hi, f0);
+#pragma unroll
+    for (int j = 1; j < NT; ++j) {
+      if (j >= ntiles) break;
+      uint32_t fj[8][2];
+      act.load(j, b, in, fj);
+      if (fast) mma_block2<FMT, true>(acc[j], lo, hi, fj);
+      else mma_block2<FMT, false>(acc[j], lo, hi, fj);
+    }
+  };
+  int b = b0;
+  if (b < nblk_full) {
+    RowChunk a_lo = row_chunk_at<FMT>(c_lo, sc_lo, b, q, true, gsc);
+    RowChunk a_hi = row_chunk_at<FMT>(c_hi, sc_hi, b, q, true, gsc);
+    uint32_t fa[8][2];
+    act.load(0, b, true, fa);
+    for (;;) {
+      const int b1 = b + step;
+      RowChunk b_lo, b_hi;
+      uint32_t fb[8][2];
+      if (b1 < nblk_full) {
+        b_lo = row_chunk_at<FMT>(c_lo, sc_lo, b1, q, true, gsc);
+        b_hi = row_chunk_at<FMT>(c_hi, sc_hi, b1, q, true, gsc);
+        act.load(0, b1, true, fb);
+      }
+      compute(a_lo, a_hi, fa, b, true);
+      if (b1 >= nblk_full) break;
+      const int b2 = b1 + step;
+      if (b2 < nblk_full) {
+        a_lo = row_chunk_at<FMT>(c_lo, sc_lo, b2, q, true, gsc);
+        a_hi = row_chunk_at<FMT>(c_hi, sc_hi, b2, q, true, gsc);
+        act.load(0, b2, true, fa);
+      }
+      compute(b_lo, b_hi, fb, b1, true);
+      if (b2 >= nblk_full) break;
+      b = b2;
+    }
+  }
+  if (tail >= 0) {
+    const bool in = 128 * tail + 32 * q < K;
+    const RowChunk lo = row_chunk_at<FMT>(c_lo, sc_lo, tail, q, in, gsc);
+    const RowChunk hi = row_chunk_at<FMT>(c_hi, sc_hi, tail, q, in, gsc);
+    uint32_t f0[8][2];
+    act.load(0, tail, in, f0);
+    compute(lo, hi, f0, tail, in);
+  }
 }
 
 // Number of 128-k blocks in which lane slice q (k in [kb + 32q, kb + 32q + 32))

@@ -52,8 +52,7 @@ struct Bank {
 
 // Workspace carve-up for T tokens (all offsets 256-byte aligned).
 // The first kStatusBytes of a workspace: the status word and the kernels'
-// device counters (small-batch routing completion at int32 index 1, the decode
-// down kernel's feature-tile counters from index 16).  Zeroed once by moe_workspace_init; every kernel
+// device counters (small-batch routing completion at int32 index 1).  Zeroed once by moe_workspace_init; every kernel
 // that counts leaves its counters at zero when it finishes.
 constexpr size_t kStatusBytes = 4096;
 
@@ -116,13 +115,10 @@ bool decode_supported(const moe_shape_t& s, int T);
 size_t decode_ypart_bytes(const moe_shape_t& s, int T);
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
-// sh_gate [T] / sh_y [T, H] (both null, or both given): the shared expert's
-// gate and output, added as sh_gate[t] * sh_y[t][f] before the bf16 rounding.
-// partial_out (nullable): the fp32 sum over the bank's experts instead of the
-// bf16 output (every element written when the bank has routed rows).
-cudaError_t launch_decode_down_combine(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                                       const Workspace& ws, uint16_t* out, float* partial_out, const float* sh_gate,
-                                       const float* sh_y, cudaStream_t stream);
+// the routing-weighted down outputs of the bank's experts' sorted rows into
+// ws.ypart [T*k, H] fp32 (combine_rows sums them)
+cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
+                               const Workspace& ws, cudaStream_t stream);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
