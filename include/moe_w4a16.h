@@ -255,8 +255,9 @@ typedef enum {
 #define MOE_NUM_STAGES 5
 /* Stage ids: 0 router logits, 1 top-k + permutation, 2 gate_up + SwiGLU,
  * 3 down projection, 4 weighted combine / output conversion.  Where one
- * kernel does two stages (small batches: routing and permutation in one) the
- * second stage's events bracket nothing and it reads zero. */
+ * kernel does two stages (small batches: routing and permutation in one; the
+ * decode path's down projection and combine in one) the second stage's
+ * events bracket nothing and it reads zero. */
 
 /* Optional extras of moe_forward / moe_forward_routed.  Every pointer may be
  * NULL; a NULL opts pointer means all defaults. */
@@ -274,21 +275,21 @@ typedef struct {
                                 captured into a CUDA graph) */
 } moe_forward_opts_t;
 
-/* moe_forward_opts_t.flags: MOE_FLAG_DETERMINISTIC makes the grouped
- * (above 32 tokens) path's combine run-to-run deterministic: every (token,
- * slot) row's weighted expert output is stored in its own fp32 row and each
- * token's k rows are summed in slot order, instead of being added into the
- * output accumulator in arrival order.  It needs the larger workspace of
- * moe_workspace_bytes_flags.  The decode path (up to 32 tokens) is always
- * deterministic. */
+/* moe_forward_opts_t.flags: MOE_FLAG_DETERMINISTIC makes the grouped path's
+ * combine run-to-run deterministic: every (token, slot) row's weighted expert
+ * output is stored in its own fp32 row and each token's k rows are summed in
+ * slot order, instead of being added into the output accumulator in arrival
+ * order.  It needs the larger workspace of moe_workspace_bytes_flags.  The
+ * decode path (up to 32 tokens) is always deterministic: its down kernel sums
+ * each token's k slot outputs in slot order. */
 #define MOE_FLAG_DETERMINISTIC 1u
 
 /* Workspace bytes moe_forward / moe_forward_routed need for T tokens. */
 MOE_API size_t moe_workspace_bytes(const moe_shape_t* shape, int T);
 
 /* Workspace bytes for T tokens with the given MOE_FLAG_* bits (flags = 0:
- * moe_workspace_bytes; MOE_FLAG_DETERMINISTIC above 32 tokens adds T*k*H*4
- * bytes for the per-row outputs). */
+ * moe_workspace_bytes; MOE_FLAG_DETERMINISTIC adds T*k*H*4 bytes for the
+ * grouped path's per-row outputs). */
 MOE_API size_t moe_workspace_bytes_flags(const moe_shape_t* shape, int T, uint32_t flags);
 
 /* Forward pass of the routed-expert layer.

@@ -119,10 +119,9 @@ Workspace carve_workspace(void* base, const moe_shape_t& s, int T, uint32_t flag
   w.block_hist = static_cast<int32_t*>(take(permute_large_hist_bytes(T, int(E), s.top_k)));
   w.act = static_cast<uint16_t*>(take(R * I * 2));
   w.out_acc = static_cast<float*>(take(size_t(T) * H * 4));
-  // per-row down outputs: the decode path's (T <= kDecodeMaxT), or the
-  // deterministic grouped combine's
-  const size_t ypart_bytes = T <= kDecodeMaxT ? decode_ypart_bytes(s, T)
-                             : (flags & MOE_FLAG_DETERMINISTIC) ? R * H * 4 : 0;
+  // per-row down outputs of the deterministic grouped combine (the decode
+  // path combines inside its down kernel)
+  const size_t ypart_bytes = (flags & MOE_FLAG_DETERMINISTIC) ? R * H * 4 : 0;
   w.ypart = static_cast<float*>(take(ypart_bytes));
   w.route_part = static_cast<float*>(take(T <= kDecodeMaxT ? route_part_bytes(T, int(H), int(E), s.top_k) : 0));
   w.bytes = off;
@@ -195,11 +194,10 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   NvtxRange range("moe.down_combine");
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
-    // routing-weighted per-row outputs, then each token's slot rows summed in order
-    MOE_TRY(launch_decode_down(s, T, dn, er, ws, stream));
+    // down products and each token's slots summed in slot order, in one kernel
+    MOE_TRY(launch_decode_down(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
-    MOE_TRY(launch_combine_rows(s, T, er, ws, ws.ypart, sh_gate, sh_y, out, partial_out, stream));
   } else if (opt_flags(o) & MOE_FLAG_DETERMINISTIC) {
     // every (token, slot) row's weighted output in its own row, then the
     // k rows of each token summed in slot order
@@ -615,7 +613,7 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   if (routed) n += perm;
   else if (T <= kDecodeMaxT) n += 1;                          // fused router + top-k + permutation
   else n += 2 + perm;                                         // router GEMM, top-k, permutation
-  n += 3;                                                     // gate_up, down, combine / finalize
+  n += decode ? 2 : 3;  // gate_up, down (+ combine / finalize for the grouped GEMMs)
   return n;
 }
 

@@ -2,15 +2,22 @@
 //
 // The time goes into streaming the touched experts' packed weights from HBM
 // ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", Measured: at concurrency 32
-// the bottleneck is weight bandwidth).  Both kernels are persistent streams of
-// 16 KB-class work units: a unit's packed rows are one or two contiguous
-// ranges of the canonical [E][N][K/2] layout, so one producer lane starts 1-D
-// bulk copies of their codes and scales into a ring of shared-memory stages
-// and every byte of several units is in flight at once.  Groups of four
-// consumer warps dequantise in registers (decode_common.cuh) and feed
-// mma.sync m16n8k16 with up to 32 tokens.  The routing state (touched
-// experts, per-expert row offsets, the rows' tokens) is read into shared
-// memory once per CTA.
+// the bottleneck is weight bandwidth).  Both kernels are persistent: one
+// producer warp per CTA starts 1-D bulk copies of 16-row weight tiles (one
+// copy per row, at a padded shared-memory stride, plus their scales) into a
+// ring of stages and keeps the next tiles' bytes in flight (and the tile after
+// the ring into L2); consumer warps dequantise in registers
+// (decode_common.cuh) and feed mma.sync m16n8k16 with up to 32 tokens.  The
+// routing state (touched experts, per-expert row offsets, the rows' tokens) is
+// read into shared memory once per CTA, and small token / activation sets are
+// staged there once in MMA fragment order.
+//
+// gate_up: CTA c takes a contiguous run of the (touched expert, 8-feature)
+// units; four warps split each unit's k-blocks and sum in shared memory.
+// down: CTA c owns 16 output features of every token and runs over all
+// touched experts, so the routing-weighted combine of a token's k expert
+// outputs happens in the CTA (in slot order, deterministic) and the output is
+// written once.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -24,28 +31,30 @@ namespace moe {
 
 namespace {
 
-constexpr int kGroupWarps = 4;  // consumer warps per work unit
+constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
 
-// Number of consumer groups (units in flight through compute) per CTA,
-// shared-memory stages per CTA, and CTAs per SM the register budget is sized
-// for (build-time tuning knobs; the defaults are the measured best).
+// Build-time tuning knobs (the defaults are the measured best): gate_up
+// consumer groups per CTA and its largest stage ring; down consumer warps per
+// CTA and its largest stage ring.
 #ifndef MOE_DEC_GROUPS
 #define MOE_DEC_GROUPS 2
 #endif
 #ifndef MOE_DEC_STAGES
-#define MOE_DEC_STAGES 4
+#define MOE_DEC_STAGES 8
 #endif
-#ifndef MOE_DEC_MIN_CTAS
-#define MOE_DEC_MIN_CTAS 2
+#ifndef MOE_DEC_DN_WARPS
+#define MOE_DEC_DN_WARPS 8
 #endif
-// registers per thread that keep MOE_DEC_MIN_CTAS CTAs per SM (65536 per SM,
-// allocated in multiples of 8 per thread); one CTA per SM above 8 tokens
-constexpr int kDecRegs = (65536 / (MOE_DEC_MIN_CTAS * (MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8;
-constexpr int kDecRegsWide = (65536 / ((MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8 > 255
-                                 ? 248 : (65536 / ((MOE_DEC_GROUPS * 4 + 1) * 32)) / 8 * 8;
-constexpr int kGroups = MOE_DEC_GROUPS;
-constexpr int kStages = MOE_DEC_STAGES;
-constexpr int kThreads = (kGroups * kGroupWarps + 1) * 32;
+#ifndef MOE_DEC_DN_STAGES
+#define MOE_DEC_DN_STAGES 32
+#endif
+constexpr int kGuGroups = MOE_DEC_GROUPS;
+constexpr int kGuMaxStages = MOE_DEC_STAGES;
+constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
+constexpr int kDnWarps = MOE_DEC_DN_WARPS;
+constexpr int kDnMaxStages = MOE_DEC_DN_STAGES;
+constexpr int kDnThreads = (kDnWarps + 1) * 32;
+constexpr int kDnRows = 16;  // output features per down tile
 
 // The routing state every CTA keeps in shared memory: the touched-expert list
 // [n, e_0, e_1, ...] and the per-expert row offsets (E + 1 entries each).
@@ -82,32 +91,37 @@ MOE_DEV void local_slice(const int* s_touched, int e_lo, int e_hi, int E, int* s
   *t_hi = s_cnt[0] + s_cnt[1];
 }
 
+template <typename T>
+MOE_DEV T* align8(void* p) {
+  return reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(p) + 7) & ~uintptr_t(7));
+}
+
 // Activation fragments of the gate_up kernel: token rows of x (staged in
-// shared memory, or read through L1) for the token tiles of one unit.
+// fragment order, or read through L1) for the token tiles of one unit.
 template <int NT, bool X_SMEM>
 struct XFrags {
   const uint16_t* x;      // global x [T, K]
   const uint8_t* x_s;     // staged rows (X_SMEM)
-  int xstride, K, q;
+  int pstride, K, q;
   int tok[NT];            // token of column 8j + g
   MOE_DEV void load(int j, int b, bool in, uint32_t (&bf)[8][2]) const {
-    if (X_SMEM) act_frags<0>(reinterpret_cast<const uint16_t*>(x_s + tok[j] * xstride) + 128 * b + 32 * q, in, bf);
-    else act_frags<1>(x + size_t(tok[j]) * K + 128 * b + 32 * q, in, bf);
+    if (X_SMEM) act_frags_staged(x_s + tok[j] * pstride + 256 * b, q, in, bf);
+    else act_frags_global<1>(x + size_t(tok[j]) * K + 128 * b + 32 * q, in, bf);
   }
 };
 
 // Activation fragments of the down kernel: the expert's bf16 SwiGLU rows p
-// (staged in shared memory, or read through L2: another kernel wrote them).
+// (staged in fragment order, or read through L2: another kernel wrote them).
 template <bool ACT_SMEM>
 struct ActFrags {
   const uint16_t* act;    // global act [T*k, K]
   const uint8_t* act_s;   // staged rows (ACT_SMEM)
-  int astride, K, q, g, p0, n_e;
+  int pstride, K, q, g, p0, n_e;
   MOE_DEV void load(int j, int b, bool in, uint32_t (&bf)[8][2]) const {
     const int c = 8 * j + g;
     const int p = p0 + (c < n_e ? c : 0);
-    if (ACT_SMEM) act_frags<0>(reinterpret_cast<const uint16_t*>(act_s + p * astride) + 128 * b + 32 * q, in, bf);
-    else act_frags<2>(act + size_t(p) * K + 128 * b + 32 * q, in, bf);
+    if (ACT_SMEM) act_frags_staged(act_s + size_t(p) * pstride + 256 * b, q, in, bf);
+    else act_frags_global<2>(act + size_t(p) * K + 128 * b + 32 * q, in, bf);
   }
 };
 
@@ -117,39 +131,61 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
   for (int i = max(0, issued - S); i < issued; ++i) mbar_wait_drain(&full[i % S], (i / S) & 1, kWaitLimitNs);
 }
 
+// Start the copies of one 16-row weight tile into `stage` (codes at the padded
+// row stride, then scales): lanes 0-15 one code row each (source rows
+// row_a + l for l < 8, row_b + l - 8 after), lanes 16 / 17 the scales of the
+// two 8-row runs (16 contiguous rows when row_b = row_a + 8: lane 16 alone).
+// Called by the whole producer warp after lane 0 announced the bytes.
+template <int FMT>
+MOE_DEV void stage_tile(const Bank& bk, long row_a, long row_b, uint8_t* stage, const StageLayout& L, uint64_t* bar,
+                        uint64_t policy, int lane) {
+  const int K = bk.K;
+  const int srow = scale_row_bytes(FMT, K);
+  const uint8_t* scales = static_cast<const uint8_t*>(bk.scales);
+  if (lane < 16) {
+    const long r = lane < 8 ? row_a + lane : row_b + lane - 8;
+    bulk_g2s_hint(stage + lane * L.crow, bk.codes + r * (K / 2), uint32_t(K / 2), bar, policy);
+  } else if (lane == 16) {
+    const int n = row_b == row_a + 8 ? 16 : 8;
+    bulk_g2s_hint(stage + L.cbytes, scales + row_a * srow, uint32_t(n * srow), bar, policy);
+  } else if (lane == 17 && row_b != row_a + 8) {
+    bulk_g2s_hint(stage + L.cbytes + 8 * srow, scales + row_b * srow, uint32_t(8 * srow), bar, policy);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // gate_up + SwiGLU.  Work unit u = (touched slot u / (I/8), features
 // f0 = 8 (u % (I/8)) .. f0 + 7): its 16 weight rows are the 8 gate rows f0..
 // and the 8 matching up rows I + f0.., staged as one 16-row tile (gate rows
 // 0-7, up rows 8-15), so the MMA's C fragment holds gate (c0, c1) and up
-// (c2, c3) of the same feature and token: SwiGLU needs no shuffle.  The CTA's
-// i-th unit goes to stage i % S and consumer group i % G; the group's four
-// warps split K (128-k blocks w, w + 4, ...), and one of them (rotating) sums
-// the four partial tiles in warp order and writes a = bf16(silu(gate) * up) to
-// act[p][f] for the expert's sorted rows p.
-// With X_SMEM (small T) the producer warp first stages the T token rows in
-// shared memory (one bulk copy per row, padded row stride).
+// (c2, c3) of the same feature and token: SwiGLU needs no shuffle.  CTA c
+// takes units [c n / grid, (c + 1) n / grid); its i-th goes to stage i % S and
+// consumer group i % G.  The group's four warps split K (128-k blocks w,
+// w + 4, ...), and one of them (rotating) sums the four partial tiles in warp
+// order and writes a = bf16(silu(gate) * up) to act[p][f] for the expert's
+// sorted rows p.  With X_SMEM (small T) the consumers first stage the T token
+// rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
-    uint16_t* __restrict__ act, uint32_t* status) {
+    uint16_t* __restrict__ act, uint32_t* status, int S) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int G = kGroups, S = kStages;
+  constexpr int G = kGuGroups;
+  constexpr int CH = NT == 1 ? 4 : 2;  // accumulator chains per token tile
   const int K = gu.K, R = T * top_k;
-  const UnitLayout L = unit_layout(FMT, K, 16);
+  const StageLayout L = stage_layout(FMT, K, 16);
   const int srow = scale_row_bytes(FMT, K);
-  const int xstride = staged_row_stride(K);
-  uint8_t* ring = smem;                                                  // [S][stage]
-  uint8_t* x_s = ring + S * L.stage_bytes;                               // [T][xstride] (X_SMEM)
-  float* red = reinterpret_cast<float*>(x_s + (X_SMEM ? T * xstride : 0));  // [G][2][4][NT][4][32]
+  const int pstride = staged_act_stride(K);
+  uint8_t* ring = smem;                                                      // [S][stage]
+  uint8_t* x_s = ring + size_t(S) * L.stage_bytes;                           // [T][pstride] (X_SMEM)
+  float* red = reinterpret_cast<float*>(x_s + (X_SMEM ? size_t(T) * pstride : 0));  // [G][2][4][NT][4][32]
   int* s_touched = reinterpret_cast<int*>(red + G * 2 * kGroupWarps * NT * 128);
   int* s_off = s_touched + (E + 1);
-  int* s_tok = s_off + (E + 1);                                          // [R] token of sorted row p
-  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_tok + R) + 7) & ~uintptr_t(7));
+  int* s_tok = s_off + (E + 1);                                              // [R] token of sorted row p
+  uint64_t* full = align8<uint64_t>(s_tok + R);
   uint64_t* empty = full + S;
-  uint64_t* x_bar = empty + S;
   __shared__ volatile int s_abort;  // raised by the first wait that gives up
   __shared__ int s_cnt[2];
 
@@ -160,7 +196,6 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
       mbar_init(&full[st], 1);
       mbar_init(&empty[st], kGroupWarps);
     }
-    mbar_init(x_bar, 1);
     fence_mbar_init();
   }
   pdl_wait();
@@ -173,61 +208,60 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
   const int ftiles = I / 8;
   const int n_units = (t_hi - t_lo) * ftiles;
-  if (int(blockIdx.x) >= n_units) return;
+  const int u_begin = int(long(n_units) * blockIdx.x / gridDim.x);
+  const int cnt = int(long(n_units) * (blockIdx.x + 1) / gridDim.x) - u_begin;
+  if (cnt <= 0) return;
 
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
-    if (X_SMEM) {
-      if (lane == 0) mbar_arrive_expect_tx(x_bar, uint32_t(T) * uint32_t(2 * K));
+    const uint64_t policy = l2_policy_evict_first();
+    const uint32_t tx = staged_bytes<FMT>(gu, 16);
+    int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;          // unit i
+    int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
+    int i = 0, st = 0, ph = 0;  // unit i's stage and that stage's use count parity
+    for (; i < cnt; ++i) {
+      if (i >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &s_abort, status))) break;
+      const long row_g = long(s_local[slot] - e_lo) * gu.N + ft * 8;
+      fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], tx);
       __syncwarp();
-      stage_bf16_rows(x_s, x, T, K, x_bar);
-    }
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      int i = 0;
-      for (;; ++i) {
-        const int u = blockIdx.x + i * gridDim.x;
-        if (u >= n_units) break;
-        const int st = i % S;
-        if (i >= S && !mbar_wait(&empty[st], ((i / S) - 1) & 1, &s_abort, status)) break;
-        const int e = s_local[u / ftiles];
-        const long row_g = long(e - e_lo) * gu.N + (u % ftiles) * 8;
-        uint8_t* stage = ring + st * L.stage_bytes;
-        fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
-        mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(gu, 16));
-        stage_rows<FMT>(gu, row_g, 8, stage, stage + L.cbytes, &full[st], policy);
-        stage_rows<FMT>(gu, row_g + I, 8, stage + 8 * (K / 2), stage + L.cbytes + 8 * srow, &full[st], policy);
+      stage_tile<FMT>(gu, row_g, row_g + I, ring + size_t(st) * L.stage_bytes, L, &full[st], policy, lane);
+      if (lane >= 18 && lane < 22 && i + S < cnt) {
         // the unit that will refill this stage, into L2 ahead of time
-        const int un = u + S * gridDim.x;
-        if (un < n_units) {
-          const long rn = long(s_local[un / ftiles] - e_lo) * gu.N + (un % ftiles) * 8;
-          prefetch_rows<FMT>(gu, rn, 8);
-          prefetch_rows<FMT>(gu, rn + I, 8);
-        }
+        const long rn = long(s_local[pslot] - e_lo) * gu.N + pft * 8 + ((lane & 1) ? I : 0);
+        if (lane < 20) prefetch_codes<FMT>(gu, rn, 8);
+        else prefetch_scales<FMT>(gu, rn, 8);
       }
-      drain_stages(full, i, S);
+      if (++st == S) st = 0, ph ^= 1;
+      if (++ft == ftiles) ft = 0, ++slot;
+      if (++pft == ftiles) pft = 0, ++pslot;
     }
+    if (lane == 0) drain_stages(full, i, S);
     return;
   }
 
   // -------------------------------------------------------------------- consumers
+  constexpr int kConsumers = G * kGroupWarps * 32;
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
-  const int nblk_full = K / 128;              // blocks where every lane slice lies inside K
-  const bool tail = (K % 128) != 0;           // a last block with slices past K
-  const bool x_ok = !X_SMEM || mbar_wait(x_bar, 0, &s_abort, status);
-  for (int i = grp, n = 0;; i += G, ++n) {
-    const int u = blockIdx.x + i * gridDim.x;
-    if (u >= n_units) break;
-    const int st = i % S;
+  if (X_SMEM) {
+    stage_act_rows<1>(x_s, x, T, K, threadIdx.x, kConsumers);
+    named_barrier_sync(1, kConsumers);
+  }
+  const int nfull = K / 128;  // blocks where every lane slice lies inside K
+  const int my_full = wj < nfull ? (nfull - wj + kGroupWarps - 1) / kGroupWarps : 0;
+  const int tail_b = ((K % 128) != 0 && nfull % kGroupWarps == wj) ? nfull : -1;
+  int slot = (u_begin + grp) / ftiles, ft = (u_begin + grp) - slot * ftiles;
+  int st = grp, ph = 0;
+  for (int i = grp, n = 0; i < cnt; i += G, ++n) {
     // warp-uniform: the MMAs below run only if every lane saw the data land
-    const bool ok = __all_sync(0xffffffffu, x_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status));
-    const int e = s_local[u / ftiles];
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, &s_abort, status));
+    const int e = s_local[slot];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-    const int f0 = (u % ftiles) * 8;
-    const uint8_t* s_c = ring + st * L.stage_bytes;
-    const uint8_t* c_gate = s_c + g * (K / 2) + 16 * q;   // rows g (gate) and g + 8 (up), lane slice
-    const uint8_t* c_up = c_gate + 8 * (K / 2);
+    const int f0 = ft * 8;
+    const uint8_t* s_c = ring + size_t(st) * L.stage_bytes;
+    const uint8_t* c_gate = s_c + g * L.crow + 16 * q;   // rows g (gate) and g + 8 (up), lane slice
+    const uint8_t* c_up = c_gate + 8 * L.crow;
     const uint8_t* sc_gate = s_c + L.cbytes + g * srow;
     const uint8_t* sc_up = sc_gate + 8 * srow;
     const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[e - e_lo] : 0.f;
@@ -235,7 +269,7 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
     XFrags<NT, X_SMEM> xf;
     xf.x = x;
     xf.x_s = x_s;
-    xf.xstride = xstride;
+    xf.pstride = pstride;
     xf.K = K;
     xf.q = q;
     // token of column 8j + g (a valid token's row for the padding columns)
@@ -244,19 +278,15 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
       const int c = 8 * j + g;
       xf.tok[j] = s_tok[p0 + (c < n_e ? c : 0)];
     }
-    float acc2[NT][2][4];
+    float acc2[NT][CH][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc2[j][0][c] = acc2[j][1][c] = 0.f;
-    if (ok)
-      stream_kblocks<FMT, NT>(acc2, wj, kGroupWarps, nblk_full, (tail && nblk_full % kGroupWarps == wj) ? nblk_full : -1,
-                              K, q, c_gate, c_up, sc_gate, sc_up, gsc, ntiles, xf);
-    float acc[NT][4];
+      for (int h = 0; h < CH; ++h)
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[j][c] = acc2[j][0][c] + acc2[j][1][c];
+        for (int c = 0; c < 4; ++c) acc2[j][h][c] = 0.f;
+    if (ok) warp_tile<FMT, NT, CH>(acc2, c_gate, c_up, sc_gate, sc_up, wj, kGroupWarps, my_full, tail_b, K, q, gsc,
+                                   ntiles, xf);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
     // the group's partial tiles, double-buffered by unit parity
@@ -264,8 +294,13 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) red_u[((wj * NT + j) * 4 + c) * 32 + lane] = acc[j][c];
-    named_barrier_sync(1 + grp, kGroupWarps * 32);
+      for (int c = 0; c < 4; ++c) {
+        float v = acc2[j][0][c];
+#pragma unroll
+        for (int h = 1; h < CH; ++h) v += acc2[j][h][c];
+        red_u[((wj * NT + j) * 4 + c) * 32 + lane] = v;
+      }
+    named_barrier_sync(2 + grp, kGroupWarps * 32);
     if (ok && wj == n % kGroupWarps) {
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -285,44 +320,52 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_gate_up_ke
         }
       }
     }
+    st += G;
+    if (st >= S) st -= S, ph ^= 1;
+    ft += G;
+    while (ft >= ftiles) ft -= ftiles, ++slot;
   }
 }
 
 // ---------------------------------------------------------------------------
-// down projection.  Work unit u = (feature tile ft = u / n of 64 output
-// features, touched slot u % n): the expert's 64 down rows (all of K = I).
-// Consumer warp w of the unit's group takes rows 16 w .. 16 w + 15 over every
-// k-block and writes w_tj * (Wd a) for each of the expert's sorted rows p
-// (fp32, scaled by the row's routing weight) to ypart[p][f].  The combine
-// kernel that follows sums each token's k rows in slot order (deterministic).
-// The weights do not depend on the gate_up kernel that runs just before: the
-// producer reads the routing state (written two launches back, and the kernel
-// in between triggers its dependents only after its own wait) and starts the
-// weight copies before the programmatic-launch wait; only the consumers wait.
-// With ACT_SMEM (small T) one consumer warp stages the T*k activation rows.
+// down projection and combine.  CTA c owns the 16 output features of tiles
+// c, c + grid, ... (H / 16 tiles).  For a tile, work unit s = the tile's 16
+// rows of the down matrix of touched expert s (all of K = I), taken by
+// consumer warp s % W; its C fragment times the routing weight of each
+// column's (token, slot) goes to ybuf[t k + j][f] in shared memory.  When the
+// tile's units are done, each token's output is the sum of its k slots in
+// slot order (plus the shared expert's gated output), rounded once to bf16,
+// or the fp32 sum (an expert-parallel shard's partial: slots of other shards'
+// experts stay zero).  The weights do not depend on the gate_up kernel that
+// runs just before: the producer reads the routing state (written two
+// launches back, and the kernel in between triggers its dependents only after
+// its own wait) and starts the weight copies before the programmatic-launch
+// wait; only the consumers wait.  With ACT_SMEM (small T) the consumers first
+// stage the T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
-constexpr int kDnRows = 64;  // output features per unit
-
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_down_kernel(
+__global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
-    const float* __restrict__ topk_w, float* __restrict__ ypart, uint32_t* status) {
+    const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
+    uint16_t* __restrict__ out, float* __restrict__ partial_out, uint32_t* status, int S) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int G = kGroups, S = kStages;
+  constexpr int W = kDnWarps;
+  constexpr int CH = NT == 1 ? 4 : 2;
   const int H = dn.N, K = dn.K;  // K = I
   const int R = T * top_k;
-  const UnitLayout L = unit_layout(FMT, K, kDnRows);
+  const StageLayout L = stage_layout(FMT, K, kDnRows);
   const int srow = scale_row_bytes(FMT, K);
-  const int astride = staged_row_stride(K);
-  uint8_t* ring = smem;                                  // [S][stage]
-  uint8_t* act_s = ring + S * L.stage_bytes;             // [R][astride] (ACT_SMEM)
-  int* s_touched = reinterpret_cast<int*>(act_s + (ACT_SMEM ? R * astride : 0));
+  const int pstride = staged_act_stride(K);
+  uint8_t* ring = smem;                                           // [S][stage]
+  uint8_t* act_s = ring + size_t(S) * L.stage_bytes;              // [R][pstride] (ACT_SMEM)
+  float* ybuf = reinterpret_cast<float*>(act_s + (ACT_SMEM ? size_t(R) * pstride : 0));  // [R][16]
+  int* s_touched = reinterpret_cast<int*>(ybuf + R * kDnRows);
   int* s_off = s_touched + (E + 1);
-  float* s_wrow = reinterpret_cast<float*>(s_off + (E + 1));  // [R] routing weight of sorted row p
-  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_wrow + R) + 7) & ~uintptr_t(7));
+  int* s_slot = s_off + (E + 1);                                  // [R] slot t k + j of sorted row p
+  float* s_w = reinterpret_cast<float*>(s_slot + R);              // [R] its routing weight
+  uint64_t* full = align8<uint64_t>(s_w + R);
   uint64_t* empty = full + S;
-  uint64_t* act_bar = empty + S;
   __shared__ volatile int s_abort;
   __shared__ int s_cnt[2];
 
@@ -331,48 +374,57 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_down_kerne
     s_abort = 0;
     for (int st = 0; st < S; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], kGroupWarps);
+      mbar_init(&empty[st], 1);
     }
-    mbar_init(act_bar, 1);
     fence_mbar_init();
   }
   // routing state: written two launches back (see above), read through L2
   load_routing(s_touched, s_off, touched, offsets, E);
-  for (int p = threadIdx.x; p < R; p += blockDim.x) s_wrow[p] = __ldcg(topk_w + __ldcg(sorted_rows + p));
+  for (int p = threadIdx.x; p < R; p += blockDim.x) {
+    const int r = __ldcg(sorted_rows + p);
+    s_slot[p] = r;
+    s_w[p] = __ldcg(topk_w + r);
+  }
+  for (int i = threadIdx.x; i < R * kDnRows; i += blockDim.x) ybuf[i] = 0.f;
   __syncthreads();
   int t_lo, t_hi;
   local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
   const int n_t = t_hi - t_lo;
-  const int ftiles = H / kDnRows;
-  const int n_units = n_t * ftiles;
-  if (int(blockIdx.x) >= n_units) {
-    pdl_wait();
-    pdl_trigger();
-    return;
-  }
+  const int ntile = H / kDnRows;
 
-  if (warp == G * kGroupWarps) {
+  if (warp == W) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+    if (n_t > 0) {
       const uint64_t policy = l2_policy_evict_first();
-      int i = 0;
-      for (;; ++i) {
-        const int u = blockIdx.x + i * gridDim.x;
-        if (u >= n_units) break;
-        const int st = i % S;
-        if (i >= S && !mbar_wait(&empty[st], ((i / S) - 1) & 1, &s_abort, status)) break;
-        const int e = s_local[u % n_t];
-        const long row0 = long(e - e_lo) * H + (u / n_t) * kDnRows;
-        uint8_t* stage = ring + st * L.stage_bytes;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&full[st], staged_bytes<FMT>(dn, kDnRows));
-        stage_rows<FMT>(dn, row0, kDnRows, stage, stage + L.cbytes, &full[st], policy);
-        // the unit that will refill this stage, into L2 ahead of time
-        const int un = u + S * gridDim.x;
-        if (un < n_units) prefetch_rows<FMT>(dn, long(s_local[un % n_t] - e_lo) * H + (un / n_t) * kDnRows, kDnRows);
+      const uint32_t tx = staged_bytes<FMT>(dn, kDnRows);
+      int ptile = blockIdx.x, ps = 0;  // unit i + S
+      for (int a = 0; a < S; ++a)
+        if (++ps == n_t) ps = 0, ptile += gridDim.x;
+      int i = 0, st = 0, ph = 0;
+      bool run = true;
+      for (int tile = blockIdx.x; run && tile < ntile; tile += gridDim.x) {
+        for (int s = 0; s < n_t; ++s, ++i) {
+          if (i >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &s_abort, status))) {
+            run = false;
+            break;
+          }
+          const long row0 = long(s_local[s] - e_lo) * H + tile * kDnRows;
+          fence_proxy_async_smem();
+          if (lane == 0) mbar_arrive_expect_tx(&full[st], tx);
+          __syncwarp();
+          stage_tile<FMT>(dn, row0, row0 + 8, ring + size_t(st) * L.stage_bytes, L, &full[st], policy, lane);
+          if (lane >= 18 && lane < 20 && ptile < ntile) {
+            // the unit that will refill this stage, into L2 ahead of time
+            const long rn = long(s_local[ps] - e_lo) * H + ptile * kDnRows;
+            if (lane == 18) prefetch_codes<FMT>(dn, rn, kDnRows);
+            else prefetch_scales<FMT>(dn, rn, kDnRows);
+          }
+          if (++st == S) st = 0, ph ^= 1;
+          if (++ps == n_t) ps = 0, ptile += gridDim.x;
+        }
       }
-      drain_stages(full, i, S);
+      if (lane == 0) drain_stages(full, i, S);
     }
     pdl_wait();
     pdl_trigger();
@@ -380,86 +432,165 @@ __global__ void __maxnreg__(NT >= 2 ? kDecRegsWide : kDecRegs) decode_down_kerne
   }
 
   // -------------------------------------------------------------------- consumers
-  pdl_wait();  // the activations (and the previous readers of ypart) of the kernels before
+  constexpr int kConsumers = W * 32;
+  pdl_wait();  // the activations (and the previous readers of the output) of the kernels before
   pdl_trigger();
-  const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
-  const int nblk_full = K / 128;
-  const int tail = (K % 128) != 0 ? nblk_full : -1;
-  if (ACT_SMEM && warp == 0) {
-    if (lane == 0) mbar_arrive_expect_tx(act_bar, uint32_t(R) * uint32_t(2 * K));
-    __syncwarp();
-    stage_bf16_rows(act_s, act, R, K, act_bar);
-  }
-  const bool act_ok = !ACT_SMEM || mbar_wait(act_bar, 0, &s_abort, status);
-  for (int i = grp;; i += G) {
-    const int u = blockIdx.x + i * gridDim.x;
-    if (u >= n_units) break;
-    const int st = i % S;
-    // warp-uniform: the MMAs below run only if every lane saw the data land
-    const bool ok = __all_sync(0xffffffffu, act_ok && mbar_wait(&full[st], (i / S) & 1, &s_abort, status));
-    const int e = s_local[u % n_t];
-    const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-    const int f0 = (u / n_t) * kDnRows + 16 * wj;  // this warp's 16 output features
-    const uint8_t* s_c = ring + st * L.stage_bytes;
-    const uint8_t* c_lo = s_c + (16 * wj + g) * (K / 2) + 16 * q;
-    const uint8_t* c_hi = c_lo + 8 * (K / 2);
-    const uint8_t* sc_lo = s_c + L.cbytes + (16 * wj + g) * srow;
-    const uint8_t* sc_hi = sc_lo + 8 * srow;
-    const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
-    const int ntiles = min(NT, (n_e + 7) / 8);
-    ActFrags<ACT_SMEM> af;
-    af.act = act;
-    af.act_s = act_s;
-    af.astride = astride;
-    af.K = K;
-    af.q = q;
-    af.g = g;
-    af.p0 = p0;
-    af.n_e = n_e;
-    float acc2[NT][2][4];
+  if (ACT_SMEM) stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kConsumers);
+  named_barrier_sync(1, kConsumers);
+  const int nfull = K / 128;
+  const int tail_b = (K % 128) != 0 ? nfull : -1;
+  int ti = 0;
+  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x, ++ti) {
+    for (int s = warp; s < n_t; s += W) {
+      const int idx = ti * n_t + s;  // the CTA's unit index
+      const int st = idx % S;
+      // warp-uniform: the MMAs below run only if every lane saw the data land
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (idx / S) & 1, &s_abort, status));
+      const int e = s_local[s];
+      const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
+      const uint8_t* s_c = ring + size_t(st) * L.stage_bytes;
+      const uint8_t* c_lo = s_c + g * L.crow + 16 * q;
+      const uint8_t* c_hi = c_lo + 8 * L.crow;
+      const uint8_t* sc_lo = s_c + L.cbytes + g * srow;
+      const uint8_t* sc_hi = sc_lo + 8 * srow;
+      const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
+      const int ntiles = min(NT, (n_e + 7) / 8);
+      ActFrags<ACT_SMEM> af;
+      af.act = act;
+      af.act_s = act_s;
+      af.pstride = pstride;
+      af.K = K;
+      af.q = q;
+      af.g = g;
+      af.p0 = p0;
+      af.n_e = n_e;
+      float acc2[NT][CH][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+      for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc2[j][0][c] = acc2[j][1][c] = 0.f;
-    if (ok) stream_kblocks<FMT, NT>(acc2, 0, 1, nblk_full, tail, K, q, c_lo, c_hi, sc_lo, sc_hi, gsc, ntiles, af);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-    if (!ok) continue;
-    // c0, c1: feature f0 + g at columns 2q, 2q+1; c2, c3: feature + 8
+        for (int h = 0; h < CH; ++h)
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      if (j >= ntiles) break;
+          for (int c = 0; c < 4; ++c) acc2[j][h][c] = 0.f;
+      if (ok) warp_tile<FMT, NT, CH>(acc2, c_lo, c_hi, sc_lo, sc_hi, 0, 1, nfull, tail_b, K, q, gsc, ntiles, af);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (!ok) continue;
+      // c0, c1: feature g at columns 2q, 2q+1; c2, c3: feature g + 8
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int col = 8 * j + 2 * q + (c & 1);
-        if (col < n_e)
-          ypart[size_t(p0 + col) * H + f0 + g + 8 * (c >> 1)] = s_wrow[p0 + col] * (acc2[j][0][c] + acc2[j][1][c]);
+      for (int j = 0; j < NT; ++j) {
+        if (j >= ntiles) break;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = 8 * j + 2 * q + (c & 1);
+          if (col < n_e) {
+            float v = acc2[j][0][c];
+#pragma unroll
+            for (int h = 1; h < CH; ++h) v += acc2[j][h][c];
+            ybuf[s_slot[p0 + col] * kDnRows + g + 8 * (c >> 1)] = s_w[p0 + col] * v;
+          }
+        }
       }
     }
+    named_barrier_sync(1, kConsumers);
+    // each token's k slots summed in slot order, two features per thread
+    for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kConsumers) {
+      const int t = o / (kDnRows / 2), f = 2 * (o % (kDnRows / 2));
+      float v0 = 0.f, v1 = 0.f;
+      for (int j = 0; j < top_k; ++j) {
+        float* yb = ybuf + (t * top_k + j) * kDnRows + f;
+        v0 += yb[0];
+        v1 += yb[1];
+        yb[0] = 0.f;
+        yb[1] = 0.f;
+      }
+      const size_t oi = size_t(t) * H + tile * kDnRows + f;
+      if (partial_out) {
+        *reinterpret_cast<float2*>(partial_out + oi) = make_float2(v0, v1);
+      } else {
+        if (sh_y) {
+          const float gg = __ldcg(sh_gate + t);
+          v0 += gg * __ldcg(sh_y + oi);
+          v1 += gg * __ldcg(sh_y + oi + 1);
+        }
+        *reinterpret_cast<uint32_t*>(out + oi) = pack_bf16x2(v0, v1);
+      }
+    }
+    named_barrier_sync(1, kConsumers);
   }
 }
 
 int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
 
-// stages + staged token rows + the partial-tile buffers + routing state + barriers
-size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows) {
-  const UnitLayout L = unit_layout(fmt, K, 16);
-  return size_t(kStages) * L.stage_bytes + size_t(x_rows) * staged_row_stride(K) +
-         size_t(kGroups) * 2 * kGroupWarps * NT * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 +
-         (2 * kStages + 1) * 8;
-}
-
-size_t down_smem(int fmt, int K, int E, int R, int act_rows) {
-  const UnitLayout L = unit_layout(fmt, K, kDnRows);
-  return size_t(kStages) * L.stage_bytes + size_t(act_rows) * staged_row_stride(K) + size_t(2 * (E + 1) + R) * 4 +
-         8 + (2 * kStages + 1) * 8;
-}
-
-// Staged token rows (gate_up) and activation rows (down) up to these sizes.
-constexpr size_t kMaxStagedX = 36 * 1024;
-constexpr size_t kMaxStagedAct = 36 * 1024;
 constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving room for static
+// Staged token rows (gate_up) and activation rows (down) up to these sizes.
+constexpr size_t kMaxStagedX = 72 * 1024;
+constexpr size_t kMaxStagedAct = 72 * 1024;
+
+int nt_of(int T) { return T <= 8 ? 1 : T <= 16 ? 2 : 4; }
+
+// gate_up: stages + staged token rows + the partial-tile buffers + routing
+// state + barriers
+size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows, int S) {
+  const StageLayout L = stage_layout(fmt, K, 16);
+  return size_t(S) * L.stage_bytes + size_t(x_rows) * staged_act_stride(K) +
+         size_t(kGuGroups) * 2 * kGroupWarps * NT * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 + 2 * size_t(S) * 8;
+}
+
+// down: stages + staged activation rows + the slot outputs + routing state +
+// barriers
+size_t down_smem(int fmt, int K, int E, int R, int act_rows, int S) {
+  const StageLayout L = stage_layout(fmt, K, kDnRows);
+  return size_t(S) * L.stage_bytes + size_t(act_rows) * staged_act_stride(K) + size_t(R) * kDnRows * 4 +
+         size_t(2 * (E + 1) + 2 * R) * 4 + 8 + 2 * size_t(S) * 8;
+}
+
+struct GuPlan {
+  bool x_smem;
+  int S;
+  size_t smem;
+};
+struct DnPlan {
+  bool act_smem;
+  int S;
+  size_t smem;
+};
+
+// The largest stage ring (a multiple of the consumer groups, at least two
+// stages per group) that fits beside the rest; S = 0 when none does.
+GuPlan gate_up_plan(const moe_shape_t& s, int T) {
+  const int R = T * s.top_k, NT = nt_of(T);
+  GuPlan p;
+  p.x_smem = size_t(T) * staged_act_stride(s.hidden) <= kMaxStagedX;
+  p.S = 0;
+  p.smem = 0;
+  for (int S = kGuMaxStages / kGuGroups * kGuGroups; S >= 2 * kGuGroups; S -= kGuGroups) {
+    const size_t b = gate_up_smem(s.fmt, s.hidden, NT, s.num_experts, R, p.x_smem ? T : 0, S);
+    if (b <= kMaxSmemPerCta) {
+      p.S = S;
+      p.smem = b;
+      break;
+    }
+  }
+  return p;
+}
+
+DnPlan down_plan(const moe_shape_t& s, int T) {
+  const int R = T * s.top_k;
+  DnPlan p;
+  p.act_smem = size_t(R) * staged_act_stride(s.inter) <= kMaxStagedAct;
+  p.S = 0;
+  p.smem = 0;
+  for (int S = kDnMaxStages / kDnWarps * kDnWarps; S >= kDnWarps; S -= kDnWarps) {
+    const size_t b = down_smem(s.fmt, s.inter, s.num_experts, R, p.act_smem ? R : 0, S);
+    if (b <= kMaxSmemPerCta) {
+      p.S = S;
+      p.smem = b;
+      break;
+    }
+  }
+  return p;
+}
 
 int sm_count_cached() {
   static std::atomic<int> cached{0};
@@ -513,17 +644,15 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 template <int FMT, int NT>
 cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const ExpertRange& er,
                        const Workspace& ws, int units, cudaStream_t stream) {
-  const int R = T * s.top_k;
-  const bool x_smem = size_t(T) * staged_row_stride(s.hidden) <= kMaxStagedX;
-  auto k = x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
-  const size_t smem = gate_up_smem(FMT, s.hidden, NT, s.num_experts, R, x_smem ? T : 0);
-  if (smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
-  cudaError_t err = allow_smem(k, smem);
+  const GuPlan p = gate_up_plan(s, T);
+  if (p.S == 0) return cudaErrorInvalidConfiguration;
+  auto k = p.x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
+  cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(k, smem, units, kThreads);
-  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k, er.lo,
-                    er.hi, (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
-                    ws.act, ws.status);
+  const int grid = persistent_grid(k, p.smem, units, kGuThreads);
+  return launch_pdl(k, dim3(grid), dim3(kGuThreads), p.smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k,
+                    er.lo, er.hi, (const int32_t*)ws.touched, (const int32_t*)ws.offsets,
+                    (const int32_t*)ws.sorted_rows, ws.act, ws.status, p.S);
 }
 
 template <int FMT>
@@ -537,43 +666,33 @@ cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Ba
 
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
-                    cudaStream_t stream) {
-  const int R = T * s.top_k;
-  const bool act_smem = size_t(R) * staged_row_stride(s.inter) <= kMaxStagedAct;
-  auto k = act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
-  const size_t smem = down_smem(FMT, s.inter, s.num_experts, R, act_smem ? R : 0);
-  if (smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
-  cudaError_t err = allow_smem(k, smem);
+                    const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out, cudaStream_t stream) {
+  const DnPlan p = down_plan(s, T);
+  if (p.S == 0) return cudaErrorInvalidConfiguration;
+  auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
+  cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
-  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.hidden / kDnRows);
-  const int grid = persistent_grid(k, smem, std::max(units, 1), kThreads);
-  return launch_pdl(k, dim3(grid), dim3(kThreads), smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
+  const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, kDnThreads);
+  return launch_pdl(k, dim3(grid), dim3(kDnThreads), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
-                    (const uint16_t*)ws.act, (const float*)ws.topk_w, ws.ypart, ws.status);
+                    (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out, ws.status,
+                    p.S);
 }
 
 template <int FMT>
 cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
+                     const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out,
                      cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, stream);
-  return down_nt<FMT, 4>(s, T, dn, er, ws, stream);
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+  return down_nt<FMT, 4>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
 }
 
 }  // namespace
 
 bool decode_supported(const moe_shape_t& s, int T) {
   if (T > kDecodeMaxT) return false;
-  const int R = T * s.top_k;
-  const int NT = T <= 8 ? 1 : T <= 16 ? 2 : 4;
-  const bool x_smem = size_t(T) * staged_row_stride(s.hidden) <= kMaxStagedX;
-  const bool act_smem = size_t(R) * staged_row_stride(s.inter) <= kMaxStagedAct;
-  return gate_up_smem(s.fmt, s.hidden, NT, s.num_experts, R, x_smem ? T : 0) <= kMaxSmemPerCta &&
-         down_smem(s.fmt, s.inter, s.num_experts, R, act_smem ? R : 0) <= kMaxSmemPerCta;
-}
-
-size_t decode_ypart_bytes(const moe_shape_t& s, int T) {
-  return T <= kDecodeMaxT ? size_t(T) * s.top_k * s.hidden * 4 : 0;
+  return gate_up_plan(s, T).S > 0 && down_plan(s, T).S > 0;
 }
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
@@ -586,11 +705,14 @@ cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x
 }
 
 cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                               const Workspace& ws, cudaStream_t stream) {
+                               const Workspace& ws, const float* sh_gate, const float* sh_y, uint16_t* out,
+                               float* partial_out, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, stream);
+  if (s.fmt == MOE_FMT_INT4_G128)
+    return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16)
+    return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
 }
 
 }  // namespace moe

@@ -1,6 +1,7 @@
 // Device helpers of the decode (small-batch) expert kernels: mma.sync
 // m16n8k16 on dequantised 4-bit weight fragments, the fragment k-permutation
-// shared by weights and activations, and the bulk-copy staging of packed rows.
+// shared by weights and activations, and the shared-memory layouts the
+// kernels stage weights and activations in.
 //
 // Fragment k-permutation.  Inside a 128-k block, lane (g = lane/4, q = lane%4)
 // owns k in [32q, 32q+32).  For MMA step s = 2*j + h (j = 32-bit code word,
@@ -22,7 +23,19 @@
 // s * 2^133 and s * 2^129 are bf16 values when s is normal and below 2^-5
 // (exponent field 1..121); they are built by adding to the exponent field.
 // Other scales (zero, subnormal, >= 2^-5) take the two-step path: the exact
-// small integer q = (128 + u) - 136, then one multiply by s.
+// small integer q = (128 + u) - 136, then one multiply by s.  The choice is
+// made once per warp and work unit, so the inner loop has no branches.
+//
+// Shared-memory layouts.
+//  * Weight rows: each staged row starts (K/2 rounded up to 128) + 64 bytes
+//    after the previous one, so the rows g and g + 1 that one 8-lane phase of
+//    a 16-byte load reads lie in opposite halves of the 32 banks.
+//  * Activation rows in fragment order: row r, k-block b starts at
+//    r * pstride + 256 b, and its 16-byte unit 4 i + q holds lane slice q's
+//    fragment words of MMA steps 2i and 2i+1, so a lane's 16 fragment words
+//    are four 16-byte loads with no permutes and four consecutive lanes read
+//    64 consecutive bytes.  pstride = 256 * blocks + 64 puts consecutive rows
+//    in opposite bank halves.
 #pragma once
 
 #include "common.cuh"
@@ -62,93 +75,84 @@ __host__ __device__ inline int scale_row_bytes(int fmt, int K) {
   return fmt == MOE_FMT_INT4_G128 ? int4_groups(K) * 2 : fmt == MOE_FMT_NVFP4_G16 ? K / 16 : K / 32;
 }
 
-// A lane's 32-k slice of one weight row at one 128-k block: its 16 code bytes
-// and what turns them into bf16 weights.
+// What turns a lane's 16 code bytes of one weight row at one 128-k block into
+// bf16 weights:
 //   INT4:  m0 = s * 2^133, m1 = s * 2^129, m2 = -8 s (bf16x2, both halves
-//          equal) and fast = 1 when those are exact, else fast = 0; sd = s in
-//          both halves (the two-step path's multiplier).
+//          equal); the two-step path multiplies by s, recovered as m0 minus
+//          the constant that added 133 to the exponent field.
 //   MXFP4: m0 = m1 = the multiplier of its 32-element block, m2 = the
 //          two-step flag.
 //   NVFP4: m0 / m1 = the multipliers of its two 16-element blocks (code words
 //          0-1 / 2-3), m2 = the two-step flag.
-// A slice past K has zero codes and zero multipliers (zero weights).
-struct RowChunk {
-  uint4 codes;
+// A slice past K has zero multipliers (and zero codes): zero weights.
+struct Mult {
   uint32_t m0, m1, m2;
-  uint32_t sd;
-  uint32_t fast;
 };
 
-// INT4 multipliers of scale bits s (see the top of this file).
-MOE_DEV void int4_mults(uint32_t s, RowChunk& rc) {
-  const uint32_t sd = s * 0x00010001u;
-  rc.sd = sd;
-  rc.m0 = sd + 0x42804280u;  // exponent + 133
-  rc.m1 = sd + 0x40804080u;  // exponent + 129
-  rc.m2 = sd + 0x81808180u;  // exponent + 3, sign set: -8 s
-  rc.fast = (s - 0x0080u < 0x3D00u - 0x0080u) ? 1u : 0u;
-}
-
-// The chunk of k-block b of one staged weight row: `codes` points at the row's
-// codes plus the lane's slice offset 16q, `scales` at the row's scales; `in` is
-// false for a slice past K; `g` is the matrix's NVFP4 global scale.
+// Multipliers of block b from the row's staged scales; `fast` is cleared when
+// the single-instruction path is not exact for them.
 template <int FMT>
-MOE_DEV RowChunk row_chunk_at(const uint8_t* codes, const uint8_t* scales, int b, int q, bool in, float g = 0.f) {
-  RowChunk rc;
-  if (in) {
-    rc.codes = *reinterpret_cast<const uint4*>(codes + 64 * b);
-    if (FMT == MOE_FMT_INT4_G128) {
-      int4_mults(reinterpret_cast<const uint16_t*>(scales)[b], rc);  // group b = k-block b
-    } else if (FMT == MOE_FMT_NVFP4_G16) {
-      // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
-      nv_mult_pair_scaled(scales + 8 * b + 2 * q, g, rc.m0, rc.m1, rc.m2);
-      rc.fast = 1u;
-    } else {
-      mx_mult(int(scales[4 * b + q]) - 127, rc.m0, rc.m2);  // the slice is one 32-element block
-      rc.m1 = rc.m0;
-      rc.fast = 1u;
-    }
-  } else {
-    rc.codes = make_uint4(0, 0, 0, 0);
-    rc.m0 = rc.m1 = rc.m2 = rc.sd = 0u;
-    rc.fast = 1u;
+MOE_DEV Mult mult_at(const uint8_t* scales, int b, int q, float gsc, bool in, bool& fast) {
+  Mult m;
+  if (!in) {
+    // zero weights on both paths (INT4's two-step multiplier m0 - C is 0)
+    m.m0 = FMT == MOE_FMT_INT4_G128 ? 0x42804280u : 0u;
+    m.m1 = m.m2 = 0u;
+    return m;
   }
-  return rc;
+  if (FMT == MOE_FMT_INT4_G128) {
+    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[b];  // group b = k-block b
+    const uint32_t sd = s * 0x00010001u;
+    m.m0 = sd + 0x42804280u;  // exponent + 133
+    m.m1 = sd + 0x40804080u;  // exponent + 129
+    m.m2 = sd + 0x81808180u;  // exponent + 3, sign set: -8 s
+    fast = fast && (s - 0x0080u < 0x3D00u - 0x0080u);
+  } else if (FMT == MOE_FMT_NVFP4_G16) {
+    // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
+    nv_mult_pair_scaled(scales + 8 * b + 2 * q, gsc, m.m0, m.m1, m.m2);
+    fast = fast && m.m2 == 0u;
+  } else {
+    mx_mult(int(scales[4 * b + q]) - 127, m.m0, m.m2);  // the slice is one 32-element block
+    m.m1 = m.m0;
+    fast = fast && m.m2 == 0u;
+  }
+  return m;
 }
 
-// The bf16 pair (nibbles i, i+4) of code word j of a chunk.
+// The bf16 pair (nibbles i, i+4) of code word j.
 template <int FMT, bool FAST>
-MOE_DEV uint32_t dq(const RowChunk& rc, uint32_t word, int i, int j) {
+MOE_DEV uint32_t dq(const Mult& m, uint32_t word, int i, int j) {
   if (FMT == MOE_FMT_INT4_G128) {
     if (FAST) {
       const uint32_t t = i >= 2 ? word >> 8 : word;
       const uint32_t v = t & ((i & 1) ? 0x00F000F0u : 0x000F000Fu);
-      return bf16x2_fma(v, (i & 1) ? rc.m1 : rc.m0, rc.m2);
+      return bf16x2_fma(v, (i & 1) ? m.m1 : m.m0, m.m2);
     }
-    return bf16x2_mul(int4_pair(word, i), rc.sd);
+    return bf16x2_mul(int4_pair(word, i), m.m0 - 0x42804280u);
   }
   // E2M1: codes as value * 2^-126; the multipliers carry 2^126 unless m2
   uint32_t v = e2m1_pair_scaled(word, i);
-  if (rc.m2) v = bf16x2_mul(v, kBf16x2Pow126);
-  return bf16x2_mul(v, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? rc.m1 : rc.m0);
+  if (!FAST && m.m2) v = bf16x2_mul(v, kBf16x2Pow126);
+  return bf16x2_mul(v, (FMT == MOE_FMT_NVFP4_G16 && j >= 2) ? m.m1 : m.m0);
 }
 
-// acc[h][4] += W(rows r, r+8; one 128-k block) x activation fragments: the
-// MMA steps of a block alternate between two accumulators (h = 0 / 1), so two
-// independent dependency chains are in flight instead of one.
-template <int FMT, bool FAST>
-MOE_DEV void mma_block2(float (&acc)[2][4], const RowChunk& lo, const RowChunk& hi, const uint32_t (&b)[8][2]) {
+// acc[c0 + h] += W(rows r, r+8; one 128-k block) x activation fragments: the
+// two MMA steps of each code word go to two accumulator chains, so chains of
+// independent MMAs are in flight instead of one.
+template <int FMT, bool FAST, int CH>
+MOE_DEV void mma_kblock(float (&acc)[CH][4], int c0, const uint4& lo, const uint4& hi, const Mult& mlo,
+                        const Mult& mhi, const uint32_t (&b)[8][2]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t wl = word_of(lo.codes, j), wh = word_of(hi.codes, j);
+    const uint32_t wl = word_of(lo, j), wh = word_of(hi, j);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t a[4];
-      a[0] = dq<FMT, FAST>(lo, wl, 2 * h, j);
-      a[1] = dq<FMT, FAST>(hi, wh, 2 * h, j);
-      a[2] = dq<FMT, FAST>(lo, wl, 2 * h + 1, j);
-      a[3] = dq<FMT, FAST>(hi, wh, 2 * h + 1, j);
-      mma_bf16_16816(acc[h], a, b[2 * j + h][0], b[2 * j + h][1]);
+      a[0] = dq<FMT, FAST>(mlo, wl, 2 * h, j);
+      a[1] = dq<FMT, FAST>(mhi, wh, 2 * h, j);
+      a[2] = dq<FMT, FAST>(mlo, wl, 2 * h + 1, j);
+      a[3] = dq<FMT, FAST>(mhi, wh, 2 * h + 1, j);
+      mma_bf16_16816(acc[c0 + h], a, b[2 * j + h][0], b[2 * j + h][1]);
     }
   }
 }
@@ -165,18 +169,18 @@ MOE_DEV void act_frags_from_raw(const uint32_t (&X)[16], uint32_t (&b)[8][2]) {
   }
 }
 
-// Activation fragments of one lane's 32-k slice (64 bytes at p) of a bf16 row.
-// SRC 0: shared memory; 1: global, read-only for the kernel's lifetime
-// (ld.global.nc); 2: global, written by an earlier kernel (ld.global.cg).
-// With VALID false the fragments are zero (slices past K).
+// Activation fragments of one lane's 32-k slice (64 bytes at p) of a bf16 row
+// in global memory.  SRC 1: read-only for the kernel's lifetime
+// (ld.global.nc); 2: written by an earlier kernel (ld.global.cg).  With
+// `valid` false the fragments are zero (slices past K).
 template <int SRC>
-MOE_DEV void act_frags(const uint16_t* p, bool valid, uint32_t (&b)[8][2]) {
+MOE_DEV void act_frags_global(const uint16_t* p, bool valid, uint32_t (&b)[8][2]) {
   uint32_t X[16];
   if (valid) {
     const uint4* v = reinterpret_cast<const uint4*>(p);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 w = SRC == 0 ? v[i] : SRC == 1 ? __ldg(v + i) : __ldcg(v + i);
+      const uint4 w = SRC == 1 ? __ldg(v + i) : __ldcg(v + i);
       X[4 * i] = w.x; X[4 * i + 1] = w.y; X[4 * i + 2] = w.z; X[4 * i + 3] = w.w;
     }
   } else {
@@ -186,87 +190,150 @@ MOE_DEV void act_frags(const uint16_t* p, bool valid, uint32_t (&b)[8][2]) {
   act_frags_from_raw(X, b);
 }
 
-// One warp's pass over the 128-k blocks b0, b0 + step, ... below nblk_full of
-// one 16-row weight tile (rows r and r + 8 of the lane: codes c_lo / c_hi and
-// scales sc_lo / sc_hi in shared memory), then the optional block `tail`
-// (>= 0) whose lane slices may lie past K.  The next block's weights and first
-// token tile's activations are loaded before the current block's math (two
-// register buffers, no copies).  `act.load(j, b, in, bf)` gives token tile j's
-// fragments of block b.  acc[j][h] are the two accumulator chains of tile j.
-template <int FMT, int NT, typename Act>
-MOE_DEV void stream_kblocks(float (&acc)[NT][2][4], int b0, int step, int nblk_full, int tail, int K, int q,
-                            const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo, const uint8_t* sc_hi,
-                            float gsc, int ntiles, const Act& act) {
-  auto compute = [&](const RowChunk& lo, const RowChunk& hi, const uint32_t (&f0)[8][2], int b, bool in) {
-    // warp-uniform: mma.sync needs the whole warp on one path (the two-step
-    // path is exact for every scale)
-    const bool fast = __all_sync(0xffffffffu, (lo.fast & hi.fast) != 0u);
-    if (fast) mma_block2<FMT, true>(acc[0], lo, hi, f0);
-    else mma_block2<FMT, false>(acc[0], lo, hi, f0);
+// Activation fragments of lane slice q of a k-block staged in fragment order
+// (`blk` = the row's block start).
+MOE_DEV void act_frags_staged(const uint8_t* blk, int q, bool valid, uint32_t (&b)[8][2]) {
 #pragma unroll
-    for (int j = 1; j < NT; ++j) {
-      if (j >= ntiles) break;
-      uint32_t fj[8][2];
-      act.load(j, b, in, fj);
-      if (fast) mma_block2<FMT, true>(acc[j], lo, hi, fj);
-      else mma_block2<FMT, false>(acc[j], lo, hi, fj);
-    }
-  };
-  int b = b0;
-  if (b < nblk_full) {
-    RowChunk a_lo = row_chunk_at<FMT>(c_lo, sc_lo, b, q, true, gsc);
-    RowChunk a_hi = row_chunk_at<FMT>(c_hi, sc_hi, b, q, true, gsc);
-    uint32_t fa[8][2];
-    act.load(0, b, true, fa);
-    for (;;) {
-      const int b1 = b + step;
-      RowChunk b_lo, b_hi;
-      uint32_t fb[8][2];
-      if (b1 < nblk_full) {
-        b_lo = row_chunk_at<FMT>(c_lo, sc_lo, b1, q, true, gsc);
-        b_hi = row_chunk_at<FMT>(c_hi, sc_hi, b1, q, true, gsc);
-        act.load(0, b1, true, fb);
-      }
-      compute(a_lo, a_hi, fa, b, true);
-      if (b1 >= nblk_full) break;
-      const int b2 = b1 + step;
-      if (b2 < nblk_full) {
-        a_lo = row_chunk_at<FMT>(c_lo, sc_lo, b2, q, true, gsc);
-        a_hi = row_chunk_at<FMT>(c_hi, sc_hi, b2, q, true, gsc);
-        act.load(0, b2, true, fa);
-      }
-      compute(b_lo, b_hi, fb, b1, true);
-      if (b2 >= nblk_full) break;
-      b = b2;
-    }
-  }
-  if (tail >= 0) {
-    const bool in = 128 * tail + 32 * q < K;
-    const RowChunk lo = row_chunk_at<FMT>(c_lo, sc_lo, tail, q, in, gsc);
-    const RowChunk hi = row_chunk_at<FMT>(c_hi, sc_hi, tail, q, in, gsc);
-    uint32_t f0[8][2];
-    act.load(0, tail, in, f0);
-    compute(lo, hi, f0, tail, in);
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = valid ? *reinterpret_cast<const uint4*>(blk + (4 * i + q) * 16) : make_uint4(0, 0, 0, 0);
+    b[2 * i][0] = v.x;
+    b[2 * i][1] = v.y;
+    b[2 * i + 1][0] = v.z;
+    b[2 * i + 1][1] = v.w;
   }
 }
 
-// Number of 128-k blocks in which lane slice q (k in [kb + 32q, kb + 32q + 32))
-// lies inside K (K a multiple of 32).
-MOE_DEV int lane_kblocks(int K, int q) { return (K - 32 * q + 127) >> 7; }
+// Number of 128-k blocks of a row of length K, and the row stride of bf16
+// rows staged in fragment order.
+__host__ __device__ inline int kblocks(int K) { return (K + 127) / 128; }
+__host__ __device__ inline int staged_act_stride(int K) { return 256 * kblocks(K) + 64; }
 
-// Row stride of bf16 rows of length K staged in shared memory: 16 bytes of
-// padding shift consecutive rows by four banks, so the eight rows of an MMA
-// fragment load do not all start in the same bank.
-__host__ __device__ inline int staged_row_stride(int K) { return 2 * K + 16; }
+// Stage `rows` bf16 rows of length K (global, row stride K) in fragment order
+// at `dst`; slices past K are zero.  Threads `tid` of `nthreads` share the
+// work, one (row, block, lane slice) of 64 bytes at a time: four adjacent
+// threads read 256 consecutive bytes and write 64-byte runs.
+template <int SRC>
+MOE_DEV void stage_act_rows(uint8_t* dst, const uint16_t* src, int rows, int K, int tid, int nthreads) {
+  const int nblk = kblocks(K);
+  const int pstride = staged_act_stride(K);
+  const int items = rows * nblk * 4;
+  for (int it = tid; it < items; it += nthreads) {
+    const int q = it & 3, rb = it >> 2;
+    const int r = rb / nblk, b = rb - r * nblk;
+    const int k0 = 128 * b + 32 * q;
+    uint32_t X[16];
+    if (k0 < K) {
+      const uint4* v = reinterpret_cast<const uint4*>(src + size_t(r) * K + k0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = SRC == 1 ? __ldg(v + i) : __ldcg(v + i);
+        X[4 * i] = w.x; X[4 * i + 1] = w.y; X[4 * i + 2] = w.z; X[4 * i + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) X[i] = 0;
+    }
+    uint32_t f[8][2];
+    act_frags_from_raw(X, f);
+    uint8_t* o = dst + size_t(r) * pstride + 256 * b + 16 * q;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4*>(o + 64 * i) = make_uint4(f[2 * i][0], f[2 * i][1], f[2 * i + 1][0], f[2 * i + 1][1]);
+  }
+}
 
-// Start one bulk copy per bf16 row of length K (rows [lane, lane+32, ...) <
-// `rows`) from global `src` into shared memory at `dst` with the padded row
-// stride, all completing on `bar`.  Called by every lane of one warp after
-// lane 0 announced rows * 2K bytes on `bar`.
-MOE_DEV void stage_bf16_rows(uint8_t* dst, const uint16_t* src, int rows, int K, uint64_t* bar) {
-  const int lane = threadIdx.x & 31;
-  const int stride = staged_row_stride(K);
-  for (int r = lane; r < rows; r += 32) bulk_g2s(dst + size_t(r) * stride, src + size_t(r) * K, uint32_t(2 * K), bar);
+// Shared-memory layout of one stage of `rows` weight rows: codes at the
+// padded row stride crow, then the rows' scales (contiguous, padded to 16).
+struct StageLayout {
+  int crow, cbytes, sbytes, stage_bytes;
+};
+
+__host__ __device__ inline StageLayout stage_layout(int fmt, int K, int rows) {
+  StageLayout l;
+  l.crow = (((K / 2) + 127) & ~127) + 64;
+  l.cbytes = rows * l.crow;
+  l.sbytes = rows * scale_row_bytes(fmt, K);
+  l.stage_bytes = l.cbytes + ((l.sbytes + 15) & ~15);
+  return l;
+}
+
+// One warp, one 16-row weight tile staged at c_lo (row r = lane/4; the tile's
+// row r + 8 at c_hi) with scales at sc_lo / sc_hi: acc[j] += W x B_j over the
+// NB k-blocks b0, b0 + bstep, ... (all inside K), for the token tiles
+// j < ntiles.  `act.load(j, b, in, frags)` gives token tile j's fragments of
+// block b.  CH accumulator chains per token tile (2 or 4).
+template <int FMT, int NT, int CH, int NB, bool FAST, typename Act>
+MOE_DEV void tile_run(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const Mult (&mlo)[NB],
+                      const Mult (&mhi)[NB], int b0, int bstep, int ntiles, const Act& act) {
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    const int b = b0 + i * bstep;
+    const uint4 lo = *reinterpret_cast<const uint4*>(c_lo + 64 * b);
+    const uint4 hi = *reinterpret_cast<const uint4*>(c_hi + 64 * b);
+    const int c0 = CH == 4 ? 2 * (i & 1) : 0;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (j > 0 && j >= ntiles) break;
+      uint32_t bf[8][2];
+      act.load(j, b, true, bf);
+      mma_kblock<FMT, FAST, CH>(acc[j], c0, lo, hi, mlo[i], mhi[i], bf);
+    }
+  }
+}
+
+// tile_run with the fast / two-step choice made once for all NB blocks.
+template <int FMT, int NT, int CH, int NB, typename Act>
+MOE_DEV void tile_blocks(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
+                         const uint8_t* sc_hi, int b0, int bstep, int q, float gsc, int ntiles, const Act& act) {
+  Mult mlo[NB], mhi[NB];
+  bool fast = true;
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    mlo[i] = mult_at<FMT>(sc_lo, b0 + i * bstep, q, gsc, true, fast);
+    mhi[i] = mult_at<FMT>(sc_hi, b0 + i * bstep, q, gsc, true, fast);
+  }
+  // warp-uniform: mma.sync needs the whole warp on one path (the two-step
+  // path is exact for every scale)
+  if (__all_sync(0xffffffffu, fast)) tile_run<FMT, NT, CH, NB, true>(acc, c_lo, c_hi, mlo, mhi, b0, bstep, ntiles, act);
+  else tile_run<FMT, NT, CH, NB, false>(acc, c_lo, c_hi, mlo, mhi, b0, bstep, ntiles, act);
+}
+
+// The last k-block b of a row whose length K ends inside it (K % 128 == 64):
+// lane slices past K contribute zero.
+template <int FMT, int NT, int CH, typename Act>
+MOE_DEV void tile_tail(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
+                       const uint8_t* sc_hi, int b, int K, int q, float gsc, int ntiles, const Act& act) {
+  const bool in = 128 * b + 32 * q < K;
+  bool fast = true;
+  Mult mlo[1], mhi[1];
+  mlo[0] = mult_at<FMT>(sc_lo, b, q, gsc, in, fast);
+  mhi[0] = mult_at<FMT>(sc_hi, b, q, gsc, in, fast);
+  const uint4 lo = in ? *reinterpret_cast<const uint4*>(c_lo + 64 * b) : make_uint4(0, 0, 0, 0);
+  const uint4 hi = in ? *reinterpret_cast<const uint4*>(c_hi + 64 * b) : make_uint4(0, 0, 0, 0);
+  const bool all_fast = __all_sync(0xffffffffu, fast);
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    if (j > 0 && j >= ntiles) break;
+    uint32_t bf[8][2];
+    act.load(j, b, in, bf);
+    if (all_fast) mma_kblock<FMT, true, CH>(acc[j], 0, lo, hi, mlo[0], mhi[0], bf);
+    else mma_kblock<FMT, false, CH>(acc[j], 0, lo, hi, mlo[0], mhi[0], bf);
+  }
+}
+
+// One warp's share of a 16-row tile: the nb full k-blocks b0, b0 + bstep, ...
+// (four at a time where possible) and, if tail_b >= 0, the partial block
+// tail_b.
+template <int FMT, int NT, int CH, typename Act>
+MOE_DEV void warp_tile(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
+                       const uint8_t* sc_hi, int b0, int bstep, int nb, int tail_b, int K, int q, float gsc,
+                       int ntiles, const Act& act) {
+  int i = 0;
+  for (; i + 4 <= nb; i += 4)
+    tile_blocks<FMT, NT, CH, 4>(acc, c_lo, c_hi, sc_lo, sc_hi, b0 + i * bstep, bstep, q, gsc, ntiles, act);
+  for (; i < nb; ++i)
+    tile_blocks<FMT, NT, CH, 1>(acc, c_lo, c_hi, sc_lo, sc_hi, b0 + i * bstep, bstep, q, gsc, ntiles, act);
+  if (tail_b >= 0) tile_tail<FMT, NT, CH>(acc, c_lo, c_hi, sc_lo, sc_hi, tail_b, K, q, gsc, ntiles, act);
 }
 
 // Bytes staged for `rows` consecutive weight rows (codes + scales).
@@ -275,38 +342,16 @@ MOE_DEV uint32_t staged_bytes(const Bank& bk, int rows) {
   return uint32_t(rows) * (bk.K / 2) + uint32_t(rows) * scale_row_bytes(FMT, bk.K);
 }
 
-// Start the two bulk copies (codes, scales) of `rows` consecutive weight rows
-// of a bank into shared memory, completing on `bar`.  Packed weights are read
-// once per launch: they are evicted first from L2.
+// Prefetch into L2 the codes and scales of `rows` consecutive weight rows
+// (one lane each: codes, scales).
 template <int FMT>
-MOE_DEV void stage_rows(const Bank& bk, long row0, int rows, uint8_t* s_codes, uint8_t* s_scales, uint64_t* bar,
-                        uint64_t policy) {
-  const uint32_t cbytes = uint32_t(rows) * (bk.K / 2);
-  const int sb = scale_row_bytes(FMT, bk.K);
-  bulk_g2s_hint(s_codes, bk.codes + row0 * (bk.K / 2), cbytes, bar, policy);
-  bulk_g2s_hint(s_scales, static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb, bar, policy);
-}
-
-// Prefetch into L2 the codes and scales of `rows` consecutive weight rows.
-template <int FMT>
-MOE_DEV void prefetch_rows(const Bank& bk, long row0, int rows) {
-  const int sb = scale_row_bytes(FMT, bk.K);
+MOE_DEV void prefetch_codes(const Bank& bk, long row0, int rows) {
   bulk_prefetch_l2(bk.codes + row0 * (bk.K / 2), uint32_t(rows) * (bk.K / 2));
-  bulk_prefetch_l2(static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb);
 }
-
-// Shared-memory layout of one staged work unit of `rows` weight rows: codes,
-// then scales padded to 16 bytes.
-struct UnitLayout {
-  int cbytes, sbytes, stage_bytes;
-};
-
-__host__ __device__ inline UnitLayout unit_layout(int fmt, int K, int rows) {
-  UnitLayout l;
-  l.cbytes = rows * (K / 2);
-  l.sbytes = rows * scale_row_bytes(fmt, K);
-  l.stage_bytes = l.cbytes + ((l.sbytes + 15) & ~15);
-  return l;
+template <int FMT>
+MOE_DEV void prefetch_scales(const Bank& bk, long row0, int rows) {
+  const int sb = scale_row_bytes(FMT, bk.K);
+  bulk_prefetch_l2(static_cast<const uint8_t*>(bk.scales) + row0 * sb, uint32_t(rows) * sb);
 }
 
 }  // namespace moe

@@ -70,7 +70,7 @@ struct Workspace {
   int32_t* block_hist;    // [nblk, E] per-block expert histograms (large-T permutation)
   uint16_t* act;          // [T*k, I] bf16 SwiGLU output, expert-sorted rows
   float* out_acc;         // [T, H] fp32 combine accumulator (grouped-GEMM path)
-  float* ypart;           // [T*k, H] fp32 per-row down outputs (decode path, T <= kDecodeMaxT)
+  float* ypart;           // [T*k, H] fp32 per-row down outputs (deterministic grouped combine)
   float* route_part;      // [H/256, T, E] fp32 split-K router partials (small-batch routing)
   size_t bytes;
 };
@@ -112,13 +112,14 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 // the decode kernels take this shape and token count (T <= kDecodeMaxT and the
 // stages fit in shared memory)
 bool decode_supported(const moe_shape_t& s, int T);
-size_t decode_ypart_bytes(const moe_shape_t& s, int T);
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
-// the routing-weighted down outputs of the bank's experts' sorted rows into
-// ws.ypart [T*k, H] fp32 (combine_rows sums them)
+// the down products of the bank's experts and the combine: out = bf16(sum
+// over each token's slots in slot order of w * y (+ sh_gate[t] * sh_y[t])),
+// or the fp32 sum over the bank's experts into partial_out (sh_* nullable)
 cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
-                               const Workspace& ws, cudaStream_t stream);
+                               const Workspace& ws, const float* sh_gate, const float* sh_y, uint16_t* out,
+                               float* partial_out, cudaStream_t stream);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile
