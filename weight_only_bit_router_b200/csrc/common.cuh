@@ -120,8 +120,7 @@ constexpr uint32_t kBf16x2Pow126 = 0x7E807E80u;  // 2^126 in both halves
 // within [2^-126, 3.9), i.e. the bf16 rounding is in the normal range and the
 // scaled value stays finite; otherwise the plain multipliers (two = 1, and
 // the caller first multiplies the codes by 2^126).
-MOE_DEV void nv_mult_pair_scaled(const uint8_t* p, float g, uint32_t& m0, uint32_t& m1, uint32_t& two) {
-  const uint16_t pair = *reinterpret_cast<const uint16_t*>(p);
+MOE_DEV void nv_mult_pair_scaled_v(uint16_t pair, float g, uint32_t& m0, uint32_t& m1, uint32_t& two) {
   uint32_t h2;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
   const float v0 = __fmul_rn(__half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu))), g);
@@ -132,6 +131,9 @@ MOE_DEV void nv_mult_pair_scaled(const uint8_t* p, float g, uint32_t& m0, uint32
   asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m0) : "f"(a));
   asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(m1) : "f"(b));
   two = fold ? 0u : 1u;
+}
+MOE_DEV void nv_mult_pair_scaled(const uint8_t* p, float g, uint32_t& m0, uint32_t& m1, uint32_t& two) {
+  nv_mult_pair_scaled_v(*reinterpret_cast<const uint16_t*>(p), g, m0, m1, two);
 }
 
 // --------------------------------------------------------------------------
@@ -170,21 +172,33 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps (issues nothing) until the phase completes or about `ns` pass, so a
+// waiting warp leaves the issue slots to the warps doing work.
+MOE_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kSuspendNs = 20000;  // longest sleep per try: 20 us
+
 // Wait for the phase of `bar` with the given parity.  Gives up (returns
 // false) once `abort` is raised by another thread of the CTA or after
 // kWaitLimitNs, in which case it raises `abort` and the global status word.
 MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* gstatus) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 255u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        if (gstatus) atomicOr(gstatus, kStatusTimeout);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      if (gstatus) atomicOr(gstatus, kStatusTimeout);
+      return false;
     }
   }
 }
@@ -193,7 +207,7 @@ MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint
 // gives up (false) after limit_ns.  Used to drain copies still in flight.
 MOE_DEV bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kSuspendNs)) {
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
   return true;

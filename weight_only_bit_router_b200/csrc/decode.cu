@@ -2,22 +2,28 @@
 //
 // The time goes into streaming the touched experts' packed weights from HBM
 // ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", Measured: at concurrency 32
-// the bottleneck is weight bandwidth).  Both kernels are persistent: one
-// producer warp per CTA starts 1-D bulk copies of 16-row weight tiles (one
-// copy per row, at a padded shared-memory stride, plus their scales) into a
-// ring of stages and keeps the next tiles' bytes in flight (and the tile after
-// the ring into L2); consumer warps dequantise in registers
-// (decode_common.cuh) and feed mma.sync m16n8k16 with up to 32 tokens.  The
-// routing state (touched experts, per-expert row offsets, the rows' tokens) is
-// read into shared memory once per CTA, and small token / activation sets are
-// staged there once in MMA fragment order.
+// the bottleneck is weight bandwidth).  Consumer warps dequantise in
+// registers (decode_common.cuh) and feed mma.sync m16n8k16 with up to 32
+// tokens; small token / activation sets are staged in shared memory once per
+// CTA in MMA fragment order, and the routing state (touched experts,
+// per-expert row offsets, the rows' tokens) is read into shared memory once
+// per CTA.
 //
-// gate_up: CTA c takes a contiguous run of the (touched expert, 8-feature)
-// units; four warps split each unit's k-blocks and sum in shared memory.
+// gate_up: persistent; CTA c takes a contiguous run of the (touched expert,
+// 16-feature) units.  One producer warp starts, per unit, two 16 KB-class
+// bulk copies (the 16 gate rows, the 16 up rows) and two of their scales into
+// a ring of shared-memory stages, and prefetches the unit that will next
+// refill the stage into L2; four consumer warps split each unit's k-blocks
+// and sum in shared memory.  Few large copies: the bulk-copy engine's cost is
+// per copy as much as per byte.
 // down: CTA c owns 16 output features of every token and runs over all
 // touched experts, so the routing-weighted combine of a token's k expert
 // outputs happens in the CTA (in slot order, deterministic) and the output is
-// written once.
+// written once.  Its 16-row weight tiles are small (16 rows x I/2 bytes), so
+// each warp loads its tiles straight into registers, the next tile's loads in
+// flight while the current one is multiplied, all of its tiles requested
+// into L2 up front, and the first tile's loads issued before the
+// programmatic-launch wait.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -32,29 +38,42 @@ namespace moe {
 namespace {
 
 constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
+constexpr int kGuFeat = 16;     // gate_up: features per work unit (16 gate + 16 up rows)
+constexpr int kGuMT = 2;        // gate_up: 16-row MMA tiles per unit
 
 // Build-time tuning knobs (the defaults are the measured best): gate_up
-// consumer groups per CTA and its largest stage ring; down consumer warps per
-// CTA and its largest stage ring.
+// consumer groups per CTA and its largest stage ring; down warps per CTA.
 #ifndef MOE_DEC_GROUPS
 #define MOE_DEC_GROUPS 2
 #endif
 #ifndef MOE_DEC_STAGES
-#define MOE_DEC_STAGES 8
+#define MOE_DEC_STAGES 4
 #endif
 #ifndef MOE_DEC_DN_WARPS
 #define MOE_DEC_DN_WARPS 8
-#endif
-#ifndef MOE_DEC_DN_STAGES
-#define MOE_DEC_DN_STAGES 32
 #endif
 constexpr int kGuGroups = MOE_DEC_GROUPS;
 constexpr int kGuMaxStages = MOE_DEC_STAGES;
 constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
 constexpr int kDnWarps = MOE_DEC_DN_WARPS;
-constexpr int kDnMaxStages = MOE_DEC_DN_STAGES;
-constexpr int kDnThreads = (kDnWarps + 1) * 32;
+constexpr int kDnThreads = kDnWarps * 32;
 constexpr int kDnRows = 16;  // output features per down tile
+
+// Offsets inside one gate_up stage: gate-row codes, 64 bytes of padding,
+// up-row codes, then gate-row and up-row scales (see decode_common.cuh).
+struct GuLayout {
+  int cA, cB, sA, sB, stage_bytes;
+};
+__host__ __device__ inline GuLayout gu_layout(int fmt, int K) {
+  const int run = kGuFeat * (K / 2), srun = kGuFeat * scale_row_bytes(fmt, K);
+  GuLayout l;
+  l.cA = 0;
+  l.cB = run + 64;
+  l.sA = 2 * run + 64;
+  l.sB = l.sA + srun;
+  l.stage_bytes = (l.sB + srun + 127) & ~127;
+  return l;
+}
 
 // The routing state every CTA keeps in shared memory: the touched-expert list
 // [n, e_0, e_1, ...] and the per-expert row offsets (E + 1 entries each).
@@ -131,40 +150,19 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
   for (int i = max(0, issued - S); i < issued; ++i) mbar_wait_drain(&full[i % S], (i / S) & 1, kWaitLimitNs);
 }
 
-// Start the copies of one 16-row weight tile into `stage` (codes at the padded
-// row stride, then scales): lanes 0-15 one code row each (source rows
-// row_a + l for l < 8, row_b + l - 8 after), lanes 16 / 17 the scales of the
-// two 8-row runs (16 contiguous rows when row_b = row_a + 8: lane 16 alone).
-// Called by the whole producer warp after lane 0 announced the bytes.
-template <int FMT>
-MOE_DEV void stage_tile(const Bank& bk, long row_a, long row_b, uint8_t* stage, const StageLayout& L, uint64_t* bar,
-                        uint64_t policy, int lane) {
-  const int K = bk.K;
-  const int srow = scale_row_bytes(FMT, K);
-  const uint8_t* scales = static_cast<const uint8_t*>(bk.scales);
-  if (lane < 16) {
-    const long r = lane < 8 ? row_a + lane : row_b + lane - 8;
-    bulk_g2s_hint(stage + lane * L.crow, bk.codes + r * (K / 2), uint32_t(K / 2), bar, policy);
-  } else if (lane == 16) {
-    const int n = row_b == row_a + 8 ? 16 : 8;
-    bulk_g2s_hint(stage + L.cbytes, scales + row_a * srow, uint32_t(n * srow), bar, policy);
-  } else if (lane == 17 && row_b != row_a + 8) {
-    bulk_g2s_hint(stage + L.cbytes + 8 * srow, scales + row_b * srow, uint32_t(8 * srow), bar, policy);
-  }
-}
-
 // ---------------------------------------------------------------------------
-// gate_up + SwiGLU.  Work unit u = (touched slot u / (I/8), features
-// f0 = 8 (u % (I/8)) .. f0 + 7): its 16 weight rows are the 8 gate rows f0..
-// and the 8 matching up rows I + f0.., staged as one 16-row tile (gate rows
-// 0-7, up rows 8-15), so the MMA's C fragment holds gate (c0, c1) and up
-// (c2, c3) of the same feature and token: SwiGLU needs no shuffle.  CTA c
-// takes units [c n / grid, (c + 1) n / grid); its i-th goes to stage i % S and
-// consumer group i % G.  The group's four warps split K (128-k blocks w,
-// w + 4, ...), and one of them (rotating) sums the four partial tiles in warp
-// order and writes a = bf16(silu(gate) * up) to act[p][f] for the expert's
-// sorted rows p.  With X_SMEM (small T) the consumers first stage the T token
-// rows in fragment order.
+// gate_up + SwiGLU.  Work unit u = (touched slot u / (I/16), features
+// f0 = 16 (u % (I/16)) .. f0 + 15): its 32 weight rows are the 16 gate rows
+// f0.. and the 16 matching up rows I + f0.., staged as two runs.  Lane g of
+// MMA tile t (features f0 + 8t ..) takes feature f0 + 8t + g's gate row and up
+// row as its two MMA rows (low / high; swapped for odd g), so the C fragment
+// holds gate and up of the same feature and token: SwiGLU needs no shuffle.
+// CTA c takes units [c n / grid, (c + 1) n / grid); its i-th goes to stage
+// i % S and consumer group i % G.  The group's four warps split K (128-k
+// blocks w, w + 4, ...), and one of them (rotating) sums the four partial
+// tiles in warp order and writes a = bf16(silu(gate) * up) to act[p][f] for
+// the expert's sorted rows p.  With X_SMEM (small T) the consumers first
+// stage the T token rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
@@ -172,16 +170,16 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
     uint16_t* __restrict__ act, uint32_t* status, int S) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int G = kGuGroups;
-  constexpr int CH = NT == 1 ? 4 : 2;  // accumulator chains per token tile
+  constexpr int G = kGuGroups, MT = kGuMT, CH = 2;
+  constexpr int kRed = kGroupWarps * NT * MT * 128;  // floats of one group's partial tiles
   const int K = gu.K, R = T * top_k;
-  const StageLayout L = stage_layout(FMT, K, 16);
+  const GuLayout L = gu_layout(FMT, K);
   const int srow = scale_row_bytes(FMT, K);
   const int pstride = staged_act_stride(K);
   uint8_t* ring = smem;                                                      // [S][stage]
   uint8_t* x_s = ring + size_t(S) * L.stage_bytes;                           // [T][pstride] (X_SMEM)
-  float* red = reinterpret_cast<float*>(x_s + (X_SMEM ? size_t(T) * pstride : 0));  // [G][2][4][NT][4][32]
-  int* s_touched = reinterpret_cast<int*>(red + G * 2 * kGroupWarps * NT * 128);
+  float* red = reinterpret_cast<float*>(x_s + (X_SMEM ? size_t(T) * pstride : 0));  // [G][2][kRed]
+  int* s_touched = reinterpret_cast<int*>(red + G * 2 * kRed);
   int* s_off = s_touched + (E + 1);
   int* s_tok = s_off + (E + 1);                                              // [R] token of sorted row p
   uint64_t* full = align8<uint64_t>(s_tok + R);
@@ -206,7 +204,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
   int t_lo, t_hi;
   local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
-  const int ftiles = I / 8;
+  const int ftiles = I / kGuFeat;
   const int n_units = (t_hi - t_lo) * ftiles;
   const int u_begin = int(long(n_units) * blockIdx.x / gridDim.x);
   const int cnt = int(long(n_units) * (blockIdx.x + 1) / gridDim.x) - u_begin;
@@ -215,22 +213,27 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
     const uint64_t policy = l2_policy_evict_first();
-    const uint32_t tx = staged_bytes<FMT>(gu, 16);
-    int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;          // unit i
+    const uint32_t run = uint32_t(kGuFeat * (K / 2)), srun = uint32_t(kGuFeat * srow);
+    const uint8_t* scales = static_cast<const uint8_t*>(gu.scales);
+    int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;                 // unit i
     int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
     int i = 0, st = 0, ph = 0;  // unit i's stage and that stage's use count parity
     for (; i < cnt; ++i) {
       if (i >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &s_abort, status))) break;
-      const long row_g = long(s_local[slot] - e_lo) * gu.N + ft * 8;
       fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], tx);
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * run + 2 * srun);
       __syncwarp();
-      stage_tile<FMT>(gu, row_g, row_g + I, ring + size_t(st) * L.stage_bytes, L, &full[st], policy, lane);
-      if (lane >= 18 && lane < 22 && i + S < cnt) {
+      if (lane < 4) {
+        // lane 0 / 1: gate / up codes; lane 2 / 3: their scales
+        const long row = long(s_local[slot] - e_lo) * gu.N + ft * kGuFeat + ((lane & 1) ? I : 0);
+        uint8_t* stage = ring + size_t(st) * L.stage_bytes;
+        if (lane < 2) bulk_g2s_hint(stage + (lane ? L.cB : L.cA), gu.codes + row * (K / 2), run, &full[st], policy);
+        else bulk_g2s_hint(stage + (lane & 1 ? L.sB : L.sA), scales + row * srow, srun, &full[st], policy);
+      } else if (lane < 8 && i + S < cnt) {
         // the unit that will refill this stage, into L2 ahead of time
-        const long rn = long(s_local[pslot] - e_lo) * gu.N + pft * 8 + ((lane & 1) ? I : 0);
-        if (lane < 20) prefetch_codes<FMT>(gu, rn, 8);
-        else prefetch_scales<FMT>(gu, rn, 8);
+        const long row = long(s_local[pslot] - e_lo) * gu.N + pft * kGuFeat + ((lane & 1) ? I : 0);
+        if (lane < 6) prefetch_codes<FMT>(gu, row, kGuFeat);
+        else prefetch_scales<FMT>(gu, row, kGuFeat);
       }
       if (++st == S) st = 0, ph ^= 1;
       if (++ft == ftiles) ft = 0, ++slot;
@@ -244,6 +247,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
   constexpr int kConsumers = G * kGroupWarps * 32;
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
+  const bool odd = (g & 1) != 0;  // this lane's low MMA row is the up row
   if (X_SMEM) {
     stage_act_rows<1>(x_s, x, T, K, threadIdx.x, kConsumers);
     named_barrier_sync(1, kConsumers);
@@ -251,6 +255,8 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
   const int nfull = K / 128;  // blocks where every lane slice lies inside K
   const int my_full = wj < nfull ? (nfull - wj + kGroupWarps - 1) / kGroupWarps : 0;
   const int tail_b = ((K % 128) != 0 && nfull % kGroupWarps == wj) ? nfull : -1;
+  const int lo_c = odd ? L.cB : L.cA, hi_c = odd ? L.cA : L.cB;
+  const int lo_s = odd ? L.sB : L.sA, hi_s = odd ? L.sA : L.sB;
   int slot = (u_begin + grp) / ftiles, ft = (u_begin + grp) - slot * ftiles;
   int st = grp, ph = 0;
   for (int i = grp, n = 0; i < cnt; i += G, ++n) {
@@ -258,12 +264,20 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, &s_abort, status));
     const int e = s_local[slot];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-    const int f0 = ft * 8;
+    const int f0 = ft * kGuFeat;
     const uint8_t* s_c = ring + size_t(st) * L.stage_bytes;
-    const uint8_t* c_gate = s_c + g * L.crow + 16 * q;   // rows g (gate) and g + 8 (up), lane slice
-    const uint8_t* c_up = c_gate + 8 * L.crow;
-    const uint8_t* sc_gate = s_c + L.cbytes + g * srow;
-    const uint8_t* sc_up = sc_gate + 8 * srow;
+    const uint8_t* c_lo[MT];
+    const uint8_t* c_hi[MT];
+    const uint8_t* sc_lo[MT];
+    const uint8_t* sc_hi[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int fi = 8 * t + g;
+      c_lo[t] = s_c + lo_c + fi * (K / 2) + 16 * q;
+      c_hi[t] = s_c + hi_c + fi * (K / 2) + 16 * q;
+      sc_lo[t] = s_c + lo_s + fi * srow;
+      sc_hi[t] = s_c + hi_s + fi * srow;
+    }
     const float gsc = FMT == MOE_FMT_NVFP4_G16 ? gu.gscale[e - e_lo] : 0.f;
     const int ntiles = min(NT, (n_e + 7) / 8);
     XFrags<NT, X_SMEM> xf;
@@ -278,45 +292,56 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
       const int c = 8 * j + g;
       xf.tok[j] = s_tok[p0 + (c < n_e ? c : 0)];
     }
-    float acc2[NT][CH][4];
+    float acc[NT][MT][CH][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int h = 0; h < CH; ++h)
+      for (int t = 0; t < MT; ++t)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc2[j][h][c] = 0.f;
-    if (ok) warp_tile<FMT, NT, CH>(acc2, c_gate, c_up, sc_gate, sc_up, wj, kGroupWarps, my_full, tail_b, K, q, gsc,
-                                   ntiles, xf);
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[j][t][h][c] = 0.f;
+    // blocks four at a time (fewer with more token tiles: registers)
+    constexpr int UNB = NT == 1 ? 4 : NT == 2 ? 2 : 1;
+    if (ok)
+      smem_unit<FMT, NT, MT, CH, UNB>(acc, c_lo, c_hi, sc_lo, sc_hi, wj, kGroupWarps, my_full, tail_b, K, q, gsc, ntiles,
+                                      xf);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
     // the group's partial tiles, double-buffered by unit parity
-    float* red_u = red + size_t((grp * 2 + (n & 1)) * kGroupWarps) * NT * 128;
+    float* red_u = red + size_t(grp * 2 + (n & 1)) * kRed;
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v = acc2[j][0][c];
+      for (int t = 0; t < MT; ++t)
 #pragma unroll
-        for (int h = 1; h < CH; ++h) v += acc2[j][h][c];
-        red_u[((wj * NT + j) * 4 + c) * 32 + lane] = v;
-      }
+        for (int c = 0; c < 4; ++c) {
+          float v = acc[j][t][0][c];
+#pragma unroll
+          for (int h = 1; h < CH; ++h) v += acc[j][t][h][c];
+          red_u[(((wj * NT + j) * MT + t) * 4 + c) * 32 + lane] = v;
+        }
     named_barrier_sync(2 + grp, kGroupWarps * 32);
     if (ok && wj == n % kGroupWarps) {
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         if (j >= ntiles) break;
-        float sum[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          sum[c] = 0.f;
+        for (int t = 0; t < MT; ++t) {
+          float sum[4];
 #pragma unroll
-          for (int w = 0; w < kGroupWarps; ++w) sum[c] += red_u[((w * NT + j) * 4 + c) * 32 + lane];
-        }
-        // c0, c1: gate of feature f0+g at columns 2q, 2q+1; c2, c3: up of the same
+          for (int c = 0; c < 4; ++c) {
+            sum[c] = 0.f;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int col = 8 * j + 2 * q + hh;
-          if (col < n_e) act[size_t(p0 + col) * I + f0 + g] = f32_to_bf16_rn(silu_mul(sum[hh], sum[2 + hh]));
+            for (int w = 0; w < kGroupWarps; ++w) sum[c] += red_u[(((w * NT + j) * MT + t) * 4 + c) * 32 + lane];
+          }
+          // c0, c1: low row at columns 2q, 2q+1; c2, c3: high row (gate low for even g)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int col = 8 * j + 2 * q + hh;
+            const float gate = odd ? sum[2 + hh] : sum[hh], up = odd ? sum[hh] : sum[2 + hh];
+            if (col < n_e) act[size_t(p0 + col) * I + f0 + 8 * t + g] = f32_to_bf16_rn(silu_mul(gate, up));
+          }
         }
       }
     }
@@ -330,54 +355,44 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
 // ---------------------------------------------------------------------------
 // down projection and combine.  CTA c owns the 16 output features of tiles
 // c, c + grid, ... (H / 16 tiles).  For a tile, work unit s = the tile's 16
-// rows of the down matrix of touched expert s (all of K = I), taken by
-// consumer warp s % W; its C fragment times the routing weight of each
-// column's (token, slot) goes to ybuf[t k + j][f] in shared memory.  When the
-// tile's units are done, each token's output is the sum of its k slots in
-// slot order (plus the shared expert's gated output), rounded once to bf16,
-// or the fp32 sum (an expert-parallel shard's partial: slots of other shards'
-// experts stay zero).  The weights do not depend on the gate_up kernel that
-// runs just before: the producer reads the routing state (written two
-// launches back, and the kernel in between triggers its dependents only after
-// its own wait) and starts the weight copies before the programmatic-launch
-// wait; only the consumers wait.  With ACT_SMEM (small T) the consumers first
-// stage the T*k activation rows in fragment order.
+// rows of the down matrix of touched expert s (all of K = I), taken by warp
+// s % W, in chunks of four 128-k blocks loaded into registers; the next
+// chunk's loads are issued before the current chunk is multiplied.  The
+// unit's C fragment times the routing weight of each column's (token, slot)
+// goes to ybuf[t k + j][f] in shared memory.  When the tile's units are
+// done, each token's output is the sum of its k slots in slot order (plus
+// the shared expert's gated output), rounded once to bf16, or the fp32 sum
+// (an expert-parallel shard's partial: slots of other shards' experts stay
+// zero).  The weights do not depend on the gate_up kernel that runs just
+// before: the routing state was written two launches back (and the kernel in
+// between triggers its dependents only after its own wait), so every warp
+// requests its tiles into L2 and loads its first chunk before the
+// programmatic-launch wait.  With ACT_SMEM (small T) the warps then stage the
+// T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool ACT_SMEM>
 __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
     const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
-    uint16_t* __restrict__ out, float* __restrict__ partial_out, uint32_t* status, int S) {
+    uint16_t* __restrict__ out, float* __restrict__ partial_out) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = kDnWarps;
   constexpr int CH = NT == 1 ? 4 : 2;
   const int H = dn.N, K = dn.K;  // K = I
   const int R = T * top_k;
-  const StageLayout L = stage_layout(FMT, K, kDnRows);
   const int srow = scale_row_bytes(FMT, K);
   const int pstride = staged_act_stride(K);
-  uint8_t* ring = smem;                                           // [S][stage]
-  uint8_t* act_s = ring + size_t(S) * L.stage_bytes;              // [R][pstride] (ACT_SMEM)
+  uint8_t* act_s = smem;                                          // [R][pstride] (ACT_SMEM)
   float* ybuf = reinterpret_cast<float*>(act_s + (ACT_SMEM ? size_t(R) * pstride : 0));  // [R][16]
   int* s_touched = reinterpret_cast<int*>(ybuf + R * kDnRows);
   int* s_off = s_touched + (E + 1);
   int* s_slot = s_off + (E + 1);                                  // [R] slot t k + j of sorted row p
   float* s_w = reinterpret_cast<float*>(s_slot + R);              // [R] its routing weight
-  uint64_t* full = align8<uint64_t>(s_w + R);
-  uint64_t* empty = full + S;
-  __shared__ volatile int s_abort;
   __shared__ int s_cnt[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    s_abort = 0;
-    for (int st = 0; st < S; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], 1);
-    }
-    fence_mbar_init();
-  }
+  const int g = lane >> 2, q = lane & 3;
   // routing state: written two launches back (see above), read through L2
   load_routing(s_touched, s_off, touched, offsets, E);
   for (int p = threadIdx.x; p < R; p += blockDim.x) {
@@ -392,68 +407,52 @@ __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
   const int n_t = t_hi - t_lo;
   const int ntile = H / kDnRows;
-
-  if (warp == W) {
-    // ---------------------------------------------------------------- producer
-    if (n_t > 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      const uint32_t tx = staged_bytes<FMT>(dn, kDnRows);
-      int ptile = blockIdx.x, ps = 0;  // unit i + S
-      for (int a = 0; a < S; ++a)
-        if (++ps == n_t) ps = 0, ptile += gridDim.x;
-      int i = 0, st = 0, ph = 0;
-      bool run = true;
-      for (int tile = blockIdx.x; run && tile < ntile; tile += gridDim.x) {
-        for (int s = 0; s < n_t; ++s, ++i) {
-          if (i >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &s_abort, status))) {
-            run = false;
-            break;
-          }
-          const long row0 = long(s_local[s] - e_lo) * H + tile * kDnRows;
-          fence_proxy_async_smem();
-          if (lane == 0) mbar_arrive_expect_tx(&full[st], tx);
-          __syncwarp();
-          stage_tile<FMT>(dn, row0, row0 + 8, ring + size_t(st) * L.stage_bytes, L, &full[st], policy, lane);
-          if (lane >= 18 && lane < 20 && ptile < ntile) {
-            // the unit that will refill this stage, into L2 ahead of time
-            const long rn = long(s_local[ps] - e_lo) * H + ptile * kDnRows;
-            if (lane == 18) prefetch_codes<FMT>(dn, rn, kDnRows);
-            else prefetch_scales<FMT>(dn, rn, kDnRows);
-          }
-          if (++st == S) st = 0, ph ^= 1;
-          if (++ps == n_t) ps = 0, ptile += gridDim.x;
-        }
-      }
-      if (lane == 0) drain_stages(full, i, S);
-    }
-    pdl_wait();
-    pdl_trigger();
-    return;
+  const int nblk = kblocks(K), nch = (nblk + 3) / 4;  // k-blocks and chunks of four per unit
+  const uint8_t* scales = static_cast<const uint8_t*>(dn.scales);
+  const int my_units = warp < n_t ? (n_t - warp + W - 1) / W : 0;  // per tile
+  const int nk = my_units * nch;                                   // chunks per tile
+  // the lane's two rows of unit m's tile, codes (+ slice offset) and scales
+  auto rows_of = [&](int tile, int m, const uint8_t*& c_lo, const uint8_t*& s_lo) {
+    const long r = long(s_local[warp + W * m] - e_lo) * H + tile * kDnRows + g;
+    c_lo = dn.codes + r * (K / 2) + 16 * q;
+    s_lo = scales + r * srow;
+  };
+  auto load = [&](RegChunk& c, int tile, int k) {
+    const int m = k / nch, ch = k - m * nch;
+    const uint8_t *c_lo, *s_lo;
+    rows_of(tile, m, c_lo, s_lo);
+    load_chunk<FMT>(c, c_lo, c_lo + 8 * (K / 2), s_lo, s_lo + 8 * srow, 4 * ch, nblk, K, q);
+  };
+  if (lane < my_units && blockIdx.x < ntile) {
+    // all of this warp's tiles of the CTA's first tile into L2
+    const long r0 = long(s_local[warp + W * lane] - e_lo) * H + blockIdx.x * kDnRows;
+    prefetch_codes<FMT>(dn, r0, kDnRows);
+    prefetch_scales<FMT>(dn, r0, kDnRows);
   }
+  RegChunk cA, cB;
+  if (nk > 0 && blockIdx.x < ntile) load(cA, blockIdx.x, 0);
 
-  // -------------------------------------------------------------------- consumers
-  constexpr int kConsumers = W * 32;
   pdl_wait();  // the activations (and the previous readers of the output) of the kernels before
   pdl_trigger();
-  const int g = lane >> 2, q = lane & 3;
-  if (ACT_SMEM) stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kConsumers);
-  named_barrier_sync(1, kConsumers);
-  const int nfull = K / 128;
-  const int tail_b = (K % 128) != 0 ? nfull : -1;
-  int ti = 0;
-  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x, ++ti) {
-    for (int s = warp; s < n_t; s += W) {
-      const int idx = ti * n_t + s;  // the CTA's unit index
-      const int st = idx % S;
-      // warp-uniform: the MMAs below run only if every lane saw the data land
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (idx / S) & 1, &s_abort, status));
-      const int e = s_local[s];
+  if (ACT_SMEM) {
+    stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kDnThreads);
+    __syncthreads();
+  }
+  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+    if (tile != int(blockIdx.x) && nk > 0) load(cA, tile, 0);
+    float acc[NT][CH][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int h = 0; h < CH; ++h)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
+    // multiply chunk k (in `cur`); after a unit's last chunk, its weighted
+    // outputs go to ybuf and the accumulators restart
+    auto step = [&](const RegChunk& cur, int k) {
+      const int m = k / nch, ch = k - m * nch;
+      const int e = s_local[warp + W * m];
       const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-      const uint8_t* s_c = ring + size_t(st) * L.stage_bytes;
-      const uint8_t* c_lo = s_c + g * L.crow + 16 * q;
-      const uint8_t* c_hi = c_lo + 8 * L.crow;
-      const uint8_t* sc_lo = s_c + L.cbytes + g * srow;
-      const uint8_t* sc_hi = sc_lo + 8 * srow;
       const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
       const int ntiles = min(NT, (n_e + 7) / 8);
       ActFrags<ACT_SMEM> af;
@@ -465,36 +464,38 @@ __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
       af.g = g;
       af.p0 = p0;
       af.n_e = n_e;
-      float acc2[NT][CH][4];
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int h = 0; h < CH; ++h)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc2[j][h][c] = 0.f;
-      if (ok) warp_tile<FMT, NT, CH>(acc2, c_lo, c_hi, sc_lo, sc_hi, 0, 1, nfull, tail_b, K, q, gsc, ntiles, af);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      if (!ok) continue;
+      chunk_mma<FMT, NT, CH>(acc, cur, 4 * ch, nblk, K, q, gsc, ntiles, af);
+      if (ch != nch - 1) return;
       // c0, c1: feature g at columns 2q, 2q+1; c2, c3: feature g + 8
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        if (j >= ntiles) break;
+        if (j < ntiles) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = 8 * j + 2 * q + (c & 1);
-          if (col < n_e) {
-            float v = acc2[j][0][c];
+          for (int c = 0; c < 4; ++c) {
+            const int col = 8 * j + 2 * q + (c & 1);
+            float v = acc[j][0][c];
 #pragma unroll
-            for (int h = 1; h < CH; ++h) v += acc2[j][h][c];
-            ybuf[s_slot[p0 + col] * kDnRows + g + 8 * (c >> 1)] = s_w[p0 + col] * v;
+            for (int h = 1; h < CH; ++h) v += acc[j][h][c];
+            if (col < n_e) ybuf[s_slot[p0 + col] * kDnRows + g + 8 * (c >> 1)] = s_w[p0 + col] * v;
           }
         }
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
       }
+    };
+    for (int k = 0; k < nk;) {
+      if (k + 1 < nk) load(cB, tile, k + 1);
+      step(cA, k);
+      if (++k >= nk) break;
+      if (k + 1 < nk) load(cA, tile, k + 1);
+      step(cB, k);
+      ++k;
     }
-    named_barrier_sync(1, kConsumers);
+    __syncthreads();
     // each token's k slots summed in slot order, two features per thread
-    for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kConsumers) {
+    for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kDnThreads) {
       const int t = o / (kDnRows / 2), f = 2 * (o % (kDnRows / 2));
       float v0 = 0.f, v1 = 0.f;
       for (int j = 0; j < top_k; ++j) {
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
         *reinterpret_cast<uint32_t*>(out + oi) = pack_bf16x2(v0, v1);
       }
     }
-    named_barrier_sync(1, kConsumers);
+    __syncthreads();
   }
 }
 
@@ -525,24 +526,21 @@ int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
 constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving room for static
 // Staged token rows (gate_up) and activation rows (down) up to these sizes.
 constexpr size_t kMaxStagedX = 72 * 1024;
-constexpr size_t kMaxStagedAct = 72 * 1024;
+constexpr size_t kMaxStagedAct = 160 * 1024;
 
 int nt_of(int T) { return T <= 8 ? 1 : T <= 16 ? 2 : 4; }
 
 // gate_up: stages + staged token rows + the partial-tile buffers + routing
 // state + barriers
 size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows, int S) {
-  const StageLayout L = stage_layout(fmt, K, 16);
-  return size_t(S) * L.stage_bytes + size_t(x_rows) * staged_act_stride(K) +
-         size_t(kGuGroups) * 2 * kGroupWarps * NT * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 + 2 * size_t(S) * 8;
+  return size_t(S) * gu_layout(fmt, K).stage_bytes + size_t(x_rows) * staged_act_stride(K) +
+         size_t(kGuGroups) * 2 * kGroupWarps * NT * kGuMT * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 +
+         2 * size_t(S) * 8;
 }
 
-// down: stages + staged activation rows + the slot outputs + routing state +
-// barriers
-size_t down_smem(int fmt, int K, int E, int R, int act_rows, int S) {
-  const StageLayout L = stage_layout(fmt, K, kDnRows);
-  return size_t(S) * L.stage_bytes + size_t(act_rows) * staged_act_stride(K) + size_t(R) * kDnRows * 4 +
-         size_t(2 * (E + 1) + 2 * R) * 4 + 8 + 2 * size_t(S) * 8;
+// down: staged activation rows + the slot outputs + routing state
+size_t down_smem(int E, int R, int K, int act_rows) {
+  return size_t(act_rows) * staged_act_stride(K) + size_t(R) * kDnRows * 4 + size_t(2 * (E + 1) + 2 * R) * 4;
 }
 
 struct GuPlan {
@@ -552,7 +550,6 @@ struct GuPlan {
 };
 struct DnPlan {
   bool act_smem;
-  int S;
   size_t smem;
 };
 
@@ -579,16 +576,7 @@ DnPlan down_plan(const moe_shape_t& s, int T) {
   const int R = T * s.top_k;
   DnPlan p;
   p.act_smem = size_t(R) * staged_act_stride(s.inter) <= kMaxStagedAct;
-  p.S = 0;
-  p.smem = 0;
-  for (int S = kDnMaxStages / kDnWarps * kDnWarps; S >= kDnWarps; S -= kDnWarps) {
-    const size_t b = down_smem(s.fmt, s.inter, s.num_experts, R, p.act_smem ? R : 0, S);
-    if (b <= kMaxSmemPerCta) {
-      p.S = S;
-      p.smem = b;
-      break;
-    }
-  }
+  p.smem = down_smem(s.num_experts, R, s.inter, p.act_smem ? R : 0);
   return p;
 }
 
@@ -668,15 +656,14 @@ template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
                     const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out, cudaStream_t stream) {
   const DnPlan p = down_plan(s, T);
-  if (p.S == 0) return cudaErrorInvalidConfiguration;
+  if (p.smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
   auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
   cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, kDnThreads);
   return launch_pdl(k, dim3(grid), dim3(kDnThreads), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
-                    (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out, ws.status,
-                    p.S);
+                    (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out);
 }
 
 template <int FMT>
@@ -692,12 +679,12 @@ cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRa
 
 bool decode_supported(const moe_shape_t& s, int T) {
   if (T > kDecodeMaxT) return false;
-  return gate_up_plan(s, T).S > 0 && down_plan(s, T).S > 0;
+  return gate_up_plan(s, T).S > 0 && down_plan(s, T).smem <= kMaxSmemPerCta;
 }
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
-  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / 8);
+  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / kGuFeat);
   if (units <= 0) return cudaSuccess;
   if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, er, ws, units, stream);
   if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, er, ws, units, stream);

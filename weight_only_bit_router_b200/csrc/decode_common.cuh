@@ -27,9 +27,13 @@
 // made once per warp and work unit, so the inner loop has no branches.
 //
 // Shared-memory layouts.
-//  * Weight rows: each staged row starts (K/2 rounded up to 128) + 64 bytes
-//    after the previous one, so the rows g and g + 1 that one 8-lane phase of
-//    a 16-byte load reads lie in opposite halves of the 32 banks.
+//  * Weight tiles (gate_up): the 16 gate rows of a unit, then 64 bytes of
+//    padding, then its 16 up rows, each run one bulk copy.  A 16-byte load of
+//    rows g and g + 1 by one 8-lane phase would hit the same bank half when
+//    both rows sit in one run (rows are a multiple of 128 bytes long); lanes
+//    with odd g therefore take the up row as their low MMA row and the gate
+//    row as their high one, so the two rows of a phase are in different runs,
+//    64 bytes apart modulo 128.
 //  * Activation rows in fragment order: row r, k-block b starts at
 //    r * pstride + 256 b, and its 16-byte unit 4 i + q holds lane slice q's
 //    fragment words of MMA steps 2i and 2i+1, so a lane's 16 fragment words
@@ -89,10 +93,30 @@ struct Mult {
   uint32_t m0, m1, m2;
 };
 
-// Multipliers of block b from the row's staged scales; `fast` is cleared when
-// the single-instruction path is not exact for them.
+// The raw scale bits of one lane slice of one weight row at k-block b: INT4
+// the bf16 scale of group b, MXFP4 the exponent byte of 32-element block
+// 4b + q, NVFP4 the two E4M3 bytes of 16-element blocks 8b + 2q, 8b + 2q + 1.
+// `row` points at the row's scales in shared memory, or in global memory
+// (read-only for the kernel's lifetime) with GLOBAL.
+template <int FMT, bool GLOBAL>
+MOE_DEV uint32_t raw_scale(const uint8_t* row, int b, int q) {
+  if (FMT == MOE_FMT_INT4_G128) {
+    const uint16_t* p = reinterpret_cast<const uint16_t*>(row) + b;
+    return GLOBAL ? __ldg(p) : *p;
+  }
+  if (FMT == MOE_FMT_NVFP4_G16) {
+    const uint16_t* p = reinterpret_cast<const uint16_t*>(row + 8 * b + 2 * q);
+    return GLOBAL ? __ldg(p) : *p;
+  }
+  const uint8_t* p = row + 4 * b + q;
+  return GLOBAL ? __ldg(p) : *p;
+}
+
+// Multipliers from raw scale bits; `fast` is cleared when the
+// single-instruction path is not exact for them.  A slice outside the row
+// (`in` false) gets zero weights.
 template <int FMT>
-MOE_DEV Mult mult_at(const uint8_t* scales, int b, int q, float gsc, bool in, bool& fast) {
+MOE_DEV Mult mult_of(uint32_t raw, float gsc, bool in, bool& fast) {
   Mult m;
   if (!in) {
     // zero weights on both paths (INT4's two-step multiplier m0 - C is 0)
@@ -101,18 +125,16 @@ MOE_DEV Mult mult_at(const uint8_t* scales, int b, int q, float gsc, bool in, bo
     return m;
   }
   if (FMT == MOE_FMT_INT4_G128) {
-    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[b];  // group b = k-block b
-    const uint32_t sd = s * 0x00010001u;
+    const uint32_t sd = raw * 0x00010001u;
     m.m0 = sd + 0x42804280u;  // exponent + 133
     m.m1 = sd + 0x40804080u;  // exponent + 129
     m.m2 = sd + 0x81808180u;  // exponent + 3, sign set: -8 s
-    fast = fast && (s - 0x0080u < 0x3D00u - 0x0080u);
+    fast = fast && (raw - 0x0080u < 0x3D00u - 0x0080u);
   } else if (FMT == MOE_FMT_NVFP4_G16) {
-    // the slice holds two 16-element blocks: 8b + 2q and 8b + 2q + 1
-    nv_mult_pair_scaled(scales + 8 * b + 2 * q, gsc, m.m0, m.m1, m.m2);
+    nv_mult_pair_scaled_v(uint16_t(raw), gsc, m.m0, m.m1, m.m2);
     fast = fast && m.m2 == 0u;
   } else {
-    mx_mult(int(scales[4 * b + q]) - 127, m.m0, m.m2);  // the slice is one 32-element block
+    mx_mult(int(raw) - 127, m.m0, m.m2);
     m.m1 = m.m0;
     fast = fast && m.m2 == 0u;
   }
@@ -242,98 +264,133 @@ MOE_DEV void stage_act_rows(uint8_t* dst, const uint16_t* src, int rows, int K, 
   }
 }
 
-// Shared-memory layout of one stage of `rows` weight rows: codes at the
-// padded row stride crow, then the rows' scales (contiguous, padded to 16).
-struct StageLayout {
-  int crow, cbytes, sbytes, stage_bytes;
-};
-
-__host__ __device__ inline StageLayout stage_layout(int fmt, int K, int rows) {
-  StageLayout l;
-  l.crow = (((K / 2) + 127) & ~127) + 64;
-  l.cbytes = rows * l.crow;
-  l.sbytes = rows * scale_row_bytes(fmt, K);
-  l.stage_bytes = l.cbytes + ((l.sbytes + 15) & ~15);
-  return l;
-}
-
-// One warp, one 16-row weight tile staged at c_lo (row r = lane/4; the tile's
-// row r + 8 at c_hi) with scales at sc_lo / sc_hi: acc[j] += W x B_j over the
-// NB k-blocks b0, b0 + bstep, ... (all inside K), for the token tiles
-// j < ntiles.  `act.load(j, b, in, frags)` gives token tile j's fragments of
-// block b.  CH accumulator chains per token tile (2 or 4).
-template <int FMT, int NT, int CH, int NB, bool FAST, typename Act>
-MOE_DEV void tile_run(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const Mult (&mlo)[NB],
-                      const Mult (&mhi)[NB], int b0, int bstep, int ntiles, const Act& act) {
+// One warp: acc[j][t] += W_t x B_j over NB k-blocks b0, b0 + bstep, ... of
+// MT 16-row weight tiles whose codes sit in shared memory (tile t: the lane's
+// row at c_lo[t], its row + 8 at c_hi[t], scales at s_lo[t] / s_hi[t]), for
+// the token tiles j < ntiles.  `act.load(j, b, in, frags)` gives token tile
+// j's fragments of block b.  With `partial` (NB = 1) the block may end inside
+// K: lane slices past K contribute zero.  The fast / two-step choice is made
+// once for all NB blocks; CH accumulator chains per tile (blocks alternate
+// between chain pairs when CH = 4).
+template <int FMT, int NT, int MT, int CH, int NB, typename Act>
+MOE_DEV void smem_blocks(float (&acc)[NT][MT][CH][4], const uint8_t* const (&c_lo)[MT],
+                         const uint8_t* const (&c_hi)[MT], const uint8_t* const (&s_lo)[MT],
+                         const uint8_t* const (&s_hi)[MT], int b0, int bstep, int K, int q, float gsc, int ntiles,
+                         bool partial, const Act& act) {
+  Mult mlo[MT][NB], mhi[MT][NB];
+  bool fast = true;
 #pragma unroll
   for (int i = 0; i < NB; ++i) {
     const int b = b0 + i * bstep;
-    const uint4 lo = *reinterpret_cast<const uint4*>(c_lo + 64 * b);
-    const uint4 hi = *reinterpret_cast<const uint4*>(c_hi + 64 * b);
+    const bool in = !partial || 128 * b + 32 * q < K;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      mlo[t][i] = mult_of<FMT>(in ? raw_scale<FMT, false>(s_lo[t], b, q) : 0u, gsc, in, fast);
+      mhi[t][i] = mult_of<FMT>(in ? raw_scale<FMT, false>(s_hi[t], b, q) : 0u, gsc, in, fast);
+    }
+  }
+  // warp-uniform: mma.sync needs the whole warp on one path (the two-step
+  // path is exact for every scale)
+  const bool all_fast = __all_sync(0xffffffffu, fast);
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    const int b = b0 + i * bstep;
+    const bool in = !partial || 128 * b + 32 * q < K;
+    uint4 lo[MT], hi[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      lo[t] = in ? *reinterpret_cast<const uint4*>(c_lo[t] + 64 * b) : make_uint4(0, 0, 0, 0);
+      hi[t] = in ? *reinterpret_cast<const uint4*>(c_hi[t] + 64 * b) : make_uint4(0, 0, 0, 0);
+    }
     const int c0 = CH == 4 ? 2 * (i & 1) : 0;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       if (j > 0 && j >= ntiles) break;
       uint32_t bf[8][2];
-      act.load(j, b, true, bf);
-      mma_kblock<FMT, FAST, CH>(acc[j], c0, lo, hi, mlo[i], mhi[i], bf);
+      act.load(j, b, in, bf);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        if (all_fast) mma_kblock<FMT, true, CH>(acc[j][t], c0, lo[t], hi[t], mlo[t][i], mhi[t][i], bf);
+        else mma_kblock<FMT, false, CH>(acc[j][t], c0, lo[t], hi[t], mlo[t][i], mhi[t][i], bf);
+      }
     }
   }
 }
 
-// tile_run with the fast / two-step choice made once for all NB blocks.
-template <int FMT, int NT, int CH, int NB, typename Act>
-MOE_DEV void tile_blocks(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
-                         const uint8_t* sc_hi, int b0, int bstep, int q, float gsc, int ntiles, const Act& act) {
-  Mult mlo[NB], mhi[NB];
-  bool fast = true;
-#pragma unroll
-  for (int i = 0; i < NB; ++i) {
-    mlo[i] = mult_at<FMT>(sc_lo, b0 + i * bstep, q, gsc, true, fast);
-    mhi[i] = mult_at<FMT>(sc_hi, b0 + i * bstep, q, gsc, true, fast);
-  }
-  // warp-uniform: mma.sync needs the whole warp on one path (the two-step
-  // path is exact for every scale)
-  if (__all_sync(0xffffffffu, fast)) tile_run<FMT, NT, CH, NB, true>(acc, c_lo, c_hi, mlo, mhi, b0, bstep, ntiles, act);
-  else tile_run<FMT, NT, CH, NB, false>(acc, c_lo, c_hi, mlo, mhi, b0, bstep, ntiles, act);
+// One warp's share of a unit staged in shared memory: the nb full k-blocks
+// b0, b0 + bstep, ... (UNB at a time where possible) and, if tail_b >= 0,
+// the partial block tail_b.
+template <int FMT, int NT, int MT, int CH, int UNB, typename Act>
+MOE_DEV void smem_unit(float (&acc)[NT][MT][CH][4], const uint8_t* const (&c_lo)[MT], const uint8_t* const (&c_hi)[MT],
+                       const uint8_t* const (&s_lo)[MT], const uint8_t* const (&s_hi)[MT], int b0, int bstep, int nb,
+                       int tail_b, int K, int q, float gsc, int ntiles, const Act& act) {
+  int i = 0;
+  for (; i + UNB <= nb; i += UNB)
+    smem_blocks<FMT, NT, MT, CH, UNB>(acc, c_lo, c_hi, s_lo, s_hi, b0 + i * bstep, bstep, K, q, gsc, ntiles, false,
+                                      act);
+  for (; i < nb; ++i)
+    smem_blocks<FMT, NT, MT, CH, 1>(acc, c_lo, c_hi, s_lo, s_hi, b0 + i * bstep, bstep, K, q, gsc, ntiles, false, act);
+  if (tail_b >= 0)
+    smem_blocks<FMT, NT, MT, CH, 1>(acc, c_lo, c_hi, s_lo, s_hi, tail_b, 1, K, q, gsc, ntiles, true, act);
 }
 
-// The last k-block b of a row whose length K ends inside it (K % 128 == 64):
-// lane slices past K contribute zero.
+// Four consecutive k-blocks b0 .. b0 + 3 of one 16-row weight tile held in
+// registers (loaded from global memory): the lane's codes of its row (lo) and
+// row + 8 (hi) and their raw scales.  Blocks at or past nblk, and lane slices
+// past K, hold zeros.
+struct RegChunk {
+  uint4 lo[4], hi[4];
+  uint32_t slo[4], shi[4];
+};
+
+// Load a RegChunk: codes_lo / codes_hi point at the two rows' codes plus the
+// lane's slice offset 16q, scales_lo / scales_hi at their scales (global,
+// read-only for the kernel's lifetime; the codes are read once, so they are
+// not kept in L1).
+template <int FMT>
+MOE_DEV void load_chunk(RegChunk& c, const uint8_t* codes_lo, const uint8_t* codes_hi, const uint8_t* scales_lo,
+                        const uint8_t* scales_hi, int b0, int nblk, int K, int q) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = b0 + i;
+    const bool in = b < nblk && 128 * b + 32 * q < K;
+    c.lo[i] = in ? ldg_nc_v4(codes_lo + 64 * b) : make_uint4(0, 0, 0, 0);
+    c.hi[i] = in ? ldg_nc_v4(codes_hi + 64 * b) : make_uint4(0, 0, 0, 0);
+    c.slo[i] = in ? raw_scale<FMT, true>(scales_lo, b, q) : 0u;
+    c.shi[i] = in ? raw_scale<FMT, true>(scales_hi, b, q) : 0u;
+  }
+}
+
+// acc[j] += W x B_j over the blocks of a RegChunk (block b0 + i for i < 4
+// while b0 + i < nblk), for the token tiles j < ntiles.
 template <int FMT, int NT, int CH, typename Act>
-MOE_DEV void tile_tail(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
-                       const uint8_t* sc_hi, int b, int K, int q, float gsc, int ntiles, const Act& act) {
-  const bool in = 128 * b + 32 * q < K;
+MOE_DEV void chunk_mma(float (&acc)[NT][CH][4], const RegChunk& c, int b0, int nblk, int K, int q, float gsc,
+                       int ntiles, const Act& act) {
+  Mult mlo[4], mhi[4];
   bool fast = true;
-  Mult mlo[1], mhi[1];
-  mlo[0] = mult_at<FMT>(sc_lo, b, q, gsc, in, fast);
-  mhi[0] = mult_at<FMT>(sc_hi, b, q, gsc, in, fast);
-  const uint4 lo = in ? *reinterpret_cast<const uint4*>(c_lo + 64 * b) : make_uint4(0, 0, 0, 0);
-  const uint4 hi = in ? *reinterpret_cast<const uint4*>(c_hi + 64 * b) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = b0 + i;
+    const bool in = b < nblk && 128 * b + 32 * q < K;
+    mlo[i] = mult_of<FMT>(c.slo[i], gsc, in, fast);
+    mhi[i] = mult_of<FMT>(c.shi[i], gsc, in, fast);
+  }
   const bool all_fast = __all_sync(0xffffffffu, fast);
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    if (j > 0 && j >= ntiles) break;
-    uint32_t bf[8][2];
-    act.load(j, b, in, bf);
-    if (all_fast) mma_kblock<FMT, true, CH>(acc[j], 0, lo, hi, mlo[0], mhi[0], bf);
-    else mma_kblock<FMT, false, CH>(acc[j], 0, lo, hi, mlo[0], mhi[0], bf);
+  for (int i = 0; i < 4; ++i) {
+    const int b = b0 + i;
+    if (b >= nblk) break;  // warp-uniform
+    const bool in = 128 * b + 32 * q < K;
+    const int c0 = CH == 4 ? 2 * (i & 1) : 0;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (j > 0 && j >= ntiles) break;
+      uint32_t bf[8][2];
+      act.load(j, b, in, bf);
+      if (all_fast) mma_kblock<FMT, true, CH>(acc[j], c0, c.lo[i], c.hi[i], mlo[i], mhi[i], bf);
+      else mma_kblock<FMT, false, CH>(acc[j], c0, c.lo[i], c.hi[i], mlo[i], mhi[i], bf);
+    }
   }
-}
-
-// One warp's share of a 16-row tile: the nb full k-blocks b0, b0 + bstep, ...
-// (four at a time where possible) and, if tail_b >= 0, the partial block
-// tail_b.
-template <int FMT, int NT, int CH, typename Act>
-MOE_DEV void warp_tile(float (&acc)[NT][CH][4], const uint8_t* c_lo, const uint8_t* c_hi, const uint8_t* sc_lo,
-                       const uint8_t* sc_hi, int b0, int bstep, int nb, int tail_b, int K, int q, float gsc,
-                       int ntiles, const Act& act) {
-  int i = 0;
-  for (; i + 4 <= nb; i += 4)
-    tile_blocks<FMT, NT, CH, 4>(acc, c_lo, c_hi, sc_lo, sc_hi, b0 + i * bstep, bstep, q, gsc, ntiles, act);
-  for (; i < nb; ++i)
-    tile_blocks<FMT, NT, CH, 1>(acc, c_lo, c_hi, sc_lo, sc_hi, b0 + i * bstep, bstep, q, gsc, ntiles, act);
-  if (tail_b >= 0) tile_tail<FMT, NT, CH>(acc, c_lo, c_hi, sc_lo, sc_hi, tail_b, K, q, gsc, ntiles, act);
 }
 
 // Bytes staged for `rows` consecutive weight rows (codes + scales).
