@@ -187,7 +187,7 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   {
     NvtxRange range("moe.gate_up");
     MOE_TRY(mark(o, 2, 0, stream));
-    if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, er, ws, stream));
+    if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, dn, er, ws, stream));
     else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
     MOE_TRY(mark(o, 2, 1, stream));
   }

@@ -203,6 +203,26 @@ MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint
   }
 }
 
+// mbar_wait for a thread off the critical path (a warp that waits for a whole
+// tile, or a producer ahead of its consumers): between tries it sleeps about
+// sleep_ns, so a long wait costs a few instructions per sleep instead of a
+// stream of polls that would take issue slots from the warps doing work.
+MOE_DEV bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* gstatus,
+                               uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      if (gstatus) atomicOr(gstatus, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // Wait for the phase of `bar` with the given parity, ignoring any abort flag;
 // gives up (false) after limit_ns.  Used to drain copies still in flight.
 MOE_DEV bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {

@@ -27,6 +27,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -58,6 +59,8 @@ constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
 constexpr int kDnWarps = MOE_DEC_DN_WARPS;
 constexpr int kDnThreads = kDnWarps * 32;
 constexpr int kDnRows = 16;  // output features per down tile
+constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
+constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch issued by gate_up
 
 // Offsets inside one gate_up stage: gate-row codes, 64 bytes of padding,
 // up-row codes, then gate-row and up-row scales (see decode_common.cuh).
@@ -168,7 +171,7 @@ template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
-    uint16_t* __restrict__ act, uint32_t* status, int S) {
+    uint16_t* __restrict__ act, uint32_t* status, int S, Bank dn) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int G = kGuGroups, MT = kGuMT, CH = 2;
   constexpr int kRed = kGroupWarps * NT * MT * 128;  // floats of one group's partial tiles
@@ -212,6 +215,19 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
 
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
+    if (dn.codes) {
+      // this CTA's share of the touched experts' down matrices into L2 for
+      // the down kernel that follows: pieces of kDnPrefetchRows rows, piece
+      // p to CTA p % grid, one lane per piece
+      const int per_e = dn.N / kDnPrefetchRows;
+      const int pieces = (t_hi - t_lo) * per_e;
+      for (int p = blockIdx.x + lane * gridDim.x; p < pieces; p += 32 * gridDim.x) {
+        const int ex = p / per_e;
+        const long row = long(s_local[ex] - e_lo) * dn.N + (p - ex * per_e) * kDnPrefetchRows;
+        prefetch_codes<FMT>(dn, row, kDnPrefetchRows);
+        prefetch_scales<FMT>(dn, row, kDnPrefetchRows);
+      }
+    }
     const uint64_t policy = l2_policy_evict_first();
     const uint32_t run = uint32_t(kGuFeat * (K / 2)), srun = uint32_t(kGuFeat * srow);
     const uint8_t* scales = static_cast<const uint8_t*>(gu.scales);
@@ -219,7 +235,9 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
     int i = 0, st = 0, ph = 0;  // unit i's stage and that stage's use count parity
     for (; i < cnt; ++i) {
-      if (i >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &s_abort, status))) break;
+      if (i >= S &&
+          !__all_sync(0xffffffffu, mbar_wait_backoff(&empty[st], ph ^ 1, &s_abort, status, kProducerSleepNs)))
+        break;
       fence_proxy_async_smem();  // earlier generic-proxy reads of this stage before the refill
       if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * run + 2 * srun);
       __syncwarp();
@@ -411,90 +429,11 @@ __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
   const uint8_t* scales = static_cast<const uint8_t*>(dn.scales);
   const int my_units = warp < n_t ? (n_t - warp + W - 1) / W : 0;  // per tile
   const int nk = my_units * nch;                                   // chunks per tile
-  // the lane's two rows of unit m's tile, codes (+ slice offset) and scales
-  auto rows_of = [&](int tile, int m, const uint8_t*& c_lo, const uint8_t*& s_lo) {
-    const long r = long(s_local[warp + W * m] - e_lo) * H + tile * kDnRows + g;
-    c_lo = dn.codes + r * (K / 2) + 16 * q;
-    s_lo = scales + r * srow;
-  };
-  auto load = [&](RegChunk& c, int tile, int k) {
-    const int m = k / nch, ch = k - m * nch;
-    const uint8_t *c_lo, *s_lo;
-    rows_of(tile, m, c_lo, s_lo);
-    load_chunk<FMT>(c, c_lo, c_lo + 8 * (K / 2), s_lo, s_lo + 8 * srow, 4 * ch, nblk, K, q);
-  };
-  if (lane < my_units && blockIdx.x < ntile) {
-    // all of this warp's tiles of the CTA's first tile into L2
-    const long r0 = long(s_local[warp + W * lane] - e_lo) * H + blockIdx.x * kDnRows;
-    prefetch_codes<FMT>(dn, r0, kDnRows);
-    prefetch_scales<FMT>(dn, r0, kDnRows);
-  }
-  RegChunk cA, cB;
-  if (nk > 0 && blockIdx.x < ntile) load(cA, blockIdx.x, 0);
-
-  pdl_wait();  // the activations (and the previous readers of the output) of the kernels before
-  pdl_trigger();
-  if (ACT_SMEM) {
-    stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kDnThreads);
+  // the tile's outputs: each token's k slots summed in slot order, two
+  // features per thread (block barriers before and after: ybuf is complete,
+  // then cleared for the next tile)
+  auto finish_tile = [&](int tile) {
     __syncthreads();
-  }
-  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
-    if (tile != int(blockIdx.x) && nk > 0) load(cA, tile, 0);
-    float acc[NT][CH][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int h = 0; h < CH; ++h)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
-    // multiply chunk k (in `cur`); after a unit's last chunk, its weighted
-    // outputs go to ybuf and the accumulators restart
-    auto step = [&](const RegChunk& cur, int k) {
-      const int m = k / nch, ch = k - m * nch;
-      const int e = s_local[warp + W * m];
-      const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-      const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
-      const int ntiles = min(NT, (n_e + 7) / 8);
-      ActFrags<ACT_SMEM> af;
-      af.act = act;
-      af.act_s = act_s;
-      af.pstride = pstride;
-      af.K = K;
-      af.q = q;
-      af.g = g;
-      af.p0 = p0;
-      af.n_e = n_e;
-      chunk_mma<FMT, NT, CH>(acc, cur, 4 * ch, nblk, K, q, gsc, ntiles, af);
-      if (ch != nch - 1) return;
-      // c0, c1: feature g at columns 2q, 2q+1; c2, c3: feature g + 8
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        if (j < ntiles) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int col = 8 * j + 2 * q + (c & 1);
-            float v = acc[j][0][c];
-#pragma unroll
-            for (int h = 1; h < CH; ++h) v += acc[j][h][c];
-            if (col < n_e) ybuf[s_slot[p0 + col] * kDnRows + g + 8 * (c >> 1)] = s_w[p0 + col] * v;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < CH; ++h)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
-      }
-    };
-    for (int k = 0; k < nk;) {
-      if (k + 1 < nk) load(cB, tile, k + 1);
-      step(cA, k);
-      if (++k >= nk) break;
-      if (k + 1 < nk) load(cA, tile, k + 1);
-      step(cB, k);
-      ++k;
-    }
-    __syncthreads();
-    // each token's k slots summed in slot order, two features per thread
     for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kDnThreads) {
       const int t = o / (kDnRows / 2), f = 2 * (o % (kDnRows / 2));
       float v0 = 0.f, v1 = 0.f;
@@ -518,7 +457,94 @@ __global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
       }
     }
     __syncthreads();
+  };
+  if (lane < my_units && blockIdx.x < ntile) {
+    // all of this warp's tiles of the CTA's first tile into L2
+    const long r0 = long(s_local[warp + W * lane] - e_lo) * H + blockIdx.x * kDnRows;
+    prefetch_codes<FMT>(dn, r0, kDnRows);
+    prefetch_scales<FMT>(dn, r0, kDnRows);
   }
+  // The tile loop; FULL (every chunk is four whole k-blocks) drops the
+  // bounds checks of the chunk loads and multiplies.
+  auto run = [&](auto full_tag) {
+    constexpr bool FULL = decltype(full_tag)::value;
+    // chunk k of this warp's units: unit m = k / nch, chunk k % nch
+    auto load = [&](RegChunk& c, int tile, int k) {
+      const int m = nch == 1 ? k : k / nch, ch = k - m * nch;
+      const long r = long(s_local[warp + W * m] - e_lo) * H + tile * kDnRows + g;
+      const uint8_t* c_lo = dn.codes + r * (K / 2) + 16 * q;
+      const uint8_t* s_lo = scales + r * srow;
+      load_chunk<FMT, FULL>(c, c_lo, c_lo + 8 * (K / 2), s_lo, s_lo + 8 * srow, 4 * ch, nblk, K, q);
+    };
+    RegChunk cA, cB;
+    if (nk > 0 && blockIdx.x < ntile) load(cA, blockIdx.x, 0);
+
+    pdl_wait();  // the activations (and the previous readers of the output) of the kernels before
+    pdl_trigger();
+    if (ACT_SMEM) {
+      stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kDnThreads);
+      __syncthreads();
+    }
+    for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+      if (tile != int(blockIdx.x) && nk > 0) load(cA, tile, 0);
+      float acc[NT][CH][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int h = 0; h < CH; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
+      // multiply chunk k (in `cur`); after a unit's last chunk, its weighted
+      // outputs go to ybuf and the accumulators restart
+      auto step = [&](const RegChunk& cur, int k) {
+        const int m = nch == 1 ? k : k / nch, ch = k - m * nch;
+        const int e = s_local[warp + W * m];
+        const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
+        const float gsc = FMT == MOE_FMT_NVFP4_G16 ? dn.gscale[e - e_lo] : 0.f;
+        const int ntiles = min(NT, (n_e + 7) / 8);
+        ActFrags<ACT_SMEM> af;
+        af.act = act;
+        af.act_s = act_s;
+        af.pstride = pstride;
+        af.K = K;
+        af.q = q;
+        af.g = g;
+        af.p0 = p0;
+        af.n_e = n_e;
+        chunk_mma<FMT, NT, CH, FULL>(acc, cur, 4 * ch, nblk, K, q, gsc, ntiles, af);
+        if (ch != nch - 1) return;
+        // c0, c1: feature g at columns 2q, 2q+1; c2, c3: feature g + 8
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (j < ntiles) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = 8 * j + 2 * q + (c & 1);
+              float v = acc[j][0][c];
+#pragma unroll
+              for (int h = 1; h < CH; ++h) v += acc[j][h][c];
+              if (col < n_e) ybuf[s_slot[p0 + col] * kDnRows + g + 8 * (c >> 1)] = s_w[p0 + col] * v;
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < CH; ++h)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
+        }
+      };
+      for (int k = 0; k < nk;) {
+        if (k + 1 < nk) load(cB, tile, k + 1);
+        step(cA, k);
+        if (++k >= nk) break;
+        if (k + 1 < nk) load(cA, tile, k + 1);
+        step(cB, k);
+        ++k;
+      }
+      finish_tile(tile);
+    }
+  };
+  if (K % 512 == 0) run(std::true_type{});
+  else run(std::false_type{});
 }
 
 int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
@@ -630,8 +656,8 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 }
 
 template <int FMT, int NT>
-cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const ExpertRange& er,
-                       const Workspace& ws, int units, cudaStream_t stream) {
+cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
+                       const ExpertRange& er, const Workspace& ws, int units, cudaStream_t stream) {
   const GuPlan p = gate_up_plan(s, T);
   if (p.S == 0) return cudaErrorInvalidConfiguration;
   auto k = p.x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
@@ -640,16 +666,16 @@ cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Ban
   const int grid = persistent_grid(k, p.smem, units, kGuThreads);
   return launch_pdl(k, dim3(grid), dim3(kGuThreads), p.smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k,
                     er.lo, er.hi, (const int32_t*)ws.touched, (const int32_t*)ws.offsets,
-                    (const int32_t*)ws.sorted_rows, ws.act, ws.status, p.S);
+                    (const int32_t*)ws.sorted_rows, ws.act, ws.status, p.S, dn);
 }
 
 template <int FMT>
-cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const ExpertRange& er,
-                        const Workspace& ws, int units, cudaStream_t stream) {
+cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
+                        const ExpertRange& er, const Workspace& ws, int units, cudaStream_t stream) {
   // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
-  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, er, ws, units, stream);
-  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, er, ws, units, stream);
-  return gate_up_nt<FMT, 4>(s, T, x, gu, er, ws, units, stream);
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, dn, er, ws, units, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, dn, er, ws, units, stream);
+  return gate_up_nt<FMT, 4>(s, T, x, gu, dn, er, ws, units, stream);
 }
 
 template <int FMT, int NT>
@@ -682,13 +708,15 @@ bool decode_supported(const moe_shape_t& s, int T) {
   return gate_up_plan(s, T).S > 0 && down_plan(s, T).smem <= kMaxSmemPerCta;
 }
 
-cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
+cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
   const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / kGuFeat);
   if (units <= 0) return cudaSuccess;
-  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, er, ws, units, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, er, ws, units, stream);
-  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, er, ws, units, stream);
+  Bank pf = dn;
+  if (s.hidden % kDnPrefetchRows) pf.codes = nullptr;  // whole pieces only
+  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, pf, er, ws, units, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, pf, er, ws, units, stream);
+  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, pf, er, ws, units, stream);
 }
 
 cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,

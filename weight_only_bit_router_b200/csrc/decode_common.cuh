@@ -346,24 +346,32 @@ struct RegChunk {
 // Load a RegChunk: codes_lo / codes_hi point at the two rows' codes plus the
 // lane's slice offset 16q, scales_lo / scales_hi at their scales (global,
 // read-only for the kernel's lifetime; the codes are read once, so they are
-// not kept in L1).
-template <int FMT>
+// not kept in L1).  FULL: all four blocks lie inside K (no checks).
+template <int FMT, bool FULL>
 MOE_DEV void load_chunk(RegChunk& c, const uint8_t* codes_lo, const uint8_t* codes_hi, const uint8_t* scales_lo,
                         const uint8_t* scales_hi, int b0, int nblk, int K, int q) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int b = b0 + i;
-    const bool in = b < nblk && 128 * b + 32 * q < K;
-    c.lo[i] = in ? ldg_nc_v4(codes_lo + 64 * b) : make_uint4(0, 0, 0, 0);
-    c.hi[i] = in ? ldg_nc_v4(codes_hi + 64 * b) : make_uint4(0, 0, 0, 0);
-    c.slo[i] = in ? raw_scale<FMT, true>(scales_lo, b, q) : 0u;
-    c.shi[i] = in ? raw_scale<FMT, true>(scales_hi, b, q) : 0u;
+    if (FULL) {
+      c.lo[i] = ldg_nc_v4(codes_lo + 64 * b);
+      c.hi[i] = ldg_nc_v4(codes_hi + 64 * b);
+      c.slo[i] = raw_scale<FMT, true>(scales_lo, b, q);
+      c.shi[i] = raw_scale<FMT, true>(scales_hi, b, q);
+    } else {
+      const bool in = b < nblk && 128 * b + 32 * q < K;
+      c.lo[i] = in ? ldg_nc_v4(codes_lo + 64 * b) : make_uint4(0, 0, 0, 0);
+      c.hi[i] = in ? ldg_nc_v4(codes_hi + 64 * b) : make_uint4(0, 0, 0, 0);
+      c.slo[i] = in ? raw_scale<FMT, true>(scales_lo, b, q) : 0u;
+      c.shi[i] = in ? raw_scale<FMT, true>(scales_hi, b, q) : 0u;
+    }
   }
 }
 
 // acc[j] += W x B_j over the blocks of a RegChunk (block b0 + i for i < 4
-// while b0 + i < nblk), for the token tiles j < ntiles.
-template <int FMT, int NT, int CH, typename Act>
+// while b0 + i < nblk), for the token tiles j < ntiles.  FULL: all four
+// blocks lie inside K.
+template <int FMT, int NT, int CH, bool FULL, typename Act>
 MOE_DEV void chunk_mma(float (&acc)[NT][CH][4], const RegChunk& c, int b0, int nblk, int K, int q, float gsc,
                        int ntiles, const Act& act) {
   Mult mlo[4], mhi[4];
@@ -371,7 +379,7 @@ MOE_DEV void chunk_mma(float (&acc)[NT][CH][4], const RegChunk& c, int b0, int n
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int b = b0 + i;
-    const bool in = b < nblk && 128 * b + 32 * q < K;
+    const bool in = FULL || (b < nblk && 128 * b + 32 * q < K);
     mlo[i] = mult_of<FMT>(c.slo[i], gsc, in, fast);
     mhi[i] = mult_of<FMT>(c.shi[i], gsc, in, fast);
   }
@@ -379,8 +387,8 @@ MOE_DEV void chunk_mma(float (&acc)[NT][CH][4], const RegChunk& c, int b0, int n
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int b = b0 + i;
-    if (b >= nblk) break;  // warp-uniform
-    const bool in = 128 * b + 32 * q < K;
+    if (!FULL && b >= nblk) break;  // warp-uniform
+    const bool in = FULL || 128 * b + 32 * q < K;
     const int c0 = CH == 4 ? 2 * (i & 1) : 0;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {

@@ -162,6 +162,12 @@ MOE_DEV void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
                : "memory");
 }
 
+// Sleep between tries of the waits off the critical path: the producers
+// (code tiles, scale rows, token rows) run ahead of the dequantisation warps,
+// and the epilogue waits for a whole tile's main loop.
+constexpr uint32_t kProducerSleepNs = 64;
+constexpr uint32_t kEpilogueSleepNs = 256;
+
 // Code tiles this many k-stages ahead of the producer are prefetched into L2.
 constexpr int kCodePrefetch = 8;
 
@@ -320,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE != kRouter) {
           // the tile's scale rows: contiguous rows of the scale plane, once per tile
           const int slot = it & 1;
-          if (!(ok = mbar_wait(&sc_empty[slot], ((it >> 1) & 1) ^ 1, abort, a.status))) break;
+          if (!(ok = mbar_wait_backoff(&sc_empty[slot], ((it >> 1) & 1) ^ 1, abort, a.status, kProducerSleepNs)))
+            break;
           const int f0 = t.fb * BM;
           const int rows = min(BM, a.M_total - f0);
           const uint32_t bytes = uint32_t(rows * sb);
@@ -342,7 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sA + s * NACC * kTileBytes, &tmap_a, &opA_full[s], ks * BK, t.fb * BM);
           } else {
             const int s = g % SC;
-            if (!(ok = mbar_wait(&codes_empty[s], ((g / SC) & 1) ^ 1, abort, a.status))) break;
+            if (!(ok = mbar_wait_backoff(&codes_empty[s], ((g / SC) & 1) ^ 1, abort, a.status, kProducerSleepNs)))
+              break;
             mbar_arrive_expect_tx(&codes_full[s], NACC * kCodeBytes);
             uint8_t* dst = sC + s * NACC * kCodeBytes;
             if (MODE == kGateUp) {
@@ -442,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_tile(a, tile, s_tile_base);
         for (int ks = 0; ks < KS; ++ks, ++g) {
           const int s = g % SB;
-          if (!(ok = mbar_wait(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status))) break;
+          if (!(ok = mbar_wait_backoff(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status, kProducerSleepNs))) break;
           mbar_arrive_expect_tx(&opB_full[s], kTileBytes);
           tma_load_2d(sB + s * kTileBytes, &tmap_b, &opB_full[s], ks * BK, t.p_begin);
         }
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int ks = 0; ks < KS; ++ks, ++g) {
         const int s = g % SB;
-        if (!(ok = mbar_wait(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status))) break;
+        if (!(ok = mbar_wait_backoff(&opB_empty[s], ((g / SB) & 1) ^ 1, abort, a.status, kProducerSleepNs))) break;
         const uint32_t base = smem_u32(sB + s * kTileBytes);
 #pragma unroll
         for (int i = 0; i < BN / 8; ++i) {
@@ -559,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
       const Tile t = decode_tile(a, tile, s_tile_base);
       const int buf = it & 1;
-      if (!(ok = mbar_wait(&acc_full[buf], (it >> 1) & 1, abort, a.status))) break;
+      if (!(ok = mbar_wait_backoff(&acc_full[buf], (it >> 1) & 1, abort, a.status, kEpilogueSleepNs))) break;
       tc_fence_after();
       const int f = t.fb * BM + r;
       const bool row_ok = f < a.M_total;

@@ -112,7 +112,9 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 // the decode kernels take this shape and token count (T <= kDecodeMaxT and the
 // stages fit in shared memory)
 bool decode_supported(const moe_shape_t& s, int T);
-cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu,
+// gate_up + SwiGLU into ws.act; also requests the touched experts' rows of
+// the down bank `dn` into L2 for the down kernel that follows
+cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
 // the down products of the bank's experts and the combine: out = bf16(sum
 // over each token's slots in slot order of w * y (+ sh_gate[t] * sh_y[t])),
