@@ -59,6 +59,11 @@ constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
 constexpr int kDnWarps = MOE_DEC_DN_WARPS;
 constexpr int kDnThreads = kDnWarps * 32;
 constexpr int kDnRows = 16;  // output features per down tile
+// registers per down thread: up to 8 tokens, room on the SM for the next
+// layer's routing kernel (256 threads x 80) while down CTAs drain; more
+// token tiles need more (two warps per SM sub-partition: at most 255)
+constexpr int kDnRegs = 160;
+constexpr int kDnRegsWide = 224;
 constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
 constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch issued by gate_up
 
@@ -215,24 +220,25 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
 
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
-    if (dn.codes) {
-      // this CTA's share of the touched experts' down matrices into L2 for
-      // the down kernel that follows: pieces of kDnPrefetchRows rows, piece
-      // p to CTA p % grid, one lane per piece
-      const int per_e = dn.N / kDnPrefetchRows;
-      const int pieces = (t_hi - t_lo) * per_e;
-      for (int p = blockIdx.x + lane * gridDim.x; p < pieces; p += 32 * gridDim.x) {
-        const int ex = p / per_e;
-        const long row = long(s_local[ex] - e_lo) * dn.N + (p - ex * per_e) * kDnPrefetchRows;
-        prefetch_codes<FMT>(dn, row, kDnPrefetchRows);
-        prefetch_scales<FMT>(dn, row, kDnPrefetchRows);
-      }
-    }
     const uint64_t policy = l2_policy_evict_first();
     const uint32_t run = uint32_t(kGuFeat * (K / 2)), srun = uint32_t(kGuFeat * srow);
     const uint8_t* scales = static_cast<const uint8_t*>(gu.scales);
     int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;                 // unit i
     int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
+    // This CTA's share of the touched experts' down matrices into L2 for the
+    // down kernel that follows: pieces of kDnPrefetchRows rows, the CTA's
+    // j-th piece is piece blockIdx.x + j * grid.
+    const int dn_per_e = dn.codes ? dn.N / kDnPrefetchRows : 0;
+    const int dn_pieces = (t_hi - t_lo) * dn_per_e;
+    auto prefetch_down = [&](int j) {
+      const int p = blockIdx.x + j * gridDim.x;
+      if (p >= dn_pieces) return;
+      const int ex = p / dn_per_e;
+      const long row = long(s_local[ex] - e_lo) * dn.N + (p - ex * dn_per_e) * kDnPrefetchRows;
+      prefetch_codes<FMT>(dn, row, kDnPrefetchRows);
+      prefetch_scales<FMT>(dn, row, kDnPrefetchRows);
+    };
+    int pf_next = 0;  // the CTA's next piece
     int i = 0, st = 0, ph = 0;  // unit i's stage and that stage's use count parity
     for (; i < cnt; ++i) {
       if (i >= S &&
@@ -247,16 +253,23 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
         uint8_t* stage = ring + size_t(st) * L.stage_bytes;
         if (lane < 2) bulk_g2s_hint(stage + (lane ? L.cB : L.cA), gu.codes + row * (K / 2), run, &full[st], policy);
         else bulk_g2s_hint(stage + (lane & 1 ? L.sB : L.sA), scales + row * srow, srun, &full[st], policy);
-      } else if (lane < 8 && i + S < cnt) {
-        // the unit that will refill this stage, into L2 ahead of time
-        const long row = long(s_local[pslot] - e_lo) * gu.N + pft * kGuFeat + ((lane & 1) ? I : 0);
-        if (lane < 6) prefetch_codes<FMT>(gu, row, kGuFeat);
-        else prefetch_scales<FMT>(gu, row, kGuFeat);
+      } else if (lane < 8) {
+        if (i + S < cnt) {
+          // the unit that will refill this stage, into L2 ahead of time
+          const long row = long(s_local[pslot] - e_lo) * gu.N + pft * kGuFeat + ((lane & 1) ? I : 0);
+          if (lane < 6) prefetch_codes<FMT>(gu, row, kGuFeat);
+          else prefetch_scales<FMT>(gu, row, kGuFeat);
+        }
+      } else if (lane < 12 && i >= S) {
+        prefetch_down(pf_next + lane - 8);  // once the ring is primed: four pieces per unit
       }
+      if (i >= S) pf_next += 4;
       if (++st == S) st = 0, ph ^= 1;
       if (++ft == ftiles) ft = 0, ++slot;
       if (++pft == ftiles) pft = 0, ++pslot;
     }
+    // the rest of the share, one piece per lane
+    for (int j = pf_next + lane; blockIdx.x + j * int(gridDim.x) < dn_pieces; j += 32) prefetch_down(j);
     if (lane == 0) drain_stages(full, i, S);
     return;
   }
@@ -389,7 +402,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
 // T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __launch_bounds__(kDnThreads, 1) decode_down_kernel(
+__global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
     const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,

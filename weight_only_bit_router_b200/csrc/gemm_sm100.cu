@@ -167,6 +167,9 @@ MOE_DEV void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
 // and the epilogue waits for a whole tile's main loop.
 constexpr uint32_t kProducerSleepNs = 64;
 constexpr uint32_t kEpilogueSleepNs = 256;
+// The MMA issuer waits on the dequantisation warps most of the time; a short
+// sleep between its tries keeps its polls from taking their issue slots.
+constexpr uint32_t kMmaSleepNs = 32;
 
 // Code tiles this many k-stages ahead of the producer are prefetched into L2.
 constexpr int kCodePrefetch = 8;
@@ -401,15 +404,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const Tile t = decode_tile(a, tile, s_tile_base);
         const int buf = it & 1;
-        if (!(ok = mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, a.status))) break;
+        if (!(ok = mbar_wait_backoff(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, a.status, kMmaSleepNs))) break;
         tc_fence_after();
         const uint32_t n16 = uint32_t((t.n + 15) & ~15);
         const uint32_t idesc = umma_idesc_bf16(BM, n16);
         const uint32_t d0 = tmem_base + uint32_t(buf * NACC * BN);
         for (int ks = 0; ks < KS; ++ks, ++g) {
           const int sa = g % SA, sbuf = g % SB;
-          if (!(ok = mbar_wait(&opA_full[sa], (g / SA) & 1, abort, a.status))) break;
-          if (!(ok = mbar_wait(&opB_full[sbuf], (g / SB) & 1, abort, a.status))) break;
+          if (!(ok = mbar_wait_backoff(&opA_full[sa], (g / SA) & 1, abort, a.status, kMmaSleepNs))) break;
+          if (!(ok = mbar_wait_backoff(&opB_full[sbuf], (g / SB) & 1, abort, a.status, kMmaSleepNs))) break;
           // the token rows landed through cp.async (generic proxy): order them
           // before the tensor core's (async proxy) reads
           fence_proxy_async_smem();
