@@ -170,7 +170,8 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // blocks w, w + 4, ...), and one of them (rotating) sums the four partial
 // tiles in warp order and writes a = bf16(silu(gate) * up) to act[p][f] for
 // the expert's sorted rows p.  With X_SMEM (small T) the consumers first
-// stage the T token rows in fragment order.
+// stage the T token rows in fragment order, before the programmatic-launch
+// wait.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
@@ -204,6 +205,11 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
     }
     fence_mbar_init();
   }
+  // The token rows do not depend on the kernel just before: every kernel of
+  // the forward waits for its predecessor before it lets its dependents
+  // launch, so x's producer finished before this kernel started.  Staged
+  // before the wait (published by the block barrier below).
+  if (X_SMEM && warp < G * kGroupWarps) stage_act_rows<1>(x_s, x, T, K, threadIdx.x, G * kGroupWarps * 32);
   pdl_wait();
   pdl_trigger();
   load_routing(s_touched, s_off, touched, offsets, E);
@@ -275,14 +281,9 @@ __global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
   }
 
   // -------------------------------------------------------------------- consumers
-  constexpr int kConsumers = G * kGroupWarps * 32;
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
   const bool odd = (g & 1) != 0;  // this lane's low MMA row is the up row
-  if (X_SMEM) {
-    stage_act_rows<1>(x_s, x, T, K, threadIdx.x, kConsumers);
-    named_barrier_sync(1, kConsumers);
-  }
   const int nfull = K / 128;  // blocks where every lane slice lies inside K
   const int my_full = wj < nfull ? (nfull - wj + kGroupWarps - 1) / kGroupWarps : 0;
   const int tail_b = ((K % 128) != 0 && nfull % kGroupWarps == wj) ? nfull : -1;

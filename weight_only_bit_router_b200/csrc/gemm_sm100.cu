@@ -248,7 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kSrow = C::SROW;
   constexpr int NACC = C::NACC;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment by an offset into the shared array (not by integer
+  // arithmetic on its address), so every access below stays a shared-memory
+  // access instead of a generic one
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;                          // [SA][NACC][16 KB]
   uint8_t* sB = sA + C::SMEM_A;                // [SB][16 KB]
   uint8_t* sC = sB + C::SMEM_B;                // [SC][NACC][4 KB]

@@ -121,16 +121,19 @@ namespace moe {
 // Top-k (k <= 8) of one token's logits row[0, E) (+ bias), E <= 256: writes
 // ids[0, k) in descending order and the renormalised softmax weights over the
 // selected (biased) logits.  `row` may point to shared or global memory.
+// Lane l holds experts 8l .. 8l + 7.  Each of the k rounds takes every lane's
+// best remaining expert (larger key, ties to the lower expert), then the
+// warp's best (max key; among lanes with it, the lowest lane: the lower
+// expert), and the winning lane marks it taken.  Short code on purpose: it
+// runs once per layer in a single CTA, often with a cold instruction cache.
 MOE_DEV void warp_topk8(const float* row, const float* __restrict__ bias, int E, int k, int32_t* ids,
                         float* wout) {
   const unsigned full = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   uint32_t key[8];
-  int slot[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = 8 * lane + i;
-    slot[i] = i;
     key[i] = 0u;  // empty: below every real key
     if (e < E) {
       float val = row[e];
@@ -138,45 +141,28 @@ MOE_DEV void warp_topk8(const float* row, const float* __restrict__ bias, int E,
       key[i] = orderable(val);
     }
   }
-  // bitonic sort, best first: larger key, or equal key and lower slot
-#pragma unroll
-  for (int size = 2; size <= 8; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int l = i ^ stride;
-        if (l > i) {
-          const bool l_better = key[l] > key[i] || (key[l] == key[i] && slot[l] < slot[i]);
-          const bool swap = ((i & size) == 0) ? l_better : !l_better;
-          const uint32_t ki = key[i], kl = key[l];
-          const int si = slot[i], sl = slot[l];
-          key[i] = swap ? kl : ki;
-          key[l] = swap ? ki : kl;
-          slot[i] = swap ? sl : si;
-          slot[l] = swap ? si : sl;
-        }
-      }
-    }
-  }
+  uint32_t taken = 0u;  // bit i: expert 8 lane + i already selected
   float my_val = 0.f;
   int my_id = 0;
 #pragma unroll 1
   for (int j = 0; j < k; ++j) {
-    const uint32_t kmax = __reduce_max_sync(full, key[0]);
-    const int wl = __ffs(__ballot_sync(full, key[0] == kmax)) - 1;
-    const int wslot = __shfl_sync(full, slot[0], wl);
-    if (lane == wl) {
+    uint32_t best = 0u;
+    int bi = 0;
 #pragma unroll
-      for (int i = 0; i < 7; ++i) {
-        key[i] = key[i + 1];
-        slot[i] = slot[i + 1];
+    for (int i = 7; i >= 0; --i) {
+      const uint32_t v = (taken >> i) & 1u ? 0u : key[i];
+      if (v >= best) {  // from the top down: ties end on the lower index
+        best = v;
+        bi = i;
       }
-      key[7] = 0u;
     }
+    const uint32_t kmax = __reduce_max_sync(full, best);
+    const int wl = __ffs(__ballot_sync(full, best == kmax)) - 1;
+    const int wi = __shfl_sync(full, bi, wl);
+    if (lane == wl) taken |= 1u << wi;
     if (lane == j) {
       my_val = from_orderable(kmax);
-      my_id = 8 * wl + wslot;
+      my_id = 8 * wl + wi;
     }
   }
   const float vmax = __shfl_sync(full, my_val, 0);
