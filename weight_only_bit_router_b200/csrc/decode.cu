@@ -39,11 +39,10 @@ namespace moe {
 namespace {
 
 constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
-constexpr int kGuFeat = 16;     // gate_up: features per work unit (16 gate + 16 up rows)
-constexpr int kGuMT = 2;        // gate_up: 16-row MMA tiles per unit
 
 // Build-time tuning knobs (the defaults are the measured best): gate_up
-// consumer groups per CTA and its largest stage ring; down warps per CTA.
+// consumer groups per CTA and its largest stage ring; down warps per CTA;
+// gate_up unit size and CTAs per SM.
 #ifndef MOE_DEC_GROUPS
 #define MOE_DEC_GROUPS 2
 #endif
@@ -53,6 +52,15 @@ constexpr int kGuMT = 2;        // gate_up: 16-row MMA tiles per unit
 #ifndef MOE_DEC_DN_WARPS
 #define MOE_DEC_DN_WARPS 8
 #endif
+#ifndef MOE_DEC_GU_MT
+#define MOE_DEC_GU_MT 2
+#endif
+#ifndef MOE_DEC_GU_CTAS
+#define MOE_DEC_GU_CTAS 1
+#endif
+constexpr int kGuMT = MOE_DEC_GU_MT;     // gate_up: 16-row MMA tiles per unit (8 features each)
+constexpr int kGuFeat = 8 * kGuMT;       // gate_up: features per unit (that many gate and up rows)
+constexpr int kGuCtas = MOE_DEC_GU_CTAS; // gate_up: CTAs per SM the registers are sized for
 constexpr int kGuGroups = MOE_DEC_GROUPS;
 constexpr int kGuMaxStages = MOE_DEC_STAGES;
 constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
@@ -174,12 +182,12 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // wait.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __launch_bounds__(kGuThreads, 1) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
     uint16_t* __restrict__ act, uint32_t* status, int S, Bank dn) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int G = kGuGroups, MT = kGuMT, CH = 2;
+  constexpr int G = kGuGroups, MT = kGuMT, CH = MT == 1 && NT == 1 ? 4 : 2;
   constexpr int kRed = kGroupWarps * NT * MT * 128;  // floats of one group's partial tiles
   const int K = gu.K, R = T * top_k;
   const GuLayout L = gu_layout(FMT, K);

@@ -48,7 +48,7 @@ constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BN = kGemmBN;    // token columns per tile (max MMA N)
 constexpr int BK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int SA_DEFAULT = 3;  // bf16 weight-operand stages (dequantised, or router weights by TMA)
-constexpr int SB = 4;          // gathered token-operand stages (copies signal their own arrival)
+constexpr int SB_DEFAULT = 4;  // gathered token-operand stages (copies signal their own arrival)
 constexpr int SC = 3;          // code stages
 constexpr int kThreads = 512;
 constexpr int kDqThreads = 256;           // dequantisation threads (warps 4-11)
@@ -57,6 +57,7 @@ constexpr int kEpiWarp0 = 12;             // first epilogue warp
 // one E4M3 byte per 16 k and, to make room, one bf16 operand stage less
 constexpr int kMaxScaleRow = 64;
 constexpr int kMaxScaleRowNv = 128;
+constexpr int kMaxScaleRowInt4 = 32;  // INT4: K <= 2048
 constexpr int kTileBytes = BM * BK * 2;   // 16 KB bf16 operand tile
 constexpr int kCodeBytes = BM * BK / 2;   // 4 KB code tile
 
@@ -85,8 +86,14 @@ struct GemmArgs {
 template <int MODE, int FMT>
 struct Cfg {
   static constexpr bool NV_WIDE = FMT == MOE_FMT_NVFP4_G16 && MODE == kGateUp;
-  static constexpr int SA = NV_WIDE ? SA_DEFAULT - 1 : SA_DEFAULT;
-  static constexpr int SROW = FMT == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv : kMaxScaleRow;
+  // Four weight-operand stages where shared memory allows (INT4 gate_up,
+  // down), one token stage less: the dequantisation of a stage waits for the
+  // tensor core to release the stage SA back, so SA covers the MMAs' latency.
+  static constexpr bool DEEP = MODE == kDown || (MODE == kGateUp && FMT == MOE_FMT_INT4_G128);
+  static constexpr int SA = NV_WIDE ? SA_DEFAULT - 1 : DEEP ? SA_DEFAULT + 1 : SA_DEFAULT;
+  static constexpr int SB = DEEP ? SB_DEFAULT - 1 : SB_DEFAULT;
+  static constexpr int SROW = FMT == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv
+                              : FMT == MOE_FMT_INT4_G128 ? kMaxScaleRowInt4 : kMaxScaleRow;
   static constexpr int NACC = MODE == kGateUp ? 2 : 1;                 // accumulators per tile
   static constexpr uint32_t TMEM_COLS = MODE == kGateUp ? 512 : 256;   // 2 buffers x NACC x BN
   static constexpr int SMEM_A = SA * NACC * kTileBytes;
@@ -245,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const GemmArgs args) {
   using C = Cfg<MODE, FMT>;
   constexpr int SA = C::SA;
+  constexpr int SB = C::SB;
   constexpr int kSrow = C::SROW;
   constexpr int NACC = C::NACC;
   extern __shared__ uint8_t smem_raw[];
@@ -846,7 +854,8 @@ bool grouped_supported(const moe_shape_t& s) {
   const auto row_bytes = [&](int K) {
     return s.fmt == MOE_FMT_INT4_G128 ? 2 * int4_groups(K) : s.fmt == MOE_FMT_NVFP4_G16 ? K / 16 : K / 32;
   };
-  const int cap = s.fmt == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv : kMaxScaleRow;
+  const int cap = s.fmt == MOE_FMT_NVFP4_G16 ? kMaxScaleRowNv
+                  : s.fmt == MOE_FMT_INT4_G128 ? kMaxScaleRowInt4 : kMaxScaleRow;
   return row_bytes(s.hidden) <= cap && row_bytes(s.inter) <= cap;
 }
 
