@@ -41,8 +41,7 @@ namespace {
 constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
 
 // Build-time tuning knobs (the defaults are the measured best): gate_up
-// consumer groups per CTA and its largest stage ring; down warps per CTA;
-// gate_up unit size and CTAs per SM.
+// consumer groups per CTA and its largest stage ring; down warps per CTA.
 #ifndef MOE_DEC_GROUPS
 #define MOE_DEC_GROUPS 2
 #endif
@@ -52,15 +51,14 @@ constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
 #ifndef MOE_DEC_DN_WARPS
 #define MOE_DEC_DN_WARPS 8
 #endif
-#ifndef MOE_DEC_GU_MT
-#define MOE_DEC_GU_MT 2
-#endif
-#ifndef MOE_DEC_GU_CTAS
-#define MOE_DEC_GU_CTAS 1
-#endif
-constexpr int kGuMT = MOE_DEC_GU_MT;     // gate_up: 16-row MMA tiles per unit (8 features each)
-constexpr int kGuFeat = 8 * kGuMT;       // gate_up: features per unit (that many gate and up rows)
-constexpr int kGuCtas = MOE_DEC_GU_CTAS; // gate_up: CTAs per SM the registers are sized for
+// gate_up unit size and CTAs per SM by token tiles (NT): with one token tile,
+// 8-feature units (one 16-row MMA tile) and registers for two CTAs per SM,
+// so twice the warps hide the latency (measured faster); more token tiles
+// need the registers of one CTA per SM and share each activation fragment
+// between two MMA tiles (16-feature units).
+__host__ __device__ constexpr int gu_mt(int NT) { return NT == 1 ? 1 : 2; }
+__host__ __device__ constexpr int gu_feat(int NT) { return 8 * gu_mt(NT); }
+constexpr int gu_ctas(int NT) { return NT == 1 ? 2 : 1; }
 constexpr int kGuGroups = MOE_DEC_GROUPS;
 constexpr int kGuMaxStages = MOE_DEC_STAGES;
 constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
@@ -80,8 +78,8 @@ constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch 
 struct GuLayout {
   int cA, cB, sA, sB, stage_bytes;
 };
-__host__ __device__ inline GuLayout gu_layout(int fmt, int K) {
-  const int run = kGuFeat * (K / 2), srun = kGuFeat * scale_row_bytes(fmt, K);
+__host__ __device__ inline GuLayout gu_layout(int fmt, int K, int feat) {
+  const int run = feat * (K / 2), srun = feat * scale_row_bytes(fmt, K);
   GuLayout l;
   l.cA = 0;
   l.cB = run + 64;
@@ -182,15 +180,15 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // wait.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool X_SMEM>
-__global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
+__global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
     uint16_t* __restrict__ act, uint32_t* status, int S, Bank dn) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int G = kGuGroups, MT = kGuMT, CH = MT == 1 && NT == 1 ? 4 : 2;
+  constexpr int G = kGuGroups, MT = gu_mt(NT), FEAT = gu_feat(NT), CH = MT == 1 && NT == 1 ? 4 : 2;
   constexpr int kRed = kGroupWarps * NT * MT * 128;  // floats of one group's partial tiles
   const int K = gu.K, R = T * top_k;
-  const GuLayout L = gu_layout(FMT, K);
+  const GuLayout L = gu_layout(FMT, K, FEAT);
   const int srow = scale_row_bytes(FMT, K);
   const int pstride = staged_act_stride(K);
   uint8_t* ring = smem;                                                      // [S][stage]
@@ -226,7 +224,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
   int t_lo, t_hi;
   local_slice(s_touched, e_lo, e_hi, E, s_cnt, &t_lo, &t_hi);
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
-  const int ftiles = I / kGuFeat;
+  const int ftiles = I / FEAT;
   const int n_units = (t_hi - t_lo) * ftiles;
   const int u_begin = int(long(n_units) * blockIdx.x / gridDim.x);
   const int cnt = int(long(n_units) * (blockIdx.x + 1) / gridDim.x) - u_begin;
@@ -235,7 +233,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
     const uint64_t policy = l2_policy_evict_first();
-    const uint32_t run = uint32_t(kGuFeat * (K / 2)), srun = uint32_t(kGuFeat * srow);
+    const uint32_t run = uint32_t(FEAT * (K / 2)), srun = uint32_t(FEAT * srow);
     const uint8_t* scales = static_cast<const uint8_t*>(gu.scales);
     int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;                 // unit i
     int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
@@ -263,16 +261,16 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
       __syncwarp();
       if (lane < 4) {
         // lane 0 / 1: gate / up codes; lane 2 / 3: their scales
-        const long row = long(s_local[slot] - e_lo) * gu.N + ft * kGuFeat + ((lane & 1) ? I : 0);
+        const long row = long(s_local[slot] - e_lo) * gu.N + ft * FEAT + ((lane & 1) ? I : 0);
         uint8_t* stage = ring + size_t(st) * L.stage_bytes;
         if (lane < 2) bulk_g2s_hint(stage + (lane ? L.cB : L.cA), gu.codes + row * (K / 2), run, &full[st], policy);
         else bulk_g2s_hint(stage + (lane & 1 ? L.sB : L.sA), scales + row * srow, srun, &full[st], policy);
       } else if (lane < 8) {
         if (i + S < cnt) {
           // the unit that will refill this stage, into L2 ahead of time
-          const long row = long(s_local[pslot] - e_lo) * gu.N + pft * kGuFeat + ((lane & 1) ? I : 0);
-          if (lane < 6) prefetch_codes<FMT>(gu, row, kGuFeat);
-          else prefetch_scales<FMT>(gu, row, kGuFeat);
+          const long row = long(s_local[pslot] - e_lo) * gu.N + pft * FEAT + ((lane & 1) ? I : 0);
+          if (lane < 6) prefetch_codes<FMT>(gu, row, FEAT);
+          else prefetch_scales<FMT>(gu, row, FEAT);
         }
       } else if (lane < 12 && i >= S) {
         prefetch_down(pf_next + lane - 8);  // once the ring is primed: four pieces per unit
@@ -304,7 +302,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtas) decode_gate_up_kernel(
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, &s_abort, status));
     const int e = s_local[slot];
     const int p0 = s_off[e], n_e = s_off[e + 1] - p0;
-    const int f0 = ft * kGuFeat;
+    const int f0 = ft * FEAT;
     const uint8_t* s_c = ring + size_t(st) * L.stage_bytes;
     const uint8_t* c_lo[MT];
     const uint8_t* c_hi[MT];
@@ -572,6 +570,8 @@ __global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
 int max_touched(int T, int k, int E) { return (long(T) * k < E) ? T * k : E; }
 
 constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving room for static
+constexpr size_t kSmemPerSm = 228 * 1024;       // shared memory of one SM
+constexpr size_t kSmemReservedPerCta = 2 * 1024;  // the system's share per CTA and the kernels' static arrays
 // Staged token rows (gate_up) and activation rows (down) up to these sizes.
 constexpr size_t kMaxStagedX = 72 * 1024;
 constexpr size_t kMaxStagedAct = 160 * 1024;
@@ -581,8 +581,8 @@ int nt_of(int T) { return T <= 8 ? 1 : T <= 16 ? 2 : 4; }
 // gate_up: stages + staged token rows + the partial-tile buffers + routing
 // state + barriers
 size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows, int S) {
-  return size_t(S) * gu_layout(fmt, K).stage_bytes + size_t(x_rows) * staged_act_stride(K) +
-         size_t(kGuGroups) * 2 * kGroupWarps * NT * kGuMT * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 +
+  return size_t(S) * gu_layout(fmt, K, gu_feat(NT)).stage_bytes + size_t(x_rows) * staged_act_stride(K) +
+         size_t(kGuGroups) * 2 * kGroupWarps * NT * gu_mt(NT) * 128 * 4 + size_t(2 * (E + 1) + R) * 4 + 8 +
          2 * size_t(S) * 8;
 }
 
@@ -609,12 +609,17 @@ GuPlan gate_up_plan(const moe_shape_t& s, int T) {
   p.x_smem = size_t(T) * staged_act_stride(s.hidden) <= kMaxStagedX;
   p.S = 0;
   p.smem = 0;
-  for (int S = kGuMaxStages / kGuGroups * kGuGroups; S >= 2 * kGuGroups; S -= kGuGroups) {
-    const size_t b = gate_up_smem(s.fmt, s.hidden, NT, s.num_experts, R, p.x_smem ? T : 0, S);
-    if (b <= kMaxSmemPerCta) {
-      p.S = S;
-      p.smem = b;
-      break;
+  // the largest ring that leaves room for gu_ctas(NT) CTAs per SM, else the
+  // largest that fits one CTA
+  const size_t shared_budget = kSmemPerSm / gu_ctas(NT) - kSmemReservedPerCta;
+  for (size_t budget : {std::min(shared_budget, kMaxSmemPerCta), kMaxSmemPerCta}) {
+    for (int S = kGuMaxStages / kGuGroups * kGuGroups; S >= 2 * kGuGroups; S -= kGuGroups) {
+      const size_t b = gate_up_smem(s.fmt, s.hidden, NT, s.num_experts, R, p.x_smem ? T : 0, S);
+      if (b <= budget) {
+        p.S = S;
+        p.smem = b;
+        return p;
+      }
     }
   }
   return p;
@@ -732,7 +737,8 @@ bool decode_supported(const moe_shape_t& s, int T) {
 
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
                                   const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
-  const int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / kGuFeat);
+  const int units =
+      std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / gu_feat(nt_of(T)));
   if (units <= 0) return cudaSuccess;
   Bank pf = dn;
   if (s.hidden % kDnPrefetchRows) pf.codes = nullptr;  // whole pieces only
