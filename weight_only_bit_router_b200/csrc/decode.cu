@@ -68,8 +68,11 @@ constexpr int kDnRows = 16;  // output features per down tile
 // registers per down thread: up to 8 tokens, room on the SM for the next
 // layer's routing kernel (256 threads x 80) while down CTAs drain; more
 // token tiles need more (two warps per SM sub-partition: at most 255)
-constexpr int kDnRegs = 160;
-constexpr int kDnRegsWide = 224;
+constexpr int kDnRegs = kDnWarps > 8 ? 128 : 160;
+constexpr int kDnRegsWide = kDnWarps > 8 ? 128 : 224;
+// With more than 8 warps the registers hold one chunk per warp (the next
+// chunk's loads are not in flight during the multiply; other warps hide them)
+constexpr bool kDnOneChunk = kDnWarps > 8;
 constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
 constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch issued by gate_up
 
@@ -552,13 +555,20 @@ __global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
             for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
         }
       };
-      for (int k = 0; k < nk;) {
-        if (k + 1 < nk) load(cB, tile, k + 1);
-        step(cA, k);
-        if (++k >= nk) break;
-        if (k + 1 < nk) load(cA, tile, k + 1);
-        step(cB, k);
-        ++k;
+      if (kDnOneChunk) {
+        for (int k = 0; k < nk; ++k) {
+          if (k > 0) load(cA, tile, k);
+          step(cA, k);
+        }
+      } else {
+        for (int k = 0; k < nk;) {
+          if (k + 1 < nk) load(cB, tile, k + 1);
+          step(cA, k);
+          if (++k >= nk) break;
+          if (k + 1 < nk) load(cA, tile, k + 1);
+          step(cB, k);
+          ++k;
+        }
       }
       finish_tile(tile);
     }
