@@ -20,10 +20,10 @@
 // touched experts, so the routing-weighted combine of a token's k expert
 // outputs happens in the CTA (in slot order, deterministic) and the output is
 // written once.  Its 16-row weight tiles are small (16 rows x I/2 bytes), so
-// each warp loads its tiles straight into registers, the next tile's loads in
-// flight while the current one is multiplied, all of its tiles requested
-// into L2 up front, and the first tile's loads issued before the
-// programmatic-launch wait.
+// each warp loads its tiles straight into registers (16 warps per CTA with
+// one chunk each up to 8 tokens; 8 warps with the next chunk's loads in
+// flight during the multiply above), the first chunk's loads issued before
+// the programmatic-launch wait; gate_up has requested the tiles into L2.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -41,15 +41,12 @@ namespace {
 constexpr int kGroupWarps = 4;  // gate_up: consumer warps per work unit
 
 // Build-time tuning knobs (the defaults are the measured best): gate_up
-// consumer groups per CTA and its largest stage ring; down warps per CTA.
+// consumer groups per CTA and its largest stage ring.
 #ifndef MOE_DEC_GROUPS
 #define MOE_DEC_GROUPS 2
 #endif
 #ifndef MOE_DEC_STAGES
 #define MOE_DEC_STAGES 4
-#endif
-#ifndef MOE_DEC_DN_WARPS
-#define MOE_DEC_DN_WARPS 8
 #endif
 // gate_up unit size and CTAs per SM by token tiles (NT): with one token tile,
 // 8-feature units (one 16-row MMA tile) and registers for two CTAs per SM,
@@ -62,17 +59,15 @@ constexpr int gu_ctas(int NT) { return NT == 1 ? 2 : 1; }
 constexpr int kGuGroups = MOE_DEC_GROUPS;
 constexpr int kGuMaxStages = MOE_DEC_STAGES;
 constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
-constexpr int kDnWarps = MOE_DEC_DN_WARPS;
-constexpr int kDnThreads = kDnWarps * 32;
 constexpr int kDnRows = 16;  // output features per down tile
-// registers per down thread: up to 8 tokens, room on the SM for the next
-// layer's routing kernel (256 threads x 80) while down CTAs drain; more
-// token tiles need more (two warps per SM sub-partition: at most 255)
-constexpr int kDnRegs = kDnWarps > 8 ? 128 : 160;
-constexpr int kDnRegsWide = kDnWarps > 8 ? 128 : 224;
-// With more than 8 warps the registers hold one chunk per warp (the next
-// chunk's loads are not in flight during the multiply; other warps hide them)
-constexpr bool kDnOneChunk = kDnWarps > 8;
+// down warps per CTA by token tiles: with one token tile 16 warps, each
+// holding one register chunk (the other warps hide its loads; measured 6 %
+// faster than 8 warps with two chunks each); more token tiles need the
+// registers of 8 warps, each with the next chunk's loads in flight during
+// the multiply.
+constexpr int dn_warps(int NT) { return NT == 1 ? 16 : 8; }
+constexpr int dn_threads(int NT) { return 32 * dn_warps(NT); }
+constexpr int dn_regs(int NT) { return NT == 1 ? 128 : 224; }  // at most 65536 / threads, 8-aligned
 constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
 constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch issued by gate_up
 
@@ -412,13 +407,14 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
 // T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
+__global__ void __maxnreg__(dn_regs(NT)) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
     const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
     uint16_t* __restrict__ out, float* __restrict__ partial_out) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int W = kDnWarps;
+  constexpr int W = dn_warps(NT), kThreads = dn_threads(NT);
+  constexpr bool kOneChunk = W > 8;
   constexpr int CH = NT == 1 ? 4 : 2;
   const int H = dn.N, K = dn.K;  // K = I
   const int R = T * top_k;
@@ -457,7 +453,7 @@ __global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
   // then cleared for the next tile)
   auto finish_tile = [&](int tile) {
     __syncthreads();
-    for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kDnThreads) {
+    for (int o = threadIdx.x; o < T * (kDnRows / 2); o += kThreads) {
       const int t = o / (kDnRows / 2), f = 2 * (o % (kDnRows / 2));
       float v0 = 0.f, v1 = 0.f;
       for (int j = 0; j < top_k; ++j) {
@@ -505,7 +501,7 @@ __global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
     pdl_wait();  // the activations (and the previous readers of the output) of the kernels before
     pdl_trigger();
     if (ACT_SMEM) {
-      stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kDnThreads);
+      stage_act_rows<2>(act_s, act, R, K, threadIdx.x, kThreads);
       __syncthreads();
     }
     for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
@@ -555,7 +551,7 @@ __global__ void __maxnreg__(NT == 1 ? kDnRegs : kDnRegsWide) decode_down_kernel(
             for (int c = 0; c < 4; ++c) acc[j][h][c] = 0.f;
         }
       };
-      if (kDnOneChunk) {
+      if (kOneChunk) {
         for (int k = 0; k < nk; ++k) {
           if (k > 0) load(cA, tile, k);
           step(cA, k);
@@ -723,8 +719,8 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRan
   auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
   cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, kDnThreads);
-  return launch_pdl(k, dim3(grid), dim3(kDnThreads), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
+  const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, dn_threads(NT));
+  return launch_pdl(k, dim3(grid), dim3(dn_threads(NT)), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
                     (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out);
 }
