@@ -611,7 +611,7 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   const int perm = (long(T) * shape->top_k <= 1024) ? 1 : 3;
   int n = 0;
   if (routed) n += perm;
-  else if (T <= kDecodeMaxT) n += 1;                          // fused router + top-k + permutation
+  else if (T <= kDecodeMaxT) n += route_small_launches(T, shape->hidden, shape->num_experts, shape->top_k);
   else n += 2 + perm;                                         // router GEMM, top-k, permutation
   n += decode ? 2 : 3;  // gate_up, down (+ combine / finalize for the grouped GEMMs)
   return n;

@@ -58,7 +58,7 @@ constexpr size_t kStatusBytes = 4096;
 
 struct Workspace {
   uint32_t* status;       // status word (device-side failures)
-  int32_t* route_counter; // CTAs done in the fused small-batch routing kernel
+  int32_t* route_counter; // CTAs done in the one-kernel small-batch routing (shapes outside the split-K form)
   float* logits;          // [T, E]
   int32_t* topk_ids;      // [T, k]
   float* topk_w;          // [T, k]
@@ -90,11 +90,15 @@ cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, i
                            cudaStream_t stream);
 
 // route.cu
-// Fused router GEMV + top-k + permutation for T <= kDecodeMaxT.
+// Router GEMV + top-k + permutation for T <= kDecodeMaxT: split-K GEMV then
+// a one-CTA finalize kernel, or one kernel for other shapes.
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream);
 // split-K partial logits of the small-batch routing kernel (0 when it does not apply)
 size_t route_part_bytes(int T, int H, int E, int k);
+// kernels launch_route_small launches: 2 (split-K GEMV + finalize) where the
+// split-K form applies, else 1
+int route_small_launches(int T, int H, int E, int k);
 cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t stream);
 // Small-T permutation (R = T*k <= 1024) in one CTA, with the touched-expert

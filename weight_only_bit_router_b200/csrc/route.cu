@@ -367,14 +367,15 @@ __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Fused small-batch routing, split-K (T <= 32, E <= 256, k <= 8).  CTA
-// (tile, s) computes, with mma.sync, the partial logits of experts
-// [16 tile, 16 tile + 16) over k in [256 s, 256 s + 256) for every token and
-// stores them; spreading the router weight over (E/16) x (H/256) CTAs keeps
-// every SM's share of it small.  The last CTA to finish (device counter) sums
-// the partials in split order (deterministic), keeps the logits in shared
-// memory, runs the merge top-k (one warp per token) and the stable
-// permutation with the whole block.
+// Small-batch routing, split-K (T <= 32, E <= 256, k <= 8), two kernels.
+// route_gemv_kernel: CTA (tile, s) computes, with mma.sync, the partial
+// logits of experts [16 tile, 16 tile + 16) over k in [256 s, 256 s + 256)
+// for every token and stores them; spreading the router weight over
+// (E/16) x (H/256) CTAs keeps every SM's share of it small.
+// route_finalize_kernel (one CTA, launched behind it and waiting at its
+// launch wait): sums the partials in split order (deterministic), keeps the
+// logits in shared memory, runs the top-k (one warp per token) and the
+// stable permutation with the whole block.
 // ---------------------------------------------------------------------------
 constexpr int kRfK = 256;  // k per CTA
 constexpr int kRfMaxT = 32, kRfMaxE = 256, kRfMaxR = kRfMaxT * 8;
@@ -546,23 +547,22 @@ __device__ void warp_permutation_32(RouteFastSmem& sm, int R, int E, int32_t* __
   }
 }
 
+// The split-K router GEMV of the small-batch routing: CTA (tile, s) stores the
+// partial logits of experts [16 tile, 16 tile + 16) over k in
+// [256 s, 256 s + 256) for every token.  The router weight does not depend on
+// the kernels before, so its fragments are loaded before the launch wait.
 template <int NT>
-__global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
-    int E, int k, float* __restrict__ logits, float* __restrict__ part, int32_t* __restrict__ ids,
-    float* __restrict__ wout, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows,
-    int32_t* __restrict__ pos, int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n,
-    int32_t* done_counter) {
-  __shared__ RouteFastSmem sm;
+__global__ void __launch_bounds__(kRsThreads) route_gemv_kernel(const uint16_t* __restrict__ x,
+                                                                const uint16_t* __restrict__ wr, int T, int H,
+                                                                int E, float* __restrict__ part) {
+  __shared__ float red[kRsWarps][4][32];  // one C fragment per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int e0 = blockIdx.x * kRsExperts, ks = blockIdx.y, KS = gridDim.y;
+  const int e0 = blockIdx.x * kRsExperts, ks = blockIdx.y;
   // warp: k-block b of this split, token tile jt
   const int b = warp & 1, jt = warp >> 1;
   const int kblk = ks * kRfK + b * 128 + 32 * q;
   const bool kin = kblk < H;
-  // the router weight does not depend on the kernels before: its fragments
-  // are loaded before the programmatic-launch wait
   uint32_t alo[8][2], ahi[8][2];
   if (jt < NT) {
     const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
@@ -583,55 +583,53 @@ __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
     }
   }
 #pragma unroll
-  for (int c = 0; c < 4; ++c) sm.u.red[warp][c][lane] = acc[c];
+  for (int c = 0; c < 4; ++c) red[warp][c][lane] = acc[c];
   __syncthreads();
   if (b == 0 && jt < NT) {
     // this CTA's partial logits of token tile jt: the two k-blocks in order
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const float v = sm.u.red[warp][c][lane] + sm.u.red[warp + 1][c][lane];
+      const float v = red[warp][c][lane] + red[warp + 1][c][lane];
       // c0, c1: expert e0+g, tokens 2q, 2q+1; c2, c3: expert e0+g+8
       const int t = jt * 8 + 2 * q + (c & 1);
       const int e = e0 + g + ((c >> 1) << 3);
       if (t < T && e < E) part[(size_t(ks) * T + t) * E + e] = v;
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    sm.last = atomicAdd(done_counter, 1) == int(gridDim.x * gridDim.y) - 1;
-  }
-  __syncthreads();
-  if (!sm.last) return;
-  __threadfence();
-  // logits = sum of the split partials, in split order; four logits per
-  // thread-step, every split's load in flight at once (KS <= kRfMaxSplits)
+}
+
+// The rest of the small-batch routing in one CTA, after the GEMV kernel has
+// finished (its launch wait): logits = the split partials summed in split
+// order (deterministic), the top k per token (one warp per token) and the
+// stable permutation.  No device counter and no fences: the kernel boundary
+// orders the partials.
+__global__ void __launch_bounds__(kRsThreads) route_finalize_kernel(
+    const float* __restrict__ part, int KS, const float* __restrict__ bias, int T, int E, int k,
+    float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos, int32_t* __restrict__ touched,
+    int32_t* __restrict__ tile_base, int block_n) {
+  __shared__ RouteFastSmem sm;
+  const int warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  // four logits per thread-step, every split's load in flight at once
   const int n4 = T * E / 4;
   const float4* part4 = reinterpret_cast<const float4*>(part);
-  for (int i0 = threadIdx.x; i0 < n4; i0 += 2 * blockDim.x) {
-    float4 v[2][kRfMaxSplits];
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    float4 v[kRfMaxSplits];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int s2 = 0; s2 < kRfMaxSplits; ++s2)
+      v[s2] = s2 < KS ? __ldcg(part4 + size_t(s2) * n4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 sum = v[0];
 #pragma unroll
-      for (int s2 = 0; s2 < kRfMaxSplits; ++s2) {
-        const int idx = i0 + h * blockDim.x;
-        v[h][s2] = (s2 < KS && idx < n4) ? __ldcg(part4 + size_t(s2) * n4 + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int idx = i0 + h * blockDim.x;
-      if (idx >= n4) continue;
-      float4 sum = v[h][0];
-#pragma unroll
-      for (int s2 = 1; s2 < kRfMaxSplits; ++s2) {
-        sum.x += v[h][s2].x;
-        sum.y += v[h][s2].y;
-        sum.z += v[h][s2].z;
-        sum.w += v[h][s2].w;
-      }
-      reinterpret_cast<float4*>(sm.u.logit)[idx] = sum;
-      reinterpret_cast<float4*>(logits)[idx] = sum;
+    for (int s2 = 1; s2 < kRfMaxSplits; ++s2) {
+      sum.x += v[s2].x;
+      sum.y += v[s2].y;
+      sum.z += v[s2].z;
+      sum.w += v[s2].w;
     }
+    reinterpret_cast<float4*>(sm.u.logit)[i] = sum;
+    reinterpret_cast<float4*>(logits)[i] = sum;
   }
   __syncthreads();
   for (int t = warp; t < T; t += kRsWarps) warp_topk8(sm.u.logit + t * E, bias, E, k, sm.ids + t * k, wout + t * k);
@@ -643,7 +641,6 @@ __global__ void __launch_bounds__(kRsThreads) route_fast_kernel(
   } else {
     block_permutation_256(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
   }
-  if (threadIdx.x == 0) *done_counter = 0;  // ready for the next call
 }
 
 // ---------------------------------------------------------------------------
@@ -804,14 +801,19 @@ template <int NT>
 cudaError_t route_fast_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                           const Workspace& ws, int block_n, cudaStream_t stream) {
   const dim3 grid((E + kRsExperts - 1) / kRsExperts, (H + kRfK - 1) / kRfK);
-  return launch_pdl(route_fast_kernel<NT>, grid, dim3(kRsThreads), 0, stream, x, wr, bias, T, H, E, k, ws.logits,
-                    ws.route_part, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched,
-                    ws.tile_base, block_n, ws.route_counter);
+  cudaError_t err = launch_pdl(route_gemv_kernel<NT>, grid, dim3(kRsThreads), 0, stream, x, wr, T, H, E,
+                               ws.route_part);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(route_finalize_kernel, dim3(1), dim3(kRsThreads), 0, stream, (const float*)ws.route_part,
+                    int(grid.y), bias, T, E, k, ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows,
+                    ws.pos, ws.touched, ws.tile_base, block_n);
 }
 
 bool route_fast_applies(int T, int H, int E, int k) {
   return T <= kRfMaxT && E <= kRfMaxE && E % 4 == 0 && k <= 8 && H <= kRfMaxSplits * kRfK;
 }
+
+int route_small_launches(int T, int H, int E, int k) { return route_fast_applies(T, H, E, k) ? 2 : 1; }
 
 size_t route_part_bytes(int T, int H, int E, int k) {
   return route_fast_applies(T, H, E, k) ? size_t((H + kRfK - 1) / kRfK) * T * E * sizeof(float) : 0;
