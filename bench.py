@@ -82,8 +82,13 @@ KERNEL_SOURCES = {
     "grouped": ("gemm_sm100.cu", "common.cuh", "internal.h"),
 }
 # DRAM bytes (read + write) per launch of a workload's dominant kernel from one
-# ncu capture: (workload, kernel) -> (bytes, kernel family, digest of its sources)
-MEASURED_TRAFFIC = {}
+# ncu capture: (workload, kernel) -> (bytes, kernel family, digest of its sources).
+# decode4 gate_up: 47.16 MB read + 0.02 MB written (2-layer stack, the same
+# per-layer work): its 32.5 MB of packed gate_up rows and the 16.3 MB of down
+# matrices it requests into L2 for the down kernel (moved earlier, not re-read).
+MEASURED_TRAFFIC = {
+    ("decode4", "gate_up"): (47_178_496, "decode", "257215440c35ab63"),
+}
 
 
 # ---------------------------------------------------------------- distributed plumbing

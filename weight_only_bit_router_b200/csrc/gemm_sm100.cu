@@ -177,6 +177,15 @@ constexpr uint32_t kEpilogueSleepNs = 256;
 // The MMA issuer waits on the dequantisation warps most of the time; a short
 // sleep between its tries keeps its polls from taking their issue slots.
 constexpr uint32_t kMmaSleepNs = 32;
+// The dequantisation warps' waits (code tiles landed, weight stage free):
+// a build-time tuning knob, 0 = plain tries with the suspend hint.
+#ifndef MOE_GEMM_DQ_SLEEP_NS
+#define MOE_GEMM_DQ_SLEEP_NS 0
+#endif
+MOE_DEV bool dq_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* gstatus) {
+  return MOE_GEMM_DQ_SLEEP_NS > 0 ? mbar_wait_backoff(bar, parity, abort, gstatus, MOE_GEMM_DQ_SLEEP_NS)
+                                  : mbar_wait(bar, parity, abort, gstatus);
+}
 
 // Code tiles this many k-stages ahead of the producer are prefetched into L2.
 constexpr int kCodePrefetch = 8;
@@ -529,13 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f = t.fb * BM + r;
         const bool valid = f < a.M_total;
         const int slot = it & 1;
-        if (!(ok = mbar_wait(&sc_full[slot], (it >> 1) & 1, abort, a.status))) break;
+        if (!(ok = dq_wait(&sc_full[slot], (it >> 1) & 1, abort, a.status))) break;
         const uint8_t* srows = sS + slot * NACC * BM * kSrow + r * sb;
         const float gsc = FMT == MOE_FMT_NVFP4_G16 ? a.gscale[t.eb] : 0.f;
         for (int ks = 0; ks < KS; ++ks, ++g) {
           const int sc = g % SC, so = g % SA;
-          if (!(ok = mbar_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
-          if (!(ok = mbar_wait(&opA_empty[so], ((g / SA) & 1) ^ 1, abort, a.status))) break;
+          if (!(ok = dq_wait(&codes_full[sc], (g / SC) & 1, abort, a.status))) break;
+          if (!(ok = dq_wait(&opA_empty[so], ((g / SA) & 1) ^ 1, abort, a.status))) break;
 #pragma unroll
           for (int c = 0; c < NACC; ++c) {
             const uint8_t* ctile = sC + (sc * NACC + c) * kCodeBytes + r * (BK / 2);
