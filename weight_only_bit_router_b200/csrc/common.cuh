@@ -447,14 +447,6 @@ MOE_DEV void red_add_u32(uint32_t* addr, uint32_t v) {
 MOE_DEV void red_add_f32(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
-// Four consecutive fp32 additions into global memory (addr 16-byte aligned).
-MOE_DEV void red_add_v4_f32(float* addr, float4 v) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-               : "memory");
-}
-
-// Prefetch the 128-byte line holding p into L1 (a later load of it hits L1).
-MOE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 MOE_DEV uint4 ldg_nc_v4(const void* p) {
   uint4 r;

@@ -495,20 +495,6 @@ __global__ void __maxnreg__(dn_regs(NT)) decode_down_kernel(
       const uint8_t* s_lo = scales + r * srow;
       load_chunk<FMT, FULL>(c, c_lo, c_lo + 8 * (K / 2), s_lo, s_lo + 8 * srow, 4 * ch, nblk, K, q);
     };
-    // the lines of chunk k into L1 (lanes q = 0, 2 take the two 128-byte
-    // lines of their rows' four blocks; lane q = 1 the rows' scales)
-    auto prefetch = [&](int tile, int k) {
-      const int m = nch == 1 ? k : k / nch, ch = k - m * nch;
-      const long r = long(s_local[warp + W * m] - e_lo) * H + tile * kDnRows + g;
-      const uint8_t* c_lo = dn.codes + r * (K / 2) + 256 * ch;
-      if ((q & 1) == 0 && 256 * ch + 64 * q < K / 2) {
-        prefetch_l1(c_lo + 64 * q);
-        prefetch_l1(c_lo + 8 * (K / 2) + 64 * q);
-      } else if (q == 1) {
-        prefetch_l1(scales + r * srow);
-        prefetch_l1(scales + (r + 8) * srow);
-      }
-    };
     RegChunk cA, cB;
     if (nk > 0 && blockIdx.x < ntile) load(cA, blockIdx.x, 0);
 
@@ -568,7 +554,6 @@ __global__ void __maxnreg__(dn_regs(NT)) decode_down_kernel(
       if (kOneChunk) {
         for (int k = 0; k < nk; ++k) {
           if (k > 0) load(cA, tile, k);
-          if (k + 1 < nk) prefetch(tile, k + 1);  // in L1 by the time it is loaded
           step(cA, k);
         }
       } else {

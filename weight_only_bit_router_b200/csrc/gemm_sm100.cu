@@ -640,27 +640,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       if (MODE == kDown) {
-        // every row of the weighted tile is staged
+        // every row of the weighted tile is staged: one bulk add per token
         fence_proxy_async_smem();
         named_barrier_sync(1, 128);
-        const int rows = min(BM, a.M_total - t.fb * BM);
-        if (a.ypart) {
-          // the row's own slot of the per-row outputs (summed in slot order
-          // later): one bulk copy per token
-          if (r < t.n) {
+        if (r < t.n) {
+          const int rows = min(BM, a.M_total - t.fb * BM);
+          if (a.ypart) {
+            // the row's own slot of the per-row outputs: summed in slot order later
             bulk_s2g(a.ypart + size_t(t.p_begin + r) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
-            bulk_commit_group();
+          } else {
+            const int tok = a.sorted_rows[t.p_begin + r] / a.top_k;
+            bulk_reduce_add_f32(a.out_acc + size_t(tok) * a.H + t.fb * BM, sD + r * BM, uint32_t(rows * 4));
           }
-        } else {
-          // added into the fp32 output: one warp per token row, 16 bytes a
-          // lane (vector reductions through L2; the bulk-copy engine's cost
-          // per copy made one bulk reduction per token row the bound)
-          for (int tt = ew; tt < t.n; tt += 4) {
-            const int tok = a.sorted_rows[t.p_begin + tt] / a.top_k;
-            for (int c = 4 * lane; c < rows; c += 128)
-              red_add_v4_f32(a.out_acc + size_t(tok) * a.H + t.fb * BM + c,
-                             *reinterpret_cast<const float4*>(sD + tt * BM + c));
-          }
+          bulk_commit_group();
         }
       }
     }
