@@ -384,8 +384,7 @@ constexpr int kRfMaxSplits = 8;  // H <= 8 * kRfK
 struct __align__(16) RouteFastSmem {
   union __align__(16) {
     float red[kRsWarps][4][32];                // GEMV: one C fragment per warp
-    float red4[kRsWarps][4][4][32];            // cluster GEMV: a warp's C fragments of up to 4 token tiles
-    float logit[kRfMaxT * kRfMaxE];             // finalize: summed logits [T][E]
+    float logit[kRfMaxT * kRfMaxE];             // last CTA: summed logits [T][E]
   } u;
   int ids[kRfMaxR];
   int rank[kRfMaxR];
@@ -644,128 +643,6 @@ __global__ void __launch_bounds__(kRsThreads) route_finalize_kernel(
   }
 }
 
-// Small-batch routing in one thread-block cluster (T <= 32, E <= 256,
-// k <= 8): no second kernel, no device counter.  CTA c of the cluster (C =
-// ceil(E/32) CTAs) computes the full logits of experts [32c, 32c + 32) for
-// every token: warp w takes MMA tile w % 2 (16 experts) and the 128-k blocks
-// w / 2, w / 2 + 4, ..., and the four k-warps of a tile are summed in warp
-// order.  After a cluster barrier, CTA 0 gathers the C CTAs' logits through
-// distributed shared memory, releases the others with a second barrier, and
-// selects the top k per token (one warp per token) and builds the stable
-// permutation.  The router weight does not depend on the kernels before: the
-// first k-block's fragments are loaded before the launch wait.
-constexpr int kRcExperts = 32;  // experts per cluster CTA
-constexpr int kRcMaxCtas = 8;   // portable cluster size: E <= 256
-
-MOE_DEV uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-MOE_DEV void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-// fp32 at shared address `local` of CTA `rank` of the cluster
-MOE_DEV float ld_cluster_f32(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
-template <int NT>
-__global__ void __launch_bounds__(kRsThreads) route_cluster_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const float* __restrict__ bias, int T, int H,
-    int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_rows, int32_t* __restrict__ pos,
-    int32_t* __restrict__ touched, int32_t* __restrict__ tile_base, int block_n) {
-  __shared__ RouteFastSmem sm;
-  __shared__ __align__(16) float s_mine[kRfMaxT][kRcExperts];  // this CTA's logits [t][expert - e0]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, q = lane & 3;
-  const uint32_t rank = cluster_ctarank();
-  const int mt = warp & 1, kw = warp >> 1;
-  const int e0 = int(rank) * kRcExperts + 16 * mt;
-  const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
-  const uint16_t* wlo = wr + size_t(r_lo ? e0 + g : 0) * H;
-  const uint16_t* whi = wr + size_t(r_hi ? e0 + g + 8 : 0) * H;
-  const int nblk = (H + 127) / 128;
-  float acc[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
-  uint32_t alo[8][2], ahi[8][2];
-  if (kw < nblk) {
-    const int kk = kw * 128 + 32 * q;
-    bf16_frags(wlo + kk, r_lo && kk < H, alo);
-    bf16_frags(whi + kk, r_hi && kk < H, ahi);
-  }
-  pdl_wait();
-  pdl_trigger();
-  for (int b = kw; b < nblk; b += 4) {
-    const int kk = b * 128 + 32 * q;
-    const bool kin = kk < H;  // H is a multiple of 64: a last half block
-    if (b != kw) {
-      bf16_frags(wlo + kk, r_lo && kin, alo);
-      bf16_frags(whi + kk, r_hi && kin, ahi);
-    }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int t = j * 8 + g;
-      uint32_t bf[8][2];
-      bf16_frags(x + size_t(t < T ? t : 0) * H + kk, t < T && kin, bf);
-#pragma unroll
-      for (int st = 0; st < 8; ++st) {
-        const uint32_t a[4] = {alo[st][0], ahi[st][0], alo[st][1], ahi[st][1]};
-        mma_16816(acc[j], a, bf[st][0], bf[st][1]);
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) sm.u.red4[warp][j][c][lane] = acc[j][c];
-  __syncthreads();
-  // warps 0 and 1 (tiles 0, 1): the tile's four k-warps summed in order
-  if (warp < 2) {
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v = sm.u.red4[warp][j][c][lane];
-#pragma unroll
-        for (int w = 1; w < 4; ++w) v += sm.u.red4[warp + 2 * w][j][c][lane];
-        // c0, c1: expert row g at tokens 2q, 2q+1; c2, c3: row g + 8
-        const int t = j * 8 + 2 * q + (c & 1);
-        if (t < T) s_mine[t][16 * warp + g + ((c >> 1) << 3)] = v;
-      }
-  }
-  cluster_sync_all();  // every CTA's logits are in its shared memory
-  if (rank == 0) {
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
-      const int t = i / E, e = i - t * E;
-      const float v = ld_cluster_f32(&s_mine[t][e % kRcExperts], uint32_t(e / kRcExperts));
-      sm.u.logit[i] = v;
-      logits[i] = v;
-    }
-  }
-  cluster_sync_all();  // CTA 0 has read the others' shared memory: they may exit
-  if (rank != 0) return;
-  __syncthreads();
-  for (int t = warp; t < T; t += kRsWarps) warp_topk8(sm.u.logit + t * E, bias, E, k, sm.ids + t * k, wout + t * k);
-  __syncthreads();
-  const int R = T * k;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) ids[r] = sm.ids[r];
-  if (R <= 32) {
-    if (warp == 0) warp_permutation_32(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
-  } else {
-    block_permutation_256(sm, R, E, offsets, sorted_rows, pos, touched, tile_base, block_n);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Large permutation, any R.  Blocks of 256 rows.
 // K1: per-block histogram + stable rank of each row inside its block.
@@ -920,29 +797,6 @@ cudaError_t route_small_nt(const uint16_t* x, const uint16_t* wr, const float* b
 #undef MOE_ROUTE_SMALL
 }
 
-// One cluster of ceil(E/32) CTAs, programmatic launch.
-template <int NT>
-cudaError_t route_cluster_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                             const Workspace& ws, int block_n, cudaStream_t stream) {
-  const int C = (E + kRcExperts - 1) / kRcExperts;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C);
-  cfg.blockDim = dim3(kRsThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(C);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, route_cluster_kernel<NT>, x, wr, bias, T, H, E, k, ws.logits, ws.topk_ids,
-                            ws.topk_w, ws.offsets, ws.sorted_rows, ws.pos, ws.touched, ws.tile_base, block_n);
-}
-
 template <int NT>
 cudaError_t route_fast_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                           const Workspace& ws, int block_n, cudaStream_t stream) {
@@ -959,14 +813,7 @@ bool route_fast_applies(int T, int H, int E, int k) {
   return T <= kRfMaxT && E <= kRfMaxE && E % 4 == 0 && k <= 8 && H <= kRfMaxSplits * kRfK;
 }
 
-// The cluster form: up to 8 CTAs of 32 experts each, k <= 8 (the warp top-k)
-bool route_cluster_applies(int T, int H, int E, int k) {
-  return T <= kRfMaxT && E <= kRcMaxCtas * kRcExperts && k <= 8 && H >= 64;
-}
-
-int route_small_launches(int T, int H, int E, int k) {
-  return route_cluster_applies(T, H, E, k) ? 1 : route_fast_applies(T, H, E, k) ? 2 : 1;
-}
+int route_small_launches(int T, int H, int E, int k) { return route_fast_applies(T, H, E, k) ? 2 : 1; }
 
 size_t route_part_bytes(int T, int H, int E, int k) {
   return route_fast_applies(T, H, E, k) ? size_t((H + kRfK - 1) / kRfK) * T * E * sizeof(float) : 0;
@@ -975,11 +822,6 @@ size_t route_part_bytes(int T, int H, int E, int k) {
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                                const Workspace& ws, int block_n, cudaStream_t stream) {
   const int nt = (T + 7) / 8;
-  if (route_cluster_applies(T, H, E, k)) {
-    if (nt <= 1) return route_cluster_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
-    if (nt <= 2) return route_cluster_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
-    return route_cluster_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
-  }
   if (route_fast_applies(T, H, E, k)) {
     if (nt <= 1) return route_fast_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
     if (nt <= 2) return route_fast_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
