@@ -9,13 +9,13 @@
 // per-expert row offsets, the rows' tokens) is read into shared memory once
 // per CTA.
 //
-// gate_up: persistent; CTA c takes a contiguous run of the (touched expert,
-// 16-feature) units.  One producer warp starts, per unit, two 16 KB-class
-// bulk copies (the 16 gate rows, the 16 up rows) and two of their scales into
-// a ring of shared-memory stages, and prefetches the unit that will next
-// refill the stage into L2; four consumer warps split each unit's k-blocks
-// and sum in shared memory.  Few large copies: the bulk-copy engine's cost is
-// per copy as much as per byte.
+// gate_up: persistent; CTA c takes the (touched expert, 8- or 16-feature)
+// units c, c + grid, ....  One producer warp starts, per unit, two bulk
+// copies (the unit's gate rows, its up rows: contiguous 8-16 KB ranges) and
+// two of their scales into a ring of shared-memory stages, and prefetches the
+// unit that will next refill the stage into L2; four consumer warps split
+// each unit's k-blocks and sum in shared memory.  Few large copies: the
+// bulk-copy engine's cost is per copy as much as per byte.
 // down: CTA c owns 16 output features of every token and runs over all
 // touched experts, so the routing-weighted combine of a token's k expert
 // outputs happens in the CTA (in slot order, deterministic) and the output is
@@ -169,8 +169,8 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // MMA tile t (features f0 + 8t ..) takes feature f0 + 8t + g's gate row and up
 // row as its two MMA rows (low / high; swapped for odd g), so the C fragment
 // holds gate and up of the same feature and token: SwiGLU needs no shuffle.
-// CTA c takes units [c n / grid, (c + 1) n / grid); its i-th goes to stage
-// i % S and consumer group i % G.  The group's four warps split K (128-k
+// CTA c takes units c, c + grid, ...; its i-th goes to stage i % S and
+// consumer group i % G.  The group's four warps split K (128-k
 // blocks w, w + 4, ...), and one of them (rotating) sums the four partial
 // tiles in warp order and writes a = bf16(silu(gate) * up) to act[p][f] for
 // the expert's sorted rows p.  With X_SMEM (small T) the consumers first
@@ -224,17 +224,28 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   const int* s_local = s_touched + 1 + t_lo;  // the bank's touched experts (global ids)
   const int ftiles = I / FEAT;
   const int n_units = (t_hi - t_lo) * ftiles;
-  const int u_begin = int(long(n_units) * blockIdx.x / gridDim.x);
-  const int cnt = int(long(n_units) * (blockIdx.x + 1) / gridDim.x) - u_begin;
+  // CTA c takes units c, c + grid, ...: a popular expert's units spread over
+  // many CTAs (its extra token tiles are work the CTAs share)
+  const int grid = int(gridDim.x);
+  const int cnt = n_units > int(blockIdx.x) ? (n_units - int(blockIdx.x) + grid - 1) / grid : 0;
   if (cnt <= 0) return;
+  const int g_slot = grid / ftiles, g_ft = grid - g_slot * ftiles;  // a step of `grid` units
+  auto advance = [&](int& sl, int& f, int steps) {  // (slot, feature tile) `steps` x grid units on
+    for (int a = 0; a < steps; ++a) {
+      sl += g_slot;
+      f += g_ft;
+      if (f >= ftiles) f -= ftiles, ++sl;
+    }
+  };
 
   if (warp == G * kGroupWarps) {
     // ---------------------------------------------------------------- producer
     const uint64_t policy = l2_policy_evict_first();
     const uint32_t run = uint32_t(FEAT * (K / 2)), srun = uint32_t(FEAT * srow);
     const uint8_t* scales = static_cast<const uint8_t*>(gu.scales);
-    int slot = u_begin / ftiles, ft = u_begin - slot * ftiles;                 // unit i
-    int pslot = (u_begin + S) / ftiles, pft = (u_begin + S) - pslot * ftiles;  // unit i + S
+    int slot = int(blockIdx.x) / ftiles, ft = int(blockIdx.x) - slot * ftiles;  // unit i
+    int pslot = slot, pft = ft;                                                // unit i + S
+    advance(pslot, pft, S);
     // This CTA's share of the touched experts' down matrices into L2 for the
     // down kernel that follows: pieces of kDnPrefetchRows rows, the CTA's
     // j-th piece is piece blockIdx.x + j * grid.
@@ -275,8 +286,8 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
       }
       if (i >= S) pf_next += 4;
       if (++st == S) st = 0, ph ^= 1;
-      if (++ft == ftiles) ft = 0, ++slot;
-      if (++pft == ftiles) pft = 0, ++pslot;
+      advance(slot, ft, 1);
+      advance(pslot, pft, 1);
     }
     // the rest of the share, one piece per lane
     for (int j = pf_next + lane; blockIdx.x + j * int(gridDim.x) < dn_pieces; j += 32) prefetch_down(j);
@@ -293,7 +304,8 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   const int tail_b = ((K % 128) != 0 && nfull % kGroupWarps == wj) ? nfull : -1;
   const int lo_c = odd ? L.cB : L.cA, hi_c = odd ? L.cA : L.cB;
   const int lo_s = odd ? L.sB : L.sA, hi_s = odd ? L.sA : L.sB;
-  int slot = (u_begin + grp) / ftiles, ft = (u_begin + grp) - slot * ftiles;
+  int slot = int(blockIdx.x) / ftiles, ft = int(blockIdx.x) - slot * ftiles;
+  advance(slot, ft, grp);
   int st = grp, ph = 0;
   for (int i = grp, n = 0; i < cnt; i += G, ++n) {
     // warp-uniform: the MMAs below run only if every lane saw the data land
@@ -383,8 +395,7 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
     }
     st += G;
     if (st >= S) st -= S, ph ^= 1;
-    ft += G;
-    while (ft >= ftiles) ft -= ftiles, ++slot;
+    advance(slot, ft, G);
   }
 }
 
