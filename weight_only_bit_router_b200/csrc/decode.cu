@@ -65,9 +65,16 @@ constexpr int kDnRows = 16;  // output features per down tile
 // faster than 8 warps with two chunks each); more token tiles need the
 // registers of 8 warps, each with the next chunk's loads in flight during
 // the multiply.
-constexpr int dn_warps(int NT) { return NT == 1 ? 16 : 8; }
-constexpr int dn_threads(int NT) { return 32 * dn_warps(NT); }
-constexpr int dn_regs(int NT) { return NT == 1 ? 128 : 224; }  // at most 65536 / threads, 8-aligned
+#ifndef MOE_DEC_DN_WIDE_INT4
+#define MOE_DEC_DN_WIDE_INT4 0
+#endif
+constexpr int dn_warps(int NT, int FMT = 0) {
+  return NT == 1 || (MOE_DEC_DN_WIDE_INT4 && FMT == MOE_FMT_INT4_G128) ? 16 : 8;
+}
+constexpr int dn_threads(int NT, int FMT = 0) { return 32 * dn_warps(NT, FMT); }
+constexpr int dn_regs(int NT, int FMT = 0) {  // at most 65536 / threads, 8-aligned
+  return dn_warps(NT, FMT) == 16 ? 128 : 224;
+}
 constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
 constexpr int kDnPrefetchRows = 64;         // down-matrix rows per L2 prefetch issued by gate_up
 
@@ -418,13 +425,13 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
 // T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool ACT_SMEM>
-__global__ void __maxnreg__(dn_regs(NT)) decode_down_kernel(
+__global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
     const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
     uint16_t* __restrict__ out, float* __restrict__ partial_out) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int W = dn_warps(NT), kThreads = dn_threads(NT);
+  constexpr int W = dn_warps(NT, FMT), kThreads = dn_threads(NT, FMT);
   constexpr bool kOneChunk = W > 8;
   constexpr int CH = NT == 1 ? 4 : 2;
   const int H = dn.N, K = dn.K;  // K = I
@@ -730,8 +737,8 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRan
   auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
   cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, dn_threads(NT));
-  return launch_pdl(k, dim3(grid), dim3(dn_threads(NT)), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
+  const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, dn_threads(NT, FMT));
+  return launch_pdl(k, dim3(grid), dim3(dn_threads(NT, FMT)), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
                     (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out);
 }

@@ -612,24 +612,34 @@ __global__ void __launch_bounds__(kRsThreads) route_finalize_kernel(
   const int warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
-  // four logits per thread-step, every split's load in flight at once
+  // four logits per thread and position, two positions per step: every
+  // split's load of both in flight at once
   const int n4 = T * E / 4;
   const float4* part4 = reinterpret_cast<const float4*>(part);
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-    float4 v[kRfMaxSplits];
+  for (int i0 = threadIdx.x; i0 < n4; i0 += 2 * blockDim.x) {
+    float4 v[2][kRfMaxSplits];
 #pragma unroll
-    for (int s2 = 0; s2 < kRfMaxSplits; ++s2)
-      v[s2] = s2 < KS ? __ldcg(part4 + size_t(s2) * n4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 sum = v[0];
+    for (int h = 0; h < 2; ++h) {
+      const int i = i0 + h * blockDim.x;
 #pragma unroll
-    for (int s2 = 1; s2 < kRfMaxSplits; ++s2) {
-      sum.x += v[s2].x;
-      sum.y += v[s2].y;
-      sum.z += v[s2].z;
-      sum.w += v[s2].w;
+      for (int s2 = 0; s2 < kRfMaxSplits; ++s2)
+        v[h][s2] = (s2 < KS && i < n4) ? __ldcg(part4 + size_t(s2) * n4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    reinterpret_cast<float4*>(sm.u.logit)[i] = sum;
-    reinterpret_cast<float4*>(logits)[i] = sum;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = i0 + h * blockDim.x;
+      if (i >= n4) break;
+      float4 sum = v[h][0];
+#pragma unroll
+      for (int s2 = 1; s2 < kRfMaxSplits; ++s2) {
+        sum.x += v[h][s2].x;
+        sum.y += v[h][s2].y;
+        sum.z += v[h][s2].z;
+        sum.w += v[h][s2].w;
+      }
+      reinterpret_cast<float4*>(sm.u.logit)[i] = sum;
+      reinterpret_cast<float4*>(logits)[i] = sum;
+    }
   }
   __syncthreads();
   for (int t = warp; t < T; t += kRsWarps) warp_topk8(sm.u.logit + t * E, bias, E, k, sm.ids + t * k, wout + t * k);
