@@ -60,19 +60,14 @@ constexpr int kGuGroups = MOE_DEC_GROUPS;
 constexpr int kGuMaxStages = MOE_DEC_STAGES;
 constexpr int kGuThreads = (kGuGroups * kGroupWarps + 1) * 32;
 constexpr int kDnRows = 16;  // output features per down tile
-// down warps per CTA by token tiles: with one token tile 16 warps, each
-// holding one register chunk (the other warps hide its loads; measured 6 %
-// faster than 8 warps with two chunks each); more token tiles need the
-// registers of 8 warps, each with the next chunk's loads in flight during
-// the multiply.
-#ifndef MOE_DEC_DN_WIDE_INT4
-#define MOE_DEC_DN_WIDE_INT4 0
-#endif
-constexpr int dn_warps(int NT, int FMT = 0) {
-  return NT == 1 || (MOE_DEC_DN_WIDE_INT4 && FMT == MOE_FMT_INT4_G128) ? 16 : 8;
-}
-constexpr int dn_threads(int NT, int FMT = 0) { return 32 * dn_warps(NT, FMT); }
-constexpr int dn_regs(int NT, int FMT = 0) {  // at most 65536 / threads, 8-aligned
+// down warps per CTA: 16, each holding one register chunk (the other warps
+// hide a chunk's loads; with one token tile measured 6 % faster than 8 warps
+// with the next chunk's loads in flight, at 32 INT4 tokens 27 % faster);
+// MXFP4 / NVFP4 with more token tiles need the registers of 8 warps, each
+// with the next chunk in flight during the multiply.
+constexpr int dn_warps(int NT, int FMT) { return NT == 1 || FMT == MOE_FMT_INT4_G128 ? 16 : 8; }
+constexpr int dn_threads(int NT, int FMT) { return 32 * dn_warps(NT, FMT); }
+constexpr int dn_regs(int NT, int FMT) {  // at most 65536 / threads, 8-aligned
   return dn_warps(NT, FMT) == 16 ? 128 : 224;
 }
 constexpr uint32_t kProducerSleepNs = 64;  // gate_up producer: sleep between tries for a free stage
