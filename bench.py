@@ -83,11 +83,14 @@ KERNEL_SOURCES = {
 }
 # DRAM bytes (read + write) per launch of a workload's dominant kernel from one
 # ncu capture: (workload, kernel) -> (bytes, kernel family, digest of its sources).
-# decode4 gate_up: 47.16 MB read + 0.02 MB written (2-layer stack, the same
+# decode4 gate_up: 47.35 MB read + 0.04 MB written (2-layer stack, the same
 # per-layer work): its 32.5 MB of packed gate_up rows and the 16.3 MB of down
 # matrices it requests into L2 for the down kernel (moved earlier, not re-read).
+# prefill gate_up: 378.06 MB read + 57.60 MB written (packed bank, x rows
+# gathered per 128-row weight tile, activations out).
 MEASURED_TRAFFIC = {
-    ("decode4", "gate_up"): (47_178_496, "decode", "257215440c35ab63"),
+    ("decode4", "gate_up"): (47_384_576, "decode", "82eecb54cbdaf490"),
+    ("prefill", "gate_up"): (435_657_216, "grouped", "559eba8651574ef6"),
 }
 
 
