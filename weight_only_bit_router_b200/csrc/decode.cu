@@ -592,8 +592,11 @@ constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving
 constexpr size_t kSmemPerSm = 228 * 1024;       // shared memory of one SM
 constexpr size_t kSmemReservedPerCta = 2 * 1024;  // the system's share per CTA and the kernels' static arrays
 // Staged token rows (gate_up) and activation rows (down) up to these sizes.
+#ifndef MOE_DEC_MAX_STAGED_ACT_KB
+#define MOE_DEC_MAX_STAGED_ACT_KB 160
+#endif
 constexpr size_t kMaxStagedX = 72 * 1024;
-constexpr size_t kMaxStagedAct = 160 * 1024;
+constexpr size_t kMaxStagedAct = size_t(MOE_DEC_MAX_STAGED_ACT_KB) * 1024;
 
 int nt_of(int T) { return T <= 8 ? 1 : T <= 16 ? 2 : 4; }
 
