@@ -83,14 +83,14 @@ KERNEL_SOURCES = {
 }
 # DRAM bytes (read + write) per launch of a workload's dominant kernel from one
 # ncu capture: (workload, kernel) -> (bytes, kernel family, digest of its sources).
-# decode4 gate_up: 47.35 MB read + 0.04 MB written (2-layer stack, the same
+# decode4 gate_up: 48.01 MB read + 0.06 MB written (2-layer stack, the same
 # per-layer work): its 32.5 MB of packed gate_up rows and the 16.3 MB of down
 # matrices it requests into L2 for the down kernel (moved earlier, not re-read).
-# prefill gate_up: 378.06 MB read + 57.60 MB written (packed bank, x rows
+# prefill gate_up: 377.57 MB read + 56.87 MB written (packed bank, x rows
 # gathered per 128-row weight tile, activations out).
 MEASURED_TRAFFIC = {
-    ("decode4", "gate_up"): (47_384_576, "decode", "82eecb54cbdaf490"),
-    ("prefill", "gate_up"): (435_657_216, "grouped", "559eba8651574ef6"),
+    ("decode4", "gate_up"): (48_062_720, "decode", "ec2beb3a72dd8dc7"),
+    ("prefill", "gate_up"): (434_441_472, "grouped", "6957f73dd9f9e7fa"),
 }
 
 
@@ -254,14 +254,18 @@ def capture_graph(fn):
 
 # ---------------------------------------------------------------- algorithmic work
 
-def layer_work(moe, shape, T: int, touched: float):
+def layer_work(moe, shape, T: int, touched: float, inter_sh: int = 0, folded: bool = False):
     """Algorithmic bytes (decode) and flops (prefill) per layer of each kernel
     stage and of the whole layer.
 
     bytes: packed weights of the touched experts streamed once + the stage's
     inputs and outputs (intermediates that the method does not define, such as
     per-row fp32 partials, are not counted); flops: 2*T*E*H for the router,
-    2*R*(2I)*H for gate_up, 2*R*H*I for down, R = T*k."""
+    2*R*(2I)*H for gate_up, 2*R*H*I for down, R = T*k.  A bf16 shared expert
+    of intermediate inter_sh adds its weights (gate_up, gate vector, down) and
+    flops to the layer; folded into the decode kernels, its gate_up rows and
+    gate to the router stage (the routing GEMV computes them) and its down
+    rows to the down stage."""
     H, I, E, k = shape.hidden, shape.inter, shape.num_experts, shape.top_k
     R = T * k
     gu_e = moe.moe_packed_bytes(shape, 0) // E
@@ -269,8 +273,17 @@ def layer_work(moe, shape, T: int, touched: float):
     router = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
     gate_up = {"bytes": touched * gu_e + T * H * 2 + R * I * 2, "flops": 2 * R * 2 * I * H}
     down = {"bytes": touched * dn_e + R * I * 2 + T * H * 2, "flops": 2 * R * H * I}
+    n_sh = 2 * inter_sh + 1 if inter_sh else 0  # gate_up rows and the gate vector
+    sh_gu = {"bytes": n_sh * H * 2, "flops": 2 * T * n_sh * H}
+    sh_dn = {"bytes": H * inter_sh * 2, "flops": 2 * T * H * inter_sh}
+    if folded:
+        for d, add in ((router, sh_gu), (down, sh_dn)):
+            d["bytes"] += add["bytes"]
+            d["flops"] += add["flops"]
     layer = {"bytes": E * H * 2 + T * H * 2 + touched * (gu_e + dn_e) + T * H * 2,
-             "flops": router["flops"] + gate_up["flops"] + down["flops"]}
+             "flops": 2 * T * E * H + 2 * R * 2 * I * H + 2 * R * H * I}
+    layer["bytes"] += sh_gu["bytes"] + sh_dn["bytes"]
+    layer["flops"] += sh_gu["flops"] + sh_dn["flops"]
     return {"router": router, "gate_up": gate_up, "down": down, "layer": layer}
 
 
@@ -442,7 +455,9 @@ def measure(moe, stack, name: str, steps: int, warmup: int, path: int, rank: int
         layer_call(l, debug={"topk_ids_out": ids_buf})
         touched.append(len(torch.unique(ids_buf)))
     avg_touched = float(np.mean(touched))
-    work = layer_work(moe, shape, T, avg_touched)
+    folded = bool(shared) and (moe.moe_forward_shared_launch_count(shape, inter_sh, T, path)
+                               == moe.moe_forward_launch_count(shape, T, path, False))
+    work = layer_work(moe, shape, T, avg_touched, inter_sh or 0, folded)
     peaks, peak_kind = load_peaks()
     decode = T <= 32 and path != moe.MOE_PATH_PREFILL
     dom = max(("router", "gate_up", "down"), key=lambda n: stage_share[n])
@@ -484,7 +499,8 @@ def measure(moe, stack, name: str, steps: int, warmup: int, path: int, rank: int
                "call": "moe_forward_host per layer, pinned host buffers"}
         del ws_h
 
-    per_layer = moe.moe_forward_launch_count(shape, T, path, False) + (3 if shared else 0)
+    per_layer = (moe.moe_forward_shared_launch_count(shape, inter_sh, T, path) if shared
+                 else moe.moe_forward_launch_count(shape, T, path, False))
     cpu = None
     if with_cpu and rank == 0 and world == 1:
         v, desc, threads, secs = oracle_sample(stack, x, bias, T, budget_s=cpu_budget, shared=shared)

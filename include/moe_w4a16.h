@@ -397,7 +397,12 @@ MOE_API size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_sh
  *   out_t = bf16( sum_j w_tj y_tj  +  g_t * (W_down_s a_s) )   one final rounding
  * The shared expert's products run on tcgen05 above 32 tokens and as a
  * split-K mma.sync product up to 32; its contribution is added to the routed
- * combine in fp32 before the output's single bf16 rounding.  Other
+ * combine in fp32 before the output's single bf16 rounding.  On the decode
+ * path with the split-K routing (up to 32 tokens, E <= 256, k <= 8,
+ * H <= 2048) and I_s <= 512 it launches no kernel of its own: its gate_up
+ * rows and gate vector are computed by the routing GEMV, its SwiGLU and gate
+ * by the gate_up kernel, its down product inside the down kernel's combine
+ * (moe_forward_shared_launch_count says which form a call takes).  Other
  * arguments, paths, errors and the workspace rules as moe_forward (workspace
  * >= moe_workspace_bytes_shared bytes; opts->flags must be 0, else
  * MOE_ERR_UNSUPPORTED). */
@@ -418,6 +423,13 @@ MOE_API moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes,
  * debug copies are not kernels and are not counted); -1 if the arguments are
  * invalid or the path does not support them. */
 MOE_API int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, int routed);
+
+/* Number of kernels moe_forward_shared launches for T tokens on `path` with
+ * a shared expert of intermediate size inter_shared: moe_forward's count,
+ * plus 3 where the shared expert runs as its own kernels (0 where it rides
+ * the decode kernels); -1 if the arguments are invalid or the path does not
+ * support them. */
+MOE_API int moe_forward_shared_launch_count(const moe_shape_t* shape, int inter_shared, int T, moe_path_t path);
 
 /* Synchronises `stream`, then reports MOE_ERR_TIMEOUT if a bounded
  * device-side wait of a previous moe_forward on this workspace expired (and

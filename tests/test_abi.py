@@ -147,6 +147,25 @@ def test_forward_validation_happens_on_the_host():
     assert moe.moe_forward_launch_count(s, 4, 3, False) == -1     # unknown path
 
 
+def test_launch_counts_with_and_without_the_folded_shared_expert():
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    dec, pre = moe.MOE_PATH_DECODE, moe.MOE_PATH_PREFILL
+    # decode: split-K routing GEMV + finalize, gate_up, down (with the combine)
+    assert moe.moe_forward_launch_count(s, 4, dec, False) == 4
+    # the shared expert rides those four kernels up to I_s = 512 on the decode path
+    for T in (1, 4, 32):
+        assert moe.moe_forward_shared_launch_count(s, 512, T, dec) == moe.moe_forward_launch_count(s, T, dec, False)
+    assert moe.moe_forward_shared_launch_count(s, 448, 8, moe.MOE_PATH_AUTO) == 4
+    # its own three kernels elsewhere: larger I_s, the grouped path, more than 32 tokens
+    assert moe.moe_forward_shared_launch_count(s, 640, 4, dec) == 4 + 3
+    assert (moe.moe_forward_shared_launch_count(s, 512, 16, pre)
+            == moe.moe_forward_launch_count(s, 16, pre, False) + 3)
+    assert (moe.moe_forward_shared_launch_count(s, 512, 64, moe.MOE_PATH_AUTO)
+            == moe.moe_forward_launch_count(s, 64, moe.MOE_PATH_AUTO, False) + 3)
+    assert moe.moe_forward_shared_launch_count(s, 96, 4, dec) == -1   # I_s not a multiple of 64
+    assert moe.moe_forward_shared_launch_count(s, 512, 64, dec) == -1  # no decode path above 32 tokens
+
+
 def test_workspace_query_with_flags():
     s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
     base = moe.moe_workspace_bytes(s, 8192)

@@ -103,10 +103,34 @@ def test_shared_tiny_layer(fmt, path):
     check_shared(layer, fmt, 64, path, seed=3)
 
 
-@pytest.mark.parametrize("T", [4, 24])
+@pytest.mark.parametrize("T", [1, 4, 24, 32])
 def test_shared_nex_decode(T):
+    # folded: the shared expert rides the routing GEMV and the two decode kernels
     layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=100 + T, device=DEV)
+    shape = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    assert moe.moe_forward_shared_launch_count(shape, 512, T, moe.MOE_PATH_AUTO) == \
+        moe.moe_forward_launch_count(shape, T, moe.MOE_PATH_AUTO, False)
     check_shared(layer, "int4_g128", 512, seed=100 + T)
+
+
+@pytest.mark.parametrize("fmt,inter_shared,T", [("mxfp4", 448, 8), ("int4_g128", 640, 4)])
+def test_shared_nex_decode_other_sizes(fmt, inter_shared, T):
+    # 448: folded, its last 128-k sub-unit half past I_s; 640: too large for
+    # the down kernel's sub-units, the shared expert's own kernels
+    layer = moe_synth.make_layer(moe_synth.NEX, T=T, seed=300 + T, device=DEV)
+    check_shared(layer, fmt, inter_shared, seed=300 + inter_shared)
+
+
+def test_shared_decode_unfolded_odd_shape():
+    # E % 4 != 0: no split-K routing, so the shared expert runs its own
+    # split-K kernels beside the decode kernels (its output added in the
+    # down kernel's combine)
+    shp = moe_synth.LayerShape(hidden=320, inter=192, num_experts=6, top_k=3)
+    shape = moe.make_shape(320, 192, 6, 3, "int4_g128")
+    assert moe.moe_forward_shared_launch_count(shape, 64, 8, moe.MOE_PATH_DECODE) == \
+        moe.moe_forward_launch_count(shape, 8, moe.MOE_PATH_DECODE, False) + 3
+    layer = moe_synth.make_layer(shp, T=8, seed=77, device=DEV)
+    check_shared(layer, "int4_g128", 64, moe.MOE_PATH_DECODE, seed=78)
 
 
 def test_shared_nex_prefill_sampled():

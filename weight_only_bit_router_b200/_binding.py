@@ -111,6 +111,8 @@ _SIGS = {
                                           ctypes.POINTER(ForwardOpts), ctypes.c_void_p]),
     "moe_forward_launch_count": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int,
                                                 ctypes.c_int]),
+    "moe_forward_shared_launch_count": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_int, ctypes.c_int,
+                                                       ctypes.c_int]),
     "moe_forward_noalloc": (ctypes.c_int, [ctypes.POINTER(MoeShape), ctypes.c_void_p, ctypes.c_int,
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_void_p]),
@@ -429,6 +431,10 @@ def moe_forward_routed(shape: MoeShape, x, topk_ids, topk_w, gate_up_packed, dow
 
 def moe_forward_launch_count(shape: MoeShape, T: int, path=MOE_PATH_AUTO, routed=False) -> int:
     return lib().moe_forward_launch_count(ctypes.byref(shape), T, path, int(routed))
+
+
+def moe_forward_shared_launch_count(shape: MoeShape, inter_shared: int, T: int, path=MOE_PATH_AUTO) -> int:
+    return lib().moe_forward_shared_launch_count(ctypes.byref(shape), inter_shared, T, path)
 
 
 def moe_noalloc_scratch_bytes() -> int:

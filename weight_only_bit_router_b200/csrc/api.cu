@@ -3,6 +3,8 @@
 #include <nvtx3/nvToolsExt.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -180,14 +182,15 @@ moe_status_t route_all(const moe_shape_t& s, int T, const uint16_t* x, const uin
 moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const void* gu_packed,
                          const void* dn_packed, const ExpertRange& er, const Workspace& ws, uint16_t* out,
                          float* partial_out, bool decode, const moe_forward_opts_t* o, cudaStream_t stream,
-                         const float* sh_gate = nullptr, const float* sh_y = nullptr) {
+                         const float* sh_gate = nullptr, const float* sh_y = nullptr,
+                         const SharedFold* sf = nullptr) {
   const int n_bank = er.hi - er.lo;
   const Bank gu = make_bank(gu_packed, s.fmt, n_bank, 2 * s.inter, s.hidden);
   const Bank dn = make_bank(dn_packed, s.fmt, n_bank, s.hidden, s.inter);
   {
     NvtxRange range("moe.gate_up");
     MOE_TRY(mark(o, 2, 0, stream));
-    if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, dn, er, ws, stream));
+    if (decode) MOE_TRY(launch_decode_gate_up(s, T, x, gu, dn, er, ws, stream, sf));
     else MOE_TRY(launch_grouped_gate_up(s, T, x, gu, er, ws, stream));
     MOE_TRY(mark(o, 2, 1, stream));
   }
@@ -195,7 +198,7 @@ moe_status_t run_experts(const moe_shape_t& s, int T, const uint16_t* x, const v
   MOE_TRY(mark(o, 3, 0, stream));
   if (decode) {
     // down products and each token's slots summed in slot order, in one kernel
-    MOE_TRY(launch_decode_down(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream));
+    MOE_TRY(launch_decode_down(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream, sf));
     MOE_TRY(mark(o, 3, 1, stream));
     MOE_TRY(mark(o, 4, 0, stream));
   } else if (opt_flags(o) & MOE_FLAG_DETERMINISTIC) {
@@ -537,9 +540,21 @@ static SharedWs carve_shared(void* base, const moe_shape_t& s, int I_s, int T) {
   w.a = static_cast<uint16_t*>(take(size_t(T) * I_s * 2));
   w.g = static_cast<float*>(take(size_t(T) * 4));
   w.y = static_cast<float*>(take(size_t(T) * s.hidden * 4 * (T <= kDecodeMaxT ? shared_gemv_splits(I_s) : 1)));
-  w.h = static_cast<float*>(take(size_t(w.splits) * T * 2 * I_s * 4));
+  // h: the split-K gate_up partials, or (folded form) the routing GEMV's
+  // partials of the gate_up rows and the gate
+  const size_t h_fold = T <= kDecodeMaxT ? size_t(route_gemv_splits(s.hidden)) * T * (2 * I_s + 1) : 0;
+  w.h = static_cast<float*>(take(std::max(size_t(w.splits) * T * 2 * I_s, h_fold) * 4));
   w.bytes = off;
   return w;
+}
+
+// The shared expert rides the small-batch kernels (routing GEMV, decode
+// gate_up and down) instead of its own three: the decode kernels and the
+// split-K routing take the shape, and its down product fits the down
+// kernel's four 128-k sub-units.
+static bool shared_folds(const moe_shape_t& s, int T, int I_s, bool decode) {
+  return decode && T <= kDecodeMaxT && I_s <= kSharedFoldMaxInter &&
+         route_fast_applies(T, s.hidden, s.num_experts, s.top_k) && decode_shared_fits(s, T);
 }
 
 size_t moe_workspace_bytes_shared(const moe_shape_t* shape, int inter_shared, int T) {
@@ -569,6 +584,20 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   if (workspace_bytes < carve_shared(nullptr, s, I_s, T).bytes) return MOE_ERR_WORKSPACE;
   const Workspace ws = carve_workspace(workspace, s, T, opt_flags(opts));
   const SharedWs sw = carve_shared(workspace, s, I_s, T);
+  if (shared_folds(s, T, I_s, decode)) {
+    const SharedFold sf{shared->gate_up, shared->gate, shared->down, I_s, route_gemv_splits(s.hidden),
+                        sw.h, sw.a, sw.g};
+    MOE_TRY(mark(opts, 0, 0, stream));
+    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream,
+                               &sf));
+    MOE_TRY(mark(opts, 0, 1, stream));
+    MOE_TRY(mark(opts, 1, 0, stream));
+    MOE_TRY(mark(opts, 1, 1, stream));
+    if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr,
+                          decode, opts, stream, nullptr, nullptr, &sf)) != MOE_OK)
+      return st;
+    return copy_debug_outputs(s, T, ws, opts, false, stream);
+  }
   // the shared expert needs only x: gate_up product, SwiGLU and gate, down
   // product (split-K mma.sync for small batches, tcgen05 above)
   if (T <= kDecodeMaxT && I_s <= 512) {
@@ -615,6 +644,14 @@ int moe_forward_launch_count(const moe_shape_t* shape, int T, moe_path_t path, i
   else n += 2 + perm;                                         // router GEMM, top-k, permutation
   n += decode ? 2 : 3;  // gate_up, down (+ combine / finalize for the grouped GEMMs)
   return n;
+}
+
+int moe_forward_shared_launch_count(const moe_shape_t* shape, int inter_shared, int T, moe_path_t path) {
+  const int n = moe_forward_launch_count(shape, T, path, 0);
+  if (n < 0 || inter_shared <= 0 || inter_shared % 64) return -1;
+  if (T == 0) return 0;
+  const bool decode = path == MOE_PATH_DECODE || (path == MOE_PATH_AUTO && decode_supported(*shape, T));
+  return n + (shared_folds(*shape, T, inter_shared, decode) ? 0 : 3);
 }
 
 moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, cudaStream_t stream) {

@@ -158,6 +158,66 @@ struct ActFrags {
   }
 };
 
+// The shared expert's SwiGLU activation and sigmoid gate from the routing
+// GEMV's split partials (summed in split order): a[t][i] = bf16(silu(h_gate)
+// * h_up), g[t] = sigmoid(z_t).  The T * I_s features, then the T gates, are
+// spread over the grid: thread `tid` of `nthreads` per CTA.
+MOE_DEV void shared_activation(const SharedFold& sf, int T, int tid, int nthreads) {
+  const int I = sf.inter, N2 = 2 * I + 1, n = T * I + T;
+  for (int e = int(blockIdx.x) * nthreads + tid; e < n; e += int(gridDim.x) * nthreads) {
+    if (e < T * I) {
+      const int t = e / I, i = e - t * I;
+      float hg = 0.f, hu = 0.f;
+      for (int sp = 0; sp < sf.splits; ++sp) {
+        const float* hs = sf.h + (size_t(sp) * T + t) * N2;
+        hg += __ldcg(hs + i);
+        hu += __ldcg(hs + I + i);
+      }
+      sf.a[size_t(t) * I + i] = f32_to_bf16_rn(silu_mul(hg, hu));
+    } else {
+      const int t = e - T * I;
+      float z = 0.f;
+      for (int sp = 0; sp < sf.splits; ++sp) z += __ldcg(sf.h + (size_t(sp) * T + t) * N2 + 2 * I);
+      sf.g[t] = 1.0f / (1.0f + expf(-z));
+    }
+  }
+}
+
+// Sub-unit i of the shared expert's down product for one 16-feature tile: the
+// tile's bf16 rows over k in [128 i, 128 i + 128) times the activation of
+// every token, one warp; ys[t][f] (fp32, 16 features per token) gets the
+// partial product.  The activation was written by the kernel before (read
+// through L2); the rows are constant.
+template <int NT>
+MOE_DEV void shared_down_part(const SharedFold& sf, int T, int tile, int i, int g, int q, float* ys) {
+  const int I = sf.inter;
+  const int k = 128 * i + 32 * q;
+  const bool kin = k < I;  // I % 64 == 0: a lane's 32-k slice is whole or past I
+  const uint16_t* w = sf.w_down + size_t(tile * kDnRows + g) * I + k;
+  uint32_t alo[8][2], ahi[8][2];
+  act_frags_global<1>(w, kin, alo);
+  act_frags_global<1>(w + size_t(8) * I, kin, ahi);
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    if (8 * j >= T) break;
+    const int t = 8 * j + g;
+    uint32_t bf[8][2];
+    act_frags_global<2>(sf.a + size_t(t < T ? t : 0) * I + k, kin && t < T, bf);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int st = 0; st < 8; ++st) {
+      const uint32_t a[4] = {alo[st][0], ahi[st][0], alo[st][1], ahi[st][1]};
+      mma_bf16_16816(acc, a, bf[st][0], bf[st][1]);
+    }
+    // c0, c1: feature g at tokens 2q, 2q+1; c2, c3: feature g + 8
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int tok = 8 * j + 2 * q + (c & 1);
+      if (tok < T) ys[tok * kDnRows + g + 8 * (c >> 1)] = acc[c];
+    }
+  }
+}
+
 // Let the last bulk copies of this CTA's producer land before its shared
 // memory is released (bounded: they complete unless the GPU is failing).
 MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
@@ -183,7 +243,7 @@ template <int FMT, int NT, bool X_SMEM>
 __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
-    uint16_t* __restrict__ act, uint32_t* status, int S, Bank dn) {
+    uint16_t* __restrict__ act, uint32_t* status, int S, Bank dn, SharedFold sf) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int G = kGuGroups, MT = gu_mt(NT), FEAT = gu_feat(NT), CH = MT == 1 && NT == 1 ? 4 : 2;
   constexpr int kRed = kGroupWarps * NT * MT * 128;  // floats of one group's partial tiles
@@ -230,7 +290,13 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   // many CTAs (its extra token tiles are work the CTAs share)
   const int grid = int(gridDim.x);
   const int cnt = n_units > int(blockIdx.x) ? (n_units - int(blockIdx.x) + grid - 1) / grid : 0;
-  if (cnt <= 0) return;
+  // the shared expert's activation and gate: consumer threads, while the
+  // producer's first copies are in flight
+  const bool consumer = warp < G * kGroupWarps;
+  if (cnt <= 0) {
+    if (sf.h && consumer) shared_activation(sf, T, threadIdx.x, G * kGroupWarps * 32);
+    return;
+  }
   const int g_slot = grid / ftiles, g_ft = grid - g_slot * ftiles;  // a step of `grid` units
   auto advance = [&](int& sl, int& f, int steps) {  // (slot, feature tile) `steps` x grid units on
     for (int a = 0; a < steps; ++a) {
@@ -298,6 +364,7 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   }
 
   // -------------------------------------------------------------------- consumers
+  if (sf.h) shared_activation(sf, T, threadIdx.x, G * kGroupWarps * 32);
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
   const bool odd = (g & 1) != 0;  // this lane's low MMA row is the up row
@@ -424,7 +491,7 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
     const float* __restrict__ topk_w, const float* __restrict__ sh_gate, const float* __restrict__ sh_y,
-    uint16_t* __restrict__ out, float* __restrict__ partial_out) {
+    uint16_t* __restrict__ out, float* __restrict__ partial_out, SharedFold sf) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = dn_warps(NT, FMT), kThreads = dn_threads(NT, FMT);
   constexpr bool kOneChunk = W > 8;
@@ -439,6 +506,8 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
   int* s_off = s_touched + (E + 1);
   int* s_slot = s_off + (E + 1);                                  // [R] slot t k + j of sorted row p
   float* s_w = reinterpret_cast<float*>(s_slot + R);              // [R] its routing weight
+  float* s_sh = s_w + R;  // [nsu][T][16] the shared expert's down sub-unit products (with sf)
+  const int nsu = sf.w_down ? (sf.inter + 127) / 128 : 0;
   __shared__ int s_cnt[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -485,6 +554,18 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
           v0 += gg * __ldcg(sh_y + oi);
           v1 += gg * __ldcg(sh_y + oi + 1);
         }
+        if (nsu) {
+          // the shared expert: its sub-units summed in k order, times the gate
+          const float* ys = s_sh + t * kDnRows + f;
+          float y0 = ys[0], y1 = ys[1];
+          for (int i = 1; i < nsu; ++i) {
+            y0 += ys[i * T * kDnRows];
+            y1 += ys[i * T * kDnRows + 1];
+          }
+          const float gg = __ldcg(sf.g + t);
+          v0 += gg * y0;
+          v1 += gg * y1;
+        }
         *reinterpret_cast<uint32_t*>(out + oi) = pack_bf16x2(v0, v1);
       }
     }
@@ -496,6 +577,8 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
     prefetch_codes<FMT>(dn, r0, kDnRows);
     prefetch_scales<FMT>(dn, r0, kDnRows);
   }
+  if (nsu && threadIdx.x == 0 && blockIdx.x < ntile)  // the shared expert's rows of the first tile
+    bulk_prefetch_l2(sf.w_down + size_t(blockIdx.x) * kDnRows * sf.inter, uint32_t(kDnRows * sf.inter * 2));
   // The tile loop; FULL (every chunk is four whole k-blocks) drops the
   // bounds checks of the chunk loads and multiplies.
   auto run = [&](auto full_tag) {
@@ -579,6 +662,9 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
           ++k;
         }
       }
+      // the shared expert's sub-units: the warps after the last routed unit's
+      for (int i = 0; i < nsu; ++i)
+        if (warp == (n_t + i) % W) shared_down_part<NT>(sf, T, tile, i, g, q, s_sh + i * T * kDnRows);
       finish_tile(tile);
     }
   };
@@ -592,8 +678,11 @@ constexpr size_t kMaxSmemPerCta = 226 * 1024;  // dynamic shared memory, leaving
 constexpr size_t kSmemPerSm = 228 * 1024;       // shared memory of one SM
 constexpr size_t kSmemReservedPerCta = 2 * 1024;  // the system's share per CTA and the kernels' static arrays
 // Staged token rows (gate_up) and activation rows (down) up to these sizes.
+// The down kernel reads the activation rows through L2 by default: staging
+// them costs a block barrier before the first multiply, which measured
+// slower (4 tokens: down stage 14.6 us without staging, 15.5 us with).
 #ifndef MOE_DEC_MAX_STAGED_ACT_KB
-#define MOE_DEC_MAX_STAGED_ACT_KB 160
+#define MOE_DEC_MAX_STAGED_ACT_KB 0
 #endif
 constexpr size_t kMaxStagedX = 72 * 1024;
 constexpr size_t kMaxStagedAct = size_t(MOE_DEC_MAX_STAGED_ACT_KB) * 1024;
@@ -608,9 +697,11 @@ size_t gate_up_smem(int fmt, int K, int NT, int E, int R, int x_rows, int S) {
          2 * size_t(S) * 8;
 }
 
-// down: staged activation rows + the slot outputs + routing state
-size_t down_smem(int E, int R, int K, int act_rows) {
-  return size_t(act_rows) * staged_act_stride(K) + size_t(R) * kDnRows * 4 + size_t(2 * (E + 1) + 2 * R) * 4;
+// down: staged activation rows + the slot outputs + routing state (+ the
+// shared expert's sub-unit products)
+size_t down_smem(int E, int R, int K, int act_rows, int T, bool shared) {
+  return size_t(act_rows) * staged_act_stride(K) + size_t(R) * kDnRows * 4 + size_t(2 * (E + 1) + 2 * R) * 4 +
+         (shared ? size_t(kSharedFoldMaxInter / 128) * T * kDnRows * 4 : 0);
 }
 
 struct GuPlan {
@@ -647,11 +738,11 @@ GuPlan gate_up_plan(const moe_shape_t& s, int T) {
   return p;
 }
 
-DnPlan down_plan(const moe_shape_t& s, int T) {
+DnPlan down_plan(const moe_shape_t& s, int T, bool shared = false) {
   const int R = T * s.top_k;
   DnPlan p;
   p.act_smem = size_t(R) * staged_act_stride(s.inter) <= kMaxStagedAct;
-  p.smem = down_smem(s.num_experts, R, s.inter, p.act_smem ? R : 0);
+  p.smem = down_smem(s.num_experts, R, s.inter, p.act_smem ? R : 0, T, shared);
   return p;
 }
 
@@ -706,7 +797,8 @@ cudaError_t allow_smem(Kern k, size_t smem) {
 
 template <int FMT, int NT>
 cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
-                       const ExpertRange& er, const Workspace& ws, int units, cudaStream_t stream) {
+                       const ExpertRange& er, const Workspace& ws, int units, const SharedFold& sf,
+                       cudaStream_t stream) {
   const GuPlan p = gate_up_plan(s, T);
   if (p.S == 0) return cudaErrorInvalidConfiguration;
   auto k = p.x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
@@ -715,22 +807,24 @@ cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Ban
   const int grid = persistent_grid(k, p.smem, units, kGuThreads);
   return launch_pdl(k, dim3(grid), dim3(kGuThreads), p.smem, stream, x, T, gu, s.inter, s.num_experts, s.top_k,
                     er.lo, er.hi, (const int32_t*)ws.touched, (const int32_t*)ws.offsets,
-                    (const int32_t*)ws.sorted_rows, ws.act, ws.status, p.S, dn);
+                    (const int32_t*)ws.sorted_rows, ws.act, ws.status, p.S, dn, sf);
 }
 
 template <int FMT>
 cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
-                        const ExpertRange& er, const Workspace& ws, int units, cudaStream_t stream) {
+                        const ExpertRange& er, const Workspace& ws, int units, const SharedFold& sf,
+                        cudaStream_t stream) {
   // token tiles of 8 held in registers: enough for the largest possible expert batch (T)
-  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, dn, er, ws, units, stream);
-  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, dn, er, ws, units, stream);
-  return gate_up_nt<FMT, 4>(s, T, x, gu, dn, er, ws, units, stream);
+  if (T <= 8) return gate_up_nt<FMT, 1>(s, T, x, gu, dn, er, ws, units, sf, stream);
+  if (T <= 16) return gate_up_nt<FMT, 2>(s, T, x, gu, dn, er, ws, units, sf, stream);
+  return gate_up_nt<FMT, 4>(s, T, x, gu, dn, er, ws, units, sf, stream);
 }
 
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
-                    const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out, cudaStream_t stream) {
-  const DnPlan p = down_plan(s, T);
+                    const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out,
+                    const SharedFold& sf, cudaStream_t stream) {
+  const DnPlan p = down_plan(s, T, sf.w_down != nullptr);
   if (p.smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
   auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
   cudaError_t err = allow_smem(k, p.smem);
@@ -738,16 +832,16 @@ cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRan
   const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, dn_threads(NT, FMT));
   return launch_pdl(k, dim3(grid), dim3(dn_threads(NT, FMT)), p.smem, stream, dn, T, s.num_experts, s.top_k, er.lo, er.hi,
                     (const int32_t*)ws.touched, (const int32_t*)ws.offsets, (const int32_t*)ws.sorted_rows,
-                    (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out);
+                    (const uint16_t*)ws.act, (const float*)ws.topk_w, sh_gate, sh_y, out, partial_out, sf);
 }
 
 template <int FMT>
 cudaError_t down_fmt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
                      const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out,
-                     cudaStream_t stream) {
-  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
-  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
-  return down_nt<FMT, 4>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+                     const SharedFold& sf, cudaStream_t stream) {
+  if (T <= 8) return down_nt<FMT, 1>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, sf, stream);
+  if (T <= 16) return down_nt<FMT, 2>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, sf, stream);
+  return down_nt<FMT, 4>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, sf, stream);
 }
 
 }  // namespace
@@ -757,27 +851,37 @@ bool decode_supported(const moe_shape_t& s, int T) {
   return gate_up_plan(s, T).S > 0 && down_plan(s, T).smem <= kMaxSmemPerCta;
 }
 
+bool decode_shared_fits(const moe_shape_t& s, int T) {
+  return decode_supported(s, T) && down_plan(s, T, true).smem <= kMaxSmemPerCta;
+}
+
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
-                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream) {
-  const int units =
-      std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / gu_feat(nt_of(T)));
-  if (units <= 0) return cudaSuccess;
+                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream,
+                                  const SharedFold* sf) {
+  const SharedFold shf = sf ? *sf : SharedFold{};
+  int units = std::min(max_touched(T, s.top_k, s.num_experts), er.hi - er.lo) * (s.inter / gu_feat(nt_of(T)));
+  if (units <= 0) {
+    if (!sf || T == 0) return cudaSuccess;
+    units = 1;  // no routed unit, but the shared expert's activation is due
+  }
   Bank pf = dn;
   if (s.hidden % kDnPrefetchRows) pf.codes = nullptr;  // whole pieces only
-  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, pf, er, ws, units, stream);
-  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, pf, er, ws, units, stream);
-  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, pf, er, ws, units, stream);
+  if (s.fmt == MOE_FMT_INT4_G128) return gate_up_fmt<MOE_FMT_INT4_G128>(s, T, x, gu, pf, er, ws, units, shf, stream);
+  if (s.fmt == MOE_FMT_NVFP4_G16) return gate_up_fmt<MOE_FMT_NVFP4_G16>(s, T, x, gu, pf, er, ws, units, shf, stream);
+  return gate_up_fmt<MOE_FMT_MXFP4_G32>(s, T, x, gu, pf, er, ws, units, shf, stream);
 }
 
 cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
                                const Workspace& ws, const float* sh_gate, const float* sh_y, uint16_t* out,
-                               float* partial_out, cudaStream_t stream) {
+                               float* partial_out, cudaStream_t stream, const SharedFold* sf) {
   if (T == 0) return cudaSuccess;
+  if (sf && partial_out) return cudaErrorInvalidValue;  // the shared term belongs to the bf16 output only
+  const SharedFold shf = sf ? *sf : SharedFold{};
   if (s.fmt == MOE_FMT_INT4_G128)
-    return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+    return down_fmt<MOE_FMT_INT4_G128>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, shf, stream);
   if (s.fmt == MOE_FMT_NVFP4_G16)
-    return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
-  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, stream);
+    return down_fmt<MOE_FMT_NVFP4_G16>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, shf, stream);
+  return down_fmt<MOE_FMT_MXFP4_G32>(s, T, dn, er, ws, sh_gate, sh_y, out, partial_out, shf, stream);
 }
 
 }  // namespace moe

@@ -80,6 +80,24 @@ struct Workspace {
 Workspace carve_workspace(void* base, const moe_shape_t& s, int T, uint32_t flags = 0);
 size_t permute_block_rows();
 
+// The bf16 shared expert folded into the small-batch kernels (T <= kDecodeMaxT
+// with the split-K routing and the decode kernels): its gate_up rows and its
+// gate vector are extra rows of the routing GEMV, the gate_up kernel turns
+// their split partials into the SwiGLU activation and the sigmoid gate, and
+// the down kernel multiplies the activation by its down matrix inside the
+// combine.  Null members: no shared expert.
+struct SharedFold {
+  const uint16_t* w_gate_up;  // [2 I_s, H] bf16 (gate rows, then up rows)
+  const uint16_t* w_gate;     // [H] bf16 shared_expert_gate
+  const uint16_t* w_down;     // [H, I_s] bf16
+  int inter;                  // I_s (a multiple of 64, at most kSharedFoldMaxInter)
+  int splits;                 // k-splits of the routing GEMV
+  float* h;                   // [splits][T][2 I_s + 1] fp32 partials: gate_up rows, then the gate logit
+  uint16_t* a;                // [T, I_s] bf16 SwiGLU activation
+  float* g;                   // [T] fp32 sigmoid gate
+};
+constexpr int kSharedFoldMaxInter = 512;  // the down kernel's four 128-k sub-units
+
 // pack.cu
 cudaError_t launch_pack(moe_format_t fmt, const uint16_t* w, int E, int N, int K, void* packed,
                         int32_t* nonfinite, cudaStream_t stream);
@@ -92,8 +110,15 @@ cudaError_t launch_dequant(moe_format_t fmt, const void* packed, int E, int N, i
 // route.cu
 // Router GEMV + top-k + permutation for T <= kDecodeMaxT: split-K GEMV then
 // a one-CTA finalize kernel, or one kernel for other shapes.
+// With `sf` (the split-K form only) the GEMV also writes the shared expert's
+// partials sf->h.
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                               const Workspace& ws, int block_n, cudaStream_t stream);
+                               const Workspace& ws, int block_n, cudaStream_t stream,
+                               const SharedFold* sf = nullptr);
+// the split-K form applies (T <= 32, E <= 256, k <= 8, H <= 2048, E % 4 == 0)
+bool route_fast_applies(int T, int H, int E, int k);
+// k-splits of its GEMV
+int route_gemv_splits(int H);
 // split-K partial logits of the small-batch routing kernel (0 when it does not apply)
 size_t route_part_bytes(int T, int H, int E, int k);
 // kernels launch_route_small launches: 2 (split-K GEMV + finalize) where the
@@ -116,16 +141,22 @@ size_t permute_large_hist_bytes(int T, int E, int k);
 // the decode kernels take this shape and token count (T <= kDecodeMaxT and the
 // stages fit in shared memory)
 bool decode_supported(const moe_shape_t& s, int T);
+// ... and with the folded shared expert's products in the down kernel
+bool decode_shared_fits(const moe_shape_t& s, int T);
 // gate_up + SwiGLU into ws.act; also requests the touched experts' rows of
-// the down bank `dn` into L2 for the down kernel that follows
+// the down bank `dn` into L2 for the down kernel that follows; with `sf`
+// also the shared expert's activation sf->a and gate sf->g
 cudaError_t launch_decode_gate_up(const moe_shape_t& s, int T, const uint16_t* x, const Bank& gu, const Bank& dn,
-                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream);
+                                  const ExpertRange& er, const Workspace& ws, cudaStream_t stream,
+                                  const SharedFold* sf = nullptr);
 // the down products of the bank's experts and the combine: out = bf16(sum
 // over each token's slots in slot order of w * y (+ sh_gate[t] * sh_y[t])),
-// or the fp32 sum over the bank's experts into partial_out (sh_* nullable)
+// or the fp32 sum over the bank's experts into partial_out (sh_* nullable);
+// with `sf` (bf16 output only) the shared term is g[t] * (W_down a[t]),
+// computed here
 cudaError_t launch_decode_down(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er,
                                const Workspace& ws, const float* sh_gate, const float* sh_y, uint16_t* out,
-                               float* partial_out, cudaStream_t stream);
+                               float* partial_out, cudaStream_t stream, const SharedFold* sf = nullptr);
 
 // gemm_sm100.cu
 constexpr int kGemmBN = 128;  // token columns per grouped-GEMM tile

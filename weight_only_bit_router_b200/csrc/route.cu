@@ -371,7 +371,10 @@ __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
 // route_gemv_kernel: CTA (tile, s) computes, with mma.sync, the partial
 // logits of experts [16 tile, 16 tile + 16) over k in [256 s, 256 s + 256)
 // for every token and stores them; spreading the router weight over
-// (E/16) x (H/256) CTAs keeps every SM's share of it small.
+// (E/16) x (H/256) CTAs keeps every SM's share of it small.  With a shared
+// expert, more CTAs (after the router's) compute the same split partials of
+// its 2 I_s gate_up rows and its gate vector (one more row) for the gate_up
+// kernel, which turns them into the shared SwiGLU and gate.
 // route_finalize_kernel (one CTA, launched behind it and waiting at its
 // launch wait): sums the partials in split order (deterministic), keeps the
 // logits in shared memory, runs the top-k (one warp per token) and the
@@ -554,25 +557,37 @@ __device__ void warp_permutation_32(RouteFastSmem& sm, int R, int E, int32_t* __
 template <int NT>
 __global__ void __launch_bounds__(kRsThreads) route_gemv_kernel(const uint16_t* __restrict__ x,
                                                                 const uint16_t* __restrict__ wr, int T, int H,
-                                                                int E, float* __restrict__ part) {
+                                                                int E, float* __restrict__ part, SharedFold sf) {
   __shared__ float red[kRsWarps][4][32];  // one C fragment per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int e0 = blockIdx.x * kRsExperts, ks = blockIdx.y;
-  // warp: k-block b of this split, token tile jt
-  const int b = warp & 1, jt = warp >> 1;
+  const int ks = blockIdx.y;
+  // warp: k-block b of this split, token tile jt of row tile rt.  Router
+  // CTAs take one 16-row tile (warps past the token tiles idle); the shared
+  // expert's CTAs (past the router's) take 4 / NT of them, every warp busy.
+  const int b = warp & 1, slot = warp >> 1, jt = slot % NT, rt = slot / NT;
+  const int tiles_r = (E + kRsExperts - 1) / kRsExperts;
+  const bool sh = int(blockIdx.x) >= tiles_r;
+  const int n_rows = sh ? 2 * sf.inter + 1 : E;  // the shared rows: gate_up rows, then the gate vector
+  const bool active = sh ? true : rt == 0;
+  const int e0 = (sh ? (int(blockIdx.x) - tiles_r) * (4 / NT) + rt : int(blockIdx.x)) * kRsExperts;
+  float* out = sh ? sf.h : part;
+  auto row_ptr = [&](int r) -> const uint16_t* {
+    if (!sh) return wr + size_t(r) * H;
+    return r < 2 * sf.inter ? sf.w_gate_up + size_t(r) * H : sf.w_gate;
+  };
   const int kblk = ks * kRfK + b * 128 + 32 * q;
   const bool kin = kblk < H;
   uint32_t alo[8][2], ahi[8][2];
-  if (jt < NT) {
-    const bool r_lo = e0 + g < E, r_hi = e0 + g + 8 < E;
-    bf16_frags(wr + size_t(r_lo ? e0 + g : 0) * H + kblk, r_lo && kin, alo);
-    bf16_frags(wr + size_t(r_hi ? e0 + g + 8 : 0) * H + kblk, r_hi && kin, ahi);
+  const bool r_lo = active && e0 + g < n_rows, r_hi = active && e0 + g + 8 < n_rows;
+  if (active) {
+    bf16_frags(row_ptr(r_lo ? e0 + g : 0) + kblk, r_lo && kin, alo);
+    bf16_frags(row_ptr(r_hi ? e0 + g + 8 : 0) + kblk, r_hi && kin, ahi);
   }
   pdl_wait();
   pdl_trigger();
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (jt < NT) {
+  if (active) {
     uint32_t bf[8][2];
     const int t = jt * 8 + g;
     bf16_frags(x + size_t(t < T ? t : 0) * H + kblk, t < T && kin, bf);
@@ -585,15 +600,15 @@ __global__ void __launch_bounds__(kRsThreads) route_gemv_kernel(const uint16_t* 
 #pragma unroll
   for (int c = 0; c < 4; ++c) red[warp][c][lane] = acc[c];
   __syncthreads();
-  if (b == 0 && jt < NT) {
-    // this CTA's partial logits of token tile jt: the two k-blocks in order
+  if (b == 0 && active) {
+    // this CTA's partial products of token tile jt: the two k-blocks in order
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const float v = red[warp][c][lane] + red[warp + 1][c][lane];
-      // c0, c1: expert e0+g, tokens 2q, 2q+1; c2, c3: expert e0+g+8
+      // c0, c1: row e0+g, tokens 2q, 2q+1; c2, c3: row e0+g+8
       const int t = jt * 8 + 2 * q + (c & 1);
       const int e = e0 + g + ((c >> 1) << 3);
-      if (t < T && e < E) part[(size_t(ks) * T + t) * E + e] = v;
+      if (t < T && e < n_rows) out[(size_t(ks) * T + t) * n_rows + e] = v;
     }
   }
 }
@@ -809,10 +824,14 @@ cudaError_t route_small_nt(const uint16_t* x, const uint16_t* wr, const float* b
 
 template <int NT>
 cudaError_t route_fast_nt(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                          const Workspace& ws, int block_n, cudaStream_t stream) {
-  const dim3 grid((E + kRsExperts - 1) / kRsExperts, (H + kRfK - 1) / kRfK);
+                          const Workspace& ws, int block_n, cudaStream_t stream, const SharedFold* sf) {
+  SharedFold none{};
+  const SharedFold& shf = sf ? *sf : none;
+  // the shared expert's 2 I_s + 1 rows in CTAs of 4 / NT 16-row tiles
+  const int sh_ctas = sf ? ((2 * sf->inter + 1 + kRsExperts - 1) / kRsExperts + 4 / NT - 1) / (4 / NT) : 0;
+  const dim3 grid((E + kRsExperts - 1) / kRsExperts + sh_ctas, route_gemv_splits(H));
   cudaError_t err = launch_pdl(route_gemv_kernel<NT>, grid, dim3(kRsThreads), 0, stream, x, wr, T, H, E,
-                               ws.route_part);
+                               ws.route_part, shf);
   if (err != cudaSuccess) return err;
   return launch_pdl(route_finalize_kernel, dim3(1), dim3(kRsThreads), 0, stream, (const float*)ws.route_part,
                     int(grid.y), bias, T, E, k, ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows,
@@ -825,18 +844,21 @@ bool route_fast_applies(int T, int H, int E, int k) {
 
 int route_small_launches(int T, int H, int E, int k) { return route_fast_applies(T, H, E, k) ? 2 : 1; }
 
+int route_gemv_splits(int H) { return (H + kRfK - 1) / kRfK; }
+
 size_t route_part_bytes(int T, int H, int E, int k) {
-  return route_fast_applies(T, H, E, k) ? size_t((H + kRfK - 1) / kRfK) * T * E * sizeof(float) : 0;
+  return route_fast_applies(T, H, E, k) ? size_t(route_gemv_splits(H)) * T * E * sizeof(float) : 0;
 }
 
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                               const Workspace& ws, int block_n, cudaStream_t stream) {
+                               const Workspace& ws, int block_n, cudaStream_t stream, const SharedFold* sf) {
   const int nt = (T + 7) / 8;
   if (route_fast_applies(T, H, E, k)) {
-    if (nt <= 1) return route_fast_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
-    if (nt <= 2) return route_fast_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
-    return route_fast_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
+    if (nt <= 1) return route_fast_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream, sf);
+    if (nt <= 2) return route_fast_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream, sf);
+    return route_fast_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream, sf);
   }
+  if (sf) return cudaErrorInvalidValue;  // the shared rows ride the split-K GEMV only
   if (nt <= 1) return route_small_nt<1>(x, wr, bias, T, H, E, k, ws, block_n, stream);
   if (nt <= 2) return route_small_nt<2>(x, wr, bias, T, H, E, k, ws, block_n, stream);
   return route_small_nt<4>(x, wr, bias, T, H, E, k, ws, block_n, stream);
