@@ -239,7 +239,7 @@ MOE_DEV void drain_stages(uint64_t* full, int issued, int S) {
 // stage the T token rows in fragment order, before the programmatic-launch
 // wait.
 // ---------------------------------------------------------------------------
-template <int FMT, int NT, bool X_SMEM>
+template <int FMT, int NT, bool X_SMEM, bool SH>
 __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel(
     const uint16_t* __restrict__ x, int T, Bank gu, int I, int E, int top_k, int e_lo, int e_hi,
     const int32_t* __restrict__ touched, const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows,
@@ -290,13 +290,10 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   // many CTAs (its extra token tiles are work the CTAs share)
   const int grid = int(gridDim.x);
   const int cnt = n_units > int(blockIdx.x) ? (n_units - int(blockIdx.x) + grid - 1) / grid : 0;
-  // the shared expert's activation and gate: consumer threads, while the
-  // producer's first copies are in flight
-  const bool consumer = warp < G * kGroupWarps;
-  if (cnt <= 0) {
-    if (sf.h && consumer) shared_activation(sf, T, threadIdx.x, G * kGroupWarps * 32);
-    return;
-  }
+  // SH: the shared expert's activation and gate, by the consumer threads
+  // while the producer's first copies are in flight
+  if (SH && warp < G * kGroupWarps) shared_activation(sf, T, threadIdx.x, G * kGroupWarps * 32);
+  if (cnt <= 0) return;
   const int g_slot = grid / ftiles, g_ft = grid - g_slot * ftiles;  // a step of `grid` units
   auto advance = [&](int& sl, int& f, int steps) {  // (slot, feature tile) `steps` x grid units on
     for (int a = 0; a < steps; ++a) {
@@ -364,7 +361,6 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
   }
 
   // -------------------------------------------------------------------- consumers
-  if (sf.h) shared_activation(sf, T, threadIdx.x, G * kGroupWarps * 32);
   const int grp = warp / kGroupWarps, wj = warp % kGroupWarps;
   const int g = lane >> 2, q = lane & 3;
   const bool odd = (g & 1) != 0;  // this lane's low MMA row is the up row
@@ -486,7 +482,7 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
 // programmatic-launch wait.  With ACT_SMEM (small T) the warps then stage the
 // T*k activation rows in fragment order.
 // ---------------------------------------------------------------------------
-template <int FMT, int NT, bool ACT_SMEM>
+template <int FMT, int NT, bool ACT_SMEM, bool SH>
 __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
     Bank dn, int T, int E, int top_k, int e_lo, int e_hi, const int32_t* __restrict__ touched,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ sorted_rows, const uint16_t* __restrict__ act,
@@ -507,7 +503,7 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
   int* s_slot = s_off + (E + 1);                                  // [R] slot t k + j of sorted row p
   float* s_w = reinterpret_cast<float*>(s_slot + R);              // [R] its routing weight
   float* s_sh = s_w + R;  // [nsu][T][16] the shared expert's down sub-unit products (with sf)
-  const int nsu = sf.w_down ? (sf.inter + 127) / 128 : 0;
+  const int nsu = SH ? (sf.inter + 127) / 128 : 0;
   __shared__ int s_cnt[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -554,7 +550,7 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
           v0 += gg * __ldcg(sh_y + oi);
           v1 += gg * __ldcg(sh_y + oi + 1);
         }
-        if (nsu) {
+        if (SH) {
           // the shared expert: its sub-units summed in k order, times the gate
           const float* ys = s_sh + t * kDnRows + f;
           float y0 = ys[0], y1 = ys[1];
@@ -577,7 +573,7 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
     prefetch_codes<FMT>(dn, r0, kDnRows);
     prefetch_scales<FMT>(dn, r0, kDnRows);
   }
-  if (nsu && threadIdx.x == 0 && blockIdx.x < ntile)  // the shared expert's rows of the first tile
+  if (SH && threadIdx.x == 0 && blockIdx.x < ntile)  // the shared expert's rows of the first tile
     bulk_prefetch_l2(sf.w_down + size_t(blockIdx.x) * kDnRows * sf.inter, uint32_t(kDnRows * sf.inter * 2));
   // The tile loop; FULL (every chunk is four whole k-blocks) drops the
   // bounds checks of the chunk loads and multiplies.
@@ -663,8 +659,9 @@ __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
         }
       }
       // the shared expert's sub-units: the warps after the last routed unit's
-      for (int i = 0; i < nsu; ++i)
-        if (warp == (n_t + i) % W) shared_down_part<NT>(sf, T, tile, i, g, q, s_sh + i * T * kDnRows);
+      if (SH)
+        for (int i = 0; i < nsu; ++i)
+          if (warp == (n_t + i) % W) shared_down_part<NT>(sf, T, tile, i, g, q, s_sh + i * T * kDnRows);
       finish_tile(tile);
     }
   };
@@ -801,7 +798,9 @@ cudaError_t gate_up_nt(const moe_shape_t& s, int T, const uint16_t* x, const Ban
                        cudaStream_t stream) {
   const GuPlan p = gate_up_plan(s, T);
   if (p.S == 0) return cudaErrorInvalidConfiguration;
-  auto k = p.x_smem ? decode_gate_up_kernel<FMT, NT, true> : decode_gate_up_kernel<FMT, NT, false>;
+  const bool sh = sf.h != nullptr;
+  auto k = p.x_smem ? (sh ? decode_gate_up_kernel<FMT, NT, true, true> : decode_gate_up_kernel<FMT, NT, true, false>)
+                    : (sh ? decode_gate_up_kernel<FMT, NT, false, true> : decode_gate_up_kernel<FMT, NT, false, false>);
   cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(k, p.smem, units, kGuThreads);
@@ -820,13 +819,24 @@ cudaError_t gate_up_fmt(const moe_shape_t& s, int T, const uint16_t* x, const Ba
   return gate_up_nt<FMT, 4>(s, T, x, gu, dn, er, ws, units, sf, stream);
 }
 
+// The down kernel's instantiation: staged activations only when the build
+// allows staging at all (MOE_DEC_MAX_STAGED_ACT_KB > 0).
+template <int FMT, int NT>
+auto down_kernel_for(bool act_smem, bool sh) {
+  if constexpr (kMaxStagedAct > 0) {
+    if (act_smem) return sh ? decode_down_kernel<FMT, NT, true, true> : decode_down_kernel<FMT, NT, true, false>;
+  }
+  (void)act_smem;
+  return sh ? decode_down_kernel<FMT, NT, false, true> : decode_down_kernel<FMT, NT, false, false>;
+}
+
 template <int FMT, int NT>
 cudaError_t down_nt(const moe_shape_t& s, int T, const Bank& dn, const ExpertRange& er, const Workspace& ws,
                     const float* sh_gate, const float* sh_y, uint16_t* out, float* partial_out,
                     const SharedFold& sf, cudaStream_t stream) {
   const DnPlan p = down_plan(s, T, sf.w_down != nullptr);
   if (p.smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
-  auto k = p.act_smem ? decode_down_kernel<FMT, NT, true> : decode_down_kernel<FMT, NT, false>;
+  auto k = down_kernel_for<FMT, NT>(p.act_smem, sf.w_down != nullptr);
   cudaError_t err = allow_smem(k, p.smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(k, p.smem, s.hidden / kDnRows, dn_threads(NT, FMT));

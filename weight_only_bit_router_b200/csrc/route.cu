@@ -554,7 +554,7 @@ __device__ void warp_permutation_32(RouteFastSmem& sm, int R, int E, int32_t* __
 // partial logits of experts [16 tile, 16 tile + 16) over k in
 // [256 s, 256 s + 256) for every token.  The router weight does not depend on
 // the kernels before, so its fragments are loaded before the launch wait.
-template <int NT>
+template <int NT, bool SH>
 __global__ void __launch_bounds__(kRsThreads) route_gemv_kernel(const uint16_t* __restrict__ x,
                                                                 const uint16_t* __restrict__ wr, int T, int H,
                                                                 int E, float* __restrict__ part, SharedFold sf) {
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(kRsThreads) route_gemv_kernel(const uint16_t* 
   // expert's CTAs (past the router's) take 4 / NT of them, every warp busy.
   const int b = warp & 1, slot = warp >> 1, jt = slot % NT, rt = slot / NT;
   const int tiles_r = (E + kRsExperts - 1) / kRsExperts;
-  const bool sh = int(blockIdx.x) >= tiles_r;
+  const bool sh = SH && int(blockIdx.x) >= tiles_r;
   const int n_rows = sh ? 2 * sf.inter + 1 : E;  // the shared rows: gate_up rows, then the gate vector
   const bool active = sh ? true : rt == 0;
   const int e0 = (sh ? (int(blockIdx.x) - tiles_r) * (4 / NT) + rt : int(blockIdx.x)) * kRsExperts;
@@ -830,8 +830,8 @@ cudaError_t route_fast_nt(const uint16_t* x, const uint16_t* wr, const float* bi
   // the shared expert's 2 I_s + 1 rows in CTAs of 4 / NT 16-row tiles
   const int sh_ctas = sf ? ((2 * sf->inter + 1 + kRsExperts - 1) / kRsExperts + 4 / NT - 1) / (4 / NT) : 0;
   const dim3 grid((E + kRsExperts - 1) / kRsExperts + sh_ctas, route_gemv_splits(H));
-  cudaError_t err = launch_pdl(route_gemv_kernel<NT>, grid, dim3(kRsThreads), 0, stream, x, wr, T, H, E,
-                               ws.route_part, shf);
+  cudaError_t err = launch_pdl(sf ? route_gemv_kernel<NT, true> : route_gemv_kernel<NT, false>, grid,
+                               dim3(kRsThreads), 0, stream, x, wr, T, H, E, ws.route_part, shf);
   if (err != cudaSuccess) return err;
   return launch_pdl(route_finalize_kernel, dim3(1), dim3(kRsThreads), 0, stream, (const float*)ws.route_part,
                     int(grid.y), bias, T, E, k, ws.logits, ws.topk_ids, ws.topk_w, ws.offsets, ws.sorted_rows,
