@@ -166,6 +166,16 @@ def test_launch_counts_with_and_without_the_folded_shared_expert():
     assert moe.moe_forward_shared_launch_count(s, 512, 64, dec) == -1  # no decode path above 32 tokens
 
 
+def test_shared_workspace_holds_the_folded_partials():
+    s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
+    for T in (1, 4, 32):
+        extra = moe.moe_workspace_bytes_shared(s, 512, T) - moe.moe_workspace_bytes(s, T)
+        # activation, gate and the routing GEMV's 8 split partials of 1,025 rows per token
+        assert extra >= T * 512 * 2 + T * 4 + 8 * T * (2 * 512 + 1) * 4
+        # and the own-kernel form's down product [T, H]
+        assert extra >= T * 512 * 2 + T * 4 + T * 2048 * 4
+
+
 def test_workspace_query_with_flags():
     s = moe.make_shape(2048, 512, 256, 8, "int4_g128")
     base = moe.moe_workspace_bytes(s, 8192)
