@@ -374,7 +374,8 @@ __global__ void __launch_bounds__(kRsThreads) route_small_kernel(
 // (E/16) x (H/256) CTAs keeps every SM's share of it small.  With a shared
 // expert, more CTAs (after the router's) compute the same split partials of
 // its 2 I_s gate_up rows and its gate vector (one more row) for the gate_up
-// kernel, which turns them into the shared SwiGLU and gate.
+// kernel, which turns them into the shared SwiGLU and gate (template
+// parameter SH: without it the kernel compiles to the router rows alone).
 // route_finalize_kernel (one CTA, launched behind it and waiting at its
 // launch wait): sums the partials in split order (deterministic), keeps the
 // logits in shared memory, runs the top-k (one warp per token) and the
