@@ -89,7 +89,7 @@ KERNEL_SOURCES = {
 # prefill gate_up: 377.57 MB read + 56.87 MB written (packed bank, x rows
 # gathered per 128-row weight tile, activations out).
 MEASURED_TRAFFIC = {
-    ("decode4", "gate_up"): (47_347_968, "decode", "f79972613908d512"),
+    ("decode4", "gate_up"): (47_347_968, "decode", "23db5b2d1058ea6c"),
     ("prefill", "gate_up"): (434_441_472, "grouped", "6957f73dd9f9e7fa"),
 }
 

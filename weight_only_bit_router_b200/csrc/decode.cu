@@ -4,10 +4,10 @@
 // ("primitive-ai/Nex-N2.5-mini-mixed-NVFP4-FP8", Measured: at concurrency 32
 // the bottleneck is weight bandwidth).  Consumer warps dequantise in
 // registers (decode_common.cuh) and feed mma.sync m16n8k16 with up to 32
-// tokens; small token / activation sets are staged in shared memory once per
-// CTA in MMA fragment order, and the routing state (touched experts,
-// per-expert row offsets, the rows' tokens) is read into shared memory once
-// per CTA.
+// tokens; small token sets are staged in shared memory once per CTA in MMA
+// fragment order (the down kernel reads its activation rows through L2), and
+// the routing state (touched experts, per-expert row offsets, the rows'
+// tokens) is read into shared memory once per CTA.
 //
 // gate_up: persistent; CTA c takes the (touched expert, 8- or 16-feature)
 // units c, c + grid, ....  One producer warp starts, per unit, two bulk
@@ -21,9 +21,14 @@
 // outputs happens in the CTA (in slot order, deterministic) and the output is
 // written once.  Its 16-row weight tiles are small (16 rows x I/2 bytes), so
 // each warp loads its tiles straight into registers (16 warps per CTA with
-// one chunk each up to 8 tokens; 8 warps with the next chunk's loads in
-// flight during the multiply above), the first chunk's loads issued before
-// the programmatic-launch wait; gate_up has requested the tiles into L2.
+// one chunk each for INT4 and up to 8 tokens in every format; otherwise 8
+// warps with the next chunk's loads in flight during the multiply), the
+// first chunk's loads issued before the programmatic-launch wait; gate_up has
+// requested the tiles into L2.
+// Template parameter SH (both kernels): the bf16 shared expert rides along;
+// gate_up turns the routing GEMV's split partials of its rows into its
+// SwiGLU activation and gate, and down adds its gated down product to the
+// combine.  Without SH neither kernel carries any of that code.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -479,8 +484,9 @@ __global__ void __launch_bounds__(kGuThreads, gu_ctas(NT)) decode_gate_up_kernel
 // before: the routing state was written two launches back (and the kernel in
 // between triggers its dependents only after its own wait), so every warp
 // requests its tiles into L2 and loads its first chunk before the
-// programmatic-launch wait.  With ACT_SMEM (small T) the warps then stage the
-// T*k activation rows in fragment order.
+// programmatic-launch wait.  With ACT_SMEM (a build with a non-zero staging
+// threshold, small T) the warps then stage the T*k activation rows in
+// fragment order; otherwise the fragments are read through L2.
 // ---------------------------------------------------------------------------
 template <int FMT, int NT, bool ACT_SMEM, bool SH>
 __global__ void __maxnreg__(dn_regs(NT, FMT)) decode_down_kernel(
