@@ -151,15 +151,18 @@ moe_status_t build_permutation(const moe_shape_t& s, int T, const Workspace& ws,
                                           ws.pos, ws.block_hist, ws.touched, ws.tile_base, kGemmBN, stream));
 }
 
-// Stages 0-1: router logits, top-k and the permutation over all E experts.
+// Stages 0-1: router logits, top-k and the permutation over all E experts
+// (with `sf`, the small-batch routing GEMV also computes the folded shared
+// expert's rows).
 moe_status_t route_all(const moe_shape_t& s, int T, const uint16_t* x, const uint16_t* router_w,
                        const float* logit_bias, const Workspace& ws, const moe_forward_opts_t* opts,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, const SharedFold* sf = nullptr) {
   NvtxRange range("moe.route");
   MOE_TRY(mark(opts, 0, 0, stream));
   if (T <= kDecodeMaxT) {
-    // router logits, top-k and the permutation in one kernel
-    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
+    // router logits, top-k and the permutation: split-K GEMV + finalize, or one kernel
+    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream,
+                               sf));
     MOE_TRY(mark(opts, 0, 1, stream));
     MOE_TRY(mark(opts, 1, 0, stream));
   } else {
@@ -587,12 +590,7 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   if (shared_folds(s, T, I_s, decode)) {
     const SharedFold sf{shared->gate_up, shared->gate, shared->down, I_s, route_gemv_splits(s.hidden),
                         sw.h, sw.a, sw.g};
-    MOE_TRY(mark(opts, 0, 0, stream));
-    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream,
-                               &sf));
-    MOE_TRY(mark(opts, 0, 1, stream));
-    MOE_TRY(mark(opts, 1, 0, stream));
-    MOE_TRY(mark(opts, 1, 1, stream));
+    if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream, &sf)) != MOE_OK) return st;
     if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr,
                           decode, opts, stream, nullptr, nullptr, &sf)) != MOE_OK)
       return st;
@@ -600,29 +598,20 @@ moe_status_t moe_forward_shared(const moe_shape_t* shape, const moe_shared_exper
   }
   // the shared expert needs only x: gate_up product, SwiGLU and gate, down
   // product (split-K mma.sync for small batches, tcgen05 above)
-  if (T <= kDecodeMaxT && I_s <= 512) {
-    MOE_TRY(launch_shared_gemv(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, stream));
-    MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, sw.splits, T, s.hidden, I_s, sw.a, sw.g, stream));
-    MOE_TRY(launch_shared_gemv(sw.a, shared->down, T, I_s, s.hidden, sw.y, stream));  // one split: I_s <= 512
-  } else {
-    MOE_TRY(launch_router_gemm(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, ws.status, stream));
-    MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, 1, T, s.hidden, I_s, sw.a, sw.g, stream));
-    MOE_TRY(launch_router_gemm(sw.a, shared->down, T, I_s, s.hidden, sw.y, ws.status, stream));
+  {
+    NvtxRange range("moe.shared_expert");
+    if (T <= kDecodeMaxT && I_s <= 512) {
+      MOE_TRY(launch_shared_gemv(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, stream));
+      MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, sw.splits, T, s.hidden, I_s, sw.a, sw.g, stream));
+      MOE_TRY(launch_shared_gemv(sw.a, shared->down, T, I_s, s.hidden, sw.y, stream));  // one split: I_s <= 512
+    } else {
+      MOE_TRY(launch_router_gemm(x, shared->gate_up, T, s.hidden, 2 * I_s, sw.h, ws.status, stream));
+      MOE_TRY(launch_shared_swiglu_gate(x, shared->gate, sw.h, 1, T, s.hidden, I_s, sw.a, sw.g, stream));
+      MOE_TRY(launch_router_gemm(sw.a, shared->down, T, I_s, s.hidden, sw.y, ws.status, stream));
+    }
   }
   // the routed experts, their combine and the shared expert's gated output
-  MOE_TRY(mark(opts, 0, 0, stream));
-  if (T <= kDecodeMaxT) {
-    MOE_TRY(launch_route_small(x, router_w, logit_bias, T, s.hidden, s.num_experts, s.top_k, ws, kGemmBN, stream));
-    MOE_TRY(mark(opts, 0, 1, stream));
-    MOE_TRY(mark(opts, 1, 0, stream));
-  } else {
-    MOE_TRY(launch_router_gemm(x, router_w, T, s.hidden, s.num_experts, ws.logits, ws.status, stream));
-    MOE_TRY(mark(opts, 0, 1, stream));
-    MOE_TRY(mark(opts, 1, 0, stream));
-    MOE_TRY(launch_topk(ws.logits, logit_bias, T, s.num_experts, s.top_k, ws.topk_ids, ws.topk_w, stream));
-    if ((st = build_permutation(s, T, ws, stream)) != MOE_OK) return st;
-  }
-  MOE_TRY(mark(opts, 1, 1, stream));
+  if ((st = route_all(s, T, x, router_w, logit_bias, ws, opts, stream)) != MOE_OK) return st;
   if ((st = run_experts(s, T, x, gate_up_packed, down_packed, ExpertRange{0, s.num_experts}, ws, out, nullptr, decode,
                         opts, stream, sw.g, sw.y)) != MOE_OK)
     return st;
