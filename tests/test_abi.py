@@ -101,6 +101,7 @@ def test_forward_shared_validation_happens_on_the_host():
                                     ws_sh if wsb is None else wsb, 256, opts, None)
     assert call(shared=None) == 1
     assert call(wsb=ws_plain) == 3                                       # the routed workspace is too small
+    assert call(wsb=ws_sh - 1) == 3                                      # one byte short of the shared part
     bad = moe.SharedExpert(96, 256, 256, 256)
     assert call(shared=ctypes.byref(bad)) == 2                           # I_s not a multiple of 64
     unaligned = moe.SharedExpert(512, 258, 256, 256)
